@@ -1,0 +1,242 @@
+/*
+ * hca.h -- C ABI of libhca, a B200 (sm_100a) implementation of DeepSeek-V4's
+ * hybrid compressed attention: CSA (overlapped block compression, lightning
+ * indexer + per-query top-k, shared-KV MQA) and HCA (heavy compression, dense
+ * shared-KV MQA), both with a sliding-window branch, partial RoPE and a
+ * per-head attention sink.
+ *
+ * Sources of the operations (page title, section / equation):
+ *   [J] juejin "DeepSeek-V4 技术报告简要解读": §2.3.1 Eq.(9)-(19) (CSA),
+ *       §2.3.2 Eq.(20)-(23) (HCA), §2.3.3 (QK norm, partial RoPE, window,
+ *       sink Eq.(27)), §4.6 (heterogeneous KV cache).
+ *   [Z] 1zeryu "DeepSeek-V4：算法架构": "Q, K, V 映射与位置编码注入",
+ *       "Sparse Attention", "CSA 选择器层代码实现" (Compressor, Indexer),
+ *       "HCA 选择函数代码实现", "输出投影".
+ *
+ * Conventions (all functions):
+ *   - Return HCA_OK (0) or a negative status; hca_last_error() gives text.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call launches nothing and changes no buffer.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous.  Nothing here synchronises except
+ *     hca_check_status().
+ *   - The caller owns every device buffer.  The library allocates no device
+ *     memory: scratch is passed as `ws` of at least the size the matching
+ *     *_workspace_size() returns (256-byte aligned).
+ *   - Tensors are dense, C-order, innermost dimension contiguous, base
+ *     pointers 16-byte aligned.  Sizes below are in elements.
+ *   - Index lists are int32; -1 marks an empty slot.
+ *   - Positions are absolute token positions; one start position per call,
+ *     shared by the whole batch.
+ *   - Device-side waits are bounded; one that expires sets the device status
+ *     word to HCA_ERR_TIMEOUT, the kernel returns, and hca_check_status()
+ *     reports it.
+ */
+#ifndef HCA_H
+#define HCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *hca_stream_t; /* cudaStream_t */
+
+enum {
+  HCA_OK = 0,
+  HCA_ERR_INVALID = -1,     /* bad shape, null / misaligned pointer, bad dtype */
+  HCA_ERR_UNSUPPORTED = -2, /* valid request this build does not implement */
+  HCA_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch, attribute) */
+  HCA_ERR_TIMEOUT = -4      /* a bounded device wait expired */
+};
+
+typedef enum { HCA_F32 = 0, HCA_BF16 = 1, HCA_FP8E4M3 = 2 } hca_dtype;
+
+/* ------------------------------------------------------------------------
+ * Attention-layer shape.  Query i of a call sits at position start_pos + i.
+ * Compressed entry s covers tokens [s*m, (s+1)*m) and is visible to query t
+ * iff (s+1)*m <= t+1 ([Z] Indexer mask, get_compress_topk_idxs).
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int B;                   /* sequences in the batch */
+  int n_h;                 /* query heads sharing one KV head ([J] Eq.(18)) */
+  int c;                   /* shared KV / head dim */
+  int rd;                  /* RoPE dims: the last rd of c ([J] §2.3.3) */
+  int w;                   /* sliding-window tokens, >= 0 */
+  int m;                   /* compression ratio m (CSA) or m' (HCA) */
+  int overlap;             /* 1: overlapped compression [J] Eq.(11)-(12) */
+  int k;                   /* top-k entries per query (CSA) */
+  int n_hI, c_I, rd_I;     /* indexer heads, head dim, RoPE dims ([J] Eq.(14)) */
+  hca_dtype dtype;         /* storage of q, KV rows and o: HCA_F32 or HCA_BF16 */
+  hca_dtype idx_key_dtype; /* indexer key cache: dtype or HCA_FP8E4M3 */
+  float scale;             /* logit scale; <= 0 selects c^-1/2 */
+  float eps;               /* RMSNorm epsilon (1e-6) */
+  float rope_theta;        /* RoPE base (10000) */
+} hca_attn_desc;
+
+/* ------------------------------------------------------------------------
+ * Block compression, [J] Eq.(11)-(12) (overlap = 1) or Eq.(22)-(23)
+ * (overlap = 0); [Z] Compressor (prefill and decode branches).
+ *
+ * Entry i, channel ch: softmax over the rows of block i (logit Z_a + B_a) and,
+ * with overlap and i > 0, the rows of block i-1 (logit Z_b + B_b); the entry
+ * is the softmax-weighted sum of the matching C_a / C_b values.  With
+ * HCA_COMPRESS_NORM the entry is then RMS-normalised (weight gamma, NULL =
+ * ones); with HCA_COMPRESS_ROPE its last rd dims are rotated at position i*m.
+ * ---------------------------------------------------------------------- */
+#define HCA_COMPRESS_NORM 1
+#define HCA_COMPRESS_ROPE 2
+
+typedef struct {
+  int B;               /* sequences */
+  int width;           /* channels per entry (c, or c_I for indexer keys) */
+  int m;               /* ratio */
+  int overlap;         /* 1 = CSA overlapped series a/b, 0 = single series */
+  int rd;              /* RoPE dims of the epilogue (<= width, even) */
+  int flags;           /* HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE */
+  float eps, rope_theta;
+  hca_dtype in_dtype;  /* C and Z rows: HCA_F32 or HCA_BF16 */
+  hca_dtype out_dtype; /* entries: HCA_F32, HCA_BF16 or HCA_FP8E4M3 */
+} hca_compress_desc;
+
+/* csa_compress -- two modes:
+ *   prefill (start_pos == 0, n >= 1): writes entries 0 .. n/m - 1 of every
+ *     sequence, and (if state_kv != NULL) leaves the compressor state ready
+ *     for decode at position n.
+ *   decode (start_pos > 0, n == 1): appends token start_pos to the state;
+ *     when (start_pos + 1) % m == 0 writes entry start_pos / m.
+ * Ca, Za [B, n, width] (row stride row_stride, sequence stride seq_stride,
+ *   in elements); Cb, Zb the overlap series (NULL when overlap == 0).
+ * Ba, Bb [m, width] fp32 position biases (Bb NULL when overlap == 0).
+ * out: entry e of sequence b at out + (b*out_seq_stride + e)*width.
+ * out_scale: fp32 [B, out_seq_stride] row scales, only for fp8 output.
+ * state_kv / state_score fp32 [B, R, 2*width] (overlap, R = 2m) or
+ *   [B, R, width] (R = m); rows 0..m-1 hold the previous block and rows
+ *   m..2m-1 the current block (overlap); columns 0..width-1 the b series,
+ *   width..2width-1 the a series; score rows carry the bias (Z + B); empty
+ *   rows are (0, -inf).  Required in decode mode, optional in prefill. */
+int csa_compress(const hca_compress_desc *d, int start_pos, int n,
+                 const void *Ca, const void *Cb, const void *Za, const void *Zb,
+                 long long row_stride, long long seq_stride,
+                 const float *Ba, const float *Bb, const float *gamma,
+                 void *out, float *out_scale, long long out_seq_stride,
+                 float *state_kv, float *state_score, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Lightning indexer score + per-query top-k, [J] Eq.(16)-(17); [Z] Indexer.
+ *   I[t,s] = sum_h wI[t,h] * ReLU(qI[t,h] . K_I[s]) over visible s, then the
+ *   min(k, V_t) highest scores (ties to the lower index), V_t = (t+1)/m.
+ * qI [B, n_q, n_hI, c_I] (dtype; RoPE already applied), wI [B, n_q, n_hI]
+ *   fp32 (already scaled), KI [B, cap, c_I] (idx_key_dtype), KI_scale
+ *   [B, cap] fp32 row scales for fp8 keys (else NULL).
+ * idx [B, n_q, k]: kept entry indices in ascending order, then -1.
+ * scores (optional, NULL to skip): fp32 [B, n_q, score_stride] with the
+ *   index scores of the visible entries (score_stride >= max V_t).
+ * Requires (start_pos + n_q) / m <= cap. */
+size_t csa_index_topk_workspace_size(const hca_attn_desc *d, int n_q, int start_pos);
+int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI,
+                   const void *KI, const float *KI_scale, int cap, int n_q,
+                   int start_pos, int32_t *idx, float *scores, long long score_stride,
+                   void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Shared-KV MQA with sink, [J] Eq.(18)-(19), (27), §2.3.3; [Z] Sparse
+ * Attention, 输出投影.  For query t (head h) the key/value rows are the
+ * window rows of tokens max(0, t-w+1) .. t followed by the compressed rows
+ * (csa_attend: idx[t, j] >= 0; hca_attend: every visible entry s < (t+1)/m).
+ *   z_j = scale * q_h . row_j ; o_h = sum_j e^{z_j} row_j / (sum_j e^{z_j} + e^{sink_h})
+ * then the last rd dims of o_h are rotated by -t.
+ * q [B, n_q, n_h, c]; kv_comp [B, cap, c]; sink [n_h] fp32; o [B, n_q, n_h, c].
+ * kv_win: prefill (win_is_ring == 0, start_pos == 0): [B, n_q, c], row t =
+ *   token t; decode (win_is_ring == 1, n_q == 1): [B, w, c] ring, token p in
+ *   slot p % w (the caller has already stored token start_pos). */
+size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos);
+int csa_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap,
+               const int32_t *idx, const void *kv_win, int win_is_ring,
+               const float *sink, int n_q, int start_pos, void *o,
+               void *ws, size_t ws_bytes, hca_stream_t stream);
+
+size_t hca_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos);
+int hca_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap,
+               const void *kv_win, int win_is_ring, const float *sink, int n_q,
+               int start_pos, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Whole layer.  Weights are stored [d_out, d_in] row-major in a.dtype.
+ * ---------------------------------------------------------------------- */
+typedef enum { HCA_LAYER_CSA = 0, HCA_LAYER_HCA = 1, HCA_LAYER_SWA = 2 } hca_layer_kind;
+
+typedef struct {
+  hca_layer_kind kind;
+  hca_attn_desc a;
+  int d;               /* d_model */
+  int d_c;             /* query compression rank ([J] Eq.(13)) */
+  const void *W_comp;  /* CSA [4c, d] = W_aKV|W_bKV|W_aZ|W_bZ; HCA [2c, d] = W_KV|W_Z */
+  const float *B_comp; /* CSA [2, m, c] = B_a, B_b; HCA [m, c] */
+  const void *W_compI; /* CSA indexer compressor [4c_I, d] */
+  const float *B_compI;/* CSA [2, m, c_I] */
+  const void *W_DQ;    /* [d_c, d]        c^Q = RMSNorm(h W_DQ)          */
+  const void *W_UQ;    /* [n_h*c, d_c]    q = c^Q W_UQ, per-head RMS, RoPE */
+  const void *W_IUQ;   /* [n_hI*c_I, d_c] q^I = c^Q W_IUQ, RoPE (CSA)     */
+  const void *W_w;     /* [n_hI, d]       w^I = h W_w * c_I^-1/2 n_hI^-1/2 */
+  const void *W_KV;    /* [c, d]          window kv = RMSNorm(h W_KV), RoPE */
+  const float *sink;   /* [n_h] */
+} hca_layer;
+
+/* Decode-time cache of one layer ([J] §4.6: fixed-size state + classical
+ * compressed cache).  All device memory, owned by the caller. */
+typedef struct {
+  int cap;             /* entries per sequence (multiple of lcm(m, m')/m) */
+  void *kv_comp;       /* [B, cap, c] a.dtype */
+  void *key_I;         /* [B, cap, c_I] idx_key_dtype (CSA) */
+  float *key_I_scale;  /* [B, cap] (fp8 keys) */
+  void *win;           /* [B, w, c] ring, token p in slot p % w */
+  float *state_kv, *state_score;   /* compressor state (see csa_compress) */
+  float *stateI_kv, *stateI_score; /* indexer compressor state (CSA) */
+} hca_cache;
+
+/* hybrid_layer_forward -- prefill of n tokens per sequence from hidden states
+ * H [B, n, d] (a.dtype) at positions 0 .. n-1; writes o [B, n, n_h, c].
+ * With cache != NULL also fills the compressed caches, the window ring and
+ * the compressor states so that decode can continue at position n. */
+size_t hybrid_layer_forward_workspace_size(const hca_layer *L, int n);
+int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *cache,
+                         void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* One decode token per sequence: the projected inputs of the new token. */
+typedef struct {
+  const void *q;       /* [B, n_h, c] normalised, RoPE'd at pos */
+  const void *qI;      /* [B, n_hI, c_I] RoPE'd at pos (CSA) */
+  const float *wI;     /* [B, n_hI] scaled (CSA) */
+  const void *kv;      /* [B, c] window row (normalised, RoPE'd at pos) */
+  const float *comp;   /* [B, 4c] (CSA: Ca|Cb|Za|Zb) or [B, 2c] (HCA: C|Z) fp32 */
+  const float *compI;  /* [B, 4c_I] (CSA) fp32 */
+} hca_token_in;
+
+/* hybrid_decode_step -- token at position pos (> 0) for every sequence:
+ * stores its window row, advances the compressor states (emitting an entry
+ * when (pos+1) % m == 0), scores and selects (CSA), and attends; writes
+ * o [B, n_h, c]. */
+size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos);
+int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache,
+                       int pos, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics.
+ * ---------------------------------------------------------------------- */
+const char *hca_last_error(void);   /* text of the last failing call (thread-local) */
+/* Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait expires.  *device_status = HCA_OK or
+ * HCA_ERR_TIMEOUT.  Returns HCA_ERR_CUDA if the synchronisation failed. */
+int hca_check_status(hca_stream_t stream, int *device_status);
+int hca_version(void);              /* (major << 16) | minor */
+/* Kernels launched by the library since load (per process), for accounting. */
+long long hca_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HCA_H */

@@ -1,0 +1,216 @@
+"""Thin ctypes binding of libhca (include/hca.h): argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels; PyTorch supplies
+device memory and streams.  Loading fails loudly if libhca.so is missing.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhca.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "hca.h")
+
+HCA_OK, HCA_ERR_INVALID, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_TIMEOUT = 0, -1, -2, -3, -4
+HCA_F32, HCA_BF16, HCA_FP8E4M3 = 0, 1, 2
+HCA_COMPRESS_NORM, HCA_COMPRESS_ROPE = 1, 2
+HCA_LAYER_CSA, HCA_LAYER_HCA, HCA_LAYER_SWA = 0, 1, 2
+
+DTYPE_CODE = {torch.float32: HCA_F32, torch.bfloat16: HCA_BF16, torch.uint8: HCA_FP8E4M3,
+              torch.float8_e4m3fn: HCA_FP8E4M3}
+
+
+class HcaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"libhca error {code}: {msg}")
+        self.code = code
+
+
+class AttnDesc(C.Structure):
+    _fields_ = [("B", C.c_int), ("n_h", C.c_int), ("c", C.c_int), ("rd", C.c_int), ("w", C.c_int),
+                ("m", C.c_int), ("overlap", C.c_int), ("k", C.c_int), ("n_hI", C.c_int),
+                ("c_I", C.c_int), ("rd_I", C.c_int), ("dtype", C.c_int), ("idx_key_dtype", C.c_int),
+                ("scale", C.c_float), ("eps", C.c_float), ("rope_theta", C.c_float)]
+
+
+class CompressDesc(C.Structure):
+    _fields_ = [("B", C.c_int), ("width", C.c_int), ("m", C.c_int), ("overlap", C.c_int),
+                ("rd", C.c_int), ("flags", C.c_int), ("eps", C.c_float), ("rope_theta", C.c_float),
+                ("in_dtype", C.c_int), ("out_dtype", C.c_int)]
+
+
+class Layer(C.Structure):
+    _fields_ = [("kind", C.c_int), ("a", AttnDesc), ("d", C.c_int), ("d_c", C.c_int),
+                ("W_comp", C.c_void_p), ("B_comp", C.c_void_p), ("W_compI", C.c_void_p),
+                ("B_compI", C.c_void_p), ("W_DQ", C.c_void_p), ("W_UQ", C.c_void_p),
+                ("W_IUQ", C.c_void_p), ("W_w", C.c_void_p), ("W_KV", C.c_void_p),
+                ("sink", C.c_void_p)]
+
+
+class Cache(C.Structure):
+    _fields_ = [("cap", C.c_int), ("kv_comp", C.c_void_p), ("key_I", C.c_void_p),
+                ("key_I_scale", C.c_void_p), ("win", C.c_void_p), ("state_kv", C.c_void_p),
+                ("state_score", C.c_void_p), ("stateI_kv", C.c_void_p), ("stateI_score", C.c_void_p)]
+
+
+class TokenIn(C.Structure):
+    _fields_ = [("q", C.c_void_p), ("qI", C.c_void_p), ("wI", C.c_void_p), ("kv", C.c_void_p),
+                ("comp", C.c_void_p), ("compI", C.c_void_p)]
+
+
+_lib = None
+VP, I, LL, SZ = C.c_void_p, C.c_int, C.c_longlong, C.c_size_t
+
+
+def _declare(L):
+    sig = {
+        "hca_last_error": (C.c_char_p, []),
+        "hca_version": (I, []),
+        "hca_launch_count": (LL, []),
+        "hca_check_status": (I, [VP, C.POINTER(C.c_int)]),
+        "csa_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
+                             VP, LL, VP, VP, VP]),
+        "csa_index_topk_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
+        "csa_index_topk": (I, [C.POINTER(AttnDesc), VP, VP, VP, VP, I, I, I, VP, VP, LL, VP, SZ, VP]),
+        "csa_attend_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
+        "csa_attend": (I, [C.POINTER(AttnDesc), VP, VP, I, VP, VP, I, VP, I, I, VP, VP, SZ, VP]),
+        "hca_attend_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
+        "hca_attend": (I, [C.POINTER(AttnDesc), VP, VP, I, VP, I, VP, I, I, VP, VP, SZ, VP]),
+        "hybrid_layer_forward_workspace_size": (SZ, [C.POINTER(Layer), I]),
+        "hybrid_layer_forward": (I, [C.POINTER(Layer), VP, I, C.POINTER(Cache), VP, VP, SZ, VP]),
+        "hybrid_decode_step_workspace_size": (SZ, [C.POINTER(Layer), I]),
+        "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
+                                   SZ, VP]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+
+
+def lib():
+    """Load libhca.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise HcaError(HCA_ERR_UNSUPPORTED,
+                           f"{LIB_PATH} is missing: build it with "
+                           "`python -m long_context_compressed_hca_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        _declare(L)
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/hca.h declares."""
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?(?:int|size_t|long long|char\s*\*|const char\s*\*)\s*\**\s*"
+                                 r"([a-z_][a-z0-9_]*)\s*\(", txt, flags=re.M)))
+
+
+def ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def stream_handle(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def check(rc: int):
+    if rc != HCA_OK:
+        raise HcaError(rc, lib().hca_last_error().decode(errors="replace"))
+    return rc
+
+
+def last_error() -> str:
+    return lib().hca_last_error().decode(errors="replace")
+
+
+def device_status(stream=None) -> int:
+    v = C.c_int(0)
+    check(lib().hca_check_status(stream_handle(stream), C.byref(v)))
+    return v.value
+
+
+def launch_count() -> int:
+    return lib().hca_launch_count()
+
+
+def attn_desc(B, n_h, c, rd, w, m, overlap=0, k=0, n_hI=0, c_I=0, rd_I=0, dtype=HCA_BF16,
+              idx_key_dtype=None, scale=0.0, eps=1e-6, rope_theta=10000.0) -> AttnDesc:
+    return AttnDesc(B, n_h, c, rd, w, m, int(overlap), k, n_hI, c_I, rd_I, dtype,
+                    dtype if idx_key_dtype is None else idx_key_dtype, scale, eps, rope_theta)
+
+
+def compress_desc(B, width, m, overlap, rd, flags, in_dtype, out_dtype, eps=1e-6,
+                  rope_theta=10000.0) -> CompressDesc:
+    return CompressDesc(B, width, m, int(overlap), rd, flags, eps, rope_theta, in_dtype, out_dtype)
+
+
+# --------------------------------------------------------------------- calls
+def csa_compress(d: CompressDesc, start_pos, n, Ca, Cb, Za, Zb, row_stride, seq_stride, Ba, Bb,
+                 gamma, out, out_scale, out_seq_stride, state_kv, state_score, stream=None):
+    return check(lib().csa_compress(C.byref(d), start_pos, n, ptr(Ca), ptr(Cb), ptr(Za), ptr(Zb),
+                                    row_stride, seq_stride, ptr(Ba), ptr(Bb), ptr(gamma), ptr(out),
+                                    ptr(out_scale), out_seq_stride, ptr(state_kv), ptr(state_score),
+                                    stream_handle(stream)))
+
+
+def csa_index_topk_workspace_size(d: AttnDesc, n_q, start_pos) -> int:
+    return lib().csa_index_topk_workspace_size(C.byref(d), n_q, start_pos)
+
+
+def csa_index_topk(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, scores=None,
+                   score_stride=0, ws=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    return check(lib().csa_index_topk(C.byref(d), ptr(qI), ptr(wI), ptr(KI), ptr(KI_scale), cap, n_q,
+                                      start_pos, ptr(idx), ptr(scores), score_stride, ptr(ws), nbytes,
+                                      stream_handle(stream)))
+
+
+def csa_attend(d: AttnDesc, q, kv_comp, cap, idx, kv_win, win_is_ring, sink, n_q, start_pos, o,
+               ws=None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    return check(lib().csa_attend(C.byref(d), ptr(q), ptr(kv_comp), cap, ptr(idx), ptr(kv_win),
+                                  int(win_is_ring), ptr(sink), n_q, start_pos, ptr(o), ptr(ws), nbytes,
+                                  stream_handle(stream)))
+
+
+def hca_attend(d: AttnDesc, q, kv_comp, cap, kv_win, win_is_ring, sink, n_q, start_pos, o, ws=None,
+               stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    return check(lib().hca_attend(C.byref(d), ptr(q), ptr(kv_comp), cap, ptr(kv_win), int(win_is_ring),
+                                  ptr(sink), n_q, start_pos, ptr(o), ptr(ws), nbytes,
+                                  stream_handle(stream)))
+
+
+def layer_workspace_size(L: Layer, n: int) -> int:
+    return lib().hybrid_layer_forward_workspace_size(C.byref(L), n)
+
+
+def hybrid_layer_forward(L: Layer, H, n, cache: Cache | None, o, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    return check(lib().hybrid_layer_forward(C.byref(L), ptr(H), n, C.byref(cache) if cache else None,
+                                            ptr(o), ptr(ws), nbytes, stream_handle(stream)))
+
+
+def decode_workspace_size(L: Layer, pos: int) -> int:
+    return lib().hybrid_decode_step_workspace_size(C.byref(L), pos)
+
+
+def hybrid_decode_step(L: Layer, x: TokenIn, cache: Cache, pos, o, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    return check(lib().hybrid_decode_step(C.byref(L), C.byref(x), C.byref(cache), pos, ptr(o), ptr(ws),
+                                          nbytes, stream_handle(stream)))

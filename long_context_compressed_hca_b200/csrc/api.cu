@@ -1,0 +1,266 @@
+// api.cu -- the extern "C" entry points of libhca: host-side validation,
+// workspace carving and dispatch to the kernels.  See include/hca.h.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+
+__device__ int g_status = 0;
+
+static thread_local char t_err[512] = "";
+static std::atomic<long long> g_launches{0};
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_err, sizeof t_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int check_launch(const char *what) {
+  count_launch(1);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return HCA_OK;
+}
+
+int *device_status_ptr() {
+  static int *ptr[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (!ptr[dev]) {
+    void *a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_status) == cudaSuccess) ptr[dev] = static_cast<int *>(a);
+  }
+  return ptr[dev];
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+namespace {
+
+size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : (t == HCA_BF16 ? 2 : 1); }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+#define REQUIRE(cond, ...)                                   \
+  do {                                                       \
+    if (!(cond)) return fail(HCA_ERR_INVALID, __VA_ARGS__);  \
+  } while (0)
+
+int check_attn_desc(const hca_attn_desc *d, bool need_indexer) {
+  REQUIRE(d != nullptr, "null descriptor");
+  REQUIRE(d->B >= 1, "B must be >= 1 (got %d)", d->B);
+  REQUIRE(d->n_h >= 1, "n_h must be >= 1");
+  REQUIRE(d->c >= 32 && d->c <= 512 && d->c % 32 == 0, "c must be a multiple of 32 in [32, 512] (got %d)", d->c);
+  REQUIRE(d->rd >= 0 && d->rd <= d->c && d->rd % 2 == 0, "rd must be even and <= c");
+  REQUIRE(d->w >= 0, "w must be >= 0");
+  REQUIRE(d->m >= 1, "m must be >= 1");
+  REQUIRE(d->dtype == HCA_F32 || d->dtype == HCA_BF16, "dtype must be HCA_F32 or HCA_BF16");
+  if (need_indexer) {
+    REQUIRE(d->k >= 1, "k must be >= 1");
+    REQUIRE(d->n_hI >= 1 && d->c_I >= 8 && d->c_I % 8 == 0, "indexer heads / dim invalid");
+    REQUIRE(d->rd_I >= 0 && d->rd_I <= d->c_I && d->rd_I % 2 == 0, "rd_I must be even and <= c_I");
+    REQUIRE(d->idx_key_dtype == HCA_F32 || d->idx_key_dtype == HCA_BF16 || d->idx_key_dtype == HCA_FP8E4M3,
+            "idx_key_dtype invalid");
+  }
+  return HCA_OK;
+}
+
+float attn_scale(const hca_attn_desc *d) { return d->scale > 0.f ? d->scale : 1.0f / sqrtf((float)d->c); }
+
+IndexParams index_params(const hca_attn_desc *d, const void *qI, const float *wI, const void *KI,
+                         const float *KI_scale, int cap, int n_q, int start_pos) {
+  IndexParams p{};
+  p.B = d->B; p.n_q = n_q; p.start_pos = start_pos; p.m = d->m; p.n_hI = d->n_hI; p.c_I = d->c_I;
+  p.cap = cap; p.k = d->k; p.qI = qI; p.wI = wI; p.KI = KI; p.KI_scale = KI_scale;
+  p.q_dtype = d->dtype; p.key_dtype = d->idx_key_dtype;
+  return p;
+}
+
+AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap,
+                           const int32_t *idx, const void *kv_win, int win_is_ring, const float *sink,
+                           int n_q, int start_pos, void *o, int csa) {
+  AttendParams p{};
+  p.B = d->B; p.n_q = n_q; p.start_pos = start_pos; p.n_h = d->n_h; p.c = d->c; p.rd = d->rd;
+  p.w = d->w; p.m = d->m; p.k = csa ? d->k : 0; p.cap = cap; p.csa = csa; p.win_is_ring = win_is_ring;
+  p.scale = attn_scale(d); p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
+  p.q = q; p.kv_comp = kv_comp; p.idx = idx; p.kv_win = kv_win; p.sink = sink; p.o = o; p.dtype = d->dtype;
+  p.status = nullptr;
+  return p;
+}
+
+int check_attend_args(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap, const void *kv_win,
+                      int win_is_ring, const float *sink, int n_q, int start_pos, const void *o) {
+  REQUIRE(n_q >= 0 && start_pos >= 0, "n_q and start_pos must be >= 0");
+  REQUIRE(q && o && sink, "q, sink and o must be non-null");
+  REQUIRE(aligned16(q) && aligned16(o), "q and o must be 16-byte aligned");
+  const int vmax = (start_pos + n_q) / d->m;
+  REQUIRE(cap >= vmax, "cap (%d) < visible entries (%d)", cap, vmax);
+  REQUIRE(vmax == 0 || (kv_comp && aligned16(kv_comp)), "kv_comp must be non-null and 16-byte aligned");
+  if (d->w > 0) REQUIRE(kv_win && aligned16(kv_win), "kv_win must be non-null and 16-byte aligned");
+  if (win_is_ring) REQUIRE(n_q <= 1, "a ring window serves one query per sequence");
+  else REQUIRE(start_pos == 0, "a token-indexed window needs start_pos == 0");
+  return HCA_OK;
+}
+
+}  // namespace
+}  // namespace hca
+
+using namespace hca;
+
+extern "C" {
+
+const char *hca_last_error(void) { return t_err; }
+
+int hca_version(void) { return (0 << 16) | 1; }
+
+long long hca_launch_count(void) { return g_launches.load(); }
+
+int hca_check_status(hca_stream_t stream, int *device_status) {
+  if (!device_status) return fail(HCA_ERR_INVALID, "null device_status");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof v);
+  if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  const int zero = 0;
+  cudaMemcpyToSymbol(g_status, &zero, sizeof zero);
+  *device_status = v;
+  return HCA_OK;
+}
+
+// ----------------------------------------------------------------- compress
+int csa_compress(const hca_compress_desc *d, int start_pos, int n, const void *Ca, const void *Cb,
+                 const void *Za, const void *Zb, long long row_stride, long long seq_stride,
+                 const float *Ba, const float *Bb, const float *gamma, void *out, float *out_scale,
+                 long long out_seq_stride, float *state_kv, float *state_score, hca_stream_t stream) {
+  REQUIRE(d != nullptr, "null descriptor");
+  REQUIRE(d->B >= 1 && d->m >= 1, "B and m must be >= 1");
+  REQUIRE(d->width >= 8 && d->width % 8 == 0, "width must be a positive multiple of 8");
+  REQUIRE(d->overlap == 0 || d->overlap == 1, "overlap must be 0 or 1");
+  REQUIRE(d->in_dtype == HCA_F32 || d->in_dtype == HCA_BF16, "in_dtype must be f32 or bf16");
+  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16 || d->out_dtype == HCA_FP8E4M3, "bad out_dtype");
+  if (d->flags & HCA_COMPRESS_ROPE)
+    REQUIRE(d->rd >= 0 && d->rd <= d->width && d->rd % 8 == 0, "rd must be a multiple of 8 and <= width");
+  REQUIRE(n >= 0 && start_pos >= 0, "n and start_pos must be >= 0");
+  REQUIRE(Ca && Za && Ba, "Ca, Za and Ba must be non-null");
+  if (d->overlap) REQUIRE(Cb && Zb && Bb, "overlap needs Cb, Zb and Bb");
+  const size_t es = esize(d->in_dtype);
+  REQUIRE(aligned16(Ca) && aligned16(Za) && (!d->overlap || (aligned16(Cb) && aligned16(Zb))),
+          "C/Z pointers must be 16-byte aligned");
+  REQUIRE(row_stride >= d->width && (row_stride * (long long)es) % 16 == 0, "row_stride invalid");
+  REQUIRE((seq_stride * (long long)es) % 16 == 0, "seq_stride must keep 16-byte alignment");
+  REQUIRE(d->out_dtype != HCA_FP8E4M3 || out_scale, "fp8 output needs out_scale");
+  CompressParams p{};
+  p.B = d->B; p.n = n; p.width = d->width; p.m = d->m; p.overlap = d->overlap;
+  p.rd = (d->flags & HCA_COMPRESS_ROPE) ? d->rd : 0; p.flags = d->flags;
+  p.eps = d->eps > 0.f ? d->eps : 1e-6f; p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
+  p.Ca = Ca; p.Cb = Cb; p.Za = Za; p.Zb = Zb; p.row_stride = row_stride; p.seq_stride = seq_stride;
+  p.Ba = Ba; p.Bb = Bb; p.gamma = gamma; p.out = out; p.out_scale = out_scale; p.out_seq_stride = out_seq_stride;
+  p.state_kv = state_kv; p.state_score = state_score; p.in_dtype = d->in_dtype; p.out_dtype = d->out_dtype;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (start_pos == 0) {
+    const int E = n / d->m;
+    if (E > 0) {
+      REQUIRE(out && aligned16(out) && out_seq_stride >= E, "out must hold n/m entries per sequence");
+      int rc = launch_compress_prefill(p, s);
+      if (rc) return rc;
+    }
+    if (state_kv || state_score) {
+      REQUIRE(state_kv && state_score, "state_kv and state_score go together");
+      return launch_compress_state_prefill(p, s);
+    }
+    return HCA_OK;
+  }
+  REQUIRE(n == 1, "decode mode (start_pos > 0) takes exactly one token");
+  REQUIRE(state_kv && state_score, "decode mode needs the compressor state");
+  if ((start_pos + 1) % d->m == 0)
+    REQUIRE(out && aligned16(out) && out_seq_stride > start_pos / d->m, "out too small for entry %d",
+            start_pos / d->m);
+  return launch_compress_decode(p, start_pos, s);
+}
+
+// ----------------------------------------------------------------- index + top-k
+size_t csa_index_topk_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
+  if (!d || d->m < 1 || n_q < 0 || start_pos < 0) return 0;
+  IndexParams p = index_params(d, nullptr, nullptr, nullptr, nullptr, 0, n_q, start_pos);
+  return topk_workspace_bytes(p);
+}
+
+int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI, const void *KI,
+                   const float *KI_scale, int cap, int n_q, int start_pos, int32_t *idx, float *scores,
+                   long long score_stride, void *ws, size_t ws_bytes, hca_stream_t stream) {
+  int rc = check_attn_desc(d, true);
+  if (rc) return rc;
+  REQUIRE(n_q >= 0 && start_pos >= 0, "n_q and start_pos must be >= 0");
+  REQUIRE(qI && wI && idx, "qI, wI and idx must be non-null");
+  const int vmax = (start_pos + n_q) / d->m;
+  REQUIRE(cap >= vmax, "cap (%d) < visible entries (%d)", cap, vmax);
+  REQUIRE(vmax == 0 || KI, "KI must be non-null");
+  REQUIRE(d->idx_key_dtype != HCA_FP8E4M3 || KI_scale, "fp8 keys need KI_scale");
+  if (scores) REQUIRE(score_stride >= vmax, "score_stride < max visible entries");
+  IndexParams p = index_params(d, qI, wI, KI, KI_scale, cap, n_q, start_pos);
+  REQUIRE(ws || topk_workspace_bytes(p) == 0, "workspace required");
+  return run_index_topk(p, idx, scores, score_stride, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ----------------------------------------------------------------- attend
+size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
+  if (!d) return 0;
+  AttendParams p = attend_params(d, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, n_q, start_pos, nullptr, 1);
+  return attend_workspace_bytes(p);
+}
+size_t hca_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
+  if (!d) return 0;
+  AttendParams p = attend_params(d, nullptr, nullptr, 0, nullptr, nullptr, 0, nullptr, n_q, start_pos, nullptr, 0);
+  return attend_workspace_bytes(p);
+}
+
+int csa_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap, const int32_t *idx,
+               const void *kv_win, int win_is_ring, const float *sink, int n_q, int start_pos, void *o,
+               void *ws, size_t ws_bytes, hca_stream_t stream) {
+  int rc = check_attn_desc(d, false);
+  if (rc) return rc;
+  REQUIRE(d->k >= 1, "k must be >= 1");
+  rc = check_attend_args(d, q, kv_comp, cap, kv_win, win_is_ring, sink, n_q, start_pos, o);
+  if (rc) return rc;
+  REQUIRE(idx || n_q == 0, "idx must be non-null");
+  AttendParams p = attend_params(d, q, kv_comp, cap, idx, kv_win, win_is_ring, sink, n_q, start_pos, o, 1);
+  p.status = device_status_ptr();
+  REQUIRE(ws_bytes >= attend_workspace_bytes(p), "workspace too small");
+  return run_attend(p, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int hca_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap, const void *kv_win,
+               int win_is_ring, const float *sink, int n_q, int start_pos, void *o, void *ws, size_t ws_bytes,
+               hca_stream_t stream) {
+  int rc = check_attn_desc(d, false);
+  if (rc) return rc;
+  rc = check_attend_args(d, q, kv_comp, cap, kv_win, win_is_ring, sink, n_q, start_pos, o);
+  if (rc) return rc;
+  AttendParams p = attend_params(d, q, kv_comp, cap, nullptr, kv_win, win_is_ring, sink, n_q, start_pos, o, 0);
+  p.status = device_status_ptr();
+  REQUIRE(ws_bytes >= attend_workspace_bytes(p), "workspace too small");
+  return run_attend(p, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,524 @@
+// attend.cu -- shared-KV MQA with a sliding-window branch and attention sink.
+//
+// For query token t and head h (juejin "DeepSeek-V4 技术报告简要解读" §2.3.1(c)
+// Eq.(18)-(19), §2.3.3 Eq.(27); 1zeryu "DeepSeek-V4：算法架构", Sparse
+// Attention / 输出投影):
+//   rows  = window rows of tokens max(0,t-w+1)..t, then the compressed rows
+//           (CSA: idx[t, j] for the first min(k, V_t) slots; HCA: entries 0..V_t-1)
+//   z_j   = scale * q_h . row_j
+//   o_h   = sum_j e^{z_j} row_j / (sum_j e^{z_j} + e^{sink_h})
+//   o_h[last rd dims] rotated by -t.
+// Every row is both key and value; all n_h heads share it.
+//
+// Two implementations:
+//   attend_tc   bf16, tcgen05.  One query token per work unit, its n_h (<= 64)
+//               heads form the M=64 rows.  Per 64-key tile: S = Q K^T into a
+//               TMEM accumulator in lane-half 1 (double buffered), softmax in
+//               registers, P (bf16) to shared memory, O += P V into a TMEM
+//               accumulator in lane-half 0 (up to 512 fp32 columns).  The key
+//               tile in shared memory serves as K (K-major) and V (MN-major).
+//               Warp roles: 4 softmax/epilogue warps, 1 MMA warp, 4 gather
+//               warps (cp.async of the selected rows into 128B-swizzled tiles).
+//   attend_simt fp32 CUDA cores, any shape (and the tiny fp32 workload).
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct KeySet {
+  int nw, nc, nk, t0, V;
+};
+
+__device__ __forceinline__ KeySet key_set(const AttendParams &p, int qi) {
+  KeySet k;
+  const int t = p.start_pos + qi;
+  k.V = (t + 1) / p.m;
+  k.nw = min(p.w, t + 1);
+  k.t0 = t - k.nw + 1;
+  k.nc = p.csa ? min(p.k, k.V) : k.V;
+  k.nk = k.nw + k.nc;
+  return k;
+}
+
+// Row pointer of key `j` of query (b, qi), or nullptr if the slot is empty.
+template <typename T>
+__device__ __forceinline__ const T *key_row(const AttendParams &p, const KeySet &ks, int b, int qi,
+                                            int j) {
+  if (j < ks.nw) {
+    const int tok = ks.t0 + j;
+    if (p.win_is_ring)
+      return reinterpret_cast<const T *>(p.kv_win) + ((long long)b * p.w + tok % p.w) * p.c;
+    return reinterpret_cast<const T *>(p.kv_win) + ((long long)b * p.n_q + tok) * p.c;
+  }
+  if (j >= ks.nk) return nullptr;
+  int e = j - ks.nw;
+  if (p.csa) {
+    e = p.idx[((long long)b * p.n_q + qi) * p.k + e];
+    if (e < 0 || e >= ks.V) return nullptr;
+  }
+  return reinterpret_cast<const T *>(p.kv_comp) + ((long long)b * p.cap + e) * p.c;
+}
+
+// ======================================================================= SIMT
+constexpr int kSimtWarps = 8;
+constexpr int kSimtKT = 16;
+
+template <typename T>
+__global__ void __launch_bounds__(kSimtWarps * 32) attend_simt(AttendParams p) {
+  extern __shared__ float ks[];   // [kSimtKT][c]
+  __shared__ int kvalid[kSimtKT];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = blockIdx.x % p.n_q, b = blockIdx.x / p.n_q;
+  const int h = blockIdx.y * kSimtWarps + warp;
+  const bool hact = h < p.n_h;
+  const int E = p.c / 32;
+  const KeySet kset = key_set(p, qi);
+  const float zs = p.scale * kLog2e;
+  float qv[16], acc[16];
+  const T *qrow = reinterpret_cast<const T *>(p.q) + (((long long)b * p.n_q + qi) * p.n_h + (hact ? h : 0)) * p.c;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    qv[i] = (i < E) ? Elt<T>::load(qrow + lane + 32 * i) * zs : 0.f;
+    acc[i] = 0.f;
+  }
+  float mrun = -INFINITY, l = 0.f;
+  for (int j0 = 0; j0 < kset.nk; j0 += kSimtKT) {
+    for (int e = threadIdx.x; e < kSimtKT * p.c; e += blockDim.x) {
+      const int r = e / p.c, col = e % p.c;
+      const T *row = key_row<T>(p, kset, b, qi, j0 + r);
+      ks[e] = row ? Elt<T>::load(row + col) : 0.f;
+      if (col == 0) kvalid[r] = row != nullptr;
+    }
+    __syncthreads();
+    const int nrow = min(kSimtKT, kset.nk - j0);
+    for (int r = 0; r < nrow; ++r) {
+      if (!kvalid[r]) continue;
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < E) part += qv[i] * ks[r * p.c + lane + 32 * i];
+      const float z = warp_sum(part);
+      const float mn = fmaxf(mrun, z);
+      const float sc = exp2f(mrun - mn);
+      const float pz = exp2f(z - mn);
+      l = l * sc + pz;
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (i < E) acc[i] = acc[i] * sc + pz * ks[r * p.c + lane + 32 * i];
+      mrun = mn;
+    }
+    __syncthreads();
+  }
+  if (!hact) return;
+  const float sink2 = p.sink[h] * kLog2e;
+  const float M = fmaxf(mrun, sink2);
+  const float sc = (mrun == -INFINITY) ? 0.f : exp2f(mrun - M);
+  const float denom = l * sc + exp2f(sink2 - M);
+  const float inv = sc / denom;
+  const int t = p.start_pos + qi;
+  T *orow = reinterpret_cast<T *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + h) * p.c;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (i >= E) continue;
+    const int col = lane + 32 * i;
+    float v = acc[i] * inv;
+    const float other = __shfl_xor_sync(0xffffffffu, v, 1);
+    if (col >= p.c - p.rd) {
+      float s, cs;
+      rope_sincos(t, (col - (p.c - p.rd)) / 2, p.rd, p.theta, &s, &cs);
+      // inverse rotation: (a, b) -> (a cos + b sin, -a sin + b cos)
+      v = (lane & 1) ? (-other * s + v * cs) : (v * cs + other * s);
+    }
+    Elt<T>::store(orow + col, v);
+  }
+}
+
+// ======================================================================= tcgen05
+namespace tc {
+constexpr int KT = 64;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarp0 = 5;
+constexpr int kProdThreads = 128;
+constexpr int kThreads = (kSoftmaxWarps + 1 + 4) * 32;
+constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
+
+struct Bars {
+  uint64_t q_full, q_empty, o_empty, mma_done;
+  uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], pv_done[2];
+};
+
+template <int C>
+struct Layout {
+  static constexpr int NKB = C / 64;
+  static constexpr uint32_t q_off = 0;
+  static constexpr uint32_t kv_off = NKB * kTileBytes;
+  static constexpr uint32_t p_off = kv_off + 2 * NKB * kTileBytes;
+  static constexpr uint32_t bar_off = p_off + 2 * kTileBytes;
+  static constexpr uint32_t misc_off = bar_off + 256;
+  static constexpr uint32_t bytes = misc_off + 2048 + 1024;  // + alignment slack
+  static constexpr uint32_t tmem_cols = C <= 128 ? 128 : (C <= 256 ? 256 : 512);
+};
+
+template <int C>
+__global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_units) {
+  using L = Layout<C>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  Bars *bars = reinterpret_cast<Bars *>(smem + L::bar_off);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
+  double *freq = reinterpret_cast<double *>(smem + L::misc_off + 8);      // [32]
+  float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // [4 warps][64]: cos, sin
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](uint64_t &b) { return smem_u32(&b); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(bars->q_full), kProdThreads);
+    mbar_init(bar(bars->q_empty), 1);
+    mbar_init(bar(bars->o_empty), kSoftmaxWarps);
+    mbar_init(bar(bars->mma_done), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(bars->kv_full[i]), kProdThreads);
+      mbar_init(bar(bars->kv_empty[i]), 1);
+      mbar_init(bar(bars->s_full[i]), 1);
+      mbar_init(bar(bars->s_empty[i]), kSoftmaxWarps);
+      mbar_init(bar(bars->p_full[i]), kSoftmaxWarps);
+      mbar_init(bar(bars->pv_done[i]), 1);
+    }
+    mbar_fence_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), L::tmem_cols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x < p.rd / 2)
+    freq[threadIdx.x] = exp2(-2.0 * (double)threadIdx.x / (double)p.rd * log2((double)p.theta));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= kProdWarp0) {
+    // ------------------------------------------------------------ gather
+    [&]() {
+    const int pt = threadIdx.x - kProdWarp0 * 32;
+    constexpr int CPR = C / 8;                 // 16-byte chunks per row
+    constexpr int RPP = kProdThreads / CPR;    // rows per pass
+    const int chunk = pt % CPR, prow = pt / CPR;
+    const uint32_t kb_off = (chunk / 8) * kTileBytes;
+    const int cc = chunk % 8;
+    uint32_t g = 0, iq = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const int b = u / p.n_q, qi = u % p.n_q;
+      const KeySet ks = key_set(p, qi);
+      const int nt = (ks.nk + KT - 1) / KT;
+      if (nt == 0) continue;
+      if (!mbar_wait(bar(bars->q_empty), (iq & 1) ^ 1, p.status)) return;
+      const __nv_bfloat16 *qbase = reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+                                   ((long long)b * p.n_q + qi) * p.n_h * C;
+      for (int r = prow; r < 64; r += RPP) {
+        const bool ok = r < p.n_h;
+        const __nv_bfloat16 *src = ok ? qbase + (long long)r * C + chunk * 8 : qbase;
+        cp_async16(sbase + L::q_off + kb_off + sw128_off(r, cc), src, ok ? 16 : 0);
+      }
+      cp_async_wait_all();
+      fence_proxy_async();
+      mbar_arrive(bar(bars->q_full));
+      for (int j = 0; j < nt; ++j, ++g) {
+        const int st = g & 1;
+        if (!mbar_wait(bar(bars->kv_empty[st]), ((g >> 1) & 1) ^ 1, p.status)) return;
+        const uint32_t tile = sbase + L::kv_off + st * L::NKB * kTileBytes + kb_off;
+        for (int r = prow; r < KT; r += RPP) {
+          const __nv_bfloat16 *row = key_row<__nv_bfloat16>(p, ks, b, qi, j * KT + r);
+          cp_async16(tile + sw128_off(r, cc), row ? row + chunk * 8 : qbase, row ? 16 : 0);
+        }
+        cp_async_wait_all();
+        fence_proxy_async();
+        mbar_arrive(bar(bars->kv_full[st]));
+      }
+      ++iq;
+    }
+    }();
+    cp_async_wait_all();
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16(64, KT, 0, 0);
+      constexpr int NPV = C < 256 ? C : 256;
+      constexpr uint32_t IDESC_PV = idesc_bf16(64, NPV, 0, 1);
+      const uint32_t tS = tmem + (16u << 16);
+      uint32_t g = 0, iq = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+        const int st = gg & 1;
+        if (!mbar_wait(bar(bars->p_full[st]), (gg >> 1) & 1, p.status)) return false;
+        if (first && !mbar_wait(bar(bars->o_empty), (iq & 1) ^ 1, p.status)) return false;
+        tc_fence_after();
+        const uint32_t pa = sbase + L::p_off + st * kTileBytes;
+        const uint32_t va = sbase + L::kv_off + st * L::NKB * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          const uint64_t adesc = sdesc_sw128(pa + kk * 32, 16, 1024);
+#pragma unroll
+          for (int nh = 0; nh < C / NPV; ++nh) {
+            const uint64_t bdesc = sdesc_sw128(va + nh * (NPV / 64) * kTileBytes + kk * 16 * 128,
+                                               kTileBytes, 1024);
+            umma_bf16(tmem + nh * NPV, adesc, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          }
+        }
+        umma_commit(bar(bars->kv_empty[st]));
+        umma_commit(bar(bars->pv_done[st]));
+        return true;
+      };
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        const int qi = u % p.n_q;
+        const KeySet ks = key_set(p, qi);
+        const int nt = (ks.nk + KT - 1) / KT;
+        if (nt == 0) continue;
+        if (!mbar_wait(bar(bars->q_full), iq & 1, p.status)) { ok = false; break; }
+        tc_fence_after();
+        for (int j = 0; j < nt && ok; ++j) {
+          const uint32_t gj = g + j;
+          const int st = gj & 1;
+          const uint32_t ph = (gj >> 1) & 1;
+          if (!mbar_wait(bar(bars->kv_full[st]), ph, p.status) || !mbar_wait(bar(bars->s_empty[st]), ph ^ 1, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t qa = sbase + L::q_off;
+          const uint32_t ka = sbase + L::kv_off + st * L::NKB * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < C / 16; ++kk) {
+            const uint32_t off = (kk / 4) * kTileBytes + (kk % 4) * 32;
+            umma_bf16(tS + st * KT, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
+                      IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(bars->s_full[st]));
+          if (j == nt - 1) umma_commit(bar(bars->q_empty));
+          if (j >= 1 && !issue_pv(gj - 1, j - 1 == 0)) ok = false;
+        }
+        if (ok && !issue_pv(g + nt - 1, nt == 1)) ok = false;
+        g += nt;
+        ++iq;
+      }
+      umma_commit(bar(bars->mma_done));
+      mbar_wait(bar(bars->mma_done), 0, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    [&]() {
+    float *rope_cs = rope_all + warp * 64;
+    const int q4 = warp;                  // TMEM lane quarter
+    const int hl = lane & 15, half = lane >> 4;
+    const int r = q4 * 16 + hl;           // head row
+    const float zs = p.scale * kLog2e;
+    const uint32_t lane_S = (uint32_t)(q4 * 32 + 16) << 16;
+    const uint32_t lane_O = (uint32_t)(q4 * 32) << 16;
+    uint32_t g = 0, iq = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const int b = u / p.n_q, qi = u % p.n_q;
+      const int t = p.start_pos + qi;
+      const KeySet ks = key_set(p, qi);
+      const int nt = (ks.nk + KT - 1) / KT;
+      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
+      if (nt == 0) {
+        if (r < p.n_h)
+          for (int col = half * (C / 2); col < (half + 1) * (C / 2); col += 8)
+            *reinterpret_cast<uint4 *>(orow + col) = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      // RoPE table of this token (inverse rotation applied in the epilogue)
+      __syncwarp();
+      if (lane < p.rd / 2) {
+        const double two_pi = 6.283185307179586476925286766559;
+        double ang = (double)t * freq[lane];
+        ang -= two_pi * floor(ang / two_pi);
+        float sn, cs;
+        sincosf((float)ang, &sn, &cs);
+        rope_cs[lane] = cs;
+        rope_cs[32 + lane] = sn;
+      }
+      __syncwarp();
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < nt; ++j) {
+        const uint32_t gj = g + j;
+        const int st = gj & 1;
+        const uint32_t ph = (gj >> 1) & 1;
+        if (!mbar_wait(bar(bars->s_full[st]), ph, p.status)) return;
+        tc_fence_after();
+        uint32_t sv[32];
+        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->s_empty[st]));
+        // this thread's 32 keys: j*64 + half*32 + x
+        float z[32];
+        float tmax = -INFINITY;
+        const int kbase = j * KT + half * 32;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int kj = kbase + x;
+          bool valid = kj < ks.nk;
+          if (valid && kj >= ks.nw && p.csa) {
+            const int e = p.idx[((long long)b * p.n_q + qi) * p.k + (kj - ks.nw)];
+            valid = e >= 0 && e < ks.V;
+          }
+          z[x] = valid ? __uint_as_float(sv[x]) * zs : -INFINITY;
+          tmax = fmaxf(tmax, z[x]);
+        }
+        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+        bool need = false;
+        float alpha = 1.f;
+        if (j == 0) {
+          m_used = (tmax == -INFINITY) ? 0.f : tmax;
+        } else if (tmax > m_used + 8.f) {
+          need = true;
+          alpha = exp2f(m_used - tmax);
+          m_used = tmax;
+          l *= alpha;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // rescale O rows of this warp after the PV of the previous tile lands
+          const uint32_t gp = gj - 1;
+          if (!mbar_wait(bar(bars->pv_done[gp & 1]), (gp >> 1) & 1, p.status)) return;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < C / 2; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld_16x32bx2_x16<C / 2>(tmem + lane_O + c0, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+            tmem_st_16x32bx2_x16<C / 2>(tmem + lane_O + c0, ov);
+          }
+          tmem_st_wait();
+        }
+        float psum = 0.f;
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float p0 = exp2f(z[x] - m_used), p1 = exp2f(z[x + 1] - m_used);
+          psum += p0 + p1;
+          pk[x / 2] = pack_bf16x2(p0, p1);
+        }
+        l += psum;
+        // P buffer `st` is free once the PV of tile gj-2 has completed
+        if (!mbar_wait(bar(bars->pv_done[st]), ph ^ 1, p.status)) return;
+        uint8_t *prow = smem + L::p_off + st * kTileBytes;
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const int chunkp = half * 4 + u4;
+          *reinterpret_cast<uint4 *>(prow + sw128_off(r, chunkp)) =
+              make_uint4(pk[u4 * 4 + 0], pk[u4 * 4 + 1], pk[u4 * 4 + 2], pk[u4 * 4 + 3]);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->p_full[st]));
+      }
+      // -------- epilogue: normalise, inverse RoPE, store
+      const uint32_t gl = g + nt - 1;
+      if (!mbar_wait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, p.status)) return;
+      tc_fence_after();
+      const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      const float sink2 = (r < p.n_h) ? p.sink[r] * kLog2e : 0.f;
+      const float inv = 1.f / (ltot + exp2f(sink2 - m_used));
+#pragma unroll 1
+      for (int c0 = 0; c0 < C / 2; c0 += 16) {
+        uint32_t ov[16];
+        tmem_ld_16x32bx2_x16<C / 2>(tmem + lane_O + c0, ov);
+        tmem_ld_wait();
+        float v[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] = __uint_as_float(ov[x]) * inv;
+        const int col0 = half * (C / 2) + c0;
+        if (col0 + 16 > C - p.rd) {
+#pragma unroll
+          for (int x = 0; x < 16; x += 2) {
+            const int col = col0 + x;
+            if (col >= C - p.rd) {
+              const int pi = (col - (C - p.rd)) / 2;
+              const float cs = rope_cs[pi], sn = rope_cs[32 + pi];
+              const float a = v[x], bb = v[x + 1];
+              v[x] = a * cs + bb * sn;
+              v[x + 1] = -a * sn + bb * cs;
+            }
+          }
+        }
+        if (r < p.n_h) {
+          uint4 w0, w1;
+          w0.x = pack_bf16x2(v[0], v[1]); w0.y = pack_bf16x2(v[2], v[3]);
+          w0.z = pack_bf16x2(v[4], v[5]); w0.w = pack_bf16x2(v[6], v[7]);
+          w1.x = pack_bf16x2(v[8], v[9]); w1.y = pack_bf16x2(v[10], v[11]);
+          w1.z = pack_bf16x2(v[12], v[13]); w1.w = pack_bf16x2(v[14], v[15]);
+          *reinterpret_cast<uint4 *>(orow + col0) = w0;
+          *reinterpret_cast<uint4 *>(orow + col0 + 8) = w1;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->o_empty));
+      g += nt;
+      ++iq;
+    }
+    }();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, L::tmem_cols);
+}
+
+template <int C>
+int launch_tc(const AttendParams &p, cudaStream_t s) {
+  const int n_units = p.B * p.n_q;
+  const size_t smem = Layout<C>::bytes;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attend_tc<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "attend_tc smem attribute: %s", cudaGetErrorString(e));
+    attr_set = true;
+  }
+  const int grid = n_units < num_sms() ? n_units : num_sms();
+  attend_tc<C><<<grid, kThreads, smem, s>>>(p, n_units);
+  return check_launch("attend_tc");
+}
+}  // namespace tc
+
+}  // namespace
+
+size_t attend_workspace_bytes(const AttendParams &p) {
+  (void)p;
+  return 0;
+}
+
+int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s) {
+  (void)ws; (void)ws_bytes;
+  if (p.B * p.n_q == 0) return HCA_OK;
+  const bool tc_ok = p.dtype == HCA_BF16 && p.n_h <= 64 && (p.c == 128 || p.c == 256 || p.c == 512) &&
+                     p.rd <= p.c / 2 && p.rd % 2 == 0 && p.rd <= 64;
+  if (tc_ok) {
+    switch (p.c) {
+      case 128: return tc::launch_tc<128>(p, s);
+      case 256: return tc::launch_tc<256>(p, s);
+      default: return tc::launch_tc<512>(p, s);
+    }
+  }
+  dim3 grid(p.B * p.n_q, (p.n_h + kSimtWarps - 1) / kSimtWarps);
+  const size_t smem = (size_t)kSimtKT * p.c * sizeof(float);
+  if (p.dtype == HCA_F32) attend_simt<float><<<grid, kSimtWarps * 32, smem, s>>>(p);
+  else attend_simt<__nv_bfloat16><<<grid, kSimtWarps * 32, smem, s>>>(p);
+  return check_launch("attend_simt");
+}
+
+}  // namespace hca

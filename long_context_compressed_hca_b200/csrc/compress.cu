@@ -1,0 +1,370 @@
+// compress.cu -- block compression of KV entries.
+//
+// CSA (juejin "DeepSeek-V4 技术报告简要解读" §2.3.1(a), Eq.(11)-(12)): entry i,
+// channel ch is the softmax over the 2m logits {Z_a rows of block i + B_a} U
+// {Z_b rows of block i-1 + B_b} applied to the matching C_a / C_b values.
+// HCA (§2.3.2, Eq.(22)-(23)): softmax over the m' rows of block i (+ B).
+// Epilogue (§2.3.3; 1zeryu "DeepSeek-V4：算法架构", Compressor): RMSNorm of the
+// entry, RoPE of its last rd dims at the block start i*m, and for fp8 output a
+// per-entry amax/448 scale.
+//
+// HBM-bound: every C/Z element is read once (16-byte vector loads), each entry
+// written once.  A thread owns 8 channels and a slice of the block's rows and
+// keeps an online (running max) softmax per channel; slices are merged in
+// shared memory.  The decode branch keeps the block's rows in a caller-owned
+// fp32 state and emits an entry when a block completes.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename Tin>
+__device__ __forceinline__ const Tin *row_ptr(const void *base, long long seq_stride,
+                                             long long row_stride, int b, long long tok) {
+  return reinterpret_cast<const Tin *>(base) + (long long)b * seq_stride + tok * row_stride;
+}
+
+// Write one finished entry (8 channels per thread) with the epilogue applied.
+// `vals` are this thread's 8 channel values; `red` is shared scratch of at
+// least `cv` floats per entry slot.  All threads of the block must call it.
+template <typename Tout>
+struct EntryWriter;
+
+template <>
+struct EntryWriter<float> {
+  static __device__ void put(float *row, int ch0, const float (&v)[8], float) { store8(row + ch0, v); }
+};
+template <>
+struct EntryWriter<__nv_bfloat16> {
+  static __device__ void put(__nv_bfloat16 *row, int ch0, const float (&v)[8], float) {
+    store8(row + ch0, v);
+  }
+};
+template <>
+struct EntryWriter<uint8_t> {
+  static __device__ void put(uint8_t *row, int ch0, const float (&v)[8], float inv_scale) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      lo |= (uint32_t)__nv_cvt_float_to_fp8(v[j] * inv_scale, __NV_SATFINITE, __NV_E4M3) << (8 * j);
+      hi |= (uint32_t)__nv_cvt_float_to_fp8(v[4 + j] * inv_scale, __NV_SATFINITE, __NV_E4M3)
+            << (8 * j);
+    }
+    *reinterpret_cast<uint2 *>(row + ch0) = make_uint2(lo, hi);
+  }
+};
+
+// Per-entry epilogue for `epb` entries handled by one block: norm, rope,
+// fp8 scale, store.  Thread t with active=true owns channels [ch0, ch0+8) of
+// entry slot `slot`.
+template <typename Tout>
+__device__ void entry_epilogue(const CompressParams &p, float (&v)[8], bool active, int slot,
+                               int cvi, int cv, int b, long long entry, long long pos,
+                               float *red /* [epb * cv] */, float *red2) {
+  const int ch0 = cvi * 8;
+  if (p.flags & HCA_COMPRESS_NORM) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += v[j] * v[j];
+    if (active) red[slot * cv + cvi] = ss;
+    __syncthreads();
+    if (active) {
+      float tot = 0.f;
+      for (int j = 0; j < cv; ++j) tot += red[slot * cv + j];
+      const float r = rsqrtf(tot / (float)p.width + p.eps);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] *= r * (p.gamma ? p.gamma[ch0 + j] : 1.f);
+    }
+    __syncthreads();
+  }
+  if ((p.flags & HCA_COMPRESS_ROPE) && p.rd > 0 && active && ch0 >= p.width - p.rd) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float s, c;
+      rope_sincos(pos, (ch0 - (p.width - p.rd)) / 2 + j, p.rd, p.theta, &s, &c);
+      const float a = v[2 * j], bb = v[2 * j + 1];
+      v[2 * j] = a * c - bb * s;
+      v[2 * j + 1] = a * s + bb * c;
+    }
+  }
+  float inv_scale = 1.f;
+  if (p.out_dtype == HCA_FP8E4M3) {
+    float am = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(v[j]));
+    if (active) red2[slot * cv + cvi] = am;
+    __syncthreads();
+    if (active) {
+      float tot = 0.f;
+      for (int j = 0; j < cv; ++j) tot = fmaxf(tot, red2[slot * cv + j]);
+      tot = fmaxf(tot, 1e-12f);
+      const float scale = tot / 448.f;
+      inv_scale = 1.f / scale;
+      if (cvi == 0) p.out_scale[(long long)b * p.out_seq_stride + entry] = scale;
+    }
+    __syncthreads();
+  }
+  if (active) {
+    Tout *row = reinterpret_cast<Tout *>(p.out) + ((long long)b * p.out_seq_stride + entry) * p.width;
+    EntryWriter<Tout>::put(row, ch0, v, inv_scale);
+  }
+}
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads)
+compress_prefill_kernel(CompressParams p, int epb, int rg) {
+  extern __shared__ float sm[];
+  const int cv = p.width / 8;
+  const int tpe = kThreads / epb;
+  const int tid = threadIdx.x;
+  const int slot = tid / tpe;
+  const int local = tid % tpe;
+  const int cvi = local % cv;
+  const int rgi = local / cv;
+  const int b = blockIdx.y;
+  const int E = p.n / p.m;
+  const long long entry = (long long)blockIdx.x * epb + slot;
+  const bool valid = entry < E && rgi < rg;
+  const int R = (p.overlap && entry > 0) ? 2 * p.m : p.m;
+
+  float mx[8], sum[8], acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { mx[j] = -INFINITY; sum[j] = 0.f; acc[j] = 0.f; }
+
+  if (valid) {
+    for (int r = rgi; r < R; r += rg) {
+      const bool a_series = r < p.m;
+      const int j = a_series ? r : r - p.m;
+      const long long tok = a_series ? entry * p.m + j : (entry - 1) * p.m + j;
+      const Tin *zp = row_ptr<Tin>(a_series ? p.Za : p.Zb, p.seq_stride, p.row_stride, b, tok);
+      const Tin *cp = row_ptr<Tin>(a_series ? p.Ca : p.Cb, p.seq_stride, p.row_stride, b, tok);
+      const float *bp = (a_series ? p.Ba : p.Bb) + (long long)j * p.width + cvi * 8;
+      float z[8], cval[8];
+      load8(zp + cvi * 8, z);
+      load8(cp + cvi * 8, cval);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float l = z[q] + bp[q];
+        const float nm = fmaxf(mx[q], l);
+        const float sc = __expf(mx[q] - nm);   // mx = -inf on the first row -> 0
+        const float e = __expf(l - nm);
+        sum[q] = sum[q] * sc + e;
+        acc[q] = acc[q] * sc + e * cval[q];
+        mx[q] = nm;
+      }
+    }
+  }
+  // merge the row-group partials of each entry slot
+  float *pm = sm;                       // [kThreads][8]
+  float *ps = sm + kThreads * 8;        // [kThreads][8]
+  float *pa = sm + 2 * kThreads * 8;    // [kThreads][8]
+  float *red = sm + 3 * kThreads * 8;   // [epb * cv]
+  float *red2 = red + epb * cv;         // [epb * cv]
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    pm[tid * 8 + q] = mx[q];
+    ps[tid * 8 + q] = sum[q];
+    pa[tid * 8 + q] = acc[q];
+  }
+  __syncthreads();
+  float v[8];
+  const bool active = valid && rgi == 0;
+  if (active) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float M = -INFINITY;
+      for (int g = 0; g < rg; ++g) M = fmaxf(M, pm[(slot * tpe + g * cv + cvi) * 8 + q]);
+      float S = 0.f, A = 0.f;
+      for (int g = 0; g < rg; ++g) {
+        const int t = (slot * tpe + g * cv + cvi) * 8 + q;
+        const float sc = (pm[t] == -INFINITY) ? 0.f : __expf(pm[t] - M);
+        S += ps[t] * sc;
+        A += pa[t] * sc;
+      }
+      v[q] = A / S;
+    }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = 0.f;
+  }
+  entry_epilogue<Tout>(p, v, active, slot, cvi, cv, b, entry, entry * p.m, red, red2);
+}
+
+// Prefill leaves the state ready for decode at position n (rows of the last
+// complete block and of the incomplete tail; empty rows (0, -inf)).
+template <typename Tin>
+__global__ void compress_state_prefill_kernel(CompressParams p) {
+  const int b = blockIdx.y;
+  const int m = p.m, W = p.width;
+  const int cutoff = (p.n / m) * m, rem = p.n - cutoff;
+  const int R = p.overlap ? 2 * m : m;
+  const int C = p.overlap ? 2 * W : W;
+  const long long total = (long long)R * C;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(e / C), col = (int)(e % C);
+    long long tok = -1;
+    int j = 0;
+    if (p.overlap) {
+      if (r < m) { if (cutoff >= m) { tok = cutoff - m + r; j = r; } }
+      else if (r - m < rem) { tok = cutoff + (r - m); j = r - m; }
+    } else if (r < rem) { tok = cutoff + r; j = r; }
+    float kv = 0.f, sc = -INFINITY;
+    if (tok >= 0) {
+      const bool b_half = p.overlap && col < W;
+      const int ch = p.overlap ? (b_half ? col : col - W) : col;
+      const Tin *cp = row_ptr<Tin>(b_half ? p.Cb : p.Ca, p.seq_stride, p.row_stride, b, tok);
+      const Tin *zp = row_ptr<Tin>(b_half ? p.Zb : p.Za, p.seq_stride, p.row_stride, b, tok);
+      const float *bp = b_half ? p.Bb : p.Ba;
+      kv = Elt<Tin>::load(cp + ch);
+      sc = Elt<Tin>::load(zp + ch) + bp[(long long)j * W + ch];
+    }
+    const long long off = ((long long)b * R + r) * C + col;
+    p.state_kv[off] = kv;
+    p.state_score[off] = sc;
+  }
+}
+
+// Decode: one block per sequence.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads) compress_decode_kernel(CompressParams p, int pos) {
+  extern __shared__ float sm[];
+  const int b = blockIdx.x;
+  const int m = p.m, W = p.width;
+  const int R = p.overlap ? 2 * m : m;
+  const int C = p.overlap ? 2 * W : W;
+  const int j = pos % m;
+  float *skv = p.state_kv + (long long)b * R * C;
+  float *ssc = p.state_score + (long long)b * R * C;
+  const Tin *ca = row_ptr<Tin>(p.Ca, p.seq_stride, 0, b, 0);
+  const Tin *za = row_ptr<Tin>(p.Za, p.seq_stride, 0, b, 0);
+  // 1. store the token's rows (value, logit + bias)
+  for (int ch = threadIdx.x; ch < W; ch += kThreads) {
+    if (p.overlap) {
+      const Tin *cb = row_ptr<Tin>(p.Cb, p.seq_stride, 0, b, 0);
+      const Tin *zb = row_ptr<Tin>(p.Zb, p.seq_stride, 0, b, 0);
+      const long long row = (long long)(m + j) * C;
+      skv[row + ch] = Elt<Tin>::load(cb + ch);
+      ssc[row + ch] = Elt<Tin>::load(zb + ch) + p.Bb[(long long)j * W + ch];
+      skv[row + W + ch] = Elt<Tin>::load(ca + ch);
+      ssc[row + W + ch] = Elt<Tin>::load(za + ch) + p.Ba[(long long)j * W + ch];
+    } else {
+      const long long row = (long long)j * C;
+      skv[row + ch] = Elt<Tin>::load(ca + ch);
+      ssc[row + ch] = Elt<Tin>::load(za + ch) + p.Ba[(long long)j * W + ch];
+    }
+  }
+  if ((pos + 1) % m != 0) return;   // uniform across the block
+  __syncthreads();
+  // 2. emit the entry: per channel softmax over the block's rows
+  float *ent = sm;                   // [W]
+  float *red = sm + W;               // [W / 8]
+  float *red2 = red + W / 8;         // [W / 8]
+  for (int ch = threadIdx.x; ch < W; ch += kThreads) {
+    float M = -INFINITY;
+    for (int r = 0; r < m; ++r) {
+      if (p.overlap) {
+        M = fmaxf(M, ssc[(long long)r * C + ch]);
+        M = fmaxf(M, ssc[(long long)(m + r) * C + W + ch]);
+      } else {
+        M = fmaxf(M, ssc[(long long)r * C + ch]);
+      }
+    }
+    float S = 0.f, A = 0.f;
+    for (int r = 0; r < m; ++r) {
+      if (p.overlap) {
+        const float e0 = __expf(ssc[(long long)r * C + ch] - M);
+        const float e1 = __expf(ssc[(long long)(m + r) * C + W + ch] - M);
+        S += e0 + e1;
+        A += e0 * skv[(long long)r * C + ch] + e1 * skv[(long long)(m + r) * C + W + ch];
+      } else {
+        const float e0 = __expf(ssc[(long long)r * C + ch] - M);
+        S += e0;
+        A += e0 * skv[(long long)r * C + ch];
+      }
+    }
+    ent[ch] = A / S;
+  }
+  __syncthreads();
+  const int cv = W / 8;
+  const bool active = threadIdx.x < cv;
+  float v[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = active ? ent[threadIdx.x * 8 + q] : 0.f;
+  const long long entry = pos / m;
+  entry_epilogue<Tout>(p, v, active, 0, active ? threadIdx.x : 0, cv, b, entry,
+                       (long long)(pos + 1 - m), red, red2);
+  __syncthreads();
+  // 3. shift the state: the finished block becomes the previous block
+  for (long long e = threadIdx.x; e < (long long)m * C; e += kThreads) {
+    if (p.overlap) {
+      skv[e] = skv[(long long)m * C + e];
+      ssc[e] = ssc[(long long)m * C + e];
+      skv[(long long)m * C + e] = 0.f;
+      ssc[(long long)m * C + e] = -INFINITY;
+    } else {
+      skv[e] = 0.f;
+      ssc[e] = -INFINITY;
+    }
+  }
+}
+
+template <typename Tin>
+int launch_prefill_t(const CompressParams &p, cudaStream_t s) {
+  const int cv = p.width / 8;
+  const int R = p.overlap ? 2 * p.m : p.m;
+  // entries per block: give each entry about cv * R threads, at most kThreads
+  int epb = 1;
+  while (epb < 32 && cv * R * epb * 2 <= kThreads && cv * epb * 2 <= kThreads) epb *= 2;
+  const int tpe = kThreads / epb;
+  int rg = tpe / cv;
+  if (rg > R) rg = R;
+  const int E = p.n / p.m;
+  if (E == 0) return HCA_OK;
+  dim3 grid((E + epb - 1) / epb, p.B);
+  const size_t smem = (size_t)(3 * kThreads * 8 + 2 * epb * cv) * sizeof(float);
+  switch (p.out_dtype) {
+    case HCA_F32: compress_prefill_kernel<Tin, float><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
+    case HCA_BF16: compress_prefill_kernel<Tin, __nv_bfloat16><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
+    default: compress_prefill_kernel<Tin, uint8_t><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
+  }
+  return check_launch("compress_prefill");
+}
+
+template <typename Tin>
+int launch_decode_t(const CompressParams &p, int pos, cudaStream_t s) {
+  const size_t smem = (size_t)(p.width + 2 * (p.width / 8)) * sizeof(float);
+  switch (p.out_dtype) {
+    case HCA_F32: compress_decode_kernel<Tin, float><<<p.B, kThreads, smem, s>>>(p, pos); break;
+    case HCA_BF16: compress_decode_kernel<Tin, __nv_bfloat16><<<p.B, kThreads, smem, s>>>(p, pos); break;
+    default: compress_decode_kernel<Tin, uint8_t><<<p.B, kThreads, smem, s>>>(p, pos); break;
+  }
+  return check_launch("compress_decode");
+}
+
+}  // namespace
+
+int launch_compress_prefill(const CompressParams &p, cudaStream_t s) {
+  return p.in_dtype == HCA_F32 ? launch_prefill_t<float>(p, s)
+                               : launch_prefill_t<__nv_bfloat16>(p, s);
+}
+
+int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s) {
+  dim3 grid(16, p.B);
+  if (p.in_dtype == HCA_F32)
+    compress_state_prefill_kernel<float><<<grid, 256, 0, s>>>(p);
+  else
+    compress_state_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+  return check_launch("compress_state_prefill");
+}
+
+int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s) {
+  return p.in_dtype == HCA_F32 ? launch_decode_t<float>(p, pos, s)
+                               : launch_decode_t<__nv_bfloat16>(p, pos, s);
+}
+
+}  // namespace hca

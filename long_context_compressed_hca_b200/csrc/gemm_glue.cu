@@ -1,0 +1,122 @@
+// gemm_glue.cu -- projections and row-wise glue of the layer path.
+//
+// The projections of juejin "DeepSeek-V4 技术报告简要解读" Eq.(9)-(10), (13)-(15),
+// (18), (20)-(21) and the window-KV projection (1zeryu "DeepSeek-V4：算法架构",
+// "Q, K, V 映射与位置编码注入") are plain GEMMs C = A B^T with weights stored
+// [d_out, d_in].  The row op fuses RMSNorm (optionally per head), partial RoPE,
+// scaling and the storage conversion that follow them.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+
+namespace {
+
+// ------------------------------------------------------------------ SIMT GEMM
+constexpr int BM = 64, BN = 64, BK = 16;
+
+template <typename Tab, typename Tc>
+__global__ void __launch_bounds__(256) gemm_simt(const Tab *A, long long lda, const Tab *B, long long ldb,
+                                                 Tc *C, long long ldc, int M, int N, int K, float alpha) {
+  __shared__ float As[BK][BM + 4];
+  __shared__ float Bs[BK][BN + 4];
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += BK) {
+    for (int e = threadIdx.x; e < BM * BK; e += 256) {
+      const int r = e / BK, kk = e % BK;
+      const int gm = m0 + r, gk = k0 + kk;
+      As[kk][r] = (gm < M && gk < K) ? Elt<Tab>::load(A + (long long)gm * lda + gk) : 0.f;
+      const int gn = n0 + r;
+      Bs[kk][r] = (gn < N && gk < K) ? Elt<Tab>::load(B + (long long)gn * ldb + gk) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * b[j];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx * 4 + j;
+      if (gn < N) Elt<Tc>::store(C + (long long)gm * ldc + gn, acc[i][j] * alpha);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ row op
+template <typename Tout>
+__global__ void row_op_kernel(RowOpParams p) {
+  extern __shared__ float red[];   // [blockDim / 32]
+  const int row = blockIdx.x;
+  const float *in = p.in + (long long)row * p.in_stride;
+  Tout *out = reinterpret_cast<Tout *>(p.out) + (long long)row * p.out_stride;
+  float r = p.scale;
+  if (p.norm) {
+    float ss = 0.f;
+    for (int c = threadIdx.x; c < p.cols; c += blockDim.x) ss += in[c] * in[c];
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
+    r *= rsqrtf(tot / (float)p.cols + p.eps);
+  }
+  const long long pos = (p.pos0 + (long long)(row / p.rows_per_pos)) % p.pos_mod;
+  // each thread handles pairs of columns so that a RoPE pair stays in one thread
+  for (int c = 2 * threadIdx.x; c < p.cols; c += 2 * blockDim.x) {
+    float a = in[c] * r * (p.gamma ? p.gamma[c] : 1.f);
+    float b = in[c + 1] * r * (p.gamma ? p.gamma[c + 1] : 1.f);
+    if (p.rd > 0 && c >= p.cols - p.rd) {
+      float s, cs;
+      rope_sincos(pos, (c - (p.cols - p.rd)) / 2, p.rd, p.theta, &s, &cs);
+      const float a2 = a * cs - b * s, b2 = a * s + b * cs;
+      a = a2; b = b2;
+    }
+    Elt<Tout>::store(out + c, a);
+    Elt<Tout>::store(out + c + 1, b);
+  }
+}
+
+}  // namespace
+
+int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long long ldb, void *C,
+                long long ldc, hca_dtype cdt, int M, int N, int K, float alpha, cudaStream_t s) {
+  if (M == 0 || N == 0) return HCA_OK;
+  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+  if (ab == HCA_F32) {
+    if (cdt == HCA_F32)
+      gemm_simt<float, float><<<grid, 256, 0, s>>>((const float *)A, lda, (const float *)Bm, ldb, (float *)C, ldc, M, N, K, alpha);
+    else
+      gemm_simt<float, __nv_bfloat16><<<grid, 256, 0, s>>>((const float *)A, lda, (const float *)Bm, ldb, (__nv_bfloat16 *)C, ldc, M, N, K, alpha);
+  } else {
+    if (cdt == HCA_F32)
+      gemm_simt<__nv_bfloat16, float><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb, (float *)C, ldc, M, N, K, alpha);
+    else
+      gemm_simt<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb, (__nv_bfloat16 *)C, ldc, M, N, K, alpha);
+  }
+  return check_launch("gemm_simt");
+}
+
+int launch_row_op(const RowOpParams &p, cudaStream_t s) {
+  if (p.rows == 0) return HCA_OK;
+  const int threads = p.cols >= 512 ? 256 : 128;
+  const size_t smem = (threads / 32) * sizeof(float);
+  if (p.out_dtype == HCA_F32) row_op_kernel<float><<<p.rows, threads, smem, s>>>(p);
+  else row_op_kernel<__nv_bfloat16><<<p.rows, threads, smem, s>>>(p);
+  return check_launch("row_op");
+}
+
+}  // namespace hca

@@ -1,0 +1,104 @@
+// internal.h -- host-side declarations shared by the libhca translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/hca.h"
+
+namespace hca {
+
+// Record an error message for hca_last_error() and return `code`.
+int fail(int code, const char *fmt, ...);
+// Map a CUDA error after a launch; counts launches.
+int check_launch(const char *what);
+void count_launch(int n = 1);
+int num_sms();
+// Device address of the status word (HCA_OK or HCA_ERR_TIMEOUT) of the current device.
+int *device_status_ptr();
+
+// ------------------------------------------------------------- compress
+struct CompressParams {
+  int B, n, width, m, overlap, rd, flags;
+  float eps, theta;
+  const void *Ca, *Cb, *Za, *Zb;
+  long long row_stride, seq_stride;
+  const float *Ba, *Bb, *gamma;
+  void *out;
+  float *out_scale;
+  long long out_seq_stride;
+  float *state_kv, *state_score;
+  hca_dtype in_dtype, out_dtype;
+};
+int launch_compress_prefill(const CompressParams &p, cudaStream_t s);
+int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s);
+int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s);
+
+// ------------------------------------------------------------- index + top-k
+struct IndexParams {
+  int B, n_q, start_pos, m, n_hI, c_I, cap, k;
+  const void *qI;          // [B, n_q, n_hI, c_I]
+  const float *wI;         // [B, n_q, n_hI]
+  const void *KI;          // [B, cap, c_I]
+  const float *KI_scale;   // [B, cap] fp8 only
+  hca_dtype q_dtype, key_dtype;
+  float *scores;           // [B, n_q, score_stride]
+  long long score_stride;
+};
+int launch_index_scores(const IndexParams &p, cudaStream_t s);
+
+struct TopkParams {
+  int rows;                // number of score rows
+  int k;
+  const float *scores;     // row r at scores + r*score_stride
+  long long score_stride;
+  const int32_t *cand_idx; // optional explicit indices per element (same layout), else implicit
+  const int *row_len;      // optional per-row valid length (else from visibility)
+  int n_q, start_pos, m;   // visibility: row r -> query (r % n_q) at position start_pos + r % n_q
+  int32_t *idx_out;        // row r at idx_out + r*idx_stride
+  long long idx_stride;
+  float *score_out;        // optional: the selected keys' scores (for two-pass merges)
+  long long elem_offset;   // index offset added to implicit indices (chunked rows)
+};
+int launch_topk(const TopkParams &p, cudaStream_t s);
+size_t topk_workspace_bytes(const IndexParams &p);
+int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
+                   void *ws, size_t ws_bytes, cudaStream_t s);
+
+// ------------------------------------------------------------- attention
+struct AttendParams {
+  int B, n_q, start_pos, n_h, c, rd, w, m, k, cap;
+  int csa;                 // 1: compressed set from idx; 0: all visible entries
+  int win_is_ring;
+  float scale, theta, sink_log2_bias;
+  const void *q;           // [B, n_q, n_h, c]
+  const void *kv_comp;     // [B, cap, c]
+  const int32_t *idx;      // [B, n_q, k]
+  const void *kv_win;      // prefill [B, n_q, c]; ring [B, w, c]
+  const float *sink;       // [n_h]
+  void *o;                 // [B, n_q, n_h, c]
+  hca_dtype dtype;
+  int *status;
+};
+size_t attend_workspace_bytes(const AttendParams &p);
+int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s);
+
+// ------------------------------------------------------------- GEMM / glue
+// C[M, N] = A[M, K] * B[N, K]^T (row-major, lda/ldb/ldc in elements).
+int launch_gemm(hca_dtype ab_dtype, const void *A, long long lda, const void *Bm, long long ldb,
+                void *C, long long ldc, hca_dtype c_dtype, int M, int N, int K, float alpha,
+                cudaStream_t s);
+// Row RMSNorm (optional) + partial RoPE (optional) + convert.  Row r of
+// `rows` rows of `cols` values; the RoPE position is (pos0 + r / rows_per_pos) % pos_mod.
+struct RowOpParams {
+  const float *in; long long in_stride;
+  void *out; long long out_stride; hca_dtype out_dtype;
+  int rows, cols;
+  int norm; const float *gamma; float eps;
+  int rd; float theta; long long pos0; int rows_per_pos; int pos_mod;
+  float scale;
+};
+int launch_row_op(const RowOpParams &p, cudaStream_t s);
+
+}  // namespace hca

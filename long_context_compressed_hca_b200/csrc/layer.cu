@@ -1,0 +1,340 @@
+// layer.cu -- one attention layer end to end: prefill from hidden states and
+// single-token decode over the caller's cache.
+//
+// Prefill (juejin "DeepSeek-V4 技术报告简要解读" §2.3.1-§2.3.3; 1zeryu
+// "DeepSeek-V4：算法架构", Q/K/V 映射, Compressor, Indexer, Sparse Attention):
+//   C/Z = H W_comp^T (fp32)            -> compressed entries (norm, RoPE at i*m)
+//   indexer C/Z = H W_compI^T (CSA)    -> indexer keys
+//   c^Q = RMSNorm(H W_DQ^T); q = per-head RMS(c^Q W_UQ^T), RoPE at t
+//   q^I = c^Q W_IUQ^T, RoPE at t; w^I = H W_w^T * c_I^-1/2 n_hI^-1/2   (CSA)
+//   window kv = RMSNorm(H W_KV^T), RoPE at t
+//   CSA: scores + top-k; attend over window + selected / all visible entries.
+// Decode (Compressor / Indexer decode branches): the token's projected rows
+// are appended to the window ring and the compressor states; an entry is
+// emitted when its block completes; then score, select and attend.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hca {
+namespace {
+
+size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : (t == HCA_BF16 ? 2 : 1); }
+
+struct Carver {
+  char *base;
+  size_t off = 0;
+  explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+  void *take(size_t bytes) {
+    void *p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  }
+};
+
+// Copy the last min(w, n) window rows of every sequence into the ring (slot p % w).
+template <typename T>
+__global__ void ring_fill_kernel(const T *kv, T *ring, int B, int n, int w, int c) {
+  const int b = blockIdx.y;
+  const int first = n > w ? n - w : 0;
+  const int rows = n - first;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < (long long)rows * c;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(e / c), col = (int)(e % c);
+    const int p = first + r;
+    ring[((long long)b * w + p % w) * c + col] = kv[((long long)b * n + p) * c + col];
+  }
+}
+
+template <typename T>
+__global__ void ring_put_kernel(const T *row, T *ring, int w, int c, int slot) {
+  const int b = blockIdx.x;
+  for (int col = threadIdx.x; col < c; col += blockDim.x)
+    ring[((long long)b * w + slot) * c + col] = row[(long long)b * c + col];
+}
+
+struct Plan {
+  // prefill buffers
+  void *CZ, *CZI, *cQ32, *cQ, *q32, *q, *qI32, *qI, *wI, *kv32, *kvw, *kvc, *keyI, *keyI_scale, *idx, *topk_ws;
+  size_t topk_bytes, total;
+  int qchunk;
+};
+
+int plan_prefill(const hca_layer *L, int n, void *ws, Plan &P) {
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA, comp = L->kind != HCA_LAYER_SWA;
+  const long long T = (long long)a.B * n;
+  const int E = comp ? n / a.m : 0;
+  const size_t es = esize(a.dtype);
+  Carver cv(ws);
+  P.CZ = comp ? cv.take(T * (csa ? 4 : 2) * a.c * 4) : nullptr;
+  P.CZI = csa ? cv.take(T * 4 * a.c_I * 4) : nullptr;
+  P.cQ32 = cv.take(T * L->d_c * 4);
+  P.cQ = cv.take(T * L->d_c * es);
+  P.qchunk = (int)(T < 8192 ? T : 8192);
+  P.q32 = cv.take((size_t)P.qchunk * a.n_h * a.c * 4);
+  P.q = cv.take(T * a.n_h * a.c * es);
+  P.qI32 = csa ? cv.take(T * a.n_hI * a.c_I * 4) : nullptr;
+  P.qI = csa ? cv.take(T * a.n_hI * a.c_I * es) : nullptr;
+  P.wI = csa ? cv.take(T * a.n_hI * 4) : nullptr;
+  P.kv32 = cv.take(T * a.c * 4);
+  P.kvw = cv.take(T * a.c * es);
+  P.kvc = comp ? cv.take((size_t)a.B * (E > 0 ? E : 1) * a.c * es) : nullptr;
+  P.keyI = csa ? cv.take((size_t)a.B * (E > 0 ? E : 1) * a.c_I * es) : nullptr;
+  P.keyI_scale = nullptr;
+  P.idx = csa ? cv.take(T * a.k * 4) : nullptr;
+  P.topk_bytes = 0;
+  if (csa) {
+    IndexParams ip{};
+    ip.B = a.B; ip.n_q = n; ip.start_pos = 0; ip.m = a.m; ip.k = a.k; ip.n_hI = a.n_hI; ip.c_I = a.c_I;
+    P.topk_bytes = topk_workspace_bytes(ip);
+  }
+  P.topk_ws = P.topk_bytes ? cv.take(P.topk_bytes) : nullptr;
+  P.total = cv.off;
+  return HCA_OK;
+}
+
+int check_layer(const hca_layer *L) {
+  if (!L) return fail(HCA_ERR_INVALID, "null layer");
+  const hca_attn_desc &a = L->a;
+  if (a.B < 1 || a.n_h < 1 || a.c < 32 || a.c > 512 || a.c % 32 || a.rd % 8 || a.rd > a.c || a.w < 0 || a.m < 1)
+    return fail(HCA_ERR_INVALID, "invalid attention shape");
+  if (a.dtype != HCA_F32 && a.dtype != HCA_BF16) return fail(HCA_ERR_INVALID, "dtype must be f32 or bf16");
+  if (L->kind == HCA_LAYER_CSA) {
+    if (a.k < 1 || a.n_hI < 1 || a.c_I < 8 || a.c_I % 8 || a.rd_I % 8 || a.rd_I > a.c_I)
+      return fail(HCA_ERR_INVALID, "invalid indexer shape");
+    if (a.overlap != 1 && a.overlap != 0) return fail(HCA_ERR_INVALID, "overlap must be 0 or 1");
+  }
+  if (L->kind != HCA_LAYER_CSA && L->kind != HCA_LAYER_HCA && L->kind != HCA_LAYER_SWA)
+    return fail(HCA_ERR_INVALID, "unknown layer kind");
+  if (!L->sink) return fail(HCA_ERR_INVALID, "sink must be non-null");
+  return HCA_OK;
+}
+
+float rope_theta(const hca_attn_desc &a) { return a.rope_theta > 0.f ? a.rope_theta : 10000.f; }
+float eps_of(const hca_attn_desc &a) { return a.eps > 0.f ? a.eps : 1e-6f; }
+
+}  // namespace
+}  // namespace hca
+
+using namespace hca;
+
+extern "C" {
+
+size_t hybrid_layer_forward_workspace_size(const hca_layer *L, int n) {
+  if (check_layer(L) || n < 0) return 0;
+  Plan P{};
+  plan_prefill(L, n, nullptr, P);
+  return P.total;
+}
+
+int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *cache, void *o, void *ws,
+                         size_t ws_bytes, hca_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA, comp = L->kind != HCA_LAYER_SWA;
+  if (n < 0 || !H || !o) return fail(HCA_ERR_INVALID, "H and o must be non-null, n >= 0");
+  if (L->d < 8 || L->d_c < 8) return fail(HCA_ERR_INVALID, "d and d_c must be >= 8");
+  if (!L->W_DQ || !L->W_UQ || !L->W_KV || (comp && (!L->W_comp || !L->B_comp)) ||
+      (csa && (!L->W_compI || !L->B_compI || !L->W_IUQ || !L->W_w)))
+    return fail(HCA_ERR_INVALID, "missing layer weight");
+  Plan P{};
+  plan_prefill(L, n, nullptr, P);
+  if (ws_bytes < P.total || !ws) return fail(HCA_ERR_INVALID, "workspace too small (%zu < %zu)", ws_bytes, P.total);
+  plan_prefill(L, n, ws, P);
+  if (n == 0) return HCA_OK;
+  const int E = comp ? n / a.m : 0;
+  if (cache && comp && cache->cap < E) return fail(HCA_ERR_INVALID, "cache cap < n/m");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long long T = (long long)a.B * n;
+  const hca_dtype dt = a.dtype;
+  const size_t es = esize(dt);
+  const float theta = rope_theta(a), eps = eps_of(a);
+
+  // ---- compressed main KV
+  void *kvc = P.kvc;
+  int cap = E > 0 ? E : 1;
+  if (cache && comp) { kvc = cache->kv_comp; cap = cache->cap; }
+  if (comp) {
+    const int ncz = csa ? 4 : 2;
+    rc = launch_gemm(dt, H, L->d, L->W_comp, L->d, P.CZ, (long long)ncz * a.c, HCA_F32, (int)T, ncz * a.c, L->d, 1.f, s);
+    if (rc) return rc;
+    hca_compress_desc cd{};
+    cd.B = a.B; cd.width = a.c; cd.m = a.m; cd.overlap = csa ? a.overlap : 0; cd.rd = a.rd;
+    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+    cd.in_dtype = HCA_F32; cd.out_dtype = dt;
+    const float *CZ = static_cast<const float *>(P.CZ);
+    const long long rs = (long long)ncz * a.c;
+    const bool ov = cd.overlap != 0;
+    // column blocks: CSA [Ca | Cb | Za | Zb]; HCA [C | Z]
+    rc = csa_compress(&cd, 0, n, CZ, ov ? CZ + a.c : nullptr, CZ + (csa ? 2 : 1) * a.c,
+                      ov ? CZ + 3 * a.c : nullptr, rs, rs * n, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
+                      nullptr, kvc, nullptr, cap, cache ? cache->state_kv : nullptr,
+                      cache ? cache->state_score : nullptr, stream);
+    if (rc) return rc;
+  }
+  // ---- indexer keys
+  void *keyI = P.keyI;
+  float *keyIs = nullptr;
+  hca_dtype kdt = dt;
+  if (csa) {
+    if (cache) { keyI = cache->key_I; keyIs = cache->key_I_scale; kdt = a.idx_key_dtype; }
+    rc = launch_gemm(dt, H, L->d, L->W_compI, L->d, P.CZI, 4LL * a.c_I, HCA_F32, (int)T, 4 * a.c_I, L->d, 1.f, s);
+    if (rc) return rc;
+    hca_compress_desc cd{};
+    cd.B = a.B; cd.width = a.c_I; cd.m = a.m; cd.overlap = a.overlap; cd.rd = a.rd_I;
+    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+    cd.in_dtype = HCA_F32; cd.out_dtype = kdt;
+    const float *CZ = static_cast<const float *>(P.CZI);
+    const long long rs = 4LL * a.c_I;
+    const bool ov = a.overlap != 0;
+    rc = csa_compress(&cd, 0, n, CZ, ov ? CZ + a.c_I : nullptr, CZ + 2 * a.c_I, ov ? CZ + 3 * a.c_I : nullptr, rs,
+                      rs * n, L->B_compI, ov ? L->B_compI + a.m * a.c_I : nullptr, nullptr, keyI, keyIs, cap,
+                      cache ? cache->stateI_kv : nullptr, cache ? cache->stateI_score : nullptr, stream);
+    if (rc) return rc;
+  }
+  // ---- queries
+  rc = launch_gemm(dt, H, L->d, L->W_DQ, L->d, P.cQ32, L->d_c, HCA_F32, (int)T, L->d_c, L->d, 1.f, s);
+  if (rc) return rc;
+  {
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.cQ32); r.in_stride = L->d_c; r.out = P.cQ; r.out_stride = L->d_c;
+    r.out_dtype = dt; r.rows = (int)T; r.cols = L->d_c; r.norm = 1; r.eps = eps; r.rd = 0; r.theta = theta;
+    r.rows_per_pos = 1; r.pos_mod = n; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  const int HC = a.n_h * a.c;
+  for (long long r0 = 0; r0 < T; r0 += P.qchunk) {
+    const int rows = (int)((T - r0) < P.qchunk ? (T - r0) : P.qchunk);
+    rc = launch_gemm(dt, static_cast<const char *>(P.cQ) + r0 * L->d_c * es, L->d_c, L->W_UQ, L->d_c, P.q32, HC,
+                     HCA_F32, rows, HC, L->d_c, 1.f, s);
+    if (rc) return rc;
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.q32); r.in_stride = a.c;
+    r.out = static_cast<char *>(P.q) + r0 * HC * es; r.out_stride = a.c; r.out_dtype = dt;
+    r.rows = rows * a.n_h; r.cols = a.c; r.norm = 1; r.eps = eps; r.rd = a.rd; r.theta = theta;
+    r.pos0 = r0 % n; r.rows_per_pos = a.n_h; r.pos_mod = n; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  if (csa) {
+    const int HI = a.n_hI * a.c_I;
+    rc = launch_gemm(dt, P.cQ, L->d_c, L->W_IUQ, L->d_c, P.qI32, HI, HCA_F32, (int)T, HI, L->d_c, 1.f, s);
+    if (rc) return rc;
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.qI32); r.in_stride = a.c_I; r.out = P.qI; r.out_stride = a.c_I;
+    r.out_dtype = dt; r.rows = (int)T * a.n_hI; r.cols = a.c_I; r.norm = 0; r.rd = a.rd_I; r.theta = theta;
+    r.rows_per_pos = a.n_hI; r.pos_mod = n; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+    const float wscale = 1.0f / sqrtf((float)a.c_I) / sqrtf((float)a.n_hI);
+    rc = launch_gemm(dt, H, L->d, L->W_w, L->d, P.wI, a.n_hI, HCA_F32, (int)T, a.n_hI, L->d, wscale, s);
+    if (rc) return rc;
+  }
+  // ---- window kv
+  rc = launch_gemm(dt, H, L->d, L->W_KV, L->d, P.kv32, a.c, HCA_F32, (int)T, a.c, L->d, 1.f, s);
+  if (rc) return rc;
+  {
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.kv32); r.in_stride = a.c; r.out = P.kvw; r.out_stride = a.c;
+    r.out_dtype = dt; r.rows = (int)T; r.cols = a.c; r.norm = 1; r.eps = eps; r.rd = a.rd; r.theta = theta;
+    r.rows_per_pos = 1; r.pos_mod = n; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  if (cache && a.w > 0 && cache->win) {
+    dim3 g(8, a.B);
+    if (dt == HCA_F32) ring_fill_kernel<float><<<g, 256, 0, s>>>((const float *)P.kvw, (float *)cache->win, a.B, n, a.w, a.c);
+    else ring_fill_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)P.kvw, (__nv_bfloat16 *)cache->win, a.B, n, a.w, a.c);
+    if ((rc = check_launch("ring_fill"))) return rc;
+  }
+  // ---- select + attend
+  hca_attn_desc ad = a;
+  if (csa) {
+    ad.idx_key_dtype = kdt;
+    rc = csa_index_topk(&ad, P.qI, static_cast<const float *>(P.wI), keyI, keyIs, cap, n, 0,
+                        static_cast<int32_t *>(P.idx), nullptr, 0, P.topk_ws, P.topk_bytes, stream);
+    if (rc) return rc;
+    return csa_attend(&ad, P.q, kvc, cap, static_cast<const int32_t *>(P.idx), P.kvw, 0, L->sink, n, 0, o,
+                      nullptr, 0, stream);
+  }
+  if (comp)
+    return hca_attend(&ad, P.q, kvc, cap, P.kvw, 0, L->sink, n, 0, o, nullptr, 0, stream);
+  // pure sliding window: an HCA attend whose compressed set is empty
+  ad.m = n + 1;
+  return hca_attend(&ad, P.q, P.kvw, 1, P.kvw, 0, L->sink, n, 0, o, nullptr, 0, stream);
+}
+
+// ----------------------------------------------------------------- decode
+size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos) {
+  if (check_layer(L) || pos < 0) return 0;
+  size_t b = 0;
+  if (L->kind == HCA_LAYER_CSA) {
+    b += (((size_t)L->a.B * L->a.k * 4) + 255) & ~(size_t)255;
+    b += csa_index_topk_workspace_size(&L->a, 1, pos);
+  }
+  return b + 256;
+}
+
+int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache, int pos, void *o, void *ws,
+                       size_t ws_bytes, hca_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA, comp = L->kind != HCA_LAYER_SWA;
+  if (!x || !cache || !o || pos < 1) return fail(HCA_ERR_INVALID, "x, cache, o must be non-null and pos >= 1");
+  if (!x->q || (a.w > 0 && (!x->kv || !cache->win)) || (comp && (!x->comp || !cache->kv_comp || !cache->state_kv)) ||
+      (csa && (!x->qI || !x->wI || !x->compI || !cache->key_I || !cache->stateI_kv)))
+    return fail(HCA_ERR_INVALID, "missing decode input or cache buffer");
+  const int E = comp ? (pos + 1) / a.m : 0;
+  if (comp && cache->cap < E) return fail(HCA_ERR_INVALID, "cache cap (%d) < entries (%d)", cache->cap, E);
+  const size_t need = hybrid_decode_step_workspace_size(L, pos);
+  if (ws_bytes < need || (need > 256 && !ws)) return fail(HCA_ERR_INVALID, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const hca_dtype dt = a.dtype;
+  const float theta = rope_theta(a), eps = eps_of(a);
+  // 1. window ring
+  if (a.w > 0) {
+    if (dt == HCA_F32) ring_put_kernel<float><<<a.B, 256, 0, s>>>((const float *)x->kv, (float *)cache->win, a.w, a.c, pos % a.w);
+    else ring_put_kernel<__nv_bfloat16><<<a.B, 256, 0, s>>>((const __nv_bfloat16 *)x->kv, (__nv_bfloat16 *)cache->win, a.w, a.c, pos % a.w);
+    if ((rc = check_launch("ring_put"))) return rc;
+  }
+  // 2. compressor states (+ entry emission)
+  if (comp) {
+    hca_compress_desc cd{};
+    cd.B = a.B; cd.width = a.c; cd.m = a.m; cd.overlap = csa ? a.overlap : 0; cd.rd = a.rd;
+    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+    cd.in_dtype = HCA_F32; cd.out_dtype = dt;
+    const int ncz = csa ? 4 : 2;
+    const float *cz = x->comp;
+    const bool ov = cd.overlap != 0;
+    rc = csa_compress(&cd, pos, 1, cz, ov ? cz + a.c : nullptr, cz + (csa ? 2 : 1) * a.c, ov ? cz + 3 * a.c : nullptr,
+                      (long long)ncz * a.c, (long long)ncz * a.c, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
+                      nullptr, cache->kv_comp, nullptr, cache->cap, cache->state_kv, cache->state_score, stream);
+    if (rc) return rc;
+  }
+  if (csa) {
+    hca_compress_desc cd{};
+    cd.B = a.B; cd.width = a.c_I; cd.m = a.m; cd.overlap = a.overlap; cd.rd = a.rd_I;
+    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+    cd.in_dtype = HCA_F32; cd.out_dtype = a.idx_key_dtype;
+    const float *cz = x->compI;
+    const bool ov = a.overlap != 0;
+    rc = csa_compress(&cd, pos, 1, cz, ov ? cz + a.c_I : nullptr, cz + 2 * a.c_I, ov ? cz + 3 * a.c_I : nullptr,
+                      4LL * a.c_I, 4LL * a.c_I, L->B_compI, ov ? L->B_compI + a.m * a.c_I : nullptr, nullptr,
+                      cache->key_I, cache->key_I_scale, cache->cap, cache->stateI_kv, cache->stateI_score, stream);
+    if (rc) return rc;
+    char *w = static_cast<char *>(ws);
+    int32_t *idx = reinterpret_cast<int32_t *>(w);
+    const size_t ib = (((size_t)a.B * a.k * 4) + 255) & ~(size_t)255;
+    rc = csa_index_topk(&a, x->qI, x->wI, cache->key_I, cache->key_I_scale, cache->cap, 1, pos, idx, nullptr, 0,
+                        w + ib, ws_bytes - ib, stream);
+    if (rc) return rc;
+    return csa_attend(&a, x->q, cache->kv_comp, cache->cap, idx, cache->win, 1, L->sink, 1, pos, o, nullptr, 0,
+                      stream);
+  }
+  if (comp)
+    return hca_attend(&a, x->q, cache->kv_comp, cache->cap, cache->win, 1, L->sink, 1, pos, o, nullptr, 0, stream);
+  hca_attn_desc ad = a;
+  ad.m = pos + 2;
+  return hca_attend(&ad, x->q, cache->win, 1, cache->win, 1, L->sink, 1, pos, o, nullptr, 0, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every symbol include/hca.h declares, and
+host-side validation rejects bad calls before anything is launched (no GPU
+needed: invalid calls return before touching the device)."""
+import ctypes
+
+import pytest
+
+from long_context_compressed_hca_b200 import binding as hb
+from long_context_compressed_hca_b200 import build as hbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    hbuild.build()
+    return hb.lib()
+
+
+def test_header_declares_the_hot_path():
+    names = set(hb.header_functions())
+    for f in ("csa_compress", "csa_index_topk", "csa_attend", "hca_attend", "hybrid_layer_forward",
+              "hybrid_decode_step", "hca_last_error", "hca_check_status"):
+        assert f in names, f
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in hb.header_functions():
+        assert hasattr(L, name), name
+    out = __import__("subprocess").run(["nm", "-D", "--defined-only", hb.LIB_PATH],
+                                       capture_output=True, text=True).stdout
+    for name in hb.header_functions():
+        assert f" T {name}" in out, name
+
+
+def test_version(L):
+    assert L.hca_version() >= 1
+
+
+def _bad(rc, text):
+    assert rc == hb.HCA_ERR_INVALID
+    assert text in hb.last_error()
+
+
+def test_compress_rejects_bad_arguments(L):
+    d = hb.compress_desc(1, 12, 4, 1, 0, 0, hb.HCA_F32, hb.HCA_F32)   # width not a multiple of 8
+    _bad(L.csa_compress(ctypes.byref(d), 0, 8, 16, 16, 16, 16, 12, 96, 16, 16, None, 16, None, 2,
+                        None, None, None), "width")
+    d = hb.compress_desc(1, 16, 4, 1, 0, 0, hb.HCA_F32, hb.HCA_F32)
+    _bad(L.csa_compress(ctypes.byref(d), 0, 8, 16, None, 16, 16, 16, 128, 16, 16, None, 16, None, 2,
+                        None, None, None), "overlap needs")
+    _bad(L.csa_compress(ctypes.byref(d), 0, 8, 24, 16, 16, 16, 16, 128, 16, 16, None, 16, None, 2,
+                        None, None, None), "aligned")
+    _bad(L.csa_compress(ctypes.byref(d), 5, 2, 16, 16, 16, 16, 16, 128, 16, 16, None, 16, None, 2,
+                        16, 16, None), "exactly one token")
+    _bad(L.csa_compress(ctypes.byref(d), 5, 1, 16, 16, 16, 16, 16, 128, 16, 16, None, 16, None, 2,
+                        None, None, None), "state")
+    d8 = hb.compress_desc(1, 16, 4, 0, 0, 0, hb.HCA_F32, hb.HCA_FP8E4M3)
+    _bad(L.csa_compress(ctypes.byref(d8), 0, 8, 16, None, 16, None, 16, 128, 16, None, None, 16,
+                        None, 2, None, None, None), "out_scale")
+
+
+def test_attend_rejects_bad_arguments(L):
+    d = hb.attn_desc(1, 4, 64, 16, 8, 4, k=4)
+    # cap smaller than the visible entries
+    _bad(L.hca_attend(ctypes.byref(d), 16, 16, 1, 16, 0, 16, 64, 0, 16, None, 0, None), "cap")
+    # ring window with several queries
+    _bad(L.hca_attend(ctypes.byref(d), 16, 16, 100, 16, 1, 16, 4, 0, 16, None, 0, None), "ring")
+    # token-indexed window at start_pos > 0
+    _bad(L.hca_attend(ctypes.byref(d), 16, 16, 100, 16, 0, 16, 1, 9, 16, None, 0, None), "start_pos")
+    dbad = hb.attn_desc(1, 4, 48, 16, 8, 4, k=4)
+    _bad(L.hca_attend(ctypes.byref(dbad), 16, 16, 100, 16, 0, 16, 4, 0, 16, None, 0, None), "multiple of 32")
+    _bad(L.csa_attend(ctypes.byref(d), 16, 16, 100, None, 16, 0, 16, 4, 0, 16, None, 0, None), "idx")
+
+
+def test_index_rejects_bad_arguments(L):
+    d = hb.attn_desc(1, 4, 64, 16, 8, 4, k=0, n_hI=4, c_I=32, rd_I=16)
+    _bad(L.csa_index_topk(ctypes.byref(d), 16, 16, 16, None, 100, 4, 0, 16, None, 0, None, 0, None), "k must")
+    d = hb.attn_desc(1, 4, 64, 16, 8, 4, k=4, n_hI=4, c_I=32, rd_I=16, idx_key_dtype=hb.HCA_FP8E4M3)
+    _bad(L.csa_index_topk(ctypes.byref(d), 16, 16, 16, None, 100, 4, 0, 16, None, 0, None, 0, None), "KI_scale")
+    d = hb.attn_desc(1, 4, 64, 16, 8, 4, k=4, n_hI=4, c_I=32, rd_I=16)
+    _bad(L.csa_index_topk(ctypes.byref(d), 16, 16, 16, None, 1, 64, 0, 16, None, 0, None, 0, None), "cap")
+
+
+def test_layer_rejects_bad_arguments(L):
+    lay = hb.Layer()
+    lay.kind = hb.HCA_LAYER_CSA
+    lay.a = hb.attn_desc(1, 4, 64, 16, 8, 4, overlap=1, k=4, n_hI=4, c_I=32, rd_I=16)
+    lay.d, lay.d_c = 64, 16
+    lay.sink = 16
+    _bad(L.hybrid_layer_forward(ctypes.byref(lay), 16, 8, None, 16, 16, 1 << 20, None), "missing layer weight")
+    assert L.hybrid_layer_forward_workspace_size(ctypes.byref(lay), 64) > 0

@@ -1,0 +1,252 @@
+"""GPU parity of whole layers: prefill from hidden states (hybrid_layer_forward)
+and single-token decode over a cache (hybrid_decode_step), against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_compressed_hca_b200 import binding as hb
+from long_context_compressed_hca_b200 import synth, workloads
+from long_context_compressed_hca_b200.layer import CacheHandle, LayerHandle, TokenInputs
+from oracle import hca_oracle as O
+from tests.helpers import GAP, TOL, assert_close, to64
+
+pytestmark = pytest.mark.gpu
+F32, BF16 = torch.float32, torch.bfloat16
+
+
+def _w64(W):
+    return {k: to64(v) for k, v in W.items()}
+
+
+def _run_layer(wl, L, dt, cuda, n=None, cache=None):
+    n = n or wl.n
+    W = synth.layer_weights(L, wl.d, wl.d_c, wl.seed, dt)
+    H = synth.hidden_states(wl.B, n, wl.d, wl.seed, dt)
+    lh = LayerHandle(L, W, wl.d, wl.d_c, dt, wl.B, device=cuda)
+    ws = torch.empty(hb.layer_workspace_size(lh.struct, n), dtype=torch.uint8, device=cuda)
+    o = torch.full((wl.B, n, L.n_h, L.c), float("nan"), dtype=dt, device=cuda)
+    hb.hybrid_layer_forward(lh.struct, H.to(cuda), n, cache.struct if cache else None, o, ws)
+    torch.cuda.synchronize()
+    return W, H, o
+
+
+def test_layer_tiny_csa_fp32(cuda):
+    wl = workloads.TINY_CSA
+    L = wl.layers[0]
+    W, H, o = _run_layer(wl, L, F32, cuda)
+    ref = O.layer_prefill(to64(H[0]), _w64(W), L, wl.d_c, return_intermediates=True)
+    ties = 0
+    for t in range(wl.n):
+        V = (t + 1) // L.m
+        if O.topk_gap(ref["scores"][t], L.k) <= GAP and V > L.k:
+            ties += 1
+            continue
+        assert_close(to64(o[0, t]), ref["o"][t], TOL[F32], f"o[{t}]")
+    assert ties < wl.n // 10
+
+
+def test_layer_hca_bf16(cuda):
+    wl = workloads.HCA_PREFILL
+    L = wl.layers[0]
+    n = 2048   # the oracle over all 8192 tokens is covered by the full-size test
+    W, H, o = _run_layer(wl, L, BF16, cuda, n=n)
+    W64 = _w64(W)
+    for b in range(wl.B):
+        toks = np.unique(np.concatenate([np.arange(0, 300), np.arange(n - 300, n),
+                                         np.random.default_rng(b).integers(0, n, 200)]))
+        ref = O.layer_prefill(to64(H[b]), W64, L, wl.d_c, tokens=toks)
+        assert_close(to64(o[b, toks]), ref, TOL[BF16], f"o[b={b}]")
+
+
+def test_layer_csa_bf16_small(cuda):
+    """CSA layer with the 64K workload's attention shapes at a short length."""
+    wl = workloads.CSA_PREFILL.with_(n=1024, d=512, d_c=256)
+    L = wl.layers[0]
+    W, H, o = _run_layer(wl, L, BF16, cuda)
+    toks = np.unique(np.concatenate([np.arange(0, 40), np.arange(wl.n - 40, wl.n),
+                                     np.random.default_rng(3).integers(0, wl.n, 60)]))
+    ref = O.layer_prefill(to64(H[0]), _w64(W), L, wl.d_c, tokens=toks, return_intermediates=True)
+    ties = 0
+    for j, t in enumerate(toks):
+        if O.topk_gap(ref["scores"][j], L.k) <= GAP and (t + 1) // L.m > L.k:
+            ties += 1
+            continue
+        assert_close(to64(o[0, t]), ref["o"][j], TOL[BF16], f"o[{t}]")
+    assert ties <= len(toks) // 10
+
+
+def test_prefill_then_decode_matches_longer_prefill(cuda):
+    """prefill(n) + decode steps n..n+r-1 reproduces prefill(n+r) at those tokens
+    (the cache and compressor states carry everything decode needs)."""
+    wl = workloads.TINY_CSA
+    L = wl.layers[0]
+    n, r = 200, 13
+    W = synth.layer_weights(L, wl.d, wl.d_c, wl.seed, F32, bias_std=0.3)
+    H = synth.hidden_states(wl.B, n + r, wl.d, wl.seed, F32)
+    lh = LayerHandle(L, W, wl.d, wl.d_c, F32, wl.B, device=cuda)
+    cache = CacheHandle(L, wl.B, cap=64, dtype=F32, device=cuda)
+    ws = torch.empty(hb.layer_workspace_size(lh.struct, n), dtype=torch.uint8, device=cuda)
+    o = torch.empty(wl.B, n, L.n_h, L.c, device=cuda)
+    hb.hybrid_layer_forward(lh.struct, H[:, :n].contiguous().to(cuda), n, cache.struct, o, ws)
+    # the decode inputs are the oracle-independent projections of the new tokens,
+    # computed here with torch in fp64 from the same weights (input preparation)
+    W64 = {k: v.double() for k, v in W.items()}
+    Hd = H.double()
+    ref = O.layer_prefill(to64(H[0]), _w64(W), L, wl.d_c, return_intermediates=True)
+    dws = torch.empty(max(hb.decode_workspace_size(lh.struct, n + r), 16), dtype=torch.uint8, device=cuda)
+    for pos in range(n, n + r):
+        h = Hd[:, pos]
+        comp = torch.cat([h @ W64[k].T for k in ("W_aKV", "W_bKV", "W_aZ", "W_bZ")], -1)
+        compI = torch.cat([h @ W64[k].T for k in ("W_IaKV", "W_IbKV", "W_IaZ", "W_IbZ")], -1)
+        x = TokenInputs(q=torch.from_numpy(ref["q"][pos]).float()[None].to(cuda).contiguous(),
+                        kv=torch.from_numpy(ref["kv_win"][pos]).float()[None].to(cuda).contiguous(),
+                        comp=comp.float().to(cuda).contiguous(), compI=compI.float().to(cuda).contiguous(),
+                        qI=torch.from_numpy(ref["qI"][pos]).float()[None].to(cuda).contiguous(),
+                        wI=torch.from_numpy(ref["wI"][pos]).float()[None].to(cuda).contiguous())
+        od = torch.empty(wl.B, L.n_h, L.c, device=cuda)
+        hb.hybrid_decode_step(lh.struct, x.struct, cache.struct, pos, od, dws)
+        torch.cuda.synchronize()
+        if O.topk_gap(ref["scores"][pos], L.k) > GAP:
+            assert_close(to64(od[0]), ref["o"][pos], 1e-4, f"decode o[{pos}]")
+    # emitted entries equal the prefill's entries
+    E = (n + r) // L.m
+    assert_close(to64(cache.kv_comp[0, :E]), ref["kv_comp"][:E], 1e-4, "kv_comp")
+    assert_close(to64(cache.key_I[0, :E]), ref["KI"][:E], 1e-4, "key_I")
+
+
+# ----------------------------------------------------------------- decode step over a synthetic cache
+def _fill_state(state_kv, state_score, overlap, m, width, prev, cur, Ba, Bb):
+    """Write the ABI's compressor-state layout from raw rows (test-side input
+    preparation): prev = (Cb, Zb) of the previous block, cur = (Ca, Cb, Za, Zb)
+    of the current block's earlier tokens."""
+    kv = torch.zeros_like(state_kv)
+    sc = torch.full_like(state_score, float("-inf"))
+    if overlap:
+        if prev is not None:
+            Cb, Zb = prev
+            kv[:, :m, :width] = Cb
+            sc[:, :m, :width] = Zb + Bb[None]
+            kv[:, :m, width:] = 7.0          # unused half of the previous block
+            sc[:, :m, width:] = 3.0
+        Ca, Cb, Za, Zb = cur
+        j = Ca.shape[1]
+        kv[:, m:m + j, :width] = Cb
+        sc[:, m:m + j, :width] = Zb + Bb[None, :j]
+        kv[:, m:m + j, width:] = Ca
+        sc[:, m:m + j, width:] = Za + Ba[None, :j]
+    else:
+        Ca, _, Za, _ = cur
+        j = Ca.shape[1]
+        kv[:, :j] = Ca
+        sc[:, :j] = Za + Ba[None, :j]
+    state_kv.copy_(kv)
+    state_score.copy_(sc)
+
+
+def _bf16_round(x):
+    return torch.from_numpy(np.asarray(x)).to(BF16).double().numpy()
+
+
+def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed, check_ties=True):
+    c, m, w = L.c, L.m, L.w
+    csa = L.kind == "csa"
+    dt = BF16
+    cap = pos // m + 4
+    Ecur = pos // m                          # complete entries before this token
+    W = synth.layer_weights(L, 256, 64, seed, dt, bias_std=0.5)
+    lh = LayerHandle(L, W, 256, 64, dt, B, idx_key_dtype=idx_key_dtype, device=cuda)
+    cache = CacheHandle(L, B, cap, dt, idx_key_dtype=idx_key_dtype, device=cuda)
+    g = lambda shape, s, std=1.0, d=torch.float32: synth.normal(shape, seed, s, std=std, dtype=d)
+    cache.kv_comp.copy_(g((B, cap, c), 100, d=dt))
+    cache.win.copy_(g((B, w, c), 101, d=dt))
+    j = pos % m
+    raw = {nm: g((B, m, c), 102 + i) for i, nm in enumerate(("pCb", "pZb", "Ca", "Cb", "Za", "Zb"))}
+    Ba, Bb = (W["B_a"], W["B_b"]) if csa else (W["B"], None)
+    _fill_state(cache.state_kv, cache.state_score, L.overlap, m, c,
+                (raw["pCb"], raw["pZb"]) if (L.overlap and Ecur > 0) else None,
+                tuple(raw[k][:, :j] for k in ("Ca", "Cb", "Za", "Zb")), Ba.float(),
+                Bb.float() if Bb is not None else None)
+    x = dict(q=g((B, L.n_h, c), 110, d=dt), kv=g((B, c), 111, d=dt), comp=g((B, (4 if csa else 2) * c), 112))
+    if csa:
+        cI = L.c_I
+        KIf = g((B, cap, cI), 120)
+        if idx_key_dtype == "fp8":
+            kb, ks = synth.fp8_rows(KIf)
+            cache.key_I.copy_(kb)
+            cache.key_I_scale.copy_(ks)
+        else:
+            cache.key_I.copy_(KIf.to(dt))
+        rawI = {nm: g((B, m, cI), 130 + i) for i, nm in enumerate(("pCb", "pZb", "Ca", "Cb", "Za", "Zb"))}
+        _fill_state(cache.stateI_kv, cache.stateI_score, L.overlap, m, cI,
+                    (rawI["pCb"], rawI["pZb"]) if Ecur > 0 else None,
+                    tuple(rawI[k][:, :j] for k in ("Ca", "Cb", "Za", "Zb")), W["B_Ia"].float(), W["B_Ib"].float())
+        x.update(qI=g((B, L.n_hI, cI), 113, d=dt), wI=g((B, L.n_hI), 114, std=cI ** -0.5 * L.n_hI ** -0.5),
+                 compI=g((B, 4 * cI), 115))
+    # host copies of the inputs (before the step mutates the cache)
+    kvc0, win0 = to64(cache.kv_comp), to64(cache.win)
+    if csa:
+        if idx_key_dtype == "fp8":
+            KI0 = O.e4m3_to_f64(cache.key_I.cpu().numpy()) * to64(cache.key_I_scale)[..., None]
+        else:
+            KI0 = to64(cache.key_I)
+    xt = TokenInputs(**{k: v.to(cuda).contiguous() for k, v in x.items()})
+    o = torch.full((B, L.n_h, c), float("nan"), dtype=dt, device=cuda)
+    ws = torch.empty(max(hb.decode_workspace_size(lh.struct, pos), 16), dtype=torch.uint8, device=cuda)
+    hb.hybrid_decode_step(lh.struct, xt.struct, cache.struct, pos, o, ws)
+    torch.cuda.synchronize()
+    emit = (pos + 1) % m == 0
+    ties = 0
+    for b in range(B):
+        comp = to64(x["comp"][b])
+        kvc = kvc0[b].copy()
+        if emit:
+            if csa:
+                Ca = np.concatenate([to64(raw["Ca"][b, :j]), comp[None, 0:c]])
+                Za = np.concatenate([to64(raw["Za"][b, :j]), comp[None, 2 * c:3 * c]])
+                prev = (to64(raw["pCb"][b]), to64(raw["pZb"][b])) if Ecur > 0 else (None, None)
+                e = O.decode_new_entry(pos, m, Ca, Za, to64(W["B_a"]), prev[0], prev[1], to64(W["B_b"]))
+            else:
+                Ca = np.concatenate([to64(raw["Ca"][b, :j]), comp[None, 0:c]])
+                Za = np.concatenate([to64(raw["Za"][b, :j]), comp[None, c:2 * c]])
+                e = O.decode_new_entry(pos, m, Ca, Za, to64(W["B"]))
+            e = O.entry_epilogue(e[None], m, first_entry=Ecur, rd=L.rd)[0]
+            assert_close(to64(cache.kv_comp[b, Ecur]), e, 2e-2, "emitted entry")
+            kvc[Ecur] = _bf16_round(e)
+        wpos = O.window_positions(pos, w)
+        win = win0[b].copy()
+        win[pos % w] = to64(x["kv"][b])
+        wrows = win[[p % w for p in wpos]]
+        kw = {}
+        if csa:
+            KI = KI0[b].copy()
+            if emit:
+                cI = L.c_I
+                cI64 = to64(x["compI"][b])
+                Ca = np.concatenate([to64(rawI["Ca"][b, :j]), cI64[None, 0:cI]])
+                Za = np.concatenate([to64(rawI["Za"][b, :j]), cI64[None, 2 * cI:3 * cI]])
+                prev = (to64(rawI["pCb"][b]), to64(rawI["pZb"][b])) if Ecur > 0 else (None, None)
+                e = O.decode_new_entry(pos, m, Ca, Za, to64(W["B_Ia"]), prev[0], prev[1], to64(W["B_Ib"]))
+                e = O.entry_epilogue(e[None], m, first_entry=Ecur, rd=L.rd_I)[0]
+                if idx_key_dtype == "fp8":
+                    sc = np.abs(e).max() / 448.0
+                    KI[Ecur] = O.e4m3_to_f64(O.e4m3_encode(e / sc)) * sc
+                else:
+                    KI[Ecur] = _bf16_round(e)
+            kw = dict(qI_t=to64(x["qI"][b]), w_t=to64(x["wI"][b]), KI=KI)
+            V = (pos + 1) // m
+            scores = O.index_scores(kw["qI_t"], kw["w_t"], KI, V)
+            if O.topk_gap(scores, L.k) <= GAP:
+                ties += 1
+                if check_ties:
+                    continue
+        ref, _ = O.layer_decode(L, pos, to64(x["q"][b]), kvc, wrows, to64(W["sink"]), **kw)
+        assert_close(to64(o[b]), ref, 2e-2, f"decode o[b={b}]")
+    return ties
+
+
+@pytest.mark.parametrize("kind,pos,kdt", [("csa", 2047, "bf16"), ("csa", 2050, "bf16"), ("csa", 3, "bf16"),
+                                           ("csa", 4099, "fp8"), ("csa", 4098, "fp8"),
+                                           ("hca", 4095, "bf16"), ("hca", 5000, "bf16"), ("hca", 130, "bf16")])
+def test_decode_step(cuda, kind, pos, kdt):
+    L = workloads.HYBRID_DECODE_128K.layers[0 if kind == "csa" else 1]
+    run_decode_case(cuda, L, 3, pos, kdt, seed=pos)
