@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid compressed attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline (one JSON line on rank 0): the 128K-context hybrid decode step
+(batch 32; one CSA layer m=4 top-k=512 indexer 8x64, then one HCA layer
+m'=128; 64 heads, KV dim 512, window 128), in us/step.  Sub-objects report
+the 64K CSA prefill (tokens/s of compression + index/top-k + attention; the
+projections are timed separately), the 1M-context decode (fp8 indexer keys)
+and the 8K HCA prefill.  Each carries the roofline of its dominant kernel.
+
+Multi-GPU (torchrun): every rank runs its own replica of the headline
+workload (no data-path collective); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_compressed_hca_b200 import binding as hb  # noqa: E402
+from long_context_compressed_hca_b200 import synth, workloads  # noqa: E402
+from long_context_compressed_hca_b200.layer import CacheHandle, LayerHandle, TokenInputs  # noqa: E402
+
+METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"]
+L2_FLUSH_BYTES = 256 << 20
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- helpers
+def dev_normal(shape, seed, stream, dtype=torch.float32, std=1.0):
+    return synth.normal_on("cuda", shape, seed, stream, std=std, dtype=dtype)
+
+
+def time_steps(step, K, flush_buf, stream, profile=False):
+    """K device-timed steps (CUDA events on `stream`), L2 flushed before each."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if profile:
+        hb.profile_enable(True)
+        hb.profile_collect()
+    l0 = hb.launch_count()
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            flush_buf.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    launches = hb.launch_count() - l0
+    kern = {}
+    if profile:
+        kern = {k: {"launches": v[0], "ms": v[1]} for k, v in hb.profile_collect().items()}
+        hb.profile_enable(False)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    return ms, launches, kern
+
+
+def dist_max(x: float) -> float:
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        t = torch.tensor([x], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+# --------------------------------------------------------------------------- decode
+class DecodeBench:
+    """One decode step per sequence over synthetic caches: CSA layer + HCA layer."""
+
+    def __init__(self, wl, seed_shift=0):
+        self.wl = wl
+        B, pos = wl.B, wl.pos
+        seed = wl.seed + seed_shift
+        self.layers, self.caches, self.inputs, self.outs, self.ws = [], [], [], [], []
+        for li, L in enumerate(wl.layers):
+            W = synth.layer_weights(L, 64, 64, seed, torch.bfloat16, layer_id=li)   # decode reads sink/biases only
+            lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=wl.idx_key_dtype)
+            lcm = 32
+            cap = ((pos // L.m + 8 + lcm - 1) // lcm) * lcm
+            ch = CacheHandle(L, B, cap, torch.bfloat16, idx_key_dtype=wl.idx_key_dtype)
+            s = 1000 * (li + 1)
+            ch.kv_comp.copy_(dev_normal(ch.kv_comp.shape, seed, s + 1, torch.bfloat16))
+            ch.win.copy_(dev_normal(ch.win.shape, seed, s + 2, torch.bfloat16))
+            ch.state_kv.copy_(dev_normal(ch.state_kv.shape, seed, s + 3))
+            ch.state_score.copy_(dev_normal(ch.state_score.shape, seed, s + 4))
+            if L.kind == "csa":
+                kf = dev_normal(ch.key_I.shape, seed, s + 5)
+                if wl.idx_key_dtype == "fp8":
+                    kb, ks = synth.fp8_rows(kf)
+                    ch.key_I.copy_(kb)
+                    ch.key_I_scale.copy_(ks)
+                else:
+                    ch.key_I.copy_(kf.to(torch.bfloat16))
+                ch.stateI_kv.copy_(dev_normal(ch.stateI_kv.shape, seed, s + 6))
+                ch.stateI_score.copy_(dev_normal(ch.stateI_score.shape, seed, s + 7))
+            x = dict(q=dev_normal((B, L.n_h, L.c), seed, s + 10, torch.bfloat16),
+                     kv=dev_normal((B, L.c), seed, s + 11, torch.bfloat16),
+                     comp=dev_normal((B, (4 if L.kind == "csa" else 2) * L.c), seed, s + 12))
+            if L.kind == "csa":
+                x.update(qI=dev_normal((B, L.n_hI, L.c_I), seed, s + 13, torch.bfloat16),
+                         wI=dev_normal((B, L.n_hI), seed, s + 14, std=L.c_I ** -0.5 * L.n_hI ** -0.5),
+                         compI=dev_normal((B, 4 * L.c_I), seed, s + 15))
+            ti = TokenInputs(**x)
+            o = torch.empty(B, L.n_h, L.c, dtype=torch.bfloat16, device="cuda")
+            ws = torch.empty(max(hb.decode_workspace_size(lh.struct, pos), 256), dtype=torch.uint8, device="cuda")
+            self.layers.append(lh)
+            self.caches.append(ch)
+            self.inputs.append(ti)
+            self.outs.append(o)
+            self.ws.append(ws)
+        # pinned host copies for the end-to-end measurement
+        self.host_in = [{k: v.cpu().pin_memory() for k, v in ti.t.items() if v is not None} for ti in self.inputs]
+        self.host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
+
+    def step(self):
+        for lh, ch, ti, o, ws in zip(self.layers, self.caches, self.inputs, self.outs, self.ws):
+            hb.hybrid_decode_step(lh.struct, ti.struct, ch.struct, self.wl.pos, o, ws)
+
+    def step_e2e(self):
+        for i, ti in enumerate(self.inputs):
+            for k, h in self.host_in[i].items():
+                ti.t[k].copy_(h, non_blocking=True)
+        self.step()
+        for o, h in zip(self.outs, self.host_out):
+            h.copy_(o, non_blocking=True)
+
+    def e2e_bytes(self):
+        hi = sum(h.numel() * h.element_size() for d in self.host_in for h in d.values())
+        ho = sum(h.numel() * h.element_size() for h in self.host_out)
+        return hi, ho
+
+    def algorithmic_bytes(self):
+        """Bytes each kernel of the step must move (the HBM roofline's
+        numerators), per launch, and their sum for the whole step."""
+        wl, B, pos = self.wl, self.wl.B, self.wl.pos
+        per = {}
+        for L in wl.layers:
+            V = (pos + 1) // L.m
+            nw = min(L.w, pos + 1)
+            qo = 2 * B * L.n_h * L.c * 2
+            if L.kind == "csa":
+                kb = 1 if wl.idx_key_dtype == "fp8" else 2
+                per["index_scores"] = B * V * (L.c_I * kb + (4 if kb == 1 else 0)) + B * L.n_hI * (L.c_I * 2 + 4)
+                per["attend_csa"] = B * (min(L.k, V) + nw) * L.c * 2 + qo
+            else:
+                per["attend_hca"] = B * (V + nw) * L.c * 2 + qo
+        return sum(per.values()), per
+
+
+def run_decode(wl, K, W, flush, stream, e2e=True):
+    b = DecodeBench(wl)
+    for _ in range(W):
+        b.step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms, launches, _ = time_steps(b.step, K, flush, stream)
+    barrier()
+    torch.cuda.synchronize()
+    # per-kernel times on the same steps (profiling pass)
+    _, _, kern = time_steps(b.step, K, flush, stream, profile=True)
+    res = dict(bench=b, ms=ms, launches=launches, kern=kern)
+    if e2e:
+        for _ in range(2):
+            b.step_e2e()
+        ems, _, _ = time_steps(b.step_e2e, K, flush, stream)
+        res["e2e_ms"] = ems
+    return res
+
+
+# --------------------------------------------------------------------------- prefill
+class PrefillBench:
+    def __init__(self, wl):
+        self.wl = wl
+        L = wl.layers[0]
+        big = synth.layer_weights_on("cuda", L, wl.d, wl.d_c, wl.seed, torch.bfloat16)
+        self.lh = LayerHandle(L, big, wl.d, wl.d_c, torch.bfloat16, wl.B)
+        self.H = dev_normal((wl.B, wl.n, wl.d), wl.seed, synth.STREAMS["H"], torch.bfloat16)
+        self.o = torch.empty(wl.B, wl.n, L.n_h, L.c, dtype=torch.bfloat16, device="cuda")
+        self.ws = torch.empty(hb.layer_workspace_size(self.lh.struct, wl.n), dtype=torch.uint8, device="cuda")
+
+    def step(self):
+        hb.hybrid_layer_forward(self.lh.struct, self.H, self.wl.n, None, self.o, self.ws)
+
+
+ATTN_PATH = ("compress_prefill", "compress_state", "index_scores", "topk", "attend")
+
+
+def prefill_flops(wl):
+    """Algorithmic FLOPs of the attention path (indexer + attention) and the
+    compression bytes, per prefill."""
+    L = wl.layers[0]
+    n, B = wl.n, wl.B
+    att = idx = 0
+    for t in range(n):
+        V = (t + 1) // L.m
+        nc = min(L.k, V) if L.kind == "csa" else V
+        att += (nc + min(L.w, t + 1)) * L.n_h * L.c * 4
+        if L.kind == "csa":
+            idx += V * L.n_hI * L.c_I * 2
+    return B * att, B * idx
+
+
+def run_prefill(wl, K, W, flush, stream):
+    b = PrefillBench(wl)
+    for _ in range(W):
+        b.step()
+    torch.cuda.synchronize()
+    ms, launches, kern = time_steps(b.step, K, flush, stream, profile=True)
+    path_ms = sum(v["ms"] for k, v in kern.items() if k.startswith(ATTN_PATH)) / K
+    glue_ms = sum(v["ms"] for k, v in kern.items() if k.startswith(("gemm", "row_op", "ring"))) / K
+    att_flops, idx_flops = prefill_flops(wl)
+    del b
+    torch.cuda.empty_cache()
+    return dict(ms=ms, launches=launches, kern=kern, path_ms=path_ms, glue_ms=glue_ms,
+                att_flops=att_flops, idx_flops=idx_flops)
+
+
+# --------------------------------------------------------------------------- oracle arm
+def oracle_decode_sample(bench: DecodeBench, n_seq: int):
+    """Time the oracle on `n_seq` sequences of one decode step (both layers)."""
+    import numpy as np
+    from oracle import hca_oracle as O
+
+    wl, pos = bench.wl, bench.wl.pos
+    data = []
+    for li, L in enumerate(wl.layers):
+        ch, ti = bench.caches[li], bench.inputs[li]
+        V = (pos + 1) // L.m
+        per = []
+        for b in range(n_seq):
+            d = dict(q=ti.t["q"][b].double().cpu().numpy(), kvc=ch.kv_comp[b, :V].double().cpu().numpy(),
+                     win=ch.win[b].double().cpu().numpy(), sink=bench.layers[li].t["sink"].double().cpu().numpy())
+            if L.kind == "csa":
+                if wl.idx_key_dtype == "fp8":
+                    d["KI"] = O.e4m3_to_f64(ch.key_I[b, :V].cpu().numpy()) * \
+                        ch.key_I_scale[b, :V].double().cpu().numpy()[:, None]
+                else:
+                    d["KI"] = ch.key_I[b, :V].double().cpu().numpy()
+                d["qI"] = ti.t["qI"][b].double().cpu().numpy()
+                d["wI"] = ti.t["wI"][b].double().cpu().numpy()
+            per.append(d)
+        data.append(per)
+    t0 = time.perf_counter()
+    for li, L in enumerate(wl.layers):
+        for d in data[li]:
+            wrows = d["win"][[p % L.w for p in O.window_positions(pos, L.w)]]
+            kw = dict(qI_t=d["qI"], w_t=d["wI"], KI=d["KI"]) if L.kind == "csa" else {}
+            O.layer_decode(L, pos, d["q"], d["kvc"], wrows, d["sink"], **kw)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- main
+def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, traffic=None):
+    ach = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm"], 4), "traffic": traffic,
+            "peak_source": f"{peaks['src']} (hbm_gbs copy test)"}
+
+
+def roofline_tensor(flops_per_launch, ms_per_launch, peaks, sustained=True, traffic=None):
+    pk = peaks["bf16_sus"] if sustained else peaks["bf16"]
+    ach = flops_per_launch / (ms_per_launch * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s",
+            "frac": round(ach / pk, 4), "traffic": traffic,
+            "peak_source": f"{peaks['src']} bf16 {'sustained' if sustained else 'burst'}"}
+
+
+def kern_ms(kern, prefix, K):
+    tot = sum(v["ms"] for k, v in kern.items() if k.startswith(prefix))
+    n = sum(v["launches"] for k, v in kern.items() if k.startswith(prefix))
+    return tot / max(n, 1), n / K
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only-headline", action="store_true")
+    ap.add_argument("--oracle-seqs", type=int, default=2)
+    args = ap.parse_args()
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    hb.lib()
+    peaks = measured_peaks()
+    wl = workloads.HYBRID_DECODE_128K
+
+    if args.impl == "reference":
+        # the oracle, as it stands, on the headline's config: each step is a
+        # bounded sample (n sequences of the 32), scaled to the whole step
+        if rank != 0:
+            if world > 1:
+                torch.distributed.destroy_process_group()
+            return
+        b = DecodeBench(wl)
+        n = args.oracle_seqs
+        for _ in range(args.warmup):
+            oracle_decode_sample(b, n)
+        times = [oracle_decode_sample(b, n) * wl.B / n * 1e6 for _ in range(args.steps)]
+        v = statistics.mean(times)
+        line = {"metric": METRIC, "value": round(v, 1), "unit": "us/step", "impl": "reference",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3,
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic",
+                "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.pos,
+                           "parallelism": "single process (CPU oracle)"},
+                "cpu_baseline": {"value": round(v, 1), "unit": "us/step", "cores": cpu_cores(), "kind": "oracle",
+                                 "sample": f"{n} of {wl.B} sequences per step (CSA+HCA layer), scaled x{wl.B / n:g}"},
+                "e2e": {"value": round(v, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    stream = torch.cuda.Stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(local if world > 1 else torch.cuda.current_device())
+    clocks.start()
+    head = run_decode(wl, args.steps, args.warmup, flush, stream)
+    clk = clocks.stop()
+    step_ms = statistics.mean(head["ms"])
+    step_ms_max = dist_max(step_ms)
+    e2e_ms = dist_max(statistics.mean(head["e2e_ms"]))
+    tot_bytes, per_bytes = head["bench"].algorithmic_bytes()
+    kern = head["kern"]
+    # dominant kernel of the step (largest share of device time) and its roofline
+    roof = None
+    if kern:
+        dom = max(kern.items(), key=lambda kv: kv[1]["ms"])[0]
+        per_launch_ms = kern[dom]["ms"] / kern[dom]["launches"]
+        key = next((k for k in per_bytes if dom.startswith(k) or k in dom), None)
+        if key is not None:
+            roof = roofline_hbm(per_bytes[key], per_launch_ms, peaks)
+            roof["algorithmic_bytes_per_launch"] = per_bytes[key]
+        else:
+            roof = {"bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s", "frac": None,
+                    "traffic": None}
+        roof["kernel"] = dom
+        roof["share_of_step"] = round(kern[dom]["ms"] / sum(v["ms"] for v in kern.values()), 3)
+    step_roof = roofline_hbm(tot_bytes, step_ms, peaks)
+    hi, ho = head["bench"].e2e_bytes()
+
+    extras = {}
+    if rank == 0 and world == 1:
+        # CPU oracle baseline on a bounded sample of the same workload
+        n = args.oracle_seqs
+        oracle_decode_sample(head["bench"], 1)
+        osec = statistics.mean(oracle_decode_sample(head["bench"], n) for _ in range(2))
+        extras["cpu_baseline"] = {"value": round(osec * wl.B / n * 1e6, 1), "unit": "us/step",
+                                  "cores": cpu_cores(), "kind": "oracle",
+                                  "sample": f"{n} of {wl.B} sequences of one step (CSA+HCA), scaled x{wl.B / n:g}"}
+    del head["bench"]
+    torch.cuda.empty_cache()
+
+    if world == 1 and not args.only_headline:
+        # 1M-context decode
+        d1 = run_decode(workloads.HYBRID_DECODE_1M, args.steps, args.warmup, flush, stream, e2e=False)
+        tb, _ = d1["bench"].algorithmic_bytes()
+        m1 = statistics.mean(d1["ms"])
+        extras["decode_1m"] = {"workload": workloads.HYBRID_DECODE_1M.name, "us_per_step": round(m1 * 1e3, 2),
+                               "roofline_step": roofline_hbm(tb, m1, peaks),
+                               "kernels": {k: round(v["ms"] / args.steps * 1e3, 2) for k, v in d1["kern"].items()}}
+        del d1
+        torch.cuda.empty_cache()
+        # prefill workloads (fewer steps: each is a whole layer)
+        for key, pwl in (("prefill_64k", workloads.CSA_PREFILL), ("hca_prefill", workloads.HCA_PREFILL)):
+            kp = max(3, min(args.steps, 5))
+            r = run_prefill(pwl, kp, 3, flush, stream)
+            att_ms, _ = kern_ms(r["kern"], "attend", kp)
+            toks = pwl.B * pwl.n
+            extras[key] = {
+                "workload": pwl.name,
+                "tokens_per_s": round(toks / (r["path_ms"] * 1e-3), 1),
+                "path_ms": round(r["path_ms"], 3),
+                "projections_ms": round(r["glue_ms"], 3),
+                "layer_ms": round(statistics.mean(r["ms"]), 3),
+                "roofline_attention": roofline_tensor(r["att_flops"], att_ms, peaks),
+                "kernels_ms": {k: round(v["ms"] / kp, 3) for k, v in r["kern"].items()},
+            }
+            if r["idx_flops"]:
+                sc_ms, _ = kern_ms(r["kern"], "index_scores", kp)
+                extras[key]["roofline_index"] = roofline_tensor(r["idx_flops"], sc_ms, peaks)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(step_ms_max * 1e3, 2), "unit": "us/step",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms_max, 5),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.pos,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "layers_per_step": "CSA(m=4,k=512,idx 8x64) + HCA(m'=128)",
+                       "l2": "flushed before every timed step (256 MiB write)"},
+            "roofline": roof,
+            "roofline_step": step_roof,
+            "e2e": {"value": round(e2e_ms * 1e3, 2), "unit": "us/step", "h2d_bytes_per_step": hi,
+                    "d2h_bytes_per_step": ho},
+            "gpu_launches": head["launches"],
+            "clocks": clk,
+            "kernels_us_per_step": {k: round(v["ms"] / args.steps * 1e3, 2) for k, v in kern.items()},
+            "throughput_tokens_per_s": round(wl.B * world / (step_ms_max * 1e-3), 1),
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -234,6 +234,13 @@ int hca_check_status(hca_stream_t stream, int *device_status);
 int hca_version(void);              /* (major << 16) | minor */
 /* Kernels launched by the library since load (per process), for accounting. */
 long long hca_launch_count(void);
+/* Per-kernel timing: with profiling on, every launch is bracketed by CUDA
+ * events on its own stream (do not enable while capturing a CUDA graph).
+ * hca_profile_collect() waits for the recorded events, writes one line per
+ * kernel name "name<TAB>launches<TAB>total_ms\n" into buf (NUL-terminated)
+ * and resets the counters.  Returns HCA_ERR_INVALID if buf is too small. */
+int hca_profile_enable(int on);
+int hca_profile_collect(char *buf, size_t len);
 
 #ifdef __cplusplus
 }

@@ -72,6 +72,8 @@ def _declare(L):
         "hca_version": (I, []),
         "hca_launch_count": (LL, []),
         "hca_check_status": (I, [VP, C.POINTER(C.c_int)]),
+        "hca_profile_enable": (I, [I]),
+        "hca_profile_collect": (I, [C.c_char_p, SZ]),
         "csa_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
                              VP, LL, VP, VP, VP]),
         "csa_index_topk_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
@@ -146,6 +148,21 @@ def device_status(stream=None) -> int:
 
 def launch_count() -> int:
     return lib().hca_launch_count()
+
+
+def profile_enable(on: bool = True):
+    check(lib().hca_profile_enable(int(on)))
+
+
+def profile_collect() -> dict:
+    """{kernel name: (launches, total ms)} since the last collect."""
+    buf = C.create_string_buffer(1 << 16)
+    check(lib().hca_profile_collect(buf, len(buf)))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.split("\t")
+        out[name] = (int(n), float(ms))
+    return out
 
 
 def attn_desc(B, n_h, c, rd, w, m, overlap=0, k=0, n_hI=0, c_I=0, rd_I=0, dtype=HCA_BF16,

@@ -1,6 +1,10 @@
 // api.cu -- the extern "C" entry points of libhca: host-side validation,
 // workspace carving and dispatch to the kernels.  See include/hca.h.
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -30,6 +34,45 @@ int check_launch(const char *what) {
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return HCA_OK;
+}
+
+// ---------------------------------------------------------------- profiler
+namespace {
+struct Pending { const char *name; cudaEvent_t a, b; };
+std::mutex g_pm;
+bool g_prof = false;
+std::vector<Pending> g_pend;
+std::vector<cudaEvent_t> g_free_events;
+std::map<std::string, std::pair<double, long long>> g_acc;
+cudaEvent_t take_event() {
+  if (!g_free_events.empty()) {
+    cudaEvent_t e = g_free_events.back();
+    g_free_events.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+LaunchScope::LaunchScope(const char *n, cudaStream_t s) : name(n), stream(s) {
+  if (!g_prof) return;
+  std::lock_guard<std::mutex> lk(g_pm);
+  cudaEvent_t a = take_event();
+  cudaEventRecord(a, s);
+  slot = (int)g_pend.size();
+  g_pend.push_back({n, a, nullptr});
+}
+
+int LaunchScope::done() {
+  if (slot >= 0) {
+    std::lock_guard<std::mutex> lk(g_pm);
+    cudaEvent_t b = take_event();
+    cudaEventRecord(b, stream);
+    if (slot < (int)g_pend.size()) g_pend[slot].b = b;
+  }
+  return check_launch(name);
 }
 
 int *device_status_ptr() {
@@ -134,6 +177,41 @@ const char *hca_last_error(void) { return t_err; }
 int hca_version(void) { return (0 << 16) | 1; }
 
 long long hca_launch_count(void) { return g_launches.load(); }
+
+int hca_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_pm);
+  g_prof = on != 0;
+  return HCA_OK;
+}
+
+int hca_profile_collect(char *buf, size_t len) {
+  std::lock_guard<std::mutex> lk(g_pm);
+  for (auto &p : g_pend) {
+    if (p.b) {
+      cudaEventSynchronize(p.b);
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+        auto &acc = g_acc[p.name];
+        acc.first += ms;
+        acc.second += 1;
+      }
+      g_free_events.push_back(p.b);
+    }
+    g_free_events.push_back(p.a);
+  }
+  g_pend.clear();
+  if (!buf || len == 0) return HCA_ERR_INVALID;
+  size_t off = 0;
+  buf[0] = 0;
+  for (auto &kv : g_acc) {
+    const int w = snprintf(buf + off, len - off, "%s\t%lld\t%.6f\n", kv.first.c_str(), kv.second.second,
+                           kv.second.first);
+    if (w < 0 || (size_t)w >= len - off) return fail(HCA_ERR_INVALID, "profile buffer too small");
+    off += (size_t)w;
+  }
+  g_acc.clear();
+  return HCA_OK;
+}
 
 int hca_check_status(hca_stream_t stream, int *device_status) {
   if (!device_status) return fail(HCA_ERR_INVALID, "null device_status");

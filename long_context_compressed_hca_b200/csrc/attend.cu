@@ -490,8 +490,9 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
     attr_set = true;
   }
   const int grid = n_units < num_sms() ? n_units : num_sms();
+  LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
   attend_tc<C><<<grid, kThreads, smem, s>>>(p, n_units);
-  return check_launch("attend_tc");
+  return ls_.done();
 }
 }  // namespace tc
 
@@ -516,9 +517,10 @@ int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s)
   }
   dim3 grid(p.B * p.n_q, (p.n_h + kSimtWarps - 1) / kSimtWarps);
   const size_t smem = (size_t)kSimtKT * p.c * sizeof(float);
+  LaunchScope ls_(p.csa ? "attend_csa_simt" : "attend_hca_simt", s);
   if (p.dtype == HCA_F32) attend_simt<float><<<grid, kSimtWarps * 32, smem, s>>>(p);
   else attend_simt<__nv_bfloat16><<<grid, kSimtWarps * 32, smem, s>>>(p);
-  return check_launch("attend_simt");
+  return ls_.done();
 }
 
 }  // namespace hca

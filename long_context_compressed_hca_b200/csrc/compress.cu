@@ -327,23 +327,25 @@ int launch_prefill_t(const CompressParams &p, cudaStream_t s) {
   if (E == 0) return HCA_OK;
   dim3 grid((E + epb - 1) / epb, p.B);
   const size_t smem = (size_t)(3 * kThreads * 8 + 2 * epb * cv) * sizeof(float);
+  LaunchScope ls_("compress_prefill", s);
   switch (p.out_dtype) {
     case HCA_F32: compress_prefill_kernel<Tin, float><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
     case HCA_BF16: compress_prefill_kernel<Tin, __nv_bfloat16><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
     default: compress_prefill_kernel<Tin, uint8_t><<<grid, kThreads, smem, s>>>(p, epb, rg); break;
   }
-  return check_launch("compress_prefill");
+  return ls_.done();
 }
 
 template <typename Tin>
 int launch_decode_t(const CompressParams &p, int pos, cudaStream_t s) {
   const size_t smem = (size_t)(p.width + 2 * (p.width / 8)) * sizeof(float);
+  LaunchScope ls_("compress_decode", s);
   switch (p.out_dtype) {
     case HCA_F32: compress_decode_kernel<Tin, float><<<p.B, kThreads, smem, s>>>(p, pos); break;
     case HCA_BF16: compress_decode_kernel<Tin, __nv_bfloat16><<<p.B, kThreads, smem, s>>>(p, pos); break;
     default: compress_decode_kernel<Tin, uint8_t><<<p.B, kThreads, smem, s>>>(p, pos); break;
   }
-  return check_launch("compress_decode");
+  return ls_.done();
 }
 
 }  // namespace
@@ -355,11 +357,12 @@ int launch_compress_prefill(const CompressParams &p, cudaStream_t s) {
 
 int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s) {
   dim3 grid(16, p.B);
+  LaunchScope ls_("compress_state", s);
   if (p.in_dtype == HCA_F32)
     compress_state_prefill_kernel<float><<<grid, 256, 0, s>>>(p);
   else
     compress_state_prefill_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
-  return check_launch("compress_state_prefill");
+  return ls_.done();
 }
 
 int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s) {

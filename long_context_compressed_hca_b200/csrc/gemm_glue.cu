@@ -96,6 +96,7 @@ int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long
                 long long ldc, hca_dtype cdt, int M, int N, int K, float alpha, cudaStream_t s) {
   if (M == 0 || N == 0) return HCA_OK;
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+  LaunchScope ls_("gemm_simt", s);
   if (ab == HCA_F32) {
     if (cdt == HCA_F32)
       gemm_simt<float, float><<<grid, 256, 0, s>>>((const float *)A, lda, (const float *)Bm, ldb, (float *)C, ldc, M, N, K, alpha);
@@ -107,16 +108,17 @@ int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long
     else
       gemm_simt<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb, (__nv_bfloat16 *)C, ldc, M, N, K, alpha);
   }
-  return check_launch("gemm_simt");
+  return ls_.done();
 }
 
 int launch_row_op(const RowOpParams &p, cudaStream_t s) {
   if (p.rows == 0) return HCA_OK;
   const int threads = p.cols >= 512 ? 256 : 128;
   const size_t smem = (threads / 32) * sizeof(float);
+  LaunchScope ls_("row_op", s);
   if (p.out_dtype == HCA_F32) row_op_kernel<float><<<p.rows, threads, smem, s>>>(p);
   else row_op_kernel<__nv_bfloat16><<<p.rows, threads, smem, s>>>(p);
-  return check_launch("row_op");
+  return ls_.done();
 }
 
 }  // namespace hca

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int ch
   __shared__ uint32_t s_digit;
   __shared__ int s_krem;
 
-  const int row = blockIdx.y, ch = blockIdx.x;
+  const int row = blockIdx.x, ch = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int V;
   if (p.row_len) V = p.row_len[row];
@@ -244,6 +244,7 @@ int launch_index_scores(const IndexParams &p, cudaStream_t s) {
   if (Vmax == 0) return HCA_OK;
   dim3 grid((Vmax + kScoreThreads - 1) / kScoreThreads, (p.n_q + kQB - 1) / kQB, p.B);
   const size_t smem = (size_t)(kQB * p.n_hI * p.c_I + kQB * p.n_hI) * sizeof(float);
+  LaunchScope ls_("index_scores_simt", s);
   if (p.q_dtype == HCA_F32) {
     if (p.key_dtype == HCA_F32) index_scores_simt<float, float><<<grid, kScoreThreads, smem, s>>>(p);
     else index_scores_simt<float, __nv_bfloat16><<<grid, kScoreThreads, smem, s>>>(p);
@@ -251,7 +252,7 @@ int launch_index_scores(const IndexParams &p, cudaStream_t s) {
     if (p.key_dtype == HCA_F32) index_scores_simt<__nv_bfloat16, float><<<grid, kScoreThreads, smem, s>>>(p);
     else index_scores_simt<__nv_bfloat16, __nv_bfloat16><<<grid, kScoreThreads, smem, s>>>(p);
   }
-  return check_launch("index_scores");
+  return ls_.done();
 }
 
 namespace {
@@ -326,8 +327,7 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t.n_q = ip.n_q; t.start_pos = ip.start_pos; t.m = ip.m;
   if (n_chunks <= 1) {
     t.idx_out = idx; t.idx_stride = ip.k;
-    topk_kernel<<<dim3(1, rows), kTopkThreads, (size_t)max(chunk, 1) * 4, s>>>(t, chunk, 1, 0);
-    return check_launch("topk");
+    return HCA_LAUNCH("topk", s, topk_kernel<<<dim3(rows, 1), kTopkThreads, (size_t)max(chunk, 1) * 4, s>>>(t, chunk, 1, 0));
   }
   // pass 1: local winners of each chunk
   const size_t c = (size_t)rows * n_chunks * ip.k;
@@ -335,8 +335,7 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   off += (c * sizeof(int32_t) + 255) & ~(size_t)255;
   float *cscore = reinterpret_cast<float *>(w + off);
   t.idx_out = cidx; t.score_out = cscore; t.idx_stride = (long long)n_chunks * ip.k;
-  topk_kernel<<<dim3(n_chunks, rows), kTopkThreads, (size_t)chunk * 4, s>>>(t, chunk, n_chunks, ip.k);
-  rc = check_launch("topk_pass1");
+  rc = HCA_LAUNCH("topk_pass1", s, topk_kernel<<<dim3(rows, n_chunks), kTopkThreads, (size_t)chunk * 4, s>>>(t, chunk, n_chunks, ip.k));
   if (rc) return rc;
   // pass 2: merge the candidate lists (chunk order == index order)
   const int clen = n_chunks * ip.k;
@@ -346,8 +345,7 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t2.row_len = nullptr; t2.n_q = 1; t2.start_pos = clen - 1; t2.m = 1;   // every row has clen elements
   t2.idx_out = idx; t2.idx_stride = ip.k;
   const size_t smem = (size_t)clen * 4;
-  topk_kernel<<<dim3(1, rows), kTopkThreads, smem, s>>>(t2, clen, 1, 0);
-  return check_launch("topk_pass2");
+  return HCA_LAUNCH("topk_pass2", s, topk_kernel<<<dim3(rows, 1), kTopkThreads, smem, s>>>(t2, clen, 1, 0));
 }
 
 }  // namespace hca

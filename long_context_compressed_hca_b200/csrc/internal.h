@@ -9,6 +9,19 @@
 
 namespace hca {
 
+// Per-kernel timing with CUDA events on the launching stream (off unless
+// hca_profile_enable(1) was called).  Usage:
+//   return HCA_LAUNCH("name", stream, kernel<<<grid, block, smem, stream>>>(args));
+struct LaunchScope {
+  int slot = -1;
+  const char *name;
+  cudaStream_t stream;
+  LaunchScope(const char *name, cudaStream_t s);
+  int done();
+};
+#define HCA_LAUNCH(name, stream, ...) \
+  ([&]() -> int { ::hca::LaunchScope _ls((name), (stream)); __VA_ARGS__; return _ls.done(); }())
+
 // Record an error message for hca_last_error() and return `code`.
 int fail(int code, const char *fmt, ...);
 // Map a CUDA error after a launch; counts launches.

@@ -241,9 +241,10 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
   }
   if (cache && a.w > 0 && cache->win) {
     dim3 g(8, a.B);
+    LaunchScope ls_("ring_fill", s);
     if (dt == HCA_F32) ring_fill_kernel<float><<<g, 256, 0, s>>>((const float *)P.kvw, (float *)cache->win, a.B, n, a.w, a.c);
     else ring_fill_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)P.kvw, (__nv_bfloat16 *)cache->win, a.B, n, a.w, a.c);
-    if ((rc = check_launch("ring_fill"))) return rc;
+    if ((rc = ls_.done())) return rc;
   }
   // ---- select + attend
   hca_attn_desc ad = a;
@@ -292,9 +293,10 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
   const float theta = rope_theta(a), eps = eps_of(a);
   // 1. window ring
   if (a.w > 0) {
+    LaunchScope ls_("ring_put", s);
     if (dt == HCA_F32) ring_put_kernel<float><<<a.B, 256, 0, s>>>((const float *)x->kv, (float *)cache->win, a.w, a.c, pos % a.w);
     else ring_put_kernel<__nv_bfloat16><<<a.B, 256, 0, s>>>((const __nv_bfloat16 *)x->kv, (__nv_bfloat16 *)cache->win, a.w, a.c, pos % a.w);
-    if ((rc = check_launch("ring_put"))) return rc;
+    if ((rc = ls_.done())) return rc;
   }
   // 2. compressor states (+ entry emission)
   if (comp) {

@@ -118,3 +118,46 @@ def layer_weights(L, d: int, d_c: int, seed: int, dtype: torch.dtype,
 
 def hidden_states(B: int, n: int, d: int, seed: int, dtype: torch.dtype) -> torch.Tensor:
     return normal((B, n, d), seed, STREAMS["H"], dtype=dtype)
+
+
+def normal_on(device, shape, seed: int, stream: int, std: float = 1.0,
+              dtype: torch.dtype = torch.float32) -> torch.Tensor:
+    """N(0, std^2) drawn directly on `device` (for large benchmark inputs)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(_sub_seed(seed, stream))
+    x = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x if dtype == torch.float32 else x.to(dtype)
+
+
+def layer_weights_on(device, L, d: int, d_c: int, seed: int, dtype: torch.dtype,
+                     layer_id: int = 0) -> dict:
+    """layer_weights() drawn directly on `device` (large benchmark layers);
+    position biases zero, sinks N(0, L.sink_std^2)."""
+    s = seed * 131 + layer_id
+
+    def w(name, d_out, d_in):
+        return normal_on(device, (d_out, d_in), s, STREAMS[name], std=d_in ** -0.5, dtype=dtype)
+
+    W = {}
+    if L.kind == "csa":
+        for nm in ("W_aKV", "W_bKV", "W_aZ", "W_bZ"):
+            W[nm] = w(nm, L.c, d)
+        W["B_a"] = torch.zeros(L.m, L.c, device=device)
+        W["B_b"] = torch.zeros(L.m, L.c, device=device)
+        for nm in ("W_IaKV", "W_IbKV", "W_IaZ", "W_IbZ"):
+            W[nm] = w(nm, L.c_I, d)
+        W["B_Ia"] = torch.zeros(L.m, L.c_I, device=device)
+        W["B_Ib"] = torch.zeros(L.m, L.c_I, device=device)
+        W["W_IUQ"] = w("W_IUQ", L.n_hI * L.c_I, d_c)
+        W["W_w"] = w("W_w", L.n_hI, d)
+    else:
+        W["W_KVc"], W["W_Zc"] = w("W_KVc", L.c, d), w("W_Zc", L.c, d)
+        W["B"] = torch.zeros(L.m, L.c, device=device)
+    W["W_DQ"] = w("W_DQ", d_c, d)
+    W["W_UQ"] = w("W_UQ", L.n_h * L.c, d_c)
+    W["W_KV"] = w("W_KV", L.c, d)
+    W["sink"] = (normal_on(device, (L.n_h,), s, STREAMS["sink"], std=L.sink_std)
+                 if L.sink_std else torch.zeros(L.n_h, device=device))
+    return W
