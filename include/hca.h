@@ -151,7 +151,10 @@ int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI,
  * q [B, n_q, n_h, c]; kv_comp [B, cap, c]; sink [n_h] fp32; o [B, n_q, n_h, c].
  * kv_win: prefill (win_is_ring == 0, start_pos == 0): [B, n_q, c], row t =
  *   token t; decode (win_is_ring == 1, n_q == 1): [B, w, c] ring, token p in
- *   slot p % w (the caller has already stored token start_pos). */
+ *   slot p % w (the caller has already stored token start_pos).
+ * ws: scratch for split-KV (few queries: each key list is cut across CTAs and
+ *   the fp32 partials are merged); *_attend_workspace_size() gives its size.
+ *   With ws == NULL or too small the call runs unsplit (same result). */
 size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos);
 int csa_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap,
                const int32_t *idx, const void *kv_win, int win_is_ring,
@@ -241,6 +244,16 @@ long long hca_launch_count(void);
  * and resets the counters.  Returns HCA_ERR_INVALID if buf is too small. */
 int hca_profile_enable(int on);
 int hca_profile_collect(char *buf, size_t len);
+/* Diagnostic trace of the tensor-core attention kernel: with enable = 1 the
+ * following attend launches accumulate, summed over CTAs, the SM cycles each
+ * role spends waiting on each pipeline barrier, plus unit / tile / rescale
+ * counts (slot order: producer Q-free, producer stage-free, MMA Q-ready, MMA
+ * tile-ready, MMA S-free, MMA P-ready, MMA O-free, softmax S-ready, softmax
+ * P-buffer-free, softmax rescale wait, softmax epilogue wait, -, epilogue
+ * cycles, total cycles, rescales, units, tiles).  host_counters (n slots,
+ * may be NULL) receives the counters (the call synchronises the device);
+ * enable >= 0 then resets them and sets the mode, enable < 0 only reads. */
+int hca_trace_attend(int enable, unsigned long long *host_counters, int n);
 
 #ifdef __cplusplus
 }

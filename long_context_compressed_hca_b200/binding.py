@@ -74,6 +74,7 @@ def _declare(L):
         "hca_check_status": (I, [VP, C.POINTER(C.c_int)]),
         "hca_profile_enable": (I, [I]),
         "hca_profile_collect": (I, [C.c_char_p, SZ]),
+        "hca_trace_attend": (I, [I, C.POINTER(C.c_ulonglong), I]),
         "csa_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
                              VP, LL, VP, VP, VP]),
         "csa_index_topk_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
@@ -163,6 +164,22 @@ def profile_collect() -> dict:
         name, n, ms = line.split("\t")
         out[name] = (int(n), float(ms))
     return out
+
+
+TRACE_SLOTS = ("prod_q_free", "prod_stage_free", "mma_q_ready", "mma_tile_ready", "mma_s_free",
+               "mma_p_ready", "mma_o_free", "smax_s_ready", "smax_pbuf_free", "smax_rescale_wait",
+               "smax_epi_wait", "-", "epilogue", "total", "rescales", "units", "tiles")
+
+
+def trace_attend(enable: int):
+    """Switch the attention wait-cycle trace on (1) / off (0) and reset it."""
+    check(lib().hca_trace_attend(enable, None, 0))
+
+
+def trace_attend_read() -> dict:
+    buf = (C.c_ulonglong * 32)()
+    check(lib().hca_trace_attend(-1, buf, 32))
+    return {k: int(buf[i]) for i, k in enumerate(TRACE_SLOTS) if k != "-"}
 
 
 def attn_desc(B, n_h, c, rd, w, m, overlap=0, k=0, n_hI=0, c_I=0, rd_I=0, dtype=HCA_BF16,

@@ -9,6 +9,8 @@
 #include <cstdio>
 #include <cstring>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -87,6 +89,27 @@ int *device_status_ptr() {
   return ptr[dev];
 }
 
+int encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                   uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
+      return fail(HCA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return HCA_OK;
+}
+
 int num_sms() {
   static int n = 0;
   if (n == 0) {
@@ -136,6 +159,7 @@ IndexParams index_params(const hca_attn_desc *d, const void *qI, const float *wI
   p.B = d->B; p.n_q = n_q; p.start_pos = start_pos; p.m = d->m; p.n_hI = d->n_hI; p.c_I = d->c_I;
   p.cap = cap; p.k = d->k; p.qI = qI; p.wI = wI; p.KI = KI; p.KI_scale = KI_scale;
   p.q_dtype = d->dtype; p.key_dtype = d->idx_key_dtype;
+  p.status = device_status_ptr();
   return p;
 }
 
@@ -148,6 +172,7 @@ AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv
   p.scale = attn_scale(d); p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
   p.q = q; p.kv_comp = kv_comp; p.idx = idx; p.kv_win = kv_win; p.sink = sink; p.o = o; p.dtype = d->dtype;
   p.status = nullptr;
+  p.nsplit = 1;
   return p;
 }
 
@@ -324,7 +349,6 @@ int csa_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int c
   REQUIRE(idx || n_q == 0, "idx must be non-null");
   AttendParams p = attend_params(d, q, kv_comp, cap, idx, kv_win, win_is_ring, sink, n_q, start_pos, o, 1);
   p.status = device_status_ptr();
-  REQUIRE(ws_bytes >= attend_workspace_bytes(p), "workspace too small");
   return run_attend(p, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -337,7 +361,6 @@ int hca_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int c
   if (rc) return rc;
   AttendParams p = attend_params(d, q, kv_comp, cap, nullptr, kv_win, win_is_ring, sink, n_q, start_pos, o, 0);
   p.status = device_status_ptr();
-  REQUIRE(ws_bytes >= attend_workspace_bytes(p), "workspace too small");
   return run_attend(p, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 

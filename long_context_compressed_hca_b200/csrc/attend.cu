@@ -30,7 +30,7 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct KeySet {
-  int nw, nc, nk, t0, V;
+  int nw, nw4, nc, nk, t0, V;   // window keys, window slots (multiple of 4), compressed, total slots
 };
 
 __device__ __forceinline__ KeySet key_set(const AttendParams &p, int qi) {
@@ -40,8 +40,38 @@ __device__ __forceinline__ KeySet key_set(const AttendParams &p, int qi) {
   k.nw = min(p.w, t + 1);
   k.t0 = t - k.nw + 1;
   k.nc = p.csa ? min(p.k, k.V) : k.V;
+  k.nw4 = k.nw;
   k.nk = k.nw + k.nc;
   return k;
+}
+
+// Key slots of the tensor-core path: window keys in slots [0, nw), padding to
+// a multiple of 4 (masked), compressed keys from slot nw4, so that every
+// group of 4 slots comes from one tensor.
+__device__ __forceinline__ KeySet key_set_tc(const AttendParams &p, int qi) {
+  KeySet k = key_set(p, qi);
+  k.nw4 = (k.nw + 3) & ~3;
+  k.nk = k.nw4 + k.nc;
+  return k;
+}
+
+// Source row of slot kk (window tensor if kk < nw4, else compressed tensor)
+// and whether it is a real key; masked slots point at a valid row.
+__device__ __forceinline__ int slot_row(const AttendParams &p, const KeySet &ks, int b, int qi, int kk,
+                                        bool &valid) {
+  if (kk < ks.nw4) {
+    valid = kk < ks.nw;
+    const int tok = valid ? ks.t0 + kk : ks.t0 + ks.nw - 1;
+    return p.win_is_ring ? b * p.w + tok % p.w : b * p.n_q + tok;
+  }
+  const int slot = kk - ks.nw4;
+  int e = slot;
+  valid = slot < ks.nc;
+  if (valid && p.csa) {
+    e = p.idx[((long long)b * p.n_q + qi) * p.k + slot];
+    valid = e >= 0 && e < ks.V;
+  }
+  return b * p.cap + (valid ? e : 0);
 }
 
 // Row pointer of key `j` of query (b, qi), or nullptr if the slot is empty.
@@ -61,6 +91,91 @@ __device__ __forceinline__ const T *key_row(const AttendParams &p, const KeySet 
     if (e < 0 || e >= ks.V) return nullptr;
   }
   return reinterpret_cast<const T *>(p.kv_comp) + ((long long)b * p.cap + e) * p.c;
+}
+
+// Tile range [j0, j0 + nt) of split `sp` of a query's key list.
+__device__ __forceinline__ void split_range(const KeySet &ks, int nsplit, int sp, int &j0, int &nt) {
+  const int all = (ks.nk + 63) / 64;
+  const int per = (all + nsplit - 1) / nsplit;
+  j0 = sp * per;
+  const int j1 = min(all, j0 + per);
+  nt = j1 > j0 ? j1 - j0 : 0;
+}
+
+// Merge the split partials of one query: o_h = sum_s 2^{m_s-M} O_s /
+// (sum_s 2^{m_s-M} l_s + 2^{sink_h-M}), then the inverse RoPE at t.
+// Block = (query, group of 4 heads); thread = 4 consecutive columns.
+template <typename T>
+__global__ void __launch_bounds__(128) attend_combine(AttendParams p) {
+  __shared__ float wsc[4][32];
+  __shared__ float inv_den[4];
+  __shared__ float rcs[64];          // cos[32], sin[32] of the token's RoPE pairs
+  const int bq = blockIdx.x, hg = blockIdx.y;
+  const int qi = bq % p.n_q, b = bq / p.n_q;
+  const int t = p.start_pos + qi;
+  const KeySet ks = key_set_tc(p, qi);
+  const int C = p.c;
+  if (threadIdx.x < 4) {
+    const int r = hg * 4 + threadIdx.x;
+    const float sink2 = p.sink[r < p.n_h ? r : 0] * kLog2e;
+    float M = sink2;
+    for (int sp = 0; sp < p.nsplit; ++sp) {
+      int j0, nt;
+      split_range(ks, p.nsplit, sp, j0, nt);
+      if (nt) M = fmaxf(M, p.part_ml[(((long long)bq * p.nsplit + sp) * 64 + r) * 2]);
+    }
+    float den = exp2f(sink2 - M);
+    for (int sp = 0; sp < p.nsplit; ++sp) {
+      int j0, nt;
+      split_range(ks, p.nsplit, sp, j0, nt);
+      float w = 0.f;
+      if (nt) {
+        const float *ml = p.part_ml + (((long long)bq * p.nsplit + sp) * 64 + r) * 2;
+        w = exp2f(ml[0] - M);
+        den += w * ml[1];
+      }
+      wsc[threadIdx.x][sp] = w;
+    }
+    inv_den[threadIdx.x] = 1.f / den;
+  } else if (threadIdx.x >= 32 && threadIdx.x - 32 < p.rd / 2) {
+    const int i = threadIdx.x - 32;
+    float sn, cs;
+    rope_sincos(t, i, p.rd, p.theta, &sn, &cs);
+    rcs[i] = cs;
+    rcs[32 + i] = sn;
+  }
+  __syncthreads();
+  const int per_head = C / 4;
+  for (int e = threadIdx.x; e < 4 * per_head; e += blockDim.x) {
+    const int hh = e / per_head, r = hg * 4 + hh;
+    const int col = 4 * (e % per_head);
+    if (r >= p.n_h) continue;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *base = p.part_o + ((long long)bq * p.nsplit * 64 + r) * C + col;
+#pragma unroll 4
+    for (int sp = 0; sp < p.nsplit; ++sp) {
+      const float w = wsc[hh][sp];
+      const float4 v = *reinterpret_cast<const float4 *>(base + (long long)sp * 64 * C);
+      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+    }
+    const float id = inv_den[hh];
+    float v[4] = {acc.x * id, acc.y * id, acc.z * id, acc.w * id};
+    if (col + 4 > C - p.rd) {
+#pragma unroll
+      for (int x = 0; x < 4; x += 2) {
+        if (col + x >= C - p.rd) {
+          const int pi = (col + x - (C - p.rd)) / 2;
+          const float cs = rcs[pi], sn = rcs[32 + pi];
+          const float a = v[x], bb = v[x + 1];
+          v[x] = a * cs + bb * sn;
+          v[x + 1] = -a * sn + bb * cs;
+        }
+      }
+    }
+    T *orow = reinterpret_cast<T *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C + col;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) Elt<T>::store(orow + x, v[x]);
+  }
 }
 
 // ======================================================================= SIMT
@@ -139,12 +254,13 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attend_simt(AttendParams p) {
 
 // ======================================================================= tcgen05
 namespace tc {
+bool g_trace_on = false;
+bool attend_trace_on() { return g_trace_on; }
 constexpr int KT = 64;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp0 = 5;
-constexpr int kProdThreads = 128;
-constexpr int kThreads = (kSoftmaxWarps + 1 + 4) * 32;
+constexpr int kThreads = (kSoftmaxWarps + 1 + 1) * 32;
 constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
 
 struct Bars {
@@ -164,8 +280,18 @@ struct Layout {
   static constexpr uint32_t tmem_cols = C <= 128 ? 128 : (C <= 256 ? 256 : 512);
 };
 
-template <int C>
-__global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_units) {
+// Trace counters (cycles, summed over CTAs) of the tensor-core kernel's waits.
+enum TraceSlot {
+  TR_P_QEMPTY, TR_P_KVEMPTY, TR_M_QFULL, TR_M_KVFULL, TR_M_SEMPTY, TR_M_PFULL, TR_M_OEMPTY,
+  TR_S_SFULL, TR_S_PBUF, TR_S_RESCALE, TR_S_EPI_WAIT, TR_S_TILE, TR_S_EPI, TR_TOTAL, TR_RESCALES, TR_UNITS,
+  TR_TILES, TR_P_ISSUE, TR_COUNT
+};
+__device__ unsigned long long g_attn_trace[32];
+
+template <int C, bool TRACE>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
+          const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmW) {
   using L = Layout<C>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -177,14 +303,25 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto bar = [&](uint64_t &b) { return smem_u32(&b); };
+  unsigned long long tr[TR_COUNT];
+  if (TRACE) for (int i = 0; i < TR_COUNT; ++i) tr[i] = 0;
+  const long long t_start = TRACE ? clock64() : 0;
+  // wait on an mbarrier, adding the cycles spent to trace slot `slot`
+  auto twait = [&](uint32_t b, uint32_t par, int slot) -> bool {
+    if (!TRACE) return mbar_wait(b, par, p.status);
+    const long long t0 = clock64();
+    const bool ok = mbar_wait(b, par, p.status);
+    tr[slot] += clock64() - t0;
+    return ok;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(bars->q_full), kProdThreads);
+    mbar_init(bar(bars->q_full), 1);
     mbar_init(bar(bars->q_empty), 1);
     mbar_init(bar(bars->o_empty), kSoftmaxWarps);
     mbar_init(bar(bars->mma_done), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(bars->kv_full[i]), kProdThreads);
+      mbar_init(bar(bars->kv_full[i]), 1);
       mbar_init(bar(bars->kv_empty[i]), 1);
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->s_empty[i]), kSoftmaxWarps);
@@ -204,48 +341,56 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kProdWarp0) {
-    // ------------------------------------------------------------ gather
+  if (warp == kProdWarp0) {
+    // ------------------------------------------------------------ TMA loads
+    // Q: 64 rows x C by 2-D tiled loads; key rows by gather4 (4 rows x 64
+    // columns per instruction) into the 128B-swizzled tile.  Lane l builds
+    // group l & 15 (slots 4g..4g+3) for half of the 64-column blocks.
     [&]() {
-    const int pt = threadIdx.x - kProdWarp0 * 32;
-    constexpr int CPR = C / 8;                 // 16-byte chunks per row
-    constexpr int RPP = kProdThreads / CPR;    // rows per pass
-    const int chunk = pt % CPR, prow = pt / CPR;
-    const uint32_t kb_off = (chunk / 8) * kTileBytes;
-    const int cc = chunk % 8;
+    constexpr int NKB = C / 64;
+    constexpr int KB_PER_LANE = NKB >= 2 ? NKB / 2 : 1;
+    const int gi = lane & 15, kbh = lane >> 4;
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmC);
+      tma_prefetch_desc(&tmW);
+    }
     uint32_t g = 0, iq = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const int b = u / p.n_q, qi = u % p.n_q;
-      const KeySet ks = key_set(p, qi);
-      const int nt = (ks.nk + KT - 1) / KT;
+      const int bq = u / p.nsplit, sp = u % p.nsplit;
+      const int b = bq / p.n_q, qi = bq % p.n_q;
+      const KeySet ks = key_set_tc(p, qi);
+      int j0, nt;
+      split_range(ks, p.nsplit, sp, j0, nt);
       if (nt == 0) continue;
-      if (!mbar_wait(bar(bars->q_empty), (iq & 1) ^ 1, p.status)) return;
-      const __nv_bfloat16 *qbase = reinterpret_cast<const __nv_bfloat16 *>(p.q) +
-                                   ((long long)b * p.n_q + qi) * p.n_h * C;
-      for (int r = prow; r < 64; r += RPP) {
-        const bool ok = r < p.n_h;
-        const __nv_bfloat16 *src = ok ? qbase + (long long)r * C + chunk * 8 : qbase;
-        cp_async16(sbase + L::q_off + kb_off + sw128_off(r, cc), src, ok ? 16 : 0);
+      if (!twait(bar(bars->q_empty), (iq & 1) ^ 1, TR_P_QEMPTY)) return;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(bars->q_full), NKB * kTileBytes);
+        for (int kb = 0; kb < NKB; ++kb)
+          tma_load_2d(sbase + L::q_off + kb * kTileBytes, &tmQ, kb * 64, (b * p.n_q + qi) * p.n_h, bar(bars->q_full));
       }
-      cp_async_wait_all();
-      fence_proxy_async();
-      mbar_arrive(bar(bars->q_full));
       for (int j = 0; j < nt; ++j, ++g) {
         const int st = g & 1;
-        if (!mbar_wait(bar(bars->kv_empty[st]), ((g >> 1) & 1) ^ 1, p.status)) return;
-        const uint32_t tile = sbase + L::kv_off + st * L::NKB * kTileBytes + kb_off;
-        for (int r = prow; r < KT; r += RPP) {
-          const __nv_bfloat16 *row = key_row<__nv_bfloat16>(p, ks, b, qi, j * KT + r);
-          cp_async16(tile + sw128_off(r, cc), row ? row + chunk * 8 : qbase, row ? 16 : 0);
+        if (!twait(bar(bars->kv_empty[st]), ((g >> 1) & 1) ^ 1, TR_P_KVEMPTY)) return;
+        const int kk0 = (j0 + j) * KT + 4 * gi;
+        bool v;
+        const int r0 = slot_row(p, ks, b, qi, kk0, v), r1 = slot_row(p, ks, b, qi, kk0 + 1, v),
+                  r2 = slot_row(p, ks, b, qi, kk0 + 2, v), r3 = slot_row(p, ks, b, qi, kk0 + 3, v);
+        const CUtensorMap *map = kk0 < ks.nw4 ? &tmW : &tmC;
+        if (lane == 0) mbar_arrive_expect_tx(bar(bars->kv_full[st]), KT * C * 2);
+        __syncwarp();
+        if (NKB >= 2 || kbh == 0) {
+          const uint32_t tile = sbase + L::kv_off + st * NKB * kTileBytes + gi * 512;
+#pragma unroll
+          for (int x = 0; x < KB_PER_LANE; ++x) {
+            const int kb = kbh * KB_PER_LANE + x;
+            tma_gather4(tile + kb * kTileBytes, map, kb * 64, r0, r1, r2, r3, bar(bars->kv_full[st]));
+          }
         }
-        cp_async_wait_all();
-        fence_proxy_async();
-        mbar_arrive(bar(bars->kv_full[st]));
       }
       ++iq;
     }
     }();
-    cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
@@ -257,8 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
       bool ok = true;
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
         const int st = gg & 1;
-        if (!mbar_wait(bar(bars->p_full[st]), (gg >> 1) & 1, p.status)) return false;
-        if (first && !mbar_wait(bar(bars->o_empty), (iq & 1) ^ 1, p.status)) return false;
+        if (!twait(bar(bars->p_full[st]), (gg >> 1) & 1, TR_M_PFULL)) return false;
+        if (first && !twait(bar(bars->o_empty), (iq & 1) ^ 1, TR_M_OEMPTY)) return false;
         tc_fence_after();
         const uint32_t pa = sbase + L::p_off + st * kTileBytes;
         const uint32_t va = sbase + L::kv_off + st * L::NKB * kTileBytes;
@@ -277,20 +422,23 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
         return true;
       };
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int qi = u % p.n_q;
-        const KeySet ks = key_set(p, qi);
-        const int nt = (ks.nk + KT - 1) / KT;
+        const int qi = (u / p.nsplit) % p.n_q;
+        const KeySet ks = key_set_tc(p, qi);
+        int j0, nt;
+        split_range(ks, p.nsplit, u % p.nsplit, j0, nt);
         if (nt == 0) continue;
-        if (!mbar_wait(bar(bars->q_full), iq & 1, p.status)) { ok = false; break; }
+        if (!twait(bar(bars->q_full), iq & 1, TR_M_QFULL)) { ok = false; break; }
+        fence_proxy_async();
         tc_fence_after();
         for (int j = 0; j < nt && ok; ++j) {
           const uint32_t gj = g + j;
           const int st = gj & 1;
           const uint32_t ph = (gj >> 1) & 1;
-          if (!mbar_wait(bar(bars->kv_full[st]), ph, p.status) || !mbar_wait(bar(bars->s_empty[st]), ph ^ 1, p.status)) {
+          if (!twait(bar(bars->kv_full[st]), ph, TR_M_KVFULL) || !twait(bar(bars->s_empty[st]), ph ^ 1, TR_M_SEMPTY)) {
             ok = false;
             break;
           }
+          fence_proxy_async();
           tc_fence_after();
           const uint32_t qa = sbase + L::q_off;
           const uint32_t ka = sbase + L::kv_off + st * L::NKB * kTileBytes;
@@ -324,10 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
     const uint32_t lane_O = (uint32_t)(q4 * 32) << 16;
     uint32_t g = 0, iq = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const int b = u / p.n_q, qi = u % p.n_q;
+      const int bq = u / p.nsplit, sp = u % p.nsplit;
+      const int b = bq / p.n_q, qi = bq % p.n_q;
       const int t = p.start_pos + qi;
-      const KeySet ks = key_set(p, qi);
-      const int nt = (ks.nk + KT - 1) / KT;
+      const KeySet ks = key_set_tc(p, qi);
+      int j0, nt;
+      split_range(ks, p.nsplit, sp, j0, nt);
+      if (nt == 0 && p.nsplit > 1) continue;   // the combine kernel skips empty ranges
       __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
       if (nt == 0) {
         if (r < p.n_h)
@@ -348,11 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
       }
       __syncwarp();
       float m_used = -INFINITY, l = 0.f;
+      if (TRACE) { tr[TR_UNITS] += 1; tr[TR_TILES] += nt; }
       for (int j = 0; j < nt; ++j) {
         const uint32_t gj = g + j;
         const int st = gj & 1;
         const uint32_t ph = (gj >> 1) & 1;
-        if (!mbar_wait(bar(bars->s_full[st]), ph, p.status)) return;
+        if (!twait(bar(bars->s_full[st]), ph, TR_S_SFULL)) return;
         tc_fence_after();
         uint32_t sv[32];
         tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
@@ -361,19 +513,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->s_empty[st]));
-        // this thread's 32 keys: j*64 + half*32 + x
+        // validity of the tile's 64 keys: lane l checks keys l and 32+l, shared by ballot
+        const int kbase = (j0 + j) * KT + half * 32;
+        uint32_t vmask;
+        {
+          const int k0 = (j0 + j) * KT + lane, k1 = k0 + 32;
+          bool v0 = false, v1 = false;
+          if (k0 < ks.nk) slot_row(p, ks, b, qi, k0, v0);
+          if (k1 < ks.nk) slot_row(p, ks, b, qi, k1, v1);
+          const uint32_t m0 = __ballot_sync(0xffffffffu, v0), m1 = __ballot_sync(0xffffffffu, v1);
+          vmask = half ? m1 : m0;
+        }
         float z[32];
         float tmax = -INFINITY;
-        const int kbase = j * KT + half * 32;
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const int kj = kbase + x;
-          bool valid = kj < ks.nk;
-          if (valid && kj >= ks.nw && p.csa) {
-            const int e = p.idx[((long long)b * p.n_q + qi) * p.k + (kj - ks.nw)];
-            valid = e >= 0 && e < ks.V;
-          }
-          z[x] = valid ? __uint_as_float(sv[x]) * zs : -INFINITY;
+          z[x] = ((vmask >> x) & 1u) ? __uint_as_float(sv[x]) * zs : -INFINITY;
           tmax = fmaxf(tmax, z[x]);
         }
         tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
@@ -390,7 +545,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
         if (__any_sync(0xffffffffu, need)) {
           // rescale O rows of this warp after the PV of the previous tile lands
           const uint32_t gp = gj - 1;
-          if (!mbar_wait(bar(bars->pv_done[gp & 1]), (gp >> 1) & 1, p.status)) return;
+          if (TRACE) tr[TR_RESCALES] += 1;
+          if (!twait(bar(bars->pv_done[gp & 1]), (gp >> 1) & 1, TR_S_RESCALE)) return;
           tc_fence_after();
 #pragma unroll 1
           for (int c0 = 0; c0 < C / 2; c0 += 16) {
@@ -413,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
         }
         l += psum;
         // P buffer `st` is free once the PV of tile gj-2 has completed
-        if (!mbar_wait(bar(bars->pv_done[st]), ph ^ 1, p.status)) return;
+        if (!twait(bar(bars->pv_done[st]), ph ^ 1, TR_S_PBUF)) return;
         uint8_t *prow = smem + L::p_off + st * kTileBytes;
 #pragma unroll
         for (int u4 = 0; u4 < 4; ++u4) {
@@ -428,9 +584,37 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
       }
       // -------- epilogue: normalise, inverse RoPE, store
       const uint32_t gl = g + nt - 1;
-      if (!mbar_wait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, p.status)) return;
+      if (!twait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, TR_S_EPI_WAIT)) return;
+      const long long te0 = TRACE ? clock64() : 0;
       tc_fence_after();
       const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      if (p.nsplit > 1) {
+        // unnormalised partial: O rows (fp32), running max (log2 units) and sum
+        const long long slot = (long long)bq * p.nsplit + sp;
+        float *po = p.part_o + (slot * 64 + r) * C;
+        if (half == 0) {
+          p.part_ml[(slot * 64 + r) * 2] = m_used;
+          p.part_ml[(slot * 64 + r) * 2 + 1] = ltot;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < C / 2; c0 += 16) {
+          uint32_t ov[16];
+          tmem_ld_16x32bx2_x16<C / 2>(tmem + lane_O + c0, ov);
+          tmem_ld_wait();
+          float4 *dst = reinterpret_cast<float4 *>(po + half * (C / 2) + c0);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            dst[x] = make_float4(__uint_as_float(ov[4 * x]), __uint_as_float(ov[4 * x + 1]),
+                                 __uint_as_float(ov[4 * x + 2]), __uint_as_float(ov[4 * x + 3]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->o_empty));
+        if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+        g += nt;
+        ++iq;
+        continue;
+      }
       const float sink2 = (r < p.n_h) ? p.sink[r] * kLog2e : 0.f;
       const float inv = 1.f / (ltot + exp2f(sink2 - m_used));
 #pragma unroll 1
@@ -468,10 +652,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bars->o_empty));
+      if (TRACE) tr[TR_S_EPI] += clock64() - te0;
       g += nt;
       ++iq;
     }
     }();
+  }
+  if (TRACE) {
+    tr[TR_TOTAL] = clock64() - t_start;
+    // one thread per role reports: producer thread 0, MMA lane 0, softmax thread 0
+    const bool rep = threadIdx.x == kProdWarp0 * 32 || threadIdx.x == kMmaWarp * 32 || threadIdx.x == 0;
+    if (rep)
+      for (int i = 0; i < TR_COUNT; ++i)
+        if (tr[i]) atomicAdd(&g_attn_trace[i], tr[i]);
   }
   tc_fence_before();
   __syncthreads();
@@ -481,39 +674,89 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc(AttendParams p, int n_u
 
 template <int C>
 int launch_tc(const AttendParams &p, cudaStream_t s) {
-  const int n_units = p.B * p.n_q;
+  const int n_units = p.B * p.n_q * p.nsplit;
   const size_t smem = Layout<C>::bytes;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attend_tc<C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "attend_tc smem attribute: %s", cudaGetErrorString(e));
     attr_set = true;
   }
   const int grid = n_units < num_sms() ? n_units : num_sms();
+  // tensor maps: q rows (box 64 x 64), compressed and window rows (box 1 x 64)
+  CUtensorMap tmQ, tmC, tmW;
+  const void *cbase = p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q);
+  const void *wbase = p.kv_win ? p.kv_win : cbase;
+  const uint64_t crows = p.kv_comp ? (uint64_t)p.B * p.cap : 1;
+  const uint64_t wrows = p.kv_win ? (uint64_t)p.B * (p.win_is_ring ? p.w : p.n_q) : crows;
+  int rc = encode_tmap_2d(&tmQ, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, (uint64_t)p.B * p.n_q * p.n_h, C * 2, 64, 64,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc) rc = encode_tmap_2d(&tmC, cbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, crows, C * 2, 64, 1,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!rc) rc = encode_tmap_2d(&tmW, wbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, wrows, C * 2, 64, 1,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
+  if (rc) return rc;
   LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
-  attend_tc<C><<<grid, kThreads, smem, s>>>(p, n_units);
+  if (attend_trace_on()) attend_tc<C, true><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
+  else attend_tc<C, false><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
   return ls_.done();
 }
 }  // namespace tc
 
 }  // namespace
 
+namespace {
+bool tc_path(const AttendParams &p) {
+  return p.dtype == HCA_BF16 && p.n_h <= 64 && (p.c == 128 || p.c == 256 || p.c == 512) && p.rd <= p.c / 2 &&
+         p.rd % 2 == 0 && p.rd <= 64;
+}
+// Splits per query: enough work units to fill the GPU when there are few queries.
+int choose_splits(const AttendParams &p) {
+  const long long q = (long long)p.B * p.n_q;
+  if (q == 0 || q >= num_sms()) return 1;
+  // longest key list among the queries (the last one)
+  const int t = p.start_pos + p.n_q - 1;
+  const int V = (t + 1) / p.m;
+  const int nk = (p.w < t + 1 ? p.w : t + 1) + (p.csa ? (p.k < V ? p.k : V) : V);
+  const int tiles = (nk + 63) / 64;
+  int ns = (int)((num_sms() + q - 1) / q);
+  if (ns > tiles / 2) ns = tiles / 2;     // keep >= 2 tiles per split
+  if (ns > 32) ns = 32;
+  return ns < 1 ? 1 : ns;
+}
+}  // namespace
+
 size_t attend_workspace_bytes(const AttendParams &p) {
-  (void)p;
-  return 0;
+  if (!tc_path(p)) return 0;
+  const int ns = choose_splits(p);
+  if (ns <= 1) return 0;
+  const size_t q = (size_t)p.B * p.n_q * ns * 64;
+  return ((q * p.c * 4 + 255) & ~(size_t)255) + ((q * 8 + 255) & ~(size_t)255);
 }
 
-int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s) {
-  (void)ws; (void)ws_bytes;
-  if (p.B * p.n_q == 0) return HCA_OK;
-  const bool tc_ok = p.dtype == HCA_BF16 && p.n_h <= 64 && (p.c == 128 || p.c == 256 || p.c == 512) &&
-                     p.rd <= p.c / 2 && p.rd % 2 == 0 && p.rd <= 64;
-  if (tc_ok) {
-    switch (p.c) {
-      case 128: return tc::launch_tc<128>(p, s);
-      case 256: return tc::launch_tc<256>(p, s);
-      default: return tc::launch_tc<512>(p, s);
+int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t s) {
+  if (p_in.B * p_in.n_q == 0) return HCA_OK;
+  AttendParams p = p_in;
+  p.nsplit = 1;
+  if (tc_path(p)) {
+    if (!p.kv_comp) p.cap = 0;   // no visible entries: masked slots then read row 0 of the dummy map
+    const int ns = choose_splits(p);
+    if (ns > 1 && ws && ws_bytes >= attend_workspace_bytes(p)) {
+      p.nsplit = ns;
+      const size_t q = (size_t)p.B * p.n_q * ns * 64;
+      p.part_o = static_cast<float *>(ws);
+      p.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + ((q * p.c * 4 + 255) & ~(size_t)255));
     }
+    int rc;
+    switch (p.c) {
+      case 128: rc = tc::launch_tc<128>(p, s); break;
+      case 256: rc = tc::launch_tc<256>(p, s); break;
+      default: rc = tc::launch_tc<512>(p, s); break;
+    }
+    if (rc || p.nsplit == 1) return rc;
+    return HCA_LAUNCH("attend_combine", s, attend_combine<__nv_bfloat16><<<dim3(p.B * p.n_q, (p.n_h + 3) / 4), 128, 0, s>>>(p));
   }
   dim3 grid(p.B * p.n_q, (p.n_h + kSimtWarps - 1) / kSimtWarps);
   const size_t smem = (size_t)kSimtKT * p.c * sizeof(float);
@@ -524,3 +767,21 @@ int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s)
 }
 
 }  // namespace hca
+
+extern "C" int hca_trace_attend(int enable, unsigned long long *host_counters, int n) {
+  using namespace hca;
+  if (host_counters && n > 0) {
+    unsigned long long buf[32];
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(buf, tc::g_attn_trace, sizeof buf) != cudaSuccess)
+      return fail(HCA_ERR_CUDA, "trace read failed");
+    for (int i = 0; i < n && i < 32; ++i) host_counters[i] = buf[i];
+  }
+  if (enable >= 0) {
+    const unsigned long long zero[32] = {0};
+    if (cudaMemcpyToSymbol(tc::g_attn_trace, zero, sizeof zero) != cudaSuccess)
+      return fail(HCA_ERR_CUDA, "trace reset failed");
+    tc::g_trace_on = enable != 0;
+  }
+  return HCA_OK;
+}

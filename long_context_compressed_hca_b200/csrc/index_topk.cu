@@ -318,7 +318,8 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   size_t off = ((size_t)rows * (size_t)Vmax * sizeof(float) + 255) & ~(size_t)255;
   int rc = ensure_topk_smem();
   if (rc) return rc;
-  rc = launch_index_scores(p, s);
+  rc = launch_index_scores_tc(p, s);
+  if (rc == HCA_ERR_UNSUPPORTED) rc = launch_index_scores(p, s);
   if (rc) return rc;
   const int chunk = topk_chunk_for(rows, Vmax, ip.k);
   const int n_chunks = Vmax > 0 ? (Vmax + chunk - 1) / chunk : 1;

@@ -1,6 +1,7 @@
 // internal.h -- host-side declarations shared by the libhca translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -28,6 +29,12 @@ int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);
 void count_launch(int n = 1);
 int num_sms();
+// Encode a 2-D tiled TMA descriptor over a row-major matrix (rows x cols
+// elements of elem_bytes, rows row_stride_bytes apart); box = box_rows x
+// box_cols elements.  Returns HCA_OK or HCA_ERR_CUDA.
+int encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint64_t cols,
+                   uint64_t rows, uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows,
+                   CUtensorMapSwizzle swizzle);
 // Device address of the status word (HCA_OK or HCA_ERR_TIMEOUT) of the current device.
 int *device_status_ptr();
 
@@ -58,8 +65,11 @@ struct IndexParams {
   hca_dtype q_dtype, key_dtype;
   float *scores;           // [B, n_q, score_stride]
   long long score_stride;
+  int *status;
 };
 int launch_index_scores(const IndexParams &p, cudaStream_t s);
+// tcgen05 scorer; returns HCA_ERR_UNSUPPORTED (launching nothing) for shapes it does not cover.
+int launch_index_scores_tc(const IndexParams &p, cudaStream_t s);
 
 struct TopkParams {
   int rows;                // number of score rows
@@ -93,6 +103,12 @@ struct AttendParams {
   void *o;                 // [B, n_q, n_h, c]
   hca_dtype dtype;
   int *status;
+  // split-KV: each query's key list is cut into nsplit tile ranges whose
+  // unnormalised partials (fp32 O rows, running max and sum) go to part_o /
+  // part_ml and are merged by a combine kernel
+  int nsplit;
+  float *part_o;           // [B*n_q, nsplit, 64, c]
+  float *part_ml;          // [B*n_q, nsplit, 64, 2]
 };
 size_t attend_workspace_bytes(const AttendParams &p);
 int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s);

@@ -271,7 +271,9 @@ size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos) {
     b += (((size_t)L->a.B * L->a.k * 4) + 255) & ~(size_t)255;
     b += csa_index_topk_workspace_size(&L->a, 1, pos);
   }
-  return b + 256;
+  const size_t att = L->kind == HCA_LAYER_CSA ? csa_attend_workspace_size(&L->a, 1, pos)
+                                              : hca_attend_workspace_size(&L->a, 1, pos);
+  return ((b + 255) & ~(size_t)255) + att + 256;
 }
 
 int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache, int pos, void *o, void *ws,
@@ -326,14 +328,17 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
     char *w = static_cast<char *>(ws);
     int32_t *idx = reinterpret_cast<int32_t *>(w);
     const size_t ib = (((size_t)a.B * a.k * 4) + 255) & ~(size_t)255;
+    const size_t tb = csa_index_topk_workspace_size(&a, 1, pos);
     rc = csa_index_topk(&a, x->qI, x->wI, cache->key_I, cache->key_I_scale, cache->cap, 1, pos, idx, nullptr, 0,
-                        w + ib, ws_bytes - ib, stream);
+                        w + ib, tb, stream);
     if (rc) return rc;
-    return csa_attend(&a, x->q, cache->kv_comp, cache->cap, idx, cache->win, 1, L->sink, 1, pos, o, nullptr, 0,
-                      stream);
+    const size_t ab = (ib + tb + 255) & ~(size_t)255;
+    return csa_attend(&a, x->q, cache->kv_comp, cache->cap, idx, cache->win, 1, L->sink, 1, pos, o, w + ab,
+                      ws_bytes - ab, stream);
   }
   if (comp)
-    return hca_attend(&a, x->q, cache->kv_comp, cache->cap, cache->win, 1, L->sink, 1, pos, o, nullptr, 0, stream);
+    return hca_attend(&a, x->q, cache->kv_comp, cache->cap, cache->win, 1, L->sink, 1, pos, o, ws, ws_bytes,
+                      stream);
   hca_attn_desc ad = a;
   ad.m = pos + 2;
   return hca_attend(&ad, x->q, cache->win, 1, cache->win, 1, L->sink, 1, pos, o, nullptr, 0, stream);

@@ -150,6 +150,8 @@ IDX_CASES = [
     (3, 1, 50000, 4, 512, 8, 64, BF16, "bf16"),      # decode-like: chunked two-pass select
     (2, 1, 70001, 4, 1024, 8, 64, BF16, "fp8"),
     (2, 5, 1000, 4, 40, 8, 64, BF16, "fp8"),
+    (1, 40, 0, 4, 16, 8, 64, BF16, "fp8"),            # prefill-shaped blocks with fp8 keys
+    (2, 530, 100, 4, 64, 8, 64, BF16, "bf16"),        # several 16-query blocks, ragged tail
 ]
 
 
