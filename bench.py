@@ -83,12 +83,11 @@ def dev_normal(shape, seed, stream, dtype=torch.float32, std=1.0):
     return synth.normal_on("cuda", shape, seed, stream, std=std, dtype=dtype)
 
 
-def time_steps(step, K, flush_buf, stream, profile=False):
-    """K device-timed steps (CUDA events on `stream`), L2 flushed before each."""
+def time_steps(step, K, flush_buf, stream, profile=False, replayed=False):
+    """K device-timed steps (CUDA events on `stream`), L2 flushed before each.
+    With profile=True the library's per-kernel events are sampled after every
+    step (this pass is for the per-kernel breakdown, not for the step time)."""
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    if profile:
-        hb.profile_enable(True)
-        hb.profile_collect()
     l0 = hb.launch_count()
     with torch.cuda.stream(stream):
         for i in range(K):
@@ -96,14 +95,27 @@ def time_steps(step, K, flush_buf, stream, profile=False):
             evs[i][0].record(stream)
             step()
             evs[i][1].record(stream)
+            if profile and replayed:
+                hb.profile_sample()        # a replayed graph re-records the same events
     torch.cuda.synchronize()
+    if profile and not replayed:
+        hb.profile_sample()
     launches = hb.launch_count() - l0
     kern = {}
     if profile:
         kern = {k: {"launches": v[0], "ms": v[1]} for k, v in hb.profile_collect().items()}
-        hb.profile_enable(False)
     ms = [a.elapsed_time(b) for a, b in evs]
     return ms, launches, kern
+
+
+def profiled(fn):
+    """Run fn with the library's per-kernel event profiling switched on."""
+    hb.profile_enable(True)
+    hb.profile_collect()
+    try:
+        return fn()
+    finally:
+        hb.profile_enable(False)
 
 
 def dist_max(x: float) -> float:
@@ -169,8 +181,20 @@ class DecodeBench:
         self.host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
 
     def step(self):
-        for lh, ch, ti, o, ws in zip(self.layers, self.caches, self.inputs, self.outs, self.ws):
-            hb.hybrid_decode_step(lh.struct, ti.struct, ch.struct, self.wl.pos, o, ws)
+        """CSA layer on the current stream, HCA layer on a side stream (the two
+        layers of the step are independent), joined before returning."""
+        cur = torch.cuda.current_stream()
+        if not hasattr(self, "side"):
+            self.side = torch.cuda.Stream()
+            self.fork, self.join = torch.cuda.Event(), torch.cuda.Event()
+        self.fork.record(cur)
+        self.side.wait_event(self.fork)
+        for i, (lh, ch, ti, o, ws) in enumerate(zip(self.layers, self.caches, self.inputs, self.outs, self.ws)):
+            st = cur if i == 0 else self.side
+            with torch.cuda.stream(st):
+                hb.hybrid_decode_step(lh.struct, ti.struct, ch.struct, self.wl.pos, o, ws)
+        self.join.record(self.side)
+        cur.wait_event(self.join)
 
     def step_e2e(self):
         for i, ti in enumerate(self.inputs):
@@ -203,24 +227,61 @@ class DecodeBench:
         return sum(per.values()), per
 
 
+def capture_graph(fn, stream):
+    """Capture fn's launches (all on `stream`) into a CUDA graph; returns replay()."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()                       # warm the host-side caches outside capture
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def run_decode(wl, K, W, flush, stream, e2e=True):
     b = DecodeBench(wl)
     for _ in range(W):
         b.step()
     torch.cuda.synchronize()
+    # the decode step's launches replayed as one CUDA graph
+    l0 = hb.launch_count()
+    graph = capture_graph(b.step, stream)
+    per_step_launches = (hb.launch_count() - l0) // 2
+    for _ in range(W):
+        graph.replay()
+    torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms, launches, _ = time_steps(b.step, K, flush, stream)
+    ms, _, _ = time_steps(graph.replay, K, flush, stream)
+    launches = per_step_launches * K
     barrier()
     torch.cuda.synchronize()
-    # per-kernel times on the same steps (profiling pass)
-    _, _, kern = time_steps(b.step, K, flush, stream, profile=True)
-    res = dict(bench=b, ms=ms, launches=launches, kern=kern)
+    # per-kernel times: a second graph captured with the library's event
+    # profiling on, replayed K times
+    def prof_pass():
+        hb.profile_enable(True)
+        pg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pg, stream=stream):
+            b.step()
+        torch.cuda.synchronize()
+        return time_steps(pg.replay, K, flush, stream, profile=True, replayed=True)[2]
+    kern = profiled(prof_pass)
+    res = dict(bench=b, ms=ms, launches=launches, kern=kern, graph=True)
     if e2e:
+        # end to end: host inputs -> device, the step (graph), outputs -> host
+        def e2e_step():
+            for i, ti in enumerate(b.inputs):
+                for k, h in b.host_in[i].items():
+                    ti.t[k].copy_(h, non_blocking=True)
+            graph.replay()
+            for o, h in zip(b.outs, b.host_out):
+                h.copy_(o, non_blocking=True)
         for _ in range(2):
-            b.step_e2e()
-        ems, _, _ = time_steps(b.step_e2e, K, flush, stream)
+            e2e_step()
+        ems, _, _ = time_steps(e2e_step, K, flush, stream)
         res["e2e_ms"] = ems
+    del graph
     return res
 
 
@@ -262,7 +323,7 @@ def run_prefill(wl, K, W, flush, stream):
     for _ in range(W):
         b.step()
     torch.cuda.synchronize()
-    ms, launches, kern = time_steps(b.step, K, flush, stream, profile=True)
+    ms, launches, kern = profiled(lambda: time_steps(b.step, K, flush, stream, profile=True))
     path_ms = sum(v["ms"] for k, v in kern.items() if k.startswith(ATTN_PATH)) / K
     glue_ms = sum(v["ms"] for k, v in kern.items() if k.startswith(("gemm", "row_op", "ring"))) / K
     att_flops, idx_flops = prefill_flops(wl)
@@ -465,7 +526,8 @@ def main():
             "config": {"workload": wl.name, "global_batch": wl.B * world, "seq_len": wl.pos,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "layers_per_step": "CSA(m=4,k=512,idx 8x64) + HCA(m'=128)",
-                       "l2": "flushed before every timed step (256 MiB write)"},
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": "decode step replayed as one CUDA graph; CSA and HCA layers on two streams"},
             "roofline": roof,
             "roofline_step": step_roof,
             "e2e": {"value": round(e2e_ms * 1e3, 2), "unit": "us/step", "h2d_bytes_per_step": hi,

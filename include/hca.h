@@ -238,11 +238,15 @@ int hca_version(void);              /* (major << 16) | minor */
 /* Kernels launched by the library since load (per process), for accounting. */
 long long hca_launch_count(void);
 /* Per-kernel timing: with profiling on, every launch is bracketed by CUDA
- * events on its own stream (do not enable while capturing a CUDA graph).
- * hca_profile_collect() waits for the recorded events, writes one line per
- * kernel name "name<TAB>launches<TAB>total_ms\n" into buf (NUL-terminated)
- * and resets the counters.  Returns HCA_ERR_INVALID if buf is too small. */
+ * events recorded on its own stream (also inside a CUDA graph capture, where
+ * the records become graph nodes).  hca_profile_sample() waits for the
+ * recorded events and adds their durations to per-kernel counters, keeping
+ * the records (call it after each replay of a captured graph, or after each
+ * step).  hca_profile_collect() writes one line per kernel name
+ * "name<TAB>launches<TAB>total_ms\n" into buf (NUL-terminated), then clears
+ * the counters and the records.  Returns HCA_ERR_INVALID if buf is too small. */
 int hca_profile_enable(int on);
+int hca_profile_sample(void);
 int hca_profile_collect(char *buf, size_t len);
 /* Diagnostic trace of the tensor-core attention kernel: with enable = 1 the
  * following attend launches accumulate, summed over CTAs, the SM cycles each

@@ -73,6 +73,7 @@ def _declare(L):
         "hca_launch_count": (LL, []),
         "hca_check_status": (I, [VP, C.POINTER(C.c_int)]),
         "hca_profile_enable": (I, [I]),
+        "hca_profile_sample": (I, []),
         "hca_profile_collect": (I, [C.c_char_p, SZ]),
         "hca_trace_attend": (I, [I, C.POINTER(C.c_ulonglong), I]),
         "csa_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
@@ -153,6 +154,10 @@ def launch_count() -> int:
 
 def profile_enable(on: bool = True):
     check(lib().hca_profile_enable(int(on)))
+
+
+def profile_sample():
+    check(lib().hca_profile_sample())
 
 
 def profile_collect() -> dict:

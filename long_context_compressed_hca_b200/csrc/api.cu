@@ -56,13 +56,21 @@ cudaEvent_t take_event() {
   cudaEventCreate(&e);
   return e;
 }
+// Inside a stream capture the record must be an external event node to be
+// timeable after the graph is replayed.
+void record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else cudaEventRecord(e, s);
+}
 }  // namespace
 
 LaunchScope::LaunchScope(const char *n, cudaStream_t s) : name(n), stream(s) {
   if (!g_prof) return;
   std::lock_guard<std::mutex> lk(g_pm);
   cudaEvent_t a = take_event();
-  cudaEventRecord(a, s);
+  record_event(a, s);
   slot = (int)g_pend.size();
   g_pend.push_back({n, a, nullptr});
 }
@@ -71,7 +79,7 @@ int LaunchScope::done() {
   if (slot >= 0) {
     std::lock_guard<std::mutex> lk(g_pm);
     cudaEvent_t b = take_event();
-    cudaEventRecord(b, stream);
+    record_event(b, stream);
     if (slot < (int)g_pend.size()) g_pend[slot].b = b;
   }
   return check_launch(name);
@@ -209,23 +217,24 @@ int hca_profile_enable(int on) {
   return HCA_OK;
 }
 
-int hca_profile_collect(char *buf, size_t len) {
+int hca_profile_sample(void) {
   std::lock_guard<std::mutex> lk(g_pm);
   for (auto &p : g_pend) {
-    if (p.b) {
-      cudaEventSynchronize(p.b);
-      float ms = 0.f;
-      if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
-        auto &acc = g_acc[p.name];
-        acc.first += ms;
-        acc.second += 1;
-      }
-      g_free_events.push_back(p.b);
+    if (!p.b) continue;
+    if (cudaEventSynchronize(p.b) != cudaSuccess) return fail(HCA_ERR_CUDA, "profile event sync failed");
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+      auto &acc = g_acc[p.name];
+      acc.first += ms;
+      acc.second += 1;
     }
-    g_free_events.push_back(p.a);
   }
-  g_pend.clear();
-  if (!buf || len == 0) return HCA_ERR_INVALID;
+  return HCA_OK;
+}
+
+int hca_profile_collect(char *buf, size_t len) {
+  std::lock_guard<std::mutex> lk(g_pm);
+  if (!buf || len == 0) return fail(HCA_ERR_INVALID, "null profile buffer");
   size_t off = 0;
   buf[0] = 0;
   for (auto &kv : g_acc) {
@@ -235,6 +244,11 @@ int hca_profile_collect(char *buf, size_t len) {
     off += (size_t)w;
   }
   g_acc.clear();
+  for (auto &p : g_pend) {
+    if (p.b) g_free_events.push_back(p.b);
+    g_free_events.push_back(p.a);
+  }
+  g_pend.clear();
   return HCA_OK;
 }
 

@@ -260,22 +260,26 @@ constexpr int KT = 64;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kProdWarp0 = 5;
-constexpr int kThreads = (kSoftmaxWarps + 1 + 1) * 32;
+constexpr int kProdWarps = 8;
+constexpr int kProdThreads = kProdWarps * 32;
+constexpr int kThreads = (kSoftmaxWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
 
 struct Bars {
   uint64_t q_full, q_empty, o_empty, mma_done;
-  uint64_t kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t kv_full[8], kv_empty[8], s_full[2], s_empty[2], p_full[2], pv_done[2];
 };
 
 template <int C>
 struct Layout {
   static constexpr int NKB = C / 64;
+  // key-tile stages: as many 64-key tiles as fit beside Q and the P buffers
+  static constexpr int NS = (C == 512) ? 2 : (C == 256 ? 5 : 8);
   static constexpr uint32_t q_off = 0;
   static constexpr uint32_t kv_off = NKB * kTileBytes;
-  static constexpr uint32_t p_off = kv_off + 2 * NKB * kTileBytes;
+  static constexpr uint32_t p_off = kv_off + NS * NKB * kTileBytes;
   static constexpr uint32_t bar_off = p_off + 2 * kTileBytes;
-  static constexpr uint32_t misc_off = bar_off + 256;
+  static constexpr uint32_t misc_off = bar_off + 512;
   static constexpr uint32_t bytes = misc_off + 2048 + 1024;  // + alignment slack
   static constexpr uint32_t tmem_cols = C <= 128 ? 128 : (C <= 256 ? 256 : 512);
 };
@@ -320,9 +324,11 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
     mbar_init(bar(bars->q_empty), 1);
     mbar_init(bar(bars->o_empty), kSoftmaxWarps);
     mbar_init(bar(bars->mma_done), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(bars->kv_full[i]), 1);
+    for (int i = 0; i < L::NS; ++i) {
+      mbar_init(bar(bars->kv_full[i]), kProdThreads);
       mbar_init(bar(bars->kv_empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->s_empty[i]), kSoftmaxWarps);
       mbar_init(bar(bars->p_full[i]), kSoftmaxWarps);
@@ -341,20 +347,23 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProdWarp0) {
-    // ------------------------------------------------------------ TMA loads
-    // Q: 64 rows x C by 2-D tiled loads; key rows by gather4 (4 rows x 64
-    // columns per instruction) into the 128B-swizzled tile.  Lane l builds
-    // group l & 15 (slots 4g..4g+3) for half of the 64-column blocks.
+  if (warp >= kProdWarp0) {
+    // ------------------------------------------------------------ loads
+    // Q: 2-D tiled TMA (thread 0).  Key rows: cp.async by 8 warps, 16-byte
+    // chunks placed at their 128B-swizzled positions; every thread resolves
+    // all of its row addresses for the tile first (independent index loads),
+    // then issues its copies and arms the stage barrier to complete when they
+    // land.
     [&]() {
     constexpr int NKB = C / 64;
-    constexpr int KB_PER_LANE = NKB >= 2 ? NKB / 2 : 1;
-    const int gi = lane & 15, kbh = lane >> 4;
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmC);
-      tma_prefetch_desc(&tmW);
-    }
+    constexpr int CPR = C / 8;                  // 16-byte chunks per row
+    constexpr int RPP = kProdThreads / CPR;     // rows per pass
+    constexpr int NR = KT / RPP;                // rows per thread per tile
+    const int pt = threadIdx.x - kProdWarp0 * 32;
+    const int chunk = pt % CPR, prow = pt / CPR;
+    const uint32_t kb_off = (chunk / 8) * kTileBytes;
+    const int cc = chunk % 8;
+    if (pt == 0) tma_prefetch_desc(&tmQ);
     uint32_t g = 0, iq = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const int bq = u / p.nsplit, sp = u % p.nsplit;
@@ -363,34 +372,36 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
       if (nt == 0) continue;
-      if (!twait(bar(bars->q_empty), (iq & 1) ^ 1, TR_P_QEMPTY)) return;
-      if (lane == 0) {
+      if (pt == 0) {
+        if (!twait(bar(bars->q_empty), (iq & 1) ^ 1, TR_P_QEMPTY)) return;
         mbar_arrive_expect_tx(bar(bars->q_full), NKB * kTileBytes);
         for (int kb = 0; kb < NKB; ++kb)
           tma_load_2d(sbase + L::q_off + kb * kTileBytes, &tmQ, kb * 64, (b * p.n_q + qi) * p.n_h, bar(bars->q_full));
       }
+      // masked slots read a real row of a real tensor (cap is 0 when kv_comp is absent)
+      const __nv_bfloat16 *cbase = reinterpret_cast<const __nv_bfloat16 *>(
+          p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q));
+      const __nv_bfloat16 *wbase = p.kv_win ? reinterpret_cast<const __nv_bfloat16 *>(p.kv_win) : cbase;
       for (int j = 0; j < nt; ++j, ++g) {
-        const int st = g & 1;
-        if (!twait(bar(bars->kv_empty[st]), ((g >> 1) & 1) ^ 1, TR_P_KVEMPTY)) return;
-        const int kk0 = (j0 + j) * KT + 4 * gi;
-        bool v;
-        const int r0 = slot_row(p, ks, b, qi, kk0, v), r1 = slot_row(p, ks, b, qi, kk0 + 1, v),
-                  r2 = slot_row(p, ks, b, qi, kk0 + 2, v), r3 = slot_row(p, ks, b, qi, kk0 + 3, v);
-        const CUtensorMap *map = kk0 < ks.nw4 ? &tmW : &tmC;
-        if (lane == 0) mbar_arrive_expect_tx(bar(bars->kv_full[st]), KT * C * 2);
-        __syncwarp();
-        if (NKB >= 2 || kbh == 0) {
-          const uint32_t tile = sbase + L::kv_off + st * NKB * kTileBytes + gi * 512;
+        const int st = g % L::NS;
+        const __nv_bfloat16 *src[NR];
 #pragma unroll
-          for (int x = 0; x < KB_PER_LANE; ++x) {
-            const int kb = kbh * KB_PER_LANE + x;
-            tma_gather4(tile + kb * kTileBytes, map, kb * 64, r0, r1, r2, r3, bar(bars->kv_full[st]));
-          }
+        for (int i = 0; i < NR; ++i) {
+          const int kk = (j0 + j) * KT + prow + i * RPP;
+          bool v;
+          const int row = slot_row(p, ks, b, qi, kk, v);
+          src[i] = (kk < ks.nw4 ? wbase : cbase) + (long long)row * C + chunk * 8;
         }
+        if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+        const uint32_t tile = sbase + L::kv_off + st * NKB * kTileBytes + kb_off;
+#pragma unroll
+        for (int i = 0; i < NR; ++i) cp_async16(tile + sw128_off(prow + i * RPP, cc), src[i], 16);
+        cp_async_arrive_noinc(bar(bars->kv_full[st]));
       }
       ++iq;
     }
     }();
+    cp_async_wait_all();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
@@ -401,23 +412,24 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       uint32_t g = 0, iq = 0;
       bool ok = true;
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-        const int st = gg & 1;
+        const int st = gg & 1;                 // S / P double buffer
+        const int kst = gg % L::NS;            // key-tile stage
         if (!twait(bar(bars->p_full[st]), (gg >> 1) & 1, TR_M_PFULL)) return false;
         if (first && !twait(bar(bars->o_empty), (iq & 1) ^ 1, TR_M_OEMPTY)) return false;
         tc_fence_after();
         const uint32_t pa = sbase + L::p_off + st * kTileBytes;
-        const uint32_t va = sbase + L::kv_off + st * L::NKB * kTileBytes;
+        const uint32_t va = sbase + L::kv_off + kst * L::NKB * kTileBytes;
+        const uint64_t pd = sdesc_sw128(pa, 16, 1024);
+        const uint64_t vd = sdesc_sw128(va, kTileBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
-          const uint64_t adesc = sdesc_sw128(pa + kk * 32, 16, 1024);
 #pragma unroll
           for (int nh = 0; nh < C / NPV; ++nh) {
-            const uint64_t bdesc = sdesc_sw128(va + nh * (NPV / 64) * kTileBytes + kk * 16 * 128,
-                                               kTileBytes, 1024);
-            umma_bf16(tmem + nh * NPV, adesc, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            const uint64_t voff = (nh * (NPV / 64) * kTileBytes + kk * 16 * 128) >> 4;
+            umma_bf16(tmem + nh * NPV, pd + ((kk * 32) >> 4), vd + voff, IDESC_PV, (first && kk == 0) ? 0u : 1u);
           }
         }
-        umma_commit(bar(bars->kv_empty[st]));
+        umma_commit(bar(bars->kv_empty[kst]));
         umma_commit(bar(bars->pv_done[st]));
         return true;
       };
@@ -434,19 +446,21 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
           const uint32_t gj = g + j;
           const int st = gj & 1;
           const uint32_t ph = (gj >> 1) & 1;
-          if (!twait(bar(bars->kv_full[st]), ph, TR_M_KVFULL) || !twait(bar(bars->s_empty[st]), ph ^ 1, TR_M_SEMPTY)) {
+          const int kst = gj % L::NS;
+          if (!twait(bar(bars->kv_full[kst]), (gj / L::NS) & 1, TR_M_KVFULL) ||
+              !twait(bar(bars->s_empty[st]), ph ^ 1, TR_M_SEMPTY)) {
             ok = false;
             break;
           }
           fence_proxy_async();
           tc_fence_after();
-          const uint32_t qa = sbase + L::q_off;
-          const uint32_t ka = sbase + L::kv_off + st * L::NKB * kTileBytes;
+          // descriptors advance by constant offsets (16-byte units in the low field)
+          const uint64_t qd = sdesc_sw128(sbase + L::q_off, 16, 1024);
+          const uint64_t kd = sdesc_sw128(sbase + L::kv_off + kst * L::NKB * kTileBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
-            const uint32_t off = (kk / 4) * kTileBytes + (kk % 4) * 32;
-            umma_bf16(tS + st * KT, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024),
-                      IDESC_S, kk > 0 ? 1u : 0u);
+            const uint64_t off = ((kk / 4) * kTileBytes + (kk % 4) * 32) >> 4;
+            umma_bf16(tS + st * KT, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar(bars->s_full[st]));
           if (j == nt - 1) umma_commit(bar(bars->q_empty));

@@ -9,7 +9,16 @@ from long_context_compressed_hca_b200 import synth
 from oracle import hca_oracle as O
 
 TOL = {torch.float32: 1e-4, torch.bfloat16: 2e-2}
-GAP = 1e-3
+GAP = 1e-3          # top-k must match exactly where the k-th/(k+1)-th gap exceeds this
+# Where the GPU and the oracle score identical stored inputs (decode over a
+# given cache), their scores agree to ~1e-6 relative, so outputs are compared
+# wherever the gap exceeds this much smaller threshold (stricter than GAP).
+GAP_STRICT = 2e-5
+# From hidden states the bf16 path stores q^I and K^I in bf16, which moves an
+# index score by up to ~1-2% relative (64-term dot products of rounded
+# operands), so end-to-end bf16 layer outputs are compared where the gap
+# exceeds this; the exact rule is applied where the stored inputs are shared.
+GAP_LAYER_BF16 = 2e-2
 
 
 def to64(t):
