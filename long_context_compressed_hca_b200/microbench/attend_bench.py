@@ -1,0 +1,72 @@
+"""Time the tensor-core attention kernel alone on a synthetic prefill batch and
+print the per-role wait-cycle trace.
+
+    python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c]
+
+Inputs are seeded N(0,1) (bf16); CSA index lists take one random visible entry
+per equal-width bucket (valid, sorted, no repeats)."""
+import sys
+
+import torch
+
+from long_context_compressed_hca_b200 import binding as hb
+from long_context_compressed_hca_b200 import synth
+
+
+def main():
+    n_q = int(sys.argv[1]) if len(sys.argv) > 1 else 2048
+    kind = sys.argv[2] if len(sys.argv) > 2 else "csa"
+    c = int(sys.argv[3]) if len(sys.argv) > 3 else 512
+    B, n_h, rd, w, m, k = 1, 64, 64, 128, 4, 512
+    cap = n_q // m + 2
+    dev = "cuda"
+    q = synth.normal_on(dev, (B, n_q, n_h, c), 1, 1, dtype=torch.bfloat16)
+    kv = synth.normal_on(dev, (B, cap, c), 1, 2, dtype=torch.bfloat16)
+    win = synth.normal_on(dev, (B, n_q, c), 1, 3, dtype=torch.bfloat16)
+    sink = synth.normal_on(dev, (n_h,), 1, 4)
+    t = torch.arange(n_q, device=dev)
+    V = (t + 1) // m
+    nsel = torch.clamp(V, max=k)
+    j = torch.arange(k, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    u = torch.rand(n_q, k, device=dev, generator=g)
+    idx = torch.floor((j[None] + u) * V[:, None].double() / nsel.clamp(min=1)[:, None].double()).long()
+    idx = torch.where(j[None] < nsel[:, None], idx, torch.full_like(idx, -1)).int()[None].contiguous()
+    o = torch.empty(B, n_q, n_h, c, dtype=torch.bfloat16, device=dev)
+    d = hb.attn_desc(B, n_h, c, rd, w, m, k=k, dtype=hb.HCA_BF16)
+
+    def run():
+        if kind == "csa":
+            hb.csa_attend(d, q, kv, cap, idx, win, 0, sink, n_q, 0, o)
+        else:
+            hb.hca_attend(d, q, kv, cap, win, 0, sink, n_q, 0, o)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / 5
+    keys = 0
+    for i in range(n_q):
+        vv = (i + 1) // m
+        keys += min(w, i + 1) + (min(k, vv) if kind == "csa" else vv)
+    flops = keys * n_h * c * 4
+    print(f"attend {kind} n_q={n_q} c={c}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s")
+    hb.trace_attend(1)
+    run()
+    tr = hb.trace_attend_read()
+    hb.trace_attend(0)
+    tot = tr["total"]   # summed over the three reporting roles
+    print({kk: (round(3 * v / tot, 3) if kk not in ("rescales", "units", "tiles", "total") else v)
+           for kk, v in tr.items()})
+    print("device status", hb.device_status())
+
+
+if __name__ == "__main__":
+    main()
