@@ -219,6 +219,14 @@ def csa_index_topk(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, 
                                       stream_handle(stream)))
 
 
+def csa_attend_workspace_size(d: AttnDesc, n_q, start_pos) -> int:
+    return lib().csa_attend_workspace_size(C.byref(d), n_q, start_pos)
+
+
+def hca_attend_workspace_size(d: AttnDesc, n_q, start_pos) -> int:
+    return lib().hca_attend_workspace_size(C.byref(d), n_q, start_pos)
+
+
 def csa_attend(d: AttnDesc, q, kv_comp, cap, idx, kv_win, win_is_ring, sink, n_q, start_pos, o,
                ws=None, stream=None):
     nbytes = ws.numel() * ws.element_size() if ws is not None else 0

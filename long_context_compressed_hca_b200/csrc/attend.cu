@@ -735,7 +735,7 @@ int choose_splits(const AttendParams &p) {
   const int V = (t + 1) / p.m;
   const int nk = (p.w < t + 1 ? p.w : t + 1) + (p.csa ? (p.k < V ? p.k : V) : V);
   const int tiles = (nk + 63) / 64;
-  int ns = (int)((num_sms() + q - 1) / q);
+  int ns = (int)(num_sms() / q);          // every unit in one wave of persistent CTAs
   if (ns > tiles / 2) ns = tiles / 2;     // keep >= 2 tiles per split
   if (ns > 32) ns = 32;
   return ns < 1 ? 1 : ns;

@@ -7,9 +7,9 @@
 // lower entry index, emitted in ascending index order and padded with -1.
 //
 // The selection is an exact radix select on the order-preserving uint32 image
-// of the fp32 scores (4 passes of 8 bits over a row held in shared memory),
-// followed by a stable compaction; rows longer than one block's shared memory
-// are cut into chunks whose local winners are merged by a second pass.
+// of the fp32 scores (up to 4 passes of 8 bits), run by a thread-block cluster
+// whose CTAs hold slices of the row in shared memory and sum their histograms
+// through distributed shared memory, followed by a stable compaction.
 #include "common.cuh"
 #include "internal.h"
 
@@ -73,168 +73,322 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
 }
 
 // ------------------------------------------------------------------ top-k
+// One thread-block cluster of C CTAs (C <= 8) selects the top-k of one row
+// segment; CTA r of the cluster holds keys [r*slice, (r+1)*slice) of the
+// segment in shared memory.  Each radix pass (8 bits, top byte first) builds
+// a CTA-local 256-bin histogram, the C histograms are summed through
+// distributed shared memory, and every CTA derives the same digit from the
+// same totals.  Once a CTA's keys that still match the threshold prefix fit
+// in kCandMax they are compacted and later passes scan only those.  The final
+// stable compaction offsets each CTA's output by the winners of the lower-
+// ranked CTAs, so the selection leaves in ascending index order with ties
+// resolved towards the lower index.  Rows longer than one segment are cut
+// into segments whose winners (order key + index) a second launch merges.
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kSliceMax = 16384;   // keys per CTA (64 KB of shared memory)
+constexpr int kCandMax = 4096;     // compacted keys per CTA (16 KB)
+constexpr int kClusterMax = 8;     // portable cluster size
 
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t u = __float_as_uint(f);
+__device__ __forceinline__ uint32_t order_bits(uint32_t u) {
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                 // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 1 for every non-NaN float
 }
-
-// Exclusive scan of one int per thread over the block; returns the prefix and
-// writes the block total to *total.
-__device__ int block_exclusive_scan(int v, int *warp_tot, int *total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tot[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int t = lane < kTopkWarps ? warp_tot[lane] : 0;
-    int u = t;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, u, o);
-      if (lane >= o) u += y;
-    }
-    if (lane < kTopkWarps) warp_tot[lane] = u - t;   // exclusive warp offsets
-    if (lane == kTopkWarps - 1) *total = u;
-  }
-  __syncthreads();
-  const int r = warp_tot[warp] + x - v;
-  __syncthreads();
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync() { cluster_arrive(); cluster_wait(); }
+// Load a 32-bit word from the same shared-memory variable in CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_ld(const void *local, uint32_t rank) {
+  uint32_t ra, v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  return v;
+}
 
-// One block selects the top-k of one (row, chunk).  Elements are read from
-// scores[row*stride + begin + i] for i < len; with cand_idx the element's
-// index is cand_idx[same offset] (-1 = absent), else elem_offset + begin + i.
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkParams p, int chunk, int n_chunks,
-                                                             long long out_chunk_stride) {
-  extern __shared__ uint32_t keys[];        // [chunk]
-  __shared__ uint32_t hist[kTopkWarps][256];
-  __shared__ uint32_t total[256];
-  __shared__ int warp_tot[32];
-  __shared__ int s_total;
+// Add one key to a shared histogram (bin 256 = no key).  The lanes that
+// share the first pending lane's bin are folded into one atomic, twice, which
+// keeps clustered scores (one dominant bin) from serialising the warp.
+__device__ __forceinline__ void hist_add(uint32_t *h, uint32_t bin) {
+  const int lane = threadIdx.x & 31;
+  unsigned active = __ballot_sync(0xffffffffu, bin != 256u);
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    if (!active) return;
+    const int leader = __ffs(active) - 1;
+    const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
+    const unsigned same = __ballot_sync(0xffffffffu, bin == lb) & active;
+    if (lane == leader) atomicAdd(&h[lb], (uint32_t)__popc(same));
+    if (same & (1u << lane)) bin = 256u;
+    active &= ~same;
+  }
+  if (active & (1u << lane)) atomicAdd(&h[bin], 1u);
+}
+
+// Copy len 32-bit words to shared memory, as order keys (KEYS: already keys).
+template <bool KEYS>
+__device__ __forceinline__ void load_keys(uint32_t *dst, const uint32_t *src, int len) {
+  const int tid = threadIdx.x;
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    const int nv = len >> 2;
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    for (int i0 = 0; i0 < nv; i0 += 4 * kTopkThreads) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = i0 + u * kTopkThreads + tid;
+        if (j < nv) v[u] = __ldg(s4 + j);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = i0 + u * kTopkThreads + tid;
+        if (j < nv) {
+          uint4 x = v[u];
+          if (!KEYS) { x.x = order_bits(x.x); x.y = order_bits(x.y); x.z = order_bits(x.z); x.w = order_bits(x.w); }
+          d4[j] = x;
+        }
+      }
+    }
+    done = nv * 4;
+  }
+  for (int i = done + tid; i < len; i += kTopkThreads) {
+    const uint32_t x = __ldg(src + i);
+    dst[i] = KEYS ? x : order_bits(x);
+  }
+}
+
+// Grid: x = C * rows * n_seg, cluster (C,1,1).  Dynamic shared memory:
+// (slice + kCandMax) words.
+__global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
+  extern __shared__ __align__(16) uint32_t dyn[];
+  uint32_t *keys = dyn;               // [slice]
+  uint32_t *cand = dyn + p.slice;     // [kCandMax]
+  __shared__ uint32_t sub[4][256];
+  __shared__ uint32_t pub[2][256];    // this CTA's histogram of pass (parity), read by the cluster
+  __shared__ uint32_t tot[256];
+  __shared__ int pub_cnt[2];          // this CTA's keys above / equal to the threshold
+  __shared__ int w_gt[kTopkWarps], w_eq[kTopkWarps];
+  __shared__ int s_total, s_krem, s_nc, s_base, s_eqb;
   __shared__ uint32_t s_digit;
-  __shared__ int s_krem;
 
-  const int row = blockIdx.x, ch = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int V;
-  if (p.row_len) V = p.row_len[row];
-  else V = (p.start_pos + row % p.n_q + 1) / p.m;
-  const long long begin = (long long)ch * chunk;
-  const int len = (int)max(0LL, min((long long)chunk, (long long)V - begin));
-  const float *src = p.scores + (long long)row * p.score_stride + begin;
-  const int32_t *csrc = p.cand_idx ? p.cand_idx + (long long)row * p.score_stride + begin : nullptr;
+  const uint32_t C = cluster_size(), rank = cluster_rank();
+  const long long unit = blockIdx.x / C;
+  const int row = (int)(unit / p.n_seg), seg = (int)(unit % p.n_seg);
+  const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
+  const long long seg_begin = (long long)seg * p.seg_len;
+  const int seg_V = (int)max(0LL, min((long long)p.seg_len, (long long)V - seg_begin));
+  const int len = max(0, min(p.slice, seg_V - (int)rank * p.slice));
+  const long long begin = seg_begin + (long long)rank * p.slice;   // element index of keys[0]
 
-  int nvalid = 0;
-  for (int i = tid; i < len; i += kTopkThreads) {
-    const bool ok = csrc ? csrc[i] >= 0 : true;
-    keys[i] = ok ? order_key(src[i]) : 0u;
-    nvalid += ok;
-  }
-  block_exclusive_scan(nvalid, warp_tot, &s_total);
-  nvalid = s_total;
-  const int K = min(p.k, nvalid);
+  if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
+  else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
+  if (tid == 0) s_nc = 0;
 
-  uint32_t T = 0;      // threshold key
-  int krem = 0;        // how many keys equal to T to keep (in list order)
-  if (K > 0 && K < nvalid) {
-    uint32_t prefix = 0, mask = 0;
-    krem = K;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < kTopkWarps * 256; i += kTopkThreads) (&hist[0][0])[i] = 0;
-      __syncthreads();
-      const int trips = (len + kTopkThreads - 1) / kTopkThreads;
-      for (int tr = 0; tr < trips; ++tr) {
-        const int i = tr * kTopkThreads + tid;
-        uint32_t bin = 256;
-        if (i < len) {
-          const uint32_t kk = keys[i];
-          if (kk != 0 && (kk & mask) == prefix) bin = (kk >> shift) & 255u;
-        }
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (bin != 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[warp][bin], __popc(peers));
+  uint32_t prefix = 0, mask = 0, T = 0;
+  int krem = p.k, K = 0;
+  bool compacted = false;
+  int nc = 0;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t *arr = compacted ? cand : keys;
+    const int n = compacted ? nc : len;
+    for (int i = tid; i < 4 * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
+      const int i = b0 + tid;
+      uint32_t bin = 256u;
+      if (i < n) {
+        const uint32_t kk = arr[i];
+        if (kk != 0 && (kk & mask) == prefix) bin = (kk >> shift) & 255u;
       }
-      __syncthreads();
-      if (tid < 256) {
-        uint32_t t = 0;
-#pragma unroll
-        for (int w = 0; w < kTopkWarps; ++w) t += hist[w][tid];
-        total[tid] = t;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane l covers bins 255-8l .. 248-8l (descending); suffix sums from the top
-        uint32_t loc[8], run = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) { run += total[255 - 8 * lane - j]; loc[j] = run; }
-        uint32_t incl = run;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const uint32_t before = incl - run;   // keys in higher bins than this lane's
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t above = before + (j ? loc[j - 1] : 0u);   // strictly higher bins
-          const uint32_t upto = before + loc[j];
-          if (above < (uint32_t)krem && upto >= (uint32_t)krem) {
-            s_digit = 255 - 8 * lane - j;
-            s_krem = krem - (int)above;
-          }
-        }
-      }
-      __syncthreads();
-      prefix |= s_digit << shift;
-      mask |= 255u << shift;
-      krem = s_krem;
-      __syncthreads();
+      hist_add(sub[warp & 3], bin);
     }
-    T = prefix;
+    __syncthreads();
+    if (tid < 256) pub[pass & 1][tid] = sub[0][tid] + sub[1][tid] + sub[2][tid] + sub[3][tid];
+    cluster_sync();
+    if (tid < 256) {
+      uint32_t t = 0;
+      for (uint32_t r = 0; r < C; ++r) t += dsmem_ld(&pub[pass & 1][tid], r);
+      tot[tid] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l covers bins 255-8l .. 248-8l (descending); suffix sums from the top
+      uint32_t loc[8], run = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) { run += tot[255 - 8 * lane - j]; loc[j] = run; }
+      uint32_t incl = run;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t before = incl - run;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t above = before + (j ? loc[j - 1] : 0u), upto = before + loc[j];
+        if (above < (uint32_t)krem && upto >= (uint32_t)krem) {
+          s_digit = 255 - 8 * lane - j;
+          s_krem = krem - (int)above;
+        }
+      }
+      if (lane == 31) s_total = (int)incl;
+    }
+    __syncthreads();
+    if (pass == 0) {
+      const int nvalid = s_total;   // the whole segment's keys (absent keys are 0)
+      if (nvalid <= p.k) { K = nvalid; krem = 0; break; }   // every key is selected, T = 0
+      if (p.k <= 0) { K = 0; krem = 0; prefix = 0xFFFFFFFFu; break; }   // none is selected
+      K = p.k;
+    }
+    const uint32_t digit = s_digit;
+    prefix |= digit << shift;
+    mask |= 255u << shift;
+    krem = s_krem;
+    if (pass < 3 && !compacted && pub[pass & 1][digit] <= (uint32_t)kCandMax) {
+      // compact this CTA's keys that match the new prefix
+      for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
+        const int i = b0 + tid;
+        const uint32_t kk = i < n ? arr[i] : 0u;
+        const bool m = kk != 0 && (kk & mask) == prefix;
+        const unsigned bal = __ballot_sync(0xffffffffu, m);
+        int at = 0;
+        if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+        if (m) cand[at] = kk;
+      }
+      nc = (int)pub[pass & 1][digit];
+      compacted = true;
+    }
+    __syncthreads();
   }
-  // stable compaction: keep key > T, and the first krem keys == T
-  const int seg = (len + kTopkThreads - 1) / kTopkThreads;
-  const int lo = min(len, tid * seg), hi = min(len, lo + seg);
-  int ceq = 0;
-  for (int i = lo; i < hi; ++i) ceq += (keys[i] == T && T != 0);
-  const int eq_base = block_exclusive_scan(ceq, warp_tot, &s_total);
-  int csel = 0, e = eq_base;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t kk = keys[i];
-    if (kk == 0) continue;
-    if (kk > T) ++csel;
-    else if (kk == T && T != 0) { if (e < krem) ++csel; ++e; }
+  if (K == p.k) T = prefix;
+
+  // count, per warp over a contiguous run of keys, those above and equal to T
+  const int wseg = ((len + kTopkThreads - 1) / kTopkThreads) * 32;
+  const int w_lo = min(len, warp * wseg), w_hi = min(len, w_lo + wseg);
+  int gt = 0, eq = 0;
+  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t kk = i < w_hi ? keys[i] : 0u;
+    gt += __popc(__ballot_sync(0xffffffffu, kk > T));
+    eq += __popc(__ballot_sync(0xffffffffu, T != 0 && kk == T));
   }
-  const int out_base = block_exclusive_scan(csel, warp_tot, &s_total);
-  int32_t *out = p.idx_out + (long long)row * p.idx_stride + (long long)ch * out_chunk_stride;
-  float *sout = p.score_out ? p.score_out + (long long)row * p.idx_stride + (long long)ch * out_chunk_stride
-                            : nullptr;
-  int o = out_base;
-  e = eq_base;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t kk = keys[i];
-    if (kk == 0) continue;
-    bool take = kk > T;
-    if (kk == T && T != 0) { take = e < krem; ++e; }
+  if (lane == 0) { w_gt[warp] = gt; w_eq[warp] = eq; }
+  __syncthreads();
+  if (tid == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < kTopkWarps; ++w) { a += w_gt[w]; b += w_eq[w]; }
+    pub_cnt[0] = a;
+    pub_cnt[1] = b;
+  }
+  cluster_sync();
+  if (tid == 0) {
+    // winners of the lower-ranked CTAs, and ties among them
+    int base = 0, eqb = 0;
+    for (uint32_t r = 0; r < rank; ++r) {
+      const int g = (int)dsmem_ld(&pub_cnt[0], r), e = (int)dsmem_ld(&pub_cnt[1], r);
+      base += g + max(0, min(krem - eqb, e));
+      eqb += e;
+    }
+    s_base = base;
+    s_eqb = eqb;
+  }
+  cluster_arrive();   // this CTA reads no other CTA's shared memory past here
+  __syncthreads();
+  int ties_before = s_eqb, sel_before = s_base;
+  for (int w = 0; w < warp; ++w) { ties_before += w_eq[w]; sel_before += w_gt[w]; }
+  sel_before += min(krem, ties_before) - min(krem, s_eqb);
+  int32_t *out = p.idx_out + row * p.out_stride + (long long)seg * p.k;
+  uint32_t *kout = p.key_out ? p.key_out + row * p.out_stride + (long long)seg * p.k : nullptr;
+  const int32_t *cidx = p.cand_idx ? p.cand_idx + row * p.in_stride + begin : nullptr;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t kk = i < w_hi ? keys[i] : 0u;
+    const bool is_eq = T != 0 && kk == T;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = kk > T || (is_eq && ties_before + __popc(eqm & lt) < krem);
+    const unsigned sm = __ballot_sync(0xffffffffu, take);
     if (take) {
-      out[o] = csrc ? csrc[i] : (int32_t)(p.elem_offset + begin + i);
-      if (sout) sout[o] = src[i];
-      ++o;
+      const int o = sel_before + __popc(sm & lt);
+      out[o] = cidx ? cidx[i] : (int32_t)(begin + i);
+      if (kout) kout[o] = kk;
     }
+    ties_before += __popc(eqm);
+    sel_before += __popc(sm);
   }
-  for (int i = K + tid; i < p.k; i += kTopkThreads) {
-    out[i] = -1;
-    if (sout) sout[i] = -INFINITY;
+  if (rank == 0)
+    for (int i = K + tid; i < p.k; i += kTopkThreads) {
+      out[i] = -1;
+      if (kout) kout[i] = 0u;
+    }
+  cluster_wait();     // keep this CTA's shared memory alive until the cluster has read it
+}
+
+struct TopkPlan {
+  int C, n_seg, seg_len, slice;
+};
+// Cluster size, segments and per-CTA slice for rows of up to Vmax keys: grow
+// the cluster (keeping >= 1024 keys per CTA) until the grid covers the SMs
+// twice or the row fits one segment of C * kSliceMax keys.
+TopkPlan plan_topk(long long rows, long long Vmax) {
+  TopkPlan t{};
+  int C = 1;
+  const long long want = 2LL * num_sms();
+  while (C < kClusterMax && Vmax >= 2048LL * C && (rows * C < want || (long long)C * kSliceMax < Vmax)) C *= 2;
+  t.C = C;
+  const long long per_seg = (long long)C * kSliceMax;
+  t.n_seg = (int)max(1LL, (Vmax + per_seg - 1) / per_seg);
+  long long seg_len = (Vmax + t.n_seg - 1) / t.n_seg;
+  seg_len = ((seg_len + 4LL * C - 1) / (4LL * C)) * (4LL * C);
+  t.seg_len = (int)max(seg_len, 4LL * C);
+  t.slice = t.seg_len / C;
+  return t;
+}
+size_t topk_smem(const TopkPlan &t) { return (size_t)(t.slice + kCandMax) * 4; }
+int ensure_topk_smem() {
+  static bool done = false;
+  if (!done) {
+    const cudaError_t e = cudaFuncSetAttribute(topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (kSliceMax + kCandMax) * 4);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k smem attribute: %s", cudaGetErrorString(e));
+    done = true;
   }
+  return HCA_OK;
+}
+int launch_topk_cluster(const char *name, const TopkParams &t, const TopkPlan &pl, long long rows, cudaStream_t s) {
+  LaunchScope ls(name, s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(rows * pl.n_seg * pl.C), 1, 1);
+  cfg.blockDim = dim3(kTopkThreads, 1, 1);
+  cfg.dynamicSmemBytes = topk_smem(pl);
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = pl.C;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster, t);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "%s launch: %s", name, cudaGetErrorString(e));
+  }
+  return ls.done();
 }
 
 }  // namespace
@@ -255,56 +409,24 @@ int launch_index_scores(const IndexParams &p, cudaStream_t s) {
   return ls_.done();
 }
 
-namespace {
-constexpr int kMaxChunk = 16384;     // 64 KB of keys per block in pass 1
-constexpr int kMaxMerge = 32768;     // candidates per row in pass 2 (128 KB)
-int topk_chunk_for(int rows, int Vmax, int k) {
-  if (Vmax <= 0) return 1;
-  int chunk = kMaxChunk;
-  // with few rows, cut each row into more chunks so that every SM has work,
-  // keeping each chunk >= 4k so the merge pass still reduces
-  const int want_blocks = 2 * num_sms();
-  while (chunk / 2 >= 4 * k && chunk / 2 >= 1024 &&
-         (long long)rows * ((Vmax + chunk - 1) / chunk) < want_blocks &&
-         (long long)((Vmax + chunk / 2 - 1) / (chunk / 2)) * k <= kMaxMerge)
-    chunk /= 2;
-  return chunk;
-}
-int ensure_topk_smem() {
-  static bool done = false;
-  if (!done) {
-    const cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               kMaxMerge * 4);
-    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k smem attribute: %s", cudaGetErrorString(e));
-    done = true;
-  }
-  return HCA_OK;
-}
-}  // namespace
 
 size_t topk_workspace_bytes(const IndexParams &p) {
-  const int rows = p.B * p.n_q;
-  const int Vmax = (p.start_pos + p.n_q) / p.m;
-  const int chunk = topk_chunk_for(rows, Vmax, p.k);
-  const int n_chunks = (Vmax + chunk - 1) / chunk;
+  const long long rows = (long long)p.B * p.n_q;
+  const long long Vmax = (p.start_pos + p.n_q) / p.m;
+  const TopkPlan pl = plan_topk(rows, Vmax);
   size_t b = (size_t)rows * (size_t)Vmax * sizeof(float);           // scores
   b = (b + 255) & ~(size_t)255;
-  if (n_chunks > 1) {
-    size_t c = (size_t)rows * n_chunks * p.k;
-    b += ((c * sizeof(int32_t) + 255) & ~(size_t)255) + ((c * sizeof(float) + 255) & ~(size_t)255);
+  if (pl.n_seg > 1) {
+    const size_t c = (size_t)rows * pl.n_seg * p.k;
+    b += 2 * ((c * sizeof(int32_t) + 255) & ~(size_t)255);          // winners' indices and keys
   }
   return b;
-}
-
-int launch_topk(const TopkParams &p, cudaStream_t s) {
-  (void)p; (void)s;
-  return HCA_ERR_UNSUPPORTED;
 }
 
 int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long long user_stride,
                    void *ws, size_t ws_bytes, cudaStream_t s) {
   if (ws_bytes < topk_workspace_bytes(ip)) return fail(HCA_ERR_INVALID, "workspace too small");
-  const int rows = ip.B * ip.n_q;
+  const long long rows = (long long)ip.B * ip.n_q;
   const int Vmax = (ip.start_pos + ip.n_q) / ip.m;
   IndexParams p = ip;
   char *w = static_cast<char *>(ws);
@@ -321,32 +443,33 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   rc = launch_index_scores_tc(p, s);
   if (rc == HCA_ERR_UNSUPPORTED) rc = launch_index_scores(p, s);
   if (rc) return rc;
-  const int chunk = topk_chunk_for(rows, Vmax, ip.k);
-  const int n_chunks = Vmax > 0 ? (Vmax + chunk - 1) / chunk : 1;
+  const TopkPlan pl = plan_topk(rows, Vmax);
   TopkParams t{};
-  t.rows = rows; t.k = ip.k; t.scores = p.scores; t.score_stride = p.score_stride;
+  t.rows = (int)rows; t.k = ip.k; t.scores = p.scores; t.in_stride = p.score_stride;
   t.n_q = ip.n_q; t.start_pos = ip.start_pos; t.m = ip.m;
-  if (n_chunks <= 1) {
-    t.idx_out = idx; t.idx_stride = ip.k;
-    return HCA_LAUNCH("topk", s, topk_kernel<<<dim3(rows, 1), kTopkThreads, (size_t)max(chunk, 1) * 4, s>>>(t, chunk, 1, 0));
+  t.n_seg = pl.n_seg; t.seg_len = pl.seg_len; t.slice = pl.slice;
+  if (pl.n_seg == 1) {
+    t.idx_out = idx; t.out_stride = ip.k;
+    return launch_topk_cluster("topk", t, pl, rows, s);
   }
-  // pass 1: local winners of each chunk
-  const size_t c = (size_t)rows * n_chunks * ip.k;
+  // pass 1: the winners of every segment, with their order keys
+  const int clen = pl.n_seg * ip.k;
+  const size_t c = (size_t)rows * clen;
   int32_t *cidx = reinterpret_cast<int32_t *>(w + off);
   off += (c * sizeof(int32_t) + 255) & ~(size_t)255;
-  float *cscore = reinterpret_cast<float *>(w + off);
-  t.idx_out = cidx; t.score_out = cscore; t.idx_stride = (long long)n_chunks * ip.k;
-  rc = HCA_LAUNCH("topk_pass1", s, topk_kernel<<<dim3(rows, n_chunks), kTopkThreads, (size_t)chunk * 4, s>>>(t, chunk, n_chunks, ip.k));
+  uint32_t *ckey = reinterpret_cast<uint32_t *>(w + off);
+  t.idx_out = cidx; t.key_out = ckey; t.out_stride = clen;
+  rc = launch_topk_cluster("topk_pass1", t, pl, rows, s);
   if (rc) return rc;
-  // pass 2: merge the candidate lists (chunk order == index order)
-  const int clen = n_chunks * ip.k;
-  if (clen > kMaxMerge) return fail(HCA_ERR_UNSUPPORTED, "top-k candidate list too long (%d)", clen);
+  // pass 2: merge the segments' winners (segment order is index order)
+  const TopkPlan pl2 = plan_topk(rows, clen);
+  if (pl2.n_seg != 1) return fail(HCA_ERR_UNSUPPORTED, "top-k candidate list too long (%d)", clen);
   TopkParams t2{};
-  t2.rows = rows; t2.k = ip.k; t2.scores = cscore; t2.score_stride = clen; t2.cand_idx = cidx;
-  t2.row_len = nullptr; t2.n_q = 1; t2.start_pos = clen - 1; t2.m = 1;   // every row has clen elements
-  t2.idx_out = idx; t2.idx_stride = ip.k;
-  const size_t smem = (size_t)clen * 4;
-  return HCA_LAUNCH("topk_pass2", s, topk_kernel<<<dim3(rows, 1), kTopkThreads, smem, s>>>(t2, clen, 1, 0));
+  t2.rows = (int)rows; t2.k = ip.k; t2.keys = ckey; t2.cand_idx = cidx; t2.in_stride = clen;
+  t2.fixed_len = clen; t2.n_q = 1; t2.m = 1;
+  t2.n_seg = 1; t2.seg_len = pl2.seg_len; t2.slice = pl2.slice;
+  t2.idx_out = idx; t2.out_stride = ip.k;
+  return launch_topk_cluster("topk_pass2", t2, pl2, rows, s);
 }
 
 }  // namespace hca

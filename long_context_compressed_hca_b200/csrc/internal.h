@@ -74,17 +74,17 @@ int launch_index_scores_tc(const IndexParams &p, cudaStream_t s);
 struct TopkParams {
   int rows;                // number of score rows
   int k;
-  const float *scores;     // row r at scores + r*score_stride
-  long long score_stride;
-  const int32_t *cand_idx; // optional explicit indices per element (same layout), else implicit
-  const int *row_len;      // optional per-row valid length (else from visibility)
-  int n_q, start_pos, m;   // visibility: row r -> query (r % n_q) at position start_pos + r % n_q
-  int32_t *idx_out;        // row r at idx_out + r*idx_stride
-  long long idx_stride;
-  float *score_out;        // optional: the selected keys' scores (for two-pass merges)
-  long long elem_offset;   // index offset added to implicit indices (chunked rows)
+  const float *scores;     // fp32 scores, row r at scores + r*in_stride; or
+  const uint32_t *keys;    // order keys (0 = absent) whose indices are in cand_idx
+  const int32_t *cand_idx; // same layout as keys
+  long long in_stride;
+  int fixed_len;           // > 0: every row has fixed_len elements
+  int n_q, start_pos, m;   // else row r -> query r % n_q at position start_pos + r % n_q, (t+1)/m entries
+  int32_t *idx_out;        // (row, segment) at idx_out + row*out_stride + segment*k
+  uint32_t *key_out;       // optional: the winners' order keys (segmented first pass)
+  long long out_stride;
+  int n_seg, seg_len, slice;   // segments per row, keys per segment, keys per CTA
 };
-int launch_topk(const TopkParams &p, cudaStream_t s);
 size_t topk_workspace_bytes(const IndexParams &p);
 int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
                    void *ws, size_t ws_bytes, cudaStream_t s);

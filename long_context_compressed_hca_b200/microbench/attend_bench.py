@@ -2,6 +2,7 @@
 print the per-role wait-cycle trace.
 
     python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c]
+    python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos]
 
 Inputs are seeded N(0,1) (bf16); CSA index lists take one random visible entry
 per equal-width bucket (valid, sorted, no repeats)."""
@@ -13,7 +14,70 @@ from long_context_compressed_hca_b200 import binding as hb
 from long_context_compressed_hca_b200 import synth
 
 
+def decode_main():
+    """One decode token per sequence over a ring window and a compressed cache
+    (the 128K decode workload's attention call), split-KV included."""
+    kind = sys.argv[2] if len(sys.argv) > 2 else "csa"
+    B = int(sys.argv[3]) if len(sys.argv) > 3 else 32
+    pos = int(sys.argv[4]) if len(sys.argv) > 4 else 131072
+    n_h, c, rd, w = 64, 512, 64, 128
+    m, k = (4, 512) if kind == "csa" else (128, 0)
+    V = (pos + 1) // m
+    cap = V + 8
+    dev = "cuda"
+    q = synth.normal_on(dev, (B, 1, n_h, c), 2, 1, dtype=torch.bfloat16)
+    kv = synth.normal_on(dev, (B, cap, c), 2, 2, dtype=torch.bfloat16)
+    ring = synth.normal_on(dev, (B, w, c), 2, 3, dtype=torch.bfloat16)
+    sink = synth.normal_on(dev, (n_h,), 2, 4)
+    idx = None
+    if kind == "csa":
+        g = torch.Generator(device=dev)
+        g.manual_seed(4)
+        j = torch.arange(k, device=dev)
+        u = torch.rand(B, k, device=dev, generator=g)
+        idx = torch.floor((j[None] + u) * (V / k)).long().clamp(max=V - 1).int()[:, None].contiguous()
+    o = torch.empty(B, 1, n_h, c, dtype=torch.bfloat16, device=dev)
+    d = hb.attn_desc(B, n_h, c, rd, w, m, k=max(k, 1), dtype=hb.HCA_BF16)
+    wsz = (hb.csa_attend_workspace_size if kind == "csa" else hb.hca_attend_workspace_size)(d, 1, pos)
+    ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
+
+    def run():
+        if kind == "csa":
+            hb.csa_attend(d, q, kv, cap, idx, ring, 1, sink, 1, pos, o, ws)
+        else:
+            hb.hca_attend(d, q, kv, cap, ring, 1, sink, 1, pos, o, ws)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    hb.profile_enable(True)
+    hb.profile_collect()
+    for _ in range(10):
+        run()
+        torch.cuda.synchronize()
+        hb.profile_sample()
+        hb.profile_collect() if False else None
+    prof = hb.profile_collect()
+    hb.profile_enable(False)
+    keys = min(w, pos + 1) + (min(k, V) if kind == "csa" else V)
+    byts = B * (keys * c * 2 + 2 * n_h * c * 2)
+    for name, (n, ms) in prof.items():
+        print(f"{name}: {ms / n * 1e3:.1f} us per launch ({n} launches)")
+    att = [v for kk, v in prof.items() if kk.startswith("attend_") and kk.endswith("tc")][0]
+    print(f"gathered+q/o bytes {byts / 1e6:.1f} MB -> {byts / (att[1] / att[0] * 1e-3) / 1e9:.0f} GB/s in the attention kernel")
+    hb.trace_attend(1)
+    run()
+    tr = hb.trace_attend_read()
+    hb.trace_attend(0)
+    tot = tr["total"]
+    print({kk: (round(3 * v / tot, 3) if kk not in ("rescales", "units", "tiles", "total") else v)
+           for kk, v in tr.items()})
+    print("device status", hb.device_status())
+
+
 def main():
+    if len(sys.argv) > 1 and sys.argv[1] == "decode":
+        return decode_main()
     n_q = int(sys.argv[1]) if len(sys.argv) > 1 else 2048
     kind = sys.argv[2] if len(sys.argv) > 2 else "csa"
     c = int(sys.argv[3]) if len(sys.argv) > 3 else 512

@@ -192,6 +192,57 @@ def test_index_topk(cuda, B, n_q, start_pos, m, k, n_hI, c_I, qdt, kdt):
             ties += check_topk_row(gi[b, i], ref, k, V)
 
 
+TIE_CASES = [
+    # B, n_q, start_pos, k, key dtype: rows span one CTA, a cluster, two segments
+    (2, 64, 0, 64, "bf16"),
+    (3, 1, 131071, 512, "bf16"),
+    (1, 2, 300000, 512, "bf16"),
+    (2, 1, 1048575, 1024, "fp8"),
+]
+
+
+@pytest.mark.parametrize("B,n_q,start_pos,k,kdt", TIE_CASES)
+def test_index_topk_exact_ties(cuda, B, n_q, start_pos, k, kdt):
+    """Entries share one of three index keys, so each row holds three score
+    values repeated thousands of times: the selection must take the whole
+    upper classes and then the lowest indices of the class that the k-th
+    score falls in (Eq.(17), ties to the lower index), across every CTA of
+    the cluster and every segment of the row."""
+    m, n_hI, c_I = 4, 8, 64
+    E = (start_pos + n_q) // m
+    cap = E + 1
+    base = synth.normal((B, 3, c_I), 77, 1)
+    s_ids = np.arange(cap)
+    cls = np.where(s_ids % 97 == 5, 0, 1 + (s_ids * 7 // 3) % 2)   # a rare class and two common ones
+    KIf = base[:, torch.from_numpy(cls)]
+    qI = rnd((B, n_q, n_hI, c_I), 78, 1, BF16)
+    wI = rnd((B, n_q, n_hI), 78, 2, std=c_I ** -0.5 * n_hI ** -0.5)
+    KI_scale = None
+    if kdt == "fp8":
+        KI, KI_scale = synth.fp8_rows(KIf)
+        KI, KI_scale = KI.to(cuda), KI_scale.to(cuda)
+        KI64 = O.e4m3_to_f64(KI.cpu().numpy()) * to64(KI_scale)[..., None]
+        kcode = hb.HCA_FP8E4M3
+    else:
+        KI = KIf.to(BF16).to(cuda)
+        KI64 = to64(KI)
+        kcode = CODE[BF16]
+    d = hb.attn_desc(B, 4, 64, 16, 8, m, k=k, n_hI=n_hI, c_I=c_I, rd_I=16, dtype=CODE[BF16], idx_key_dtype=kcode)
+    ws = torch.empty(hb.csa_index_topk_workspace_size(d, n_q, start_pos), dtype=torch.uint8, device=cuda)
+    idx = torch.full((B, n_q, k), -7, dtype=torch.int32, device=cuda)
+    hb.csa_index_topk(d, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, None, 0, ws)
+    torch.cuda.synchronize()
+    q64, w64, gi = to64(qI), to64(wI), idx.cpu().numpy()
+    for b in range(B):
+        for i in range(n_q):
+            V = (start_pos + i + 1) // m
+            ref = O.index_scores(q64[b, i], w64[b, i], KI64[b], V)
+            vals = np.unique(ref)
+            if len(vals) > 1:   # the classes are far apart, so fp32 cannot reorder them
+                assert np.diff(vals).min() > 1e-3 * np.abs(vals).max()
+            np.testing.assert_array_equal(gi[b, i], O.topk_select(ref, k))
+
+
 # ----------------------------------------------------------------- attention
 ATT_CASES = [
     # kind, dtype, B, n_q, n_h, c, rd, w, m, k
