@@ -141,6 +141,28 @@ int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI,
                    int start_pos, int32_t *idx, float *scores, long long score_stride,
                    void *ws, size_t ws_bytes, hca_stream_t stream);
 
+/* The papers have no counterpart to this call: it is csa_index_topk (same
+ * arguments, same results) for callers that cannot allocate or hand in a
+ * workspace, e.g. an allocator's own out-of-memory path or a loop that must
+ * not call cudaMalloc/cudaFree (they synchronise the device).  Its scratch is
+ * a fixed device array of HCA_STATIC_SCRATCH_BYTES (8 MiB) per device, inside
+ * the library; it allocates nothing.
+ *   Needs csa_index_topk_workspace_size(d, n_q, start_pos) <=
+ *   HCA_STATIC_SCRATCH_BYTES (about B*n_q*((start_pos+n_q)/m)*4 bytes, e.g. a
+ *   decode step of 32 sequences at 131072 tokens with m = 4); a larger call
+ *   fails with HCA_ERR_INVALID and a message naming both sizes.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make it before any stream capture that includes
+ *   this call.  The array is not cleared between calls and needs no clearing.
+ *   The array is shared by every call on a device: calls that may overlap in
+ *   time (different streams or host threads without ordering between them)
+ *   race on it and must be serialised by the caller. */
+#define HCA_STATIC_SCRATCH_BYTES (8u << 20)
+int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const float *wI,
+                                  const void *KI, const float *KI_scale, int cap, int n_q,
+                                  int start_pos, int32_t *idx, float *scores, long long score_stride,
+                                  hca_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Shared-KV MQA with sink, [J] Eq.(18)-(19), (27), §2.3.3; [Z] Sparse
  * Attention, 输出投影.  For query t (head h) the key/value rows are the

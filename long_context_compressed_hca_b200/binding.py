@@ -80,6 +80,7 @@ def _declare(L):
                              VP, LL, VP, VP, VP]),
         "csa_index_topk_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
         "csa_index_topk": (I, [C.POINTER(AttnDesc), VP, VP, VP, VP, I, I, I, VP, VP, LL, VP, SZ, VP]),
+        "csa_index_topk_static_scratch": (I, [C.POINTER(AttnDesc), VP, VP, VP, VP, I, I, I, VP, VP, LL, VP]),
         "csa_attend_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
         "csa_attend": (I, [C.POINTER(AttnDesc), VP, VP, I, VP, VP, I, VP, I, I, VP, VP, SZ, VP]),
         "hca_attend_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
@@ -217,6 +218,17 @@ def csa_index_topk(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, 
     return check(lib().csa_index_topk(C.byref(d), ptr(qI), ptr(wI), ptr(KI), ptr(KI_scale), cap, n_q,
                                       start_pos, ptr(idx), ptr(scores), score_stride, ptr(ws), nbytes,
                                       stream_handle(stream)))
+
+
+# Size of the library's fixed scratch array used by csa_index_topk_static_scratch.
+STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def csa_index_topk_static_scratch(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, scores=None,
+                                  score_stride=0, stream=None):
+    return check(lib().csa_index_topk_static_scratch(C.byref(d), ptr(qI), ptr(wI), ptr(KI), ptr(KI_scale), cap,
+                                                     n_q, start_pos, ptr(idx), ptr(scores), score_stride,
+                                                     stream_handle(stream)))
 
 
 def csa_attend_workspace_size(d: AttnDesc, n_q, start_pos) -> int:

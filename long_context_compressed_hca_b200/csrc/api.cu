@@ -340,6 +340,22 @@ int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI, cons
   return run_index_topk(p, idx, scores, score_stride, ws, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
+int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const float *wI, const void *KI,
+                                  const float *KI_scale, int cap, int n_q, int start_pos, int32_t *idx,
+                                  float *scores, long long score_stride, hca_stream_t stream) {
+  int rc = check_attn_desc(d, true);
+  if (rc) return rc;
+  REQUIRE(n_q >= 0 && start_pos >= 0, "n_q and start_pos must be >= 0");
+  REQUIRE(qI && wI && idx, "qI, wI and idx must be non-null");
+  const int vmax = (start_pos + n_q) / d->m;
+  REQUIRE(cap >= vmax, "cap (%d) < visible entries (%d)", cap, vmax);
+  REQUIRE(vmax == 0 || KI, "KI must be non-null");
+  REQUIRE(d->idx_key_dtype != HCA_FP8E4M3 || KI_scale, "fp8 keys need KI_scale");
+  if (scores) REQUIRE(score_stride >= vmax, "score_stride < max visible entries");
+  IndexParams p = index_params(d, qI, wI, KI, KI_scale, cap, n_q, start_pos);
+  return run_index_topk_static(p, idx, scores, score_stride, static_cast<cudaStream_t>(stream));
+}
+
 // ----------------------------------------------------------------- attend
 size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
   if (!d) return 0;

@@ -10,6 +10,8 @@
 // of the fp32 scores (up to 4 passes of 8 bits), run by a thread-block cluster
 // whose CTAs hold slices of the row in shared memory and sum their histograms
 // through distributed shared memory, followed by a stable compaction.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -470,6 +472,57 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t2.n_seg = 1; t2.seg_len = pl2.seg_len; t2.slice = pl2.slice;
   t2.idx_out = idx; t2.out_stride = ip.k;
   return launch_topk_cluster("topk_pass2", t2, pl2, rows, s);
+}
+
+
+// ------------------------------------------------- static-scratch variant
+// Scratch for callers that cannot hand in a workspace: code that runs while
+// the caller's device allocator is itself busy (an out-of-memory handler, an
+// allocator hook), hosts whose device memory is reserved up front with no
+// room for a per-call buffer, and loops that must not call cudaMalloc /
+// cudaFree because those calls synchronise the device.  One array per device
+// (per process): calls that overlap in time on one device -- two streams, two
+// host threads, or a graph replay next to a direct call -- would share it and
+// race, so such callers must order their calls (one stream, or events).
+// Nothing in it must start at zero: the scorer writes every visible score of
+// every row before the selection reads it, and a segmented selection's first
+// launch writes every winner slot (padding included) before the merge reads it.
+namespace {
+static __device__ __align__(256) unsigned char g_index_topk_scratch[HCA_STATIC_SCRATCH_BYTES];
+
+// Device address of the scratch on the current device, looked up once per
+// device (the lookup may load the module, so it must not run during capture).
+int static_scratch(void **out) {
+  static std::mutex mu;
+  static void *cached[64] = {nullptr};
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(HCA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cached[dev]) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress((void **)&ptr, g_index_topk_scratch);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    cached[dev] = ptr;
+  }
+  *out = cached[dev];
+  return HCA_OK;
+}
+}  // namespace
+
+int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
+                          cudaStream_t s) {
+  const size_t need = topk_workspace_bytes(p);
+  if (need > (size_t)HCA_STATIC_SCRATCH_BYTES)
+    return fail(HCA_ERR_INVALID,
+                "csa_index_topk_static_scratch: this call needs %zu bytes of scratch (B*n_q rows x %d visible "
+                "entries x 4 bytes, plus segment winners), the static scratch holds %zu; use csa_index_topk",
+                need, (p.start_pos + p.n_q) / p.m, (size_t)HCA_STATIC_SCRATCH_BYTES);
+  void *scratch = nullptr;
+  const int rc = static_scratch(&scratch);
+  if (rc) return rc;
+  return run_index_topk(p, idx, user_scores, user_stride, scratch, (size_t)HCA_STATIC_SCRATCH_BYTES, s);
 }
 
 }  // namespace hca

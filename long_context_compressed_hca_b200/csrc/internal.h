@@ -88,6 +88,10 @@ struct TopkParams {
 size_t topk_workspace_bytes(const IndexParams &p);
 int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
                    void *ws, size_t ws_bytes, cudaStream_t s);
+// csa_index_topk with its scratch in a file-scope device array of
+// HCA_STATIC_SCRATCH_BYTES; fails with HCA_ERR_INVALID when the call needs more.
+int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
+                          cudaStream_t s);
 
 // ------------------------------------------------------------- attention
 struct AttendParams {
