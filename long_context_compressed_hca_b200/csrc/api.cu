@@ -181,6 +181,7 @@ AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv
   p.q = q; p.kv_comp = kv_comp; p.idx = idx; p.kv_win = kv_win; p.sink = sink; p.o = o; p.dtype = d->dtype;
   p.status = nullptr;
   p.nsplit = 1;
+  p.cluster = 0;
   return p;
 }
 

@@ -264,10 +264,13 @@ constexpr int kProdWarps = 8;
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kThreads = (kSoftmaxWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
+constexpr int kMaxClusterSplits = 8;         // portable cluster size
 
 struct Bars {
   uint64_t q_full, q_empty, o_empty, mma_done;
   uint64_t kv_full[8], kv_empty[8], s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t mg_ready, mg_full;    // cluster merge: peers' buffers free / peers' partials delivered
+  uint64_t mg_stage, mg_wt;      // cluster merge: this CTA's blocks staged / merge weights written
 };
 
 template <int C>
@@ -288,9 +291,194 @@ struct Layout {
 enum TraceSlot {
   TR_P_QEMPTY, TR_P_KVEMPTY, TR_M_QFULL, TR_M_KVFULL, TR_M_SEMPTY, TR_M_PFULL, TR_M_OEMPTY,
   TR_S_SFULL, TR_S_PBUF, TR_S_RESCALE, TR_S_EPI_WAIT, TR_S_TILE, TR_S_EPI, TR_TOTAL, TR_RESCALES, TR_UNITS,
-  TR_TILES, TR_P_ISSUE, TR_COUNT
+  TR_TILES, TR_P_ISSUE, TR_S_MERGE_READY, TR_S_MERGE_FULL, TR_S_PUSH, TR_S_WEIGHTS, TR_S_MERGE_LOOP, TR_COUNT
 };
 __device__ unsigned long long g_attn_trace[32];
+
+// Named barrier over the 4 softmax warps (warps 0-3).
+__device__ __forceinline__ void softmax_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
+}
+
+// ---------------------------------------------------------------- cluster merge
+// With nsplit <= 8 the splits of one query form a thread-block cluster (one
+// unit per CTA).  CTA `sp` owns output columns [sp*per, (sp+1)*per).  After
+// its last P.V, each CTA stages its unnormalised O rows (bf16) and per-row
+// (max, sum) as one block per owner, then one thread sends every other
+// owner its block with a bulk shared-to-distributed-shared copy that
+// completes on the owner's mg_full barrier.  Copies into a peer start only
+// once every CTA of the cluster has reported (mg_ready) that its tiles are
+// done, since the blocks overlay the Q and key-tile buffers.  The owner
+// forms  o = sum_i 2^{m_i-M} O_i / (sum_i 2^{m_i-M} l_i + 2^{sink-M})  for its
+// columns, applies the inverse RoPE and stores bf16.  The 4 softmax warps and
+// the 8 load warps (idle by then) share the work: 3 warps per TMEM lane
+// quarter read O, 384 threads merge.  All waits are bounded.
+__host__ __device__ constexpr int merge_cols(int C, int ns) { return ((C / ns + 15) / 16) * 16; }
+__host__ __device__ constexpr int merge_pitch(int C, int ns) { return merge_cols(C, ns) + 8; }   // bf16 elements
+// one owner's block: O [64][pitch] bf16, then (max, sum) [64] float2
+__host__ __device__ constexpr uint32_t merge_blk(int C, int ns) { return 64u * merge_pitch(C, ns) * 2 + 64 * 8; }
+// staged blocks [ns], received blocks [ns] (own slot unused), weights [64][8] fp32
+__host__ __device__ constexpr uint32_t merge_bytes(int C, int ns) { return 2u * ns * merge_blk(C, ns) + 64 * 8 * 4; }
+template <int C>
+__host__ __device__ constexpr bool merge_fits() {
+  for (int ns = 2; ns <= kMaxClusterSplits; ++ns)
+    if (merge_bytes(C, ns) > Layout<C>::p_off) return false;
+  return true;
+}
+constexpr int kMergeThreads = (kSoftmaxWarps + kProdWarps) * 32;
+
+// Bounded rendezvous of the 12 merge warps (softmax warps 0-3, load warps
+// 5-12) on a one-shot mbarrier that counts one arrival per warp.
+__device__ __forceinline__ bool merge_sync(uint64_t *b, int *status) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(smem_u32(b));
+  return mbar_wait(smem_u32(b), 0, status);
+}
+__device__ __forceinline__ void bulk_s2c(uint32_t dst_cluster, uint32_t src, uint32_t bytes, uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src), "r"(bytes), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Called by the 12 merge warps once the softmax warps have written every
+// staged block's (max, sum) and all have waited for the unit's last P.V.
+template <int C>
+__device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *smem, Bars *bars, uint32_t tmem,
+                                              int nt, int sp, int b, int qi, const float *rope_cs,
+                                              unsigned long long *trace) {
+  static_assert(merge_fits<C>(), "merge buffers overlap the P buffers");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = (warp < kSoftmaxWarps ? warp : warp - 1) * 32 + lane;   // 0..383
+  const int quarter = warp & 3, third = warp < kSoftmaxWarps ? 0 : 1 + (warp - kProdWarp0) / 4;
+  const int hl = lane & 15, half = lane >> 4;
+  const int r = quarter * 16 + hl;
+  const int ns = p.nsplit;
+  const int per = merge_cols(C, ns), pitch = merge_pitch(C, ns);
+  const uint32_t blk = merge_blk(C, ns);
+  uint8_t *stage = smem;                      // [ns] blocks
+  uint8_t *recv = smem + ns * blk;            // [ns] blocks
+  float *wt = reinterpret_cast<float *>(smem + 2 * ns * blk);
+  long long tw = trace ? clock64() : 0;
+  // ---- stage O (bf16), 16 columns per TMEM load
+  if (nt > 0) {
+    tc_fence_after();
+    const uint32_t tq = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int k = third; k < C / 32; k += 3) {
+      uint32_t ov[16];
+      tmem_ld_16x32bx2_x16<C / 2>(tq + 16 * k, ov);
+      tmem_ld_wait();
+      const int col0 = half * (C / 2) + 16 * k;
+      const int owner = col0 / per;
+      __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(stage + owner * blk) + r * pitch + (col0 - owner * per);
+      uint4 w0, w1;
+      w0.x = pack_bf16x2(__uint_as_float(ov[0]), __uint_as_float(ov[1]));
+      w0.y = pack_bf16x2(__uint_as_float(ov[2]), __uint_as_float(ov[3]));
+      w0.z = pack_bf16x2(__uint_as_float(ov[4]), __uint_as_float(ov[5]));
+      w0.w = pack_bf16x2(__uint_as_float(ov[6]), __uint_as_float(ov[7]));
+      w1.x = pack_bf16x2(__uint_as_float(ov[8]), __uint_as_float(ov[9]));
+      w1.y = pack_bf16x2(__uint_as_float(ov[10]), __uint_as_float(ov[11]));
+      w1.z = pack_bf16x2(__uint_as_float(ov[12]), __uint_as_float(ov[13]));
+      w1.w = pack_bf16x2(__uint_as_float(ov[14]), __uint_as_float(ov[15]));
+      reinterpret_cast<uint4 *>(dst)[0] = w0;
+      reinterpret_cast<uint4 *>(dst)[1] = w1;
+    }
+    tc_fence_before();
+  }
+  fence_proxy_async();   // staged blocks are read by the bulk-copy engine
+  if (!merge_sync(&bars->mg_stage, p.status)) return false;
+  if (trace) { const long long t = clock64(); trace[2] += t - tw; tw = t; }
+  // ---- every CTA's tiles are done -> send each owner its block
+  bool sent = false;
+  if (mt == 0) {
+    for (int j = 0; j < ns; ++j) mbar_arrive_cluster(cluster_map(smem_u32(&bars->mg_ready), j));
+    if (mbar_wait_cluster(smem_u32(&bars->mg_ready), 0, p.status)) {
+      for (int j = 0; j < ns; ++j)
+        if (j != sp)
+          bulk_s2c(cluster_map(smem_u32(recv + sp * blk), j), smem_u32(stage + j * blk), blk,
+                   cluster_map(smem_u32(&bars->mg_full), j));
+      bulk_commit();
+      sent = true;
+    }
+  }
+  if (trace) { const long long t = clock64(); trace[0] += t - tw; tw = t; }
+  bool ok = mbar_wait_cluster(smem_u32(&bars->mg_full), 0, p.status);
+  if (trace) { const long long t = clock64(); trace[1] += t - tw; tw = t; }
+  if (ok) {
+    // ---- merge weights of every head row
+    auto ml_of = [&](int i, int row) -> float2 {
+      const uint8_t *base = (i == sp ? stage + i * blk : recv + i * blk);
+      return reinterpret_cast<const float2 *>(base + 64u * pitch * 2)[row];
+    };
+    if (mt < 64) {
+      const float sink2 = mt < p.n_h ? p.sink[mt] * kLog2e : 0.f;
+      float M = sink2;
+      for (int i = 0; i < ns; ++i) {
+        const float2 v = ml_of(i, mt);
+        if (v.y > 0.f) M = fmaxf(M, v.x);
+      }
+      float den = exp2f(sink2 - M);
+      float e[kMaxClusterSplits];
+#pragma unroll
+      for (int i = 0; i < kMaxClusterSplits; ++i) {
+        const float2 v = i < ns ? ml_of(i, mt) : make_float2(0.f, 0.f);
+        e[i] = v.y > 0.f ? exp2f(v.x - M) : 0.f;
+        den += e[i] * v.y;
+      }
+      const float inv = 1.f / den;
+#pragma unroll
+      for (int i = 0; i < kMaxClusterSplits; ++i) wt[mt * 8 + i] = e[i] * inv;
+    }
+    ok = merge_sync(&bars->mg_wt, p.status);
+  }
+  if (ok) {
+    if (trace) { const long long t = clock64(); trace[3] += t - tw; tw = t; }
+    // ---- this CTA's columns of every head row, 8 columns per item
+    const int c_lo = min(C, sp * per), c_hi = min(C, c_lo + per);
+    const int ngr = (c_hi - c_lo) / 8;
+    for (int it = mt; it < 64 * ngr; it += kMergeThreads) {
+      const int row = it / ngr, cg = c_lo + 8 * (it % ngr);
+      if (row >= p.n_h) continue;
+      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < ns; ++i) {
+        const float w = wt[row * 8 + i];
+        if (w == 0.f) continue;
+        const uint8_t *base = (i == sp ? stage + i * blk : recv + i * blk);
+        const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(base) +
+                                                         row * pitch + (cg - c_lo));
+        o[0] += w * bf16_lo(v.x); o[1] += w * bf16_hi(v.x);
+        o[2] += w * bf16_lo(v.y); o[3] += w * bf16_hi(v.y);
+        o[4] += w * bf16_lo(v.z); o[5] += w * bf16_hi(v.z);
+        o[6] += w * bf16_lo(v.w); o[7] += w * bf16_hi(v.w);
+      }
+      if (cg + 8 > C - p.rd) {
+#pragma unroll
+        for (int x = 0; x < 8; x += 2) {
+          const int col = cg + x;
+          if (col >= C - p.rd) {
+            const int pi = (col - (C - p.rd)) / 2;
+            const float cs = rope_cs[pi], sn = rope_cs[32 + pi];
+            const float aa = o[x], bb = o[x + 1];
+            o[x] = aa * cs + bb * sn;
+            o[x + 1] = -aa * sn + bb * cs;
+          }
+        }
+      }
+      uint4 w4;
+      w4.x = pack_bf16x2(o[0], o[1]); w4.y = pack_bf16x2(o[2], o[3]);
+      w4.z = pack_bf16x2(o[4], o[5]); w4.w = pack_bf16x2(o[6], o[7]);
+      *reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                                 (((long long)b * p.n_q + qi) * p.n_h + row) * C + cg) = w4;
+    }
+    if (trace) trace[4] += clock64() - tw;
+  }
+  // the staged blocks must have been read before this CTA leaves
+  if (sent) bulk_wait_read_all();
+  return ok;
+}
 
 template <int C, bool TRACE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -334,6 +522,12 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(bars->p_full[i]), kSoftmaxWarps);
       mbar_init(bar(bars->pv_done[i]), 1);
     }
+    if (p.cluster) {
+      mbar_init(bar(bars->mg_ready), p.nsplit);
+      mbar_init(bar(bars->mg_full), 1);
+      mbar_init(bar(bars->mg_stage), kMergeThreads / 32);
+      mbar_init(bar(bars->mg_wt), kMergeThreads / 32);
+    }
     mbar_fence_init();
   }
   if (warp == kMmaWarp) {
@@ -346,6 +540,11 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // peers arrive on this CTA's merge barriers only after every CTA initialised its own
+  if (p.cluster) {
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(bar(bars->mg_full), (p.nsplit - 1) * merge_blk(C, p.nsplit));
+    cluster_sync();
+  }
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ loads
@@ -402,6 +601,24 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
     }
     }();
     cp_async_wait_all();
+    if (p.cluster) {
+      // one unit per CTA: join the merge once its last P.V has landed
+      const int u = blockIdx.x;
+      const int bq = u / p.nsplit, sp = u % p.nsplit;
+      const int b = bq / p.n_q, qi = bq % p.n_q;
+      const KeySet ks = key_set_tc(p, qi);
+      int j0, nt;
+      split_range(ks, p.nsplit, sp, j0, nt);
+      bool ok = true;
+      if (nt > 0) {
+        const uint32_t gl = nt - 1;
+        ok = mbar_wait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, p.status);
+      }
+      if (ok) {
+        // the softmax warps' (max, sum) writes and RoPE table are ordered by the merge barrier
+        cluster_merge<C>(p, smem, bars, tmem, nt, sp, b, qi, rope_all, nullptr);
+      }
+    }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
@@ -492,9 +709,9 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       const KeySet ks = key_set_tc(p, qi);
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
-      if (nt == 0 && p.nsplit > 1) continue;   // the combine kernel skips empty ranges
+      if (nt == 0 && p.nsplit > 1 && !p.cluster) continue;   // the combine kernel skips empty ranges
       __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
-      if (nt == 0) {
+      if (nt == 0 && !p.cluster) {
         if (r < p.n_h)
           for (int col = half * (C / 2); col < (half + 1) * (C / 2); col += 8)
             *reinterpret_cast<uint4 *>(orow + col) = make_uint4(0, 0, 0, 0);
@@ -597,11 +814,30 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         if (lane == 0) mbar_arrive(bar(bars->p_full[st]));
       }
       // -------- epilogue: normalise, inverse RoPE, store
-      const uint32_t gl = g + nt - 1;
-      if (!twait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, TR_S_EPI_WAIT)) return;
+      if (nt > 0) {
+        const uint32_t gl = g + nt - 1;
+        if (!twait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, TR_S_EPI_WAIT)) return;
+      }
       const long long te0 = TRACE ? clock64() : 0;
       tc_fence_after();
       const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      if (p.cluster) {
+        // (max, sum) of this row into every owner's block, then the shared merge
+        if (half == 0) {
+          const uint32_t blk = merge_blk(C, p.nsplit);
+          const int pitch = merge_pitch(C, p.nsplit);
+          for (int j = 0; j < p.nsplit; ++j)
+            reinterpret_cast<float2 *>(smem + j * blk + 64u * pitch * 2)[r] =
+                make_float2(nt > 0 ? m_used : -INFINITY, nt > 0 ? ltot : 0.f);
+        }
+        if (!cluster_merge<C>(p, smem, bars, tmem, nt, sp, b, qi, rope_all,
+                              TRACE ? &tr[TR_S_MERGE_READY] : nullptr))
+          return;
+        if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+        g += nt;
+        ++iq;
+        continue;
+      }
       if (p.nsplit > 1) {
         // unnormalised partial: O rows (fp32), running max (log2 units) and sum
         const long long slot = (long long)bq * p.nsplit + sp;
@@ -687,18 +923,54 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
 }
 
 template <int C>
-int launch_tc(const AttendParams &p, cudaStream_t s) {
-  const int n_units = p.B * p.n_q * p.nsplit;
-  const size_t smem = Layout<C>::bytes;
+int ensure_attr() {
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int smem = (int)Layout<C>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_tc<C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      e = cudaFuncSetAttribute(attend_tc<C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "attend_tc smem attribute: %s", cudaGetErrorString(e));
     attr_set = true;
   }
-  const int grid = n_units < num_sms() ? n_units : num_sms();
+  return HCA_OK;
+}
+
+// How many clusters of `ns` CTAs can be resident at once (0 if unknown).
+template <int C>
+int max_active_clusters(int ns) {
+  static int cache[kMaxClusterSplits + 1] = {0};
+  if (ns < 1 || ns > kMaxClusterSplits) return 0;
+  if (cache[ns]) return cache[ns];
+  if (ensure_attr<C>()) return 0;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ns * 64, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Layout<C>::bytes;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = ns;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<C, false>, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cache[ns] = n;
+  return n;
+}
+
+template <int C>
+int launch_tc(const AttendParams &p, cudaStream_t s) {
+  const int n_units = p.B * p.n_q * p.nsplit;
+  const size_t smem = Layout<C>::bytes;
+  int rc0 = ensure_attr<C>();
+  if (rc0) return rc0;
+  // cluster merge: one unit per CTA, a query's splits form one cluster
+  const int grid = p.cluster ? n_units : (n_units < num_sms() ? n_units : num_sms());
   // tensor maps: q rows (box 64 x 64), compressed and window rows (box 1 x 64)
   CUtensorMap tmQ, tmC, tmW;
   const void *cbase = p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q);
@@ -713,6 +985,28 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
                                CU_TENSOR_MAP_SWIZZLE_128B);
   if (rc) return rc;
   LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
+  if (p.cluster) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = p.nsplit;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e = attend_trace_on()
+                              ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units, tmQ, tmC, tmW)
+                              : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units, tmQ, tmC, tmW);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return fail(HCA_ERR_CUDA, "attend_tc cluster launch: %s", cudaGetErrorString(e));
+    }
+    return ls_.done();
+  }
   if (attend_trace_on()) attend_tc<C, true><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
   else attend_tc<C, false><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
   return ls_.done();
@@ -727,7 +1021,7 @@ bool tc_path(const AttendParams &p) {
          p.rd % 2 == 0 && p.rd <= 64;
 }
 // Splits per query: enough work units to fill the GPU when there are few queries.
-int choose_splits(const AttendParams &p) {
+int choose_splits_raw(const AttendParams &p) {
   const long long q = (long long)p.B * p.n_q;
   if (q == 0 || q >= num_sms()) return 1;
   // longest key list among the queries (the last one)
@@ -740,12 +1034,45 @@ int choose_splits(const AttendParams &p) {
   if (ns > 32) ns = 32;
   return ns < 1 ? 1 : ns;
 }
+int max_active_clusters_for(const AttendParams &p, int ns) {
+  switch (p.c) {
+    case 128: return tc::max_active_clusters<128>(ns);
+    case 256: return tc::max_active_clusters<256>(ns);
+    default: return tc::max_active_clusters<512>(ns);
+  }
+}
+// Split plan: with at most 8 splits per query the splits of a query run as
+// one thread-block cluster and merge through distributed shared memory (no
+// workspace, no combine launch); the split count is lowered until all the
+// clusters are resident at once.  More splits go through the workspace and
+// the combine kernel when the caller gave one, else are cut to 8.
+struct SplitPlan {
+  int ns, cluster;
+};
+SplitPlan plan_splits(const AttendParams &p, bool have_ws) {
+  SplitPlan sp{choose_splits_raw(p), 0};
+  if (sp.ns <= 1 || (sp.ns > tc::kMaxClusterSplits && have_ws)) return sp;
+  if (sp.ns > tc::kMaxClusterSplits) sp.ns = tc::kMaxClusterSplits;
+  {
+    const long long q = (long long)p.B * p.n_q;
+    int ns = sp.ns;
+    while (ns > 1) {
+      const int fit = max_active_clusters_for(p, ns);
+      if (fit == 0 || fit >= q) break;   // unknown occupancy: keep the split count
+      --ns;
+    }
+    sp.ns = ns;
+    sp.cluster = ns > 1;
+  }
+  return sp;
+}
 }  // namespace
 
 size_t attend_workspace_bytes(const AttendParams &p) {
   if (!tc_path(p)) return 0;
-  const int ns = choose_splits(p);
-  if (ns <= 1) return 0;
+  const SplitPlan sp = plan_splits(p, true);
+  const int ns = sp.ns;
+  if (ns <= 1 || sp.cluster) return 0;
   const size_t q = (size_t)p.B * p.n_q * ns * 64;
   return ((q * p.c * 4 + 255) & ~(size_t)255) + ((q * 8 + 255) & ~(size_t)255);
 }
@@ -754,10 +1081,15 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
   if (p_in.B * p_in.n_q == 0) return HCA_OK;
   AttendParams p = p_in;
   p.nsplit = 1;
+  p.cluster = 0;
   if (tc_path(p)) {
     if (!p.kv_comp) p.cap = 0;   // no visible entries: masked slots then read row 0 of the dummy map
-    const int ns = choose_splits(p);
-    if (ns > 1 && ws && ws_bytes >= attend_workspace_bytes(p)) {
+    const SplitPlan sp = plan_splits(p, ws && ws_bytes >= attend_workspace_bytes(p));
+    const int ns = sp.ns;
+    if (sp.cluster) {
+      p.nsplit = ns;
+      p.cluster = 1;
+    } else if (ns > 1 && ws && ws_bytes >= attend_workspace_bytes(p)) {
       p.nsplit = ns;
       const size_t q = (size_t)p.B * p.n_q * ns * 64;
       p.part_o = static_cast<float *>(ws);
@@ -769,7 +1101,7 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
       case 256: rc = tc::launch_tc<256>(p, s); break;
       default: rc = tc::launch_tc<512>(p, s); break;
     }
-    if (rc || p.nsplit == 1) return rc;
+    if (rc || p.nsplit == 1 || p.cluster) return rc;
     return HCA_LAUNCH("attend_combine", s, attend_combine<__nv_bfloat16><<<dim3(p.B * p.n_q, (p.n_h + 3) / 4), 128, 0, s>>>(p));
   }
   dim3 grid(p.B * p.n_q, (p.n_h + kSimtWarps - 1) / kSimtWarps);

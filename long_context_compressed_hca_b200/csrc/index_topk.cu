@@ -96,25 +96,12 @@ __device__ __forceinline__ uint32_t order_bits(uint32_t u) {
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                 // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 1 for every non-NaN float
 }
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_sync() { cluster_arrive(); cluster_wait(); }
-// Load a 32-bit word from the same shared-memory variable in CTA `rank`.
+// Load from the same shared-memory variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t dsmem_ld(const void *local, uint32_t rank) {
-  uint32_t ra, v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
-  return v;
+  return ld_dsmem_u32(cluster_map(smem_u32(local), rank));
+}
+__device__ __forceinline__ uint4 dsmem_ld4(const void *local, uint32_t rank) {
+  return ld_dsmem_u32x4(cluster_map(smem_u32(local), rank));
 }
 
 // Add one key to a shared histogram (bin 256 = no key).  The lanes that
@@ -177,15 +164,16 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   uint32_t *keys = dyn;               // [slice]
   uint32_t *cand = dyn + p.slice;     // [kCandMax]
   __shared__ uint32_t sub[4][256];
-  __shared__ uint32_t pub[2][256];    // this CTA's histogram of pass (parity), read by the cluster
-  __shared__ uint32_t tot[256];
+  __shared__ __align__(16) uint32_t pub[2][256];   // this CTA's histogram of pass (parity), read by the cluster
+  __shared__ __align__(16) uint32_t tot[256];
   __shared__ int pub_cnt[2];          // this CTA's keys above / equal to the threshold
+  __shared__ int peer_cnt[kClusterMax][2];
   __shared__ int w_gt[kTopkWarps], w_eq[kTopkWarps];
   __shared__ int s_total, s_krem, s_nc, s_base, s_eqb;
   __shared__ uint32_t s_digit;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t C = cluster_size(), rank = cluster_rank();
+  const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
   const long long unit = blockIdx.x / C;
   const int row = (int)(unit / p.n_seg), seg = (int)(unit % p.n_seg);
   const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
@@ -220,10 +208,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     __syncthreads();
     if (tid < 256) pub[pass & 1][tid] = sub[0][tid] + sub[1][tid] + sub[2][tid] + sub[3][tid];
     cluster_sync();
-    if (tid < 256) {
-      uint32_t t = 0;
-      for (uint32_t r = 0; r < C; ++r) t += dsmem_ld(&pub[pass & 1][tid], r);
-      tot[tid] = t;
+    if (tid < 64) {
+      // 4 bins per thread; the C loads are issued before any is summed
+      uint4 v[kClusterMax];
+#pragma unroll
+      for (int r = 0; r < kClusterMax; ++r)
+        if (r < (int)C) v[r] = dsmem_ld4(&pub[pass & 1][4 * tid], r);
+      uint4 t = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int r = 0; r < kClusterMax; ++r)
+        if (r < (int)C) { t.x += v[r].x; t.y += v[r].y; t.z += v[r].z; t.w += v[r].w; }
+      *reinterpret_cast<uint4 *>(&tot[4 * tid]) = t;
     }
     __syncthreads();
     if (warp == 0) {
@@ -297,18 +292,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     pub_cnt[1] = b;
   }
   cluster_sync();
+  if (tid < (int)rank) {
+    peer_cnt[tid][0] = (int)dsmem_ld(&pub_cnt[0], tid);
+    peer_cnt[tid][1] = (int)dsmem_ld(&pub_cnt[1], tid);
+  }
+  cluster_arrive();   // this CTA reads no other CTA's shared memory past here
+  __syncthreads();
   if (tid == 0) {
     // winners of the lower-ranked CTAs, and ties among them
     int base = 0, eqb = 0;
     for (uint32_t r = 0; r < rank; ++r) {
-      const int g = (int)dsmem_ld(&pub_cnt[0], r), e = (int)dsmem_ld(&pub_cnt[1], r);
-      base += g + max(0, min(krem - eqb, e));
-      eqb += e;
+      base += peer_cnt[r][0] + max(0, min(krem - eqb, peer_cnt[r][1]));
+      eqb += peer_cnt[r][1];
     }
     s_base = base;
     s_eqb = eqb;
   }
-  cluster_arrive();   // this CTA reads no other CTA's shared memory past here
   __syncthreads();
   int ties_before = s_eqb, sel_before = s_base;
   for (int w = 0; w < warp; ++w) { ties_before += w_eq[w]; sel_before += w_gt[w]; }

@@ -108,9 +108,12 @@ struct AttendParams {
   hca_dtype dtype;
   int *status;
   // split-KV: each query's key list is cut into nsplit tile ranges whose
-  // unnormalised partials (fp32 O rows, running max and sum) go to part_o /
-  // part_ml and are merged by a combine kernel
+  // unnormalised partials (fp32 O rows, running max and sum) are merged
+  // either by the CTAs of one thread-block cluster through distributed shared
+  // memory (cluster = 1, nsplit <= 8) or through part_o / part_ml and a
+  // combine kernel (cluster = 0)
   int nsplit;
+  int cluster;
   float *part_o;           // [B*n_q, nsplit, 64, c]
   float *part_ml;          // [B*n_q, nsplit, 64, 2]
 };

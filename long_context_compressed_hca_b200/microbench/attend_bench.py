@@ -41,12 +41,37 @@ def decode_main():
     wsz = (hb.csa_attend_workspace_size if kind == "csa" else hb.hca_attend_workspace_size)(d, 1, pos)
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 
-    def run():
+    def run(use_ws=True):
+        w = ws if use_ws else None
         if kind == "csa":
-            hb.csa_attend(d, q, kv, cap, idx, ring, 1, sink, 1, pos, o, ws)
+            hb.csa_attend(d, q, kv, cap, idx, ring, 1, sink, 1, pos, o, w)
         else:
-            hb.hca_attend(d, q, kv, cap, ring, 1, sink, 1, pos, o, ws)
+            hb.hca_attend(d, q, kv, cap, ring, 1, sink, 1, pos, o, w)
 
+    # device time per call from CUDA-graph replays (no host work in the interval):
+    # with the workspace (fp32 partials + combine kernel) and without it (cluster merge)
+    outs = {}
+    for use_ws in (True, False):
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            for _ in range(3):
+                run(use_ws)
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=st):
+                for _ in range(10):
+                    run(use_ws)
+            gr.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for _ in range(5):
+                gr.replay()
+            e1.record(st)
+            torch.cuda.synchronize()
+            outs[use_ws] = o.clone()
+        print(f"{'workspace + combine' if use_ws else 'cluster merge'}: {e0.elapsed_time(e1) / 50 * 1e3:.2f} us per call")
+    print("max |workspace - cluster| =", (outs[True].float() - outs[False].float()).abs().max().item())
     for _ in range(3):
         run()
     torch.cuda.synchronize()
@@ -66,7 +91,7 @@ def decode_main():
     att = [v for kk, v in prof.items() if kk.startswith("attend_") and kk.endswith("tc")][0]
     print(f"gathered+q/o bytes {byts / 1e6:.1f} MB -> {byts / (att[1] / att[0] * 1e-3) / 1e9:.0f} GB/s in the attention kernel")
     hb.trace_attend(1)
-    run()
+    run(False)
     tr = hb.trace_attend_read()
     hb.trace_attend(0)
     tot = tr["total"]
@@ -123,7 +148,7 @@ def main():
     flops = keys * n_h * c * 4
     print(f"attend {kind} n_q={n_q} c={c}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s")
     hb.trace_attend(1)
-    run()
+    run(False)
     tr = hb.trace_attend_read()
     hb.trace_attend(0)
     tot = tr["total"]   # summed over the three reporting roles

@@ -314,6 +314,20 @@ def test_attend_decode_ring(cuda, kind, pos):
         assert_close(to64(o[b, 0]), ref, 2e-2, f"o[{b}]")
 
 
+@pytest.mark.parametrize("kind,B,pos", [("csa", 5, 1700), ("hca", 2, 100000), ("csa", 32, 131071)])
+def test_attend_decode_cluster_merge(cuda, kind, B, pos):
+    """Decode with few sequences: each query's key tiles are split over the
+    CTAs of one cluster (here 4 splits of 9 tiles, the last one empty; 7
+    splits; the 128K batch) and merged through distributed shared memory."""
+    n_h, c, rd, w = 64, 512, 64, 128
+    m, k = (4, 512) if kind == "csa" else (128, 0)
+    q, kv_comp, kv_win, sink, idx, o = _run_attend(kind, BF16, B, 1, n_h, c, rd, w, m, k, cuda,
+                                                   start_pos=pos, ring=True)
+    for b in range(0, B, max(1, B // 4)):
+        ref = _ref_attend(kind, q, kv_comp, kv_win, sink, idx, b, 0, pos, w, m, k, rd, True)
+        assert_close(to64(o[b, 0]), ref, 2e-2, f"o[{b}]")
+
+
 def test_attend_is_deterministic(cuda):
     runs = [_run_attend("csa", BF16, 1, 64, 64, 512, 64, 128, 4, 128, cuda)[-1] for _ in range(2)]
     assert torch.equal(runs[0], runs[1])
