@@ -200,6 +200,45 @@ int check_attend_args(const hca_attn_desc *d, const void *q, const void *kv_comp
 }
 
 }  // namespace
+int compress_params(const hca_compress_desc *d, int start_pos, int n, const void *Ca, const void *Cb,
+                    const void *Za, const void *Zb, long long row_stride, long long seq_stride, const float *Ba,
+                    const float *Bb, const float *gamma, void *out, float *out_scale, long long out_seq_stride,
+                    float *state_kv, float *state_score, CompressParams *pp) {
+  REQUIRE(d != nullptr, "null descriptor");
+  REQUIRE(d->B >= 1 && d->m >= 1, "B and m must be >= 1");
+  REQUIRE(d->width >= 8 && d->width % 8 == 0, "width must be a positive multiple of 8");
+  REQUIRE(d->overlap == 0 || d->overlap == 1, "overlap must be 0 or 1");
+  REQUIRE(d->in_dtype == HCA_F32 || d->in_dtype == HCA_BF16, "in_dtype must be f32 or bf16");
+  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16 || d->out_dtype == HCA_FP8E4M3, "bad out_dtype");
+  if (d->flags & HCA_COMPRESS_ROPE)
+    REQUIRE(d->rd >= 0 && d->rd <= d->width && d->rd % 8 == 0, "rd must be a multiple of 8 and <= width");
+  REQUIRE(n >= 0 && start_pos >= 0, "n and start_pos must be >= 0");
+  REQUIRE(Ca && Za && Ba, "Ca, Za and Ba must be non-null");
+  if (d->overlap) REQUIRE(Cb && Zb && Bb, "overlap needs Cb, Zb and Bb");
+  const size_t es = esize(d->in_dtype);
+  REQUIRE(aligned16(Ca) && aligned16(Za) && (!d->overlap || (aligned16(Cb) && aligned16(Zb))),
+          "C/Z pointers must be 16-byte aligned");
+  REQUIRE(row_stride >= d->width && (row_stride * (long long)es) % 16 == 0, "row_stride invalid");
+  REQUIRE((seq_stride * (long long)es) % 16 == 0, "seq_stride must keep 16-byte alignment");
+  REQUIRE(d->out_dtype != HCA_FP8E4M3 || out_scale, "fp8 output needs out_scale");
+  if (start_pos > 0) {
+    REQUIRE(n == 1, "decode mode (start_pos > 0) takes exactly one token");
+    REQUIRE(state_kv && state_score, "decode mode needs the compressor state");
+    if ((start_pos + 1) % d->m == 0)
+      REQUIRE(out && aligned16(out) && out_seq_stride > start_pos / d->m, "out too small for entry %d",
+              start_pos / d->m);
+  }
+  CompressParams p{};
+  p.B = d->B; p.n = n; p.width = d->width; p.m = d->m; p.overlap = d->overlap;
+  p.rd = (d->flags & HCA_COMPRESS_ROPE) ? d->rd : 0; p.flags = d->flags;
+  p.eps = d->eps > 0.f ? d->eps : 1e-6f; p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
+  p.Ca = Ca; p.Cb = Cb; p.Za = Za; p.Zb = Zb; p.row_stride = row_stride; p.seq_stride = seq_stride;
+  p.Ba = Ba; p.Bb = Bb; p.gamma = gamma; p.out = out; p.out_scale = out_scale; p.out_seq_stride = out_seq_stride;
+  p.state_kv = state_kv; p.state_score = state_score; p.in_dtype = d->in_dtype; p.out_dtype = d->out_dtype;
+  *pp = p;
+  return HCA_OK;
+}
+
 }  // namespace hca
 
 using namespace hca;
@@ -271,36 +310,16 @@ int csa_compress(const hca_compress_desc *d, int start_pos, int n, const void *C
                  const void *Za, const void *Zb, long long row_stride, long long seq_stride,
                  const float *Ba, const float *Bb, const float *gamma, void *out, float *out_scale,
                  long long out_seq_stride, float *state_kv, float *state_score, hca_stream_t stream) {
-  REQUIRE(d != nullptr, "null descriptor");
-  REQUIRE(d->B >= 1 && d->m >= 1, "B and m must be >= 1");
-  REQUIRE(d->width >= 8 && d->width % 8 == 0, "width must be a positive multiple of 8");
-  REQUIRE(d->overlap == 0 || d->overlap == 1, "overlap must be 0 or 1");
-  REQUIRE(d->in_dtype == HCA_F32 || d->in_dtype == HCA_BF16, "in_dtype must be f32 or bf16");
-  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16 || d->out_dtype == HCA_FP8E4M3, "bad out_dtype");
-  if (d->flags & HCA_COMPRESS_ROPE)
-    REQUIRE(d->rd >= 0 && d->rd <= d->width && d->rd % 8 == 0, "rd must be a multiple of 8 and <= width");
-  REQUIRE(n >= 0 && start_pos >= 0, "n and start_pos must be >= 0");
-  REQUIRE(Ca && Za && Ba, "Ca, Za and Ba must be non-null");
-  if (d->overlap) REQUIRE(Cb && Zb && Bb, "overlap needs Cb, Zb and Bb");
-  const size_t es = esize(d->in_dtype);
-  REQUIRE(aligned16(Ca) && aligned16(Za) && (!d->overlap || (aligned16(Cb) && aligned16(Zb))),
-          "C/Z pointers must be 16-byte aligned");
-  REQUIRE(row_stride >= d->width && (row_stride * (long long)es) % 16 == 0, "row_stride invalid");
-  REQUIRE((seq_stride * (long long)es) % 16 == 0, "seq_stride must keep 16-byte alignment");
-  REQUIRE(d->out_dtype != HCA_FP8E4M3 || out_scale, "fp8 output needs out_scale");
   CompressParams p{};
-  p.B = d->B; p.n = n; p.width = d->width; p.m = d->m; p.overlap = d->overlap;
-  p.rd = (d->flags & HCA_COMPRESS_ROPE) ? d->rd : 0; p.flags = d->flags;
-  p.eps = d->eps > 0.f ? d->eps : 1e-6f; p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
-  p.Ca = Ca; p.Cb = Cb; p.Za = Za; p.Zb = Zb; p.row_stride = row_stride; p.seq_stride = seq_stride;
-  p.Ba = Ba; p.Bb = Bb; p.gamma = gamma; p.out = out; p.out_scale = out_scale; p.out_seq_stride = out_seq_stride;
-  p.state_kv = state_kv; p.state_score = state_score; p.in_dtype = d->in_dtype; p.out_dtype = d->out_dtype;
+  int rc = compress_params(d, start_pos, n, Ca, Cb, Za, Zb, row_stride, seq_stride, Ba, Bb, gamma, out, out_scale,
+                           out_seq_stride, state_kv, state_score, &p);
+  if (rc) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (start_pos == 0) {
     const int E = n / d->m;
     if (E > 0) {
       REQUIRE(out && aligned16(out) && out_seq_stride >= E, "out must hold n/m entries per sequence");
-      int rc = launch_compress_prefill(p, s);
+      rc = launch_compress_prefill(p, s);
       if (rc) return rc;
     }
     if (state_kv || state_score) {
@@ -309,11 +328,6 @@ int csa_compress(const hca_compress_desc *d, int start_pos, int n, const void *C
     }
     return HCA_OK;
   }
-  REQUIRE(n == 1, "decode mode (start_pos > 0) takes exactly one token");
-  REQUIRE(state_kv && state_score, "decode mode needs the compressor state");
-  if ((start_pos + 1) % d->m == 0)
-    REQUIRE(out && aligned16(out) && out_seq_stride > start_pos / d->m, "out too small for entry %d",
-            start_pos / d->m);
   return launch_compress_decode(p, start_pos, s);
 }
 

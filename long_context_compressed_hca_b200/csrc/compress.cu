@@ -229,11 +229,9 @@ __global__ void compress_state_prefill_kernel(CompressParams p) {
   }
 }
 
-// Decode: one block per sequence.
+// Decode: one block per sequence.  `sm` holds (width + width/4) floats.
 template <typename Tin, typename Tout>
-__global__ void __launch_bounds__(kThreads) compress_decode_kernel(CompressParams p, int pos) {
-  extern __shared__ float sm[];
-  const int b = blockIdx.x;
+__device__ __forceinline__ void compress_decode_block(const CompressParams &p, int pos, int b, float *sm) {
   const int m = p.m, W = p.width;
   const int R = p.overlap ? 2 * m : m;
   const int C = p.overlap ? 2 * W : W;
@@ -313,6 +311,31 @@ __global__ void __launch_bounds__(kThreads) compress_decode_kernel(CompressParam
   }
 }
 
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads) compress_decode_kernel(CompressParams p, int pos) {
+  extern __shared__ float sm[];
+  compress_decode_block<Tin, Tout>(p, pos, blockIdx.x, sm);
+}
+
+// One decode token of one layer in one launch: blockIdx.y = 0 advances the
+// main compressor, 1 the indexer compressor (when present), the last part
+// writes the token's window row into the ring.  blockIdx.x = sequence.
+template <typename Tin, typename TA, typename TB, typename Tw>
+__global__ void __launch_bounds__(kThreads) decode_ingest_kernel(CompressParams pa, CompressParams pb, int has_b,
+                                                                 IngestRing ring, int pos) {
+  extern __shared__ float sm[];
+  const int b = blockIdx.x, part = blockIdx.y;
+  if (part == 0 && pa.B > 0) {
+    compress_decode_block<Tin, TA>(pa, pos, b, sm);
+  } else if (part == 1 && has_b) {
+    compress_decode_block<Tin, TB>(pb, pos, b, sm);
+  } else if (ring.ring) {
+    const Tw *row = reinterpret_cast<const Tw *>(ring.row) + (long long)b * ring.c;
+    Tw *dst = reinterpret_cast<Tw *>(ring.ring) + ((long long)b * ring.w + ring.slot) * ring.c;
+    for (int col = threadIdx.x; col < ring.c; col += kThreads) dst[col] = row[col];
+  }
+}
+
 template <typename Tin>
 int launch_prefill_t(const CompressParams &p, cudaStream_t s) {
   const int cv = p.width / 8;
@@ -368,6 +391,40 @@ int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s) {
 int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s) {
   return p.in_dtype == HCA_F32 ? launch_decode_t<float>(p, pos, s)
                                : launch_decode_t<__nv_bfloat16>(p, pos, s);
+}
+
+int launch_decode_ingest(const CompressParams *pa, const CompressParams *pb, const IngestRing &ring, int B, int pos,
+                         cudaStream_t s) {
+  const int parts = (pa ? 1 : 0) + (pb ? 1 : 0) + (ring.ring ? 1 : 0);
+  if (parts == 0 || B == 0) return HCA_OK;
+  CompressParams a = pa ? *pa : CompressParams{};
+  CompressParams bb = pb ? *pb : CompressParams{};
+  if (!pa) a.B = 0;
+  // part indices: 0 = main (may be empty), 1 = indexer (may be absent), last = ring
+  const int ny = pb ? (ring.ring ? 3 : 2) : (ring.ring ? 2 : 1);
+  const int wmax = (pa ? a.width : 0) > (pb ? bb.width : 0) ? (pa ? a.width : 0) : (pb ? bb.width : 0);
+  const size_t smem = (size_t)(wmax + 2 * (wmax / 8)) * sizeof(float);
+  const hca_dtype ta = pa ? a.out_dtype : (ring.dtype == HCA_F32 ? HCA_F32 : HCA_BF16);
+  const hca_dtype tb = pb ? bb.out_dtype : ta;
+  const bool in32 = (pa ? a.in_dtype : (pb ? bb.in_dtype : HCA_F32)) == HCA_F32;
+  if (!in32) return fail(HCA_ERR_UNSUPPORTED, "decode ingest takes fp32 compressor inputs");
+  if (ring.ring && ring.dtype != ta) return fail(HCA_ERR_UNSUPPORTED, "window dtype must match the entry dtype");
+  const dim3 grid(B, ny);
+  LaunchScope ls_("decode_ingest", s);
+  const int hb = pb ? 1 : 0;
+  if (ta == HCA_F32 && tb == HCA_F32)
+    decode_ingest_kernel<float, float, float, float><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  else if (ta == HCA_BF16 && tb == HCA_BF16)
+    decode_ingest_kernel<float, __nv_bfloat16, __nv_bfloat16, __nv_bfloat16><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  else if (ta == HCA_BF16 && tb == HCA_FP8E4M3)
+    decode_ingest_kernel<float, __nv_bfloat16, uint8_t, __nv_bfloat16><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  else if (ta == HCA_F32 && tb == HCA_FP8E4M3)
+    decode_ingest_kernel<float, float, uint8_t, float><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  else if (ta == HCA_F32 && tb == HCA_BF16)
+    decode_ingest_kernel<float, float, __nv_bfloat16, float><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  else
+    decode_ingest_kernel<float, __nv_bfloat16, float, __nv_bfloat16><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
+  return ls_.done();
 }
 
 }  // namespace hca

@@ -95,6 +95,10 @@ __global__ void row_op_kernel(RowOpParams p) {
 int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long long ldb, void *C,
                 long long ldc, hca_dtype cdt, int M, int N, int K, float alpha, cudaStream_t s) {
   if (M == 0 || N == 0) return HCA_OK;
+  if (ab == HCA_BF16) {
+    const int rc = launch_gemm_tc(A, lda, Bm, ldb, C, ldc, cdt, M, N, K, alpha, s);
+    if (rc != HCA_ERR_UNSUPPORTED) return rc;
+  }
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
   LaunchScope ls_("gemm_simt", s);
   if (ab == HCA_F32) {

@@ -78,9 +78,9 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
 // One thread-block cluster of C CTAs (C <= 8) selects the top-k of one row
 // segment; CTA r of the cluster holds keys [r*slice, (r+1)*slice) of the
 // segment in shared memory.  Each radix pass (8 bits, top byte first) builds
-// a CTA-local 256-bin histogram, the C histograms are summed through
-// distributed shared memory, and every CTA derives the same digit from the
-// same totals.  Once a CTA's keys that still match the threshold prefix fit
+// a CTA-local 256-bin histogram that every CTA stores into every peer's
+// inbox (distributed shared memory, stores only), so that after one cluster
+// barrier every CTA sums the same C histograms and derives the same digit.  Once a CTA's keys that still match the threshold prefix fit
 // in kCandMax they are compacted and later passes scan only those.  The final
 // stable compaction offsets each CTA's output by the winners of the lower-
 // ranked CTAs, so the selection leaves in ascending index order with ties
@@ -96,14 +96,6 @@ __device__ __forceinline__ uint32_t order_bits(uint32_t u) {
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                 // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 1 for every non-NaN float
 }
-// Load from the same shared-memory variable in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t dsmem_ld(const void *local, uint32_t rank) {
-  return ld_dsmem_u32(cluster_map(smem_u32(local), rank));
-}
-__device__ __forceinline__ uint4 dsmem_ld4(const void *local, uint32_t rank) {
-  return ld_dsmem_u32x4(cluster_map(smem_u32(local), rank));
-}
-
 // Add one key to a shared histogram (bin 256 = no key).  The lanes that
 // share the first pending lane's bin are folded into one atomic, twice, which
 // keeps clustered scores (one dominant bin) from serialising the warp.
@@ -163,11 +155,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   extern __shared__ __align__(16) uint32_t dyn[];
   uint32_t *keys = dyn;               // [slice]
   uint32_t *cand = dyn + p.slice;     // [kCandMax]
-  __shared__ uint32_t sub[4][256];
-  __shared__ __align__(16) uint32_t pub[2][256];   // this CTA's histogram of pass (parity), read by the cluster
+  __shared__ __align__(16) uint32_t sub[4][256];    // this CTA's histogram, 4 copies
+  __shared__ __align__(16) uint32_t mine[256];      // this CTA's histogram of the current pass
+  // every CTA's histogram of pass (parity), written by that CTA into each peer
+  __shared__ __align__(16) uint32_t inbox[2][kClusterMax][256];
   __shared__ __align__(16) uint32_t tot[256];
-  __shared__ int pub_cnt[2];          // this CTA's keys above / equal to the threshold
-  __shared__ int peer_cnt[kClusterMax][2];
+  __shared__ __align__(8) int peer_cnt[kClusterMax][2];   // every CTA's keys above / equal to the threshold
   __shared__ int w_gt[kTopkWarps], w_eq[kTopkWarps];
   __shared__ int s_total, s_krem, s_nc, s_base, s_eqb;
   __shared__ uint32_t s_digit;
@@ -185,6 +178,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
   else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
   if (tid == 0) s_nc = 0;
+  for (int i = tid; i < 4 * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
+  __syncthreads();
 
   uint32_t prefix = 0, mask = 0, T = 0;
   int krem = p.k, K = 0;
@@ -194,8 +189,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     const int shift = 24 - 8 * pass;
     const uint32_t *arr = compacted ? cand : keys;
     const int n = compacted ? nc : len;
-    for (int i = tid; i < 4 * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
-    __syncthreads();
     for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
       const int i = b0 + tid;
       uint32_t bin = 256u;
@@ -206,18 +199,28 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
       hist_add(sub[warp & 3], bin);
     }
     __syncthreads();
-    if (tid < 256) pub[pass & 1][tid] = sub[0][tid] + sub[1][tid] + sub[2][tid] + sub[3][tid];
-    cluster_sync();
     if (tid < 64) {
-      // 4 bins per thread; the C loads are issued before any is summed
-      uint4 v[kClusterMax];
+      // 4 bins per thread: sum (and clear) the 4 copies, then store the counts
+      // into every CTA's inbox slot for this rank
+      uint4 c = make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int r = 0; r < kClusterMax; ++r)
-        if (r < (int)C) v[r] = dsmem_ld4(&pub[pass & 1][4 * tid], r);
+      for (int w = 0; w < 4; ++w) {
+        uint4 *sp4 = reinterpret_cast<uint4 *>(&sub[w][4 * tid]);
+        const uint4 v = *sp4;
+        c.x += v.x; c.y += v.y; c.z += v.z; c.w += v.w;
+        *sp4 = make_uint4(0, 0, 0, 0);
+      }
+      *reinterpret_cast<uint4 *>(&mine[4 * tid]) = c;
+      const uint32_t a = smem_u32(&inbox[pass & 1][rank][4 * tid]);
+      for (uint32_t r = 0; r < C; ++r) st_dsmem_u32x4(cluster_map(a, r), c);
+    }
+    cluster_sync();   // every CTA's counts have landed in every inbox
+    if (tid < 64) {
       uint4 t = make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int r = 0; r < kClusterMax; ++r)
-        if (r < (int)C) { t.x += v[r].x; t.y += v[r].y; t.z += v[r].z; t.w += v[r].w; }
+      for (uint32_t r = 0; r < C; ++r) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(&inbox[pass & 1][r][4 * tid]);
+        t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+      }
       *reinterpret_cast<uint4 *>(&tot[4 * tid]) = t;
     }
     __syncthreads();
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     prefix |= digit << shift;
     mask |= 255u << shift;
     krem = s_krem;
-    if (pass < 3 && !compacted && pub[pass & 1][digit] <= (uint32_t)kCandMax) {
+    if (pass < 3 && !compacted && mine[digit] <= (uint32_t)kCandMax) {
       // compact this CTA's keys that match the new prefix
       for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
         const int i = b0 + tid;
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
         at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
         if (m) cand[at] = kk;
       }
-      nc = (int)pub[pass & 1][digit];
+      nc = (int)mine[digit];
       compacted = true;
     }
     __syncthreads();
@@ -288,16 +291,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   if (tid == 0) {
     int a = 0, b = 0;
     for (int w = 0; w < kTopkWarps; ++w) { a += w_gt[w]; b += w_eq[w]; }
-    pub_cnt[0] = a;
-    pub_cnt[1] = b;
+    const uint32_t at = smem_u32(&peer_cnt[rank][0]);
+    for (uint32_t r = 0; r < C; ++r) st_dsmem_u32x2(cluster_map(at, r), (uint32_t)a, (uint32_t)b);
   }
+  // every CTA's counts have landed; no CTA touches another's shared memory after this
   cluster_sync();
-  if (tid < (int)rank) {
-    peer_cnt[tid][0] = (int)dsmem_ld(&pub_cnt[0], tid);
-    peer_cnt[tid][1] = (int)dsmem_ld(&pub_cnt[1], tid);
-  }
-  cluster_arrive();   // this CTA reads no other CTA's shared memory past here
-  __syncthreads();
   if (tid == 0) {
     // winners of the lower-ranked CTAs, and ties among them
     int base = 0, eqb = 0;
@@ -336,7 +334,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
       out[i] = -1;
       if (kout) kout[i] = 0u;
     }
-  cluster_wait();     // keep this CTA's shared memory alive until the cluster has read it
 }
 
 struct TopkPlan {

@@ -54,6 +54,22 @@ struct CompressParams {
 int launch_compress_prefill(const CompressParams &p, cudaStream_t s);
 int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s);
 int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s);
+// Validate a compressor call and fill its parameters (no launch).
+int compress_params(const hca_compress_desc *d, int start_pos, int n, const void *Ca, const void *Cb,
+                    const void *Za, const void *Zb, long long row_stride, long long seq_stride, const float *Ba,
+                    const float *Bb, const float *gamma, void *out, float *out_scale, long long out_seq_stride,
+                    float *state_kv, float *state_score, CompressParams *p);
+// Window ring write of one decode token: row [B, c] -> ring[b, slot] of [B, w, c].
+struct IngestRing {
+  const void *row;
+  void *ring;
+  int w, c, slot;
+  hca_dtype dtype;
+};
+// One launch per decode token of a layer: main compressor (pa, may be NULL),
+// indexer compressor (pb, may be NULL) and the ring write (ring.ring may be NULL).
+int launch_decode_ingest(const CompressParams *pa, const CompressParams *pb, const IngestRing &ring, int B, int pos,
+                         cudaStream_t s);
 
 // ------------------------------------------------------------- index + top-k
 struct IndexParams {
@@ -125,6 +141,10 @@ int run_attend(const AttendParams &p, void *ws, size_t ws_bytes, cudaStream_t s)
 int launch_gemm(hca_dtype ab_dtype, const void *A, long long lda, const void *Bm, long long ldb,
                 void *C, long long ldc, hca_dtype c_dtype, int M, int N, int K, float alpha,
                 cudaStream_t s);
+// tcgen05 path of launch_gemm for bf16 A/B (M >= 128, N >= 256, K >= 64, 16-byte
+// aligned rows); HCA_ERR_UNSUPPORTED (nothing launched) otherwise.
+int launch_gemm_tc(const void *A, long long lda, const void *Bm, long long ldb, void *C, long long ldc,
+                   hca_dtype c_dtype, int M, int N, int K, float alpha, cudaStream_t s);
 // Row RMSNorm (optional) + partial RoPE (optional) + convert.  Row r of
 // `rows` rows of `cols` values; the RoPE position is (pos0 + r / rows_per_pos) % pos_mod.
 struct RowOpParams {

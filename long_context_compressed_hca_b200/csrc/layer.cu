@@ -45,12 +45,6 @@ __global__ void ring_fill_kernel(const T *kv, T *ring, int B, int n, int w, int 
   }
 }
 
-template <typename T>
-__global__ void ring_put_kernel(const T *row, T *ring, int w, int c, int slot) {
-  const int b = blockIdx.x;
-  for (int col = threadIdx.x; col < c; col += blockDim.x)
-    ring[((long long)b * w + slot) * c + col] = row[(long long)b * c + col];
-}
 
 struct Plan {
   // prefill buffers
@@ -293,38 +287,43 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const hca_dtype dt = a.dtype;
   const float theta = rope_theta(a), eps = eps_of(a);
-  // 1. window ring
-  if (a.w > 0) {
-    LaunchScope ls_("ring_put", s);
-    if (dt == HCA_F32) ring_put_kernel<float><<<a.B, 256, 0, s>>>((const float *)x->kv, (float *)cache->win, a.w, a.c, pos % a.w);
-    else ring_put_kernel<__nv_bfloat16><<<a.B, 256, 0, s>>>((const __nv_bfloat16 *)x->kv, (__nv_bfloat16 *)cache->win, a.w, a.c, pos % a.w);
-    if ((rc = ls_.done())) return rc;
-  }
-  // 2. compressor states (+ entry emission)
-  if (comp) {
-    hca_compress_desc cd{};
-    cd.B = a.B; cd.width = a.c; cd.m = a.m; cd.overlap = csa ? a.overlap : 0; cd.rd = a.rd;
-    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
-    cd.in_dtype = HCA_F32; cd.out_dtype = dt;
-    const int ncz = csa ? 4 : 2;
-    const float *cz = x->comp;
-    const bool ov = cd.overlap != 0;
-    rc = csa_compress(&cd, pos, 1, cz, ov ? cz + a.c : nullptr, cz + (csa ? 2 : 1) * a.c, ov ? cz + 3 * a.c : nullptr,
-                      (long long)ncz * a.c, (long long)ncz * a.c, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
-                      nullptr, cache->kv_comp, nullptr, cache->cap, cache->state_kv, cache->state_score, stream);
+  // 1. one launch: window ring write, compressor states (+ entry emission) of
+  //    the main and (CSA) indexer compressors
+  {
+    CompressParams pm{}, pi{};
+    if (comp) {
+      hca_compress_desc cd{};
+      cd.B = a.B; cd.width = a.c; cd.m = a.m; cd.overlap = csa ? a.overlap : 0; cd.rd = a.rd;
+      cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+      cd.in_dtype = HCA_F32; cd.out_dtype = dt;
+      const int ncz = csa ? 4 : 2;
+      const float *cz = x->comp;
+      const bool ov = cd.overlap != 0;
+      rc = compress_params(&cd, pos, 1, cz, ov ? cz + a.c : nullptr, cz + (csa ? 2 : 1) * a.c, ov ? cz + 3 * a.c : nullptr,
+                           (long long)ncz * a.c, (long long)ncz * a.c, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
+                           nullptr, cache->kv_comp, nullptr, cache->cap, cache->state_kv, cache->state_score, &pm);
+      if (rc) return rc;
+    }
+    if (csa) {
+      hca_compress_desc cd{};
+      cd.B = a.B; cd.width = a.c_I; cd.m = a.m; cd.overlap = a.overlap; cd.rd = a.rd_I;
+      cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
+      cd.in_dtype = HCA_F32; cd.out_dtype = a.idx_key_dtype;
+      const float *cz = x->compI;
+      const bool ov = a.overlap != 0;
+      rc = compress_params(&cd, pos, 1, cz, ov ? cz + a.c_I : nullptr, cz + 2 * a.c_I, ov ? cz + 3 * a.c_I : nullptr,
+                           4LL * a.c_I, 4LL * a.c_I, L->B_compI, ov ? L->B_compI + a.m * a.c_I : nullptr, nullptr,
+                           cache->key_I, cache->key_I_scale, cache->cap, cache->stateI_kv, cache->stateI_score, &pi);
+      if (rc) return rc;
+    }
+    IngestRing ring{};
+    if (a.w > 0) {
+      ring.row = x->kv; ring.ring = cache->win; ring.w = a.w; ring.c = a.c; ring.slot = pos % a.w; ring.dtype = dt;
+    }
+    rc = launch_decode_ingest(comp ? &pm : nullptr, csa ? &pi : nullptr, ring, a.B, pos, s);
     if (rc) return rc;
   }
   if (csa) {
-    hca_compress_desc cd{};
-    cd.B = a.B; cd.width = a.c_I; cd.m = a.m; cd.overlap = a.overlap; cd.rd = a.rd_I;
-    cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps; cd.rope_theta = theta;
-    cd.in_dtype = HCA_F32; cd.out_dtype = a.idx_key_dtype;
-    const float *cz = x->compI;
-    const bool ov = a.overlap != 0;
-    rc = csa_compress(&cd, pos, 1, cz, ov ? cz + a.c_I : nullptr, cz + 2 * a.c_I, ov ? cz + 3 * a.c_I : nullptr,
-                      4LL * a.c_I, 4LL * a.c_I, L->B_compI, ov ? L->B_compI + a.m * a.c_I : nullptr, nullptr,
-                      cache->key_I, cache->key_I_scale, cache->cap, cache->stateI_kv, cache->stateI_score, stream);
-    if (rc) return rc;
     char *w = static_cast<char *>(ws);
     int32_t *idx = reinterpret_cast<int32_t *>(w);
     const size_t ib = (((size_t)a.B * a.k * 4) + 255) & ~(size_t)255;
