@@ -57,36 +57,78 @@ __global__ void __launch_bounds__(256) gemm_simt(const Tab *A, long long lda, co
 }
 
 // ------------------------------------------------------------------ row op
+// One warp per row: optional RMS normalisation, gamma, scale, RoPE of the
+// last rd columns (interleaved pairs) and conversion.  cols % 4 == 0 rows
+// use 16-byte loads; a RoPE pair always sits inside one thread's 4 columns.
+constexpr int kRowWarps = 8;
+
 template <typename Tout>
-__global__ void row_op_kernel(RowOpParams p) {
-  extern __shared__ float red[];   // [blockDim / 32]
-  const int row = blockIdx.x;
-  const float *in = p.in + (long long)row * p.in_stride;
-  Tout *out = reinterpret_cast<Tout *>(p.out) + (long long)row * p.out_stride;
+__device__ __forceinline__ void store_cols4(Tout *dst, const float (&v)[4]);
+template <>
+__device__ __forceinline__ void store_cols4<float>(float *dst, const float (&v)[4]) {
+  *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void store_cols4<__nv_bfloat16>(__nv_bfloat16 *dst, const float (&v)[4]) {
+  *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+
+template <typename Tout, bool VEC>
+__global__ void __launch_bounds__(kRowWarps * 32) row_op_kernel(RowOpParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5);
+  if (row >= p.rows) return;
+  const float *in = p.in + row * p.in_stride;
+  Tout *out = reinterpret_cast<Tout *>(p.out) + row * p.out_stride;
   float r = p.scale;
   if (p.norm) {
     float ss = 0.f;
-    for (int c = threadIdx.x; c < p.cols; c += blockDim.x) ss += in[c] * in[c];
-    ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    float tot = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) tot += red[w];
-    r *= rsqrtf(tot / (float)p.cols + p.eps);
-  }
-  const long long pos = (p.pos0 + (long long)(row / p.rows_per_pos)) % p.pos_mod;
-  // each thread handles pairs of columns so that a RoPE pair stays in one thread
-  for (int c = 2 * threadIdx.x; c < p.cols; c += 2 * blockDim.x) {
-    float a = in[c] * r * (p.gamma ? p.gamma[c] : 1.f);
-    float b = in[c + 1] * r * (p.gamma ? p.gamma[c + 1] : 1.f);
-    if (p.rd > 0 && c >= p.cols - p.rd) {
-      float s, cs;
-      rope_sincos(pos, (c - (p.cols - p.rd)) / 2, p.rd, p.theta, &s, &cs);
-      const float a2 = a * cs - b * s, b2 = a * s + b * cs;
-      a = a2; b = b2;
+    if (VEC) {
+      for (int c = 4 * lane; c < p.cols; c += 128) {
+        const float4 v = *reinterpret_cast<const float4 *>(in + c);
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+    } else {
+      for (int c = lane; c < p.cols; c += 32) ss += in[c] * in[c];
     }
-    Elt<Tout>::store(out + c, a);
-    Elt<Tout>::store(out + c + 1, b);
+    ss = warp_sum(ss);
+    r *= rsqrtf(ss / (float)p.cols + p.eps);
+  }
+  const long long pos = (p.pos0 + row / p.rows_per_pos) % p.pos_mod;
+  const int c_rope = p.rd > 0 ? p.cols - p.rd : p.cols;
+  if (VEC) {
+    for (int c = 4 * lane; c < p.cols; c += 128) {
+      const float4 x = *reinterpret_cast<const float4 *>(in + c);
+      float v[4] = {x.x * r, x.y * r, x.z * r, x.w * r};
+      if (p.gamma) {
+        const float4 g = *reinterpret_cast<const float4 *>(p.gamma + c);
+        v[0] *= g.x; v[1] *= g.y; v[2] *= g.z; v[3] *= g.w;
+      }
+      if (c >= c_rope) {
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+          float s, cs;
+          rope_sincos(pos, (c + j - c_rope) / 2, p.rd, p.theta, &s, &cs);
+          const float a = v[j], b = v[j + 1];
+          v[j] = a * cs - b * s;
+          v[j + 1] = a * s + b * cs;
+        }
+      }
+      store_cols4<Tout>(out + c, v);
+    }
+  } else {
+    for (int c = 2 * lane; c < p.cols; c += 64) {
+      float a = in[c] * r * (p.gamma ? p.gamma[c] : 1.f);
+      float b = in[c + 1] * r * (p.gamma ? p.gamma[c + 1] : 1.f);
+      if (c >= c_rope) {
+        float s, cs;
+        rope_sincos(pos, (c - c_rope) / 2, p.rd, p.theta, &s, &cs);
+        const float a2 = a * cs - b * s, b2 = a * s + b * cs;
+        a = a2; b = b2;
+      }
+      Elt<Tout>::store(out + c, a);
+      Elt<Tout>::store(out + c + 1, b);
+    }
   }
 }
 
@@ -117,11 +159,18 @@ int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long
 
 int launch_row_op(const RowOpParams &p, cudaStream_t s) {
   if (p.rows == 0) return HCA_OK;
-  const int threads = p.cols >= 512 ? 256 : 128;
-  const size_t smem = (threads / 32) * sizeof(float);
+  const bool vec = p.cols % 4 == 0 && p.in_stride % 4 == 0 && p.out_stride % 4 == 0 &&
+                   (reinterpret_cast<uintptr_t>(p.in) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0 &&
+                   (!p.gamma || (reinterpret_cast<uintptr_t>(p.gamma) & 15) == 0);
+  const unsigned grid = (unsigned)((p.rows + kRowWarps - 1) / kRowWarps);
   LaunchScope ls_("row_op", s);
-  if (p.out_dtype == HCA_F32) row_op_kernel<float><<<p.rows, threads, smem, s>>>(p);
-  else row_op_kernel<__nv_bfloat16><<<p.rows, threads, smem, s>>>(p);
+  if (p.out_dtype == HCA_F32) {
+    if (vec) row_op_kernel<float, true><<<grid, kRowWarps * 32, 0, s>>>(p);
+    else row_op_kernel<float, false><<<grid, kRowWarps * 32, 0, s>>>(p);
+  } else {
+    if (vec) row_op_kernel<__nv_bfloat16, true><<<grid, kRowWarps * 32, 0, s>>>(p);
+    else row_op_kernel<__nv_bfloat16, false><<<grid, kRowWarps * 32, 0, s>>>(p);
+  }
   return ls_.done();
 }
 
