@@ -170,7 +170,9 @@ class DecodeBench:
                          compI=dev_normal((B, 4 * L.c_I), seed, s + 15))
             ti = TokenInputs(**x)
             o = torch.empty(B, L.n_h, L.c, dtype=torch.bfloat16, device="cuda")
-            ws = torch.empty(max(hb.decode_workspace_size(lh.struct, pos), 256), dtype=torch.uint8, device="cuda")
+            # sized for the 128 consecutive positions the step sweep visits
+            ws = torch.empty(max(hb.decode_workspace_size(lh.struct, pos + 128), 256), dtype=torch.uint8,
+                             device="cuda")
             self.layers.append(lh)
             self.caches.append(ch)
             self.inputs.append(ti)
@@ -180,9 +182,11 @@ class DecodeBench:
         self.host_in = [{k: v.cpu().pin_memory() for k, v in ti.t.items() if v is not None} for ti in self.inputs]
         self.host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
 
-    def step(self):
+    def step(self, pos=None):
         """CSA layer on the current stream, HCA layer on a side stream (the two
-        layers of the step are independent), joined before returning."""
+        layers of the step are independent), joined before returning.  `pos`
+        overrides the workload's token position."""
+        pos = self.wl.pos if pos is None else pos
         cur = torch.cuda.current_stream()
         if not hasattr(self, "side"):
             self.side = torch.cuda.Stream()
@@ -192,7 +196,7 @@ class DecodeBench:
         for i, (lh, ch, ti, o, ws) in enumerate(zip(self.layers, self.caches, self.inputs, self.outs, self.ws)):
             st = cur if i == 0 else self.side
             with torch.cuda.stream(st):
-                hb.hybrid_decode_step(lh.struct, ti.struct, ch.struct, self.wl.pos, o, ws)
+                hb.hybrid_decode_step(lh.struct, ti.struct, ch.struct, pos, o, ws)
         self.join.record(self.side)
         cur.wait_event(self.join)
 
@@ -221,10 +225,13 @@ class DecodeBench:
             if L.kind == "csa":
                 kb = 1 if wl.idx_key_dtype == "fp8" else 2
                 per["index_scores"] = B * V * (L.c_I * kb + (4 if kb == 1 else 0)) + B * L.n_hI * (L.c_I * 2 + 4)
+                per["topk"] = B * V * 4 + B * L.k * 4          # scores in, indices out
                 per["attend_csa"] = B * (min(L.k, V) + nw) * L.c * 2 + qo
             else:
                 per["attend_hca"] = B * (V + nw) * L.c * 2 + qo
-        return sum(per.values()), per
+        # the step's total counts the method's own streams (keys, rows, q/o), not the scores
+        # the selection reads back
+        return sum(v for k, v in per.items() if k != "topk"), per
 
 
 def capture_graph(fn, stream):
@@ -239,7 +246,31 @@ def capture_graph(fn, stream):
     return g
 
 
-def run_decode(wl, K, W, flush, stream, e2e=True):
+def time_step_sweep(b, K, W, flush, stream):
+    """The emitting step (both compressors close a block: pos+1 a multiple of
+    128) and the mean over 128 consecutive steps pos..pos+127 (32 CSA entries
+    and one HCA entry emitted), each step its own captured graph."""
+    wl = b.wl
+    pe = ((wl.pos + 1 + 127) // 128) * 128 - 1
+    ge = capture_graph(lambda: b.step(pe), stream)
+    for _ in range(W):
+        ge.replay()
+    ems, _, _ = time_steps(ge.replay, K, flush, stream)
+    graphs = [capture_graph(lambda p=p: b.step(p), stream) for p in range(wl.pos, wl.pos + 128)]
+
+    def seq():
+        for g in graphs:
+            g.replay()
+    seq()
+    torch.cuda.synchronize()
+    reps = max(2, min(K, 5))
+    sms, _, _ = time_steps(seq, reps, flush, stream)
+    del graphs, ge
+    return dict(emit_pos=pe, emit_us=round(statistics.mean(ems) * 1e3, 2),
+                mean_128_us=round(statistics.mean(sms) / 128 * 1e3, 2), mean_128_reps=reps)
+
+
+def run_decode(wl, K, W, flush, stream, e2e=True, sweep=False):
     b = DecodeBench(wl)
     for _ in range(W):
         b.step()
@@ -282,6 +313,8 @@ def run_decode(wl, K, W, flush, stream, e2e=True):
         ems, _, _ = time_steps(e2e_step, K, flush, stream)
         res["e2e_ms"] = ems
     del graph
+    if sweep:
+        res["sweep"] = time_step_sweep(b, K, W, flush, stream)
     return res
 
 
@@ -452,7 +485,7 @@ def main():
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     clocks = ClockSampler(local if world > 1 else torch.cuda.current_device())
     clocks.start()
-    head = run_decode(wl, args.steps, args.warmup, flush, stream)
+    head = run_decode(wl, args.steps, args.warmup, flush, stream, sweep=not args.only_headline)
     clk = clocks.stop()
     step_ms = statistics.mean(head["ms"])
     step_ms_max = dist_max(step_ms)
@@ -477,6 +510,8 @@ def main():
     hi, ho = head["bench"].e2e_bytes()
 
     extras = {}
+    if "sweep" in head:
+        extras["decode_steps"] = dict(steady_us=round(step_ms * 1e3, 2), steady_pos=wl.pos, **head["sweep"])
     if rank == 0 and world == 1:
         # CPU oracle baseline on a bounded sample of the same workload
         n = args.oracle_seqs
@@ -499,7 +534,8 @@ def main():
         del d1
         torch.cuda.empty_cache()
         # prefill workloads (fewer steps: each is a whole layer)
-        for key, pwl in (("prefill_64k", workloads.CSA_PREFILL), ("hca_prefill", workloads.HCA_PREFILL)):
+        for key, pwl in (("prefill_64k", workloads.CSA_PREFILL), ("prefill_128k", workloads.CSA_PREFILL_128K),
+                         ("hca_prefill", workloads.HCA_PREFILL)):
             kp = max(3, min(args.steps, 5))
             r = run_prefill(pwl, kp, 3, flush, stream)
             att_ms, _ = kern_ms(r["kern"], "attend", kp)

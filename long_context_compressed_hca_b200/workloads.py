@@ -74,6 +74,13 @@ CSA_PREFILL = Workload(
     layers=(LayerShape("csa", m=4, n_h=64, c=512, rd=64, w=128, k=512, n_hI=8, c_I=64),),
 )
 
+# The same CSA layer prefilled over 128K tokens.
+CSA_PREFILL_128K = Workload(
+    name="csa_prefill_bf16_b1_s131072", seed=2, dtype="bf16", B=1, mode="prefill",
+    n=131072, d=4096, d_c=1024,
+    layers=(LayerShape("csa", m=4, n_h=64, c=512, rd=64, w=128, k=512, n_hI=8, c_I=64),),
+)
+
 # Hybrid decode at 128K: one CSA layer then one HCA layer per step.
 HYBRID_DECODE_128K = Workload(
     name="hybrid_decode_bf16_b32_ctx131072", seed=3, dtype="bf16", B=32, mode="decode",
