@@ -256,6 +256,13 @@ const char *hca_last_error(void);   /* text of the last failing call (thread-loc
  * kernels set when a bounded wait expires.  *device_status = HCA_OK or
  * HCA_ERR_TIMEOUT.  Returns HCA_ERR_CUDA if the synchronisation failed. */
 int hca_check_status(hca_stream_t stream, int *device_status);
+/* Failure-detection self-test (no counterpart in the papers): launches one
+ * block whose single mbarrier wait can never complete.  The wait gives up
+ * after limit_ns (1 ms .. 2 s), sets the status word to HCA_ERR_TIMEOUT and
+ * the kernel returns, exactly as an expired wait in the production kernels
+ * does; the CUDA context stays usable.  Returns HCA_ERR_INVALID for a limit
+ * out of range, else the launch status. */
+int hca_selftest_wait(unsigned long long limit_ns, hca_stream_t stream);
 int hca_version(void);              /* (major << 16) | minor */
 /* Kernels launched by the library since load (per process), for accounting. */
 long long hca_launch_count(void);

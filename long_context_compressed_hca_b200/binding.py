@@ -72,6 +72,7 @@ def _declare(L):
         "hca_version": (I, []),
         "hca_launch_count": (LL, []),
         "hca_check_status": (I, [VP, C.POINTER(C.c_int)]),
+        "hca_selftest_wait": (I, [C.c_ulonglong, VP]),
         "hca_profile_enable": (I, [I]),
         "hca_profile_sample": (I, []),
         "hca_profile_collect": (I, [C.c_char_p, SZ]),
@@ -147,6 +148,11 @@ def device_status(stream=None) -> int:
     v = C.c_int(0)
     check(lib().hca_check_status(stream_handle(stream), C.byref(v)))
     return v.value
+
+
+def selftest_wait(limit_ns: int, stream=None):
+    """Launch the bounded-wait self-test kernel (its wait always expires)."""
+    return check(lib().hca_selftest_wait(limit_ns, stream_handle(stream)))
 
 
 def launch_count() -> int:

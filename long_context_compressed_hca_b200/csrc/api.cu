@@ -239,6 +239,25 @@ int compress_params(const hca_compress_desc *d, int start_pos, int n, const void
   return HCA_OK;
 }
 
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// ever arrives on; the wait gives up after limit_ns, sets the status word to
+// HCA_ERR_TIMEOUT and the kernel returns like any expired production wait.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, int *status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  mbar_fence_init();
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(b, 0)) return;   // cannot happen: nothing arrives
+    if ((it & 255u) == 0 && global_ns() - t0 > limit_ns) {
+      set_timeout_status(status);
+      return;
+    }
+  }
+}
+
 }  // namespace hca
 
 using namespace hca;
@@ -290,6 +309,14 @@ int hca_profile_collect(char *buf, size_t len) {
   }
   g_pend.clear();
   return HCA_OK;
+}
+
+int hca_selftest_wait(unsigned long long limit_ns, hca_stream_t stream) {
+  REQUIRE(limit_ns >= 1000000ull && limit_ns <= kWaitLimitNs, "limit_ns must be within [1 ms, 2 s]");
+  int *status = device_status_ptr();
+  REQUIRE(status != nullptr, "no device status word");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return HCA_LAUNCH("selftest_wait", s, selftest_wait_kernel<<<1, 32, 0, s>>>(limit_ns, status));
 }
 
 int hca_check_status(hca_stream_t stream, int *device_status) {

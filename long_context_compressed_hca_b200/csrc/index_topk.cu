@@ -77,44 +77,33 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
 // ------------------------------------------------------------------ top-k
 // One thread-block cluster of C CTAs (C <= 8) selects the top-k of one row
 // segment; CTA r of the cluster holds keys [r*slice, (r+1)*slice) of the
-// segment in shared memory.  Each radix pass (8 bits, top byte first) builds
-// a CTA-local 256-bin histogram that every CTA stores into every peer's
-// inbox (distributed shared memory, stores only), so that after one cluster
-// barrier every CTA sums the same C histograms and derives the same digit.  Once a CTA's keys that still match the threshold prefix fit
-// in kCandMax they are compacted and later passes scan only those.  The final
-// stable compaction offsets each CTA's output by the winners of the lower-
-// ranked CTAs, so the selection leaves in ascending index order with ties
-// resolved towards the lower index.  Rows longer than one segment are cut
-// into segments whose winners (order key + index) a second launch merges.
+// segment in shared memory.  The radix select takes three digits of the
+// order key: bits 31..21 (2048 bins), 20..10 (2048 bins) and 9..0.  The wide
+// first digit already separates scores of one binade, so after it only the
+// keys of the threshold's bin (compacted into kCandMax slots when they fit)
+// take part in the later passes.  With C > 1 every CTA adds its non-empty
+// bins into every CTA's copy of the cluster histogram with distributed-
+// shared-memory atomics (double-buffered by pass parity), so that after one
+// cluster barrier each CTA derives the same digit on its own.  The final stable compaction offsets each CTA's output by the
+// winners of the lower-ranked CTAs, so the selection leaves in ascending
+// index order with ties resolved towards the lower index.  Rows longer than
+// one segment are cut into segments whose winners (order key + index) a
+// second launch merges.
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kSliceMax = 16384;   // keys per CTA (64 KB of shared memory)
-constexpr int kCandMax = 4096;     // compacted keys per CTA (16 KB)
+constexpr int kCandMax = 2048;     // compacted keys per CTA (8 KB)
 constexpr int kClusterMax = 8;     // portable cluster size
+constexpr int kBinsMax = 2048;
+constexpr uint32_t kNoBin = 0xFFFFFFFFu;
+// digit p covers bits [shift, shift + width)
+__device__ __forceinline__ int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
+__device__ __forceinline__ int digit_width(int pass) { return pass == 2 ? 10 : 11; }
 
 __device__ __forceinline__ uint32_t order_bits(uint32_t u) {
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                 // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 1 for every non-NaN float
 }
-// Add one key to a shared histogram (bin 256 = no key).  The lanes that
-// share the first pending lane's bin are folded into one atomic, twice, which
-// keeps clustered scores (one dominant bin) from serialising the warp.
-__device__ __forceinline__ void hist_add(uint32_t *h, uint32_t bin) {
-  const int lane = threadIdx.x & 31;
-  unsigned active = __ballot_sync(0xffffffffu, bin != 256u);
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    if (!active) return;
-    const int leader = __ffs(active) - 1;
-    const uint32_t lb = __shfl_sync(0xffffffffu, bin, leader);
-    const unsigned same = __ballot_sync(0xffffffffu, bin == lb) & active;
-    if (lane == leader) atomicAdd(&h[lb], (uint32_t)__popc(same));
-    if (same & (1u << lane)) bin = 256u;
-    active &= ~same;
-  }
-  if (active & (1u << lane)) atomicAdd(&h[bin], 1u);
-}
-
 // Copy len 32-bit words to shared memory, as order keys (KEYS: already keys).
 template <bool KEYS>
 __device__ __forceinline__ void load_keys(uint32_t *dst, const uint32_t *src, int len) {
@@ -149,21 +138,66 @@ __device__ __forceinline__ void load_keys(uint32_t *dst, const uint32_t *src, in
   }
 }
 
+// Over the histogram h[0..nb) taken from the top bin down: the bin in which
+// the krem-th largest key falls, krem within that bin, and the histogram's
+// total.  All threads call; results land in out[0..2] (digit, krem, total).
+__device__ void find_digit(const uint32_t *h, int nb, int krem, int *warp_tot, int *out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (nb + kTopkThreads - 1) / kTopkThreads;
+  const int hi = nb - 1 - tid * per;                       // this thread's bins: hi, hi-1, ..., > hi-per
+  int sum = 0;
+  for (int j = 0; j < per; ++j)
+    if (hi - j >= 0) sum += (int)h[hi - j];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = lane < kTopkWarps ? warp_tot[lane] : 0;
+    int u = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, u, o);
+      if (lane >= o) u += y;
+    }
+    if (lane < kTopkWarps) warp_tot[lane] = u - t;          // exclusive warp offsets
+    if (lane == kTopkWarps - 1) out[2] = u;                  // total
+  }
+  __syncthreads();
+  int above = warp_tot[warp] + incl - sum;                   // keys in higher bins than this thread's
+  if (above < krem && above + sum >= krem) {
+    for (int j = 0; j < per; ++j) {
+      const int b = hi - j;
+      if (b < 0) break;
+      const int c = (int)h[b];
+      if (above + c >= krem) {
+        out[0] = b;
+        out[1] = krem - above;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
 // Grid: x = C * rows * n_seg, cluster (C,1,1).  Dynamic shared memory:
 // (slice + kCandMax) words.
 __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   extern __shared__ __align__(16) uint32_t dyn[];
   uint32_t *keys = dyn;               // [slice]
   uint32_t *cand = dyn + p.slice;     // [kCandMax]
-  __shared__ __align__(16) uint32_t sub[4][256];    // this CTA's histogram, 4 copies
-  __shared__ __align__(16) uint32_t mine[256];      // this CTA's histogram of the current pass
-  // every CTA's histogram of pass (parity), written by that CTA into each peer
-  __shared__ __align__(16) uint32_t inbox[2][kClusterMax][256];
-  __shared__ __align__(16) uint32_t tot[256];
+  __shared__ __align__(16) uint32_t hist[kBinsMax];       // this CTA's histogram
+  __shared__ __align__(16) uint32_t total[2][kBinsMax];   // the cluster's histogram, by pass parity
+  __shared__ int warp_tot[32];
+  __shared__ __align__(16) int res[4];                 // digit, krem, total of the current pass
   __shared__ __align__(8) int peer_cnt[kClusterMax][2];   // every CTA's keys above / equal to the threshold
   __shared__ int w_gt[kTopkWarps], w_eq[kTopkWarps];
-  __shared__ int s_total, s_krem, s_nc, s_base, s_eqb;
-  __shared__ uint32_t s_digit;
+  __shared__ int s_nc, s_base, s_eqb;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
@@ -177,87 +211,64 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
 
   if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
   else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
+  for (int i = tid; i < kBinsMax; i += kTopkThreads) {
+    hist[i] = 0;
+    total[0][i] = 0;
+    total[1][i] = 0;
+  }
   if (tid == 0) s_nc = 0;
-  for (int i = tid; i < 4 * 256; i += kTopkThreads) (&sub[0][0])[i] = 0;
-  __syncthreads();
+  if (C > 1) cluster_sync();   // every CTA's totals are clear before anyone adds into them
+  else __syncthreads();
 
   uint32_t prefix = 0, mask = 0, T = 0;
   int krem = p.k, K = 0;
   bool compacted = false;
   int nc = 0;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = digit_shift(pass), nb = 1 << digit_width(pass);
     const uint32_t *arr = compacted ? cand : keys;
     const int n = compacted ? nc : len;
     for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
       const int i = b0 + tid;
-      uint32_t bin = 256u;
+      uint32_t bin = kNoBin;
       if (i < n) {
         const uint32_t kk = arr[i];
-        if (kk != 0 && (kk & mask) == prefix) bin = (kk >> shift) & 255u;
+        if (kk != 0 && (kk & mask) == prefix) bin = (kk >> shift) & (uint32_t)(nb - 1);
       }
-      hist_add(sub[warp & 3], bin);
+      if (bin != kNoBin) atomicAdd(&hist[bin], 1u);
     }
     __syncthreads();
-    if (tid < 64) {
-      // 4 bins per thread: sum (and clear) the 4 copies, then store the counts
-      // into every CTA's inbox slot for this rank
-      uint4 c = make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint4 *sp4 = reinterpret_cast<uint4 *>(&sub[w][4 * tid]);
-        const uint4 v = *sp4;
-        c.x += v.x; c.y += v.y; c.z += v.z; c.w += v.w;
-        *sp4 = make_uint4(0, 0, 0, 0);
+    if (C > 1) {
+      // add this CTA's non-empty bins into every CTA's total of this pass; a
+      // total is cleared two passes before it is reused, with a cluster
+      // barrier in between
+      uint32_t *tp = total[pass & 1];
+      const uint32_t t0 = smem_u32(tp);
+      for (int b = tid; b < nb; b += kTopkThreads) {
+        const uint32_t c = hist[b];
+        if (c)
+          for (uint32_t r = 0; r < C; ++r)
+            asm volatile("red.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_map(t0 + 4u * b, r)), "r"(c)
+                         : "memory");
       }
-      *reinterpret_cast<uint4 *>(&mine[4 * tid]) = c;
-      const uint32_t a = smem_u32(&inbox[pass & 1][rank][4 * tid]);
-      for (uint32_t r = 0; r < C; ++r) st_dsmem_u32x4(cluster_map(a, r), c);
+      cluster_sync();
+      find_digit(tp, nb, krem, warp_tot, res);
+      for (int b = tid; b < nb; b += kTopkThreads) tp[b] = 0;
+    } else {
+      find_digit(hist, nb, krem, warp_tot, res);
     }
-    cluster_sync();   // every CTA's counts have landed in every inbox
-    if (tid < 64) {
-      uint4 t = make_uint4(0, 0, 0, 0);
-      for (uint32_t r = 0; r < C; ++r) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(&inbox[pass & 1][r][4 * tid]);
-        t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
-      }
-      *reinterpret_cast<uint4 *>(&tot[4 * tid]) = t;
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l covers bins 255-8l .. 248-8l (descending); suffix sums from the top
-      uint32_t loc[8], run = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { run += tot[255 - 8 * lane - j]; loc[j] = run; }
-      uint32_t incl = run;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const uint32_t before = incl - run;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t above = before + (j ? loc[j - 1] : 0u), upto = before + loc[j];
-        if (above < (uint32_t)krem && upto >= (uint32_t)krem) {
-          s_digit = 255 - 8 * lane - j;
-          s_krem = krem - (int)above;
-        }
-      }
-      if (lane == 31) s_total = (int)incl;
-    }
-    __syncthreads();
     if (pass == 0) {
-      const int nvalid = s_total;   // the whole segment's keys (absent keys are 0)
+      const int nvalid = res[2];   // the whole segment's keys (absent keys are 0)
       if (nvalid <= p.k) { K = nvalid; krem = 0; break; }   // every key is selected, T = 0
       if (p.k <= 0) { K = 0; krem = 0; prefix = 0xFFFFFFFFu; break; }   // none is selected
       K = p.k;
     }
-    const uint32_t digit = s_digit;
+    const uint32_t digit = (uint32_t)res[0];
     prefix |= digit << shift;
-    mask |= 255u << shift;
-    krem = s_krem;
-    if (pass < 3 && !compacted && mine[digit] <= (uint32_t)kCandMax) {
+    mask |= (uint32_t)(nb - 1) << shift;
+    krem = res[1];
+    const uint32_t local_in_bin = hist[digit];
+    if (pass < 2 && !compacted && local_in_bin <= (uint32_t)kCandMax) {
       // compact this CTA's keys that match the new prefix
       for (int b0 = 0; b0 < n; b0 += kTopkThreads) {
         const int i = b0 + tid;
@@ -269,9 +280,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
         at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
         if (m) cand[at] = kk;
       }
-      nc = (int)mine[digit];
+      nc = (int)local_in_bin;
       compacted = true;
     }
+    __syncthreads();   // every thread has read hist[digit]
+    for (int b = tid; b < nb; b += kTopkThreads) hist[b] = 0;
     __syncthreads();
   }
   if (K == p.k) T = prefix;
@@ -295,7 +308,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     for (uint32_t r = 0; r < C; ++r) st_dsmem_u32x2(cluster_map(at, r), (uint32_t)a, (uint32_t)b);
   }
   // every CTA's counts have landed; no CTA touches another's shared memory after this
-  cluster_sync();
+  if (C > 1) cluster_sync();
+  else __syncthreads();
   if (tid == 0) {
     // winners of the lower-ranked CTAs, and ties among them
     int base = 0, eqb = 0;
