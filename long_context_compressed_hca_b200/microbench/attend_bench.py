@@ -148,7 +148,7 @@ def main():
     flops = keys * n_h * c * 4
     print(f"attend {kind} n_q={n_q} c={c}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s")
     hb.trace_attend(1)
-    run(False)
+    run()
     tr = hb.trace_attend_read()
     hb.trace_attend(0)
     tot = tr["total"]   # summed over the three reporting roles
