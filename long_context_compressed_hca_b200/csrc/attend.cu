@@ -291,7 +291,11 @@ struct Layout {
 enum TraceSlot {
   TR_P_QEMPTY, TR_P_KVEMPTY, TR_M_QFULL, TR_M_KVFULL, TR_M_SEMPTY, TR_M_PFULL, TR_M_OEMPTY,
   TR_S_SFULL, TR_S_PBUF, TR_S_RESCALE, TR_S_EPI_WAIT, TR_S_TILE, TR_S_EPI, TR_TOTAL, TR_RESCALES, TR_UNITS,
-  TR_TILES, TR_P_ISSUE, TR_S_MERGE_READY, TR_S_MERGE_FULL, TR_S_PUSH, TR_S_WEIGHTS, TR_S_MERGE_LOOP, TR_COUNT
+  TR_TILES, TR_P_ISSUE, TR_S_MERGE_READY, TR_S_MERGE_FULL, TR_S_PUSH, TR_S_WEIGHTS, TR_S_MERGE_LOOP,
+  // timeline of each CTA's first unit (ns, summed over CTAs): setup, until the
+  // first S, the tiles, the epilogue/merge, until exit; then the earliest
+  // entry (stored inverted) and the latest exit over all CTAs, and the CTA count
+  TR_T_SETUP, TR_T_FIRST_S, TR_T_TILES, TR_T_EPI, TR_T_EXIT, TR_T_ENTRY_INV, TR_T_EXIT_MAX, TR_T_CTAS, TR_COUNT
 };
 __device__ unsigned long long g_attn_trace[32];
 
@@ -498,6 +502,8 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
   unsigned long long tr[TR_COUNT];
   if (TRACE) for (int i = 0; i < TR_COUNT; ++i) tr[i] = 0;
   const long long t_start = TRACE ? clock64() : 0;
+  unsigned long long ts[6] = {0, 0, 0, 0, 0, 0};   // timeline stamps (thread 0, first unit)
+  if (TRACE && threadIdx.x == 0) ts[0] = global_ns();
   // wait on an mbarrier, adding the cycles spent to trace slot `slot`
   auto twait = [&](uint32_t b, uint32_t par, int slot) -> bool {
     if (!TRACE) return mbar_wait(b, par, p.status);
@@ -545,6 +551,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
     if (threadIdx.x == 0) mbar_arrive_expect_tx(bar(bars->mg_full), (p.nsplit - 1) * merge_blk(C, p.nsplit));
     cluster_sync();
   }
+  if (TRACE && threadIdx.x == 0) ts[1] = global_ns();
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ loads
@@ -736,6 +743,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         const int st = gj & 1;
         const uint32_t ph = (gj >> 1) & 1;
         if (!twait(bar(bars->s_full[st]), ph, TR_S_SFULL)) return;
+        if (TRACE && threadIdx.x == 0 && j == 0 && ts[2] == 0) ts[2] = global_ns();
         tc_fence_after();
         uint32_t sv[32];
         tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
@@ -818,6 +826,10 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         const uint32_t gl = g + nt - 1;
         if (!twait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, TR_S_EPI_WAIT)) return;
       }
+      if (TRACE && threadIdx.x == 0 && ts[3] == 0) {
+        ts[3] = global_ns();
+        if (ts[2] == 0) ts[2] = ts[3];
+      }
       const long long te0 = TRACE ? clock64() : 0;
       tc_fence_after();
       const float ltot = l + __shfl_xor_sync(0xffffffffu, l, 16);
@@ -834,6 +846,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
                               TRACE ? &tr[TR_S_MERGE_READY] : nullptr))
           return;
         if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+        if (TRACE && threadIdx.x == 0 && ts[4] == 0) ts[4] = global_ns();
         g += nt;
         ++iq;
         continue;
@@ -861,6 +874,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->o_empty));
         if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+        if (TRACE && threadIdx.x == 0 && ts[4] == 0) ts[4] = global_ns();
         g += nt;
         ++iq;
         continue;
@@ -903,6 +917,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bars->o_empty));
       if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+      if (TRACE && threadIdx.x == 0 && ts[4] == 0) ts[4] = global_ns();
       g += nt;
       ++iq;
     }
@@ -919,6 +934,17 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (TRACE && threadIdx.x == 0 && ts[4] != 0) {
+    ts[5] = global_ns();
+    atomicAdd(&g_attn_trace[TR_T_SETUP], ts[1] - ts[0]);
+    atomicAdd(&g_attn_trace[TR_T_FIRST_S], ts[2] - ts[1]);
+    atomicAdd(&g_attn_trace[TR_T_TILES], ts[3] - ts[2]);
+    atomicAdd(&g_attn_trace[TR_T_EPI], ts[4] - ts[3]);
+    atomicAdd(&g_attn_trace[TR_T_EXIT], ts[5] - ts[4]);
+    atomicMax(&g_attn_trace[TR_T_ENTRY_INV], ~ts[0]);
+    atomicMax(&g_attn_trace[TR_T_EXIT_MAX], ts[5]);
+    atomicAdd(&g_attn_trace[TR_T_CTAS], 1ull);
+  }
   if (warp == kMmaWarp) tmem_dealloc(tmem, L::tmem_cols);
 }
 

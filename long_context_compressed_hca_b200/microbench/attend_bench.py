@@ -95,8 +95,14 @@ def decode_main():
     tr = hb.trace_attend_read()
     hb.trace_attend(0)
     tot = tr["total"]
+    tl = {kk for kk in tr if kk.startswith("t_")}
     print({kk: (round(3 * v / tot, 3) if kk not in ("rescales", "units", "tiles", "total") else v)
-           for kk, v in tr.items()})
+           for kk, v in tr.items() if kk not in tl})
+    n = max(tr["t_ctas"], 1)
+    span = (tr["t_exit_max"] - ((~tr["t_entry_inv"]) & (2 ** 64 - 1))) / 1e3
+    print("per-CTA timeline (us):", {kk[2:]: round(tr[kk] / n / 1e3, 2)
+                                      for kk in ("t_setup", "t_first_s", "t_tiles", "t_epilogue", "t_exit")},
+          f"first entry -> last exit {span:.2f} us over {tr['t_ctas']} CTAs")
     print("device status", hb.device_status())
 
 
