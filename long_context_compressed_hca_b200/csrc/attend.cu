@@ -276,15 +276,19 @@ struct Bars {
 template <int C>
 struct Layout {
   static constexpr int NKB = C / 64;
-  // key-tile stages: as many 64-key tiles as fit beside Q and the P buffers
-  static constexpr int NS = (C == 512) ? 2 : (C == 256 ? 5 : 8);
-  static constexpr uint32_t q_off = 0;
-  static constexpr uint32_t kv_off = NKB * kTileBytes;
+  // key-tile stages: Q lives in tensor memory, so the stages take what the P
+  // buffers leave (192 KB for C = 512 and 256)
+  static constexpr int NS = (C == 512) ? 3 : (C == 256 ? 6 : 8);
+  static constexpr uint32_t kv_off = 0;
   static constexpr uint32_t p_off = kv_off + NS * NKB * kTileBytes;
   static constexpr uint32_t bar_off = p_off + 2 * kTileBytes;
   static constexpr uint32_t misc_off = bar_off + 512;
   static constexpr uint32_t bytes = misc_off + 2048 + 1024;  // + alignment slack
-  static constexpr uint32_t tmem_cols = C <= 128 ? 128 : (C <= 256 ? 256 : 512);
+  // tensor memory: O in lane-half 0, columns [0, C); in lane-half 1 the S
+  // double buffer at columns [0, 128) and Q (bf16, two per column) at
+  // [q_col, q_col + C/2), the lanes of S as the A operand of S = Q K^T needs
+  static constexpr uint32_t tmem_cols = 512;
+  static constexpr uint32_t q_col = 2 * KT;
 };
 
 // Trace counters (cycles, summed over CTAs) of the tensor-core kernel's waits.
@@ -486,8 +490,7 @@ __device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *sm
 
 template <int C, bool TRACE>
 __global__ void __launch_bounds__(kThreads, 1)
-attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
-          const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmW) {
+attend_tc(AttendParams p, int n_units) {
   using L = Layout<C>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -514,7 +517,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(bars->q_full), 1);
+    mbar_init(bar(bars->q_full), kSoftmaxWarps);
     mbar_init(bar(bars->q_empty), 1);
     mbar_init(bar(bars->o_empty), kSoftmaxWarps);
     mbar_init(bar(bars->mma_done), 1);
@@ -569,8 +572,7 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
     const int chunk = pt % CPR, prow = pt / CPR;
     const uint32_t kb_off = (chunk / 8) * kTileBytes;
     const int cc = chunk % 8;
-    if (pt == 0) tma_prefetch_desc(&tmQ);
-    uint32_t g = 0, iq = 0;
+    uint32_t g = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const int bq = u / p.nsplit, sp = u % p.nsplit;
       const int b = bq / p.n_q, qi = bq % p.n_q;
@@ -578,12 +580,6 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
       if (nt == 0) continue;
-      if (pt == 0) {
-        if (!twait(bar(bars->q_empty), (iq & 1) ^ 1, TR_P_QEMPTY)) return;
-        mbar_arrive_expect_tx(bar(bars->q_full), NKB * kTileBytes);
-        for (int kb = 0; kb < NKB; ++kb)
-          tma_load_2d(sbase + L::q_off + kb * kTileBytes, &tmQ, kb * 64, (b * p.n_q + qi) * p.n_h, bar(bars->q_full));
-      }
       // masked slots read a real row of a real tensor (cap is 0 when kv_comp is absent)
       const __nv_bfloat16 *cbase = reinterpret_cast<const __nv_bfloat16 *>(
           p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q));
@@ -604,7 +600,6 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         for (int i = 0; i < NR; ++i) cp_async16(tile + sw128_off(prow + i * RPP, cc), src[i], 16);
         cp_async_arrive_noinc(bar(bars->kv_full[st]));
       }
-      ++iq;
     }
     }();
     cp_async_wait_all();
@@ -616,11 +611,11 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       const KeySet ks = key_set_tc(p, qi);
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
+      // the unit's last P.V has landed once the MMA warp's final commit has
+      // (a parity wait on pv_done is only meaningful one phase ahead of the
+      // last phase this thread has seen, and this thread has seen none)
       bool ok = true;
-      if (nt > 0) {
-        const uint32_t gl = nt - 1;
-        ok = mbar_wait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, p.status);
-      }
+      if (nt > 0) ok = mbar_wait(bar(bars->mma_done), 0, p.status);
       if (ok) {
         // the softmax warps' (max, sum) writes and RoPE table are ordered by the merge barrier
         cluster_merge<C>(p, smem, bars, tmem, nt, sp, b, qi, rope_all, nullptr);
@@ -678,13 +673,13 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
           }
           fence_proxy_async();
           tc_fence_after();
-          // descriptors advance by constant offsets (16-byte units in the low field)
-          const uint64_t qd = sdesc_sw128(sbase + L::q_off, 16, 1024);
+          // K descriptor advances by constant offsets (16-byte units in the low
+          // field); Q (A operand, tensor memory) by 8 columns = 16 bf16 per step
           const uint64_t kd = sdesc_sw128(sbase + L::kv_off + kst * L::NKB * kTileBytes, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint64_t off = ((kk / 4) * kTileBytes + (kk % 4) * 32) >> 4;
-            umma_bf16(tS + st * KT, qd + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            umma_bf16_ts(tS + st * KT, tS + L::q_col + 8 * kk, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar(bars->s_full[st]));
           if (j == nt - 1) umma_commit(bar(bars->q_empty));
@@ -708,6 +703,51 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
     const float zs = p.scale * kLog2e;
     const uint32_t lane_S = (uint32_t)(q4 * 32 + 16) << 16;
     const uint32_t lane_O = (uint32_t)(q4 * 32) << 16;
+    // Q of a unit into tensor memory (lane-half 1, columns q_col..): thread
+    // (hl, half) stores head row r, bf16 dims [half*C/2, (half+1)*C/2), read
+    // from global in rounds of 16 words with the next round's loads in flight
+    uint32_t nq = 0;                      // Q writes so far (q_empty parity)
+    auto write_q = [&](int uq) -> bool {
+      if (nq > 0 && !twait(bar(bars->q_empty), (nq - 1) & 1, TR_P_QEMPTY)) return false;
+      tc_fence_after();
+      const int bqq = uq / p.nsplit;
+      const bool live = r < p.n_h;
+      const uint4 *src = reinterpret_cast<const uint4 *>(
+          reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((long long)bqq * p.n_h + (live ? r : 0)) * C + half * (C / 2));
+      const uint32_t tq = tmem + lane_S + L::q_col;
+      constexpr int ROUNDS = C / 64;      // 16 words (4 x 16 B) per round
+      uint4 cur[4], nxt[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) cur[x] = live ? __ldg(src + x) : make_uint4(0, 0, 0, 0);
+#pragma unroll 1
+      for (int rd = 0; rd < ROUNDS; ++rd) {
+        if (rd + 1 < ROUNDS) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) nxt[x] = live ? __ldg(src + 4 * (rd + 1) + x) : make_uint4(0, 0, 0, 0);
+        }
+        tmem_st_16x32bx2_x16<C / 4>(tq + 16 * rd, *reinterpret_cast<const uint32_t(*)[16]>(&cur[0]));
+        if (rd + 1 < ROUNDS) {
+#pragma unroll
+          for (int x = 0; x < 4; ++x) cur[x] = nxt[x];
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->q_full));
+      ++nq;
+      return true;
+    };
+    // the next unit of this CTA with key tiles (its Q is written ahead), or -1
+    auto next_unit = [&](int u0) -> int {
+      for (int uu = u0 + gridDim.x; uu < n_units; uu += gridDim.x) {
+        int a0, an;
+        split_range(key_set_tc(p, (uu / p.nsplit) % p.n_q), p.nsplit, uu % p.nsplit, a0, an);
+        if (an > 0) return uu;
+      }
+      return -1;
+    };
+    int q_ready_u = -1;                   // unit whose Q is already in tensor memory
     uint32_t g = 0, iq = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const int bq = u / p.nsplit, sp = u % p.nsplit;
@@ -716,6 +756,10 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
       const KeySet ks = key_set_tc(p, qi);
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
+      if (nt > 0 && q_ready_u != u) {
+        if (!write_q(u)) return;
+        q_ready_u = u;
+      }
       if (nt == 0 && p.nsplit > 1 && !p.cluster) continue;   // the combine kernel skips empty ranges
       __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
       if (nt == 0 && !p.cluster) {
@@ -820,6 +864,15 @@ attend_tc(AttendParams p, int n_units, const __grid_constant__ CUtensorMap tmQ,
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->p_full[st]));
+        if (j == nt - 1) {
+          // the unit's last S has been read: write the next unit's Q now, so
+          // its first S overlaps this unit's last P.V and epilogue
+          const int un = next_unit(u);
+          if (un >= 0) {
+            if (!write_q(un)) return;
+            q_ready_u = un;
+          }
+        }
       }
       // -------- epilogue: normalise, inverse RoPE, store
       if (nt > 0) {
@@ -997,19 +1050,6 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
   if (rc0) return rc0;
   // cluster merge: one unit per CTA, a query's splits form one cluster
   const int grid = p.cluster ? n_units : (n_units < num_sms() ? n_units : num_sms());
-  // tensor maps: q rows (box 64 x 64), compressed and window rows (box 1 x 64)
-  CUtensorMap tmQ, tmC, tmW;
-  const void *cbase = p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q);
-  const void *wbase = p.kv_win ? p.kv_win : cbase;
-  const uint64_t crows = p.kv_comp ? (uint64_t)p.B * p.cap : 1;
-  const uint64_t wrows = p.kv_win ? (uint64_t)p.B * (p.win_is_ring ? p.w : p.n_q) : crows;
-  int rc = encode_tmap_2d(&tmQ, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, (uint64_t)p.B * p.n_q * p.n_h, C * 2, 64, 64,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!rc) rc = encode_tmap_2d(&tmC, cbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, crows, C * 2, 64, 1,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!rc) rc = encode_tmap_2d(&tmW, wbase, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, C, wrows, C * 2, 64, 1,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-  if (rc) return rc;
   LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
   if (p.cluster) {
     cudaLaunchConfig_t cfg{};
@@ -1025,16 +1065,16 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     const cudaError_t e = attend_trace_on()
-                              ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units, tmQ, tmC, tmW)
-                              : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units, tmQ, tmC, tmW);
+                              ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units)
+                              : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units);
     if (e != cudaSuccess) {
       (void)cudaGetLastError();
       return fail(HCA_ERR_CUDA, "attend_tc cluster launch: %s", cudaGetErrorString(e));
     }
     return ls_.done();
   }
-  if (attend_trace_on()) attend_tc<C, true><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
-  else attend_tc<C, false><<<grid, kThreads, smem, s>>>(p, n_units, tmQ, tmC, tmW);
+  if (attend_trace_on()) attend_tc<C, true><<<grid, kThreads, smem, s>>>(p, n_units);
+  else attend_tc<C, false><<<grid, kThreads, smem, s>>>(p, n_units);
   return ls_.done();
 }
 }  // namespace tc
