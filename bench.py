@@ -410,6 +410,12 @@ def cpu_cores():
 
 
 # --------------------------------------------------------------------------- main
+# DRAM bytes (read + write) per launch of the decode kernels at the 128K batch-32 workload,
+# from single ncu captures (profiles/*_b32.md); None where no capture covers the kernel.
+TRAFFIC_128K = {"index_scores": 134_297_600 + 5_803_264, "topk": 4_247_808, "attend_csa": 23_256_832,
+                "attend_hca": None}
+
+
 def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, traffic=None):
     ach = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"], "unit": "GB/s",
@@ -499,7 +505,8 @@ def main():
         per_launch_ms = kern[dom]["ms"] / kern[dom]["launches"]
         key = next((k for k in per_bytes if dom.startswith(k) or k in dom), None)
         if key is not None:
-            roof = roofline_hbm(per_bytes[key], per_launch_ms, peaks)
+            roof = roofline_hbm(per_bytes[key], per_launch_ms, peaks,
+                                traffic=TRAFFIC_128K.get(key) if wl is workloads.HYBRID_DECODE_128K else None)
             roof["algorithmic_bytes_per_launch"] = per_bytes[key]
         else:
             roof = {"bound": "hbm", "achieved": None, "peak": peaks["hbm"], "unit": "GB/s", "frac": None,
