@@ -705,7 +705,7 @@ attend_tc(AttendParams p, int n_units) {
     const uint32_t lane_O = (uint32_t)(q4 * 32) << 16;
     // Q of a unit into tensor memory (lane-half 1, columns q_col..): thread
     // (hl, half) stores head row r, bf16 dims [half*C/2, (half+1)*C/2), read
-    // from global in rounds of 16 words with the next round's loads in flight
+    // from global in batches of 16 x 16 B whose loads are all in flight
     uint32_t nq = 0;                      // Q writes so far (q_empty parity)
     auto write_q = [&](int uq) -> bool {
       if (nq > 0 && !twait(bar(bars->q_empty), (nq - 1) & 1, TR_P_QEMPTY)) return false;
@@ -715,21 +715,16 @@ attend_tc(AttendParams p, int n_units) {
       const uint4 *src = reinterpret_cast<const uint4 *>(
           reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((long long)bqq * p.n_h + (live ? r : 0)) * C + half * (C / 2));
       const uint32_t tq = tmem + lane_S + L::q_col;
-      constexpr int ROUNDS = C / 64;      // 16 words (4 x 16 B) per round
-      uint4 cur[4], nxt[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) cur[x] = live ? __ldg(src + x) : make_uint4(0, 0, 0, 0);
+      // C/16 uint4 (C/4 words) per thread, in batches of 16 uint4 whose loads are all in flight
+      constexpr int PER = C / 16, BATCH = PER < 16 ? PER : 16;
 #pragma unroll 1
-      for (int rd = 0; rd < ROUNDS; ++rd) {
-        if (rd + 1 < ROUNDS) {
+      for (int b0 = 0; b0 < PER; b0 += BATCH) {
+        uint4 v[BATCH];
 #pragma unroll
-          for (int x = 0; x < 4; ++x) nxt[x] = live ? __ldg(src + 4 * (rd + 1) + x) : make_uint4(0, 0, 0, 0);
-        }
-        tmem_st_16x32bx2_x16<C / 4>(tq + 16 * rd, *reinterpret_cast<const uint32_t(*)[16]>(&cur[0]));
-        if (rd + 1 < ROUNDS) {
+        for (int x = 0; x < BATCH; ++x) v[x] = live ? __ldg(src + b0 + x) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int x = 0; x < 4; ++x) cur[x] = nxt[x];
-        }
+        for (int y = 0; y < BATCH / 4; ++y)
+          tmem_st_16x32bx2_x16<C / 4>(tq + 4 * (b0 + 4 * y), *reinterpret_cast<const uint32_t(*)[16]>(&v[4 * y]));
       }
       tmem_st_wait();
       tc_fence_before();
