@@ -276,8 +276,9 @@ int launch_index_scores_tc(const IndexParams &p, cudaStream_t s) {
   // every SM streams keys
   const int n_qb = (p.n_q + 1) / 2;
   const int tiles = (Vmax + kRowsA - 1) / kRowsA;
+  // two resident blocks per SM: stay within one wave
   const long long want = 2LL * num_sms();
-  int units = (int)((want + (long long)p.B * n_qb - 1) / ((long long)p.B * n_qb));
+  int units = (int)(want / ((long long)p.B * n_qb));
   if (units > tiles) units = tiles;
   if (units < 1) units = 1;
   const int tpu = (tiles + units - 1) / units;
