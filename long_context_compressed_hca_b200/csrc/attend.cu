@@ -554,6 +554,7 @@ attend_tc(AttendParams p, int n_units) {
     if (threadIdx.x == 0) mbar_arrive_expect_tx(bar(bars->mg_full), (p.nsplit - 1) * merge_blk(C, p.nsplit));
     cluster_sync();
   }
+  pdl_wait();   // indices, caches and queries of the previous launch are complete
   if (TRACE && threadIdx.x == 0) ts[1] = global_ns();
 
   if (warp >= kProdWarp0) {
@@ -1046,30 +1047,26 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
   // cluster merge: one unit per CTA, a query's splits form one cluster
   const int grid = p.cluster ? n_units : (n_units < num_sms() ? n_units : num_sms());
   LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
-  if (p.cluster) {
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = p.nsplit;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    const cudaError_t e = attend_trace_on()
-                              ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units)
-                              : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units);
-    if (e != cudaSuccess) {
-      (void)cudaGetLastError();
-      return fail(HCA_ERR_CUDA, "attend_tc cluster launch: %s", cudaGetErrorString(e));
-    }
-    return ls_.done();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = p.cluster ? p.nsplit : 1;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = p.cluster ? 2 : 1;
+  const cudaError_t e = attend_trace_on() ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units)
+                                          : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "attend_tc launch: %s", cudaGetErrorString(e));
   }
-  if (attend_trace_on()) attend_tc<C, true><<<grid, kThreads, smem, s>>>(p, n_units);
-  else attend_tc<C, false><<<grid, kThreads, smem, s>>>(p, n_units);
   return ls_.done();
 }
 }  // namespace tc

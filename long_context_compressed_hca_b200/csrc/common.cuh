@@ -81,6 +81,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
   }
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: pdl_trigger lets the next kernel of the
+// stream (launched with programmatic stream serialization) be scheduled and run
+// its prologue; pdl_wait blocks until the previous kernel has completed and its
+// writes are visible.  Both are no-ops for launches without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -325,6 +325,7 @@ __global__ void __launch_bounds__(kThreads) decode_ingest_kernel(CompressParams 
                                                                  IngestRing ring, int pos) {
   extern __shared__ float sm[];
   const int b = blockIdx.x, part = blockIdx.y;
+  pdl_trigger();   // the layer's next kernel may start its prologue
   if (part == 0 && pa.B > 0) {
     compress_decode_block<Tin, TA>(pa, pos, b, sm);
   } else if (part == 1 && has_b) {

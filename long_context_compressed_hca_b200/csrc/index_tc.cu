@@ -99,6 +99,8 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const long long key_row0 = (long long)b * p.cap + e_begin;
+  pdl_trigger();   // the selection may start its prologue
+  pdl_wait();      // keys and queries of the previous launch are complete
 
   if (warp == 0) {
     // ------------------------------------------------ loads
@@ -254,7 +256,21 @@ int launch_tc_t(const IndexParams &p, int QB, int tiles_per_unit, int units_per_
   a.wI = p.wI; a.KI_scale = p.KI_scale; a.scores = p.scores; a.score_stride = p.score_stride; a.status = p.status;
   const long long grid = (long long)p.B * a.n_qb * units_per_qb;
   LaunchScope ls_(FP8 ? "index_scores_tc_fp8" : "index_scores_tc", s);
-  index_scores_tc<N, FP8, S><<<(unsigned)grid, L::threads, L::bytes, s>>>(a, tmK, tmQ);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(L::threads, 1, 1);
+  cfg.dynamicSmemBytes = L::bytes;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, index_scores_tc<N, FP8, S>, a, tmK, tmQ);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "index_scores_tc launch: %s", cudaGetErrorString(e));
+  }
   return ls_.done();
 }
 

@@ -209,6 +209,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   const int len = max(0, min(p.slice, seg_V - (int)rank * p.slice));
   const long long begin = seg_begin + (long long)rank * p.slice;   // element index of keys[0]
 
+  pdl_trigger();   // the attention may start its prologue
+  pdl_wait();      // the scores of the previous launch are complete
   if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
   else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
   for (int i = tid; i < kBinsMax; i += kTopkThreads) {
@@ -388,13 +390,15 @@ int launch_topk_cluster(const char *name, const TopkParams &t, const TopkPlan &p
   cfg.blockDim = dim3(kTopkThreads, 1, 1);
   cfg.dynamicSmemBytes = topk_smem(pl);
   cfg.stream = s;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = pl.C;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_cluster, t);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
