@@ -20,6 +20,8 @@
 //               Warp roles: 4 softmax/epilogue warps, 1 MMA warp, 4 gather
 //               warps (cp.async of the selected rows into 128B-swizzled tiles).
 //   attend_simt fp32 CUDA cores, any shape (and the tiny fp32 workload).
+#include <cmath>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -270,7 +272,7 @@ struct Bars {
   uint64_t q_full, q_empty, o_empty, mma_done;
   uint64_t kv_full[8], kv_empty[8], s_full[2], s_empty[2], p_full[2], pv_done[2];
   uint64_t mg_ready, mg_full;    // cluster merge: peers' buffers free / peers' partials delivered
-  uint64_t mg_stage, mg_wt;      // cluster merge: this CTA's blocks staged / merge weights written
+  uint64_t mg_stage;             // cluster merge: this CTA's blocks staged
 };
 
 template <int C>
@@ -325,8 +327,8 @@ __host__ __device__ constexpr int merge_cols(int C, int ns) { return ((C / ns + 
 __host__ __device__ constexpr int merge_pitch(int C, int ns) { return merge_cols(C, ns) + 8; }   // bf16 elements
 // one owner's block: O [64][pitch] bf16, then (max, sum) [64] float2
 __host__ __device__ constexpr uint32_t merge_blk(int C, int ns) { return 64u * merge_pitch(C, ns) * 2 + 64 * 8; }
-// staged blocks [ns], received blocks [ns] (own slot unused), weights [64][8] fp32
-__host__ __device__ constexpr uint32_t merge_bytes(int C, int ns) { return 2u * ns * merge_blk(C, ns) + 64 * 8 * 4; }
+// staged blocks [ns], received blocks [ns] (own slot unused)
+__host__ __device__ constexpr uint32_t merge_bytes(int C, int ns) { return 2u * ns * merge_blk(C, ns); }
 template <int C>
 __host__ __device__ constexpr bool merge_fits() {
   for (int ns = 2; ns <= kMaxClusterSplits; ++ns)
@@ -369,7 +371,6 @@ __device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *sm
   const uint32_t blk = merge_blk(C, ns);
   uint8_t *stage = smem;                      // [ns] blocks
   uint8_t *recv = smem + ns * blk;            // [ns] blocks
-  float *wt = reinterpret_cast<float *>(smem + 2 * ns * blk);
   long long tw = trace ? clock64() : 0;
   // ---- stage O (bf16), 16 columns per TMEM load
   if (nt > 0) {
@@ -416,43 +417,37 @@ __device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *sm
   bool ok = mbar_wait_cluster(smem_u32(&bars->mg_full), 0, p.status);
   if (trace) { const long long t = clock64(); trace[1] += t - tw; tw = t; }
   if (ok) {
-    // ---- merge weights of every head row
     auto ml_of = [&](int i, int row) -> float2 {
       const uint8_t *base = (i == sp ? stage + i * blk : recv + i * blk);
       return reinterpret_cast<const float2 *>(base + 64u * pitch * 2)[row];
     };
-    if (mt < 64) {
-      const float sink2 = mt < p.n_h ? p.sink[mt] * kLog2e : 0.f;
-      float M = sink2;
-      for (int i = 0; i < ns; ++i) {
-        const float2 v = ml_of(i, mt);
-        if (v.y > 0.f) M = fmaxf(M, v.x);
-      }
-      float den = exp2f(sink2 - M);
-      float e[kMaxClusterSplits];
-#pragma unroll
-      for (int i = 0; i < kMaxClusterSplits; ++i) {
-        const float2 v = i < ns ? ml_of(i, mt) : make_float2(0.f, 0.f);
-        e[i] = v.y > 0.f ? exp2f(v.x - M) : 0.f;
-        den += e[i] * v.y;
-      }
-      const float inv = 1.f / den;
-#pragma unroll
-      for (int i = 0; i < kMaxClusterSplits; ++i) wt[mt * 8 + i] = e[i] * inv;
-    }
-    ok = merge_sync(&bars->mg_wt, p.status);
-  }
-  if (ok) {
-    if (trace) { const long long t = clock64(); trace[3] += t - tw; tw = t; }
-    // ---- this CTA's columns of every head row, 8 columns per item
+    // ---- this CTA's columns of every head row, 8 columns per item; each item
+    // derives its row's merge weights from the (max, sum) pairs itself
     const int c_lo = min(C, sp * per), c_hi = min(C, c_lo + per);
     const int ngr = (c_hi - c_lo) / 8;
     for (int it = mt; it < 64 * ngr; it += kMergeThreads) {
       const int row = it / ngr, cg = c_lo + 8 * (it % ngr);
       if (row >= p.n_h) continue;
+      const float sink2 = p.sink[row] * kLog2e;
+      float mi[kMaxClusterSplits], li[kMaxClusterSplits];
+      float M = sink2;
+#pragma unroll
+      for (int i = 0; i < kMaxClusterSplits; ++i) {
+        const float2 v = i < ns ? ml_of(i, row) : make_float2(-INFINITY, 0.f);
+        mi[i] = v.x;
+        li[i] = v.y;
+        if (v.y > 0.f) M = fmaxf(M, v.x);
+      }
+      float den = exp2f(sink2 - M);
+#pragma unroll
+      for (int i = 0; i < kMaxClusterSplits; ++i) {
+        mi[i] = li[i] > 0.f ? exp2f(mi[i] - M) : 0.f;   // now the unnormalised weight
+        den += mi[i] * li[i];
+      }
+      const float inv = 1.f / den;
       float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int i = 0; i < ns; ++i) {
-        const float w = wt[row * 8 + i];
+        const float w = mi[i] * inv;
         if (w == 0.f) continue;
         const uint8_t *base = (i == sp ? stage + i * blk : recv + i * blk);
         const uint4 v = *reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(base) +
@@ -535,7 +530,6 @@ attend_tc(AttendParams p, int n_units) {
       mbar_init(bar(bars->mg_ready), p.nsplit);
       mbar_init(bar(bars->mg_full), 1);
       mbar_init(bar(bars->mg_stage), kMergeThreads / 32);
-      mbar_init(bar(bars->mg_wt), kMergeThreads / 32);
     }
     mbar_fence_init();
   }
@@ -543,8 +537,7 @@ attend_tc(AttendParams p, int n_units) {
     tmem_alloc(smem_u32(tmem_slot), L::tmem_cols);
     tmem_relinquish();
   }
-  if (threadIdx.x < p.rd / 2)
-    freq[threadIdx.x] = exp2(-2.0 * (double)threadIdx.x / (double)p.rd * log2((double)p.theta));
+  if (threadIdx.x < p.rd / 2) freq[threadIdx.x] = p.rope_freq[threadIdx.x];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1138,6 +1131,8 @@ size_t attend_workspace_bytes(const AttendParams &p) {
 int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t s) {
   if (p_in.B * p_in.n_q == 0) return HCA_OK;
   AttendParams p = p_in;
+  for (int i = 0; i < 32; ++i)
+    p.rope_freq[i] = i < p.rd / 2 ? std::exp2(-2.0 * i / (double)p.rd * std::log2((double)p.theta)) : 0.0;
   p.nsplit = 1;
   p.cluster = 0;
   if (tc_path(p)) {

@@ -262,28 +262,43 @@ __device__ __forceinline__ void compress_decode_block(const CompressParams &p, i
   float *ent = sm;                   // [W]
   float *red = sm + W;               // [W / 8]
   float *red2 = red + W / 8;         // [W / 8]
+  // one online pass over the block's rows, 8 rows per step with their loads
+  // issued together (an HCA block has 128 rows)
   for (int ch = threadIdx.x; ch < W; ch += kThreads) {
-    float M = -INFINITY;
-    for (int r = 0; r < m; ++r) {
-      if (p.overlap) {
-        M = fmaxf(M, ssc[(long long)r * C + ch]);
-        M = fmaxf(M, ssc[(long long)(m + r) * C + W + ch]);
-      } else {
-        M = fmaxf(M, ssc[(long long)r * C + ch]);
+    float M = -INFINITY, S = 0.f, A = 0.f;
+    for (int r0 = 0; r0 < m; r0 += 8) {
+      float za[8], va[8], zb[8], vb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + u;
+        za[u] = -INFINITY; va[u] = 0.f; zb[u] = -INFINITY; vb[u] = 0.f;
+        if (r < m) {
+          if (p.overlap) {
+            zb[u] = ssc[(long long)r * C + ch];
+            vb[u] = skv[(long long)r * C + ch];
+            za[u] = ssc[(long long)(m + r) * C + W + ch];
+            va[u] = skv[(long long)(m + r) * C + W + ch];
+          } else {
+            za[u] = ssc[(long long)r * C + ch];
+            va[u] = skv[(long long)r * C + ch];
+          }
+        }
       }
-    }
-    float S = 0.f, A = 0.f;
-    for (int r = 0; r < m; ++r) {
-      if (p.overlap) {
-        const float e0 = __expf(ssc[(long long)r * C + ch] - M);
-        const float e1 = __expf(ssc[(long long)(m + r) * C + W + ch] - M);
-        S += e0 + e1;
-        A += e0 * skv[(long long)r * C + ch] + e1 * skv[(long long)(m + r) * C + W + ch];
-      } else {
-        const float e0 = __expf(ssc[(long long)r * C + ch] - M);
-        S += e0;
-        A += e0 * skv[(long long)r * C + ch];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx = fmaxf(mx, fmaxf(za[u], zb[u]));
+      if (mx == -INFINITY) continue;
+      const float Mn = fmaxf(M, mx);
+      const float sc = __expf(M - Mn);   // 0 while M is still -inf
+      S *= sc;
+      A *= sc;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float ea = __expf(za[u] - Mn), eb = __expf(zb[u] - Mn);
+        S += ea + eb;
+        A += ea * va[u] + eb * vb[u];
       }
+      M = Mn;
     }
     ent[ch] = A / S;
   }

@@ -115,6 +115,7 @@ struct AttendParams {
   int csa;                 // 1: compressed set from idx; 0: all visible entries
   int win_is_ring;
   float scale, theta, sink_log2_bias;
+  double rope_freq[32];    // theta^(-2i/rd) for the rd/2 rotated pairs (host-computed)
   const void *q;           // [B, n_q, n_h, c]
   const void *kv_comp;     // [B, cap, c]
   const int32_t *idx;      // [B, n_q, k]

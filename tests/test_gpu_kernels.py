@@ -90,7 +90,8 @@ def test_compress_prefill(cuda, overlap, m, width, n, in_dt, out_dt, flags, rd):
                 np.testing.assert_allclose(sc[b, r], za, rtol=1e-6, atol=1e-6)
 
 
-@pytest.mark.parametrize("overlap,m,width,n0,steps", [(1, 4, 64, 10, 23), (0, 8, 128, 5, 30), (1, 4, 512, 64, 9)])
+@pytest.mark.parametrize("overlap,m,width,n0,steps", [(1, 4, 64, 10, 23), (0, 8, 128, 5, 30), (1, 4, 512, 64, 9),
+                                                      (0, 128, 128, 100, 160)])
 def test_compress_decode_matches_prefill(cuda, overlap, m, width, n0, steps):
     """prefill(n0) then one decode step per token == prefill(n0 + steps)."""
     B = 2
