@@ -749,6 +749,17 @@ attend_tc(AttendParams p, int n_units) {
         if (!write_q(u)) return;
         q_ready_u = u;
       }
+      {
+        // pull the next unit's Q rows towards L2 now; they are written to tensor
+        // memory after this unit's last S
+        const int un = next_unit(u);
+        if (un >= 0 && r < p.n_h) {
+          const char *nq = reinterpret_cast<const char *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+                                                          ((long long)(un / p.nsplit) * p.n_h + r) * C + half * (C / 2));
+#pragma unroll
+          for (int x = 0; x < C / 128; ++x) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * x));
+        }
+      }
       if (nt == 0 && p.nsplit > 1 && !p.cluster) continue;   // the combine kernel skips empty ranges
       __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
       if (nt == 0 && !p.cluster) {
