@@ -574,6 +574,18 @@ attend_tc(AttendParams p, int n_units) {
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
       if (nt == 0) continue;
+      if (p.csa && pt < 32) {
+        // index lists: this unit's into L1 (read tile by tile below), the next
+        // unit's of this CTA into L2
+        const int32_t *il = p.idx + ((long long)b * p.n_q + qi) * p.k;
+        const int lines = (p.k * 4 + 127) / 128;
+        for (int x = pt; x < lines; x += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(il + 32 * x));
+        const int un = u + gridDim.x;
+        if (un < n_units) {
+          const int32_t *nl = p.idx + (long long)(un / p.nsplit) * p.k;
+          for (int x = pt; x < lines; x += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(nl + 32 * x));
+        }
+      }
       // masked slots read a real row of a real tensor (cap is 0 when kv_comp is absent)
       const __nv_bfloat16 *cbase = reinterpret_cast<const __nv_bfloat16 *>(
           p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q));
