@@ -174,9 +174,12 @@ int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const 
  * kv_win: prefill (win_is_ring == 0, start_pos == 0): [B, n_q, c], row t =
  *   token t; decode (win_is_ring == 1, n_q == 1): [B, w, c] ring, token p in
  *   slot p % w (the caller has already stored token start_pos).
- * ws: scratch for split-KV (few queries: each key list is cut across CTAs and
- *   the fp32 partials are merged); *_attend_workspace_size() gives its size.
- *   With ws == NULL or too small the call runs unsplit (same result). */
+ * Few queries (decode): each query's key list is cut across up to 8 CTAs of a
+ *   thread-block cluster whose partials are merged on chip; no scratch needed.
+ * ws: scratch only for a query cut into more than 8 pieces (fp32 partials +
+ *   a merge launch); *_attend_workspace_size() gives its size (0 when not
+ *   needed).  With ws == NULL or too small such a call is cut into 8 pieces
+ *   instead (same result up to fp32 rounding order). */
 size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos);
 int csa_attend(const hca_attn_desc *d, const void *q, const void *kv_comp, int cap,
                const int32_t *idx, const void *kv_win, int win_is_ring,

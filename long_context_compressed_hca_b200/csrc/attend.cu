@@ -12,13 +12,17 @@
 //
 // Two implementations:
 //   attend_tc   bf16, tcgen05.  One query token per work unit, its n_h (<= 64)
-//               heads form the M=64 rows.  Per 64-key tile: S = Q K^T into a
-//               TMEM accumulator in lane-half 1 (double buffered), softmax in
-//               registers, P (bf16) to shared memory, O += P V into a TMEM
-//               accumulator in lane-half 0 (up to 512 fp32 columns).  The key
-//               tile in shared memory serves as K (K-major) and V (MN-major).
-//               Warp roles: 4 softmax/epilogue warps, 1 MMA warp, 4 gather
-//               warps (cp.async of the selected rows into 128B-swizzled tiles).
+//               heads form the M=64 rows.  Q sits in tensor memory (written by
+//               the softmax warps) and is the A operand of S = Q K^T, which
+//               lands per 64-key tile in a TMEM accumulator in lane-half 1
+//               (double buffered); softmax in registers, P (bf16) to shared
+//               memory, O += P V into a TMEM accumulator in lane-half 0 (up to
+//               512 fp32 columns).  The key tile in shared memory (3 stages at
+//               c = 512) serves as K (K-major) and V (MN-major).  Warp roles:
+//               4 softmax/epilogue warps, 1 MMA warp, 8 gather warps (cp.async
+//               of the selected rows into 128B-swizzled tiles).  Few queries:
+//               a query's tiles are split over the CTAs of a cluster and
+//               merged in distributed shared memory.
 //   attend_simt fp32 CUDA cores, any shape (and the tiny fp32 workload).
 #include <cmath>
 
