@@ -15,8 +15,7 @@ order and notation of the pages:
        sets), "CSA 选择器层代码实现" (Compressor, Indexer), "HCA 选择函数代码实现"
        (visible-entry rule), "输出投影" (inverse RoPE on the output).
 
-Readings taken where the pages are silent or disagree (each is listed in
-the design doc with its justification):
+Readings taken where the pages are silent or disagree:
   * visibility: entry s is visible to query t iff (s+1)*m <= t+1 ([Z] Indexer
     mask and get_compress_topk_idxs; [J] Eq.(16)'s s < floor(t/m) with 1-based t);
   * RoPE: theta = 10000, interleaved pairs (2i, 2i+1) of the last rd dims,
