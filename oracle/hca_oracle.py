@@ -333,6 +333,30 @@ def layer_prefill(H, W: dict, L, d_c: int, eps: float = 1e-6, theta: float = 100
 # ---------------------------------------------------------------------------
 
 
+# ---------------------------------------------------------------------------
+# grouped output projection  ([J] §2.3.1(d); [Z] 输出投影)
+# ---------------------------------------------------------------------------
+
+
+def output_projection(o, wo_a, wo_b, g: int) -> np.ndarray:
+    """The attention output of one token, o [n_h, c] (inverse RoPE already
+    applied), split into g groups of n_h/g heads; group i's flattened
+    n_h*c/g values go through wo_a[i] ([d_g, n_h*c/g]) to d_g values, the g
+    results are concatenated (group order) and wo_b ([d, g*d_g]) maps them
+    to the layer output [d].  o may carry leading token dims."""
+    o = np.asarray(o, np.float64)
+    lead = o.shape[:-2]
+    n_h, c = o.shape[-2:]
+    wo_a = np.asarray(wo_a, np.float64)
+    wo_b = np.asarray(wo_b, np.float64)
+    d_g = wo_a.shape[1]
+    grp = o.reshape(lead + (g, n_h * c // g))
+    mid = np.empty(lead + (g, d_g))
+    for i in range(g):
+        mid[..., i, :] = grp[..., i, :] @ wo_a[i].T
+    return mid.reshape(lead + (g * d_g,)) @ wo_b.T
+
+
 def decode_new_entry(pos: int, m: int, cur_Ca, cur_Za, Ba, prev_Cb=None, prev_Zb=None, Bb=None):
     """The entry a decode step emits, or None.
 

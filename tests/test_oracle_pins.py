@@ -393,3 +393,50 @@ def test_decode_emission_equals_prefill_entries():
         if e is not None:
             got.append(e)
     np.testing.assert_allclose(np.stack(got), ref, atol=1e-14)
+
+
+# ----------------------------------------------------------- grouped output projection
+def test_output_projection_equals_block_diagonal_projection():
+    """Grouping = one projection whose first matrix is block diagonal over the
+    groups (assembled here element by element, not by the grouping code)."""
+    rng = np.random.default_rng(7)
+    n_h, c, g, d_g, d = 8, 6, 4, 5, 9
+    o = rng.normal(size=(3, n_h, c))
+    wo_a = rng.normal(size=(g, d_g, n_h * c // g))
+    wo_b = rng.normal(size=(d, g * d_g))
+    big = np.zeros((g * d_g, n_h * c))
+    w = n_h * c // g
+    for i in range(g):
+        for r in range(d_g):
+            for j in range(w):
+                big[i * d_g + r, i * w + j] = wo_a[i, r, j]
+    ref = np.stack([wo_b @ (big @ o[t].reshape(-1)) for t in range(3)])
+    np.testing.assert_allclose(O.output_projection(o, wo_a, wo_b, g), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_output_projection_group_permutation_invariance():
+    """Relabelling the groups (heads, wo_a blocks and wo_b column blocks
+    together) leaves the output unchanged; swapping only the heads does not."""
+    rng = np.random.default_rng(8)
+    n_h, c, g, d_g, d = 8, 4, 4, 3, 5
+    o = rng.normal(size=(n_h, c))
+    wo_a = rng.normal(size=(g, d_g, n_h * c // g))
+    wo_b = rng.normal(size=(d, g * d_g))
+    perm = np.array([2, 0, 3, 1])
+    hpg = n_h // g
+    o_p = o.reshape(g, hpg, c)[perm].reshape(n_h, c)
+    wb_p = wo_b.reshape(d, g, d_g)[:, perm].reshape(d, g * d_g)
+    base = O.output_projection(o, wo_a, wo_b, g)
+    np.testing.assert_allclose(O.output_projection(o_p, wo_a[perm], wb_p, g), base, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(O.output_projection(o_p, wo_a, wo_b, g), base)
+
+
+def test_output_projection_identity_weights_flatten():
+    """d_g = n_h*c/g with identity blocks and wo_b = I returns o flattened."""
+    rng = np.random.default_rng(9)
+    n_h, c, g = 4, 3, 2
+    w = n_h * c // g
+    o = rng.normal(size=(n_h, c))
+    wo_a = np.stack([np.eye(w)] * g)
+    wo_b = np.eye(g * w)
+    np.testing.assert_allclose(O.output_projection(o, wo_a, wo_b, g), o.reshape(-1), rtol=0, atol=0)
