@@ -367,6 +367,31 @@ def run_prefill(wl, K, W, flush, stream):
                 att_flops=att_flops, idx_flops=idx_flops)
 
 
+# --------------------------------------------------------------------------- output projection
+def run_oproj(T, K, W, flush, stream):
+    """Grouped output projection of T tokens at the CSA layer's widths
+    (64 heads x 512, g = 8 groups, d_g = 1024, d = 4096): 2*T*(n_h*c*d_g + g*d_g*d) FLOP."""
+    n_h, c, g, d_g, d = 64, 512, 8, 1024, 4096
+    gw = n_h * c // g
+    o = dev_normal((T, n_h, c), 7, 1, torch.bfloat16)
+    wo_a = dev_normal((g, d_g, gw), 7, 2, torch.bfloat16, std=gw ** -0.5)
+    wo_b = dev_normal((d, g * d_g), 7, 3, torch.bfloat16, std=(g * d_g) ** -0.5)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    desc = hb.oproj_desc(T, n_h, c, g, d_g, d, hb.HCA_BF16, hb.HCA_BF16)
+    ws = torch.empty(hb.output_projection_workspace_size(desc), dtype=torch.uint8, device="cuda")
+
+    def step():
+        hb.output_projection(desc, o, wo_a, wo_b, out, ws)
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    ms, _, _ = time_steps(step, K, flush, stream)
+    flops = 2.0 * T * (n_h * c * d_g + g * d_g * d)
+    del o, wo_a, wo_b, out, ws
+    torch.cuda.empty_cache()
+    return statistics.mean(ms), flops
+
+
 # --------------------------------------------------------------------------- oracle arm
 def oracle_decode_sample(bench: DecodeBench, n_seq: int):
     """Time the oracle on `n_seq` sequences of one decode step (both layers)."""
@@ -560,6 +585,12 @@ def main():
             if r["idx_flops"]:
                 sc_ms, _ = kern_ms(r["kern"], "index_scores", kp)
                 extras[key]["roofline_index"] = roofline_tensor(r["idx_flops"], sc_ms, peaks)
+
+    if world == 1 and not args.only_headline:
+        oms, ofl = run_oproj(65536, max(3, min(args.steps, 5)), 3, flush, stream)
+        extras["output_projection_64k"] = {
+            "workload": "grouped output projection, 65536 tokens, 64x512 -> 8x1024 -> 4096, bf16",
+            "ms": round(oms, 3), "roofline": roofline_tensor(ofl, oms, peaks)}
 
     if rank == 0:
         line = {

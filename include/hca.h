@@ -252,6 +252,23 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
                        int pos, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Grouped output projection, [J] §2.3.1(d); [Z] 输出投影 -- the step after the
+ * attention.  o [T, n_h, c] (inverse RoPE already applied, dtype) is split into
+ * g groups of n_h/g consecutive heads; group i's n_h*c/g values go through
+ * wo_a[i] to d_g values:  mid_i = o_i . wo_a[i]^T  (wo_a [g, d_g, n_h*c/g]);
+ * out [T, d] = concat_i(mid_i) . wo_b^T  (wo_b [d, g*d_g]).  Weights are
+ * row-major in dtype (f32 or bf16); out is f32 or bf16 (out_dtype).  The
+ * intermediate [T, g*d_g] is kept in ws in dtype (bf16 rounding for bf16).
+ * Requires n_h % g == 0; pointers 16-byte aligned. */
+typedef struct {
+  int T, n_h, c, g, d_g, d;
+  hca_dtype dtype, out_dtype;
+} hca_oproj_desc;
+size_t hca_output_projection_workspace_size(const hca_oproj_desc *d);
+int hca_output_projection(const hca_oproj_desc *d, const void *o, const void *wo_a, const void *wo_b,
+                          void *out, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status and diagnostics.
  * ---------------------------------------------------------------------- */
 const char *hca_last_error(void);   /* text of the last failing call (thread-local) */

@@ -57,6 +57,11 @@ class Cache(C.Structure):
                 ("state_score", C.c_void_p), ("stateI_kv", C.c_void_p), ("stateI_score", C.c_void_p)]
 
 
+class OprojDesc(C.Structure):
+    _fields_ = [("T", C.c_int), ("n_h", C.c_int), ("c", C.c_int), ("g", C.c_int), ("d_g", C.c_int),
+                ("d", C.c_int), ("dtype", C.c_int), ("out_dtype", C.c_int)]
+
+
 class TokenIn(C.Structure):
     _fields_ = [("q", C.c_void_p), ("qI", C.c_void_p), ("wI", C.c_void_p), ("kv", C.c_void_p),
                 ("comp", C.c_void_p), ("compI", C.c_void_p)]
@@ -89,6 +94,8 @@ def _declare(L):
         "hybrid_layer_forward_workspace_size": (SZ, [C.POINTER(Layer), I]),
         "hybrid_layer_forward": (I, [C.POINTER(Layer), VP, I, C.POINTER(Cache), VP, VP, SZ, VP]),
         "hybrid_decode_step_workspace_size": (SZ, [C.POINTER(Layer), I]),
+        "hca_output_projection_workspace_size": (SZ, [C.POINTER(OprojDesc)]),
+        "hca_output_projection": (I, [C.POINTER(OprojDesc), VP, VP, VP, VP, VP, SZ, VP]),
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
     }
@@ -281,3 +288,17 @@ def hybrid_decode_step(L: Layer, x: TokenIn, cache: Cache, pos, o, ws, stream=No
     nbytes = ws.numel() * ws.element_size()
     return check(lib().hybrid_decode_step(C.byref(L), C.byref(x), C.byref(cache), pos, ptr(o), ptr(ws),
                                           nbytes, stream_handle(stream)))
+
+
+def oproj_desc(T, n_h, c, g, d_g, d, dtype=HCA_BF16, out_dtype=HCA_F32) -> OprojDesc:
+    return OprojDesc(T, n_h, c, g, d_g, d, dtype, out_dtype)
+
+
+def output_projection_workspace_size(d: OprojDesc) -> int:
+    return lib().hca_output_projection_workspace_size(C.byref(d))
+
+
+def output_projection(d: OprojDesc, o, wo_a, wo_b, out, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws is not None else 0
+    return check(lib().hca_output_projection(C.byref(d), ptr(o), ptr(wo_a), ptr(wo_b), ptr(out), ptr(ws), nbytes,
+                                             stream_handle(stream)))

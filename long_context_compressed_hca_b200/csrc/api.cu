@@ -398,6 +398,40 @@ int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const 
   return run_index_topk_static(p, idx, scores, score_stride, static_cast<cudaStream_t>(stream));
 }
 
+// ----------------------------------------------------------------- output projection
+size_t hca_output_projection_workspace_size(const hca_oproj_desc *d) {
+  if (!d || d->T < 0 || d->g < 1 || d->d_g < 1) return 0;
+  const size_t b = (size_t)d->T * d->g * d->d_g * esize(d->dtype);
+  return (b + 255) & ~(size_t)255;
+}
+
+int hca_output_projection(const hca_oproj_desc *d, const void *o, const void *wo_a, const void *wo_b, void *out,
+                          void *ws, size_t ws_bytes, hca_stream_t stream) {
+  REQUIRE(d != nullptr, "null descriptor");
+  REQUIRE(d->T >= 0 && d->n_h >= 1 && d->c >= 1 && d->g >= 1 && d->d_g >= 1 && d->d >= 1, "bad shape");
+  REQUIRE(d->n_h % d->g == 0, "n_h (%d) must be a multiple of g (%d)", d->n_h, d->g);
+  REQUIRE(d->dtype == HCA_F32 || d->dtype == HCA_BF16, "dtype must be f32 or bf16");
+  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16, "out_dtype must be f32 or bf16");
+  if (d->T == 0) return HCA_OK;
+  REQUIRE(o && wo_a && wo_b && out, "o, wo_a, wo_b and out must be non-null");
+  REQUIRE(aligned16(o) && aligned16(wo_a) && aligned16(wo_b) && aligned16(out), "pointers must be 16-byte aligned");
+  REQUIRE(ws && ws_bytes >= hca_output_projection_workspace_size(d), "workspace too small");
+  const int gw = d->n_h / d->g * d->c;          // values per group
+  const int mid_n = d->g * d->d_g;
+  const size_t es = esize(d->dtype);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const char *ob = static_cast<const char *>(o);
+  const char *wa = static_cast<const char *>(wo_a);
+  char *mid = static_cast<char *>(ws);
+  for (int i = 0; i < d->g; ++i) {
+    const int rc = launch_gemm(d->dtype, ob + (size_t)i * gw * es, (long long)d->n_h * d->c,
+                               wa + (size_t)i * d->d_g * gw * es, gw, mid + (size_t)i * d->d_g * es, mid_n, d->dtype,
+                               d->T, d->d_g, gw, 1.f, s);
+    if (rc) return rc;
+  }
+  return launch_gemm(d->dtype, mid, mid_n, wo_b, mid_n, out, d->d, d->out_dtype, d->T, d->d, mid_n, 1.f, s);
+}
+
 // ----------------------------------------------------------------- attend
 size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
   if (!d) return 0;
