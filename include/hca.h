@@ -19,7 +19,11 @@
  *     invalid call launches nothing and changes no buffer.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and is asynchronous.  Nothing here synchronises except
- *     hca_check_status().
+ *     hca_check_status() and the diagnostics (hca_profile_sample,
+ *     hca_trace_attend with counters).
+ *   - Stream order is kept: a library kernel may be scheduled while the
+ *     library kernel before it finishes (programmatic dependent launch), but
+ *     it waits for that kernel's completion before touching any buffer.
  *   - The caller owns every device buffer.  The library allocates no device
  *     memory: scratch is passed as `ws` of at least the size the matching
  *     *_workspace_size() returns (256-byte aligned).
