@@ -472,9 +472,9 @@ def cpu_cores():
 
 # --------------------------------------------------------------------------- main
 # DRAM bytes (read + write) per launch of the decode kernels at the 128K batch-32 workload,
-# from single ncu captures (profiles/*_b32.md); None where no capture covers the kernel.
-TRAFFIC_128K = {"index_scores": 134_297_600 + 5_803_264, "topk": 4_247_808, "attend_csa": 23_256_832,
-                "attend_hca": None}
+# from single ncu captures (profiles/*_b32.md); None where no capture covers the kernel as it is.
+TRAFFIC_128K = {"index_scores": 134_289_408 + 4_679_680, "topk": None, "attend_csa": 23_249_920 + 1_536,
+                "attend_hca": 39_961_600 + 5_376}
 
 
 def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, traffic=None):

@@ -244,6 +244,51 @@ def test_index_topk_exact_ties(cuda, B, n_q, start_pos, k, kdt):
             np.testing.assert_array_equal(gi[b, i], O.topk_select(ref, k))
 
 
+POW2_CASES = [
+    # start_pos (one query, m = 4): a cluster of 8 CTAs (32768 entries) and of 4 (12500)
+    131071,
+    49999,
+]
+
+
+@pytest.mark.parametrize("start_pos", POW2_CASES)
+def test_index_topk_pow2_classes(cuda, start_pos):
+    """Every index key is one key scaled by a power of two, so with positive
+    head weights each score is that key's score times the same power of two,
+    exactly: the scores form classes of equal values one binade apart.  Row 0
+    puts the k-th score inside a class of 1500 entries scattered over the
+    row (ties across CTAs, resolved towards the lower index, Eq.(17)); row 1
+    ends the top k exactly at a class boundary."""
+    B, n_q, m, k, n_hI, c_I = 2, 1, 4, 512, 8, 64
+    E = (start_pos + n_q) // m
+    cap = E + 1
+    rng = np.random.default_rng(start_pos)
+    expo = np.zeros((B, cap), dtype=np.int64)
+    for b, sizes in enumerate(((100, 300, 1500), (100, 412))):
+        perm = rng.permutation(E)
+        e = rng.integers(0, 9, size=cap)          # the bulk: exponents 0..8
+        at = 0
+        for j, n in enumerate(sizes):             # the top classes: exponents 11, 10, 9
+            e[perm[at:at + n]] = 11 - j
+            at += n
+        expo[b] = e
+    base = synth.normal((B, 1, c_I), 91, 1).to(BF16).float()
+    KI = (base * torch.from_numpy(np.exp2(expo)).float()[..., None]).to(BF16).to(cuda)
+    qI = rnd((B, n_q, n_hI, c_I), 91, 2, BF16)
+    wI = rnd((B, n_q, n_hI), 91, 3, std=c_I ** -0.5).abs().to(cuda)
+    d = hb.attn_desc(B, 4, 64, 16, 8, m, k=k, n_hI=n_hI, c_I=c_I, rd_I=16, dtype=CODE[BF16],
+                     idx_key_dtype=CODE[BF16])
+    ws = torch.empty(hb.csa_index_topk_workspace_size(d, n_q, start_pos), dtype=torch.uint8, device=cuda)
+    idx = torch.full((B, n_q, k), -7, dtype=torch.int32, device=cuda)
+    hb.csa_index_topk(d, qI, wI, KI, None, cap, n_q, start_pos, idx, None, 0, ws)
+    torch.cuda.synchronize()
+    q64, w64, K64, gi = to64(qI), to64(wI), to64(KI), idx.cpu().numpy()
+    for b in range(B):
+        ref = O.index_scores(q64[b, 0], w64[b, 0], K64[b], E)
+        assert ref.max() > 0 and len(np.unique(ref)) <= 12
+        np.testing.assert_array_equal(gi[b, 0], O.topk_select(ref, k))
+
+
 # ----------------------------------------------------------------- attention
 ATT_CASES = [
     # kind, dtype, B, n_q, n_h, c, rd, w, m, k
