@@ -133,17 +133,36 @@ def barrier():
 
 
 # --------------------------------------------------------------------------- decode
+# The HCA layer of a decode step runs on a side stream next to the CSA layer's
+# ingest -> indexer -> top-k -> attention chain, the step's critical path.  Per
+# workload: the CTA budgets of the CSA and HCA attention calls (0 = every SM) and
+# whether the HCA stream has the higher priority.  Measured in alternating runs on
+# one box (us per step):
+#   128K batch 32: every SM, equal priority 122; HCA first 118; HCA 32 CTAs (one
+#                  split per query) + HCA first 112.5; HCA 32 CTAs at equal priority 120
+#   1M batch 4:    every SM 148 (HCA: 32 splits through the fp32 workspace + combine);
+#                  HCA 32 CTAs (8 splits, cluster merge) at equal priority 128, HCA first
+#                  145; CSA 32 CTAs as well (8 splits instead of 9 + combine) 124, 16: 131
+LAYER_CTAS = {workloads.HYBRID_DECODE_128K.name: (0, 32, True),
+              workloads.HYBRID_DECODE_1M.name: (32, 32, False)}
+
+
 class DecodeBench:
     """One decode step per sequence over synthetic caches: CSA layer + HCA layer."""
 
-    def __init__(self, wl, seed_shift=0):
+    def __init__(self, wl, seed_shift=0, side_ctas=None, side_high=None):
         self.wl = wl
         B, pos = wl.B, wl.pos
         seed = wl.seed + seed_shift
+        main_ctas, ctas, high = LAYER_CTAS.get(wl.name, (0, 0, False))
+        self.main_ctas = main_ctas
+        self.side_ctas = ctas if side_ctas is None else side_ctas
+        self.side_high = high if side_high is None else side_high
         self.layers, self.caches, self.inputs, self.outs, self.ws = [], [], [], [], []
         for li, L in enumerate(wl.layers):
             W = synth.layer_weights(L, 64, 64, seed, torch.bfloat16, layer_id=li)   # decode reads sink/biases only
-            lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=wl.idx_key_dtype)
+            lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=wl.idx_key_dtype,
+                             max_ctas=self.side_ctas if li > 0 else self.main_ctas)
             lcm = 32
             cap = ((pos // L.m + 8 + lcm - 1) // lcm) * lcm
             ch = CacheHandle(L, B, cap, torch.bfloat16, idx_key_dtype=wl.idx_key_dtype)
@@ -197,7 +216,8 @@ class DecodeBench:
         inputs, outs = bufs if bufs is not None else (self.inputs, self.outs)
         cur = torch.cuda.current_stream()
         if not hasattr(self, "side"):
-            self.side = torch.cuda.Stream()
+            lo, hi = torch.cuda.Stream.priority_range()
+            self.side = torch.cuda.Stream(priority=hi if self.side_high else lo)
             self.fork, self.join = torch.cuda.Event(), torch.cuda.Event()
         self.fork.record(cur)
         self.side.wait_event(self.fork)
@@ -345,7 +365,8 @@ def run_decode(wl, K, W, flush, stream, e2e=True, sweep=False):
         torch.cuda.synchronize()
         return time_steps(pg.replay, K, flush, stream, profile=True, replayed=True)[2]
     kern = profiled(prof_pass)
-    res = dict(bench=b, ms=ms, launches=launches, kern=kern, graph=True)
+    res = dict(bench=b, ms=ms, launches=launches, kern=kern, graph=True, side_ctas=b.side_ctas,
+               side_high=b.side_high, main_ctas=b.main_ctas)
     if e2e:
         res["e2e_ms"] = [time_e2e_pipelined(b, K, W, stream)]
     del graph
@@ -473,8 +494,8 @@ def cpu_cores():
 # --------------------------------------------------------------------------- main
 # DRAM bytes (read + write) per launch of the decode kernels at the 128K batch-32 workload,
 # from single ncu captures (profiles/*_b32.md); None where no capture covers the kernel as it is.
-TRAFFIC_128K = {"index_scores": 134_289_408 + 4_679_680, "topk": None, "attend_csa": 23_249_920 + 1_536,
-                "attend_hca": 39_961_600 + 5_376}
+TRAFFIC_128K = {"index_scores": 134_289_408 + 4_679_680, "topk": 4_248_576, "attend_csa": 23_249_920 + 1_536,
+                "attend_hca": 39_943_680 + 11_008}   # at the bench's budget of 32 CTAs
 
 
 def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, traffic=None):
@@ -597,6 +618,9 @@ def main():
         tb, _ = d1["bench"].algorithmic_bytes()
         m1 = statistics.mean(d1["ms"])
         extras["decode_1m"] = {"workload": workloads.HYBRID_DECODE_1M.name, "us_per_step": round(m1 * 1e3, 2),
+                               "launch": f"attention budgets: CSA {d1['main_ctas'] or 'all'} CTAs, HCA "
+                                         f"{d1['side_ctas'] or 'all'} CTAs on a side stream of "
+                                         f"{'high' if d1['side_high'] else 'equal'} priority",
                                "roofline_step": roofline_hbm(tb, m1, peaks),
                                "kernels": {k: round(v["ms"] / args.steps * 1e3, 2) for k, v in d1["kern"].items()}}
         del d1
@@ -637,7 +661,9 @@ def main():
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "layers_per_step": "CSA(m=4,k=512,idx 8x64) + HCA(m'=128)",
                        "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "decode step replayed as one CUDA graph; CSA and HCA layers on two streams"},
+                       "launch": "decode step replayed as one CUDA graph; CSA layer on the main stream, HCA layer "
+                                 f"on a {'high-priority ' if head['side_high'] else ''}side stream "
+                                 f"(attention budget {head['side_ctas'] or 'all'} CTAs)"},
             "roofline": roof,
             "roofline_step": step_roof,
             "e2e": {"value": round(e2e_ms * 1e3, 2), "unit": "us/step", "h2d_bytes_per_step": hi,

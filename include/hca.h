@@ -78,6 +78,10 @@ typedef struct {
   float scale;             /* logit scale; <= 0 selects c^-1/2 */
   float eps;               /* RMSNorm epsilon (1e-6) */
   float rope_theta;        /* RoPE base (10000) */
+  int max_ctas;            /* attention only: at most this many CTAs (one per SM) per
+                              call, which also bounds the split-KV count per query;
+                              0 = every SM.  For a caller that runs another layer's
+                              kernels on a second stream at the same time. */
 } hca_attn_desc;
 
 /* ------------------------------------------------------------------------

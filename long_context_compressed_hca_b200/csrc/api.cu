@@ -149,6 +149,7 @@ int check_attn_desc(const hca_attn_desc *d, bool need_indexer) {
   REQUIRE(d->w >= 0, "w must be >= 0");
   REQUIRE(d->m >= 1, "m must be >= 1");
   REQUIRE(d->dtype == HCA_F32 || d->dtype == HCA_BF16, "dtype must be HCA_F32 or HCA_BF16");
+  REQUIRE(d->max_ctas >= 0, "max_ctas must be >= 0 (0 = every SM)");
   if (need_indexer) {
     REQUIRE(d->k >= 1, "k must be >= 1");
     REQUIRE(d->n_hI >= 1 && d->c_I >= 8 && d->c_I % 8 == 0, "indexer heads / dim invalid");
@@ -182,6 +183,7 @@ AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv
   p.status = nullptr;
   p.nsplit = 1;
   p.cluster = 0;
+  p.max_ctas = d->max_ctas;
   return p;
 }
 

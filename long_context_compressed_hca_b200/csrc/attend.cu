@@ -258,6 +258,12 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attend_simt(AttendParams p) {
   }
 }
 
+// CTAs one call may occupy: the caller's budget, else every SM.
+inline int sm_budget(const AttendParams &p) {
+  const int n = num_sms();
+  return p.max_ctas > 0 && p.max_ctas < n ? p.max_ctas : n;
+}
+
 // ======================================================================= tcgen05
 namespace tc {
 bool g_trace_on = false;
@@ -1065,7 +1071,7 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
   int rc0 = ensure_attr<C>();
   if (rc0) return rc0;
   // cluster merge: one unit per CTA, a query's splits form one cluster
-  const int grid = p.cluster ? n_units : (n_units < num_sms() ? n_units : num_sms());
+  const int grid = p.cluster ? n_units : (n_units < sm_budget(p) ? n_units : sm_budget(p));
   LaunchScope ls_(p.csa ? "attend_csa_tc" : "attend_hca_tc", s);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -1101,13 +1107,14 @@ bool tc_path(const AttendParams &p) {
 // Splits per query: enough work units to fill the GPU when there are few queries.
 int choose_splits_raw(const AttendParams &p) {
   const long long q = (long long)p.B * p.n_q;
-  if (q == 0 || q >= num_sms()) return 1;
+  const int sms = sm_budget(p);
+  if (q == 0 || q >= sms) return 1;
   // longest key list among the queries (the last one)
   const int t = p.start_pos + p.n_q - 1;
   const int V = (t + 1) / p.m;
   const int nk = (p.w < t + 1 ? p.w : t + 1) + (p.csa ? (p.k < V ? p.k : V) : V);
   const int tiles = (nk + 63) / 64;
-  int ns = (int)(num_sms() / q);          // every unit in one wave of persistent CTAs
+  int ns = (int)(sms / q);                // every unit in one wave of persistent CTAs
   if (ns > tiles / 2) ns = tiles / 2;     // keep >= 2 tiles per split
   if (ns > 32) ns = 32;
   return ns < 1 ? 1 : ns;

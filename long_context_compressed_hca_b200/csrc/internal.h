@@ -131,6 +131,7 @@ struct AttendParams {
   // combine kernel (cluster = 0)
   int nsplit;
   int cluster;
+  int max_ctas;            // CTA budget of the call (0 = every SM)
   float *part_o;           // [B*n_q, nsplit, 64, c]
   float *part_ml;          // [B*n_q, nsplit, 64, 2]
 };

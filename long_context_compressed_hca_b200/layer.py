@@ -19,7 +19,7 @@ class LayerHandle:
     """One attention layer: weights on `device` plus the hca_layer struct."""
 
     def __init__(self, L, W: dict, d: int, d_c: int, dtype: torch.dtype, B: int,
-                 idx_key_dtype: str = "bf16", device="cuda"):
+                 idx_key_dtype: str = "bf16", device="cuda", max_ctas: int = 0):
         self.shape, self.d, self.d_c, self.dtype, self.B = L, d, d_c, dtype, B
         dev = lambda t, dt=None: t.to(device=device, dtype=dt or t.dtype).contiguous()
         csa = L.kind == "csa"
@@ -41,7 +41,7 @@ class LayerHandle:
         self.idx_key_dtype = idx_key_dtype
         self.desc = hb.attn_desc(B, L.n_h, L.c, L.rd, L.w, L.m, overlap=L.overlap, k=L.k,
                                  n_hI=L.n_hI, c_I=L.c_I, rd_I=L.rd_I if csa else 0,
-                                 dtype=_code(dtype), idx_key_dtype=kdt)
+                                 dtype=_code(dtype), idx_key_dtype=kdt, max_ctas=max_ctas)
         g = lambda nm: hb.ptr(self.t.get(nm))
         self.struct = hb.Layer(hb.HCA_LAYER_CSA if csa else hb.HCA_LAYER_HCA, self.desc, d, d_c,
                                g("W_comp"), g("B_comp"), g("W_compI"), g("B_compI"), g("W_DQ"),

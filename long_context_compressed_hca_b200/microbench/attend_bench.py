@@ -2,7 +2,7 @@
 print the per-role wait-cycle trace.
 
     python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c]
-    python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos]
+    python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos] [max_ctas]
 
 Inputs are seeded N(0,1) (bf16); CSA index lists take one random visible entry
 per equal-width bucket (valid, sorted, no repeats)."""
@@ -20,6 +20,7 @@ def decode_main():
     kind = sys.argv[2] if len(sys.argv) > 2 else "csa"
     B = int(sys.argv[3]) if len(sys.argv) > 3 else 32
     pos = int(sys.argv[4]) if len(sys.argv) > 4 else 131072
+    max_ctas = int(sys.argv[5]) if len(sys.argv) > 5 else 0
     n_h, c, rd, w = 64, 512, 64, 128
     m, k = (4, 512) if kind == "csa" else (128, 0)
     V = (pos + 1) // m
@@ -37,7 +38,7 @@ def decode_main():
         u = torch.rand(B, k, device=dev, generator=g)
         idx = torch.floor((j[None] + u) * (V / k)).long().clamp(max=V - 1).int()[:, None].contiguous()
     o = torch.empty(B, 1, n_h, c, dtype=torch.bfloat16, device=dev)
-    d = hb.attn_desc(B, n_h, c, rd, w, m, k=max(k, 1), dtype=hb.HCA_BF16)
+    d = hb.attn_desc(B, n_h, c, rd, w, m, k=max(k, 1), dtype=hb.HCA_BF16, max_ctas=max_ctas)
     wsz = (hb.csa_attend_workspace_size if kind == "csa" else hb.hca_attend_workspace_size)(d, 1, pos)
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 

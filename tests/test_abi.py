@@ -69,6 +69,8 @@ def test_attend_rejects_bad_arguments(L):
     dbad = hb.attn_desc(1, 4, 48, 16, 8, 4, k=4)
     _bad(L.hca_attend(ctypes.byref(dbad), 16, 16, 100, 16, 0, 16, 4, 0, 16, None, 0, None), "multiple of 32")
     _bad(L.csa_attend(ctypes.byref(d), 16, 16, 100, None, 16, 0, 16, 4, 0, 16, None, 0, None), "idx")
+    dneg = hb.attn_desc(1, 4, 64, 16, 8, 4, k=4, max_ctas=-1)
+    _bad(L.hca_attend(ctypes.byref(dneg), 16, 16, 100, 16, 0, 16, 4, 0, 16, None, 0, None), "max_ctas")
 
 
 def test_index_rejects_bad_arguments(L):

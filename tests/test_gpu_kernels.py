@@ -302,7 +302,7 @@ ATT_CASES = [
 ]
 
 
-def _run_attend(kind, dt, B, n_q, n_h, c, rd, w, m, k, cuda, start_pos=0, ring=False, seed=5):
+def _run_attend(kind, dt, B, n_q, n_h, c, rd, w, m, k, cuda, start_pos=0, ring=False, seed=5, max_ctas=0):
     cap = (start_pos + n_q) // m + 2
     q = rnd((B, n_q, n_h, c), seed, 1, dt)
     kv_comp = rnd((B, cap, c), seed, 2, dt)
@@ -310,7 +310,7 @@ def _run_attend(kind, dt, B, n_q, n_h, c, rd, w, m, k, cuda, start_pos=0, ring=F
     sink = rnd((n_h,), seed, 4)
     idx = random_idx(B, n_q, start_pos, m, k, seed) if kind == "csa" else None
     o = torch.full((B, n_q, n_h, c), float("nan"), dtype=dt, device=cuda)
-    d = hb.attn_desc(B, n_h, c, rd, w, m, k=k, dtype=CODE[dt])
+    d = hb.attn_desc(B, n_h, c, rd, w, m, k=k, dtype=CODE[dt], max_ctas=max_ctas)
     if kind == "csa":
         hb.csa_attend(d, q, kv_comp, cap, idx, kv_win, ring, sink, n_q, start_pos, o)
     else:
@@ -372,6 +372,30 @@ def test_attend_decode_cluster_merge(cuda, kind, B, pos):
     for b in range(0, B, max(1, B // 4)):
         ref = _ref_attend(kind, q, kv_comp, kv_win, sink, idx, b, 0, pos, w, m, k, rd, True)
         assert_close(to64(o[b, 0]), ref, 2e-2, f"o[{b}]")
+
+
+@pytest.mark.parametrize("kind,B,pos,max_ctas", [("hca", 32, 131071, 64), ("hca", 32, 131071, 32),
+                                                 ("hca", 2, 100000, 6), ("csa", 5, 1700, 12)])
+def test_attend_decode_cta_budget(cuda, kind, B, pos, max_ctas):
+    """A CTA budget (max_ctas) bounds the splits per query -- 2, 1, 3 and 2
+    here instead of 4, 4, 7 and 4 -- without changing what is computed."""
+    n_h, c, rd, w = 64, 512, 64, 128
+    m, k = (4, 512) if kind == "csa" else (128, 0)
+    q, kv_comp, kv_win, sink, idx, o = _run_attend(kind, BF16, B, 1, n_h, c, rd, w, m, k, cuda,
+                                                   start_pos=pos, ring=True, max_ctas=max_ctas)
+    for b in range(0, B, max(1, B // 4)):
+        ref = _ref_attend(kind, q, kv_comp, kv_win, sink, idx, b, 0, pos, w, m, k, rd, True)
+        assert_close(to64(o[b, 0]), ref, 2e-2, f"o[{b}]")
+
+
+def test_attend_prefill_cta_budget(cuda):
+    """Prefill under a budget of 5 CTAs: the persistent grid shrinks to 5 and
+    each CTA works through 30 of the 150 query units."""
+    kind, dt, B, n_q, n_h, c, rd, w, m, k = "csa", BF16, 1, 150, 64, 512, 64, 37, 4, 100
+    q, kv_comp, kv_win, sink, idx, o = _run_attend(kind, dt, B, n_q, n_h, c, rd, w, m, k, cuda, max_ctas=5)
+    for i in (0, 1, 77, n_q - 1):
+        ref = _ref_attend(kind, q, kv_comp, kv_win, sink, idx, 0, i, 0, w, m, k, rd, False)
+        assert_close(to64(o[0, i]), ref, TOL[dt], f"o[0,{i}]")
 
 
 def test_attend_is_deterministic(cuda):
