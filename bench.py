@@ -147,6 +147,23 @@ LAYER_CTAS = {workloads.HYBRID_DECODE_128K.name: (0, 32, True),
               workloads.HYBRID_DECODE_1M.name: (32, 32, False)}
 
 
+def packed(tensors):
+    """Copies of `tensors` in one device buffer (each at a 256-byte aligned
+    offset): the buffer and the views, so that a step's inputs or outputs move
+    between host and device in one copy."""
+    offs, tot = [], 0
+    for t in tensors:
+        offs.append(tot)
+        tot += (t.numel() * t.element_size() + 255) // 256 * 256
+    flat = torch.empty(tot, dtype=torch.uint8, device="cuda")
+    views = []
+    for t, o in zip(tensors, offs):
+        v = flat[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views.append(v)
+    return flat, views
+
+
 class DecodeBench:
     """One decode step per sequence over synthetic caches: CSA layer + HCA layer."""
 
@@ -158,7 +175,7 @@ class DecodeBench:
         self.main_ctas = main_ctas
         self.side_ctas = ctas if side_ctas is None else side_ctas
         self.side_high = high if side_high is None else side_high
-        self.layers, self.caches, self.inputs, self.outs, self.ws = [], [], [], [], []
+        self.layers, self.caches, self.x, self.outs, self.ws = [], [], [], [], []
         for li, L in enumerate(wl.layers):
             W = synth.layer_weights(L, 64, 64, seed, torch.bfloat16, layer_id=li)   # decode reads sink/biases only
             lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=wl.idx_key_dtype,
@@ -188,25 +205,32 @@ class DecodeBench:
                 x.update(qI=dev_normal((B, L.n_hI, L.c_I), seed, s + 13, torch.bfloat16),
                          wI=dev_normal((B, L.n_hI), seed, s + 14, std=L.c_I ** -0.5 * L.n_hI ** -0.5),
                          compI=dev_normal((B, 4 * L.c_I), seed, s + 15))
-            ti = TokenInputs(**x)
+            self.x.append(x)
             o = torch.empty(B, L.n_h, L.c, dtype=torch.bfloat16, device="cuda")
             # sized for the 128 consecutive positions the step sweep visits
             ws = torch.empty(max(hb.decode_workspace_size(lh.struct, pos + 128), 256), dtype=torch.uint8,
                              device="cuda")
             self.layers.append(lh)
             self.caches.append(ch)
-            self.inputs.append(ti)
             self.outs.append(o)
             self.ws.append(ws)
         # pinned host copies for the end-to-end measurement
-        self.host_in = [{k: v.cpu().pin_memory() for k, v in ti.t.items() if v is not None} for ti in self.inputs]
-        self.host_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in self.outs]
+        self.in_flat, self.inputs, self.out_flat, self.outs = self.buffer_set()
+        self.host_in = self.in_flat.cpu().pin_memory()
+        self.host_out = torch.empty(self.out_flat.shape, dtype=torch.uint8).pin_memory()
 
     def buffer_set(self):
-        """Another set of per-step device inputs and outputs (same shapes), for
-        host I/O that overlaps the neighbouring steps."""
-        ins = [TokenInputs(**{k: v.clone() for k, v in ti.t.items() if v is not None}) for ti in self.inputs]
-        return ins, [torch.empty_like(o) for o in self.outs]
+        """A set of per-step device inputs and outputs: every layer's token
+        inputs packed in one buffer and its outputs in another.  Returns
+        (input buffer, TokenInputs per layer, output buffer, output per layer)."""
+        names = [[k for k, v in x.items() if v is not None] for x in self.x]
+        in_flat, views = packed([x[k] for x, ks in zip(self.x, names) for k in ks])
+        ins, at = [], 0
+        for ks in names:
+            ins.append(TokenInputs(**dict(zip(ks, views[at:at + len(ks)]))))
+            at += len(ks)
+        out_flat, outs = packed(self.outs)
+        return in_flat, ins, out_flat, outs
 
     def step(self, pos=None, bufs=None):
         """CSA layer on the current stream, HCA layer on a side stream (the two
@@ -229,9 +253,7 @@ class DecodeBench:
         cur.wait_event(self.join)
 
     def e2e_bytes(self):
-        hi = sum(h.numel() * h.element_size() for d in self.host_in for h in d.values())
-        ho = sum(h.numel() * h.element_size() for h in self.host_out)
-        return hi, ho
+        return self.host_in.numel(), self.host_out.numel()
 
     def algorithmic_bytes(self):
         """Bytes each kernel of the step must move (the HBM roofline's
@@ -296,21 +318,19 @@ def time_e2e_pipelined(b, K, W, stream):
     outputs back.  Two device buffer sets and three streams let the copies of
     neighbouring steps overlap the step, as a serving loop would; returns the
     device time per step over K steps."""
-    sets = [(b.inputs, b.outs), b.buffer_set()]
-    graphs = [capture_graph(lambda bs=bs: b.step(bufs=bs), stream) for bs in sets]
-    hout = [[torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs] for _, outs in sets]
+    sets = [(b.in_flat, b.inputs, b.out_flat, b.outs), b.buffer_set()]
+    graphs = [capture_graph(lambda bs=bs: b.step(bufs=(bs[1], bs[3])), stream) for bs in sets]
+    hout = [b.host_out, torch.empty_like(b.host_out).pin_memory()]
     s_in, s_c, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     e_in, e_done, e_out = ([torch.cuda.Event() for _ in sets] for _ in range(3))
 
     def one(i):
         k = i % 2
-        ins, outs = sets[k]
+        in_flat, _, out_flat, _ = sets[k]
         with torch.cuda.stream(s_in):
             if i >= 2:
                 s_in.wait_event(e_done[k])          # this set's previous step has read its inputs
-            for li, ti in enumerate(ins):
-                for name, h in b.host_in[li].items():
-                    ti.t[name].copy_(h, non_blocking=True)
+            in_flat.copy_(b.host_in, non_blocking=True)
             e_in[k].record(s_in)
         with torch.cuda.stream(s_c):
             s_c.wait_event(e_in[k])
@@ -320,8 +340,7 @@ def time_e2e_pipelined(b, K, W, stream):
             e_done[k].record(s_c)
         with torch.cuda.stream(s_out):
             s_out.wait_event(e_done[k])
-            for o, h in zip(outs, hout[k]):
-                h.copy_(o, non_blocking=True)
+            hout[k].copy_(out_flat, non_blocking=True)
             e_out[k].record(s_out)
 
     for i in range(W):
@@ -494,7 +513,7 @@ def cpu_cores():
 # --------------------------------------------------------------------------- main
 # DRAM bytes (read + write) per launch of the decode kernels at the 128K batch-32 workload,
 # from single ncu captures (profiles/*_b32.md); None where no capture covers the kernel as it is.
-TRAFFIC_128K = {"index_scores": 134_289_408 + 4_679_680, "topk": 4_248_576, "attend_csa": 23_249_920 + 1_536,
+TRAFFIC_128K = {"index_scores": 134_291_200 + 4_877_056, "topk": 4_248_576, "attend_csa": 23_249_920 + 1_536,
                 "attend_hca": 39_943_680 + 11_008}   # at the bench's budget of 32 CTAs
 
 

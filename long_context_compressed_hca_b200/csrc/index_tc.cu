@@ -292,8 +292,12 @@ int launch_index_scores_tc(const IndexParams &p, cudaStream_t s) {
   // every SM streams keys
   const int n_qb = (p.n_q + 1) / 2;
   const int tiles = (Vmax + kRowsA - 1) / kRowsA;
-  // two resident blocks per SM: stay within one wave
-  const long long want = 2LL * num_sms();
+  // two resident blocks per SM.  With many query pairs, four waves of them: units
+  // small enough for the grid to balance over the SMs that another stream's
+  // kernels leave free (32 sequences in the two-layer decode step, the other
+  // layer's attention beside it: one wave 112 us per step, four waves 106 us).
+  // With few (4 sequences at 1M entries) one wave, which measured faster there.
+  const long long want = ((long long)p.B * n_qb >= 16 ? 8LL : 2LL) * num_sms();
   int units = (int)(want / ((long long)p.B * n_qb));
   if (units > tiles) units = tiles;
   if (units < 1) units = 1;
