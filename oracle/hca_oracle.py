@@ -27,7 +27,10 @@ Readings taken where the pages are silent or disagree:
   * top-k keeps min(k, V_t) entries, ties to the lower index, output in
     ascending index order, -1 padding ([J] Eq.(17), [Z] Indexer);
   * the Hadamard rotation of indexer q/k is orthonormal and omitted; no FP4
-    simulation; no intermediate rounding (exact arithmetic).
+    simulation; no intermediate rounding (exact arithmetic);
+  * mixed-precision KV rows: e4m3 codes with one fp32 scale (block amax / 448)
+    per 64 non-RoPE channels, decided in fp32, all-zero blocks with scale 0;
+    the RoPE channels in bf16 (nearest, ties to even).
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, brute force and invariants (no page prints a worked example).
@@ -414,3 +417,63 @@ def e4m3_encode(x) -> np.ndarray:
     pick_hi = (dhi < dlo) | ((dhi == dlo) & ((codes[hi] & 1) == 0))
     out = np.where(pick_hi, codes[hi], codes[lo])
     return out.astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# mixed-precision KV rows ([J] §2.3.4 效率对比: RoPE dims kept in BF16, the
+# other dims in FP8, which nearly halves the KV cache; [Z] "Q, K, V 映射与位置
+# 编码注入" and the Compressor: after RoPE, the non-RoPE dims of every KV row
+# are quantised to FP8 in blocks of 64 channels)
+# ---------------------------------------------------------------------------
+KV_FP8_BLOCK = 64
+
+
+def bf16_encode(x) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even); returns
+    the bit patterns (uint16).  From the format: 8 significant bits, exponent
+    range of fp32 (subnormal spacing 2^-133), overflow to infinity."""
+    x = np.asarray(x, np.float64)
+    m, e = np.frexp(x)                                    # x = m * 2^e, 0.5 <= |m| < 1
+    q = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)         # 8 significant bits, ties to even
+    sub = np.ldexp(np.rint(np.ldexp(x, 133)), -133)      # below 2^-126: fixed spacing 2^-133
+    q = np.where(np.abs(x) < 2.0 ** -126, sub, q)
+    q = np.where(np.abs(q) >= 2.0 ** 128, np.copysign(np.inf, x), q)
+    with np.errstate(over="ignore"):
+        f = q.astype(np.float32)                         # exact: q has at most 8 significant bits
+    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+def kv_row_quant(row, rd: int, block: int = KV_FP8_BLOCK):
+    """Store KV rows (last axis = c channels) in the mixed format.
+
+    The first c - rd channels, in blocks of `block`: scale = block amax / 448
+    and code = e4m3(x / scale), so the block's largest magnitude maps to 448;
+    these decisions are taken in fp32 (the row rounded to fp32, the scale and
+    the quotient each rounded to fp32, then nearest e4m3 with ties to even);
+    an all-zero block gets scale 0 and codes 0.  The last rd (RoPE) channels:
+    bf16, nearest with ties to even.  Returns (codes uint8 [..., c-rd],
+    scales float32 [..., (c-rd)/block], rope bf16 bits uint16 [..., rd])."""
+    x = np.asarray(row, np.float64)
+    c = x.shape[-1]
+    nq = c - rd
+    assert nq >= 0 and nq % block == 0, "c - rd must be a multiple of the block"
+    xb = x[..., :nq].astype(np.float32).reshape(*x.shape[:-1], nq // block, block)
+    amax = np.abs(xb).max(axis=-1, keepdims=True)
+    scale = (amax / np.float32(448.0)).astype(np.float32)
+    quot = (xb / np.where(scale > 0, scale, np.float32(1.0))).astype(np.float32)
+    codes = e4m3_encode(quot.astype(np.float64)).reshape(*x.shape[:-1], nq)
+    return codes, scale[..., 0], bf16_encode(x[..., nq:])
+
+
+def kv_row_dequant(codes, scales, rope_bits, block: int = KV_FP8_BLOCK) -> np.ndarray:
+    """The float64 KV rows a reader of the mixed format sees: each fp8 code
+    times its block's scale, then the bf16 RoPE channels."""
+    v = e4m3_to_f64(codes)
+    sc = np.repeat(np.asarray(scales, np.float64), block, axis=-1)
+    return np.concatenate([v * sc, bf16_bits_to_f64(rope_bits)], axis=-1)
+
+
+def mixed_kv_row_bytes(c: int, rd: int, block: int = KV_FP8_BLOCK) -> int:
+    """Bytes one row occupies in the mixed format: fp8 codes, fp32 block
+    scales and bf16 RoPE channels."""
+    return (c - rd) + 4 * ((c - rd) // block) + 2 * rd

@@ -440,3 +440,77 @@ def test_output_projection_identity_weights_flatten():
     wo_a = np.stack([np.eye(w)] * g)
     wo_b = np.eye(g * w)
     np.testing.assert_allclose(O.output_projection(o, wo_a, wo_b, g), o.reshape(-1), rtol=0, atol=0)
+
+
+# ----------------------------------------------------------------- mixed-precision KV rows
+
+def test_bf16_encode_matches_torch_and_hand_ties():
+    # float32 inputs: torch's float32 -> bf16 conversion is nearest, ties to even
+    x = (torch.randn(20000) * torch.exp2(torch.randint(-30, 30, (20000,)).float())).float()
+    ref = synth.bf16_bits(x.to(torch.bfloat16)).numpy()
+    np.testing.assert_array_equal(O.bf16_encode(x.double().numpy()).astype(np.int64), ref)
+    # ties by hand: 1 + 2^-8 lies halfway between 1 (even) and 1 + 2^-7 (odd);
+    # 1 + 3*2^-8 halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even)
+    assert O.bf16_encode(1 + 2 ** -8) == 0x3F80
+    assert O.bf16_encode(1 + 3 * 2 ** -8) == 0x3F82
+    assert O.bf16_encode(-(1 + 2 ** -8 + 2 ** -40)) == 0xBF81        # just above the tie
+    assert O.bf16_encode(2.0 ** -133) == 0x0001 and O.bf16_encode(3.5e38) == 0x7F80
+
+
+def test_kv_quant_exact_on_the_grid():
+    """Rows built from e4m3 values times a power-of-two scale, each block
+    holding +-448, with bf16-exact RoPE channels, come back bit for bit."""
+    c, rd = 512, 64
+    codes = rng.integers(0, 0x7E, size=(5, c - rd))
+    codes[:, ::64] = 0x7E                                   # every block's amax is 448
+    sign = np.where(rng.random((5, c - rd)) < 0.5, -1.0, 1.0)
+    scale = 2.0 ** rng.integers(-8, 4, size=(5, (c - rd) // 64))
+    x = sign * O.e4m3_to_f64(codes) * np.repeat(scale, 64, axis=1)
+    rope = O.bf16_bits_to_f64(O.bf16_encode(rng.standard_normal((5, rd))))
+    row = np.concatenate([x, rope], axis=1)
+    q, s, r = O.kv_row_quant(row, rd)
+    np.testing.assert_array_equal(s, scale)
+    np.testing.assert_array_equal(O.kv_row_dequant(q, s, r), row)
+
+
+def test_kv_quant_error_bound_and_block_amax():
+    """e4m3 keeps 3 mantissa bits: a normal value is within 2^-4 of itself
+    relative, a subnormal one within half the spacing 2^-9 (times the scale);
+    the block's largest magnitude maps to 448 exactly."""
+    c, rd = 512, 64
+    row = rng.standard_normal((64, c)) * np.exp(rng.uniform(-6, 6, size=(64, 1)))
+    q, s, r = O.kv_row_quant(row, rd)
+    d = O.kv_row_dequant(q, s, r)
+    x32 = row[:, :c - rd].astype(np.float32).astype(np.float64)
+    sc = np.repeat(s.astype(np.float64), 64, axis=1)
+    err = np.abs(d[:, :c - rd] - x32)
+    assert (err <= 2.0 ** -4 * np.abs(x32) * (1 + 2 ** -20) + sc * 2.0 ** -10).all()
+    blocks = np.abs(x32).reshape(64, -1, 64)
+    at = blocks.argmax(axis=2)
+    top = np.take_along_axis(q.reshape(64, -1, 64), at[..., None], axis=2)[..., 0]
+    assert ((top & 0x7F) == 0x7E).all()
+    # RoPE channels: exactly the bf16 rounding
+    np.testing.assert_array_equal(r, O.bf16_encode(row[:, c - rd:]))
+
+
+def test_kv_quant_blocks_are_independent_and_zero_blocks():
+    c, rd = 256, 64
+    row = rng.standard_normal(c)
+    row[64:128] = 0.0                                       # an all-zero block
+    q, s, r = O.kv_row_quant(row, rd)
+    assert s[1] == 0 and (q[64:128] == 0).all()
+    np.testing.assert_array_equal(O.kv_row_dequant(q, s, r)[64:128], 0.0)
+    row2 = row.copy()
+    row2[130] *= 7.0                                        # touches block 2 only
+    q2, s2, r2 = O.kv_row_quant(row2, rd)
+    np.testing.assert_array_equal(np.delete(q2, np.s_[128:192]), np.delete(q, np.s_[128:192]))
+    np.testing.assert_array_equal(np.delete(s2, 2), np.delete(s, 2))
+    assert s2[2] != s[2]
+    np.testing.assert_array_equal(r2, r)
+
+
+def test_mixed_kv_row_bytes_nearly_halve_the_cache():
+    """[J] §2.3.4: BF16 RoPE dims + FP8 for the rest nearly halves the KV
+    cache: 448 fp8 bytes + 7 fp32 scales + 64 bf16 values = 604 of 1024."""
+    assert O.mixed_kv_row_bytes(512, 64) == 448 + 28 + 128 == 604
+    assert 0.5 < O.mixed_kv_row_bytes(512, 64) / (512 * 2) < 0.6
