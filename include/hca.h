@@ -305,6 +305,33 @@ long long hca_launch_count(void);
 int hca_profile_enable(int on);
 int hca_profile_sample(void);
 int hca_profile_collect(char *buf, size_t len);
+/* ------------------------------------------------------------------------
+ * Mixed-precision KV rows, [J] §2.3.4 (the KV cache keeps the RoPE dims in
+ * BF16 and the other dims in FP8, nearly halving it); [Z] "Q, K, V 映射与位置
+ * 编码注入" and Compressor (after RoPE, the non-RoPE dims of each KV row are
+ * quantised to FP8 in blocks of 64 channels).
+ *
+ * Record of one row, hca_kv_mixed_row_bytes(c, rd) bytes (a multiple of 16):
+ *   bytes [0, c-rd)                 e4m3 codes of channels 0 .. c-rd-1
+ *   bytes [c-rd, c+rd)              channels c-rd .. c-1 (the RoPE dims) as bf16
+ *   bytes [c+rd, c+rd+(c-rd)/16)    one fp32 scale per 64 code channels
+ *   then zero bytes up to the record size (c = 512, rd = 64: 604 -> 608 bytes).
+ * Block scale = block amax / 448 and code = nearest e4m3 (ties to even,
+ * saturating) of x / scale, both divisions rounded to fp32; zero is stored
+ * as +0 and an all-zero block gets scale 0.  Shapes: c <= 512, rd a multiple
+ * of 16, c - rd a multiple of 64.  Inputs must be finite.
+ * ---------------------------------------------------------------------- */
+/* Record bytes of one row; 0 when (c, rd) is unsupported. */
+size_t hca_kv_mixed_row_bytes(int c, int rd);
+/* x: [rows, c] HCA_F32 or HCA_BF16 rows (row stride c, 16-byte aligned);
+ * out: rows consecutive records (16-byte aligned, caller-owned).  rows = 0
+ * is a no-op.  HCA_ERR_INVALID for a bad shape, dtype or pointer. */
+int hca_kv_quant_mixed(const void *x, hca_dtype x_dtype, long long rows, int c, int rd, void *out,
+                       hca_stream_t stream);
+/* in: rows records; out: [rows, c] bf16 rows, each code channel
+ * bf16(fp32(code * scale)) (nearest, ties to even), the RoPE channels copied. */
+int hca_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, hca_stream_t stream);
+
 /* Diagnostic trace of the tensor-core attention kernel: with enable = 1 the
  * following attend launches accumulate, summed over CTAs, the SM cycles each
  * role spends waiting on each pipeline barrier, plus unit / tile / rescale

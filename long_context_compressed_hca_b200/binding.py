@@ -98,6 +98,9 @@ def _declare(L):
         "hca_output_projection": (I, [C.POINTER(OprojDesc), VP, VP, VP, VP, VP, SZ, VP]),
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
+        "hca_kv_mixed_row_bytes": (SZ, [I, I]),
+        "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
+        "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -296,6 +299,19 @@ def oproj_desc(T, n_h, c, g, d_g, d, dtype=HCA_BF16, out_dtype=HCA_F32) -> Oproj
 
 def output_projection_workspace_size(d: OprojDesc) -> int:
     return lib().hca_output_projection_workspace_size(C.byref(d))
+
+
+def kv_mixed_row_bytes(c, rd) -> int:
+    """Bytes of one row record in the mixed-precision KV format (0 = unsupported)."""
+    return lib().hca_kv_mixed_row_bytes(c, rd)
+
+
+def kv_quant_mixed(x, x_dtype, rows, c, rd, out, stream=None):
+    return check(lib().hca_kv_quant_mixed(ptr(x), x_dtype, rows, c, rd, ptr(out), stream_handle(stream)))
+
+
+def kv_dequant_mixed(inp, rows, c, rd, out, stream=None):
+    return check(lib().hca_kv_dequant_mixed(ptr(inp), rows, c, rd, ptr(out), stream_handle(stream)))
 
 
 def output_projection(d: OprojDesc, o, wo_a, wo_b, out, ws, stream=None):

@@ -434,6 +434,31 @@ int hca_output_projection(const hca_oproj_desc *d, const void *o, const void *wo
   return launch_gemm(d->dtype, mid, mid_n, wo_b, mid_n, out, d->d, d->out_dtype, d->T, d->d, mid_n, 1.f, s);
 }
 
+// ------------------------------------------------------ mixed-precision KV
+size_t hca_kv_mixed_row_bytes(int c, int rd) { return kv_mixed_row_bytes(c, rd); }
+
+int hca_kv_quant_mixed(const void *x, hca_dtype x_dtype, long long rows, int c, int rd, void *out,
+                       hca_stream_t stream) {
+  REQUIRE(kv_mixed_row_bytes(c, rd) > 0, "unsupported (c, rd) = (%d, %d): need c <= 512, rd %% 16 == 0, "
+          "(c - rd) %% 64 == 0", c, rd);
+  REQUIRE(rows >= 0, "rows must be >= 0");
+  REQUIRE(x_dtype == HCA_F32 || x_dtype == HCA_BF16, "x_dtype must be HCA_F32 or HCA_BF16");
+  if (rows == 0) return HCA_OK;
+  REQUIRE(x && out, "x and out must be non-null");
+  REQUIRE(aligned16(x) && aligned16(out), "x and out must be 16-byte aligned");
+  return launch_kv_quant_mixed(x, x_dtype, rows, c, rd, out, static_cast<cudaStream_t>(stream));
+}
+
+int hca_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, hca_stream_t stream) {
+  REQUIRE(kv_mixed_row_bytes(c, rd) > 0, "unsupported (c, rd) = (%d, %d): need c <= 512, rd %% 16 == 0, "
+          "(c - rd) %% 64 == 0", c, rd);
+  REQUIRE(rows >= 0, "rows must be >= 0");
+  if (rows == 0) return HCA_OK;
+  REQUIRE(in && out, "in and out must be non-null");
+  REQUIRE(aligned16(in) && aligned16(out), "in and out must be 16-byte aligned");
+  return launch_kv_dequant_mixed(in, rows, c, rd, out, static_cast<cudaStream_t>(stream));
+}
+
 // ----------------------------------------------------------------- attend
 size_t csa_attend_workspace_size(const hca_attn_desc *d, int n_q, int start_pos) {
   if (!d) return 0;

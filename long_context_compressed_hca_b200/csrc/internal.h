@@ -109,6 +109,12 @@ int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long 
 int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
                           cudaStream_t s);
 
+// ------------------------------------------------------- mixed-precision KV
+// Record bytes of one row (0 for unsupported shapes) and the two HBM streams.
+size_t kv_mixed_row_bytes(int c, int rd);
+int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, int rd, void *out, cudaStream_t s);
+int launch_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, cudaStream_t s);
+
 // ------------------------------------------------------------- attention
 struct AttendParams {
   int B, n_q, start_pos, n_h, c, rd, w, m, k, cap;

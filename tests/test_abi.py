@@ -90,3 +90,17 @@ def test_layer_rejects_bad_arguments(L):
     lay.sink = 16
     _bad(L.hybrid_layer_forward(ctypes.byref(lay), 16, 8, None, 16, 16, 1 << 20, None), "missing layer weight")
     assert L.hybrid_layer_forward_workspace_size(ctypes.byref(lay), 64) > 0
+
+
+def test_kv_mixed_sizes_and_rejections(L):
+    assert L.hca_kv_mixed_row_bytes(512, 64) == 608          # 448 + 128 + 28 = 604, padded to 16
+    assert L.hca_kv_mixed_row_bytes(128, 64) == 208          # 64 + 128 + 4 = 196 -> 208
+    for c, rd in ((512, 60), (640, 64), (512, 32), (64, 80)):
+        assert L.hca_kv_mixed_row_bytes(c, rd) == 0, (c, rd)
+    _bad(L.hca_kv_quant_mixed(16, hb.HCA_BF16, 4, 512, 32, 16, None), "unsupported")
+    _bad(L.hca_kv_quant_mixed(16, hb.HCA_FP8E4M3, 4, 512, 64, 16, None), "x_dtype")
+    _bad(L.hca_kv_quant_mixed(16, hb.HCA_BF16, -1, 512, 64, 16, None), "rows")
+    _bad(L.hca_kv_quant_mixed(24, hb.HCA_BF16, 4, 512, 64, 16, None), "aligned")
+    _bad(L.hca_kv_quant_mixed(None, hb.HCA_BF16, 4, 512, 64, 16, None), "non-null")
+    _bad(L.hca_kv_dequant_mixed(16, 4, 512, 64, 40, None), "aligned")
+    assert L.hca_kv_dequant_mixed(None, 0, 512, 64, None, None) == hb.HCA_OK   # empty call
