@@ -30,7 +30,10 @@ Readings taken where the pages are silent or disagree:
     simulation; no intermediate rounding (exact arithmetic);
   * mixed-precision KV rows: e4m3 codes with one fp32 scale (block amax / 448)
     per 64 non-RoPE channels, decided in fp32, all-zero blocks with scale 0;
-    the RoPE channels in bf16 (nearest, ties to even).
+    the RoPE channels in bf16 (nearest, ties to even);
+  * FP4 indexer path: orthonormal Sylvester-Hadamard rotation, E2M1 (ties to
+    even, saturating at 6) with one power-of-two scale 2^(floor(log2 amax)-2)
+    per 32 values, scores rounded to bf16 before the selection.
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, brute force and invariants (no page prints a worked example).
@@ -477,3 +480,87 @@ def mixed_kv_row_bytes(c: int, rd: int, block: int = KV_FP8_BLOCK) -> int:
     """Bytes one row occupies in the mixed format: fp8 codes, fp32 block
     scales and bf16 RoPE channels."""
     return (c - rd) + 4 * ((c - rd) // block) + 2 * rd
+
+
+# ---------------------------------------------------------------------------
+# FP4 indexer path ([J] §4.4 FP4 量化感知训练: the CSA indexer's QK activations
+# are cached, loaded and multiplied in FP4, FP4 (E2M1) sub-blocks of 1 x 32
+# carry fine-grained scales that FP8's two extra exponent bits absorb, so FP4
+# -> FP8 dequantisation is lossless; the index scores go from FP32 to BF16.
+# [Z] Indexer and its Compressor: q and the compressed keys are rotated by a
+# Hadamard transform (rotate_activation) before the FP4 simulation)
+# ---------------------------------------------------------------------------
+FP4_BLOCK = 32
+E2M1_MAGNITUDES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def hadamard(n: int) -> np.ndarray:
+    """The n x n Sylvester-Hadamard matrix scaled by n^-1/2 (orthonormal and
+    symmetric); n a power of two."""
+    assert n >= 1 and n & (n - 1) == 0
+    h = np.ones((1, 1))
+    while h.shape[0] < n:
+        h = np.block([[h, h], [h, -h]])
+    return h / np.sqrt(n)
+
+
+def hadamard_rotate(x) -> np.ndarray:
+    """Rotate the last axis by the orthonormal Hadamard matrix."""
+    x = np.asarray(x, np.float64)
+    return x @ hadamard(x.shape[-1])
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """Nearest FP4 E2M1 value (sign, 2 exponent bits with bias 1, 1 mantissa
+    bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even mantissa,
+    saturating at +-6; returns the 4-bit codes (sign in bit 3)."""
+    x = np.asarray(x, np.float64)
+    a = np.minimum(np.abs(x), 6.0)
+    hi = np.clip(np.searchsorted(E2M1_MAGNITUDES, a, side="left"), 0, 7)
+    lo = np.clip(hi - 1, 0, 7)
+    dlo, dhi = a - E2M1_MAGNITUDES[lo], E2M1_MAGNITUDES[hi] - a
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & ((hi & 1) == 0))   # code parity = mantissa bit
+    mag = np.where(pick_hi, hi, lo)
+    return (np.where((x < 0) & (mag > 0), 8, 0) + mag).astype(np.uint8)
+
+
+def e2m1_to_f64(codes) -> np.ndarray:
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    return np.where(c & 8, -1.0, 1.0) * E2M1_MAGNITUDES[c & 7]
+
+
+def fp4_block_quant(x, block: int = FP4_BLOCK):
+    """FP4 with one power-of-two scale per `block` consecutive values of the
+    last axis (the OCP MX layout, reading of "1 x 32 sub-blocks whose scales
+    FP8 absorbs losslessly"): scale = 2^(floor(log2 amax) - 2), so the block's
+    largest magnitude lands in [4, 8) before rounding, codes = E2M1 of
+    x / scale; an all-zero block gets scale 1.  Returns (codes [...], scale
+    exponents int [..., n/block])."""
+    x = np.asarray(x, np.float64)
+    n = x.shape[-1]
+    assert n % block == 0
+    xb = x.reshape(*x.shape[:-1], n // block, block)
+    amax = np.abs(xb).max(axis=-1)
+    e = np.where(amax > 0, np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - 2, 0).astype(np.int64)
+    codes = e2m1_encode(xb / np.ldexp(1.0, e)[..., None])
+    return codes.reshape(x.shape), e
+
+
+def fp4_block_dequant(codes, exps, block: int = FP4_BLOCK) -> np.ndarray:
+    v = e2m1_to_f64(codes)
+    return v * np.repeat(np.ldexp(1.0, np.asarray(exps)), block, axis=-1)
+
+
+def fp4_simulate(x, block: int = FP4_BLOCK) -> np.ndarray:
+    """Quantise to FP4 blocks and back (the indexer's FP4 simulation)."""
+    c, e = fp4_block_quant(x, block)
+    return fp4_block_dequant(c, e, block)
+
+
+def index_scores_fp4(qI_t, w_t, KI, V: int) -> np.ndarray:
+    """Index scores on the FP4 path: q^I and K^I rotated by the Hadamard
+    transform and FP4-simulated, Eq.(16) over them, the result rounded to
+    BF16 (the top-k then runs on the BF16 scores, ties to the lower index)."""
+    qr = fp4_simulate(hadamard_rotate(qI_t))
+    kr = fp4_simulate(hadamard_rotate(np.asarray(KI, np.float64)[:V]))
+    return bf16_bits_to_f64(bf16_encode(index_scores(qr, w_t, kr, V)))

@@ -514,3 +514,84 @@ def test_mixed_kv_row_bytes_nearly_halve_the_cache():
     cache: 448 fp8 bytes + 7 fp32 scales + 64 bf16 values = 604 of 1024."""
     assert O.mixed_kv_row_bytes(512, 64) == 448 + 28 + 128 == 604
     assert 0.5 < O.mixed_kv_row_bytes(512, 64) / (512 * 2) < 0.6
+
+
+# ----------------------------------------------------------------- FP4 indexer path
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 64, 128])
+def test_hadamard_orthonormal_symmetric(n):
+    h = O.hadamard(n)
+    np.testing.assert_allclose(h @ h.T, np.eye(n), atol=1e-12)
+    np.testing.assert_array_equal(h, h.T)
+    assert np.all(np.abs(np.abs(h) - n ** -0.5) < 1e-15)
+
+
+def test_hadamard_rotation_closed_form_and_dot_products():
+    a, b = 3.0, -1.25
+    np.testing.assert_allclose(O.hadamard_rotate([a, b]), [(a + b) / 2 ** 0.5, (a - b) / 2 ** 0.5])
+    q, k = rng.standard_normal((5, 64)), rng.standard_normal((7, 64))
+    np.testing.assert_allclose(O.hadamard_rotate(q) @ O.hadamard_rotate(k).T, q @ k.T, atol=1e-11)
+    # the exact index scores do not see the rotation
+    w = rng.standard_normal(5)
+    np.testing.assert_allclose(O.index_scores(O.hadamard_rotate(q), w, O.hadamard_rotate(k), 7),
+                               O.index_scores(q, w, k, 7), atol=1e-11)
+
+
+def test_e2m1_table_ties_and_saturation():
+    np.testing.assert_array_equal(O.e2m1_to_f64(np.arange(16)),
+                                  [0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+    # halfway cases go to the even mantissa (code bit 0 clear)
+    ties = {0.25: 0.0, 0.75: 1.0, 1.25: 1.0, 1.75: 2.0, 2.5: 2.0, 3.5: 4.0, 5.0: 4.0}
+    for x, want in ties.items():
+        assert O.e2m1_to_f64(O.e2m1_encode(x)) == want, x
+        assert O.e2m1_to_f64(O.e2m1_encode(-x)) == -want, -x
+    assert O.e2m1_to_f64(O.e2m1_encode(7.9)) == 6.0 and O.e2m1_to_f64(O.e2m1_encode(-1e9)) == -6.0
+    # round trip of every non-negative-zero code, and nearest by brute force
+    codes = np.array([c for c in range(16) if c != 8])
+    np.testing.assert_array_equal(O.e2m1_encode(O.e2m1_to_f64(codes)), codes)
+    x = rng.uniform(-6, 6, 5000)
+    got = O.e2m1_to_f64(O.e2m1_encode(x))
+    vals = np.unique(O.e2m1_to_f64(np.arange(16)))
+    best = np.abs(x[:, None] - vals[None]).min(axis=1)
+    np.testing.assert_allclose(np.abs(got - x), best, atol=0)
+
+
+def test_fp4_into_e4m3_is_lossless():
+    """[J] §4.4: FP8 (E4M3) has two more exponent bits, so FP4 values times
+    their power-of-two block scales are E4M3 values (within E4M3's range)."""
+    for k in range(-7, 7):
+        v = O.e2m1_to_f64(np.arange(16)) * 2.0 ** k
+        v = v[np.abs(v) <= 448]
+        np.testing.assert_array_equal(O.e4m3_to_f64(O.e4m3_encode(v)), v)
+
+
+def test_fp4_block_quant_scale_grid_and_error():
+    x = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-5, 5, (16, 1)))
+    codes, e = O.fp4_block_quant(x)
+    amax = np.abs(x.reshape(16, 4, 32)).max(axis=-1)
+    r = amax / np.ldexp(1.0, e)
+    assert np.all((r >= 4) & (r < 8))
+    xh = O.fp4_block_dequant(codes, e)
+    s = np.repeat(np.ldexp(1.0, e), 32, axis=1)
+    assert np.all(np.abs(xh - x) <= 2 * s)                           # saturation region (6, 8)
+    inside = np.abs(x) <= 6 * s
+    assert np.all(np.abs(xh - x)[inside] <= s[inside])              # half the widest spacing (2)
+    # values on the grid come back exactly; an all-zero block stays zero
+    g = O.e2m1_to_f64(rng.integers(0, 16, (3, 64))) * 2.0 ** 3
+    g[:, ::32] = 6 * 2.0 ** 3
+    np.testing.assert_array_equal(O.fp4_simulate(g), g)
+    z = np.zeros((1, 32))
+    np.testing.assert_array_equal(O.fp4_simulate(z), z)
+
+
+def test_index_scores_fp4_bf16_and_power_of_two_scaling():
+    q, k = rng.standard_normal((8, 64)), rng.standard_normal((40, 64))
+    w = np.abs(rng.standard_normal(8)) * 0.05
+    sc = O.index_scores_fp4(q, w, k, 40)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(O.bf16_encode(sc)), sc)   # BF16 values
+    # FP4 block scales are powers of two and BF16 rounding is scale-free: scaling
+    # q by 2^j scales every score by 2^j exactly
+    np.testing.assert_array_equal(O.index_scores_fp4(4 * q, w, k, 40), 4 * sc)
+    # the FP4 path stays close to the exact scores on this data
+    ex = O.index_scores(q, w, k, 40)
+    assert np.abs(sc - ex).max() <= 0.25 * np.abs(ex).max()
