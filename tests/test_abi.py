@@ -104,3 +104,27 @@ def test_kv_mixed_sizes_and_rejections(L):
     _bad(L.hca_kv_quant_mixed(None, hb.HCA_BF16, 4, 512, 64, 16, None), "non-null")
     _bad(L.hca_kv_dequant_mixed(16, 4, 512, 64, 40, None), "aligned")
     assert L.hca_kv_dequant_mixed(None, 0, 512, 64, None, None) == hb.HCA_OK   # empty call
+
+
+def test_attention_cta_budget_sets_the_split_plan(L):
+    """The CTA budget bounds the split-KV count per query, visible here through
+    the workspace a call needs: splits beyond 8 go through an fp32 workspace
+    of q * splits * 64 rows of c floats (+ 64 (max, sum) pairs each); up to 8
+    merge inside a thread-block cluster and need none.  4 sequences at the 1M
+    position: HCA has 130 key tiles per query, CSA (k = 1024) 18."""
+    def ws(kind, max_ctas):
+        k = 1024 if kind == "csa" else 0
+        m = 4 if kind == "csa" else 128
+        d = hb.attn_desc(4, 64, 512, 64, 128, m, k=k, dtype=hb.HCA_BF16, max_ctas=max_ctas)
+        f = L.csa_attend_workspace_size if kind == "csa" else L.hca_attend_workspace_size
+        return f(ctypes.byref(d), 1, 1048576)
+
+    def split_ws(ns, q=4, c=512):
+        return q * ns * 64 * c * 4 + q * ns * 64 * 8
+    sms = 148
+    assert ws("hca", 0) == split_ws(min(sms // 4, 65, 32))       # 32 splits
+    assert ws("hca", 64) == split_ws(16)
+    assert ws("hca", 32) == 0                                    # 8 splits: cluster merge
+    assert ws("hca", 4) == 0                                     # 1 split
+    assert ws("csa", 0) == split_ws(9)                           # 18 tiles -> 9 splits
+    assert ws("csa", 32) == 0
