@@ -8,7 +8,8 @@
  * Sources of the operations (page title, section / equation):
  *   [J] juejin "DeepSeek-V4 技术报告简要解读": §2.3.1 Eq.(9)-(19) (CSA),
  *       §2.3.2 Eq.(20)-(23) (HCA), §2.3.3 (QK norm, partial RoPE, window,
- *       sink Eq.(27)), §4.6 (heterogeneous KV cache).
+ *       sink Eq.(27)), §2.3.4 (mixed-precision KV storage), §4.4 (FP4
+ *       indexer path, deferred), §4.6 (heterogeneous KV cache).
  *   [Z] 1zeryu "DeepSeek-V4：算法架构": "Q, K, V 映射与位置编码注入",
  *       "Sparse Attention", "CSA 选择器层代码实现" (Compressor, Indexer),
  *       "HCA 选择函数代码实现", "输出投影".
