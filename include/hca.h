@@ -52,7 +52,7 @@ typedef void *hca_stream_t; /* cudaStream_t */
 enum {
   HCA_OK = 0,
   HCA_ERR_INVALID = -1,     /* bad shape, null / misaligned pointer, bad dtype */
-  HCA_ERR_UNSUPPORTED = -2, /* valid request this build does not implement */
+  HCA_ERR_UNSUPPORTED = -2, /* valid request the library does not implement */
   HCA_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch, attribute) */
   HCA_ERR_TIMEOUT = -4      /* a bounded device wait expired */
 };
