@@ -431,6 +431,25 @@ def test_output_projection_group_permutation_invariance():
     assert not np.allclose(O.output_projection(o_p, wo_a, wo_b, g), base)
 
 
+def test_output_projection_hand_example():
+    """Two heads of one channel, two groups of one output each, a square wo_b
+    (so a transposed operand would still fit): mid = (a p, b q), out = wo_b mid."""
+    a, b, p, q = 2.0, -3.0, 5.0, 7.0
+    o = np.array([[a], [b]])
+    wo_a = np.array([[[p]], [[q]]])
+    wo_b = np.array([[1.0, 2.0], [3.0, 4.0]])
+    np.testing.assert_array_equal(O.output_projection(o, wo_a, wo_b, 2),
+                                  [a * p + 2 * b * q, 3 * a * p + 4 * b * q])
+
+
+def test_window_positions_hand_table():
+    """Reading 10: the window of query t is tokens max(0, t-w+1) .. t, its own
+    token included (w rows once t >= w-1)."""
+    table = {(5, 3): [3, 4, 5], (1, 3): [0, 1], (0, 1): [0], (7, 1): [7], (4, 0): []}
+    for (t, w), want in table.items():
+        np.testing.assert_array_equal(O.window_positions(t, w), want)
+
+
 def test_output_projection_identity_weights_flatten():
     """d_g = n_h*c/g with identity blocks and wo_b = I returns o flattened."""
     rng = np.random.default_rng(9)
@@ -501,7 +520,7 @@ def test_kv_quant_blocks_are_independent_and_zero_blocks():
     assert s[1] == 0 and (q[64:128] == 0).all()
     np.testing.assert_array_equal(O.kv_row_dequant(q, s, r)[64:128], 0.0)
     row2 = row.copy()
-    row2[130] *= 7.0                                        # touches block 2 only
+    row2[130] = 10.0 * np.abs(row[128:192]).max()           # block 2's new amax, no other block
     q2, s2, r2 = O.kv_row_quant(row2, rd)
     np.testing.assert_array_equal(np.delete(q2, np.s_[128:192]), np.delete(q, np.s_[128:192]))
     np.testing.assert_array_equal(np.delete(s2, 2), np.delete(s, 2))
