@@ -262,7 +262,82 @@ def oproj_wo_b_transposed(o, wo_a, wo_b, g):
     return ORIG["output_projection"](o, wo_a, wo_b.T if wo_b.shape[0] == wo_b.shape[1] else wo_b, g)
 
 
+def decode_emit_at_block_start(pos, m, cur_Ca, cur_Za, Ba, prev_Cb=None, prev_Zb=None, Bb=None):
+    if pos % m != 0:
+        return None
+    r = np.asarray(cur_Ca).shape[0]          # the rows present so far, their biases only
+    return O.compress_entry(cur_Ca, cur_Za, np.asarray(Ba)[:r], prev_Cb, prev_Zb, Bb)
+
+
+def e4m3_bias_8(bits):
+    b = np.asarray(bits).astype(np.int64) & 0xFF
+    s = np.where(b >> 7, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    f = (b & 7).astype(np.float64)
+    v = s * np.where(e == 0, np.ldexp(f / 8.0, -7), np.ldexp(1.0 + f / 8.0, (e - 8).astype(np.int64)))
+    return np.where((e == 15) & ((b & 7) == 7), np.nan, v)
+
+
+def bf16_decode_shift_15(bits):
+    b = np.asarray(bits).astype(np.uint32) << np.uint32(15)
+    return b.view(np.float32).astype(np.float64)
+
+
+def fp4_scores_keys_not_rotated(qI_t, w_t, KI, V):
+    qr = O.fp4_simulate(O.hadamard_rotate(qI_t))
+    kr = O.fp4_simulate(np.asarray(KI, np.float64)[:V])
+    return O.bf16_bits_to_f64(O.bf16_encode(O.index_scores(qr, w_t, kr, V)))
+
+
+def fp4_scores_not_rounded(qI_t, w_t, KI, V):
+    qr = O.fp4_simulate(O.hadamard_rotate(qI_t))
+    kr = O.fp4_simulate(O.hadamard_rotate(np.asarray(KI, np.float64)[:V]))
+    return O.index_scores(qr, w_t, kr, V)
+
+
+def fp4_blocks_of_16(x, block=32):
+    return ORIG["fp4_block_quant"](x, 16)
+
+
+def kv_quant_blocks_of_32(row, rd, block=64):
+    return ORIG["kv_row_quant"](row, rd, 32)
+
+
+def topk_pads_with_low_scores(scores, k):
+    # keeps k entries even when fewer are visible (indices past the visible set)
+    s = np.asarray(scores, np.float64)
+    V = s.shape[0]
+    order = np.lexsort((np.arange(V), -s))
+    kept = np.sort(order[:min(k, V)])
+    out = np.arange(k, dtype=np.int32) + V
+    out[:kept.shape[0]] = kept
+    return out
+
+
+def compress_entry0_with_zero_row(Ca_blk, Za_blk, Ba, Cb_prev=None, Zb_prev=None, Bb=None):
+    # entry 0's missing b-half as a zero value with logit 0 instead of -inf
+    if Cb_prev is None and np.asarray(Ca_blk).shape[0] > 1:
+        z = np.zeros((1, np.asarray(Ca_blk).shape[1]))
+        return ORIG["compress_entry"](Ca_blk, Za_blk, Ba, z, z, np.zeros_like(z))
+    return ORIG["compress_entry"](Ca_blk, Za_blk, Ba, Cb_prev, Zb_prev, Bb)
+
+
+def e2m1_sign_bit_2(codes):
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    return np.where(c & 4, -1.0, 1.0) * O.E2M1_MAGNITUDES[c & 7]
+
+
 MUTATIONS = {
+    "decode: emission at the block start": ("decode_new_entry", decode_emit_at_block_start),
+    "e4m3: exponent bias 8": ("e4m3_to_f64", e4m3_bias_8),
+    "bf16: decoded with a 15-bit shift": ("bf16_bits_to_f64", bf16_decode_shift_15),
+    "fp4 scores: keys not rotated": ("index_scores_fp4", fp4_scores_keys_not_rotated),
+    "fp4 scores: not rounded to bf16": ("index_scores_fp4", fp4_scores_not_rounded),
+    "fp4: blocks of 16": ("fp4_block_quant", fp4_blocks_of_16),
+    "mixed KV: blocks of 32": ("kv_row_quant", kv_quant_blocks_of_32),
+    "top-k: padded with invisible entries": ("topk_select", topk_pads_with_low_scores),
+    "compress: entry 0 with a zero b row": ("compress_entry", compress_entry0_with_zero_row),
+    "e2m1: sign in bit 2": ("e2m1_to_f64", e2m1_sign_bit_2),
     "rope: rotation sign": ("rope", rope_sign),
     "rope: frequency theta^(-i/rd)": ("rope", rope_frequency),
     "rope: half-split pairs": ("rope", rope_half_split_pairs),

@@ -383,7 +383,7 @@ def test_decode_emission_equals_prefill_entries():
     Ca, Cb, Za, Zb = (rng.standard_normal((n, c)) for _ in range(4))
     Ba, Bb = rng.standard_normal((m, c)), rng.standard_normal((m, c))
     ref = O.compress_prefill(Ca, Za, Ba, m, Cb, Zb, Bb)
-    got = []
+    got, at = [], []
     for pos in range(n):
         b = pos // m
         blk = slice(b * m, pos + 1)
@@ -392,6 +392,8 @@ def test_decode_emission_equals_prefill_entries():
                                Cb[prev] if prev else None, Zb[prev] if prev else None, Bb)
         if e is not None:
             got.append(e)
+            at.append(pos)
+    assert at == list(range(m - 1, n, m))          # a block's entry appears with its last token
     np.testing.assert_allclose(np.stack(got), ref, atol=1e-14)
 
 
@@ -587,6 +589,7 @@ def test_fp4_into_e4m3_is_lossless():
 def test_fp4_block_quant_scale_grid_and_error():
     x = rng.standard_normal((16, 128)) * np.exp(rng.uniform(-5, 5, (16, 1)))
     codes, e = O.fp4_block_quant(x)
+    assert codes.shape == x.shape and e.shape == (16, 4)            # one scale per 32 values
     amax = np.abs(x.reshape(16, 4, 32)).max(axis=-1)
     r = amax / np.ldexp(1.0, e)
     assert np.all((r >= 4) & (r < 8))
