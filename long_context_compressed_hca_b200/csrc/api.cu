@@ -118,15 +118,27 @@ int encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, u
   return HCA_OK;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+int device_slot() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    (void)cudaGetLastError();
+    return 0;
   }
-  return n;
+  return dev;
+}
+
+int num_sms() {
+  static int n[kMaxDevices] = {0};
+  const int d = device_slot();
+  if (n[d] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || v <= 0) {
+      (void)cudaGetLastError();
+      v = 148;
+    }
+    n[d] = v;
+  }
+  return n[d];
 }
 
 namespace {

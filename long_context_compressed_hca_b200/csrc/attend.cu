@@ -1025,7 +1025,8 @@ attend_tc(AttendParams p, int n_units) {
 
 template <int C>
 int ensure_attr() {
-  static bool attr_set = false;
+  static bool attr_set_dev[kMaxDevices] = {false};
+  bool &attr_set = attr_set_dev[device_slot()];
   if (!attr_set) {
     const int smem = (int)Layout<C>::bytes;
     cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1040,8 +1041,9 @@ int ensure_attr() {
 // How many clusters of `ns` CTAs can be resident at once (0 if unknown).
 template <int C>
 int max_active_clusters(int ns) {
-  static int cache[kMaxClusterSplits + 1] = {0};
+  static int cache_dev[kMaxDevices][kMaxClusterSplits + 1] = {{0}};
   if (ns < 1 || ns > kMaxClusterSplits) return 0;
+  int *cache = cache_dev[device_slot()];
   if (cache[ns]) return cache[ns];
   if (ensure_attr<C>()) return 0;
   cudaLaunchConfig_t cfg{};

@@ -374,7 +374,8 @@ TopkPlan plan_topk(long long rows, long long Vmax) {
 }
 size_t topk_smem(const TopkPlan &t) { return (size_t)(t.slice + kCandMax) * 4; }
 int ensure_topk_smem() {
-  static bool done = false;
+  static bool done_dev[kMaxDevices] = {false};
+  bool &done = done_dev[device_slot()];
   if (!done) {
     const cudaError_t e = cudaFuncSetAttribute(topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (kSliceMax + kCandMax) * 4);

@@ -29,6 +29,11 @@ int fail(int code, const char *fmt, ...);
 int check_launch(const char *what);
 void count_launch(int n = 1);
 int num_sms();
+// The current device's slot in per-device caches (0 .. kMaxDevices-1; 0 when
+// the device cannot be read).  Kernel attributes, occupancy figures and the SM
+// count are cached per device, so one process may drive several devices.
+constexpr int kMaxDevices = 64;
+int device_slot();
 // Encode a 2-D tiled TMA descriptor over a row-major matrix (rows x cols
 // elements of elem_bytes, rows row_stride_bytes apart); box = box_rows x
 // box_cols elements.  Returns HCA_OK or HCA_ERR_CUDA.
