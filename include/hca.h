@@ -333,6 +333,20 @@ int hca_kv_quant_mixed(const void *x, hca_dtype x_dtype, long long rows, int c, 
  * bf16(fp32(code * scale)) (nearest, ties to even), the RoPE channels copied. */
 int hca_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, hca_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * FP4 indexer activations, [J] §4.4 (the indexer's QK activations in FP4 E2M1
+ * with scales per 1 x 32 sub-block that FP8 absorbs losslessly, i.e. powers of
+ * two); [Z] Indexer (q^I and the keys Hadamard-rotated first).
+ *
+ * x: [rows, n] HCA_F32 or HCA_BF16 (n = 64); out: [rows, n] bf16.  Each row is
+ * rotated by the orthonormal Hadamard matrix (butterflies of strides 1, 2, ...
+ * in fp32, then the exact scale n^-1/2), cut into blocks of 32 with scale
+ * 2^(floor(log2 amax) - 2), rounded to E2M1 (nearest, ties to even, saturating
+ * at 6; zero as +0) and written as bf16 -- exact, since every E2M1 value times
+ * a power of two is a bf16 value.  rows = 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+int hca_fp4_rotate_quant(const void *x, hca_dtype x_dtype, long long rows, int n, void *out, hca_stream_t stream);
+
 /* Diagnostic trace of the tensor-core attention kernel: with enable = 1 the
  * following attend launches accumulate, summed over CTAs, the SM cycles each
  * role spends waiting on each pipeline barrier, plus unit / tile / rescale

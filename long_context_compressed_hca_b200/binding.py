@@ -99,6 +99,7 @@ def _declare(L):
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
         "hca_kv_mixed_row_bytes": (SZ, [I, I]),
+        "hca_fp4_rotate_quant": (I, [VP, I, LL, I, VP, VP]),
         "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
         "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
     }
@@ -299,6 +300,10 @@ def oproj_desc(T, n_h, c, g, d_g, d, dtype=HCA_BF16, out_dtype=HCA_F32) -> Oproj
 
 def output_projection_workspace_size(d: OprojDesc) -> int:
     return lib().hca_output_projection_workspace_size(C.byref(d))
+
+
+def fp4_rotate_quant(x, x_dtype, rows, n, out, stream=None):
+    return check(lib().hca_fp4_rotate_quant(ptr(x), x_dtype, rows, n, ptr(out), stream_handle(stream)))
 
 
 def kv_mixed_row_bytes(c, rd) -> int:

@@ -446,6 +446,17 @@ int hca_output_projection(const hca_oproj_desc *d, const void *o, const void *wo
   return launch_gemm(d->dtype, mid, mid_n, wo_b, mid_n, out, d->d, d->out_dtype, d->T, d->d, mid_n, 1.f, s);
 }
 
+// ------------------------------------------------------------ FP4 indexer
+int hca_fp4_rotate_quant(const void *x, hca_dtype x_dtype, long long rows, int n, void *out, hca_stream_t stream) {
+  REQUIRE(n == 64, "n must be 64 (the indexer head dim), got %d", n);
+  REQUIRE(rows >= 0, "rows must be >= 0");
+  REQUIRE(x_dtype == HCA_F32 || x_dtype == HCA_BF16, "x_dtype must be HCA_F32 or HCA_BF16");
+  if (rows == 0) return HCA_OK;
+  REQUIRE(x && out, "x and out must be non-null");
+  REQUIRE(aligned16(x) && aligned16(out), "x and out must be 16-byte aligned");
+  return launch_fp4_rotate_quant(x, x_dtype, rows, out, static_cast<cudaStream_t>(stream));
+}
+
 // ------------------------------------------------------ mixed-precision KV
 size_t hca_kv_mixed_row_bytes(int c, int rd) { return kv_mixed_row_bytes(c, rd); }
 

@@ -114,6 +114,10 @@ int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long 
 int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
                           cudaStream_t s);
 
+// ------------------------------------------------------------ FP4 indexer
+// Rows of 64: Hadamard rotation, FP4 blocks of 32, written as exact bf16 values.
+int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s);
+
 // ------------------------------------------------------- mixed-precision KV
 // Record bytes of one row (0 for unsupported shapes) and the two HBM streams.
 size_t kv_mixed_row_bytes(int c, int rd);

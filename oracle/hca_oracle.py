@@ -564,3 +564,30 @@ def index_scores_fp4(qI_t, w_t, KI, V: int) -> np.ndarray:
     qr = fp4_simulate(hadamard_rotate(qI_t))
     kr = fp4_simulate(hadamard_rotate(np.asarray(KI, np.float64)[:V]))
     return bf16_bits_to_f64(bf16_encode(index_scores(qr, w_t, kr, V)))
+
+
+
+def hadamard_rotate_fwht32(x) -> np.ndarray:
+    """The Hadamard rotation of the last axis (a power of two) as the GPU takes
+    it, for decisions made on its result: fast Walsh-Hadamard butterflies in
+    fp32, strides 1, 2, 4, ... (lower element a, upper b: a + b, a - b, each
+    rounded to fp32), then the exact scale n^-1/2 for n = 4^j.  Equal to
+    hadamard_rotate up to fp32 rounding."""
+    y = np.array(np.asarray(x, np.float64).astype(np.float32), copy=True)
+    n = y.shape[-1]
+    assert n & (n - 1) == 0 and (n.bit_length() - 1) % 2 == 0, "n must be a power of 4"
+    s = 1
+    while s < n:
+        v = y.reshape(*y.shape[:-1], n // (2 * s), 2, s)
+        a, b = v[..., 0, :].copy(), v[..., 1, :].copy()
+        v[..., 0, :] = a + b
+        v[..., 1, :] = a - b
+        y = v.reshape(*y.shape[:-1], n)
+        s *= 2
+    return (y * np.float32(2.0 ** (-(n.bit_length() - 1) // 2))).astype(np.float64)
+
+
+def fp4_rotate_quant_gpu_order(x, block: int = FP4_BLOCK) -> np.ndarray:
+    """The FP4 values (as float64) of rows rotated in the GPU's fp32 order and
+    block-quantised: what an indexer stores for q^I / K^I on the FP4 path."""
+    return fp4_simulate(hadamard_rotate_fwht32(x), block)

@@ -128,3 +128,10 @@ def test_attention_cta_budget_sets_the_split_plan(L):
     assert ws("hca", 4) == 0                                     # 1 split
     assert ws("csa", 0) == split_ws(9)                           # 18 tiles -> 9 splits
     assert ws("csa", 32) == 0
+
+
+def test_fp4_rotate_quant_rejects_bad_arguments(L):
+    _bad(L.hca_fp4_rotate_quant(16, hb.HCA_BF16, 4, 32, 16, None), "n must be 64")
+    _bad(L.hca_fp4_rotate_quant(16, hb.HCA_FP8E4M3, 4, 64, 16, None), "x_dtype")
+    _bad(L.hca_fp4_rotate_quant(24, hb.HCA_BF16, 4, 64, 16, None), "aligned")
+    assert L.hca_fp4_rotate_quant(None, hb.HCA_BF16, 0, 64, None, None) == hb.HCA_OK

@@ -617,3 +617,24 @@ def test_index_scores_fp4_bf16_and_power_of_two_scaling():
     # the FP4 path stays close to the exact scores on this data
     ex = O.index_scores(q, w, k, 40)
     assert np.abs(sc - ex).max() <= 0.25 * np.abs(ex).max()
+
+
+def test_fwht32_matches_the_hadamard_matrix():
+    x = rng.standard_normal((50, 64)) * 10
+    np.testing.assert_allclose(O.hadamard_rotate_fwht32(x), O.hadamard_rotate(x.astype(np.float32)),
+                               rtol=0, atol=1e-5 * np.abs(x).max())
+    # small integers: every butterfly sum is exact in fp32, so the two agree exactly
+    xi = rng.integers(-50, 50, (20, 64)).astype(np.float64)
+    np.testing.assert_array_equal(O.hadamard_rotate_fwht32(xi), O.hadamard_rotate(xi))
+    # the butterfly order of the 4-point case by hand: [a+b+c+d, a-b+c-d, a+b-c-d, a-b-c+d] / 2
+    a, b, c, d = 1.0, 2.0, 4.0, 8.0
+    np.testing.assert_array_equal(O.hadamard_rotate_fwht32([a, b, c, d]),
+                                  np.array([a + b + c + d, a - b + c - d, a + b - c - d, a - b - c + d]) / 2)
+
+
+def test_fp4_rotate_quant_values_are_bf16_and_fp4():
+    x = rng.standard_normal((30, 64))
+    y = O.fp4_rotate_quant_gpu_order(x)
+    np.testing.assert_array_equal(O.bf16_bits_to_f64(O.bf16_encode(y)), y)      # exact in bf16
+    codes, e = O.fp4_block_quant(y)
+    np.testing.assert_array_equal(O.fp4_block_dequant(codes, e), y)             # already on the grid
