@@ -132,6 +132,14 @@ int csa_compress(const hca_compress_desc *d, int start_pos, int n,
                  const float *Ba, const float *Bb, const float *gamma,
                  void *out, float *out_scale, long long out_seq_stride,
                  float *state_kv, float *state_score, hca_stream_t stream);
+/* hca_compress -- the same call under the HCA name (overlap = 0, ratio m'):
+ * [J] Eq.(22)-(23); identical arguments and behaviour to csa_compress. */
+int hca_compress(const hca_compress_desc *d, int start_pos, int n,
+                 const void *Ca, const void *Cb, const void *Za, const void *Zb,
+                 long long row_stride, long long seq_stride,
+                 const float *Ba, const float *Bb, const float *gamma,
+                 void *out, float *out_scale, long long out_seq_stride,
+                 float *state_kv, float *state_score, hca_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Lightning indexer score + per-query top-k, [J] Eq.(16)-(17); [Z] Indexer.
@@ -167,6 +175,9 @@ int csa_index_topk(const hca_attn_desc *d, const void *qI, const float *wI,
  *   time (different streams or host threads without ordering between them)
  *   race on it and must be serialised by the caller. */
 #define HCA_STATIC_SCRATCH_BYTES (8u << 20)
+/* HCA_STATIC_SCRATCH_BYTES as this build of the library has it (for callers
+ * that load the library without its header, e.g. through ctypes). */
+size_t hca_static_scratch_bytes(void);
 int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const float *wI,
                                   const void *KI, const float *KI_scale, int cap, int n_q,
                                   int start_pos, int32_t *idx, float *scores, long long score_stride,
@@ -259,6 +270,27 @@ typedef struct {
 size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos);
 int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache,
                        int pos, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* Where the two calls above leave their intermediate results inside the
+ * caller's workspace, so that a caller can inspect the selection and the
+ * stored operands after the call (they stay until the workspace is reused).
+ * decode = 0 describes hybrid_layer_forward(L, ., n, ...), decode = 1
+ * hybrid_decode_step(L, ., ., pos = n, ...).  Each field is a byte offset
+ * from ws, or -1 when the call has no such buffer (another layer kind, decode,
+ * or a prefill with a cache, which stores entries and keys in the cache):
+ *   idx     [B, n_q, k] int32   kept entries (CSA), ascending, -1 padded
+ *   q       [B, n, n_h, c]      queries, normalised and RoPE'd   (a.dtype)
+ *   qI      [B, n, n_hI, c_I]   index queries, RoPE'd           (a.dtype)
+ *   wI      [B, n, n_hI] fp32   index weights (scaled)
+ *   key_I   [B, n/m, c_I]       indexer keys                     (a.dtype)
+ *   kv_comp [B, n/m, c]         compressed entries               (a.dtype)
+ *   kv_win  [B, n, c]           window rows, normalised, RoPE'd  (a.dtype)
+ * (n_q = n for prefill, 1 for decode.)  Returns HCA_ERR_INVALID for a bad
+ * layer, n < 0 (prefill) or n < 1 (decode). */
+typedef struct {
+  long long idx, q, qI, wI, key_I, kv_comp, kv_win;
+} hca_ws_map;
+int hybrid_workspace_map(const hca_layer *L, int n, int decode, hca_ws_map *map);
 
 /* ------------------------------------------------------------------------
  * Grouped output projection, [J] §2.3.1(d); [Z] 输出投影 -- the step after the

@@ -19,6 +19,8 @@ HCA_OK, HCA_ERR_INVALID, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_TIMEOUT = 0,
 HCA_F32, HCA_BF16, HCA_FP8E4M3 = 0, 1, 2
 HCA_COMPRESS_NORM, HCA_COMPRESS_ROPE = 1, 2
 HCA_LAYER_CSA, HCA_LAYER_HCA, HCA_LAYER_SWA = 0, 1, 2
+# HCA_STATIC_SCRATCH_BYTES of include/hca.h; lib() checks that the loaded library agrees.
+STATIC_SCRATCH_BYTES = 8 << 20
 
 DTYPE_CODE = {torch.float32: HCA_F32, torch.bfloat16: HCA_BF16, torch.uint8: HCA_FP8E4M3,
               torch.float8_e4m3fn: HCA_FP8E4M3}
@@ -62,6 +64,10 @@ class OprojDesc(C.Structure):
                 ("d", C.c_int), ("dtype", C.c_int), ("out_dtype", C.c_int)]
 
 
+class WsMap(C.Structure):
+    _fields_ = [(f, C.c_longlong) for f in ("idx", "q", "qI", "wI", "key_I", "kv_comp", "kv_win")]
+
+
 class TokenIn(C.Structure):
     _fields_ = [("q", C.c_void_p), ("qI", C.c_void_p), ("wI", C.c_void_p), ("kv", C.c_void_p),
                 ("comp", C.c_void_p), ("compI", C.c_void_p)]
@@ -99,6 +105,10 @@ def _declare(L):
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
         "hca_kv_mixed_row_bytes": (SZ, [I, I]),
+        "hca_static_scratch_bytes": (SZ, []),
+        "hca_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
+                             VP, LL, VP, VP, VP]),
+        "hybrid_workspace_map": (I, [C.POINTER(Layer), I, I, C.POINTER(WsMap)]),
         "hca_fp4_rotate_quant": (I, [VP, I, LL, I, VP, VP]),
         "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
         "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
@@ -119,6 +129,9 @@ def lib():
                            "`python -m long_context_compressed_hca_b200.build`")
         L = C.CDLL(LIB_PATH)
         _declare(L)
+        if L.hca_static_scratch_bytes() != STATIC_SCRATCH_BYTES:
+            raise HcaError(HCA_ERR_UNSUPPORTED, "libhca.so was built with a different static scratch size "
+                           f"({L.hca_static_scratch_bytes()} != {STATIC_SCRATCH_BYTES}): rebuild it")
         _lib = L
     return _lib
 
@@ -220,8 +233,9 @@ def compress_desc(B, width, m, overlap, rd, flags, in_dtype, out_dtype, eps=1e-6
 
 # --------------------------------------------------------------------- calls
 def csa_compress(d: CompressDesc, start_pos, n, Ca, Cb, Za, Zb, row_stride, seq_stride, Ba, Bb,
-                 gamma, out, out_scale, out_seq_stride, state_kv, state_score, stream=None):
-    return check(lib().csa_compress(C.byref(d), start_pos, n, ptr(Ca), ptr(Cb), ptr(Za), ptr(Zb),
+                 gamma, out, out_scale, out_seq_stride, state_kv, state_score, stream=None, hca_name=False):
+    fn = lib().hca_compress if hca_name else lib().csa_compress
+    return check(fn(C.byref(d), start_pos, n, ptr(Ca), ptr(Cb), ptr(Za), ptr(Zb),
                                     row_stride, seq_stride, ptr(Ba), ptr(Bb), ptr(gamma), ptr(out),
                                     ptr(out_scale), out_seq_stride, ptr(state_kv), ptr(state_score),
                                     stream_handle(stream)))
@@ -239,8 +253,9 @@ def csa_index_topk(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, 
                                       stream_handle(stream)))
 
 
-# Size of the library's fixed scratch array used by csa_index_topk_static_scratch.
-STATIC_SCRATCH_BYTES = 8 << 20
+def static_scratch_bytes() -> int:
+    """Size of the library's fixed scratch array (csa_index_topk_static_scratch)."""
+    return lib().hca_static_scratch_bytes()
 
 
 def csa_index_topk_static_scratch(d: AttnDesc, qI, wI, KI, KI_scale, cap, n_q, start_pos, idx, scores=None,
@@ -276,6 +291,24 @@ def hca_attend(d: AttnDesc, q, kv_comp, cap, kv_win, win_is_ring, sink, n_q, sta
 
 def layer_workspace_size(L: Layer, n: int) -> int:
     return lib().hybrid_layer_forward_workspace_size(C.byref(L), n)
+
+
+def workspace_map(L: Layer, n: int, decode: bool = False) -> dict:
+    """Byte offsets of the intermediates hybrid_layer_forward (decode=False,
+    n tokens) or hybrid_decode_step (decode=True, pos n) leaves in its
+    workspace; None where the call has no such buffer."""
+    m = WsMap()
+    check(lib().hybrid_workspace_map(C.byref(L), n, int(decode), C.byref(m)))
+    return {f: (getattr(m, f) if getattr(m, f) >= 0 else None) for f, _ in WsMap._fields_}
+
+
+def ws_view(ws, offset: int, shape, dtype):
+    """A tensor view of `shape` / `dtype` at byte `offset` of a uint8 workspace."""
+    n = 1
+    for x in shape:
+        n *= x
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    return ws[offset:offset + nbytes].view(dtype).view(*shape)
 
 
 def hybrid_layer_forward(L: Layer, H, n, cache: Cache | None, o, ws, stream=None):

@@ -86,7 +86,7 @@ int LaunchScope::done() {
 }
 
 int *device_status_ptr() {
-  static int *ptr[64] = {nullptr};
+  static std::atomic<int *> ptr[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return nullptr;
@@ -128,7 +128,7 @@ int device_slot() {
 }
 
 int num_sms() {
-  static int n[kMaxDevices] = {0};
+  static std::atomic<int> n[kMaxDevices];
   const int d = device_slot();
   if (n[d] == 0) {
     int v = 0;
@@ -280,7 +280,9 @@ extern "C" {
 
 const char *hca_last_error(void) { return t_err; }
 
-int hca_version(void) { return (0 << 16) | 1; }
+int hca_version(void) { return (0 << 16) | 2; }
+
+size_t hca_static_scratch_bytes(void) { return (size_t)HCA_STATIC_SCRATCH_BYTES; }
 
 long long hca_launch_count(void) { return g_launches.load(); }
 
@@ -370,6 +372,14 @@ int csa_compress(const hca_compress_desc *d, int start_pos, int n, const void *C
     return HCA_OK;
   }
   return launch_compress_decode(p, start_pos, s);
+}
+
+int hca_compress(const hca_compress_desc *d, int start_pos, int n, const void *Ca, const void *Cb,
+                 const void *Za, const void *Zb, long long row_stride, long long seq_stride,
+                 const float *Ba, const float *Bb, const float *gamma, void *out, float *out_scale,
+                 long long out_seq_stride, float *state_kv, float *state_score, hca_stream_t stream) {
+  return csa_compress(d, start_pos, n, Ca, Cb, Za, Zb, row_stride, seq_stride, Ba, Bb, gamma, out, out_scale,
+                      out_seq_stride, state_kv, state_score, stream);
 }
 
 // ----------------------------------------------------------------- index + top-k

@@ -1025,8 +1025,8 @@ attend_tc(AttendParams p, int n_units) {
 
 template <int C>
 int ensure_attr() {
-  static bool attr_set_dev[kMaxDevices] = {false};
-  bool &attr_set = attr_set_dev[device_slot()];
+  static std::atomic<bool> attr_set_dev[kMaxDevices];
+  std::atomic<bool> &attr_set = attr_set_dev[device_slot()];
   if (!attr_set) {
     const int smem = (int)Layout<C>::bytes;
     cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1041,9 +1041,9 @@ int ensure_attr() {
 // How many clusters of `ns` CTAs can be resident at once (0 if unknown).
 template <int C>
 int max_active_clusters(int ns) {
-  static int cache_dev[kMaxDevices][kMaxClusterSplits + 1] = {{0}};
+  static std::atomic<int> cache_dev[kMaxDevices][kMaxClusterSplits + 1];
   if (ns < 1 || ns > kMaxClusterSplits) return 0;
-  int *cache = cache_dev[device_slot()];
+  std::atomic<int> *cache = cache_dev[device_slot()];
   if (cache[ns]) return cache[ns];
   if (ensure_attr<C>()) return 0;
   cudaLaunchConfig_t cfg{};

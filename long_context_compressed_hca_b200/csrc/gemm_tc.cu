@@ -157,8 +157,8 @@ int launch_gemm_tc(const void *A, long long lda, const void *Bm, long long ldb, 
   if (M < BM || N < BN || K < BK || (lda * 2) % 16 || (ldb * 2) % 16 ||
       (reinterpret_cast<uintptr_t>(A) & 15) || (reinterpret_cast<uintptr_t>(Bm) & 15))
     return HCA_ERR_UNSUPPORTED;
-  static bool attr_dev[kMaxDevices] = {false};
-  bool &attr = attr_dev[device_slot()];
+  static std::atomic<bool> attr_dev[kMaxDevices];
+  std::atomic<bool> &attr = attr_dev[device_slot()];
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmem);

@@ -231,8 +231,8 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
 template <int N, bool FP8, int S>
 int launch_tc_t(const IndexParams &p, int QB, int tiles_per_unit, int units_per_qb, cudaStream_t s) {
   using L = TcIdxLayout<N, FP8, S>;
-  static bool attr_dev[kMaxDevices] = {false};
-  bool &attr = attr_dev[device_slot()];
+  static std::atomic<bool> attr_dev[kMaxDevices];
+  std::atomic<bool> &attr = attr_dev[device_slot()];
   if (!attr) {
     const cudaError_t e = cudaFuncSetAttribute(index_scores_tc<N, FP8, S>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::bytes);

@@ -7,7 +7,7 @@
 // lower entry index, emitted in ascending index order and padded with -1.
 //
 // The selection is an exact radix select on the order-preserving uint32 image
-// of the fp32 scores (up to 4 passes of 8 bits), run by a thread-block cluster
+// of the fp32 scores (three digits of 11, 11 and 10 bits, 2048 bins), run by a thread-block cluster
 // whose CTAs hold slices of the row in shared memory and sum their histograms
 // through distributed shared memory, followed by a stable compaction.
 #include <mutex>
@@ -374,8 +374,8 @@ TopkPlan plan_topk(long long rows, long long Vmax) {
 }
 size_t topk_smem(const TopkPlan &t) { return (size_t)(t.slice + kCandMax) * 4; }
 int ensure_topk_smem() {
-  static bool done_dev[kMaxDevices] = {false};
-  bool &done = done_dev[device_slot()];
+  static std::atomic<bool> done_dev[kMaxDevices];
+  std::atomic<bool> &done = done_dev[device_slot()];
   if (!done) {
     const cudaError_t e = cudaFuncSetAttribute(topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (kSliceMax + kCandMax) * 4);

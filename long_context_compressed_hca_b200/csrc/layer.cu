@@ -257,6 +257,33 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
   return hca_attend(&ad, P.q, P.kvw, 1, P.kvw, 0, L->sink, n, 0, o, nullptr, 0, stream);
 }
 
+int hybrid_workspace_map(const hca_layer *L, int n, int decode, hca_ws_map *map) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  if (!map) return fail(HCA_ERR_INVALID, "null map");
+  if (n < (decode ? 1 : 0)) return fail(HCA_ERR_INVALID, "n must be >= %d", decode ? 1 : 0);
+  const bool csa = L->kind == HCA_LAYER_CSA, comp = L->kind != HCA_LAYER_SWA;
+  *map = hca_ws_map{-1, -1, -1, -1, -1, -1, -1};
+  if (decode) {
+    // hybrid_decode_step keeps the CSA index lists at the start of its workspace
+    if (csa) map->idx = 0;
+    return HCA_OK;
+  }
+  // plan against a stand-in base address and report the distances from it
+  char *const base = reinterpret_cast<char *>(uintptr_t(1) << 40);
+  Plan P{};
+  plan_prefill(L, n, base, P);
+  auto off = [&](void *p) -> long long { return p ? (long long)(static_cast<char *>(p) - base) : -1; };
+  map->idx = csa ? off(P.idx) : -1;
+  map->q = off(P.q);
+  map->qI = csa ? off(P.qI) : -1;
+  map->wI = csa ? off(P.wI) : -1;
+  map->key_I = csa ? off(P.keyI) : -1;
+  map->kv_comp = comp ? off(P.kvc) : -1;
+  map->kv_win = off(P.kvw);
+  return HCA_OK;
+}
+
 // ----------------------------------------------------------------- decode
 size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos) {
   if (check_layer(L) || pos < 0) return 0;

@@ -78,3 +78,34 @@ def check_topk_row(gpu_idx, ref_scores, k, V):
     tol = 1e-5 * max(abs(kth), 1e-30) + 1e-7 * np.abs(ref_scores).max()
     assert (np.abs(ref_scores[diff] - kth) <= tol).all(), "selection differs beyond the tie"
     return True
+
+
+def check_selection_bound(gpu_idx, s_exact, s_shared, k, V):
+    """The GPU's selection against the oracle's fp64 scores s_exact when the
+    GPU stored its index operands in a narrower type: s_shared are the oracle's
+    scores over the GPU's stored (rounded) operands, delta the largest change
+    that rounding made to any score of the row.  A selection exact for
+    s_shared keeps only entries whose s_exact is >= the fp64 k-th score minus
+    2*delta (each side moves by at most delta), which is asserted."""
+    n = min(k, V)
+    if n >= V or n == 0:
+        return 0.0
+    sel = np.asarray(gpu_idx)[:n]
+    s_exact = np.asarray(s_exact, np.float64)
+    delta = float(np.abs(s_exact - np.asarray(s_shared, np.float64)).max())
+    kth = np.sort(s_exact)[::-1][n - 1]
+    slack = 2 * delta + 1e-6 * float(np.abs(s_exact).max())
+    worst = float(kth - s_exact[sel].min())
+    assert worst <= slack, f"a kept entry lies {worst:.3e} below the fp64 k-th score (allowed {slack:.3e})"
+    return delta
+
+
+def oracle_attend_over(q_t, win_rows, kv_comp, sel, sink, c, t, rd):
+    """The oracle's attention output of query t over its window rows and the
+    compressed rows `sel` (the GPU's own selection, already validated against
+    the oracle's), so that near-tie selections leave no output unchecked."""
+    sel = np.asarray(sel)
+    sel = sel[sel >= 0]
+    rows = np.concatenate([np.asarray(win_rows, np.float64).reshape(-1, c),
+                           np.asarray(kv_comp, np.float64)[sel]], axis=0)
+    return O.attend_output(q_t, rows, sink, c ** -0.5, t, rd)

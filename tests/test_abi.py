@@ -135,3 +135,49 @@ def test_fp4_rotate_quant_rejects_bad_arguments(L):
     _bad(L.hca_fp4_rotate_quant(16, hb.HCA_FP8E4M3, 4, 64, 16, None), "x_dtype")
     _bad(L.hca_fp4_rotate_quant(24, hb.HCA_BF16, 4, 64, 16, None), "aligned")
     assert L.hca_fp4_rotate_quant(None, hb.HCA_BF16, 0, 64, None, None) == hb.HCA_OK
+
+
+def test_static_scratch_size_matches_header(L):
+    assert L.hca_static_scratch_bytes() == hb.STATIC_SCRATCH_BYTES == hb.static_scratch_bytes()
+
+
+def test_hca_compress_alias_validates_like_csa_compress(L):
+    d = hb.compress_desc(1, 12, 4, 0, 0, 0, hb.HCA_F32, hb.HCA_F32)   # width not a multiple of 8
+    _bad(L.hca_compress(ctypes.byref(d), 0, 8, 16, None, 16, None, 12, 96, 16, None, None, 16, None, 2,
+                        None, None, None), "width")
+
+
+def test_workspace_map_places_intermediates_inside_the_workspace(L):
+    """hybrid_workspace_map: every prefill intermediate lies inside the
+    workspace hybrid_layer_forward_workspace_size asks for, 256-byte aligned,
+    without overlaps; decode keeps its index lists at offset 0."""
+    from long_context_compressed_hca_b200 import workloads
+    for wl in (workloads.TINY_CSA, workloads.CSA_PREFILL.with_(n=4096, d=512, d_c=256), workloads.HCA_PREFILL):
+        Ls = wl.layers[0]
+        csa = Ls.kind == "csa"
+        lay = hb.Layer()
+        lay.kind = hb.HCA_LAYER_CSA if csa else hb.HCA_LAYER_HCA
+        lay.a = hb.attn_desc(wl.B, Ls.n_h, Ls.c, Ls.rd, Ls.w, Ls.m, overlap=Ls.overlap, k=Ls.k,
+                             n_hI=Ls.n_hI, c_I=Ls.c_I, rd_I=Ls.rd_I if csa else 0, dtype=hb.HCA_BF16)
+        lay.d, lay.d_c = wl.d, wl.d_c
+        lay.sink = 16
+        n = wl.n
+        total = L.hybrid_layer_forward_workspace_size(ctypes.byref(lay), n)
+        mp = hb.workspace_map(lay, n)
+        B, E = wl.B, max(n // Ls.m, 1)
+        sizes = dict(q=B * n * Ls.n_h * Ls.c * 2, kv_win=B * n * Ls.c * 2, kv_comp=B * E * Ls.c * 2)
+        if csa:
+            sizes.update(idx=B * n * Ls.k * 4, qI=B * n * Ls.n_hI * Ls.c_I * 2, wI=B * n * Ls.n_hI * 4,
+                         key_I=B * E * Ls.c_I * 2)
+        else:
+            assert mp["idx"] is None and mp["qI"] is None and mp["key_I"] is None
+        spans = []
+        for key, size in sizes.items():
+            off = mp[key]
+            assert off is not None and off % 256 == 0 and off + size <= total, (wl.name, key, off, size, total)
+            spans.append((off, off + size))
+        spans.sort()
+        assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:])), spans
+        dm = hb.workspace_map(lay, 131072, decode=True)
+        assert (dm["idx"] == 0) if csa else (dm["idx"] is None)
+        assert L.hybrid_workspace_map(ctypes.byref(lay), 0, 1, ctypes.byref(hb.WsMap())) == hb.HCA_ERR_INVALID

@@ -57,8 +57,9 @@ def test_compress_prefill(cuda, overlap, m, width, n, in_dt, out_dt, flags, rd):
     skv = torch.empty(B, R, Cw, device=cuda)
     ssc = torch.empty(B, R, Cw, device=cuda)
     d = hb.compress_desc(B, width, m, overlap, rd, flags, CODE[in_dt], CODE[out_dt])
+    # the non-overlapped (HCA) cases go through the hca_compress name of the same call
     hb.csa_compress(d, 0, n, Ca, Cb if overlap else None, Za, Zb if overlap else None, width, n * width,
-                    Ba, Bb if overlap else None, None, out, None, max(E, 1), skv, ssc)
+                    Ba, Bb if overlap else None, None, out, None, max(E, 1), skv, ssc, hca_name=not overlap)
     torch.cuda.synchronize()
     for b in range(B):
         ref = _ref_entries(Ca, Cb, Za, Zb, Ba, Bb, m, overlap, flags, rd, b)

@@ -8,7 +8,8 @@ from long_context_compressed_hca_b200 import binding as hb
 from long_context_compressed_hca_b200 import synth, workloads
 from long_context_compressed_hca_b200.layer import CacheHandle, LayerHandle, TokenInputs
 from oracle import hca_oracle as O
-from tests.helpers import GAP, GAP_LAYER_BF16, GAP_STRICT, TOL, assert_close, to64
+from tests.helpers import (GAP, GAP_LAYER_BF16, TOL, assert_close, check_selection_bound, check_topk_row,
+                           oracle_attend_over, to64)
 
 pytestmark = pytest.mark.gpu
 F32, BF16 = torch.float32, torch.bfloat16
@@ -18,7 +19,7 @@ def _w64(W):
     return {k: to64(v) for k, v in W.items()}
 
 
-def _run_layer(wl, L, dt, cuda, n=None, cache=None):
+def _run_layer(wl, L, dt, cuda, n=None, cache=None, keep_ws=False):
     n = n or wl.n
     W = synth.layer_weights(L, wl.d, wl.d_c, wl.seed, dt)
     H = synth.hidden_states(wl.B, n, wl.d, wl.seed, dt)
@@ -27,52 +28,111 @@ def _run_layer(wl, L, dt, cuda, n=None, cache=None):
     o = torch.full((wl.B, n, L.n_h, L.c), float("nan"), dtype=dt, device=cuda)
     hb.hybrid_layer_forward(lh.struct, H.to(cuda), n, cache.struct if cache else None, o, ws)
     torch.cuda.synchronize()
+    if keep_ws:
+        return W, H, o, lh, ws
     return W, H, o
+
+
+class PrefillIntermediates:
+    """The GPU's stored intermediates of one hybrid_layer_forward call (no
+    cache), read through hybrid_workspace_map."""
+
+    def __init__(self, lh, ws, L, B, n, dt):
+        mp = hb.workspace_map(lh.struct, n)
+        E = max(n // L.m, 1)
+        v = lambda key, shape, d: hb.ws_view(ws, mp[key], shape, d) if mp[key] is not None else None
+        self.q = v("q", (B, n, L.n_h, L.c), dt)
+        self.kv_win = v("kv_win", (B, n, L.c), dt)
+        self.kv_comp = v("kv_comp", (B, E, L.c), dt)
+        self.idx = v("idx", (B, n, L.k), torch.int32) if L.kind == "csa" else None
+        if L.kind == "csa":
+            self.qI = v("qI", (B, n, L.n_hI, L.c_I), dt)
+            self.wI = v("wI", (B, n, L.n_hI), torch.float32)
+            self.KI = v("key_I", (B, E, L.c_I), dt)
+
+
+def check_prefill_tokens(L, W64, H64, gi: PrefillIntermediates, o, b, toks, d_c, tol):
+    """Every sampled token of sequence b, with nothing skipped:
+      - the stored intermediates (queries, window rows, compressed entries,
+        indexer queries / keys) against the oracle's;
+      - CSA: the GPU's top-k against the oracle's selection over the GPU's
+        stored index operands (bit-exact where the k-th/(k+1)-th gap exceeds
+        1e-3, else within the tie), and bounded against the fp64 scores;
+      - the output against the oracle's attention over the GPU's selection.
+    Returns (tokens checked, near ties among them)."""
+    ref = O.layer_prefill(H64, W64, L, d_c, tokens=toks, return_intermediates=True)
+    E = (int(toks.max()) + 1) // L.m
+    assert_close(to64(gi.q[b, toks]), ref["q"], tol, "q")
+    need = sorted(ref["kv_win"])
+    assert_close(to64(gi.kv_win[b, need]), np.stack([ref["kv_win"][p] for p in need]), tol, "window rows")
+    if E:
+        assert_close(to64(gi.kv_comp[b, :E]), ref["kv_comp"][:E], tol, "kv_comp")
+    sink = W64["sink"]
+    ties = 0
+    if L.kind == "csa":
+        if E:
+            assert_close(to64(gi.KI[b, :E]), ref["KI"][:E], tol, "key_I")
+        assert_close(to64(gi.qI[b, toks]), ref["qI"], tol, "qI")
+        wref = ref["wI"]
+        assert_close(to64(gi.wI[b, toks]), wref, 1e-2 * np.abs(wref).max(), "wI")
+        KIg = to64(gi.KI[b])
+        idx = gi.idx[b, toks].cpu().numpy()
+        qIg, wIg = to64(gi.qI[b, toks]), to64(gi.wI[b, toks])
+    for j, t in enumerate(toks):
+        t = int(t)
+        V = (t + 1) // L.m
+        sel = None
+        if L.kind == "csa":
+            s_shared = O.index_scores(qIg[j], wIg[j], KIg, V)
+            ties += check_topk_row(idx[j], s_shared, L.k, V)
+            check_selection_bound(idx[j], ref["scores"][j], s_shared, L.k, V)
+            sel = idx[j]
+        else:
+            sel = np.arange(V)
+        wrows = [ref["kv_win"][p] for p in O.window_positions(t, L.w)]
+        o_ref = oracle_attend_over(ref["q"][j], wrows, ref["kv_comp"], sel, sink, L.c, t, L.rd)
+        assert_close(to64(o[b, t]), o_ref, tol, f"o[{b},{t}]")
+        if L.kind != "csa" or O.topk_gap(ref["scores"][j], L.k) > GAP_LAYER_BF16 or V <= L.k:
+            # where the fp64 selection is unambiguous the output also matches the plain oracle
+            assert_close(to64(o[b, t]), ref["o"][j], tol, f"o[{b},{t}] (oracle selection)")
+    return len(toks), ties
 
 
 def test_layer_tiny_csa_fp32(cuda):
     wl = workloads.TINY_CSA
     L = wl.layers[0]
-    W, H, o = _run_layer(wl, L, F32, cuda)
-    ref = O.layer_prefill(to64(H[0]), _w64(W), L, wl.d_c, return_intermediates=True)
-    ties = 0
-    for t in range(wl.n):
-        V = (t + 1) // L.m
-        if O.topk_gap(ref["scores"][t], L.k) <= GAP and V > L.k:
-            ties += 1
-            continue
-        assert_close(to64(o[0, t]), ref["o"][t], TOL[F32], f"o[{t}]")
-    assert ties < wl.n // 10
+    W, H, o, lh, ws = _run_layer(wl, L, F32, cuda, keep_ws=True)
+    gi = PrefillIntermediates(lh, ws, L, wl.B, wl.n, F32)
+    checked, ties = check_prefill_tokens(L, _w64(W), to64(H[0]), gi, o, 0, np.arange(wl.n), wl.d_c, TOL[F32])
+    print(f"tiny CSA fp32: {checked} tokens checked, {ties} near ties (checked within the tie)")
 
 
 def test_layer_hca_bf16(cuda):
     wl = workloads.HCA_PREFILL
     L = wl.layers[0]
     n = 2048   # the oracle over all 8192 tokens is covered by the full-size test
-    W, H, o = _run_layer(wl, L, BF16, cuda, n=n)
+    W, H, o, lh, ws = _run_layer(wl, L, BF16, cuda, n=n, keep_ws=True)
+    gi = PrefillIntermediates(lh, ws, L, wl.B, n, BF16)
     W64 = _w64(W)
     for b in range(wl.B):
         toks = np.unique(np.concatenate([np.arange(0, 300), np.arange(n - 300, n),
                                          np.random.default_rng(b).integers(0, n, 200)]))
-        ref = O.layer_prefill(to64(H[b]), W64, L, wl.d_c, tokens=toks)
-        assert_close(to64(o[b, toks]), ref, TOL[BF16], f"o[b={b}]")
+        check_prefill_tokens(L, W64, to64(H[b]), gi, o, b, toks, wl.d_c, TOL[BF16])
 
 
 def test_layer_csa_bf16_small(cuda):
-    """CSA layer with the 64K workload's attention shapes at a short length."""
-    wl = workloads.CSA_PREFILL.with_(n=1024, d=512, d_c=256)
+    """CSA layer with the 64K workload's attention shapes at 4096 tokens, where
+    queries past token 2047 see more than k = 512 entries, so the selection
+    drops entries on every such token."""
+    wl = workloads.CSA_PREFILL.with_(n=4096, d=512, d_c=256)
     L = wl.layers[0]
-    W, H, o = _run_layer(wl, L, BF16, cuda)
-    toks = np.unique(np.concatenate([np.arange(0, 40), np.arange(wl.n - 40, wl.n),
-                                     np.random.default_rng(3).integers(0, wl.n, 60)]))
-    ref = O.layer_prefill(to64(H[0]), _w64(W), L, wl.d_c, tokens=toks, return_intermediates=True)
-    ties = 0
-    for j, t in enumerate(toks):
-        if O.topk_gap(ref["scores"][j], L.k) <= GAP_LAYER_BF16 and (t + 1) // L.m > L.k:
-            ties += 1
-            continue
-        assert_close(to64(o[0, t]), ref["o"][j], TOL[BF16], f"o[{t}]")
-    print(f"near ties: {ties} of {len(toks)}")
+    W, H, o, lh, ws = _run_layer(wl, L, BF16, cuda, keep_ws=True)
+    gi = PrefillIntermediates(lh, ws, L, wl.B, wl.n, BF16)
+    toks = np.unique(np.concatenate([np.arange(0, 40), np.arange(2040, 2060), np.arange(wl.n - 40, wl.n),
+                                     np.random.default_rng(3).integers(0, wl.n, 80)]))
+    checked, ties = check_prefill_tokens(L, _w64(W), to64(H[0]), gi, o, 0, toks, wl.d_c, TOL[BF16])
+    assert sum((int(t) + 1) // L.m > L.k for t in toks) >= 60
+    print(f"CSA bf16 4096 tokens: {checked} tokens checked, {ties} near ties (checked within the tie)")
 
 
 def test_prefill_then_decode_matches_longer_prefill(cuda):
@@ -195,6 +255,9 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
     torch.cuda.synchronize()
     emit = (pos + 1) % m == 0
     ties = 0
+    if csa:
+        mp = hb.workspace_map(lh.struct, pos, decode=True)
+        gidx = hb.ws_view(ws, mp["idx"], (B, 1, L.k), torch.int32).cpu().numpy()
     for b in range(B):
         comp = to64(x["comp"][b])
         kvc = to64(kvc0[b][:(pos + 1) // m + 1])
@@ -238,8 +301,13 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
             kw = dict(qI_t=to64(x["qI"][b]), w_t=to64(x["wI"][b]), KI=KI)
             V = (pos + 1) // m
             scores = O.index_scores(kw["qI_t"], kw["w_t"], KI, V)
-            if V > L.k and O.topk_gap(scores, L.k) <= GAP_STRICT:
-                ties += 1
+            # the step's own selection (it keeps the index lists at the start of
+            # its workspace): exact where the gap rule applies, else within the tie
+            gsel = gidx[b, 0]
+            ties += check_topk_row(gsel, scores, L.k, V)
+            o_sel = oracle_attend_over(to64(x["q"][b]), wrows, kvc, gsel, to64(W["sink"]), c, pos, L.rd)
+            assert_close(to64(o[b]), o_sel, 2e-2, f"decode o[b={b}] (over the GPU's selection)")
+            if V > L.k and O.topk_gap(scores, L.k) <= GAP:
                 continue
         ref, _ = O.layer_decode(L, pos, to64(x["q"][b]), kvc, wrows, to64(W["sink"]), **kw)
         assert_close(to64(o[b]), ref, 2e-2, f"decode o[b={b}]")

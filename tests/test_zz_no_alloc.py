@@ -53,7 +53,7 @@ def _with_workspace(d, qI, wI, KI, KI_scale, cap, B, n_q, start_pos, k, cuda):
 
 @pytest.mark.parametrize("B,n_q,start_pos,k,kdt", CASES)
 def test_static_scratch_matches_workspace_call(cuda, B, n_q, start_pos, k, kdt):
-    assert hb.csa_index_topk_workspace_size(_desc(B, k, kdt), n_q, start_pos) <= hb.STATIC_SCRATCH_BYTES
+    assert hb.csa_index_topk_workspace_size(_desc(B, k, kdt), n_q, start_pos) <= hb.static_scratch_bytes()
     E = max((start_pos + n_q) // 4, 1)
     runs = []
     # two calls in a row on different inputs, each into its own outputs
@@ -82,7 +82,7 @@ def test_static_scratch_refuses_calls_beyond_its_size(cuda):
     # 65 sequences at 128K tokens need 65 * 32768 * 4 bytes of scores > 8 MiB
     B, n_q, start_pos, k = 65, 1, 131071, 512
     args = _inputs(B, n_q, start_pos, k, "bf16", 13, cuda)
-    assert hb.csa_index_topk_workspace_size(args[0], n_q, start_pos) > hb.STATIC_SCRATCH_BYTES
+    assert hb.csa_index_topk_workspace_size(args[0], n_q, start_pos) > hb.static_scratch_bytes()
     idx = torch.full((B, n_q, k), -7, dtype=torch.int32, device=cuda)
     with pytest.raises(hb.HcaError) as e:
         hb.csa_index_topk_static_scratch(*args, n_q, start_pos, idx)
