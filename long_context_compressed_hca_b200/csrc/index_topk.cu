@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
 // index order with ties resolved towards the lower index.  Rows longer than
 // one segment are cut into segments whose winners (order key + index) a
 // second launch merges.
+bool g_topk_row_enabled = true;   // one CTA per row where the row fits (else clusters)
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kSliceMax = 16384;   // keys per CTA (64 KB of shared memory)
@@ -352,6 +353,272 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
     }
 }
 
+// ------------------------------------------------------------ one CTA per row
+// Rows of up to kRowMax keys: one CTA holds the whole row in shared memory
+// and needs no cluster exchange.  The radix digits are taken over the
+// distance of each order key from the row's smallest key, with the first
+// digit placed at the highest bit in which the row's keys differ, so the
+// 2048 bins of the first pass spread over the row's actual range instead of
+// the few quarter-binades the top bits of a float would give.  After the
+// first pass the keys of the threshold's bin are compacted (when they fit in
+// kRowCand slots) and the later passes read only those.  The final pass
+// emits every key above the threshold and the lowest-indexed ties, in
+// ascending index order (per-warp runs of the row, offsets by a block scan).
+constexpr int kRowMax = 36864;     // keys per row held in shared memory (144 KB)
+constexpr int kRowCand = 8192;     // compacted candidate keys (32 KB)
+
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, int *warp_buf, int *total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_buf[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = lane < NW ? warp_buf[lane] : 0;
+    int u = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, u, o);
+      if (lane >= o) u += y;
+    }
+    if (lane < NW) warp_buf[lane] = u - t;
+    if (lane == NW - 1) *total = u;
+  }
+  __syncthreads();
+  const int r = warp_buf[warp] + incl - v;
+  __syncthreads();   // warp_buf may be reused by the caller
+  return r;
+}
+
+// The bin (counted from the top) of the krem-th largest key of histogram
+// h[0..nb), and krem within that bin: out[0] = bin, out[1] = krem in bin.
+template <int NT>
+__device__ __forceinline__ void row_find_digit(const uint32_t *h, int nb, int krem, int *warp_buf, int *scan_tot,
+                                               int *out) {
+  const int per = (nb + NT - 1) / NT;
+  const int hi = nb - 1 - (int)threadIdx.x * per;   // this thread's bins hi, hi-1, ..., > hi-per
+  int sum = 0;
+  for (int j = 0; j < per; ++j)
+    if (hi - j >= 0) sum += (int)h[hi - j];
+  int above = block_exclusive_scan<NT>(sum, warp_buf, scan_tot);
+  if (above < krem && above + sum >= krem) {
+    for (int j = 0; j < per; ++j) {
+      const int b = hi - j;
+      if (b < 0) break;
+      const int c = (int)h[b];
+      if (above + c >= krem) {
+        out[0] = b;
+        out[1] = krem - above;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// Grid: one CTA per row.  Dynamic shared memory: (row_pad + kRowCand) words,
+// row_pad = the launch's longest row rounded up to a multiple of 4.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
+  constexpr int NW = NT / 32;
+  extern __shared__ __align__(16) uint32_t dyn[];
+  uint32_t *keys = dyn;                       // [row_pad]
+  uint32_t *cand = dyn + p.slice;             // [kRowCand]
+  __shared__ uint32_t hist[kBinsMax];
+  __shared__ int warp_buf[32];
+  __shared__ int res[2];
+  __shared__ int scan_tot;
+  __shared__ uint32_t red_min[NW], red_max[NW];
+  __shared__ int s_nc;
+  __shared__ int w_gt[NW], w_eq[NW];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = blockIdx.x;
+  const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
+  int32_t *out = p.idx_out + (long long)row * p.out_stride;
+  pdl_trigger();   // the attention may start its prologue
+  pdl_wait();      // the scores of the previous launch are complete
+  if (p.k <= 0) return;
+
+  // ---- the row as order keys, with its smallest and largest key
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  {
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(p.scores) + (long long)row * p.in_stride;
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+      const int nv = V >> 2;
+      const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+      uint4 *d4 = reinterpret_cast<uint4 *>(keys);
+      for (int i0 = 0; i0 < nv; i0 += 4 * NT) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = i0 + u * NT + tid;
+          if (j < nv) v[u] = __ldg(s4 + j);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = i0 + u * NT + tid;
+          if (j < nv) {
+            uint4 x = v[u];
+            x.x = order_bits(x.x); x.y = order_bits(x.y); x.z = order_bits(x.z); x.w = order_bits(x.w);
+            kmin = min(kmin, min(min(x.x, x.y), min(x.z, x.w)));
+            kmax = max(kmax, max(max(x.x, x.y), max(x.z, x.w)));
+            d4[j] = x;
+          }
+        }
+      }
+      done = nv * 4;
+    }
+    for (int i = done + tid; i < V; i += NT) {
+      const uint32_t x = order_bits(__ldg(src + i));
+      kmin = min(kmin, x);
+      kmax = max(kmax, x);
+      keys[i] = x;
+    }
+  }
+  for (int i = tid; i < kBinsMax; i += NT) hist[i] = 0;
+  if (tid == 0) s_nc = 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
+  __syncthreads();
+  kmin = red_min[0];
+  kmax = red_max[0];
+  for (int w = 1; w < NW; ++w) { kmin = min(kmin, red_min[w]); kmax = max(kmax, red_max[w]); }
+
+  // ---- threshold T (an order key) and krem, the ties at T to keep
+  uint32_t T = 0;   // every key is >= 1: T = 0 keeps them all
+  int krem = 0;
+  if (V > p.k && p.k > 0) {
+    const uint32_t range = kmax - kmin;
+    const int nbits = range ? 32 - __clz(range) : 0;
+    uint32_t prefix = 0;   // (key - kmin) >> shift of the keys still in play
+    int shift = nbits;
+    krem = p.k;
+    bool compacted = false;
+    int nc = 0;
+    while (shift > 0) {
+      const int width = shift > 11 ? 11 : shift;
+      const int nshift = shift - width;
+      const int nb = 1 << width;
+      const uint32_t *arr = compacted ? cand : keys;
+      const int n = compacted ? nc : V;
+      for (int i = tid; i < n; i += NT) {
+        const uint32_t v = arr[i] - kmin;
+        if (shift >= 32 || (v >> shift) == prefix) atomicAdd(&hist[(v >> nshift) & (uint32_t)(nb - 1)], 1u);
+      }
+      __syncthreads();
+      row_find_digit<NT>(hist, nb, krem, warp_buf, &scan_tot, res);
+      const uint32_t digit = (uint32_t)res[0];
+      krem = res[1];
+      const uint32_t in_bin = hist[digit];
+      const uint32_t nprefix = (prefix << width) | digit;
+      if (!compacted && nshift > 0 && in_bin <= (uint32_t)kRowCand) {
+        // the keys of the threshold's bin, in any order
+        for (int i0 = 0; i0 < n; i0 += NT) {
+          const int i = i0 + tid;
+          const uint32_t kk = i < n ? arr[i] : 0u;
+          const bool m = i < n && ((kk - kmin) >> nshift) == nprefix;
+          const unsigned bal = __ballot_sync(0xffffffffu, m);
+          int at = 0;
+          if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
+          at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+          if (m) cand[at] = kk;
+        }
+        nc = (int)in_bin;
+        compacted = true;
+      }
+      __syncthreads();   // every thread has read hist[digit]
+      for (int i = tid; i < nb; i += NT) hist[i] = 0;
+      __syncthreads();
+      prefix = nprefix;
+      shift = nshift;
+    }
+    T = kmin + prefix;     // all bits decided: the k-th largest key
+    if (nbits == 0) T = kmin;
+  }
+
+  // ---- emit: keys above T and the first krem keys equal to T, ascending
+  const int wseg = ((V + NT - 1) / NT) * 32;   // a contiguous run of keys per warp
+  const int w_lo = min(V, warp * wseg), w_hi = min(V, w_lo + wseg);
+  int gt = 0, eq = 0;
+  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t kk = i < w_hi ? keys[i] : 0u;
+    gt += __popc(__ballot_sync(0xffffffffu, kk > T));
+    eq += __popc(__ballot_sync(0xffffffffu, T != 0 && kk == T));
+  }
+  if (lane == 0) { w_gt[warp] = gt; w_eq[warp] = eq; }
+  __syncthreads();
+  int ties_before = 0, sel_before = 0;
+  for (int w = 0; w < warp; ++w) { ties_before += w_eq[w]; sel_before += w_gt[w]; }
+  sel_before += min(krem, ties_before);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t kk = i < w_hi ? keys[i] : 0u;
+    const bool is_eq = T != 0 && kk == T;
+    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
+    const bool take = kk > T || (is_eq && ties_before + __popc(eqm & lt) < krem);
+    const unsigned sm = __ballot_sync(0xffffffffu, take);
+    if (take) out[sel_before + __popc(sm & lt)] = i;
+    ties_before += __popc(eqm);
+    sel_before += __popc(sm);
+  }
+  const int K = V < p.k ? V : p.k;
+  for (int i = K + tid; i < p.k; i += NT) out[i] = -1;
+}
+
+template <int NT>
+int launch_topk_row_t(const TopkParams &t, long long rows, int row_pad, cudaStream_t s) {
+  const size_t smem = (size_t)(row_pad + kRowCand) * 4;
+  static std::atomic<bool> attr_dev[kMaxDevices];
+  std::atomic<bool> &attr = attr_dev[device_slot()];
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(topk_row<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (kRowMax + kRowCand) * 4);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k row smem attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  LaunchScope ls("topk", s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)rows, 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  TopkParams tp = t;
+  tp.slice = row_pad;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_row<NT>, tp);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "topk_row launch: %s", cudaGetErrorString(e));
+  }
+  return ls.done();
+}
+// One CTA per row for rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise).
+int launch_topk_row(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
+  if (Vmax > kRowMax || rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
+  const int row_pad = ((Vmax + 3) / 4) * 4;
+  if (Vmax > 4096) return launch_topk_row_t<1024>(t, rows, row_pad, s);
+  return launch_topk_row_t<256>(t, rows, row_pad, s);
+}
+
 struct TopkPlan {
   int C, n_seg, seg_len, slice;
 };
@@ -465,6 +732,10 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t.rows = (int)rows; t.k = ip.k; t.scores = p.scores; t.in_stride = p.score_stride;
   t.n_q = ip.n_q; t.start_pos = ip.start_pos; t.m = ip.m;
   t.n_seg = pl.n_seg; t.seg_len = pl.seg_len; t.slice = pl.slice;
+  if (Vmax <= kRowMax && g_topk_row_enabled) {
+    t.idx_out = idx; t.out_stride = ip.k;
+    return launch_topk_row(t, rows, Vmax, s);
+  }
   if (pl.n_seg == 1) {
     t.idx_out = idx; t.out_stride = ip.k;
     return launch_topk_cluster("topk", t, pl, rows, s);

@@ -195,9 +195,13 @@ def test_index_topk(cuda, B, n_q, start_pos, m, k, n_hI, c_I, qdt, kdt):
 
 
 TIE_CASES = [
-    # B, n_q, start_pos, k, key dtype: rows span one CTA, a cluster, two segments
+    # B, n_q, start_pos, k, key dtype.  Rows of up to 36864 keys: one CTA per
+    # row (256 threads up to 4096 keys, else 1024); longer rows: a cluster per
+    # row segment (one segment, then two, then the 1M rows' segments + merge)
     (2, 64, 0, 64, "bf16"),
+    (2, 8, 16000, 64, "bf16"),
     (3, 1, 131071, 512, "bf16"),
+    (2, 1, 163839, 512, "bf16"),
     (1, 2, 300000, 512, "bf16"),
     (2, 1, 1048575, 1024, "fp8"),
 ]
