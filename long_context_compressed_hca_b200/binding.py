@@ -99,6 +99,7 @@ def _declare(L):
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
         "hca_kv_mixed_row_bytes": (SZ, [I, I]),
+        "hca_step_trace": (I, [VP, SZ]),
         "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
         "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
     }
@@ -299,6 +300,26 @@ def oproj_desc(T, n_h, c, g, d_g, d, dtype=HCA_BF16, out_dtype=HCA_F32) -> Oproj
 
 def output_projection_workspace_size(d: OprojDesc) -> int:
     return lib().hca_output_projection_workspace_size(C.byref(d))
+
+
+STEP_TRACE_KERNELS = {1: "ingest", 2: "indexer", 3: "top-k", 4: "attend CSA", 5: "attend HCA"}
+
+
+def step_trace(buf):
+    """Point the decode-step kernels at `buf` (a zeroed uint64 device tensor:
+    counter, then 4 words per CTA record), or switch the trace off (None)."""
+    nbytes = buf.numel() * buf.element_size() if buf is not None else 0
+    return check(lib().hca_step_trace(ptr(buf), nbytes))
+
+
+def step_trace_records(buf):
+    """The records of a trace buffer as a list of dicts (host copy)."""
+    h = buf.cpu().numpy().view("uint64")
+    n = min(int(h[0]), (h.shape[0] - 1) // 4)
+    recs = h[1:1 + 4 * n].reshape(n, 4)
+    return [{"kernel": STEP_TRACE_KERNELS.get(int(r[3] >> 48), str(int(r[3] >> 48))),
+             "sm": int((r[3] >> 32) & 0xFFFF), "cta": int(r[3] & 0xFFFFFFFF),
+             "entry": int(r[0]), "ready": int(r[1]), "exit": int(r[2])} for r in recs]
 
 
 def kv_mixed_row_bytes(c, rd) -> int:

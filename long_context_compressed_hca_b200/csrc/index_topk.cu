@@ -209,8 +209,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   const int len = max(0, min(p.slice, seg_V - (int)rank * p.slice));
   const long long begin = seg_begin + (long long)rank * p.slice;   // element index of keys[0]
 
+  const unsigned long long st_entry = global_ns();
   pdl_trigger();   // the attention may start its prologue
   pdl_wait();      // the scores of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
   if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
   else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
   for (int i = tid; i < kBinsMax; i += kTopkThreads) {
@@ -350,6 +352,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
       out[i] = -1;
       if (kout) kout[i] = 0u;
     }
+  if (step_trace_on()) {
+    __syncthreads();
+    if (tid == 0) step_trace_record(ST_TOPK, st_entry, st_ready);
+  }
 }
 
 struct TopkPlan {
@@ -538,5 +544,7 @@ int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores
   if (rc) return rc;
   return run_index_topk(p, idx, user_scores, user_stride, scratch, (size_t)HCA_STATIC_SCRATCH_BYTES, s);
 }
+
+int step_trace_set_index_topk(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca

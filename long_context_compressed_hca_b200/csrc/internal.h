@@ -109,6 +109,13 @@ int run_index_topk(const IndexParams &p, int32_t *idx, float *user_scores, long 
 int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores, long long user_stride,
                           cudaStream_t s);
 
+// ------------------------------------------------------------- step trace
+// Point the traced kernels of each translation unit at a record buffer (NULL = off).
+int step_trace_set_attend(void *buf, unsigned long long cap);
+int step_trace_set_index_tc(void *buf, unsigned long long cap);
+int step_trace_set_index_topk(void *buf, unsigned long long cap);
+int step_trace_set_compress(void *buf, unsigned long long cap);
+
 // ------------------------------------------------------- mixed-precision KV
 // Record bytes of one row (0 for unsupported shapes) and the two HBM streams.
 size_t kv_mixed_row_bytes(int c, int rd);
