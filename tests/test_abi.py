@@ -128,3 +128,8 @@ def test_attention_cta_budget_sets_the_split_plan(L):
     assert ws("hca", 4) == 0                                     # 1 split
     assert ws("csa", 0) == split_ws(9)                           # 18 tiles -> 9 splits
     assert ws("csa", 32) == 0
+
+
+def test_step_trace_rejects_bad_buffers(L):
+    _bad(L.hca_step_trace(12, 1024), "8-byte aligned")
+    _bad(L.hca_step_trace(16, 32), "8-byte aligned")
