@@ -379,6 +379,17 @@ int hca_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *ou
  * ---------------------------------------------------------------------- */
 int hca_fp4_rotate_quant(const void *x, hca_dtype x_dtype, long long rows, int n, void *out, hca_stream_t stream);
 
+/* Diagnostic timeline of the decode step's kernels (ingest, indexer, top-k,
+ * attention): with buf set, thread 0 of every CTA of those kernels appends
+ * one record of four uint64 -- entry time, time after its wait for the
+ * previous kernel, exit time (all %globaltimer ns) and kernel << 48 | SM << 32
+ * | CTA index (kernel: 1 ingest, 2 indexer, 3 top-k, 4 CSA attention, 5 HCA
+ * attention) -- at buf + 8 + 32 * i, where i comes from the uint64 counter at
+ * buf[0] (records past the capacity are counted, not written).  The caller
+ * zeroes buf and reads it after synchronising.  buf = NULL switches it off.
+ * Synchronises the device (it sets a device variable per source file). */
+int hca_step_trace(void *buf, size_t bytes);
+
 /* Diagnostic trace of the tensor-core attention kernel: with enable = 1 the
  * following attend launches accumulate, summed over CTAs, the SM cycles each
  * role spends waiting on each pipeline barrier, plus unit / tile / rescale

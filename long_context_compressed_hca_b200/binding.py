@@ -110,6 +110,8 @@ def _declare(L):
                              VP, LL, VP, VP, VP]),
         "hybrid_workspace_map": (I, [C.POINTER(Layer), I, I, C.POINTER(WsMap)]),
         "hca_fp4_rotate_quant": (I, [VP, I, LL, I, VP, VP]),
+
+        "hca_step_trace": (I, [VP, SZ]),
         "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
         "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
     }
@@ -337,6 +339,26 @@ def output_projection_workspace_size(d: OprojDesc) -> int:
 
 def fp4_rotate_quant(x, x_dtype, rows, n, out, stream=None):
     return check(lib().hca_fp4_rotate_quant(ptr(x), x_dtype, rows, n, ptr(out), stream_handle(stream)))
+
+
+STEP_TRACE_KERNELS = {1: "ingest", 2: "indexer", 3: "top-k", 4: "attend CSA", 5: "attend HCA"}
+
+
+def step_trace(buf):
+    """Point the decode-step kernels at `buf` (a zeroed uint64 device tensor:
+    counter, then 4 words per CTA record), or switch the trace off (None)."""
+    nbytes = buf.numel() * buf.element_size() if buf is not None else 0
+    return check(lib().hca_step_trace(ptr(buf), nbytes))
+
+
+def step_trace_records(buf):
+    """The records of a trace buffer as a list of dicts (host copy)."""
+    h = buf.cpu().numpy().view("uint64")
+    n = min(int(h[0]), (h.shape[0] - 1) // 4)
+    recs = h[1:1 + 4 * n].reshape(n, 4)
+    return [{"kernel": STEP_TRACE_KERNELS.get(int(r[3] >> 48), str(int(r[3] >> 48))),
+             "sm": int((r[3] >> 32) & 0xFFFF), "cta": int(r[3] & 0xFFFFFFFF),
+             "entry": int(r[0]), "ready": int(r[1]), "exit": int(r[2])} for r in recs]
 
 
 def kv_mixed_row_bytes(c, rd) -> int:

@@ -467,6 +467,19 @@ int hca_fp4_rotate_quant(const void *x, hca_dtype x_dtype, long long rows, int n
   return launch_fp4_rotate_quant(x, x_dtype, rows, out, static_cast<cudaStream_t>(stream));
 }
 
+// ------------------------------------------------------------- step trace
+int hca_step_trace(void *buf, size_t bytes) {
+  REQUIRE(buf == nullptr || ((reinterpret_cast<uintptr_t>(buf) & 7u) == 0 && bytes >= 40),
+          "buf must be 8-byte aligned and hold the counter and at least one record (40 bytes)");
+  const unsigned long long cap = buf ? (unsigned long long)((bytes - 8) / 32) : 0ull;
+  int rc = step_trace_set_attend(buf, cap);
+  if (!rc) rc = step_trace_set_index_tc(buf, cap);
+  if (!rc) rc = step_trace_set_index_topk(buf, cap);
+  if (!rc) rc = step_trace_set_compress(buf, cap);
+  if (rc) return fail(rc, "could not set the step trace buffer");
+  return HCA_OK;
+}
+
 // ------------------------------------------------------ mixed-precision KV
 size_t hca_kv_mixed_row_bytes(int c, int rd) { return kv_mixed_row_bytes(c, rd); }
 

@@ -506,6 +506,7 @@ attend_tc(AttendParams p, int n_units) {
   float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // [4 warps][64]: cos, sin
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned long long st_entry = global_ns();
   auto bar = [&](uint64_t &b) { return smem_u32(&b); };
   unsigned long long tr[TR_COUNT];
   if (TRACE) for (int i = 0; i < TR_COUNT; ++i) tr[i] = 0;
@@ -558,6 +559,7 @@ attend_tc(AttendParams p, int n_units) {
     cluster_sync();
   }
   pdl_wait();   // indices, caches and queries of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
   if (TRACE && threadIdx.x == 0) ts[1] = global_ns();
 
   if (warp >= kProdWarp0) {
@@ -1020,6 +1022,7 @@ attend_tc(AttendParams p, int n_units) {
     atomicMax(&g_attn_trace[TR_T_EXIT_MAX], ts[5]);
     atomicAdd(&g_attn_trace[TR_T_CTAS], 1ull);
   }
+  if (threadIdx.x == 0) step_trace_record(p.csa ? ST_ATTEND_CSA : ST_ATTEND_HCA, st_entry, st_ready);
   if (warp == kMmaWarp) tmem_dealloc(tmem, L::tmem_cols);
 }
 
@@ -1200,6 +1203,8 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
   else attend_simt<__nv_bfloat16><<<grid, kSimtWarps * 32, smem, s>>>(p);
   return ls_.done();
 }
+
+int step_trace_set_attend(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca
 

@@ -89,6 +89,42 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ---------------------------------------------------------------- step trace
+// Diagnostic timeline of the decode step's kernels: when a buffer is set
+// (hca_step_trace), CTA thread 0 of each traced kernel appends one record
+// {entry ns, ready ns (after its dependent-launch wait), exit ns, id} with
+// id = kernel << 48 | SM << 32 | blockIdx.x; buf[0] counts records.  One
+// copy of the setting per translation unit (no relocatable device code).
+struct StepTrace {
+  unsigned long long *buf;
+  unsigned long long cap;
+};
+static __device__ StepTrace g_step_trace;
+enum StepTraceKernel { ST_INGEST = 1, ST_INDEX = 2, ST_TOPK = 3, ST_ATTEND_CSA = 4, ST_ATTEND_HCA = 5 };
+__device__ __forceinline__ bool step_trace_on() { return g_step_trace.buf != nullptr; }
+__device__ __forceinline__ void step_trace_record(unsigned kernel, unsigned long long t_entry,
+                                                  unsigned long long t_ready) {
+  const StepTrace t = g_step_trace;
+  if (!t.buf) return;
+  unsigned long long t_exit;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_exit));
+  unsigned sm;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+  const unsigned long long i = atomicAdd(t.buf, 1ull);
+  if (i < t.cap) {
+    unsigned long long *r = t.buf + 1 + 4 * i;
+    r[0] = t_entry;
+    r[1] = t_ready;
+    r[2] = t_exit;
+    r[3] = ((unsigned long long)kernel << 48) | ((unsigned long long)sm << 32) | blockIdx.x;
+  }
+}
+// Host: point this translation unit's kernels at `buf` (NULL = off).
+static inline int step_trace_set_here(void *buf, unsigned long long cap) {
+  const StepTrace t{static_cast<unsigned long long *>(buf), cap};
+  return cudaMemcpyToSymbol(g_step_trace, &t, sizeof t) == cudaSuccess ? HCA_OK : HCA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -340,6 +340,7 @@ __global__ void __launch_bounds__(kThreads) decode_ingest_kernel(CompressParams 
                                                                  IngestRing ring, int pos) {
   extern __shared__ float sm[];
   const int b = blockIdx.x, part = blockIdx.y;
+  const unsigned long long st_entry = global_ns();
   pdl_trigger();   // the layer's next kernel may start its prologue
   if (part == 0 && pa.B > 0) {
     compress_decode_block<Tin, TA>(pa, pos, b, sm);
@@ -349,6 +350,10 @@ __global__ void __launch_bounds__(kThreads) decode_ingest_kernel(CompressParams 
     const Tw *row = reinterpret_cast<const Tw *>(ring.row) + (long long)b * ring.c;
     Tw *dst = reinterpret_cast<Tw *>(ring.ring) + ((long long)b * ring.w + ring.slot) * ring.c;
     for (int col = threadIdx.x; col < ring.c; col += kThreads) dst[col] = row[col];
+  }
+  if (step_trace_on()) {
+    __syncthreads();
+    if (threadIdx.x == 0) step_trace_record(ST_INGEST, st_entry, st_entry);
   }
 }
 
@@ -442,5 +447,7 @@ int launch_decode_ingest(const CompressParams *pa, const CompressParams *pb, con
     decode_ingest_kernel<float, __nv_bfloat16, float, __nv_bfloat16><<<grid, kThreads, smem, s>>>(a, bb, hb, ring, pos);
   return ls_.done();
 }
+
+int step_trace_set_compress(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca

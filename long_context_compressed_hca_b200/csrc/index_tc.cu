@@ -61,6 +61,7 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
             acc_empty = 4 * S + 3;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned long long st_entry = global_ns();
   // work unit: (sequence, query block, tile range)
   int u = blockIdx.x;
   const int nunits_per_b = p.n_qb * p.units_per_qb;
@@ -101,6 +102,7 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
   const long long key_row0 = (long long)b * p.cap + e_begin;
   pdl_trigger();   // the selection may start its prologue
   pdl_wait();      // keys and queries of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
 
   if (warp == 0) {
     // ------------------------------------------------ loads
@@ -225,6 +227,7 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) step_trace_record(ST_INDEX, st_entry, st_ready);
   if (warp == 1) tmem_dealloc(tmem, L::tmem_cols);
 }
 
@@ -306,5 +309,7 @@ int launch_index_scores_tc(const IndexParams &p, cudaStream_t s) {
   units = (tiles + tpu - 1) / tpu;
   return fp8 ? launch_tc_t<16, true, 6>(p, 2, tpu, units, s) : launch_tc_t<16, false, 6>(p, 2, tpu, units, s);
 }
+
+int step_trace_set_index_tc(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca

@@ -210,8 +210,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
   const int len = max(0, min(p.slice, seg_V - (int)rank * p.slice));
   const long long begin = seg_begin + (long long)rank * p.slice;   // element index of keys[0]
 
+  const unsigned long long st_entry = global_ns();
   pdl_trigger();   // the attention may start its prologue
   pdl_wait();      // the scores of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
   if (p.keys) load_keys<true>(keys, p.keys + row * p.in_stride + begin, len);
   else load_keys<false>(keys, reinterpret_cast<const uint32_t *>(p.scores) + row * p.in_stride + begin, len);
   for (int i = tid; i < kBinsMax; i += kTopkThreads) {
@@ -351,6 +353,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
       out[i] = -1;
       if (kout) kout[i] = 0u;
     }
+  if (step_trace_on()) {
+    __syncthreads();
+    if (tid == 0) step_trace_record(ST_TOPK, st_entry, st_ready);
+  }
 }
 
 // ------------------------------------------------------------ one CTA per row
@@ -443,8 +449,10 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   const int row = blockIdx.x;
   const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
   int32_t *out = p.idx_out + (long long)row * p.out_stride;
+  const unsigned long long st_entry = global_ns();
   pdl_trigger();   // the attention may start its prologue
   pdl_wait();      // the scores of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
   if (p.k <= 0) return;
 
   // ---- the row as order keys, with its smallest and largest key
@@ -578,6 +586,10 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   }
   const int K = V < p.k ? V : p.k;
   for (int i = K + tid; i < p.k; i += NT) out[i] = -1;
+  if (step_trace_on()) {
+    __syncthreads();
+    if (tid == 0) step_trace_record(ST_TOPK, st_entry, st_ready);
+  }
 }
 
 template <int NT>
@@ -810,5 +822,7 @@ int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores
   if (rc) return rc;
   return run_index_topk(p, idx, user_scores, user_stride, scratch, (size_t)HCA_STATIC_SCRATCH_BYTES, s);
 }
+
+int step_trace_set_index_topk(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca

@@ -119,6 +119,12 @@ int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores
 // ------------------------------------------------------------ FP4 indexer
 // Rows of 64: Hadamard rotation, FP4 blocks of 32, written as exact bf16 values.
 int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s);
+// ------------------------------------------------------------- step trace
+// Point the traced kernels of each translation unit at a record buffer (NULL = off).
+int step_trace_set_attend(void *buf, unsigned long long cap);
+int step_trace_set_index_tc(void *buf, unsigned long long cap);
+int step_trace_set_index_topk(void *buf, unsigned long long cap);
+int step_trace_set_compress(void *buf, unsigned long long cap);
 
 // ------------------------------------------------------- mixed-precision KV
 // Record bytes of one row (0 for unsupported shapes) and the two HBM streams.

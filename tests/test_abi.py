@@ -181,3 +181,8 @@ def test_workspace_map_places_intermediates_inside_the_workspace(L):
         dm = hb.workspace_map(lay, 131072, decode=True)
         assert (dm["idx"] == 0) if csa else (dm["idx"] is None)
         assert L.hybrid_workspace_map(ctypes.byref(lay), 0, 1, ctypes.byref(hb.WsMap())) == hb.HCA_ERR_INVALID
+
+
+def test_step_trace_rejects_bad_buffers(L):
+    _bad(L.hca_step_trace(12, 1024), "8-byte aligned")
+    _bad(L.hca_step_trace(16, 32), "8-byte aligned")
