@@ -101,6 +101,10 @@ constexpr uint32_t kNoBin = 0xFFFFFFFFu;
 __device__ __forceinline__ int digit_shift(int pass) { return pass == 0 ? 21 : (pass == 1 ? 10 : 0); }
 __device__ __forceinline__ int digit_width(int pass) { return pass == 2 ? 10 : 11; }
 
+// The float of an order key (inverse of order_bits; -0 comes back as +0).
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 __device__ __forceinline__ uint32_t order_bits(uint32_t u) {
   if ((u & 0x7FFFFFFFu) == 0) u = 0;                 // -0 == +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // >= 1 for every non-NaN float
@@ -509,13 +513,88 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   uint32_t T = 0;   // every key is >= 1: T = 0 keeps them all
   int krem = 0;
   if (V > p.k && p.k > 0) {
-    const uint32_t range = kmax - kmin;
-    const int nbits = range ? 32 - __clz(range) : 0;
-    uint32_t prefix = 0;   // (key - kmin) >> shift of the keys still in play
-    int shift = nbits;
     krem = p.k;
+    // pass A: 2048 equal-width bins of the score over [lo, hi].  The bin is a
+    // monotone function of the score (rounded subtraction and product keep
+    // the order), so the bin holding the k-th largest score bounds the
+    // threshold; the scores' bell shape spreads them thinly over the bins,
+    // which keeps same-address atomics rare
+    const float lo = key_float(kmin), hi = key_float(kmax);
+    const float scale = (float)kBinsMax / (hi - lo);
+    const bool linear = kmin != kmax && scale > 0.f && scale < INFINITY;
+    auto lin_bin = [&](uint32_t kk) -> uint32_t {
+      const float x = (key_float(kk) - lo) * scale;
+      return x < (float)(kBinsMax - 1) ? (uint32_t)x : (uint32_t)(kBinsMax - 1);
+    };
+    uint32_t lbin = 0;
     bool compacted = false;
     int nc = 0;
+    uint32_t cmin = kmin, cmax = kmax;   // key range of the keys still in play
+    if (linear) {
+      for (int i0 = 0; i0 < V; i0 += NT) {
+        const int i = i0 + tid;
+        const bool valid = i < V;
+        const uint32_t bin = valid ? lin_bin(keys[i]) : 0xFFFFFFFFu;
+        // a warp whose 32 keys share one bin adds them at once (rows of ties)
+        if (__all_sync(0xffffffffu, bin == __shfl_sync(0xffffffffu, bin, 0))) {
+          if (lane == 0 && valid) atomicAdd(&hist[bin], 32u);
+        } else if (valid) {
+          atomicAdd(&hist[bin], 1u);
+        }
+      }
+      __syncthreads();
+      row_find_digit<NT>(hist, kBinsMax, krem, warp_buf, &scan_tot, res);
+      lbin = (uint32_t)res[0];
+      krem = res[1];
+      const uint32_t in_bin = hist[lbin];
+      cmin = 0xFFFFFFFFu;
+      cmax = 0u;
+      if (in_bin <= (uint32_t)kRowCand) {
+        for (int i0 = 0; i0 < V; i0 += NT) {
+          const int i = i0 + tid;
+          const uint32_t kk = i < V ? keys[i] : 0u;
+          const bool m = i < V && lin_bin(kk) == lbin;
+          const unsigned bal = __ballot_sync(0xffffffffu, m);
+          int at = 0;
+          if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
+          at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
+          if (m) {
+            cand[at] = kk;
+            cmin = min(cmin, kk);
+            cmax = max(cmax, kk);
+          }
+        }
+        nc = (int)in_bin;
+        compacted = true;
+      } else {
+        for (int i = tid; i < V; i += NT) {
+          const uint32_t kk = keys[i];
+          if (lin_bin(kk) == lbin) { cmin = min(cmin, kk); cmax = max(cmax, kk); }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+        cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+      }
+      __syncthreads();   // every thread has read hist[lbin]; red_* free again
+      if (lane == 0) { red_min[warp] = cmin; red_max[warp] = cmax; }
+      for (int i = tid; i < kBinsMax; i += NT) hist[i] = 0;
+      __syncthreads();
+      cmin = red_min[0];
+      cmax = red_max[0];
+      for (int w = 1; w < NW; ++w) { cmin = min(cmin, red_min[w]); cmax = max(cmax, red_max[w]); }
+    }
+    // passes B: exact radix digits over the distance of each remaining key
+    // from the smallest one, the first digit at their highest differing bit
+    const uint32_t range = cmax - cmin;
+    const int nbits = range ? 32 - __clz(range) : 0;
+    uint32_t prefix = 0;   // (key - cmin) >> shift of the keys still in play
+    int shift = nbits;
+    auto in_play = [&](uint32_t kk) -> bool {
+      if (!compacted && linear && lin_bin(kk) != lbin) return false;
+      return shift >= 32 || ((kk - cmin) >> shift) == prefix;
+    };
     while (shift > 0) {
       const int width = shift > 11 ? 11 : shift;
       const int nshift = shift - width;
@@ -523,8 +602,8 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       const uint32_t *arr = compacted ? cand : keys;
       const int n = compacted ? nc : V;
       for (int i = tid; i < n; i += NT) {
-        const uint32_t v = arr[i] - kmin;
-        if (shift >= 32 || (v >> shift) == prefix) atomicAdd(&hist[(v >> nshift) & (uint32_t)(nb - 1)], 1u);
+        const uint32_t kk = arr[i];
+        if (in_play(kk)) atomicAdd(&hist[((kk - cmin) >> nshift) & (uint32_t)(nb - 1)], 1u);
       }
       __syncthreads();
       row_find_digit<NT>(hist, nb, krem, warp_buf, &scan_tot, res);
@@ -537,7 +616,7 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
         for (int i0 = 0; i0 < n; i0 += NT) {
           const int i = i0 + tid;
           const uint32_t kk = i < n ? arr[i] : 0u;
-          const bool m = i < n && ((kk - kmin) >> nshift) == nprefix;
+          const bool m = i < n && in_play(kk) && ((kk - cmin) >> nshift) == nprefix;
           const unsigned bal = __ballot_sync(0xffffffffu, m);
           int at = 0;
           if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
@@ -553,8 +632,7 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       prefix = nprefix;
       shift = nshift;
     }
-    T = kmin + prefix;     // all bits decided: the k-th largest key
-    if (nbits == 0) T = kmin;
+    T = cmin + prefix;     // all bits decided: the k-th largest key
   }
 
   // ---- emit: keys above T and the first krem keys equal to T, ascending
