@@ -364,18 +364,27 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cluster(TopkParams p) {
 }
 
 // ------------------------------------------------------------ one CTA per row
-// Rows of up to kRowMax keys: one CTA holds the whole row in shared memory
-// and needs no cluster exchange.  The radix digits are taken over the
-// distance of each order key from the row's smallest key, with the first
-// digit placed at the highest bit in which the row's keys differ, so the
-// 2048 bins of the first pass spread over the row's actual range instead of
-// the few quarter-binades the top bits of a float would give.  After the
-// first pass the keys of the threshold's bin are compacted (when they fit in
-// kRowCand slots) and the later passes read only those.  The final pass
-// emits every key above the threshold and the lowest-indexed ties, in
-// ascending index order (per-warp runs of the row, offsets by a block scan).
-constexpr int kRowMax = 36864;     // keys per row held in shared memory (144 KB)
-constexpr int kRowCand = 8192;     // compacted candidate keys (32 KB)
+// Rows of up to 32 * NT keys: one CTA holds the whole row in registers (eight
+// 16-byte loads per thread, all in flight at once) and selects in one pass:
+//   1. a sample of the row (one key per thread, spread over the whole row)
+//      gives two thresholds t_hi > t_lo between which the k-th largest score
+//      falls with high probability (sample ranks of about k*S/V -+ 3 sigma);
+//   2. every key is compared with them: keys above t_hi are marked as winners
+//      in a bit mask of the row, keys in [t_lo, t_hi] are compacted into a
+//      band list (a few times k keys);
+//   3. if the counts confirm that the k-th score lies in the band, an exact
+//      radix select over the band's order keys finds the threshold key T and
+//      the number of ties at T to keep; otherwise (ties or an unlucky sample)
+//      the same exact select runs over the whole row held in registers;
+//   4. the winners' and the kept ties' bits are emitted in ascending index
+//      order (ties to the lower index) by a block scan over the mask words.
+// Every decision is exact: the thresholds only decide how much of the row the
+// exact select has to look at.
+constexpr int kRowRegs = 8;        // 16-byte loads per thread: rows of up to 32 * NT keys
+constexpr int kRowMaxNT = 1024;
+constexpr int kRowMax = 32 * kRowMaxNT;
+constexpr int kRowCand = 4096;     // band keys held in shared memory (order key + index)
+constexpr int kRowSample = 1024;   // at most one sample key per thread
 
 template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_buf, int *total) {
@@ -406,7 +415,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_buf, int *t
   return r;
 }
 
-// The bin (counted from the top) of the krem-th largest key of histogram
+// The bin (counted from the top) of the krem-th largest element of histogram
 // h[0..nb), and krem within that bin: out[0] = bin, out[1] = krem in bin.
 template <int NT>
 __device__ __forceinline__ void row_find_digit(const uint32_t *h, int nb, int krem, int *warp_buf, int *scan_tot,
@@ -433,25 +442,67 @@ __device__ __forceinline__ void row_find_digit(const uint32_t *h, int nb, int kr
   __syncthreads();
 }
 
-// Grid: one CTA per row.  Dynamic shared memory: (row_pad + kRowCand) words,
-// row_pad = the launch's longest row rounded up to a multiple of 4.
+// Shared state of one row's selection.
+struct RowSel {
+  uint32_t hist[kBinsMax];
+  int warp_buf[32];
+  int res[2];
+  int scan_tot;
+  int s_above, s_nc;
+  uint32_t s_min, s_max;
+};
+
+// Exact radix select of the krem-th largest order key among a set of keys
+// that each(f) visits (every thread calls f on its share of the keys; 0 =
+// no key).  Distances from kmin are taken in digits of up to 11 bits from
+// their highest differing bit.  Returns T (the key) and, in *krem, how many
+// keys equal to T are kept.
+template <int NT, typename Each>
+__device__ uint32_t radix_select(RowSel &sh, uint32_t kmin, uint32_t kmax, int *krem, Each each) {
+  const int tid = threadIdx.x;
+  const uint32_t range = kmax - kmin;
+  const int nbits = range ? 32 - __clz(range) : 0;
+  uint32_t prefix = 0;
+  int shift = nbits;
+  while (shift > 0) {
+    const int width = shift > 11 ? 11 : shift;
+    const int nshift = shift - width;
+    const int nb = 1 << width;
+    each([&](uint32_t kk) {
+      if (kk == 0 || kk < kmin || kk > kmax) return;
+      const uint32_t v = kk - kmin;
+      if (shift >= 32 || (v >> shift) == prefix) atomicAdd(&sh.hist[(v >> nshift) & (uint32_t)(nb - 1)], 1u);
+    });
+    __syncthreads();
+    row_find_digit<NT>(sh.hist, nb, *krem, sh.warp_buf, &sh.scan_tot, sh.res);
+    const uint32_t digit = (uint32_t)sh.res[0];
+    *krem = sh.res[1];
+    __syncthreads();   // every thread has read res
+    for (int i = tid; i < nb; i += NT) sh.hist[i] = 0;
+    __syncthreads();
+    prefix = (prefix << width) | digit;
+    shift = nshift;
+  }
+  return kmin + prefix;
+}
+
+// Grid: one CTA per row.  Dynamic shared memory: 2 * words + 2 * kRowCand
+// words (winner and tie masks of the row, band keys and indices).
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   constexpr int NW = NT / 32;
   extern __shared__ __align__(16) uint32_t dyn[];
-  uint32_t *keys = dyn;                       // [row_pad]
-  uint32_t *cand = dyn + p.slice;             // [kRowCand]
-  __shared__ uint32_t hist[kBinsMax];
-  __shared__ int warp_buf[32];
-  __shared__ int res[2];
-  __shared__ int scan_tot;
-  __shared__ uint32_t red_min[NW], red_max[NW];
-  __shared__ int s_nc;
-  __shared__ int w_gt[NW], w_eq[NW];
+  __shared__ RowSel sh;
+  __shared__ uint32_t red_a[NW], red_b[NW];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;
   const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
+  const int nwords = (V + 31) >> 5;
+  uint32_t *win = dyn;                        // [nwords_max]
+  uint32_t *tie = dyn + p.slice;              // [nwords_max]
+  uint32_t *band_key = dyn + 2 * p.slice;     // [kRowCand]
+  uint32_t *band_idx = band_key + kRowCand;   // [kRowCand]
   int32_t *out = p.idx_out + (long long)row * p.out_stride;
   const unsigned long long st_entry = global_ns();
   pdl_trigger();   // the attention may start its prologue
@@ -459,208 +510,215 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   const unsigned long long st_ready = global_ns();
   if (p.k <= 0) return;
 
-  // ---- the row as order keys, with its smallest and largest key
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  {
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(p.scores) + (long long)row * p.in_stride;
-    int done = 0;
-    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-      const int nv = V >> 2;
-      const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-      uint4 *d4 = reinterpret_cast<uint4 *>(keys);
-      for (int i0 = 0; i0 < nv; i0 += 4 * NT) {
-        uint4 v[4];
+  // ---- the row in registers: thread t holds keys 4t + 4NT*j + e (as floats)
+  const float *src = p.scores + (long long)row * p.in_stride;
+  float x[kRowRegs][4];
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = i0 + u * NT + tid;
-          if (j < nv) v[u] = __ldg(s4 + j);
-        }
+  for (int j = 0; j < kRowRegs; ++j) {
+    const int i = 4 * tid + 4 * NT * j;
+    if (vec && i + 3 < V) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i));
+      x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
+    } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = i0 + u * NT + tid;
-          if (j < nv) {
-            uint4 x = v[u];
-            x.x = order_bits(x.x); x.y = order_bits(x.y); x.z = order_bits(x.z); x.w = order_bits(x.w);
-            kmin = min(kmin, min(min(x.x, x.y), min(x.z, x.w)));
-            kmax = max(kmax, max(max(x.x, x.y), max(x.z, x.w)));
-            d4[j] = x;
-          }
-        }
-      }
-      done = nv * 4;
-    }
-    for (int i = done + tid; i < V; i += NT) {
-      const uint32_t x = order_bits(__ldg(src + i));
-      kmin = min(kmin, x);
-      kmax = max(kmax, x);
-      keys[i] = x;
+      for (int e = 0; e < 4; ++e) x[j][e] = i + e < V ? __ldg(src + i + e) : 0.f;
     }
   }
-  for (int i = tid; i < kBinsMax; i += NT) hist[i] = 0;
-  if (tid == 0) s_nc = 0;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-  }
-  if (lane == 0) { red_min[warp] = kmin; red_max[warp] = kmax; }
-  __syncthreads();
-  kmin = red_min[0];
-  kmax = red_max[0];
-  for (int w = 1; w < NW; ++w) { kmin = min(kmin, red_min[w]); kmax = max(kmax, red_max[w]); }
+  for (int w = tid; w < nwords; w += NT) { win[w] = 0u; tie[w] = 0u; }
+  for (int i = tid; i < kBinsMax; i += NT) sh.hist[i] = 0u;
+  if (tid == 0) { sh.s_above = 0; sh.s_nc = 0; }
 
-  // ---- threshold T (an order key) and krem, the ties at T to keep
-  uint32_t T = 0;   // every key is >= 1: T = 0 keeps them all
-  int krem = 0;
-  if (V > p.k && p.k > 0) {
-    krem = p.k;
-    // pass A: 2048 equal-width bins of the score over [lo, hi].  The bin is a
-    // monotone function of the score (rounded subtraction and product keep
-    // the order), so the bin holding the k-th largest score bounds the
-    // threshold; the scores' bell shape spreads them thinly over the bins,
-    // which keeps same-address atomics rare
-    const float lo = key_float(kmin), hi = key_float(kmax);
+  int krem = 0;        // ties at T to keep
+  uint32_t T = 0;      // the k-th largest order key (0: every key is kept)
+  bool banded = false;
+  if (V > p.k) {
+    // ---- 1. sample: thread t contributes key 4t + 4NT*(t % 8) (its register j = t % 8)
+    const int js = tid % kRowRegs;
+    const int is = 4 * tid + 4 * NT * js;
+    const bool has_s = is < V && tid < kRowSample;
+    float sv = 0.f;
+#pragma unroll
+    for (int j = 0; j < kRowRegs; ++j)
+      if (j == js) sv = x[j][0];
+    uint32_t smin = has_s ? order_bits(__float_as_uint(sv)) : 0xFFFFFFFFu;
+    uint32_t smax = has_s ? smin : 0u;
+    int ns = has_s ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+      smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+      ns += __shfl_xor_sync(0xffffffffu, ns, o);
+    }
+    if (lane == 0) { red_a[warp] = smin; red_b[warp] = smax; sh.warp_buf[warp] = ns; }
+    __syncthreads();
+    smin = red_a[0]; smax = red_b[0]; ns = sh.warp_buf[0];
+    for (int w = 1; w < NW; ++w) { smin = min(smin, red_a[w]); smax = max(smax, red_b[w]); ns += sh.warp_buf[w]; }
+    __syncthreads();
+    const float lo = key_float(smin), hi = key_float(smax);
     const float scale = (float)kBinsMax / (hi - lo);
-    const bool linear = kmin != kmax && scale > 0.f && scale < INFINITY;
-    auto lin_bin = [&](uint32_t kk) -> uint32_t {
-      const float x = (key_float(kk) - lo) * scale;
-      return x < (float)(kBinsMax - 1) ? (uint32_t)x : (uint32_t)(kBinsMax - 1);
-    };
-    uint32_t lbin = 0;
-    bool compacted = false;
-    int nc = 0;
-    uint32_t cmin = kmin, cmax = kmax;   // key range of the keys still in play
-    if (linear) {
-      for (int i0 = 0; i0 < V; i0 += NT) {
-        const int i = i0 + tid;
-        const bool valid = i < V;
-        const uint32_t bin = valid ? lin_bin(keys[i]) : 0xFFFFFFFFu;
-        // a warp whose 32 keys share one bin adds them at once (rows of ties)
-        if (__all_sync(0xffffffffu, bin == __shfl_sync(0xffffffffu, bin, 0))) {
-          if (lane == 0 && valid) atomicAdd(&hist[bin], 32u);
-        } else if (valid) {
-          atomicAdd(&hist[bin], 1u);
-        }
+    if (ns >= 64 && smin != smax && scale > 0.f && scale < INFINITY) {
+      // 2048 equal-width bins of the sample values; ranks from the top
+      if (has_s) {
+        const float f = (key_float(order_bits(__float_as_uint(sv))) - lo) * scale;
+        const uint32_t b = f >= (float)(kBinsMax - 1) ? (uint32_t)(kBinsMax - 1) : (f > 0.f ? (uint32_t)f : 0u);
+        atomicAdd(&sh.hist[b], 1u);
       }
       __syncthreads();
-      row_find_digit<NT>(hist, kBinsMax, krem, warp_buf, &scan_tot, res);
-      lbin = (uint32_t)res[0];
-      krem = res[1];
-      const uint32_t in_bin = hist[lbin];
-      cmin = 0xFFFFFFFFu;
-      cmax = 0u;
-      if (in_bin <= (uint32_t)kRowCand) {
-        for (int i0 = 0; i0 < V; i0 += NT) {
-          const int i = i0 + tid;
-          const uint32_t kk = i < V ? keys[i] : 0u;
-          const bool m = i < V && lin_bin(kk) == lbin;
-          const unsigned bal = __ballot_sync(0xffffffffu, m);
-          int at = 0;
-          if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
-          at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
-          if (m) {
-            cand[at] = kk;
-            cmin = min(cmin, kk);
-            cmax = max(cmax, kk);
+      const float q = (float)p.k * (float)ns / (float)V;   // sample keys expected above the k-th
+      const int r_hi = max(1, (int)floorf(q - 3.f * sqrtf(q)));
+      const int r_lo = min(ns, (int)ceilf(q + 3.f * sqrtf(q) + 2.f));
+      row_find_digit<NT>(sh.hist, kBinsMax, r_hi, sh.warp_buf, &sh.scan_tot, sh.res);
+      const int b_hi = sh.res[0];
+      __syncthreads();
+      row_find_digit<NT>(sh.hist, kBinsMax, r_lo, sh.warp_buf, &sh.scan_tot, sh.res);
+      const int b_lo = sh.res[0];
+      __syncthreads();
+      for (int i = tid; i < kBinsMax; i += NT) sh.hist[i] = 0u;
+      // thresholds at the bin edges: above t_hi = winners, [t_lo, t_hi] = band
+      const float t_hi = lo + (float)(b_hi + 1) / scale;
+      const float t_lo = lo + (float)b_lo / scale;
+      // ---- 2. one pass over the row
+      int above = 0;
+      const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+      for (int j = 0; j < kRowRegs; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * tid + 4 * NT * j + e;
+          const bool valid = i < V;
+          const float v = x[j][e];
+          const bool up = valid && v > t_hi;
+          const bool inb = valid && !up && v >= t_lo;
+          const unsigned bu = __ballot_sync(0xffffffffu, up);
+          above += __popc(bu);
+          if (up) atomicOr(&win[i >> 5], 1u << (i & 31));
+          const unsigned bb = __ballot_sync(0xffffffffu, inb);
+          if (bb) {
+            int at = 0;
+            if (lane == 0) at = atomicAdd(&sh.s_nc, __popc(bb));
+            at = __shfl_sync(0xffffffffu, at, 0) + __popc(bb & lt);
+            if (inb && at < kRowCand) {
+              band_key[at] = order_bits(__float_as_uint(v));
+              band_idx[at] = (uint32_t)i;
+            }
           }
         }
-        nc = (int)in_bin;
-        compacted = true;
-      } else {
-        for (int i = tid; i < V; i += NT) {
-          const uint32_t kk = keys[i];
-          if (lin_bin(kk) == lbin) { cmin = min(cmin, kk); cmax = max(cmax, kk); }
-        }
       }
+      if (lane == 0) atomicAdd(&sh.s_above, above);
+      __syncthreads();
+      const int na = sh.s_above, nc = sh.s_nc;
+      banded = na < p.k && na + nc >= p.k && nc <= kRowCand;
+      if (banded) {
+        // ---- 3. exact select within the band
+        uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
+        for (int i = tid; i < nc; i += NT) { cmin = min(cmin, band_key[i]); cmax = max(cmax, band_key[i]); }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+          cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+        }
+        if (lane == 0) { red_a[warp] = cmin; red_b[warp] = cmax; }
+        __syncthreads();
+        cmin = red_a[0]; cmax = red_b[0];
+        for (int w = 1; w < NW; ++w) { cmin = min(cmin, red_a[w]); cmax = max(cmax, red_b[w]); }
+        krem = p.k - na;
+        T = radix_select<NT>(sh, cmin, cmax, &krem, [&](auto f) {
+          for (int i = tid; i < nc; i += NT) f(band_key[i]);
+        });
+        for (int i = tid; i < nc; i += NT) {
+          const uint32_t kk = band_key[i], ix = band_idx[i];
+          if (kk > T) atomicOr(&win[ix >> 5], 1u << (ix & 31));
+          else if (kk == T) atomicOr(&tie[ix >> 5], 1u << (ix & 31));
+        }
+      } else {
+        // the band missed the k-th score: clear the winner marks
+        for (int w = tid; w < nwords; w += NT) win[w] = 0u;
+      }
+      __syncthreads();
+    }
+    if (!banded) {
+      // ---- 3'. exact select over the whole row (registers)
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+      for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * tid + 4 * NT * j + e < V) {
+            const uint32_t kk = order_bits(__float_as_uint(x[j][e]));
+            kmin = min(kmin, kk);
+            kmax = max(kmax, kk);
+          }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
-        cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
-        cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
       }
-      __syncthreads();   // every thread has read hist[lbin]; red_* free again
-      if (lane == 0) { red_min[warp] = cmin; red_max[warp] = cmax; }
-      for (int i = tid; i < kBinsMax; i += NT) hist[i] = 0;
+      if (lane == 0) { red_a[warp] = kmin; red_b[warp] = kmax; }
       __syncthreads();
-      cmin = red_min[0];
-      cmax = red_max[0];
-      for (int w = 1; w < NW; ++w) { cmin = min(cmin, red_min[w]); cmax = max(cmax, red_max[w]); }
-    }
-    // passes B: exact radix digits over the distance of each remaining key
-    // from the smallest one, the first digit at their highest differing bit
-    const uint32_t range = cmax - cmin;
-    const int nbits = range ? 32 - __clz(range) : 0;
-    uint32_t prefix = 0;   // (key - cmin) >> shift of the keys still in play
-    int shift = nbits;
-    auto in_play = [&](uint32_t kk) -> bool {
-      if (!compacted && linear && lin_bin(kk) != lbin) return false;
-      return shift >= 32 || ((kk - cmin) >> shift) == prefix;
-    };
-    while (shift > 0) {
-      const int width = shift > 11 ? 11 : shift;
-      const int nshift = shift - width;
-      const int nb = 1 << width;
-      const uint32_t *arr = compacted ? cand : keys;
-      const int n = compacted ? nc : V;
-      for (int i = tid; i < n; i += NT) {
-        const uint32_t kk = arr[i];
-        if (in_play(kk)) atomicAdd(&hist[((kk - cmin) >> nshift) & (uint32_t)(nb - 1)], 1u);
-      }
-      __syncthreads();
-      row_find_digit<NT>(hist, nb, krem, warp_buf, &scan_tot, res);
-      const uint32_t digit = (uint32_t)res[0];
-      krem = res[1];
-      const uint32_t in_bin = hist[digit];
-      const uint32_t nprefix = (prefix << width) | digit;
-      if (!compacted && nshift > 0 && in_bin <= (uint32_t)kRowCand) {
-        // the keys of the threshold's bin, in any order
-        for (int i0 = 0; i0 < n; i0 += NT) {
-          const int i = i0 + tid;
-          const uint32_t kk = i < n ? arr[i] : 0u;
-          const bool m = i < n && in_play(kk) && ((kk - cmin) >> nshift) == nprefix;
-          const unsigned bal = __ballot_sync(0xffffffffu, m);
-          int at = 0;
-          if (lane == 0 && bal) at = atomicAdd(&s_nc, __popc(bal));
-          at = __shfl_sync(0xffffffffu, at, 0) + __popc(bal & ((1u << lane) - 1u));
-          if (m) cand[at] = kk;
+      kmin = red_a[0]; kmax = red_b[0];
+      for (int w = 1; w < NW; ++w) { kmin = min(kmin, red_a[w]); kmax = max(kmax, red_b[w]); }
+      krem = p.k;
+      T = radix_select<NT>(sh, kmin, kmax, &krem, [&](auto f) {
+#pragma unroll
+        for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (4 * tid + 4 * NT * j + e < V) f(order_bits(__float_as_uint(x[j][e])));
+      });
+#pragma unroll
+      for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * tid + 4 * NT * j + e;
+          if (i < V) {
+            const uint32_t kk = order_bits(__float_as_uint(x[j][e]));
+            if (kk > T) atomicOr(&win[i >> 5], 1u << (i & 31));
+            else if (kk == T) atomicOr(&tie[i >> 5], 1u << (i & 31));
+          }
         }
-        nc = (int)in_bin;
-        compacted = true;
-      }
-      __syncthreads();   // every thread has read hist[digit]
-      for (int i = tid; i < nb; i += NT) hist[i] = 0;
       __syncthreads();
-      prefix = nprefix;
-      shift = nshift;
     }
-    T = cmin + prefix;     // all bits decided: the k-th largest key
+  } else {
+    // every key is kept
+    for (int w = tid; w < nwords; w += NT) win[w] = (w < (V >> 5)) ? 0xFFFFFFFFu : ((1u << (V & 31)) - 1u);
+    __syncthreads();
   }
 
-  // ---- emit: keys above T and the first krem keys equal to T, ascending
-  const int wseg = ((V + NT - 1) / NT) * 32;   // a contiguous run of keys per warp
-  const int w_lo = min(V, warp * wseg), w_hi = min(V, w_lo + wseg);
-  int gt = 0, eq = 0;
-  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t kk = i < w_hi ? keys[i] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, kk > T));
-    eq += __popc(__ballot_sync(0xffffffffu, T != 0 && kk == T));
+  // ---- 4. emit the winners and the first krem ties in ascending index order
+  constexpr int kWordsPerThread = (kRowMax / 32 + NT - 1) / NT;
+  const int wpt = (nwords + NT - 1) / NT;
+  const int w0 = tid * wpt;
+  int my_ties = 0;
+  for (int u = 0; u < wpt && u < kWordsPerThread; ++u)
+    if (w0 + u < nwords) my_ties += __popc(tie[w0 + u]);
+  int ties_before = block_exclusive_scan<NT>(my_ties, sh.warp_buf, &sh.scan_tot);
+  int my_sel = 0;
+  {
+    int tb = ties_before;
+    for (int u = 0; u < wpt && u < kWordsPerThread; ++u)
+      if (w0 + u < nwords) {
+        const int nt = __popc(tie[w0 + u]);
+        my_sel += __popc(win[w0 + u]) + max(0, min(nt, krem - tb));
+        tb += nt;
+      }
   }
-  if (lane == 0) { w_gt[warp] = gt; w_eq[warp] = eq; }
-  __syncthreads();
-  int ties_before = 0, sel_before = 0;
-  for (int w = 0; w < warp; ++w) { ties_before += w_eq[w]; sel_before += w_gt[w]; }
-  sel_before += min(krem, ties_before);
-  const unsigned lt = (1u << lane) - 1u;
-  for (int i0 = w_lo; i0 < w_hi; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t kk = i < w_hi ? keys[i] : 0u;
-    const bool is_eq = T != 0 && kk == T;
-    const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-    const bool take = kk > T || (is_eq && ties_before + __popc(eqm & lt) < krem);
-    const unsigned sm = __ballot_sync(0xffffffffu, take);
-    if (take) out[sel_before + __popc(sm & lt)] = i;
-    ties_before += __popc(eqm);
-    sel_before += __popc(sm);
+  int at = block_exclusive_scan<NT>(my_sel, sh.warp_buf, &sh.scan_tot);
+  for (int u = 0; u < wpt && u < kWordsPerThread; ++u) {
+    const int w = w0 + u;
+    if (w >= nwords) break;
+    uint32_t wm = win[w], tm = tie[w];
+    while (wm | tm) {
+      const int bw = wm ? __ffs(wm) - 1 : 32, bt = tm ? __ffs(tm) - 1 : 32;
+      if (bw < bt) {
+        out[at++] = w * 32 + bw;
+        wm &= wm - 1u;
+      } else {
+        if (ties_before < krem) out[at++] = w * 32 + bt;
+        ++ties_before;
+        tm &= tm - 1u;
+      }
+    }
   }
   const int K = V < p.k ? V : p.k;
   for (int i = K + tid; i < p.k; i += NT) out[i] = -1;
@@ -671,13 +729,14 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
 }
 
 template <int NT>
-int launch_topk_row_t(const TopkParams &t, long long rows, int row_pad, cudaStream_t s) {
-  const size_t smem = (size_t)(row_pad + kRowCand) * 4;
+int launch_topk_row_t(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
+  const int words = (Vmax + 31) / 32;
+  const size_t smem = (size_t)(2 * words + 2 * kRowCand) * 4;
   static std::atomic<bool> attr_dev[kMaxDevices];
   std::atomic<bool> &attr = attr_dev[device_slot()];
   if (!attr) {
     const cudaError_t e = cudaFuncSetAttribute(topk_row<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (kRowMax + kRowCand) * 4);
+                                               (2 * (kRowMax / 32) + 2 * kRowCand) * 4);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k row smem attribute: %s", cudaGetErrorString(e));
     attr = true;
   }
@@ -693,7 +752,7 @@ int launch_topk_row_t(const TopkParams &t, long long rows, int row_pad, cudaStre
   cfg.attrs = at;
   cfg.numAttrs = 1;
   TopkParams tp = t;
-  tp.slice = row_pad;
+  tp.slice = words;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_row<NT>, tp);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
@@ -704,9 +763,10 @@ int launch_topk_row_t(const TopkParams &t, long long rows, int row_pad, cudaStre
 // One CTA per row for rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise).
 int launch_topk_row(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
   if (Vmax > kRowMax || rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
-  const int row_pad = ((Vmax + 3) / 4) * 4;
-  if (Vmax > 4096) return launch_topk_row_t<1024>(t, rows, row_pad, s);
-  return launch_topk_row_t<256>(t, rows, row_pad, s);
+  if (Vmax <= 32 * 128) return launch_topk_row_t<128>(t, rows, Vmax, s);
+  if (Vmax <= 32 * 256) return launch_topk_row_t<256>(t, rows, Vmax, s);
+  if (Vmax <= 32 * 512) return launch_topk_row_t<512>(t, rows, Vmax, s);
+  return launch_topk_row_t<1024>(t, rows, Vmax, s);
 }
 
 struct TopkPlan {
