@@ -191,9 +191,12 @@ int csa_index_topk_static_scratch(const hca_attn_desc *d, const void *qI, const 
  *   z_j = scale * q_h . row_j ; o_h = sum_j e^{z_j} row_j / (sum_j e^{z_j} + e^{sink_h})
  * then the last rd dims of o_h are rotated by -t.
  * q [B, n_q, n_h, c]; kv_comp [B, cap, c]; sink [n_h] fp32; o [B, n_q, n_h, c].
- * kv_win: prefill (win_is_ring == 0, start_pos == 0): [B, n_q, c], row t =
- *   token t; decode (win_is_ring == 1, n_q == 1): [B, w, c] ring, token p in
- *   slot p % w (the caller has already stored token start_pos).
+ * kv_win: token rows (win_is_ring == 0): [B, h + n_q, c], row r = token
+ *   start_pos - h + r, where h = min(w - 1, start_pos) is the halo of window
+ *   rows before the first query (h = 0 for a prefill from position 0; a
+ *   context-parallel rank starting at start_pos > 0 passes its halo);
+ *   decode (win_is_ring == 1, n_q == 1): [B, w, c] ring, token p in slot
+ *   p % w (the caller has already stored token start_pos).
  * Few queries (decode): each query's key list is cut across up to 8 CTAs of a
  *   thread-block cluster whose partials are merged on chip; no scratch needed.
  * ws: scratch only for a query cut into more than 8 pieces (fp32 partials +
@@ -270,6 +273,35 @@ typedef struct {
 size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos);
 int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache,
                        int pos, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Context-parallel prefill ([J] §4.5, the two-stage communication for
+ * compressed attention; ranhao §6): the tokens of a long prefill are cut into
+ * contiguous ranges, one per rank.  Stage 1 compresses each range on its own
+ * (hybrid_cp_compress); the caller then all-gathers the ranks' entries and
+ * indexer keys (one collective, e.g. NCCL); stage 2 scores, selects and
+ * attends the range's queries against the gathered caches (hybrid_cp_attend).
+ * A rank owns tokens [t0, t0 + n_loc) of every sequence (t0 a multiple of m)
+ * and is given H [B, h + n_loc, d] (a.dtype): its rows preceded by the
+ * h = hybrid_cp_halo(L, t0) rows of the tokens before t0 (the window rows of
+ * its first queries, and for CSA the previous block, whose b series the
+ * range's first entry needs).  Compressed layers only (CSA, HCA); a CSA
+ * window must cover the overlap block (w - 1 >= m).
+ * ---------------------------------------------------------------------- */
+/* h = min(t0, max(w - 1, m if the layer's compression overlaps else 0)). */
+int hybrid_cp_halo(const hca_layer *L, int t0);
+size_t hybrid_cp_workspace_size(const hca_layer *L, int t0, int n_loc);
+/* Stage 1: entries t0/m .. (t0 + n_loc)/m - 1 of every sequence, normalised
+ * and RoPE'd at their global positions, to kv_comp [B, out_cap, c] (a.dtype)
+ * and, CSA, key_I [B, out_cap, c_I] (idx_key_dtype; key_I_scale [B, out_cap]
+ * fp32 for fp8 keys), slots 0 .. n_loc/m - 1. */
+int hybrid_cp_compress(const hca_layer *L, const void *H, int t0, int n_loc, void *kv_comp, void *key_I,
+                       float *key_I_scale, int out_cap, void *ws, size_t ws_bytes, hca_stream_t stream);
+/* Stage 2: o [B, n_loc, n_h, c] of the range's queries against the gathered
+ * caches kv_comp [B, cap, c] and (CSA) key_I [B, cap, c_I] (+ key_I_scale),
+ * which must hold entries 0 .. (t0 + n_loc)/m - 1 (cap >= that). */
+int hybrid_cp_attend(const hca_layer *L, const void *H, int t0, int n_loc, const void *kv_comp, const void *key_I,
+                     const float *key_I_scale, int cap, void *o, void *ws, size_t ws_bytes, hca_stream_t stream);
 
 /* Where the two calls above leave their intermediate results inside the
  * caller's workspace, so that a caller can inspect the selection and the

@@ -112,6 +112,10 @@ def _declare(L):
         "hca_fp4_rotate_quant": (I, [VP, I, LL, I, VP, VP]),
 
         "hca_step_trace": (I, [VP, SZ]),
+        "hybrid_cp_halo": (I, [C.POINTER(Layer), I]),
+        "hybrid_cp_workspace_size": (SZ, [C.POINTER(Layer), I, I]),
+        "hybrid_cp_compress": (I, [C.POINTER(Layer), VP, I, I, VP, VP, VP, I, VP, SZ, VP]),
+        "hybrid_cp_attend": (I, [C.POINTER(Layer), VP, I, I, VP, VP, VP, I, VP, VP, SZ, VP]),
         "hca_kv_quant_mixed": (I, [VP, I, LL, I, I, VP, VP]),
         "hca_kv_dequant_mixed": (I, [VP, LL, I, I, VP, VP]),
     }
@@ -293,6 +297,22 @@ def hca_attend(d: AttnDesc, q, kv_comp, cap, kv_win, win_is_ring, sink, n_q, sta
 
 def layer_workspace_size(L: Layer, n: int) -> int:
     return lib().hybrid_layer_forward_workspace_size(C.byref(L), n)
+
+
+def ctypes_byref(x):
+    return C.byref(x)
+
+
+def hybrid_cp_compress(L: Layer, H, t0, n_loc, kv_comp, key_I, key_I_scale, out_cap, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    return check(lib().hybrid_cp_compress(C.byref(L), ptr(H), t0, n_loc, ptr(kv_comp), ptr(key_I), ptr(key_I_scale),
+                                          out_cap, ptr(ws), nbytes, stream_handle(stream)))
+
+
+def hybrid_cp_attend(L: Layer, H, t0, n_loc, kv_comp, key_I, key_I_scale, cap, o, ws, stream=None):
+    nbytes = ws.numel() * ws.element_size()
+    return check(lib().hybrid_cp_attend(C.byref(L), ptr(H), t0, n_loc, ptr(kv_comp), ptr(key_I), ptr(key_I_scale),
+                                        cap, ptr(o), ptr(ws), nbytes, stream_handle(stream)))
 
 
 def workspace_map(L: Layer, n: int, decode: bool = False) -> dict:

@@ -192,6 +192,11 @@ AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv
   p.w = d->w; p.m = d->m; p.k = csa ? d->k : 0; p.cap = cap; p.csa = csa; p.win_is_ring = win_is_ring;
   p.scale = attn_scale(d); p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
   p.q = q; p.kv_comp = kv_comp; p.idx = idx; p.kv_win = kv_win; p.sink = sink; p.o = o; p.dtype = d->dtype;
+  // token-indexed window: the rows of tokens start_pos - h .. start_pos + n_q - 1,
+  // h = min(w - 1, start_pos) (the halo before the first query)
+  const int halo = d->w > 0 ? (d->w - 1 < start_pos ? d->w - 1 : start_pos) : 0;
+  p.win_tok0 = start_pos - halo;
+  p.win_rows = n_q + halo;
   p.status = nullptr;
   p.nsplit = 1;
   p.cluster = 0;
@@ -209,7 +214,6 @@ int check_attend_args(const hca_attn_desc *d, const void *q, const void *kv_comp
   REQUIRE(vmax == 0 || (kv_comp && aligned16(kv_comp)), "kv_comp must be non-null and 16-byte aligned");
   if (d->w > 0) REQUIRE(kv_win && aligned16(kv_win), "kv_win must be non-null and 16-byte aligned");
   if (win_is_ring) REQUIRE(n_q <= 1, "a ring window serves one query per sequence");
-  else REQUIRE(start_pos == 0, "a token-indexed window needs start_pos == 0");
   return HCA_OK;
 }
 

@@ -68,7 +68,7 @@ __device__ __forceinline__ int slot_row(const AttendParams &p, const KeySet &ks,
   if (kk < ks.nw4) {
     valid = kk < ks.nw;
     const int tok = valid ? ks.t0 + kk : ks.t0 + ks.nw - 1;
-    return p.win_is_ring ? b * p.w + tok % p.w : b * p.n_q + tok;
+    return p.win_is_ring ? b * p.w + tok % p.w : b * p.win_rows + (tok - p.win_tok0);
   }
   const int slot = kk - ks.nw4;
   int e = slot;
@@ -88,7 +88,7 @@ __device__ __forceinline__ const T *key_row(const AttendParams &p, const KeySet 
     const int tok = ks.t0 + j;
     if (p.win_is_ring)
       return reinterpret_cast<const T *>(p.kv_win) + ((long long)b * p.w + tok % p.w) * p.c;
-    return reinterpret_cast<const T *>(p.kv_win) + ((long long)b * p.n_q + tok) * p.c;
+    return reinterpret_cast<const T *>(p.kv_win) + ((long long)b * p.win_rows + (tok - p.win_tok0)) * p.c;
   }
   if (j >= ks.nk) return nullptr;
   int e = j - ks.nw;

@@ -127,7 +127,7 @@ compress_prefill_kernel(CompressParams p, int epb, int rg) {
   const int rgi = local / cv;
   const int b = blockIdx.y;
   const int E = p.n / p.m;
-  const long long entry = (long long)blockIdx.x * epb + slot;
+  const long long entry = p.e_first + (long long)blockIdx.x * epb + slot;
   const bool valid = entry < E && rgi < rg;
   const int R = (p.overlap && entry > 0) ? 2 * p.m : p.m;
 
@@ -191,7 +191,7 @@ compress_prefill_kernel(CompressParams p, int epb, int rg) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) v[q] = 0.f;
   }
-  entry_epilogue<Tout>(p, v, active, slot, cvi, cv, b, entry, entry * p.m, red, red2);
+  entry_epilogue<Tout>(p, v, active, slot, cvi, cv, b, entry - p.e_first, (p.e_pos0 + entry) * p.m, red, red2);
 }
 
 // Prefill leaves the state ready for decode at position n (rows of the last
@@ -367,9 +367,9 @@ int launch_prefill_t(const CompressParams &p, cudaStream_t s) {
   const int tpe = kThreads / epb;
   int rg = tpe / cv;
   if (rg > R) rg = R;
-  const int E = p.n / p.m;
-  if (E == 0) return HCA_OK;
-  dim3 grid((E + epb - 1) / epb, p.B);
+  const long long E = p.n / p.m - p.e_first;   // entries written
+  if (E <= 0) return HCA_OK;
+  dim3 grid((unsigned)((E + epb - 1) / epb), p.B);
   const size_t smem = (size_t)(3 * kThreads * 8 + 2 * epb * cv) * sizeof(float);
   LaunchScope ls_("compress_prefill", s);
   switch (p.out_dtype) {

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) row_op_kernel(RowOpParams p) {
     ss = warp_sum(ss);
     r *= rsqrtf(ss / (float)p.cols + p.eps);
   }
-  const long long pos = (p.pos0 + row / p.rows_per_pos) % p.pos_mod;
+  const long long pos = p.pos_base + (p.pos0 + row / p.rows_per_pos) % p.pos_mod;
   const int c_rope = p.rd > 0 ? p.cols - p.rd : p.cols;
   if (VEC) {
     for (int c = 4 * lane; c < p.cols; c += 128) {

@@ -57,6 +57,10 @@ struct CompressParams {
   long long out_seq_stride;
   float *state_kv, *state_score;
   hca_dtype in_dtype, out_dtype;
+  // prefill of a token range: local entries below e_first only feed the next
+  // entry's b series and are not written (entry e goes to out slot e - e_first);
+  // entry e sits at RoPE position (e_pos0 + e) * m
+  long long e_first, e_pos0;
 };
 int launch_compress_prefill(const CompressParams &p, cudaStream_t s);
 int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s);
@@ -142,7 +146,8 @@ struct AttendParams {
   const void *q;           // [B, n_q, n_h, c]
   const void *kv_comp;     // [B, cap, c]
   const int32_t *idx;      // [B, n_q, k]
-  const void *kv_win;      // prefill [B, n_q, c]; ring [B, w, c]
+  const void *kv_win;      // token rows [B, win_rows, c] (row r = token win_tok0 + r); ring [B, w, c]
+  int win_tok0, win_rows;  // token-indexed window: first token and rows per sequence
   const float *sink;       // [n_h]
   void *o;                 // [B, n_q, n_h, c]
   hca_dtype dtype;
@@ -178,6 +183,7 @@ struct RowOpParams {
   int rows, cols;
   int norm; const float *gamma; float eps;
   int rd; float theta; long long pos0; int rows_per_pos; int pos_mod;
+  long long pos_base;   // RoPE position = pos_base + (pos0 + row / rows_per_pos) % pos_mod
   float scale;
 };
 int launch_row_op(const RowOpParams &p, cudaStream_t s);

@@ -257,6 +257,223 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
   return hca_attend(&ad, P.q, P.kvw, 1, P.kvw, 0, L->sink, n, 0, o, nullptr, 0, stream);
 }
 
+// ----------------------------------------------------------- context parallel
+// A rank's share of a context-parallel prefill: tokens [t0, t0 + n_loc) of
+// every sequence, with h = hybrid_cp_halo(L, t0) rows of the previous tokens.
+namespace {
+int cp_block_halo(const hca_layer *L) {
+  return (L->kind == HCA_LAYER_CSA && L->a.overlap) ? L->a.m : 0;
+}
+int cp_check(const hca_layer *L, const void *H, int t0, int n_loc) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  if (!H) return fail(HCA_ERR_INVALID, "H must be non-null");
+  if (t0 < 0 || n_loc < 1) return fail(HCA_ERR_INVALID, "t0 must be >= 0 and n_loc >= 1");
+  if (L->kind == HCA_LAYER_SWA) return fail(HCA_ERR_UNSUPPORTED, "context-parallel prefill needs a compressed layer");
+  if (t0 % a.m) return fail(HCA_ERR_INVALID, "t0 (%d) must start a compression block (m = %d)", t0, a.m);
+  if (cp_block_halo(L) > 0 && a.w - 1 < cp_block_halo(L))
+    return fail(HCA_ERR_UNSUPPORTED, "the window (w = %d) must cover the overlap block (m = %d)", a.w, a.m);
+  if (L->d < 8 || L->d_c < 8) return fail(HCA_ERR_INVALID, "d and d_c must be >= 8");
+  return HCA_OK;
+}
+struct CpPlan {
+  void *CZ, *CZI, *cQ32, *cQ, *q32, *q, *qI32, *qI, *wI, *kv32, *kvw, *idx, *topk_ws;
+  size_t topk_bytes, total;
+  int qchunk;
+};
+void plan_cp(const hca_layer *L, int t0, int n_loc, void *ws, CpPlan &P) {
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA;
+  const int h = hybrid_cp_halo(L, t0);
+  const long long R = (long long)a.B * (h + n_loc);   // rows with the halo
+  const long long T = (long long)a.B * n_loc;         // the rank's own rows
+  const size_t es = esize(a.dtype);
+  Carver cv(ws);
+  P.CZ = cv.take(R * (csa ? 4 : 2) * a.c * 4);
+  P.CZI = csa ? cv.take(R * 4 * a.c_I * 4) : nullptr;
+  P.cQ32 = cv.take(T * L->d_c * 4);
+  P.cQ = cv.take(T * L->d_c * es);
+  P.qchunk = (int)(n_loc < 8192 ? n_loc : 8192);
+  P.q32 = cv.take((size_t)P.qchunk * a.n_h * a.c * 4);
+  P.q = cv.take(T * a.n_h * a.c * es);
+  P.qI32 = csa ? cv.take(T * a.n_hI * a.c_I * 4) : nullptr;
+  P.qI = csa ? cv.take(T * a.n_hI * a.c_I * es) : nullptr;
+  P.wI = csa ? cv.take(T * a.n_hI * 4) : nullptr;
+  P.kv32 = cv.take(R * a.c * 4);
+  P.kvw = cv.take(R * a.c * es);
+  P.idx = csa ? cv.take(T * a.k * 4) : nullptr;
+  P.topk_bytes = 0;
+  if (csa) {
+    IndexParams ip{};
+    ip.B = a.B; ip.n_q = n_loc; ip.start_pos = t0; ip.m = a.m; ip.k = a.k; ip.n_hI = a.n_hI; ip.c_I = a.c_I;
+    P.topk_bytes = topk_workspace_bytes(ip);
+  }
+  P.topk_ws = P.topk_bytes ? cv.take(P.topk_bytes) : nullptr;
+  P.total = cv.off;
+}
+// Entries of the rank's complete blocks from the projected C/Z rows (with the
+// halo): rows start at token t0 - h; the compression reads from t0 - hb (the
+// previous block, whose b series the first entry needs) and writes entries
+// t0/m .. (t0 + n_loc)/m - 1 to out slots 0 ...
+int cp_compress_series(const hca_layer *L, int t0, int n_loc, int h, const float *CZ, int width, int ncz,
+                       const float *Bias, hca_dtype out_dt, int rd, void *out, float *out_scale, long long out_cap,
+                       cudaStream_t s) {
+  const hca_attn_desc &a = L->a;
+  const bool ov = L->kind == HCA_LAYER_CSA && a.overlap;
+  const int hb = (ov && t0 > 0) ? a.m : 0;
+  hca_compress_desc cd{};
+  cd.B = a.B; cd.width = width; cd.m = a.m; cd.overlap = ov ? 1 : 0; cd.rd = rd;
+  cd.flags = HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE; cd.eps = eps_of(a); cd.rope_theta = rope_theta(a);
+  cd.in_dtype = HCA_F32; cd.out_dtype = out_dt;
+  const long long rs = (long long)ncz * width;
+  const float *base = CZ + (long long)(h - hb) * rs;
+  // column blocks: CSA [Ca | Cb | Za | Zb]; HCA [C | Z]
+  const float *Ca = base, *Cb = ov ? base + width : nullptr;
+  const float *Za = base + (ov ? 2 : 1) * width, *Zb = ov ? base + 3 * width : nullptr;
+  CompressParams p{};
+  int rc = compress_params(&cd, 0, hb + n_loc, Ca, Cb, Za, Zb, rs, rs * (h + n_loc), Bias,
+                           ov ? Bias + a.m * width : nullptr, nullptr, out, out_scale, out_cap, nullptr, nullptr, &p);
+  if (rc) return rc;
+  p.e_first = hb / a.m;
+  p.e_pos0 = (t0 - hb) / a.m;
+  return launch_compress_prefill(p, s);
+}
+}  // namespace
+
+int hybrid_cp_halo(const hca_layer *L, int t0) {
+  if (!L || t0 <= 0) return 0;
+  const int need = L->a.w - 1 > cp_block_halo(L) ? L->a.w - 1 : cp_block_halo(L);
+  return need < t0 ? need : t0;
+}
+
+size_t hybrid_cp_workspace_size(const hca_layer *L, int t0, int n_loc) {
+  if (check_layer(L) || t0 < 0 || n_loc < 1) return 0;
+  CpPlan P{};
+  plan_cp(L, t0, n_loc, nullptr, P);
+  return P.total;
+}
+
+int hybrid_cp_compress(const hca_layer *L, const void *H, int t0, int n_loc, void *kv_comp, void *key_I,
+                       float *key_I_scale, int out_cap, void *ws, size_t ws_bytes, hca_stream_t stream) {
+  int rc = cp_check(L, H, t0, n_loc);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA;
+  const int E_loc = n_loc / a.m;
+  if (!L->W_comp || !L->B_comp || (csa && (!L->W_compI || !L->B_compI))) return fail(HCA_ERR_INVALID, "missing layer weight");
+  if (E_loc > 0 && (!kv_comp || (csa && !key_I))) return fail(HCA_ERR_INVALID, "kv_comp and key_I must be non-null");
+  if (out_cap < E_loc) return fail(HCA_ERR_INVALID, "out_cap (%d) < entries of the range (%d)", out_cap, E_loc);
+  if (csa && a.idx_key_dtype == HCA_FP8E4M3 && !key_I_scale) return fail(HCA_ERR_INVALID, "fp8 keys need key_I_scale");
+  CpPlan P{};
+  plan_cp(L, t0, n_loc, nullptr, P);
+  if (!ws || ws_bytes < P.total) return fail(HCA_ERR_INVALID, "workspace too small (%zu < %zu)", ws_bytes, P.total);
+  plan_cp(L, t0, n_loc, ws, P);
+  if (E_loc == 0) return HCA_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int h = hybrid_cp_halo(L, t0);
+  const int R = a.B * (h + n_loc);
+  const int ncz = csa ? 4 : 2;
+  rc = launch_gemm(a.dtype, H, L->d, L->W_comp, L->d, P.CZ, (long long)ncz * a.c, HCA_F32, R, ncz * a.c, L->d, 1.f, s);
+  if (rc) return rc;
+  rc = cp_compress_series(L, t0, n_loc, h, static_cast<const float *>(P.CZ), a.c, ncz, L->B_comp, a.dtype, a.rd,
+                          kv_comp, nullptr, out_cap, s);
+  if (rc || !csa) return rc;
+  rc = launch_gemm(a.dtype, H, L->d, L->W_compI, L->d, P.CZI, 4LL * a.c_I, HCA_F32, R, 4 * a.c_I, L->d, 1.f, s);
+  if (rc) return rc;
+  return cp_compress_series(L, t0, n_loc, h, static_cast<const float *>(P.CZI), a.c_I, 4, L->B_compI, a.idx_key_dtype,
+                            a.rd_I, key_I, key_I_scale, out_cap, s);
+}
+
+int hybrid_cp_attend(const hca_layer *L, const void *H, int t0, int n_loc, const void *kv_comp, const void *key_I,
+                     const float *key_I_scale, int cap, void *o, void *ws, size_t ws_bytes, hca_stream_t stream) {
+  int rc = cp_check(L, H, t0, n_loc);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA;
+  if (!o) return fail(HCA_ERR_INVALID, "o must be non-null");
+  if (!L->W_DQ || !L->W_UQ || !L->W_KV || (csa && (!L->W_IUQ || !L->W_w))) return fail(HCA_ERR_INVALID, "missing layer weight");
+  const int Vmax = (t0 + n_loc) / a.m;
+  if (cap < Vmax) return fail(HCA_ERR_INVALID, "cap (%d) < entries visible to the range (%d)", cap, Vmax);
+  if (Vmax > 0 && (!kv_comp || (csa && !key_I))) return fail(HCA_ERR_INVALID, "kv_comp and key_I must be non-null");
+  CpPlan P{};
+  plan_cp(L, t0, n_loc, nullptr, P);
+  if (!ws || ws_bytes < P.total) return fail(HCA_ERR_INVALID, "workspace too small (%zu < %zu)", ws_bytes, P.total);
+  plan_cp(L, t0, n_loc, ws, P);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const hca_dtype dt = a.dtype;
+  const size_t es = esize(dt);
+  const float theta = rope_theta(a), eps = eps_of(a);
+  const int h = hybrid_cp_halo(L, t0);
+  const char *Hb = static_cast<const char *>(H);
+  const long long hrow = (long long)L->d * es;
+  // ---- queries of the rank's own tokens (per sequence: its rows follow the halo)
+  for (int b = 0; b < a.B; ++b) {
+    rc = launch_gemm(dt, Hb + ((long long)b * (h + n_loc) + h) * hrow, L->d, L->W_DQ, L->d,
+                     static_cast<float *>(P.cQ32) + (long long)b * n_loc * L->d_c, L->d_c, HCA_F32, n_loc, L->d_c, L->d,
+                     1.f, s);
+    if (rc) return rc;
+  }
+  const long long T = (long long)a.B * n_loc;
+  {
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.cQ32); r.in_stride = L->d_c; r.out = P.cQ; r.out_stride = L->d_c;
+    r.out_dtype = dt; r.rows = (int)T; r.cols = L->d_c; r.norm = 1; r.eps = eps; r.rd = 0; r.theta = theta;
+    r.rows_per_pos = 1; r.pos_mod = n_loc; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  const int HC = a.n_h * a.c;
+  for (long long r0 = 0; r0 < T; r0 += P.qchunk) {
+    const int rows = (int)((T - r0) < P.qchunk ? (T - r0) : P.qchunk);
+    rc = launch_gemm(dt, static_cast<const char *>(P.cQ) + r0 * L->d_c * es, L->d_c, L->W_UQ, L->d_c, P.q32, HC,
+                     HCA_F32, rows, HC, L->d_c, 1.f, s);
+    if (rc) return rc;
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.q32); r.in_stride = a.c;
+    r.out = static_cast<char *>(P.q) + r0 * HC * es; r.out_stride = a.c; r.out_dtype = dt;
+    r.rows = rows * a.n_h; r.cols = a.c; r.norm = 1; r.eps = eps; r.rd = a.rd; r.theta = theta;
+    r.pos0 = r0 % n_loc; r.rows_per_pos = a.n_h; r.pos_mod = n_loc; r.pos_base = t0; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  if (csa) {
+    const int HI = a.n_hI * a.c_I;
+    rc = launch_gemm(dt, P.cQ, L->d_c, L->W_IUQ, L->d_c, P.qI32, HI, HCA_F32, (int)T, HI, L->d_c, 1.f, s);
+    if (rc) return rc;
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.qI32); r.in_stride = a.c_I; r.out = P.qI; r.out_stride = a.c_I;
+    r.out_dtype = dt; r.rows = (int)T * a.n_hI; r.cols = a.c_I; r.norm = 0; r.rd = a.rd_I; r.theta = theta;
+    r.rows_per_pos = a.n_hI; r.pos_mod = n_loc; r.pos_base = t0; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+    const float wscale = 1.0f / sqrtf((float)a.c_I) / sqrtf((float)a.n_hI);
+    for (int b = 0; b < a.B; ++b) {
+      rc = launch_gemm(dt, Hb + ((long long)b * (h + n_loc) + h) * hrow, L->d, L->W_w, L->d,
+                       static_cast<float *>(P.wI) + (long long)b * n_loc * a.n_hI, a.n_hI, HCA_F32, n_loc, a.n_hI,
+                       L->d, wscale, s);
+      if (rc) return rc;
+    }
+  }
+  // ---- window rows of the halo and the rank's tokens: [B, h + n_loc, c] at tokens t0 - h ..
+  const int R = a.B * (h + n_loc);
+  rc = launch_gemm(dt, H, L->d, L->W_KV, L->d, P.kv32, a.c, HCA_F32, R, a.c, L->d, 1.f, s);
+  if (rc) return rc;
+  {
+    RowOpParams r{};
+    r.in = static_cast<const float *>(P.kv32); r.in_stride = a.c; r.out = P.kvw; r.out_stride = a.c;
+    r.out_dtype = dt; r.rows = R; r.cols = a.c; r.norm = 1; r.eps = eps; r.rd = a.rd; r.theta = theta;
+    r.rows_per_pos = 1; r.pos_mod = h + n_loc; r.pos_base = t0 - h; r.scale = 1.f;
+    if ((rc = launch_row_op(r, s))) return rc;
+  }
+  // ---- select and attend against the gathered caches
+  if (csa) {
+    rc = csa_index_topk(&a, P.qI, static_cast<const float *>(P.wI), key_I, key_I_scale, cap, n_loc, t0,
+                        static_cast<int32_t *>(P.idx), nullptr, 0, P.topk_ws, P.topk_bytes, stream);
+    if (rc) return rc;
+    return csa_attend(&a, P.q, kv_comp, cap, static_cast<const int32_t *>(P.idx), P.kvw, 0, L->sink, n_loc, t0, o,
+                      nullptr, 0, stream);
+  }
+  return hca_attend(&a, P.q, kv_comp, cap, P.kvw, 0, L->sink, n_loc, t0, o, nullptr, 0, stream);
+}
+
 int hybrid_workspace_map(const hca_layer *L, int n, int decode, hca_ws_map *map) {
   int rc = check_layer(L);
   if (rc) return rc;

@@ -64,8 +64,6 @@ def test_attend_rejects_bad_arguments(L):
     _bad(L.hca_attend(ctypes.byref(d), 16, 16, 1, 16, 0, 16, 64, 0, 16, None, 0, None), "cap")
     # ring window with several queries
     _bad(L.hca_attend(ctypes.byref(d), 16, 16, 100, 16, 1, 16, 4, 0, 16, None, 0, None), "ring")
-    # token-indexed window at start_pos > 0
-    _bad(L.hca_attend(ctypes.byref(d), 16, 16, 100, 16, 0, 16, 1, 9, 16, None, 0, None), "start_pos")
     dbad = hb.attn_desc(1, 4, 48, 16, 8, 4, k=4)
     _bad(L.hca_attend(ctypes.byref(dbad), 16, 16, 100, 16, 0, 16, 4, 0, 16, None, 0, None), "multiple of 32")
     _bad(L.csa_attend(ctypes.byref(d), 16, 16, 100, None, 16, 0, 16, 4, 0, 16, None, 0, None), "idx")
