@@ -57,7 +57,13 @@ enum {
   HCA_ERR_TIMEOUT = -4      /* a bounded device wait expired */
 };
 
-typedef enum { HCA_F32 = 0, HCA_BF16 = 1, HCA_FP8E4M3 = 2 } hca_dtype;
+/* HCA_FP4: the FP4 indexer path ([J] §4.4; [Z] Indexer) -- indexer keys that
+ * are Hadamard-rotated and FP4-quantised (E2M1, one power-of-two scale per 32
+ * values, see hca_fp4_rotate_quant), carried exactly as bf16 values.  As an
+ * idx_key_dtype it also rotates and quantises q^I inside csa_index_topk and
+ * rounds the index scores to bf16 before the selection; as a compressor
+ * out_dtype (width 64) the entries are rotated and quantised when written. */
+typedef enum { HCA_F32 = 0, HCA_BF16 = 1, HCA_FP8E4M3 = 2, HCA_FP4 = 3 } hca_dtype;
 
 /* ------------------------------------------------------------------------
  * Attention-layer shape.  Query i of a call sits at position start_pos + i.
@@ -107,7 +113,7 @@ typedef struct {
   int flags;           /* HCA_COMPRESS_NORM | HCA_COMPRESS_ROPE */
   float eps, rope_theta;
   hca_dtype in_dtype;  /* C and Z rows: HCA_F32 or HCA_BF16 */
-  hca_dtype out_dtype; /* entries: HCA_F32, HCA_BF16 or HCA_FP8E4M3 */
+  hca_dtype out_dtype; /* entries: HCA_F32, HCA_BF16, HCA_FP8E4M3 or HCA_FP4 (width 64) */
 } hca_compress_desc;
 
 /* csa_compress -- two modes:
@@ -149,6 +155,10 @@ int hca_compress(const hca_compress_desc *d, int start_pos, int n,
  *   fp32 (already scaled), KI [B, cap, c_I] (idx_key_dtype), KI_scale
  *   [B, cap] fp32 row scales for fp8 keys (else NULL).
  * idx [B, n_q, k]: kept entry indices in ascending order, then -1.
+ * idx_key_dtype HCA_FP4 (c_I = 64): KI holds rotated FP4 keys (bf16 storage,
+ *   as csa_compress writes them); q^I is rotated and FP4-quantised in ws, the
+ *   scores are rounded to bf16 (nearest, ties to even) before the selection
+ *   (ties still to the lower index) and in the optional scores output.
  * scores (optional, NULL to skip): fp32 [B, n_q, score_stride] with the
  *   index scores of the visible entries (score_stride >= max V_t).
  * Requires (start_pos + n_q) / m <= cap. */

@@ -16,7 +16,7 @@ LIB_PATH = os.path.join(HERE, "libhca.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "hca.h")
 
 HCA_OK, HCA_ERR_INVALID, HCA_ERR_UNSUPPORTED, HCA_ERR_CUDA, HCA_ERR_TIMEOUT = 0, -1, -2, -3, -4
-HCA_F32, HCA_BF16, HCA_FP8E4M3 = 0, 1, 2
+HCA_F32, HCA_BF16, HCA_FP8E4M3, HCA_FP4 = 0, 1, 2, 3
 HCA_COMPRESS_NORM, HCA_COMPRESS_ROPE = 1, 2
 HCA_LAYER_CSA, HCA_LAYER_HCA, HCA_LAYER_SWA = 0, 1, 2
 # HCA_STATIC_SCRATCH_BYTES of include/hca.h; lib() checks that the loaded library agrees.

@@ -143,7 +143,7 @@ int num_sms() {
 
 namespace {
 
-size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : (t == HCA_BF16 ? 2 : 1); }
+size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : ((t == HCA_BF16 || t == HCA_FP4) ? 2 : 1); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
@@ -166,8 +166,10 @@ int check_attn_desc(const hca_attn_desc *d, bool need_indexer) {
     REQUIRE(d->k >= 1, "k must be >= 1");
     REQUIRE(d->n_hI >= 1 && d->c_I >= 8 && d->c_I % 8 == 0, "indexer heads / dim invalid");
     REQUIRE(d->rd_I >= 0 && d->rd_I <= d->c_I && d->rd_I % 2 == 0, "rd_I must be even and <= c_I");
-    REQUIRE(d->idx_key_dtype == HCA_F32 || d->idx_key_dtype == HCA_BF16 || d->idx_key_dtype == HCA_FP8E4M3,
+    REQUIRE(d->idx_key_dtype == HCA_F32 || d->idx_key_dtype == HCA_BF16 || d->idx_key_dtype == HCA_FP8E4M3 ||
+                d->idx_key_dtype == HCA_FP4,
             "idx_key_dtype invalid");
+    REQUIRE(d->idx_key_dtype != HCA_FP4 || d->c_I == 64, "the FP4 indexer path needs c_I == 64");
   }
   return HCA_OK;
 }
@@ -227,7 +229,9 @@ int compress_params(const hca_compress_desc *d, int start_pos, int n, const void
   REQUIRE(d->width >= 8 && d->width % 8 == 0, "width must be a positive multiple of 8");
   REQUIRE(d->overlap == 0 || d->overlap == 1, "overlap must be 0 or 1");
   REQUIRE(d->in_dtype == HCA_F32 || d->in_dtype == HCA_BF16, "in_dtype must be f32 or bf16");
-  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16 || d->out_dtype == HCA_FP8E4M3, "bad out_dtype");
+  REQUIRE(d->out_dtype == HCA_F32 || d->out_dtype == HCA_BF16 || d->out_dtype == HCA_FP8E4M3 ||
+              d->out_dtype == HCA_FP4, "bad out_dtype");
+  REQUIRE(d->out_dtype != HCA_FP4 || d->width == 64, "FP4 entries need width 64");
   if (d->flags & HCA_COMPRESS_ROPE)
     REQUIRE(d->rd >= 0 && d->rd <= d->width && d->rd % 8 == 0, "rd must be a multiple of 8 and <= width");
   REQUIRE(n >= 0 && start_pos >= 0, "n and start_pos must be >= 0");

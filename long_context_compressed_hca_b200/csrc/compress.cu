@@ -394,9 +394,19 @@ int launch_decode_t(const CompressParams &p, int pos, cudaStream_t s) {
 
 }  // namespace
 
-int launch_compress_prefill(const CompressParams &p, cudaStream_t s) {
-  return p.in_dtype == HCA_F32 ? launch_prefill_t<float>(p, s)
-                               : launch_prefill_t<__nv_bfloat16>(p, s);
+// FP4 keys (HCA_FP4): the entries are written in bf16 and then rotated and
+// FP4-quantised in place (Hadamard, blocks of 32; width 64).
+int launch_decode_ingest_t(const CompressParams *pa, const CompressParams *pb, CompressParams a, CompressParams bb,
+                           const IngestRing &ring, int B, int pos, cudaStream_t s);
+
+int launch_compress_prefill(const CompressParams &p0, cudaStream_t s) {
+  CompressParams p = p0;
+  if (p.out_dtype == HCA_FP4) p.out_dtype = HCA_BF16;
+  const int rc = p.in_dtype == HCA_F32 ? launch_prefill_t<float>(p, s) : launch_prefill_t<__nv_bfloat16>(p, s);
+  if (rc || p0.out_dtype != HCA_FP4) return rc;
+  const long long E = p.n / p.m - p.e_first;
+  if (E <= 0) return HCA_OK;
+  return launch_fp4_rotate_quant(p.out, HCA_BF16, (long long)p.B * E, p.out, s, E, p.out_seq_stride);
 }
 
 int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s) {
@@ -409,9 +419,14 @@ int launch_compress_state_prefill(const CompressParams &p, cudaStream_t s) {
   return ls_.done();
 }
 
-int launch_compress_decode(const CompressParams &p, int pos, cudaStream_t s) {
-  return p.in_dtype == HCA_F32 ? launch_decode_t<float>(p, pos, s)
-                               : launch_decode_t<__nv_bfloat16>(p, pos, s);
+int launch_compress_decode(const CompressParams &p0, int pos, cudaStream_t s) {
+  CompressParams p = p0;
+  if (p.out_dtype == HCA_FP4) p.out_dtype = HCA_BF16;
+  const int rc = p.in_dtype == HCA_F32 ? launch_decode_t<float>(p, pos, s) : launch_decode_t<__nv_bfloat16>(p, pos, s);
+  if (rc || p0.out_dtype != HCA_FP4 || (pos + 1) % p.m != 0) return rc;
+  // the entry this token completed, one row per sequence
+  void *row = static_cast<__nv_bfloat16 *>(p.out) + (long long)(pos / p.m) * p.width;
+  return launch_fp4_rotate_quant(row, HCA_BF16, p.B, row, s, 1, p.out_seq_stride);
 }
 
 int launch_decode_ingest(const CompressParams *pa, const CompressParams *pb, const IngestRing &ring, int B, int pos,
@@ -420,6 +435,18 @@ int launch_decode_ingest(const CompressParams *pa, const CompressParams *pb, con
   if (parts == 0 || B == 0) return HCA_OK;
   CompressParams a = pa ? *pa : CompressParams{};
   CompressParams bb = pb ? *pb : CompressParams{};
+  // FP4 indexer keys: the emitted key is written in bf16, then rotated and
+  // FP4-quantised in place by a second launch (emitting steps only)
+  const bool fp4 = pb && bb.out_dtype == HCA_FP4;
+  if (fp4) bb.out_dtype = HCA_BF16;
+  const int rc = launch_decode_ingest_t(pa ? &a : nullptr, pb ? &bb : nullptr, a, bb, ring, B, pos, s);
+  if (rc || !fp4 || (pos + 1) % bb.m != 0) return rc;
+  void *row = static_cast<__nv_bfloat16 *>(bb.out) + (long long)(pos / bb.m) * bb.width;
+  return launch_fp4_rotate_quant(row, HCA_BF16, B, row, s, 1, bb.out_seq_stride);
+}
+
+int launch_decode_ingest_t(const CompressParams *pa, const CompressParams *pb, CompressParams a, CompressParams bb,
+                           const IngestRing &ring, int B, int pos, cudaStream_t s) {
   if (!pa) a.B = 0;
   // part indices: 0 = main (may be empty), 1 = indexer (may be absent), last = ring
   const int ny = pb ? (ring.ring ? 3 : 2) : (ring.ring ? 2 : 1);

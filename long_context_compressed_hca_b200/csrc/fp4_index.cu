@@ -59,12 +59,18 @@ __device__ __forceinline__ float e2m1_round(float q) {
   return r == 0.0f ? 0.0f : copysignf(r, q);   // zero is stored as +0
 }
 
+// Row r of `rows` sits at row (r / per_seq) * seq_rows + r % per_seq of x and
+// out (rows of 64 values; per_seq = rows and seq_rows = 0 for dense rows).
+// x and out may be the same buffer: a warp reads its whole row before it
+// writes it.
 template <typename T>
-__global__ void __launch_bounds__(kFp4Warps * 32) fp4_rotate_quant_kernel(const T *__restrict__ x, long long rows,
-                                                                            __nv_bfloat16 *__restrict__ out) {
+__global__ void __launch_bounds__(kFp4Warps * 32) fp4_rotate_quant_kernel(const T *x, long long rows,
+                                                                            long long per_seq, long long seq_rows,
+                                                                            __nv_bfloat16 *out) {
   const int lane = threadIdx.x & 31;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+  for (long long r0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r0 < rows; r0 += nwarps) {
+    const long long r = (r0 / per_seq) * seq_rows + r0 % per_seq;
     float a, b;
     load2(x + r * 64 + 2 * lane, a, b);
     // stride 1: the lane's own pair
@@ -103,18 +109,20 @@ __global__ void __launch_bounds__(kFp4Warps * 32) fp4_rotate_quant_kernel(const 
 
 }  // namespace
 
-int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s) {
+int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s,
+                            long long per_seq, long long seq_rows) {
   if (rows == 0) return HCA_OK;
+  if (per_seq <= 0) { per_seq = rows; seq_rows = 0; }
   const long long blocks = (rows + kFp4Warps - 1) / kFp4Warps;
   const int grid = (int)(blocks < (long long)num_sms() * 16 ? blocks : (long long)num_sms() * 16);
   __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
   if (dt == HCA_F32)
     return HCA_LAUNCH("fp4_rotate_quant", s,
                       fp4_rotate_quant_kernel<float><<<grid, kFp4Warps * 32, 0, s>>>(
-                          static_cast<const float *>(x), rows, o));
+                          static_cast<const float *>(x), rows, per_seq, seq_rows, o));
   return HCA_LAUNCH("fp4_rotate_quant", s,
                     fp4_rotate_quant_kernel<__nv_bfloat16><<<grid, kFp4Warps * 32, 0, s>>>(
-                        static_cast<const __nv_bfloat16 *>(x), rows, o));
+                        static_cast<const __nv_bfloat16 *>(x), rows, per_seq, seq_rows, o));
 }
 
 }  // namespace hca

@@ -30,6 +30,7 @@ struct TcIdxArgs {
   float *scores;
   long long score_stride;
   int *status;
+  int round_bf16;
 };
 
 template <int N, bool FP8, int S>
@@ -180,8 +181,10 @@ index_scores_tc(TcIdxArgs p, const __grid_constant__ CUtensorMap tmK, const __gr
 #pragma unroll
             for (int x = 0; x < 8; ++x) sacc += wsm[jq * 8 + x] * fmaxf(__uint_as_float(r[x]), 0.f);
             const int t = p.start_pos + q0 + jq;
+            float v = sacc * kscale;
+            if (p.round_bf16) v = __bfloat162float(__float2bfloat16_rn(v));
             if (e < e_end && e < (t + 1) / p.m)
-              p.scores[((long long)b * p.n_q + q0 + jq) * p.score_stride + e] = sacc * kscale;
+              p.scores[((long long)b * p.n_q + q0 + jq) * p.score_stride + e] = v;
           }
         }
         tc_fence_before();
@@ -258,6 +261,7 @@ int launch_tc_t(const IndexParams &p, int QB, int tiles_per_unit, int units_per_
   a.B = p.B; a.n_q = p.n_q; a.start_pos = p.start_pos; a.m = p.m; a.n_hI = p.n_hI; a.cap = p.cap; a.QB = QB;
   a.tiles_per_unit = tiles_per_unit; a.units_per_qb = units_per_qb; a.n_qb = (p.n_q + QB - 1) / QB;
   a.wI = p.wI; a.KI_scale = p.KI_scale; a.scores = p.scores; a.score_stride = p.score_stride; a.status = p.status;
+  a.round_bf16 = p.round_bf16;
   const long long grid = (long long)p.B * a.n_qb * units_per_qb;
   LaunchScope ls_(FP8 ? "index_scores_tc_fp8" : "index_scores_tc", s);
   cudaLaunchConfig_t cfg{};

@@ -69,8 +69,9 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
   }
   for (int j = 0; j < nq; ++j) {
     const int t = p.start_pos + q0 + j;
-    if (s < (t + 1) / p.m)
-      p.scores[((long long)b * p.n_q + q0 + j) * p.score_stride + s] = acc[j] * kscale;
+    float v = acc[j] * kscale;
+    if (p.round_bf16) v = __bfloat162float(__float2bfloat16_rn(v));
+    if (s < (t + 1) / p.m) p.scores[((long long)b * p.n_q + q0 + j) * p.score_stride + s] = v;
   }
 }
 
@@ -578,33 +579,47 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       // thresholds at the bin edges: above t_hi = winners, [t_lo, t_hi] = band
       const float t_hi = lo + (float)(b_hi + 1) / scale;
       const float t_lo = lo + (float)b_lo / scale;
-      // ---- 2. one pass over the row
-      int above = 0;
-      const unsigned lt = (1u << lane) - 1u;
+      // ---- 2. one pass over the row: count, then place (no per-key votes)
+      int above = 0, inband = 0;
 #pragma unroll
-      for (int j = 0; j < kRowRegs; ++j) {
+      for (int j = 0; j < kRowRegs; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int i = 4 * tid + 4 * NT * j + e;
-          const bool valid = i < V;
+          const bool valid = 4 * tid + 4 * NT * j + e < V;
           const float v = x[j][e];
-          const bool up = valid && v > t_hi;
-          const bool inb = valid && !up && v >= t_lo;
-          const unsigned bu = __ballot_sync(0xffffffffu, up);
-          above += __popc(bu);
-          if (up) atomicOr(&win[i >> 5], 1u << (i & 31));
-          const unsigned bb = __ballot_sync(0xffffffffu, inb);
-          if (bb) {
-            int at = 0;
-            if (lane == 0) at = atomicAdd(&sh.s_nc, __popc(bb));
-            at = __shfl_sync(0xffffffffu, at, 0) + __popc(bb & lt);
-            if (inb && at < kRowCand) {
-              band_key[at] = order_bits(__float_as_uint(v));
-              band_idx[at] = (uint32_t)i;
+          above += (valid && v > t_hi) ? 1 : 0;
+          inband += (valid && v <= t_hi && v >= t_lo) ? 1 : 0;
+        }
+      // band slots: warp-inclusive scan of the per-thread counts, one atomic per warp
+      int incl = inband;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int wbase = 0;
+      if (lane == 31 && incl) wbase = atomicAdd(&sh.s_nc, incl);
+      int at = __shfl_sync(0xffffffffu, wbase, 31) + incl - inband;
+      if (above | inband) {
+#pragma unroll
+        for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 4 * tid + 4 * NT * j + e;
+            const float v = x[j][e];
+            if (i < V && v > t_hi) {
+              atomicOr(&win[i >> 5], 1u << (i & 31));
+            } else if (i < V && v >= t_lo) {
+              if (at < kRowCand) {
+                band_key[at] = order_bits(__float_as_uint(v));
+                band_idx[at] = (uint32_t)i;
+              }
+              ++at;
             }
           }
-        }
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
       if (lane == 0) atomicAdd(&sh.s_above, above);
       __syncthreads();
       const int na = sh.s_above, nc = sh.s_nc;
@@ -844,17 +859,22 @@ int launch_index_scores(const IndexParams &p, cudaStream_t s) {
 }
 
 
+// FP4 path: the rotated, quantised q^I (bf16) after everything else.
+size_t fp4_q_bytes(const IndexParams &p) {
+  return p.key_dtype == HCA_FP4 ? (((size_t)p.B * p.n_q * p.n_hI * 64 * 2 + 255) & ~(size_t)255) : 0;
+}
+
 size_t topk_workspace_bytes(const IndexParams &p) {
   const long long rows = (long long)p.B * p.n_q;
   const long long Vmax = (p.start_pos + p.n_q) / p.m;
   const TopkPlan pl = plan_topk(rows, Vmax);
   size_t b = (size_t)rows * (size_t)Vmax * sizeof(float);           // scores
   b = (b + 255) & ~(size_t)255;
-  if (pl.n_seg > 1) {
+  if (pl.n_seg > 1 && !(Vmax <= kRowMax && g_topk_row_enabled)) {
     const size_t c = (size_t)rows * pl.n_seg * p.k;
     b += 2 * ((c * sizeof(int32_t) + 255) & ~(size_t)255);          // winners' indices and keys
   }
-  return b;
+  return b + fp4_q_bytes(p);
 }
 
 int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long long user_stride,
@@ -874,6 +894,18 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   size_t off = ((size_t)rows * (size_t)Vmax * sizeof(float) + 255) & ~(size_t)255;
   int rc = ensure_topk_smem();
   if (rc) return rc;
+  if (ip.key_dtype == HCA_FP4) {
+    // FP4 path: rotate and quantise q^I into the end of the workspace, then
+    // score the exact bf16 images of both FP4 operands and round to bf16
+    const size_t qb = fp4_q_bytes(ip);
+    __nv_bfloat16 *q4 = reinterpret_cast<__nv_bfloat16 *>(w + topk_workspace_bytes(ip) - qb);
+    rc = launch_fp4_rotate_quant(ip.qI, ip.q_dtype, (long long)ip.B * ip.n_q * ip.n_hI, q4, s);
+    if (rc) return rc;
+    p.qI = q4;
+    p.q_dtype = HCA_BF16;
+    p.key_dtype = HCA_BF16;
+    p.round_bf16 = 1;
+  }
   rc = launch_index_scores_tc(p, s);
   if (rc == HCA_ERR_UNSUPPORTED) rc = launch_index_scores(p, s);
   if (rc) return rc;

@@ -93,6 +93,7 @@ struct IndexParams {
   float *scores;           // [B, n_q, score_stride]
   long long score_stride;
   int *status;
+  int round_bf16;          // FP4 path: scores rounded to bf16 (nearest even) when written
 };
 int launch_index_scores(const IndexParams &p, cudaStream_t s);
 // tcgen05 scorer; returns HCA_ERR_UNSUPPORTED (launching nothing) for shapes it does not cover.
@@ -122,7 +123,9 @@ int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores
 
 // ------------------------------------------------------------ FP4 indexer
 // Rows of 64: Hadamard rotation, FP4 blocks of 32, written as exact bf16 values.
-int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s);
+// Strided rows: row r at (r / per_seq) * seq_rows + r % per_seq (per_seq <= 0: dense).
+int launch_fp4_rotate_quant(const void *x, hca_dtype dt, long long rows, void *out, cudaStream_t s,
+                            long long per_seq = 0, long long seq_rows = 0);
 // ------------------------------------------------------------- step trace
 // Point the traced kernels of each translation unit at a record buffer (NULL = off).
 int step_trace_set_attend(void *buf, unsigned long long cap);

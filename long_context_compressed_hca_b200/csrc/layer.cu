@@ -18,7 +18,7 @@
 namespace hca {
 namespace {
 
-size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : (t == HCA_BF16 ? 2 : 1); }
+size_t esize(hca_dtype t) { return t == HCA_F32 ? 4 : ((t == HCA_BF16 || t == HCA_FP4) ? 2 : 1); }
 
 struct Carver {
   char *base;
@@ -80,6 +80,7 @@ int plan_prefill(const hca_layer *L, int n, void *ws, Plan &P) {
   if (csa) {
     IndexParams ip{};
     ip.B = a.B; ip.n_q = n; ip.start_pos = 0; ip.m = a.m; ip.k = a.k; ip.n_hI = a.n_hI; ip.c_I = a.c_I;
+    ip.key_dtype = a.idx_key_dtype;
     P.topk_bytes = topk_workspace_bytes(ip);
   }
   P.topk_ws = P.topk_bytes ? cv.take(P.topk_bytes) : nullptr;
@@ -170,7 +171,8 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
   // ---- indexer keys
   void *keyI = P.keyI;
   float *keyIs = nullptr;
-  hca_dtype kdt = dt;
+  // without a cache the keys stay in the workspace in dtype, or FP4 (bf16 storage)
+  hca_dtype kdt = a.idx_key_dtype == HCA_FP4 ? HCA_FP4 : dt;
   if (csa) {
     if (cache) { keyI = cache->key_I; keyIs = cache->key_I_scale; kdt = a.idx_key_dtype; }
     rc = launch_gemm(dt, H, L->d, L->W_compI, L->d, P.CZI, 4LL * a.c_I, HCA_F32, (int)T, 4 * a.c_I, L->d, 1.f, s);
@@ -307,6 +309,7 @@ void plan_cp(const hca_layer *L, int t0, int n_loc, void *ws, CpPlan &P) {
   if (csa) {
     IndexParams ip{};
     ip.B = a.B; ip.n_q = n_loc; ip.start_pos = t0; ip.m = a.m; ip.k = a.k; ip.n_hI = a.n_hI; ip.c_I = a.c_I;
+    ip.key_dtype = a.idx_key_dtype;
     P.topk_bytes = topk_workspace_bytes(ip);
   }
   P.topk_ws = P.topk_bytes ? cv.take(P.topk_bytes) : nullptr;

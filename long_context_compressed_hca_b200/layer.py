@@ -37,7 +37,7 @@ class LayerHandle:
         for nm in ("W_DQ", "W_UQ", "W_KV"):
             self.t[nm] = dev(W[nm], dtype)
         self.t["sink"] = dev(W["sink"], torch.float32)
-        kdt = {"bf16": _code(dtype), "fp8": hb.HCA_FP8E4M3}[idx_key_dtype] if csa else _code(dtype)
+        kdt = {"bf16": _code(dtype), "fp8": hb.HCA_FP8E4M3, "fp4": hb.HCA_FP4}[idx_key_dtype] if csa else _code(dtype)
         self.idx_key_dtype = idx_key_dtype
         self.desc = hb.attn_desc(B, L.n_h, L.c, L.rd, L.w, L.m, overlap=L.overlap, k=L.k,
                                  n_hI=L.n_hI, c_I=L.c_I, rd_I=L.rd_I if csa else 0,
@@ -63,7 +63,8 @@ class CacheHandle:
         self.state_score = torch.full((B, R, Cw), float("-inf"), device=device)
         self.key_I = self.key_I_scale = self.stateI_kv = self.stateI_score = None
         if L.kind == "csa":
-            kdt = torch.uint8 if idx_key_dtype == "fp8" else dtype
+            # fp8: e4m3 bytes + row scales; fp4: rotated FP4 values carried in bf16
+            kdt = torch.uint8 if idx_key_dtype == "fp8" else (torch.bfloat16 if idx_key_dtype == "fp4" else dtype)
             self.key_I = z(B, cap, L.c_I, dt=kdt)
             if idx_key_dtype == "fp8":
                 self.key_I_scale = z(B, cap)
