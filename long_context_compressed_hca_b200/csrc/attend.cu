@@ -277,10 +277,15 @@ constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kThreads = (kSoftmaxWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
 constexpr int kMaxClusterSplits = 8;         // portable cluster size
+// S / P buffers and how many S tiles the MMA issue runs ahead of P.V: with S
+// of tiles j+1 and j+2 queued behind P.V(j-1), the softmax of tile j hides
+// behind two tiles of tensor work
+constexpr int kSP = 3;
+constexpr int kLookahead = 2;
 
 struct Bars {
   uint64_t q_full, q_empty, o_empty, mma_done;
-  uint64_t kv_full[8], kv_empty[8], s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t kv_full[8], kv_empty[8], s_full[3], s_empty[3], p_full[3], pv_done[3];
   uint64_t mg_ready, mg_full;    // cluster merge: peers' buffers free / peers' partials delivered
   uint64_t mg_stage;             // cluster merge: this CTA's blocks staged
 };
@@ -293,14 +298,17 @@ struct Layout {
   static constexpr int NS = (C == 512) ? 3 : (C == 256 ? 6 : 8);
   static constexpr uint32_t kv_off = 0;
   static constexpr uint32_t p_off = kv_off + NS * NKB * kTileBytes;
-  static constexpr uint32_t bar_off = p_off + 2 * kTileBytes;
+  static constexpr uint32_t bar_off = p_off + kSP * kTileBytes;
   static constexpr uint32_t misc_off = bar_off + 512;
   static constexpr uint32_t bytes = misc_off + 2048 + 1024;  // + alignment slack
-  // tensor memory: O in lane-half 0, columns [0, C); in lane-half 1 the S
-  // double buffer at columns [0, 128) and Q (bf16, two per column) at
-  // [q_col, q_col + C/2), the lanes of S as the A operand of S = Q K^T needs
+  // tensor memory: O in lane-half 0, columns [0, C); in lane-half 1 S buffers
+  // 0 and 1 at columns [0, 128), Q (bf16, two per column) at [q_col, q_col +
+  // C/2), the lanes of S as the A operand of S = Q K^T needs, and S buffer 2
+  // after Q
   static constexpr uint32_t tmem_cols = 512;
   static constexpr uint32_t q_col = 2 * KT;
+  static_assert(q_col + C / 2 + KT <= tmem_cols, "S buffers and Q exceed tensor memory");
+  static constexpr __host__ __device__ uint32_t s_col(int b) { return b < 2 ? b * KT : q_col + C / 2; }
 };
 
 // Trace counters (cycles, summed over CTAs) of the tensor-core kernel's waits.
@@ -531,7 +539,7 @@ attend_tc(AttendParams p, int n_units) {
       mbar_init(bar(bars->kv_full[i]), kProdThreads);
       mbar_init(bar(bars->kv_empty[i]), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSP; ++i) {
       mbar_init(bar(bars->s_full[i]), 1);
       mbar_init(bar(bars->s_empty[i]), kSoftmaxWarps);
       mbar_init(bar(bars->p_full[i]), kSoftmaxWarps);
@@ -649,9 +657,9 @@ attend_tc(AttendParams p, int n_units) {
       uint32_t g = 0, iq = 0;
       bool ok = true;
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-        const int st = gg & 1;                 // S / P double buffer
+        const int st = gg % kSP;               // S / P buffer
         const int kst = gg % L::NS;            // key-tile stage
-        if (!twait(bar(bars->p_full[st]), (gg >> 1) & 1, TR_M_PFULL)) return false;
+        if (!twait(bar(bars->p_full[st]), (gg / kSP) & 1, TR_M_PFULL)) return false;
         if (first && !twait(bar(bars->o_empty), (iq & 1) ^ 1, TR_M_OEMPTY)) return false;
         tc_fence_after();
         const uint32_t pa = sbase + L::p_off + st * kTileBytes;
@@ -679,10 +687,14 @@ attend_tc(AttendParams p, int n_units) {
         if (!twait(bar(bars->q_full), iq & 1, TR_M_QFULL)) { ok = false; break; }
         fence_proxy_async();
         tc_fence_after();
+        // S of tile j, then P.V of tile j - kLookahead; the unit's last P.Vs
+        // are issued before the next unit's Q is awaited (its epilogue waits
+        // for them)
+        int npv = 0;                           // P.Vs of this unit issued
         for (int j = 0; j < nt && ok; ++j) {
           const uint32_t gj = g + j;
-          const int st = gj & 1;
-          const uint32_t ph = (gj >> 1) & 1;
+          const int st = gj % kSP;
+          const uint32_t ph = (gj / kSP) & 1;
           const int kst = gj % L::NS;
           if (!twait(bar(bars->kv_full[kst]), (gj / L::NS) & 1, TR_M_KVFULL) ||
               !twait(bar(bars->s_empty[st]), ph ^ 1, TR_M_SEMPTY)) {
@@ -694,16 +706,21 @@ attend_tc(AttendParams p, int n_units) {
           // K descriptor advances by constant offsets (16-byte units in the low
           // field); Q (A operand, tensor memory) by 8 columns = 16 bf16 per step
           const uint64_t kd = sdesc_sw128(sbase + L::kv_off + kst * L::NKB * kTileBytes, 16, 1024);
+          const uint32_t sd = tS + L::s_col(st);
 #pragma unroll
           for (int kk = 0; kk < C / 16; ++kk) {
             const uint64_t off = ((kk / 4) * kTileBytes + (kk % 4) * 32) >> 4;
-            umma_bf16_ts(tS + st * KT, tS + L::q_col + 8 * kk, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+            umma_bf16_ts(sd, tS + L::q_col + 8 * kk, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar(bars->s_full[st]));
           if (j == nt - 1) umma_commit(bar(bars->q_empty));
-          if (j >= 1 && !issue_pv(gj - 1, j - 1 == 0)) ok = false;
+          if (j >= kLookahead) {
+            if (!issue_pv(g + npv, npv == 0)) ok = false;
+            ++npv;
+          }
         }
-        if (ok && !issue_pv(g + nt - 1, nt == 1)) ok = false;
+        for (; ok && npv < nt; ++npv)
+          if (!issue_pv(g + npv, npv == 0)) ok = false;
         g += nt;
         ++iq;
       }
@@ -808,14 +825,14 @@ attend_tc(AttendParams p, int n_units) {
       if (TRACE) { tr[TR_UNITS] += 1; tr[TR_TILES] += nt; }
       for (int j = 0; j < nt; ++j) {
         const uint32_t gj = g + j;
-        const int st = gj & 1;
-        const uint32_t ph = (gj >> 1) & 1;
+        const int st = gj % kSP;
+        const uint32_t ph = (gj / kSP) & 1;
         if (!twait(bar(bars->s_full[st]), ph, TR_S_SFULL)) return;
         if (TRACE && threadIdx.x == 0 && j == 0 && ts[2] == 0) ts[2] = global_ns();
         tc_fence_after();
         uint32_t sv[32];
-        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
-        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + st * KT + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + L::s_col(st), *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld_16x32bx2_x16<32>(tmem + lane_S + L::s_col(st) + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
@@ -853,7 +870,7 @@ attend_tc(AttendParams p, int n_units) {
           // rescale O rows of this warp after the PV of the previous tile lands
           const uint32_t gp = gj - 1;
           if (TRACE) tr[TR_RESCALES] += 1;
-          if (!twait(bar(bars->pv_done[gp & 1]), (gp >> 1) & 1, TR_S_RESCALE)) return;
+          if (!twait(bar(bars->pv_done[gp % kSP]), (gp / kSP) & 1, TR_S_RESCALE)) return;
           tc_fence_after();
 #pragma unroll 1
           for (int c0 = 0; c0 < C / 2; c0 += 16) {
@@ -875,7 +892,7 @@ attend_tc(AttendParams p, int n_units) {
           pk[x / 2] = pack_bf16x2(p0, p1);
         }
         l += psum;
-        // P buffer `st` is free once the PV of tile gj-2 has completed
+        // P buffer `st` is free once the PV of tile gj-3 has completed
         if (!twait(bar(bars->pv_done[st]), ph ^ 1, TR_S_PBUF)) return;
         uint8_t *prow = smem + L::p_off + st * kTileBytes;
 #pragma unroll
@@ -901,7 +918,7 @@ attend_tc(AttendParams p, int n_units) {
       // -------- epilogue: normalise, inverse RoPE, store
       if (nt > 0) {
         const uint32_t gl = g + nt - 1;
-        if (!twait(bar(bars->pv_done[gl & 1]), (gl >> 1) & 1, TR_S_EPI_WAIT)) return;
+        if (!twait(bar(bars->pv_done[gl % kSP]), (gl / kSP) & 1, TR_S_EPI_WAIT)) return;
       }
       if (TRACE && threadIdx.x == 0 && ts[3] == 0) {
         ts[3] = global_ns();
