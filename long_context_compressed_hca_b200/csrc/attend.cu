@@ -277,11 +277,12 @@ constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kThreads = (kSoftmaxWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = 64 * 128;   // 64 rows x 128 B (one 64-column block)
 constexpr int kMaxClusterSplits = 8;         // portable cluster size
-// S / P buffers and how many S tiles the MMA issue runs ahead of P.V: with S
-// of tiles j+1 and j+2 queued behind P.V(j-1), the softmax of tile j hides
-// behind two tiles of tensor work
-constexpr int kSP = 3;
-constexpr int kLookahead = 2;
+// S / P buffers and how many S tiles the MMA issue runs ahead of P.V.  Two
+// tiles ahead measured slower than one (the third key stage then refills only
+// after P.V(j-1) and the gathers stall the tensor pipe), so one: S(j+1) is
+// queued behind P.V(j-1) while the softmax of tile j runs.
+constexpr int kSP = 2;
+constexpr int kLookahead = 1;
 
 struct Bars {
   uint64_t q_full, q_empty, o_empty, mma_done;

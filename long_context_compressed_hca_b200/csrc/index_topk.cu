@@ -743,6 +743,356 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   }
 }
 
+// ------------------------------------------------------ a cluster per row
+// Few long rows (decode): the row is cut over the C CTAs of a thread-block
+// cluster, each holding 32 keys per thread in registers, so that every pass
+// over the keys runs on C SMs.  CTA 0 owns the row's selection state: the
+// others send it their sample keys (step 1), receive the two thresholds
+// (step 2), and send it their band keys and winner bits (step 3) through
+// distributed shared memory; CTA 0 then selects within the band and emits
+// (step 4).  Three cluster barriers in all.  If the band missed the k-th
+// score, CTA 0 selects exactly over the whole row read back from memory.
+__device__ __forceinline__ void st_dsmem_f32(uint32_t a, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_dsmem_u32(uint32_t a, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t atom_add_dsmem_u32(uint32_t a, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(a), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void red_or_dsmem_u32(uint32_t a, uint32_t v) {
+  asm volatile("red.shared::cluster.or.b32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
+}
+
+struct RowcShared {
+  RowSel sh;
+  float thr[2];        // t_hi, t_lo (sent by CTA 0)
+  int band_ok;         // the sample gave thresholds
+  uint32_t base;       // this CTA's first band slot in CTA 0
+  uint32_t red_a[32], red_b[32];
+};
+
+// Emission of CTA 0: winners and the first krem ties of the masks, ascending.
+template <int NT>
+__device__ void emit_masks(RowSel &sh, const uint32_t *win, const uint32_t *tie, int nwords, int krem, int V, int k,
+                           int32_t *out) {
+  const int tid = threadIdx.x;
+  const int wpt = (nwords + NT - 1) / NT;
+  const int w0 = tid * wpt;
+  int my_ties = 0;
+  for (int u = 0; u < wpt; ++u)
+    if (w0 + u < nwords) my_ties += __popc(tie[w0 + u]);
+  int ties_before = block_exclusive_scan<NT>(my_ties, sh.warp_buf, &sh.scan_tot);
+  int my_sel = 0;
+  {
+    int tb = ties_before;
+    for (int u = 0; u < wpt; ++u)
+      if (w0 + u < nwords) {
+        const int nt = __popc(tie[w0 + u]);
+        my_sel += __popc(win[w0 + u]) + max(0, min(nt, krem - tb));
+        tb += nt;
+      }
+  }
+  int at = block_exclusive_scan<NT>(my_sel, sh.warp_buf, &sh.scan_tot);
+  for (int u = 0; u < wpt; ++u) {
+    const int w = w0 + u;
+    if (w >= nwords) break;
+    uint32_t wm = win[w], tm = tie[w];
+    while (wm | tm) {
+      const int bw = wm ? __ffs(wm) - 1 : 32, bt = tm ? __ffs(tm) - 1 : 32;
+      if (bw < bt) {
+        out[at++] = w * 32 + bw;
+        wm &= wm - 1u;
+      } else {
+        if (ties_before < krem) out[at++] = w * 32 + bt;
+        ++ties_before;
+        tm &= tm - 1u;
+      }
+    }
+  }
+  const int K = V < k ? V : k;
+  for (int i = K + tid; i < k; i += NT) out[i] = -1;
+}
+
+// Grid: C CTAs per row, cluster (C,1,1).  Dynamic shared memory: 2 * words +
+// 2 * kRowCand + C * NT words (masks, band, samples; used in CTA 0).
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_rowc(TopkParams p) {
+  constexpr int NW = NT / 32;
+  extern __shared__ __align__(16) uint32_t dyn[];
+  __shared__ RowcShared rs;
+  RowSel &sh = rs.sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t C = cluster_nctarank(), rank = cluster_ctarank();
+  const int row = blockIdx.x / C;
+  const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + row % p.n_q + 1) / p.m;
+  const int nwords = (V + 31) >> 5;
+  const int per_cta = 32 * NT;
+  const int base = (int)rank * per_cta;                  // first key of this CTA
+  uint32_t *win = dyn;                                   // [words]        (CTA 0)
+  uint32_t *tie = dyn + p.slice;                         // [words]        (CTA 0)
+  uint32_t *band_key = dyn + 2 * p.slice;                // [kRowCand]     (CTA 0)
+  uint32_t *band_idx = band_key + kRowCand;              // [kRowCand]     (CTA 0)
+  float *samples = reinterpret_cast<float *>(band_idx + kRowCand);   // [C * NT] (CTA 0)
+  int32_t *out = p.idx_out + (long long)row * p.out_stride;
+  const unsigned long long st_entry = global_ns();
+  pdl_trigger();
+  pdl_wait();
+  const unsigned long long st_ready = global_ns();
+  // every row of a launch has V > k (the host sends short rows elsewhere)
+  const float *src = p.scores + (long long)row * p.in_stride;
+  float x[kRowRegs][4];
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+#pragma unroll
+  for (int j = 0; j < kRowRegs; ++j) {
+    const int i = base + 4 * tid + 4 * NT * j;
+    if (vec && i + 3 < V) {
+      const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i));
+      x[j][0] = v.x; x[j][1] = v.y; x[j][2] = v.z; x[j][3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[j][e] = i + e < V ? __ldg(src + i + e) : 0.f;
+    }
+  }
+  if (rank == 0) {
+    for (int w = tid; w < nwords; w += NT) { win[w] = 0u; tie[w] = 0u; }
+    for (int i = tid; i < kBinsMax; i += NT) sh.hist[i] = 0u;
+    if (tid == 0) { sh.s_above = 0; sh.s_nc = 0; }
+  }
+  // ---- 1. one sample key per thread into CTA 0 (NaN marks "no key")
+  {
+    const int js = tid % kRowRegs;
+    const int is = base + 4 * tid + 4 * NT * js;
+    float sv = __uint_as_float(0x7FC00000u);
+#pragma unroll
+    for (int j = 0; j < kRowRegs; ++j)
+      if (j == js && is < V) sv = x[j][0];
+    st_dsmem_f32(cluster_map(smem_u32(samples + rank * NT + tid), 0), sv);
+  }
+  cluster_sync();
+  // ---- 2. CTA 0: thresholds from the sample, sent to every CTA
+  if (rank == 0) {
+    const int S = (int)C * NT;
+    uint32_t smin = 0xFFFFFFFFu, smax = 0u;
+    int ns = 0;
+    for (int i = tid; i < S; i += NT) {
+      const float v = samples[i];
+      if (v == v) {
+        const uint32_t kk = order_bits(__float_as_uint(v));
+        smin = min(smin, kk);
+        smax = max(smax, kk);
+        ++ns;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      smin = min(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+      smax = max(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+      ns += __shfl_xor_sync(0xffffffffu, ns, o);
+    }
+    if (lane == 0) { rs.red_a[warp] = smin; rs.red_b[warp] = smax; sh.warp_buf[warp] = ns; }
+    __syncthreads();
+    smin = rs.red_a[0]; smax = rs.red_b[0]; ns = sh.warp_buf[0];
+    for (int w = 1; w < NW; ++w) { smin = min(smin, rs.red_a[w]); smax = max(smax, rs.red_b[w]); ns += sh.warp_buf[w]; }
+    __syncthreads();
+    const float lo = key_float(smin), hi = key_float(smax);
+    const float scale = (float)kBinsMax / (hi - lo);
+    const bool ok = ns >= 64 && smin != smax && scale > 0.f && scale < INFINITY;
+    float t_hi = 0.f, t_lo = 0.f;
+    if (ok) {
+      for (int i = tid; i < S; i += NT) {
+        const float v = samples[i];
+        if (v == v) {
+          const float f = (key_float(order_bits(__float_as_uint(v))) - lo) * scale;
+          atomicAdd(&sh.hist[f >= (float)(kBinsMax - 1) ? (uint32_t)(kBinsMax - 1) : (f > 0.f ? (uint32_t)f : 0u)], 1u);
+        }
+      }
+      __syncthreads();
+      const float q = (float)p.k * (float)ns / (float)V;
+      const int r_hi = max(1, (int)floorf(q - 3.f * sqrtf(q)));
+      const int r_lo = min(ns, (int)ceilf(q + 3.f * sqrtf(q) + 2.f));
+      row_find_digit<NT>(sh.hist, kBinsMax, r_hi, sh.warp_buf, &sh.scan_tot, sh.res);
+      const int b_hi = sh.res[0];
+      __syncthreads();
+      row_find_digit<NT>(sh.hist, kBinsMax, r_lo, sh.warp_buf, &sh.scan_tot, sh.res);
+      const int b_lo = sh.res[0];
+      __syncthreads();
+      for (int i = tid; i < kBinsMax; i += NT) sh.hist[i] = 0u;
+      t_hi = lo + (float)(b_hi + 1) / scale;
+      t_lo = lo + (float)b_lo / scale;
+    }
+    if (tid < (int)C) {
+      const uint32_t r = (uint32_t)tid;
+      st_dsmem_f32(cluster_map(smem_u32(&rs.thr[0]), r), t_hi);
+      st_dsmem_f32(cluster_map(smem_u32(&rs.thr[1]), r), t_lo);
+      st_dsmem_u32(cluster_map(smem_u32(&rs.band_ok), r), ok ? 1u : 0u);
+    }
+  }
+  cluster_sync();
+  // ---- 3. every CTA: winners' bits and band keys into CTA 0
+  if (rs.band_ok) {
+    const float t_hi = rs.thr[0], t_lo = rs.thr[1];
+    int above = 0, inband = 0;
+#pragma unroll
+    for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool valid = base + 4 * tid + 4 * NT * j + e < V;
+        const float v = x[j][e];
+        above += (valid && v > t_hi) ? 1 : 0;
+        inband += (valid && v <= t_hi && v >= t_lo) ? 1 : 0;
+      }
+    const int off = block_exclusive_scan<NT>(inband, sh.warp_buf, &sh.scan_tot);
+    const int tot = sh.scan_tot;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    if (lane == 0 && above) atom_add_dsmem_u32(cluster_map(smem_u32(&sh.s_above), 0), (uint32_t)above);
+    if (tid == 0) rs.base = tot ? atom_add_dsmem_u32(cluster_map(smem_u32(&sh.s_nc), 0), (uint32_t)tot) : 0u;
+    __syncthreads();
+    int at = (int)rs.base + off;
+    if (above | inband) {
+      const uint32_t wmap = cluster_map(smem_u32(win), 0);
+      const uint32_t kmap = cluster_map(smem_u32(band_key), 0);
+      const uint32_t imap = cluster_map(smem_u32(band_idx), 0);
+#pragma unroll
+      for (int j = 0; j < kRowRegs; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = base + 4 * tid + 4 * NT * j + e;
+          const float v = x[j][e];
+          if (i < V && v > t_hi) {
+            red_or_dsmem_u32(wmap + 4u * (uint32_t)(i >> 5), 1u << (i & 31));
+          } else if (i < V && v >= t_lo) {
+            if (at < kRowCand) {
+              st_dsmem_u32(kmap + 4u * (uint32_t)at, order_bits(__float_as_uint(v)));
+              st_dsmem_u32(imap + 4u * (uint32_t)at, (uint32_t)i);
+            }
+            ++at;
+          }
+        }
+    }
+  }
+  cluster_sync();   // after this no CTA touches another's shared memory
+  if (rank == 0) {
+    // ---- 4. CTA 0: exact selection within the band, or over the whole row
+    const int na = sh.s_above, nc = sh.s_nc;
+    const bool banded = rs.band_ok && na < p.k && na + nc >= p.k && nc <= kRowCand;
+    int krem;
+    uint32_t T;
+    if (banded) {
+      uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
+      for (int i = tid; i < nc; i += NT) { cmin = min(cmin, band_key[i]); cmax = max(cmax, band_key[i]); }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cmin = min(cmin, __shfl_xor_sync(0xffffffffu, cmin, o));
+        cmax = max(cmax, __shfl_xor_sync(0xffffffffu, cmax, o));
+      }
+      if (lane == 0) { rs.red_a[warp] = cmin; rs.red_b[warp] = cmax; }
+      __syncthreads();
+      cmin = rs.red_a[0]; cmax = rs.red_b[0];
+      for (int w = 1; w < NW; ++w) { cmin = min(cmin, rs.red_a[w]); cmax = max(cmax, rs.red_b[w]); }
+      krem = p.k - na;
+      T = radix_select<NT>(sh, cmin, cmax, &krem, [&](auto f) {
+        for (int i = tid; i < nc; i += NT) f(band_key[i]);
+      });
+      for (int i = tid; i < nc; i += NT) {
+        const uint32_t kk = band_key[i], ix = band_idx[i];
+        if (kk > T) atomicOr(&win[ix >> 5], 1u << (ix & 31));
+        else if (kk == T) atomicOr(&tie[ix >> 5], 1u << (ix & 31));
+      }
+    } else {
+      // the whole row, read back from memory (rare: heavy ties, a bad sample)
+      for (int w = tid; w < nwords; w += NT) win[w] = 0u;
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+      for (int i = tid; i < V; i += NT) {
+        const uint32_t kk = order_bits(__float_as_uint(src[i]));
+        kmin = min(kmin, kk);
+        kmax = max(kmax, kk);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+      }
+      if (lane == 0) { rs.red_a[warp] = kmin; rs.red_b[warp] = kmax; }
+      __syncthreads();
+      kmin = rs.red_a[0]; kmax = rs.red_b[0];
+      for (int w = 1; w < NW; ++w) { kmin = min(kmin, rs.red_a[w]); kmax = max(kmax, rs.red_b[w]); }
+      krem = p.k;
+      T = radix_select<NT>(sh, kmin, kmax, &krem, [&](auto f) {
+        for (int i = tid; i < V; i += NT) f(order_bits(__float_as_uint(src[i])));
+      });
+      for (int i = tid; i < V; i += NT) {
+        const uint32_t kk = order_bits(__float_as_uint(src[i]));
+        if (kk > T) atomicOr(&win[i >> 5], 1u << (i & 31));
+        else if (kk == T) atomicOr(&tie[i >> 5], 1u << (i & 31));
+      }
+    }
+    __syncthreads();
+    emit_masks<NT>(sh, win, tie, nwords, krem, V, p.k, out);
+  }
+  if (step_trace_on()) {
+    __syncthreads();
+    if (tid == 0) step_trace_record(ST_TOPK, st_entry, st_ready);
+  }
+}
+
+template <int NT>
+int launch_topk_rowc_t(const TopkParams &t, long long rows, int Vmax, int C, cudaStream_t s) {
+  const int words = (Vmax + 31) / 32;
+  const size_t smem = (size_t)(2 * words + 2 * kRowCand + C * NT) * 4;
+  static std::atomic<bool> attr_dev[kMaxDevices];
+  std::atomic<bool> &attr = attr_dev[device_slot()];
+  if (!attr) {
+    const int max_words = kClusterMax * 32 * NT / 32;
+    const cudaError_t e = cudaFuncSetAttribute(topk_rowc<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (2 * max_words + 2 * kRowCand + kClusterMax * NT) * 4);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k cluster-row smem attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  LaunchScope ls("topk", s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)(rows * C), 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = C;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  TopkParams tp = t;
+  tp.slice = words;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_rowc<NT>, tp);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "topk_rowc launch: %s", cudaGetErrorString(e));
+  }
+  return ls.done();
+}
+// Rows all longer than k and few of them (decode): a cluster of C CTAs per
+// row, C the smallest power of two (<= 8) giving every CTA at most 32 * NT
+// keys.  HCA_ERR_UNSUPPORTED when the rows do not fit.
+int launch_topk_rowc(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
+  const int NTs[2] = {128, 1024};
+  for (int v = 0; v < 2; ++v) {
+    const int NT = NTs[v];
+    int C = 1;
+    while (C < kClusterMax && (long long)C * 32 * NT < Vmax) C *= 2;
+    if ((long long)C * 32 * NT < Vmax) continue;
+    if (C < 2) C = 2;
+    return NT == 128 ? launch_topk_rowc_t<128>(t, rows, Vmax, C, s) : launch_topk_rowc_t<1024>(t, rows, Vmax, C, s);
+  }
+  return HCA_ERR_UNSUPPORTED;
+}
+
 template <int NT>
 int launch_topk_row_t(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
   const int words = (Vmax + 31) / 32;
@@ -914,6 +1264,13 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t.rows = (int)rows; t.k = ip.k; t.scores = p.scores; t.in_stride = p.score_stride;
   t.n_q = ip.n_q; t.start_pos = ip.start_pos; t.m = ip.m;
   t.n_seg = pl.n_seg; t.seg_len = pl.seg_len; t.slice = pl.slice;
+  // few rows, all longer than k (decode): a cluster per row
+  const int Vmin = (ip.start_pos + 1) / ip.m;
+  if (Vmin > ip.k && rows * 8 <= 2LL * num_sms() && Vmax > 4096) {
+    t.idx_out = idx; t.out_stride = ip.k;
+    rc = launch_topk_rowc(t, rows, Vmax, s);
+    if (rc != HCA_ERR_UNSUPPORTED) return rc;
+  }
   if (Vmax <= kRowMax && g_topk_row_enabled) {
     t.idx_out = idx; t.out_stride = ip.k;
     return launch_topk_row(t, rows, Vmax, s);

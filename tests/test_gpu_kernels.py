@@ -195,14 +195,16 @@ def test_index_topk(cuda, B, n_q, start_pos, m, k, n_hI, c_I, qdt, kdt):
 
 
 TIE_CASES = [
-    # B, n_q, start_pos, k, key dtype.  Rows of up to 36864 keys: one CTA per
-    # row (256 threads up to 4096 keys, else 1024); longer rows: a cluster per
-    # row segment (one segment, then two, then the 1M rows' segments + merge)
+    # B, n_q, start_pos, k, key dtype.  Many rows of up to 32768 keys: one CTA
+    # per row (128..1024 threads); few rows all longer than k: a cluster of
+    # CTAs per row (up to 262144 keys); many long rows: a cluster per row
+    # segment (the 64 rows of 50000 keys)
     (2, 64, 0, 64, "bf16"),
     (2, 8, 16000, 64, "bf16"),
     (3, 1, 131071, 512, "bf16"),
     (2, 1, 163839, 512, "bf16"),
     (1, 2, 300000, 512, "bf16"),
+    (1, 64, 200000, 512, "bf16"),
     (2, 1, 1048575, 1024, "fp8"),
 ]
 
