@@ -89,6 +89,12 @@ typedef struct {
                               call, which also bounds the split-KV count per query;
                               0 = every SM.  For a caller that runs another layer's
                               kernels on a second stream at the same time. */
+  int kv_mixed;            /* 1: the compressed KV rows and the window rows the layer
+                              keeps are mixed-precision records (hca_kv_quant_mixed;
+                              [J] §2.3.4): csa_attend / hca_attend read kv_comp and
+                              kv_win as records of hca_kv_mixed_row_bytes(c, rd)
+                              bytes and dequantise them on load (dtype HCA_BF16,
+                              n_h <= 64, c in {128, 256, 512}).  0: dtype rows. */
 } hca_attn_desc;
 
 /* ------------------------------------------------------------------------

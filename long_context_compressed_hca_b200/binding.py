@@ -36,7 +36,8 @@ class AttnDesc(C.Structure):
     _fields_ = [("B", C.c_int), ("n_h", C.c_int), ("c", C.c_int), ("rd", C.c_int), ("w", C.c_int),
                 ("m", C.c_int), ("overlap", C.c_int), ("k", C.c_int), ("n_hI", C.c_int),
                 ("c_I", C.c_int), ("rd_I", C.c_int), ("dtype", C.c_int), ("idx_key_dtype", C.c_int),
-                ("scale", C.c_float), ("eps", C.c_float), ("rope_theta", C.c_float), ("max_ctas", C.c_int)]
+                ("scale", C.c_float), ("eps", C.c_float), ("rope_theta", C.c_float), ("max_ctas", C.c_int),
+                ("kv_mixed", C.c_int)]
 
 
 class CompressDesc(C.Structure):
@@ -227,9 +228,10 @@ def trace_attend_read() -> dict:
 
 
 def attn_desc(B, n_h, c, rd, w, m, overlap=0, k=0, n_hI=0, c_I=0, rd_I=0, dtype=HCA_BF16,
-              idx_key_dtype=None, scale=0.0, eps=1e-6, rope_theta=10000.0, max_ctas=0) -> AttnDesc:
+              idx_key_dtype=None, scale=0.0, eps=1e-6, rope_theta=10000.0, max_ctas=0, kv_mixed=0) -> AttnDesc:
     return AttnDesc(B, n_h, c, rd, w, m, int(overlap), k, n_hI, c_I, rd_I, dtype,
-                    dtype if idx_key_dtype is None else idx_key_dtype, scale, eps, rope_theta, max_ctas)
+                    dtype if idx_key_dtype is None else idx_key_dtype, scale, eps, rope_theta, max_ctas,
+                    int(kv_mixed))
 
 
 def compress_desc(B, width, m, overlap, rd, flags, in_dtype, out_dtype, eps=1e-6,

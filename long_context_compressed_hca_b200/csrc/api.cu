@@ -162,6 +162,12 @@ int check_attn_desc(const hca_attn_desc *d, bool need_indexer) {
   REQUIRE(d->m >= 1, "m must be >= 1");
   REQUIRE(d->dtype == HCA_F32 || d->dtype == HCA_BF16, "dtype must be HCA_F32 or HCA_BF16");
   REQUIRE(d->max_ctas >= 0, "max_ctas must be >= 0 (0 = every SM)");
+  REQUIRE(d->kv_mixed == 0 || d->kv_mixed == 1, "kv_mixed must be 0 or 1");
+  if (d->kv_mixed) {
+    REQUIRE(d->dtype == HCA_BF16, "mixed-precision KV rows need dtype HCA_BF16");
+    REQUIRE(kv_mixed_row_bytes(d->c, d->rd) > 0, "mixed-precision KV rows need c - rd a multiple of 64 and rd a "
+            "multiple of 16 (c = %d, rd = %d)", d->c, d->rd);
+  }
   if (need_indexer) {
     REQUIRE(d->k >= 1, "k must be >= 1");
     REQUIRE(d->n_hI >= 1 && d->c_I >= 8 && d->c_I % 8 == 0, "indexer heads / dim invalid");
@@ -193,6 +199,8 @@ AttendParams attend_params(const hca_attn_desc *d, const void *q, const void *kv
   p.B = d->B; p.n_q = n_q; p.start_pos = start_pos; p.n_h = d->n_h; p.c = d->c; p.rd = d->rd;
   p.w = d->w; p.m = d->m; p.k = csa ? d->k : 0; p.cap = cap; p.csa = csa; p.win_is_ring = win_is_ring;
   p.scale = attn_scale(d); p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
+  p.kv_mixed = d->kv_mixed ? 1 : 0;
+  p.rec = d->kv_mixed ? (int)kv_mixed_row_bytes(d->c, d->rd) : 0;
   p.q = q; p.kv_comp = kv_comp; p.idx = idx; p.kv_win = kv_win; p.sink = sink; p.o = o; p.dtype = d->dtype;
   // token-indexed window: the rows of tokens start_pos - h .. start_pos + n_q - 1,
   // h = min(w - 1, start_pos) (the halo before the first query)

@@ -502,7 +502,7 @@ __device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *sm
   return ok;
 }
 
-template <int C, bool TRACE>
+template <int C, bool TRACE, bool MIX>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc(AttendParams p, int n_units) {
   using L = Layout<C>;
@@ -611,6 +611,66 @@ attend_tc(AttendParams p, int n_units) {
       const __nv_bfloat16 *cbase = reinterpret_cast<const __nv_bfloat16 *>(
           p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q));
       const __nv_bfloat16 *wbase = p.kv_win ? reinterpret_cast<const __nv_bfloat16 *>(p.kv_win) : cbase;
+      if (MIX) {
+        // mixed-precision records: a thread whose chunk holds FP8 codes loads
+        // its 8 codes and their block scale for all of its rows (independent
+        // loads, all in flight), waits for the stage, and writes the bf16
+        // values code x scale; a thread of the bf16 RoPE channels copies them
+        const uint8_t *crec = reinterpret_cast<const uint8_t *>(p.kv_comp ? p.kv_comp : (p.kv_win ? p.kv_win : p.q));
+        const uint8_t *wrec = p.kv_win ? reinterpret_cast<const uint8_t *>(p.kv_win) : crec;
+        const int ch0 = chunk * 8, nq = C - p.rd;
+        const bool code = ch0 < nq;
+        const int col_off = code ? ch0 : nq + 2 * (ch0 - nq);
+        const int sc_off = C + p.rd + 4 * (ch0 / 64);
+        for (int j = 0; j < nt; ++j, ++g) {
+          const int st = g % L::NS;
+          const uint32_t tile = sbase + L::kv_off + st * NKB * kTileBytes + kb_off;
+          if (code) {
+            uint2 cw[NR];
+            float sc[NR];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              const int kk = (j0 + j) * KT + prow + i * RPP;
+              bool v;
+              const int row = slot_row(p, ks, b, qi, kk, v);
+              const uint8_t *rp = (kk < ks.nw4 ? wrec : crec) + (long long)row * p.rec;
+              cw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + col_off));
+              sc[i] = __ldg(reinterpret_cast<const float *>(rp + sc_off));
+            }
+            if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              const uint32_t w2[2] = {cw[i].x, cw[i].y};
+              uint32_t o[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const uint32_t pair = (w2[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+                const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)pair, __NV_E4M3)));
+                o[h] = pack_bf16x2(f.x * sc[i], f.y * sc[i]);
+              }
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(tile + sw128_off(prow + i * RPP, cc)),
+                           "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                           : "memory");
+            }
+            fence_proxy_async();   // the tensor cores read the tile through the async proxy
+            mbar_arrive(bar(bars->kv_full[st]));
+          } else {
+            const uint8_t *src8[NR];
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              const int kk = (j0 + j) * KT + prow + i * RPP;
+              bool v;
+              const int row = slot_row(p, ks, b, qi, kk, v);
+              src8[i] = (kk < ks.nw4 ? wrec : crec) + (long long)row * p.rec + col_off;
+            }
+            if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+#pragma unroll
+            for (int i = 0; i < NR; ++i) cp_async16(tile + sw128_off(prow + i * RPP, cc), src8[i], 16);
+            cp_async_arrive_noinc(bar(bars->kv_full[st]));
+          }
+        }
+        continue;
+      }
       for (int j = 0; j < nt; ++j, ++g) {
         const int st = g % L::NS;
         const __nv_bfloat16 *src[NR];
@@ -1050,9 +1110,13 @@ int ensure_attr() {
   std::atomic<bool> &attr_set = attr_set_dev[device_slot()];
   if (!attr_set) {
     const int smem = (int)Layout<C>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_tc<C, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(attend_tc<C, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attend_tc<C, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attend_tc<C, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "attend_tc smem attribute: %s", cudaGetErrorString(e));
     attr_set = true;
   }
@@ -1079,7 +1143,7 @@ int max_active_clusters(int ns) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<C, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<C, false, false>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     n = 0;
   }
@@ -1110,8 +1174,11 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
   at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = p.cluster ? 2 : 1;
-  const cudaError_t e = attend_trace_on() ? cudaLaunchKernelEx(&cfg, attend_tc<C, true>, p, n_units)
-                                          : cudaLaunchKernelEx(&cfg, attend_tc<C, false>, p, n_units);
+  const bool tr = attend_trace_on();
+  const cudaError_t e = p.kv_mixed ? (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, true, true>, p, n_units)
+                                         : cudaLaunchKernelEx(&cfg, attend_tc<C, false, true>, p, n_units))
+                                   : (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, true, false>, p, n_units)
+                                         : cudaLaunchKernelEx(&cfg, attend_tc<C, false, false>, p, n_units));
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return fail(HCA_ERR_CUDA, "attend_tc launch: %s", cudaGetErrorString(e));
@@ -1192,6 +1259,8 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
     p.rope_freq[i] = i < p.rd / 2 ? std::exp2(-2.0 * i / (double)p.rd * std::log2((double)p.theta)) : 0.0;
   p.nsplit = 1;
   p.cluster = 0;
+  if (p.kv_mixed && !tc_path(p))
+    return fail(HCA_ERR_UNSUPPORTED, "mixed-precision KV rows need the tensor-core path (bf16, n_h <= 64, c in {128, 256, 512})");
   if (tc_path(p)) {
     if (!p.kv_comp) p.cap = 0;   // no visible entries: masked slots then read row 0 of the dummy map
     const SplitPlan sp = plan_splits(p, ws && ws_bytes >= attend_workspace_bytes(p));

@@ -489,7 +489,7 @@ __device__ uint32_t radix_select(RowSel &sh, uint32_t kmin, uint32_t kmax, int *
 
 // Grid: one CTA per row.  Dynamic shared memory: 2 * words + 2 * kRowCand
 // words (winner and tie masks of the row, band keys and indices).
-template <int NT>
+template <int NT, int RR>
 __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   constexpr int NW = NT / 32;
   extern __shared__ __align__(16) uint32_t dyn[];
@@ -513,10 +513,10 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
 
   // ---- the row in registers: thread t holds keys 4t + 4NT*j + e (as floats)
   const float *src = p.scores + (long long)row * p.in_stride;
-  float x[kRowRegs][4];
+  float x[RR][4];
   const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
 #pragma unroll
-  for (int j = 0; j < kRowRegs; ++j) {
+  for (int j = 0; j < RR; ++j) {
     const int i = 4 * tid + 4 * NT * j;
     if (vec && i + 3 < V) {
       const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i));
@@ -535,12 +535,12 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   bool banded = false;
   if (V > p.k) {
     // ---- 1. sample: thread t contributes key 4t + 4NT*(t % 8) (its register j = t % 8)
-    const int js = tid % kRowRegs;
+    const int js = tid % RR;
     const int is = 4 * tid + 4 * NT * js;
     const bool has_s = is < V && tid < kRowSample;
     float sv = 0.f;
 #pragma unroll
-    for (int j = 0; j < kRowRegs; ++j)
+    for (int j = 0; j < RR; ++j)
       if (j == js) sv = x[j][0];
     uint32_t smin = has_s ? order_bits(__float_as_uint(sv)) : 0xFFFFFFFFu;
     uint32_t smax = has_s ? smin : 0u;
@@ -582,7 +582,7 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       // ---- 2. one pass over the row: count, then place (no per-key votes)
       int above = 0, inband = 0;
 #pragma unroll
-      for (int j = 0; j < kRowRegs; ++j)
+      for (int j = 0; j < RR; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool valid = 4 * tid + 4 * NT * j + e < V;
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       int at = __shfl_sync(0xffffffffu, wbase, 31) + incl - inband;
       if (above | inband) {
 #pragma unroll
-        for (int j = 0; j < kRowRegs; ++j)
+        for (int j = 0; j < RR; ++j)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 4 * tid + 4 * NT * j + e;
@@ -656,7 +656,7 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       // ---- 3'. exact select over the whole row (registers)
       uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
 #pragma unroll
-      for (int j = 0; j < kRowRegs; ++j)
+      for (int j = 0; j < RR; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (4 * tid + 4 * NT * j + e < V) {
@@ -676,13 +676,13 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
       krem = p.k;
       T = radix_select<NT>(sh, kmin, kmax, &krem, [&](auto f) {
 #pragma unroll
-        for (int j = 0; j < kRowRegs; ++j)
+        for (int j = 0; j < RR; ++j)
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             if (4 * tid + 4 * NT * j + e < V) f(order_bits(__float_as_uint(x[j][e])));
       });
 #pragma unroll
-      for (int j = 0; j < kRowRegs; ++j)
+      for (int j = 0; j < RR; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = 4 * tid + 4 * NT * j + e;
@@ -839,7 +839,6 @@ __global__ void __launch_bounds__(NT) topk_rowc(TopkParams p) {
   float *samples = reinterpret_cast<float *>(band_idx + kRowCand);   // [C * NT] (CTA 0)
   int32_t *out = p.idx_out + (long long)row * p.out_stride;
   const unsigned long long st_entry = global_ns();
-  pdl_trigger();
   pdl_wait();
   const unsigned long long st_ready = global_ns();
   // every row of a launch has V > k (the host sends short rows elsewhere)
@@ -976,6 +975,9 @@ __global__ void __launch_bounds__(NT) topk_rowc(TopkParams p) {
     }
   }
   cluster_sync();   // after this no CTA touches another's shared memory
+  // the attention may now start its prologue: scheduling it earlier let its
+  // CTAs take the SMs that clusters still waiting for placement needed
+  pdl_trigger();
   if (rank == 0) {
     // ---- 4. CTA 0: exact selection within the band, or over the whole row
     const int na = sh.s_above, nc = sh.s_nc;
@@ -1093,14 +1095,14 @@ int launch_topk_rowc(const TopkParams &t, long long rows, int Vmax, cudaStream_t
   return HCA_ERR_UNSUPPORTED;
 }
 
-template <int NT>
+template <int NT, int RR>
 int launch_topk_row_t(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
   const int words = (Vmax + 31) / 32;
   const size_t smem = (size_t)(2 * words + 2 * kRowCand) * 4;
   static std::atomic<bool> attr_dev[kMaxDevices];
   std::atomic<bool> &attr = attr_dev[device_slot()];
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(topk_row<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(topk_row<NT, RR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (2 * (kRowMax / 32) + 2 * kRowCand) * 4);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k row smem attribute: %s", cudaGetErrorString(e));
     attr = true;
@@ -1118,20 +1120,21 @@ int launch_topk_row_t(const TopkParams &t, long long rows, int Vmax, cudaStream_
   cfg.numAttrs = 1;
   TopkParams tp = t;
   tp.slice = words;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_row<NT>, tp);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_row<NT, RR>, tp);
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return fail(HCA_ERR_CUDA, "topk_row launch: %s", cudaGetErrorString(e));
   }
   return ls.done();
 }
-// One CTA per row for rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise).
+// One CTA per row for rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise);
+// the longest rows take 64 keys per thread in 512 threads (no register spills).
 int launch_topk_row(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
   if (Vmax > kRowMax || rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
-  if (Vmax <= 32 * 128) return launch_topk_row_t<128>(t, rows, Vmax, s);
-  if (Vmax <= 32 * 256) return launch_topk_row_t<256>(t, rows, Vmax, s);
-  if (Vmax <= 32 * 512) return launch_topk_row_t<512>(t, rows, Vmax, s);
-  return launch_topk_row_t<1024>(t, rows, Vmax, s);
+  if (Vmax <= 32 * 128) return launch_topk_row_t<128, 8>(t, rows, Vmax, s);
+  if (Vmax <= 32 * 256) return launch_topk_row_t<256, 8>(t, rows, Vmax, s);
+  if (Vmax <= 32 * 512) return launch_topk_row_t<512, 8>(t, rows, Vmax, s);
+  return launch_topk_row_t<512, 16>(t, rows, Vmax, s);
 }
 
 struct TopkPlan {
@@ -1266,7 +1269,7 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t.n_seg = pl.n_seg; t.seg_len = pl.seg_len; t.slice = pl.slice;
   // few rows, all longer than k (decode): a cluster per row
   const int Vmin = (ip.start_pos + 1) / ip.m;
-  if (Vmin > ip.k && rows * 8 <= 2LL * num_sms() && Vmax > 4096) {
+  if (Vmin > ip.k && rows * 8 <= 2LL * num_sms() && Vmax > kRowMax) {
     t.idx_out = idx; t.out_stride = ip.k;
     rc = launch_topk_rowc(t, rows, Vmax, s);
     if (rc != HCA_ERR_UNSUPPORTED) return rc;

@@ -151,6 +151,8 @@ struct AttendParams {
   const int32_t *idx;      // [B, n_q, k]
   const void *kv_win;      // token rows [B, win_rows, c] (row r = token win_tok0 + r); ring [B, w, c]
   int win_tok0, win_rows;  // token-indexed window: first token and rows per sequence
+  int kv_mixed;            // 1: kv_comp and kv_win hold mixed-precision records of `rec` bytes
+  int rec;
   const float *sink;       // [n_h]
   void *o;                 // [B, n_q, n_h, c]
   hca_dtype dtype;
