@@ -309,7 +309,8 @@ __device__ __forceinline__ void compress_decode_block(const CompressParams &p, i
 #pragma unroll
   for (int q = 0; q < 8; ++q) v[q] = active ? ent[threadIdx.x * 8 + q] : 0.f;
   const long long entry = pos / m;
-  entry_epilogue<Tout>(p, v, active, 0, active ? threadIdx.x : 0, cv, b, entry,
+  // the entry goes to out slot entry - e_first (e_first = entry: a one-row scratch)
+  entry_epilogue<Tout>(p, v, active, 0, active ? threadIdx.x : 0, cv, b, entry - p.e_first,
                        (long long)(pos + 1 - m), red, red2);
   __syncthreads();
   // 3. shift the state: the finished block becomes the previous block

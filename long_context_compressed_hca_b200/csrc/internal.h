@@ -136,7 +136,9 @@ int step_trace_set_compress(void *buf, unsigned long long cap);
 // ------------------------------------------------------- mixed-precision KV
 // Record bytes of one row (0 for unsupported shapes) and the two HBM streams.
 size_t kv_mixed_row_bytes(int c, int rd);
-int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, int rd, void *out, cudaStream_t s);
+// Output row r at record (r / per_seq) * seq_rows + r % per_seq (per_seq <= 0: dense).
+int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, int rd, void *out, cudaStream_t s,
+                          long long per_seq = 0, long long seq_rows = 0);
 int launch_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, cudaStream_t s);
 
 // ------------------------------------------------------------- attention

@@ -58,7 +58,7 @@ __device__ __forceinline__ void store_bf16x16(unsigned char *dst, const float *v
 template <typename T>
 __global__ void __launch_bounds__(kKvWarps * 32) kv_quant_mixed_kernel(const T *__restrict__ x, long long rows,
                                                                          int c, int rd, unsigned char *__restrict__ out,
-                                                                         int rec) {
+                                                                         int rec, long long per_seq, long long seq_rows) {
   const int lane = threadIdx.x & 31;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int nq = c - rd, ncl = nq / 16, L = c / 16;
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kKvWarps * 32) kv_quant_mixed_kernel(const T *
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = 0.f;
     }
-    unsigned char *rp = out + r * rec;
+    unsigned char *rp = out + ((r / per_seq) * seq_rows + r % per_seq) * rec;
     // the amax of this lane's block (lanes 4b .. 4b+3 hold block b)
     float amax = 0.f;
     if (lane < ncl) {
@@ -144,17 +144,19 @@ size_t kv_mixed_row_bytes(int c, int rd) {
   return (payload + 15) & ~(size_t)15;
 }
 
-int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, int rd, void *out, cudaStream_t s) {
+int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, int rd, void *out, cudaStream_t s,
+                          long long per_seq, long long seq_rows) {
   if (rows == 0) return HCA_OK;
+  if (per_seq <= 0) { per_seq = rows; seq_rows = 0; }
   const int rec = (int)kv_mixed_row_bytes(c, rd);
   unsigned char *o = static_cast<unsigned char *>(out);
   if (dt == HCA_F32)
     return HCA_LAUNCH("kv_quant_mixed", s,
                       kv_quant_mixed_kernel<float><<<kv_grid(rows), kKvWarps * 32, 0, s>>>(
-                          static_cast<const float *>(x), rows, c, rd, o, rec));
+                          static_cast<const float *>(x), rows, c, rd, o, rec, per_seq, seq_rows));
   return HCA_LAUNCH("kv_quant_mixed", s,
                     kv_quant_mixed_kernel<__nv_bfloat16><<<kv_grid(rows), kKvWarps * 32, 0, s>>>(
-                        static_cast<const __nv_bfloat16 *>(x), rows, c, rd, o, rec));
+                        static_cast<const __nv_bfloat16 *>(x), rows, c, rd, o, rec, per_seq, seq_rows));
 }
 
 int launch_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, cudaStream_t s) {

@@ -149,7 +149,8 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
   // ---- compressed main KV
   void *kvc = P.kvc;
   int cap = E > 0 ? E : 1;
-  if (cache && comp) { kvc = cache->kv_comp; cap = cache->cap; }
+  // a mixed-precision cache is filled from the bf16 entries after compression
+  if (cache && comp && !a.kv_mixed) { kvc = cache->kv_comp; cap = cache->cap; }
   if (comp) {
     const int ncz = csa ? 4 : 2;
     rc = launch_gemm(dt, H, L->d, L->W_comp, L->d, P.CZ, (long long)ncz * a.c, HCA_F32, (int)T, ncz * a.c, L->d, 1.f, s);
@@ -167,6 +168,10 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
                       nullptr, kvc, nullptr, cap, cache ? cache->state_kv : nullptr,
                       cache ? cache->state_score : nullptr, stream);
     if (rc) return rc;
+    if (cache && a.kv_mixed && E > 0) {
+      rc = launch_kv_quant_mixed(P.kvc, dt, (long long)a.B * E, a.c, a.rd, cache->kv_comp, s, E, cache->cap);
+      if (rc) return rc;
+    }
   }
   // ---- indexer keys
   void *keyI = P.keyI;
@@ -235,15 +240,31 @@ int hybrid_layer_forward(const hca_layer *L, const void *H, int n, hca_cache *ca
     r.rows_per_pos = 1; r.pos_mod = n; r.scale = 1.f;
     if ((rc = launch_row_op(r, s))) return rc;
   }
-  if (cache && a.w > 0 && cache->win) {
+  if (cache && a.w > 0 && cache->win && a.kv_mixed) {
+    // the last min(w, n) window rows of every sequence as records in ring slot
+    // p % w: at most two runs of consecutive slots per sequence
+    const int rec = (int)kv_mixed_row_bytes(a.c, a.rd);
+    const int first = n > a.w ? n - a.w : 0;
+    for (int b = 0; b < a.B; ++b) {
+      int p0 = first;
+      while (p0 < n) {
+        const int run = (a.w - p0 % a.w) < (n - p0) ? (a.w - p0 % a.w) : (n - p0);
+        rc = launch_kv_quant_mixed(static_cast<const char *>(P.kvw) + ((long long)b * n + p0) * a.c * es, dt, run, a.c,
+                                   a.rd, static_cast<char *>(cache->win) + ((long long)b * a.w + p0 % a.w) * rec, s);
+        if (rc) return rc;
+        p0 += run;
+      }
+    }
+  } else if (cache && a.w > 0 && cache->win) {
     dim3 g(8, a.B);
     LaunchScope ls_("ring_fill", s);
     if (dt == HCA_F32) ring_fill_kernel<float><<<g, 256, 0, s>>>((const float *)P.kvw, (float *)cache->win, a.B, n, a.w, a.c);
     else ring_fill_kernel<__nv_bfloat16><<<g, 256, 0, s>>>((const __nv_bfloat16 *)P.kvw, (__nv_bfloat16 *)cache->win, a.B, n, a.w, a.c);
     if ((rc = ls_.done())) return rc;
   }
-  // ---- select + attend
+  // ---- select + attend (on the bf16 rows of this call, also with a mixed-precision cache)
   hca_attn_desc ad = a;
+  ad.kv_mixed = 0;
   if (csa) {
     ad.idx_key_dtype = kdt;
     rc = csa_index_topk(&ad, P.qI, static_cast<const float *>(P.wI), keyI, keyIs, cap, n, 0,
@@ -466,15 +487,18 @@ int hybrid_cp_attend(const hca_layer *L, const void *H, int t0, int n_loc, const
     r.rows_per_pos = 1; r.pos_mod = h + n_loc; r.pos_base = t0 - h; r.scale = 1.f;
     if ((rc = launch_row_op(r, s))) return rc;
   }
-  // ---- select and attend against the gathered caches
+  // ---- select and attend against the gathered caches (bf16 rows: the
+  // stages exchange dtype entries even when the decode cache is mixed)
+  hca_attn_desc ad = a;
+  ad.kv_mixed = 0;
   if (csa) {
-    rc = csa_index_topk(&a, P.qI, static_cast<const float *>(P.wI), key_I, key_I_scale, cap, n_loc, t0,
+    rc = csa_index_topk(&ad, P.qI, static_cast<const float *>(P.wI), key_I, key_I_scale, cap, n_loc, t0,
                         static_cast<int32_t *>(P.idx), nullptr, 0, P.topk_ws, P.topk_bytes, stream);
     if (rc) return rc;
-    return csa_attend(&a, P.q, kv_comp, cap, static_cast<const int32_t *>(P.idx), P.kvw, 0, L->sink, n_loc, t0, o,
+    return csa_attend(&ad, P.q, kv_comp, cap, static_cast<const int32_t *>(P.idx), P.kvw, 0, L->sink, n_loc, t0, o,
                       nullptr, 0, stream);
   }
-  return hca_attend(&a, P.q, kv_comp, cap, P.kvw, 0, L->sink, n_loc, t0, o, nullptr, 0, stream);
+  return hca_attend(&ad, P.q, kv_comp, cap, P.kvw, 0, L->sink, n_loc, t0, o, nullptr, 0, stream);
 }
 
 int hybrid_workspace_map(const hca_layer *L, int n, int decode, hca_ws_map *map) {
@@ -514,7 +538,9 @@ size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos) {
   }
   const size_t att = L->kind == HCA_LAYER_CSA ? csa_attend_workspace_size(&L->a, 1, pos)
                                               : hca_attend_workspace_size(&L->a, 1, pos);
-  return ((b + 255) & ~(size_t)255) + att + 256;
+  // mixed-precision KV: the emitted entry in bf16 before it is quantised
+  const size_t mix = L->a.kv_mixed ? ((((size_t)L->a.B * L->a.c * 2) + 255) & ~(size_t)255) : 0;
+  return ((b + 255) & ~(size_t)255) + att + 256 + mix;
 }
 
 int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cache, int pos, void *o, void *ws,
@@ -534,6 +560,9 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const hca_dtype dt = a.dtype;
   const float theta = rope_theta(a), eps = eps_of(a);
+  void *mix_entry = a.kv_mixed ? static_cast<char *>(ws) + (need - ((((size_t)a.B * a.c * 2) + 255) & ~(size_t)255))
+                               : nullptr;
+  const int rec = a.kv_mixed ? (int)kv_mixed_row_bytes(a.c, a.rd) : 0;
   // 1. one launch: window ring write, compressor states (+ entry emission) of
   //    the main and (CSA) indexer compressors
   {
@@ -548,8 +577,11 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
       const bool ov = cd.overlap != 0;
       rc = compress_params(&cd, pos, 1, cz, ov ? cz + a.c : nullptr, cz + (csa ? 2 : 1) * a.c, ov ? cz + 3 * a.c : nullptr,
                            (long long)ncz * a.c, (long long)ncz * a.c, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
-                           nullptr, cache->kv_comp, nullptr, cache->cap, cache->state_kv, cache->state_score, &pm);
+                           nullptr, a.kv_mixed ? mix_entry : cache->kv_comp, nullptr, a.kv_mixed ? 1 : cache->cap,
+                           cache->state_kv, cache->state_score, &pm);
       if (rc) return rc;
+      // mixed-precision KV: the emitted entry lands in a one-row bf16 scratch
+      if (a.kv_mixed) pm.e_first = pos / a.m;
     }
     if (csa) {
       hca_compress_desc cd{};
@@ -564,11 +596,26 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
       if (rc) return rc;
     }
     IngestRing ring{};
-    if (a.w > 0) {
+    if (a.w > 0 && !a.kv_mixed) {
       ring.row = x->kv; ring.ring = cache->win; ring.w = a.w; ring.c = a.c; ring.slot = pos % a.w; ring.dtype = dt;
     }
-    rc = launch_decode_ingest(comp ? &pm : nullptr, csa ? &pi : nullptr, ring, a.B, pos, s);
-    if (rc) return rc;
+    if (comp || csa || ring.ring) {
+      rc = launch_decode_ingest(comp ? &pm : nullptr, csa ? &pi : nullptr, ring, a.B, pos, s);
+      if (rc) return rc;
+    }
+    if (a.kv_mixed) {
+      // the token's window row and (on a block's last token) the new entry, as records
+      if (a.w > 0) {
+        rc = launch_kv_quant_mixed(x->kv, dt, a.B, a.c, a.rd, static_cast<char *>(cache->win) + (size_t)(pos % a.w) * rec,
+                                   s, 1, a.w);
+        if (rc) return rc;
+      }
+      if (comp && (pos + 1) % a.m == 0) {
+        rc = launch_kv_quant_mixed(mix_entry, dt, a.B, a.c, a.rd,
+                                   static_cast<char *>(cache->kv_comp) + (size_t)(pos / a.m) * rec, s, 1, cache->cap);
+        if (rc) return rc;
+      }
+    }
   }
   if (csa) {
     char *w = static_cast<char *>(ws);

@@ -19,7 +19,7 @@ class LayerHandle:
     """One attention layer: weights on `device` plus the hca_layer struct."""
 
     def __init__(self, L, W: dict, d: int, d_c: int, dtype: torch.dtype, B: int,
-                 idx_key_dtype: str = "bf16", device="cuda", max_ctas: int = 0):
+                 idx_key_dtype: str = "bf16", device="cuda", max_ctas: int = 0, kv_mixed: bool = False):
         self.shape, self.d, self.d_c, self.dtype, self.B = L, d, d_c, dtype, B
         dev = lambda t, dt=None: t.to(device=device, dtype=dt or t.dtype).contiguous()
         csa = L.kind == "csa"
@@ -41,7 +41,7 @@ class LayerHandle:
         self.idx_key_dtype = idx_key_dtype
         self.desc = hb.attn_desc(B, L.n_h, L.c, L.rd, L.w, L.m, overlap=L.overlap, k=L.k,
                                  n_hI=L.n_hI, c_I=L.c_I, rd_I=L.rd_I if csa else 0,
-                                 dtype=_code(dtype), idx_key_dtype=kdt, max_ctas=max_ctas)
+                                 dtype=_code(dtype), idx_key_dtype=kdt, max_ctas=max_ctas, kv_mixed=int(kv_mixed))
         g = lambda nm: hb.ptr(self.t.get(nm))
         self.struct = hb.Layer(hb.HCA_LAYER_CSA if csa else hb.HCA_LAYER_HCA, self.desc, d, d_c,
                                g("W_comp"), g("B_comp"), g("W_compI"), g("B_compI"), g("W_DQ"),
@@ -52,11 +52,17 @@ class CacheHandle:
     """Decode cache of one layer (caller-owned device buffers)."""
 
     def __init__(self, L, B: int, cap: int, dtype: torch.dtype, idx_key_dtype: str = "bf16",
-                 device="cuda"):
+                 device="cuda", kv_mixed: bool = False):
         self.shape, self.B, self.cap = L, B, cap
         z = lambda *s, dt=torch.float32: torch.zeros(*s, dtype=dt, device=device)
-        self.kv_comp = z(B, cap, L.c, dt=dtype)
-        self.win = z(B, max(L.w, 1), L.c, dt=dtype)
+        if kv_mixed:
+            # mixed-precision records (hca_kv_mixed_row_bytes per row)
+            rec = hb.kv_mixed_row_bytes(L.c, L.rd)
+            self.kv_comp = z(B, cap, rec, dt=torch.uint8)
+            self.win = z(B, max(L.w, 1), rec, dt=torch.uint8)
+        else:
+            self.kv_comp = z(B, cap, L.c, dt=dtype)
+            self.win = z(B, max(L.w, 1), L.c, dt=dtype)
         R = 2 * L.m if L.overlap else L.m
         Cw = 2 * L.c if L.overlap else L.c
         self.state_kv = z(B, R, Cw)

@@ -212,19 +212,31 @@ def _bf16_round(x):
     return torch.from_numpy(np.asarray(x)).to(BF16).double().numpy()
 
 
-def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
+def _mixed(x64, rd):
+    """Rows as a reader of the mixed-precision KV format sees them (the oracle's
+    own quantisation of the same bf16 rows)."""
+    return O.kv_row_dequant(*O.kv_row_quant(np.asarray(x64, np.float64), rd))
+
+
+def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed, kv_mixed=False):
     c, m, w = L.c, L.m, L.w
     csa = L.kind == "csa"
     dt = BF16
     cap = pos // m + 4
     Ecur = pos // m                          # complete entries before this token
     W = synth.layer_weights(L, 256, 64, seed, dt, bias_std=0.5)
-    lh = LayerHandle(L, W, 256, 64, dt, B, idx_key_dtype=idx_key_dtype, device=cuda)
-    cache = CacheHandle(L, B, cap, dt, idx_key_dtype=idx_key_dtype, device=cuda)
+    lh = LayerHandle(L, W, 256, 64, dt, B, idx_key_dtype=idx_key_dtype, device=cuda, kv_mixed=kv_mixed)
+    cache = CacheHandle(L, B, cap, dt, idx_key_dtype=idx_key_dtype, device=cuda, kv_mixed=kv_mixed)
     g = lambda shape, s, std=1.0, d=torch.float32: synth.normal(shape, seed, s, std=std, dtype=d)
     gd = lambda shape, s, d=torch.float32: synth.normal_on(cuda, shape, seed, s, dtype=d)
-    cache.kv_comp.copy_(gd((B, cap, c), 100, d=dt))
-    cache.win.copy_(g((B, w, c), 101, d=dt))
+    kvc_rows = gd((B, cap, c), 100, d=dt)
+    win_rows = g((B, w, c), 101, d=dt).to(cuda)
+    if kv_mixed:
+        hb.kv_quant_mixed(kvc_rows, hb.HCA_BF16, B * cap, c, L.rd, cache.kv_comp)
+        hb.kv_quant_mixed(win_rows, hb.HCA_BF16, B * w, c, L.rd, cache.win)
+    else:
+        cache.kv_comp.copy_(kvc_rows)
+        cache.win.copy_(win_rows)
     j = pos % m
     raw = {nm: g((B, m, c), 102 + i) for i, nm in enumerate(("pCb", "pZb", "Ca", "Cb", "Za", "Zb"))}
     Ba, Bb = (W["B_a"], W["B_b"]) if csa else (W["B"], None)
@@ -248,8 +260,8 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
                     tuple(rawI[k][:, :j] for k in ("Ca", "Cb", "Za", "Zb")), W["B_Ia"].float(), W["B_Ib"].float())
         x.update(qI=g((B, L.n_hI, cI), 113, d=dt), wI=g((B, L.n_hI), 114, std=cI ** -0.5 * L.n_hI ** -0.5),
                  compI=g((B, 4 * cI), 115))
-    # device copies of the inputs the step mutates (host copies are made per sequence)
-    kvc0, win0 = cache.kv_comp.clone(), cache.win.clone()
+    # the bf16 rows behind the cache (the step mutates the cache; host copies are made per sequence)
+    kvc0, win0 = kvc_rows, win_rows
     if csa:
         KI0 = cache.key_I.clone()
         KI0s = cache.key_I_scale.clone() if idx_key_dtype == "fp8" else None
@@ -263,9 +275,12 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
     if csa:
         mp = hb.workspace_map(lh.struct, pos, decode=True)
         gidx = hb.ws_view(ws, mp["idx"], (B, 1, L.k), torch.int32).cpu().numpy()
+    rec = hb.kv_mixed_row_bytes(c, L.rd) if kv_mixed else 0
     for b in range(B):
         comp = to64(x["comp"][b])
         kvc = to64(kvc0[b][:(pos + 1) // m + 1])
+        if kv_mixed:
+            kvc = _mixed(kvc, L.rd)
         if emit:
             if csa:
                 Ca = np.concatenate([to64(raw["Ca"][b, :j]), comp[None, 0:c]])
@@ -277,11 +292,24 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
                 Za = np.concatenate([to64(raw["Za"][b, :j]), comp[None, c:2 * c]])
                 e = O.decode_new_entry(pos, m, Ca, Za, to64(W["B"]))
             e = O.entry_epilogue(e[None], m, first_entry=Ecur, rd=L.rd)[0]
-            assert_close(to64(cache.kv_comp[b, Ecur]), e, 2e-2, "emitted entry")
-            kvc[Ecur] = _bf16_round(e)
+            if kv_mixed:
+                # the emitted record, read back: the oracle's quantisation of the
+                # bf16 entry (a value may sit one e4m3 step away where the two
+                # bf16 entries differ in their last bit)
+                got = torch.empty(1, c, dtype=BF16, device=cuda)
+                hb.kv_dequant_mixed(cache.kv_comp[b, Ecur].contiguous(), 1, c, L.rd, got)
+                ref = _mixed(_bf16_round(e)[None], L.rd)[0]
+                d = np.abs(to64(got[0]) - ref)
+                assert (d <= 0.126 * np.abs(ref) + 1e-6).all() and (d == 0).mean() >= 0.95, "emitted record"
+                kvc[Ecur] = ref
+            else:
+                assert_close(to64(cache.kv_comp[b, Ecur]), e, 2e-2, "emitted entry")
+                kvc[Ecur] = _bf16_round(e)
         wpos = O.window_positions(pos, w)
         win = to64(win0[b])
         win[pos % w] = to64(x["kv"][b])
+        if kv_mixed:
+            win = _mixed(win, L.rd)
         wrows = win[[p % w for p in wpos]]
         kw = {}
         if csa:
@@ -325,3 +353,13 @@ def run_decode_case(cuda, L, B, pos, idx_key_dtype, seed):
 def test_decode_step(cuda, kind, pos, kdt):
     L = workloads.HYBRID_DECODE_128K.layers[0 if kind == "csa" else 1]
     run_decode_case(cuda, L, 3, pos, kdt, seed=pos)
+
+
+@pytest.mark.parametrize("kind,pos", [("csa", 2047), ("csa", 2050), ("hca", 4095), ("hca", 5000)])
+def test_decode_step_mixed_kv(cuda, kind, pos):
+    """A decode step over a mixed-precision KV cache ([J] §2.3.4): the step
+    stores its window row and (on a block's last token) its new entry as
+    records, and the attention reads records; checked against the oracle over
+    the oracle's own quantisation of the same rows."""
+    L = workloads.HYBRID_DECODE_128K.layers[0 if kind == "csa" else 1]
+    run_decode_case(cuda, L, 3, pos, "bf16", seed=pos + 7, kv_mixed=True)
