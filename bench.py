@@ -167,8 +167,10 @@ def packed(tensors):
 class DecodeBench:
     """One decode step per sequence over synthetic caches: CSA layer + HCA layer."""
 
-    def __init__(self, wl, seed_shift=0, side_ctas=None, side_high=None):
+    def __init__(self, wl, seed_shift=0, side_ctas=None, side_high=None, kv_mixed=False, idx_key_dtype=None):
         self.wl = wl
+        self.kv_mixed = kv_mixed
+        self.idx_key_dtype = idx_key_dtype or wl.idx_key_dtype
         B, pos = wl.B, wl.pos
         seed = wl.seed + seed_shift
         main_ctas, ctas, high = LAYER_CTAS.get(wl.name, (0, 0, False))
@@ -178,22 +180,33 @@ class DecodeBench:
         self.layers, self.caches, self.x, self.outs, self.ws = [], [], [], [], []
         for li, L in enumerate(wl.layers):
             W = synth.layer_weights(L, 64, 64, seed, torch.bfloat16, layer_id=li)   # decode reads sink/biases only
-            lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=wl.idx_key_dtype,
-                             max_ctas=self.side_ctas if li > 0 else self.main_ctas)
+            lh = LayerHandle(L, W, 64, 64, torch.bfloat16, B, idx_key_dtype=self.idx_key_dtype,
+                             max_ctas=self.side_ctas if li > 0 else self.main_ctas, kv_mixed=kv_mixed)
             lcm = 32
             cap = ((pos // L.m + 8 + lcm - 1) // lcm) * lcm
-            ch = CacheHandle(L, B, cap, torch.bfloat16, idx_key_dtype=wl.idx_key_dtype)
+            ch = CacheHandle(L, B, cap, torch.bfloat16, idx_key_dtype=self.idx_key_dtype, kv_mixed=kv_mixed)
             s = 1000 * (li + 1)
-            ch.kv_comp.copy_(dev_normal(ch.kv_comp.shape, seed, s + 1, torch.bfloat16))
-            ch.win.copy_(dev_normal(ch.win.shape, seed, s + 2, torch.bfloat16))
+            if kv_mixed:
+                # mixed-precision records of N(0,1) rows
+                for buf, sid in ((ch.kv_comp, 1), (ch.win, 2)):
+                    rows = buf.shape[0] * buf.shape[1]
+                    hb.kv_quant_mixed(dev_normal((rows, L.c), seed, s + sid, torch.bfloat16), hb.HCA_BF16, rows,
+                                      L.c, L.rd, buf)
+            else:
+                ch.kv_comp.copy_(dev_normal(ch.kv_comp.shape, seed, s + 1, torch.bfloat16))
+                ch.win.copy_(dev_normal(ch.win.shape, seed, s + 2, torch.bfloat16))
             ch.state_kv.copy_(dev_normal(ch.state_kv.shape, seed, s + 3))
             ch.state_score.copy_(dev_normal(ch.state_score.shape, seed, s + 4))
             if L.kind == "csa":
                 kf = dev_normal(ch.key_I.shape, seed, s + 5)
-                if wl.idx_key_dtype == "fp8":
+                if self.idx_key_dtype == "fp8":
                     kb, ks = synth.fp8_rows(kf)
                     ch.key_I.copy_(kb)
                     ch.key_I_scale.copy_(ks)
+                elif self.idx_key_dtype == "fp4":
+                    # rotated FP4 keys (carried in bf16), as the compressor stores them
+                    rows = kf.shape[0] * kf.shape[1]
+                    hb.fp4_rotate_quant(kf.contiguous(), hb.HCA_F32, rows, kf.shape[2], ch.key_I)
                 else:
                     ch.key_I.copy_(kf.to(torch.bfloat16))
                 ch.stateI_kv.copy_(dev_normal(ch.stateI_kv.shape, seed, s + 6))
@@ -264,13 +277,14 @@ class DecodeBench:
             V = (pos + 1) // L.m
             nw = min(L.w, pos + 1)
             qo = 2 * B * L.n_h * L.c * 2
+            row = hb.kv_mixed_row_bytes(L.c, L.rd) if self.kv_mixed else L.c * 2   # bytes per KV row
             if L.kind == "csa":
-                kb = 1 if wl.idx_key_dtype == "fp8" else 2
+                kb = 1 if self.idx_key_dtype == "fp8" else 2
                 per["index_scores"] = B * V * (L.c_I * kb + (4 if kb == 1 else 0)) + B * L.n_hI * (L.c_I * 2 + 4)
                 per["topk"] = B * V * 4 + B * L.k * 4          # scores in, indices out
-                per["attend_csa"] = B * (min(L.k, V) + nw) * L.c * 2 + qo
+                per["attend_csa"] = B * (min(L.k, V) + nw) * row + qo
             else:
-                per["attend_hca"] = B * (V + nw) * L.c * 2 + qo
+                per["attend_hca"] = B * (V + nw) * row + qo
         # the step's total counts the method's own streams (keys, rows, q/o), not the scores
         # the selection reads back
         return sum(v for k, v in per.items() if k != "topk"), per
@@ -356,8 +370,8 @@ def time_e2e_pipelined(b, K, W, stream):
     return t0.elapsed_time(t1) / K
 
 
-def run_decode(wl, K, W, flush, stream, e2e=True, sweep=False):
-    b = DecodeBench(wl)
+def run_decode(wl, K, W, flush, stream, e2e=True, sweep=False, **variant):
+    b = DecodeBench(wl, **variant)
     for _ in range(W):
         b.step()
     torch.cuda.synchronize()
@@ -524,12 +538,14 @@ def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, traffic=None):
             "peak_source": f"{peaks['src']} (hbm_gbs copy test)"}
 
 
-def roofline_tensor(flops_per_launch, ms_per_launch, peaks, sustained=True, traffic=None):
-    pk = peaks["bf16_sus"] if sustained else peaks["bf16"]
+def roofline_tensor(flops_per_launch, ms_per_launch, peaks, traffic=None):
+    """Against the dense bf16 peak measured as a burst (the kernels are timed
+    alone within a layer of tens of ms); the sustained-peak fraction beside it."""
     ach = flops_per_launch / (ms_per_launch * 1e-3) / 1e12
-    return {"bound": "tensor", "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s",
-            "frac": round(ach / pk, 4), "traffic": traffic,
-            "peak_source": f"{peaks['src']} bf16 {'sustained' if sustained else 'burst'}"}
+    return {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16"], "unit": "TFLOP/s",
+            "frac": round(ach / peaks["bf16"], 4), "traffic": traffic,
+            "peak_source": f"{peaks['src']} dense bf16 (cuBLAS burst)",
+            "frac_of_sustained": round(ach / peaks["bf16_sus"], 4), "peak_sustained": peaks["bf16_sus"]}
 
 
 def kern_ms(kern, prefix, K):
@@ -644,6 +660,21 @@ def main():
                                "kernels": {k: round(v["ms"] / args.steps * 1e3, 2) for k, v in d1["kern"].items()}}
         del d1
         torch.cuda.empty_cache()
+        # the 128K step with the pages' storage formats: mixed-precision KV rows
+        # (f2: e4m3 + block scales, RoPE dims bf16) and the FP4 indexer path
+        # (f4: rotated FP4 keys carried in bf16, bf16 scores)
+        for key, variant in (("decode_128k_mixed_kv", dict(kv_mixed=True)),
+                             ("decode_128k_fp4_indexer", dict(idx_key_dtype="fp4"))):
+            dv = run_decode(wl, args.steps, args.warmup, flush, stream, e2e=False, **variant)
+            tb, pb = dv["bench"].algorithmic_bytes()
+            mv = statistics.mean(dv["ms"])
+            extras[key] = {"workload": wl.name + ("_kvmixed" if "kv_mixed" in variant else "_fp4idx"),
+                           "us_per_step": round(mv * 1e3, 2), "algorithmic_bytes_per_step": tb,
+                           "attention_row_bytes": hb.kv_mixed_row_bytes(512, 64) if "kv_mixed" in variant else 1024,
+                           "roofline_step": roofline_hbm(tb, mv, peaks),
+                           "kernels": {k: round(v["ms"] / args.steps * 1e3, 2) for k, v in dv["kern"].items()}}
+            del dv
+            torch.cuda.empty_cache()
         # prefill workloads (fewer steps: each is a whole layer)
         for key, pwl in (("prefill_64k", workloads.CSA_PREFILL), ("prefill_128k", workloads.CSA_PREFILL_128K),
                          ("hca_prefill", workloads.HCA_PREFILL)):
