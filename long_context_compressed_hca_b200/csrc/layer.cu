@@ -577,11 +577,15 @@ int hybrid_decode_step(const hca_layer *L, const hca_token_in *x, hca_cache *cac
       const bool ov = cd.overlap != 0;
       rc = compress_params(&cd, pos, 1, cz, ov ? cz + a.c : nullptr, cz + (csa ? 2 : 1) * a.c, ov ? cz + 3 * a.c : nullptr,
                            (long long)ncz * a.c, (long long)ncz * a.c, L->B_comp, ov ? L->B_comp + a.m * a.c : nullptr,
-                           nullptr, a.kv_mixed ? mix_entry : cache->kv_comp, nullptr, a.kv_mixed ? 1 : cache->cap,
-                           cache->state_kv, cache->state_score, &pm);
+                           nullptr, cache->kv_comp, nullptr, cache->cap, cache->state_kv, cache->state_score, &pm);
       if (rc) return rc;
-      // mixed-precision KV: the emitted entry lands in a one-row bf16 scratch
-      if (a.kv_mixed) pm.e_first = pos / a.m;
+      if (a.kv_mixed) {
+        // mixed-precision KV: the emitted entry lands in a one-row bf16 scratch
+        // per sequence (quantised into the cache below)
+        pm.out = mix_entry;
+        pm.out_seq_stride = 1;
+        pm.e_first = pos / a.m;
+      }
     }
     if (csa) {
       hca_compress_desc cd{};
