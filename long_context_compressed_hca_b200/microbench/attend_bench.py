@@ -2,7 +2,7 @@
 print the per-role wait-cycle trace.
 
     python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c]
-    python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos] [max_ctas]
+    python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos] [max_ctas] [mixed]
 
 Inputs are seeded N(0,1) (bf16); CSA index lists take one random visible entry
 per equal-width bucket (valid, sorted, no repeats)."""
@@ -21,6 +21,7 @@ def decode_main():
     B = int(sys.argv[3]) if len(sys.argv) > 3 else 32
     pos = int(sys.argv[4]) if len(sys.argv) > 4 else 131072
     max_ctas = int(sys.argv[5]) if len(sys.argv) > 5 else 0
+    mixed = len(sys.argv) > 6 and sys.argv[6] == "mixed"   # mixed-precision KV records
     n_h, c, rd, w = 64, 512, 64, 128
     m, k = (4, 512) if kind == "csa" else (128, 0)
     V = (pos + 1) // m
@@ -29,6 +30,13 @@ def decode_main():
     q = synth.normal_on(dev, (B, 1, n_h, c), 2, 1, dtype=torch.bfloat16)
     kv = synth.normal_on(dev, (B, cap, c), 2, 2, dtype=torch.bfloat16)
     ring = synth.normal_on(dev, (B, w, c), 2, 3, dtype=torch.bfloat16)
+    if mixed:
+        rec = hb.kv_mixed_row_bytes(c, rd)
+        kvr = torch.empty(B * cap * rec, dtype=torch.uint8, device=dev)
+        rr = torch.empty(B * w * rec, dtype=torch.uint8, device=dev)
+        hb.kv_quant_mixed(kv, hb.HCA_BF16, B * cap, c, rd, kvr)
+        hb.kv_quant_mixed(ring, hb.HCA_BF16, B * w, c, rd, rr)
+        kv, ring = kvr, rr
     sink = synth.normal_on(dev, (n_h,), 2, 4)
     idx = None
     if kind == "csa":
@@ -38,7 +46,7 @@ def decode_main():
         u = torch.rand(B, k, device=dev, generator=g)
         idx = torch.floor((j[None] + u) * (V / k)).long().clamp(max=V - 1).int()[:, None].contiguous()
     o = torch.empty(B, 1, n_h, c, dtype=torch.bfloat16, device=dev)
-    d = hb.attn_desc(B, n_h, c, rd, w, m, k=max(k, 1), dtype=hb.HCA_BF16, max_ctas=max_ctas)
+    d = hb.attn_desc(B, n_h, c, rd, w, m, k=max(k, 1), dtype=hb.HCA_BF16, max_ctas=max_ctas, kv_mixed=int(mixed))
     wsz = (hb.csa_attend_workspace_size if kind == "csa" else hb.hca_attend_workspace_size)(d, 1, pos)
     ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
 
@@ -86,7 +94,7 @@ def decode_main():
     prof = hb.profile_collect()
     hb.profile_enable(False)
     keys = min(w, pos + 1) + (min(k, V) if kind == "csa" else V)
-    byts = B * (keys * c * 2 + 2 * n_h * c * 2)
+    byts = B * (keys * (hb.kv_mixed_row_bytes(c, rd) if mixed else c * 2) + 2 * n_h * c * 2)
     for name, (n, ms) in prof.items():
         print(f"{name}: {ms / n * 1e3:.1f} us per launch ({n} launches)")
     att = [v for kk, v in prof.items() if kk.startswith("attend_") and kk.endswith("tc")][0]
