@@ -449,6 +449,19 @@ int hca_step_trace(void *buf, size_t bytes);
  * enable >= 0 then resets them and sets the mode, enable < 0 only reads. */
 int hca_trace_attend(int enable, unsigned long long *host_counters, int n);
 
+/* Which kernel runs the top-k selection of csa_index_topk (and of the layer
+ * calls that use it), for tests and measurements: 0 = chosen by shape (the
+ * default), 1 = one CTA per row (rows of up to 32768 keys in registers),
+ * 2 = one warp per row (rows of up to 32768 keys; many rows), 3 = the
+ * segmented cluster radix select, 4 = one thread-block cluster per row
+ * (rows all longer than k).  A mode whose kernel does not take the shape
+ * falls back to the segmented select, so every mode is exact for every
+ * shape.  Returns the previous mode;
+ * mode < 0 only reads it.  Process-wide setting (not per device or stream);
+ * workspace sizes depend on it for mode 3, so size workspaces after setting
+ * it.  Errors: HCA_ERR_INVALID for mode > 4. */
+int hca_topk_kernel(int mode);
+
 #ifdef __cplusplus
 }
 #endif

@@ -89,6 +89,7 @@ def _declare(L):
         "hca_profile_sample": (I, []),
         "hca_profile_collect": (I, [C.c_char_p, SZ]),
         "hca_trace_attend": (I, [I, C.POINTER(C.c_ulonglong), I]),
+        "hca_topk_kernel": (I, [I]),
         "csa_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
                              VP, LL, VP, VP, VP]),
         "csa_index_topk_workspace_size": (SZ, [C.POINTER(AttnDesc), I, I]),
@@ -214,6 +215,17 @@ TRACE_SLOTS = ("prod_q_free", "prod_stage_free", "mma_q_ready", "mma_tile_ready"
                "smax_epi_wait", "-", "epilogue", "total", "rescales", "units", "tiles", "-",
                "merge_wait_ready", "merge_wait_full", "merge_push", "merge_weights", "merge_loop",
                "t_setup", "t_first_s", "t_tiles", "t_epilogue", "t_exit", "t_entry_inv", "t_exit_max", "t_ctas")
+
+
+TOPK_AUTO, TOPK_ROW, TOPK_WARP, TOPK_CLUSTER, TOPK_ROW_CLUSTER = 0, 1, 2, 3, 4
+
+
+def topk_kernel(mode: int = -1) -> int:
+    """Select the top-k kernel (TOPK_*; -1 only reads); returns the previous mode."""
+    r = lib().hca_topk_kernel(mode)
+    if r < 0:
+        check(r)
+    return r
 
 
 def trace_attend(enable: int):

@@ -6,10 +6,13 @@
 // Selection (Eq.(17)): the min(k, V_t) highest scores, ties broken towards the
 // lower entry index, emitted in ascending index order and padded with -1.
 //
-// The selection is an exact radix select on the order-preserving uint32 image
-// of the fp32 scores (three digits of 11, 11 and 10 bits, 2048 bins), run by a thread-block cluster
-// whose CTAs hold slices of the row in shared memory and sum their histograms
-// through distributed shared memory, followed by a stable compaction.
+// The selection is exact on the order-preserving uint32 image of the fp32
+// scores, by one of four kernels chosen by shape: many rows (prefill) take a
+// warp per row (sampled thresholds, one pass, radix select within the band);
+// a few rows of up to 32768 keys a CTA per row (the row in registers); a few
+// longer rows a thread-block cluster per row; the general fallback is a
+// segmented radix select (digits of 11, 11 and 10 bits) by thread-block
+// clusters that sum their histograms through distributed shared memory.
 #include <mutex>
 
 #include "common.cuh"
@@ -90,7 +93,9 @@ __global__ void __launch_bounds__(kScoreThreads) index_scores_simt(IndexParams p
 // index order with ties resolved towards the lower index.  Rows longer than
 // one segment are cut into segments whose winners (order key + index) a
 // second launch merges.
-bool g_topk_row_enabled = true;   // one CTA per row where the row fits (else clusters)
+// selection kernel: 0 = by shape, 1 = a CTA per row, 2 = a warp per row,
+// 3 = the segmented cluster select, 4 = a cluster per row (hca_topk_kernel)
+int g_topk_kernel = 0;
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kSliceMax = 16384;   // keys per CTA (64 KB of shared memory)
@@ -743,6 +748,320 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
   }
 }
 
+// ------------------------------------------------------- a warp per row
+// Many rows (prefill): each warp of a CTA selects one row, with no block-wide
+// barrier, so that many rows are in flight per SM and the pass over the
+// scores runs at the memory rate.  Per row:
+//   1. a sample of the row (128 evenly spaced runs of 8 keys, one 32-byte
+//      sector each; the whole row when it has at most 1024 keys) gives, by
+//      bisection on the order keys, two thresholds: keys above hiK are
+//      winners, keys in [loK, hiK] are the band, which holds the k-th largest
+//      unless the sample misled (then step 3's fallback decides);
+//   2. one pass over the row (4 keys per lane per step, 128 consecutive keys
+//      per warp step, 8 steps' loads in flight): winners go to a bit mask of the row, band keys (order
+//      key + index) to a list in shared memory in ascending index order;
+//   3. if the winners number below k and winners + band reach k (and the band
+//      fitted its list), an exact radix select over the band finds the k-th
+//      largest key T and how many keys equal to T are kept (krem); the band's
+//      keys above T and its first krem keys equal to T (lowest indices) join
+//      the mask.  Otherwise an exact radix select over the whole row (read
+//      again from memory) decides, and a last pass marks the mask;
+//   4. the mask's bits are emitted in ascending index order.
+// Every decision is exact; the sample only decides how much of the row the
+// exact select looks at.
+constexpr int kWarpRowWarps = 8;                 // warps (rows) per CTA
+constexpr int kWarpRowMaxWords = kRowMax / 32;   // mask words of the longest row
+constexpr int kWarpRowCand = 1536;               // band keys held per warp
+constexpr int kWarpRowSample = 1024;             // sample keys per row (32 per lane)
+constexpr int kWarpRowUnroll = 8;                // 16-byte loads in flight per lane
+// 13 KB per warp: two CTAs of 8 warps fit an SM
+struct WarpRowSmem {
+  uint32_t mask[kWarpRowMaxWords];
+  uint32_t cand_key[kWarpRowCand];
+  uint16_t cand_idx[kWarpRowCand];   // indices < kRowMax = 32768
+};
+static_assert(kRowMax <= 65536, "band indices are 16-bit");
+
+// Spread the 8 bits of b to bit positions 0, 4, 8, ..., 28.
+__device__ __forceinline__ uint32_t spread4(uint32_t b) {
+  b = (b | (b << 12)) & 0x000F000Fu;
+  b = (b | (b << 6)) & 0x03030303u;
+  b = (b | (b << 3)) & 0x11111111u;
+  return b;
+}
+
+// The r-th largest (r >= 1) of the warp's sample keys (NS per lane), found
+// bit by bit: the largest key value x with at least r sample keys >= x.
+template <int NS>
+__device__ __forceinline__ uint32_t warp_rank_key(const uint32_t (&s)[NS], int r) {
+  uint32_t x = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t c = x | (1u << bit);
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < NS; ++i) n += s[i] >= c ? 1 : 0;
+    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)n) >= r) x = c;
+  }
+  return x;
+}
+
+// Exact radix select (digits of up to 8 bits from the highest bit in which
+// kmin and kmax differ) of the krem-th largest key among those each(f)
+// visits (every lane calls f on its share), with a 256-bin histogram in
+// shared memory.  Returns the key; *krem becomes how many keys equal to it
+// are kept.
+template <typename Each>
+__device__ uint32_t warp_radix_select(uint32_t *hist, uint32_t kmin, uint32_t kmax, int *krem, Each each) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t range = kmax - kmin;
+  int shift = range ? 32 - __clz(range) : 0;
+  uint32_t prefix = 0;
+  while (shift > 0) {
+    const int width = shift > 8 ? 8 : shift;
+    const int nshift = shift - width;
+    for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+    __syncwarp();
+    each([&](uint32_t kk) {
+      if (kk < kmin || kk > kmax) return;
+      const uint32_t v = kk - kmin;
+      if (shift >= 32 || (v >> shift) == prefix) atomicAdd(&hist[(v >> nshift) & ((1u << width) - 1u)], 1u);
+    });
+    __syncwarp();
+    // lane l holds bins 255-8l .. 248-8l (from the top); counts above each lane's bins
+    uint32_t h[8];
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      h[j] = hist[255 - 8 * lane - j];
+      sum += (int)h[j];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int above = incl - sum;
+    int found = -1, kin = 0;
+    if (above < *krem && incl >= *krem) {
+      int a = above;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (found < 0 && a + (int)h[j] >= *krem) {
+          found = 255 - 8 * lane - j;
+          kin = *krem - a;
+        }
+        a += (int)h[j];
+      }
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+    const int src = __ffs(who) - 1;
+    const int digit = __shfl_sync(0xffffffffu, found, src);
+    *krem = __shfl_sync(0xffffffffu, kin, src);
+    prefix = (prefix << width) | (uint32_t)digit;
+    shift = nshift;
+    __syncwarp();
+  }
+  return kmin + prefix;
+}
+
+__global__ void __launch_bounds__(kWarpRowWarps * 32) topk_warp(TopkParams p) {
+  extern __shared__ __align__(16) uint8_t dyn_raw[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WarpRowSmem &sm = reinterpret_cast<WarpRowSmem *>(dyn_raw)[warp];
+  __shared__ uint32_t hist_all[kWarpRowWarps][256];
+  uint32_t *hist = hist_all[warp];
+  const long long row = (long long)blockIdx.x * kWarpRowWarps + warp;
+  const unsigned long long st_entry = global_ns();
+  pdl_trigger();   // the attention may start its prologue
+  pdl_wait();      // the scores of the previous launch are complete
+  const unsigned long long st_ready = global_ns();
+  if (row >= p.rows || p.k <= 0) return;
+  const int V = p.fixed_len > 0 ? p.fixed_len : (p.start_pos + (int)(row % p.n_q) + 1) / p.m;
+  const int k = p.k;
+  int32_t *out = p.idx_out + row * p.out_stride;
+  const float *src = p.scores + row * p.in_stride;
+  const uint32_t *srcu = reinterpret_cast<const uint32_t *>(src);
+  const int nwords = (V + 31) >> 5;
+  if (V <= k) {
+    for (int i = lane; i < k; i += 32) out[i] = i < V ? i : -1;
+    return;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+
+  // ---- 1. sample and thresholds
+  constexpr int NS = kWarpRowSample / 32;
+  const int S = V < kWarpRowSample ? V : kWarpRowSample;
+  uint32_t s[NS];
+  if (V <= kWarpRowSample) {
+#pragma unroll
+    for (int i = 0; i < NS; ++i) s[i] = 32 * i + lane < V ? order_bits(__ldg(srcu + 32 * i + lane)) : 0u;
+  } else {
+    // lane l reads runs 4l .. 4l+3; run j starts at the multiple of 8 at or
+    // below (2j+1) V / 256, kept inside the row
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = 4 * lane + r;
+      const int st = min(V - 8, (int)(((long long)(2 * j + 1) * V) / 256) & ~7);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[8 * r + e] = order_bits(__ldg(srcu + st + e));
+    }
+  }
+  const float q = (float)k * (float)S / (float)V;   // sample keys expected above the k-th
+  const float mg = 2.6f * sqrtf(q) + 1.f;
+  const int r_hi = max(1, (int)floorf(q - mg));
+  const int r_lo = min(S, (int)ceilf(q + mg));
+  // winners: keys > hiK (none when the sample's top is within the margin);
+  // band: keys in [loK, hiK]
+  const uint32_t hiK = q - mg >= 1.f ? warp_rank_key<NS>(s, r_hi) : 0xFFFFFFFFu;
+  const uint32_t loK = warp_rank_key<NS>(s, r_lo);
+
+  // ---- 2. one pass: winner bits and band keys
+  int nwin = 0, ncand = 0;
+  const int steps = (V + 127) >> 7;
+#pragma unroll 1
+  for (int st0 = 0; st0 < steps; st0 += kWarpRowUnroll) {
+    uint32_t kv[kWarpRowUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kWarpRowUnroll; ++u) {
+      const int i0 = (st0 + u) * 128 + 4 * lane;
+      if (vec && i0 + 3 < V) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(srcu + i0));
+        kv[u][0] = w.x; kv[u][1] = w.y; kv[u][2] = w.z; kv[u][3] = w.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) kv[u][e] = i0 + e < V ? __ldg(srcu + i0 + e) : 0u;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kWarpRowUnroll; ++u) {
+      const int st = st0 + u;
+      if (st >= steps) break;
+      const int i0 = st * 128 + 4 * lane;
+      uint32_t bw[4], bc[4];
+      int my_c = 0;
+      bool isc[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool valid = i0 + e < V;
+        const uint32_t ok = order_bits(kv[u][e]);
+        kv[u][e] = ok;
+        const bool w = valid && ok > hiK;
+        isc[e] = valid && !w && ok >= loK;
+        bw[e] = __ballot_sync(0xffffffffu, w);
+        bc[e] = __ballot_sync(0xffffffffu, isc[e]);
+        my_c += isc[e] ? 1 : 0;
+      }
+      if (lane < 4) {
+        const int sh = 8 * lane;
+        sm.mask[st * 4 + lane] = spread4((bw[0] >> sh) & 0xFFu) | (spread4((bw[1] >> sh) & 0xFFu) << 1) |
+                                 (spread4((bw[2] >> sh) & 0xFFu) << 2) | (spread4((bw[3] >> sh) & 0xFFu) << 3);
+      }
+      nwin += __popc(bw[0]) + __popc(bw[1]) + __popc(bw[2]) + __popc(bw[3]);
+      if (bc[0] | bc[1] | bc[2] | bc[3]) {
+        int at = ncand + __popc(bc[0] & lt) + __popc(bc[1] & lt) + __popc(bc[2] & lt) + __popc(bc[3] & lt);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (isc[e]) {
+            if (at < kWarpRowCand) {
+              sm.cand_key[at] = kv[u][e];
+              sm.cand_idx[at] = (uint16_t)(i0 + e);
+            }
+            ++at;
+          }
+        ncand += __popc(bc[0]) + __popc(bc[1]) + __popc(bc[2]) + __popc(bc[3]);
+      }
+    }
+  }
+  __syncwarp();
+
+  // ---- 3. the k-th largest key T and the ties kept
+  if (nwin < k && nwin + ncand >= k && ncand <= kWarpRowCand) {
+    uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
+    for (int i = lane; i < ncand; i += 32) {
+      cmin = min(cmin, sm.cand_key[i]);
+      cmax = max(cmax, sm.cand_key[i]);
+    }
+    cmin = __reduce_min_sync(0xffffffffu, cmin);
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
+    int krem = k - nwin;
+    const uint32_t T = warp_radix_select(hist, cmin, cmax, &krem, [&](auto f) {
+      for (int i = lane; i < ncand; i += 32) f(sm.cand_key[i]);
+    });
+    // band keys above T, then the first krem keys equal to T (index order)
+    int ties = 0;
+    for (int c0 = 0; c0 < ncand; c0 += 32) {
+      const int i = c0 + lane;
+      const uint32_t kk = i < ncand ? sm.cand_key[i] : 0u;
+      const bool gt = i < ncand && kk > T, eq = i < ncand && kk == T;
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && ties + __popc(be & lt) < krem);
+      if (take) {
+        const uint32_t ix = sm.cand_idx[i];
+        atomicOr(&sm.mask[ix >> 5], 1u << (ix & 31));
+      }
+      ties += __popc(be);
+    }
+  } else {
+    // the band missed: exact select over the whole row, read again
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = lane; i < V; i += 32) {
+      const uint32_t kk = order_bits(__ldg(srcu + i));
+      kmin = min(kmin, kk);
+      kmax = max(kmax, kk);
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    int krem = k;
+    const uint32_t T = warp_radix_select(hist, kmin, kmax, &krem, [&](auto f) {
+      for (int i = lane; i < V; i += 32) f(order_bits(__ldg(srcu + i)));
+    });
+    // mark: keys above T, then the first krem keys equal to T in index order
+    int ties = 0;
+    for (int w0 = 0; w0 < nwords; ++w0) {
+      const int i = 32 * w0 + lane;
+      const uint32_t kk = i < V ? order_bits(__ldg(srcu + i)) : 0u;
+      const bool gt = i < V && kk > T, eq = i < V && kk == T;
+      const uint32_t be = __ballot_sync(0xffffffffu, eq);
+      const bool take = gt || (eq && ties + __popc(be & lt) < krem);
+      const uint32_t word = __ballot_sync(0xffffffffu, take);
+      if (lane == 0) sm.mask[w0] = word;
+      ties += __popc(be);
+    }
+  }
+  __syncwarp();
+
+  // ---- 4. emit in ascending index order (exactly k bits are set): lane l
+  // takes words [l*wpl, (l+1)*wpl)
+  const int wpl = (nwords + 31) >> 5;
+  int cnt = 0;
+  for (int j = 0; j < wpl; ++j) {
+    const int w = lane * wpl + j;
+    if (w < nwords) cnt += __popc(sm.mask[w]);
+  }
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int at = incl - cnt;
+  for (int j = 0; j < wpl; ++j) {
+    const int w = lane * wpl + j;
+    if (w >= nwords) break;
+    uint32_t m = sm.mask[w];
+    while (m) {
+      const int b = __ffs(m) - 1;
+      if (at < k) out[at] = 32 * w + b;
+      ++at;
+      m &= m - 1u;
+    }
+  }
+  if (step_trace_on() && lane == 0) step_trace_record(ST_TOPK, st_entry, st_ready);
+}
+
 // ------------------------------------------------------ a cluster per row
 // Few long rows (decode): the row is cut over the C CTAs of a thread-block
 // cluster, each holding 32 keys per thread in registers, so that every pass
@@ -1127,6 +1446,35 @@ int launch_topk_row_t(const TopkParams &t, long long rows, int Vmax, cudaStream_
   }
   return ls.done();
 }
+// A warp per row for many rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise).
+int launch_topk_warp(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
+  if (Vmax > kRowMax || rows > 0x7FFFFFFFLL) return HCA_ERR_UNSUPPORTED;
+  const size_t smem = kWarpRowWarps * sizeof(WarpRowSmem);
+  static std::atomic<bool> attr_dev[kMaxDevices];
+  std::atomic<bool> &attr = attr_dev[device_slot()];
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k warp smem attribute: %s", cudaGetErrorString(e));
+    attr = true;
+  }
+  LaunchScope ls("topk", s);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)((rows + kWarpRowWarps - 1) / kWarpRowWarps), 1, 1);
+  cfg.blockDim = dim3(kWarpRowWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_warp, t);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return fail(HCA_ERR_CUDA, "topk_warp launch: %s", cudaGetErrorString(e));
+  }
+  return ls.done();
+}
 // One CTA per row for rows of up to kRowMax keys (HCA_ERR_UNSUPPORTED otherwise);
 // the longest rows take 64 keys per thread in 512 threads (no register spills).
 int launch_topk_row(const TopkParams &t, long long rows, int Vmax, cudaStream_t s) {
@@ -1223,7 +1571,7 @@ size_t topk_workspace_bytes(const IndexParams &p) {
   const TopkPlan pl = plan_topk(rows, Vmax);
   size_t b = (size_t)rows * (size_t)Vmax * sizeof(float);           // scores
   b = (b + 255) & ~(size_t)255;
-  if (pl.n_seg > 1 && !(Vmax <= kRowMax && g_topk_row_enabled)) {
+  if (pl.n_seg > 1 && !(Vmax <= kRowMax && g_topk_kernel != 3)) {
     const size_t c = (size_t)rows * pl.n_seg * p.k;
     b += 2 * ((c * sizeof(int32_t) + 255) & ~(size_t)255);          // winners' indices and keys
   }
@@ -1267,14 +1615,20 @@ int run_index_topk(const IndexParams &ip, int32_t *idx, float *user_scores, long
   t.rows = (int)rows; t.k = ip.k; t.scores = p.scores; t.in_stride = p.score_stride;
   t.n_q = ip.n_q; t.start_pos = ip.start_pos; t.m = ip.m;
   t.n_seg = pl.n_seg; t.seg_len = pl.seg_len; t.slice = pl.slice;
+  const int force = g_topk_kernel;
   // few rows, all longer than k (decode): a cluster per row
   const int Vmin = (ip.start_pos + 1) / ip.m;
-  if (Vmin > ip.k && rows * 8 <= 2LL * num_sms() && Vmax > kRowMax) {
+  if ((force == 0 && Vmin > ip.k && rows * 8 <= 2LL * num_sms() && Vmax > kRowMax) || (force == 4 && Vmin > ip.k)) {
     t.idx_out = idx; t.out_stride = ip.k;
     rc = launch_topk_rowc(t, rows, Vmax, s);
     if (rc != HCA_ERR_UNSUPPORTED) return rc;
   }
-  if (Vmax <= kRowMax && g_topk_row_enabled) {
+  // many rows (prefill): a warp per row
+  if (((force == 0 && rows >= 2LL * num_sms()) || force == 2) && Vmax <= kRowMax) {
+    t.idx_out = idx; t.out_stride = ip.k;
+    return launch_topk_warp(t, rows, Vmax, s);
+  }
+  if ((force == 0 || force == 1) && Vmax <= kRowMax) {
     t.idx_out = idx; t.out_stride = ip.k;
     return launch_topk_row(t, rows, Vmax, s);
   }
@@ -1356,3 +1710,11 @@ int run_index_topk_static(const IndexParams &p, int32_t *idx, float *user_scores
 int step_trace_set_index_topk(void *buf, unsigned long long cap) { return step_trace_set_here(buf, cap); }
 
 }  // namespace hca
+
+extern "C" int hca_topk_kernel(int mode) {
+  using namespace hca;
+  if (mode > 4) return fail(HCA_ERR_INVALID, "top-k kernel mode %d (0..4)", mode);
+  const int prev = g_topk_kernel;
+  if (mode >= 0) g_topk_kernel = mode;
+  return prev;
+}

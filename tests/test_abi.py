@@ -184,3 +184,13 @@ def test_workspace_map_places_intermediates_inside_the_workspace(L):
 def test_step_trace_rejects_bad_buffers(L):
     _bad(L.hca_step_trace(12, 1024), "8-byte aligned")
     _bad(L.hca_step_trace(16, 32), "8-byte aligned")
+
+
+def test_topk_kernel_knob_round_trip(L):
+    prev = hb.topk_kernel(hb.TOPK_WARP)
+    try:
+        assert hb.topk_kernel(-1) == hb.TOPK_WARP
+    finally:
+        hb.topk_kernel(prev)
+    assert hb.topk_kernel(-1) == prev
+    _bad(L.hca_topk_kernel(5), "top-k kernel mode")
