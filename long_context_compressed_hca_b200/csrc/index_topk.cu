@@ -752,20 +752,23 @@ __global__ void __launch_bounds__(NT) topk_row(TopkParams p) {
 // Many rows (prefill): each warp of a CTA selects one row, with no block-wide
 // barrier, so that many rows are in flight per SM and the pass over the
 // scores runs at the memory rate.  Per row:
-//   1. a sample of the row (128 evenly spaced runs of 8 keys, one 32-byte
-//      sector each; the whole row when it has at most 1024 keys) gives, by
-//      bisection on the order keys, two thresholds: keys above hiK are
+//   1. a sample of the row (32 to 128 evenly spaced runs of 8 keys, one
+//      32-byte sector each; the whole row when it has at most 1024 keys) gives, by
+//      radix select over the sample, two thresholds: keys above hiK are
 //      winners, keys in [loK, hiK] are the band, which holds the k-th largest
 //      unless the sample misled (then step 3's fallback decides);
-//   2. one pass over the row (4 keys per lane per step, 128 consecutive keys
-//      per warp step, 8 steps' loads in flight): winners go to a bit mask of the row, band keys (order
+//   2. one pass over the row (128 consecutive keys per warp step, 4 per lane,
+//      8 steps' loads in flight): winners go to a bit mask of the row, band keys (order
 //      key + index) to a list in shared memory in ascending index order;
 //   3. if the winners number below k and winners + band reach k (and the band
 //      fitted its list), an exact radix select over the band finds the k-th
 //      largest key T and how many keys equal to T are kept (krem); the band's
 //      keys above T and its first krem keys equal to T (lowest indices) join
-//      the mask.  Otherwise an exact radix select over the whole row (read
-//      again from memory) decides, and a last pass marks the mask;
+//      the mask.  Otherwise (rare) counting passes over the row narrow the
+//      range that holds the k-th largest, 256 bins at a time, until its bin
+//      fits the band list (the band pass then runs again on that bin) or is a
+//      single key value (a last pass marks the keys above it and its first
+//      ties);
 //   4. the mask's bits are emitted in ascending index order.
 // Every decision is exact; the sample only decides how much of the row the
 // exact select looks at.
@@ -773,7 +776,7 @@ constexpr int kWarpRowWarps = 8;                 // warps (rows) per CTA
 constexpr int kWarpRowMaxWords = kRowMax / 32;   // mask words of the longest row
 constexpr int kWarpRowCand = 1536;               // band keys held per warp
 constexpr int kWarpRowSample = 1024;             // sample keys per row (32 per lane)
-constexpr int kWarpRowUnroll = 8;                // 16-byte loads in flight per lane
+constexpr int kWarpRowUnroll = 8;                // steps whose loads are in flight together
 // 13 KB per warp: two CTAs of 8 warps fit an SM
 struct WarpRowSmem {
   uint32_t mask[kWarpRowMaxWords];
@@ -781,30 +784,7 @@ struct WarpRowSmem {
   uint16_t cand_idx[kWarpRowCand];   // indices < kRowMax = 32768
 };
 static_assert(kRowMax <= 65536, "band indices are 16-bit");
-
-// Spread the 8 bits of b to bit positions 0, 4, 8, ..., 28.
-__device__ __forceinline__ uint32_t spread4(uint32_t b) {
-  b = (b | (b << 12)) & 0x000F000Fu;
-  b = (b | (b << 6)) & 0x03030303u;
-  b = (b | (b << 3)) & 0x11111111u;
-  return b;
-}
-
-// The r-th largest (r >= 1) of the warp's sample keys (NS per lane), found
-// bit by bit: the largest key value x with at least r sample keys >= x.
-template <int NS>
-__device__ __forceinline__ uint32_t warp_rank_key(const uint32_t (&s)[NS], int r) {
-  uint32_t x = 0;
-#pragma unroll 1
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t c = x | (1u << bit);
-    int n = 0;
-#pragma unroll
-    for (int i = 0; i < NS; ++i) n += s[i] >= c ? 1 : 0;
-    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)n) >= r) x = c;
-  }
-  return x;
-}
+static_assert(kWarpRowSample <= kWarpRowCand, "the sample is held in the band list");
 
 // Exact radix select (digits of up to 8 bits from the highest bit in which
 // kmin and kmax differ) of the krem-th largest key among those each(f)
@@ -889,96 +869,198 @@ __global__ void __launch_bounds__(kWarpRowWarps * 32) topk_warp(TopkParams p) {
     return;
   }
   const uint32_t lt = (1u << lane) - 1u;
-  const bool vec = (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-
-  // ---- 1. sample and thresholds
-  constexpr int NS = kWarpRowSample / 32;
-  const int S = V < kWarpRowSample ? V : kWarpRowSample;
-  uint32_t s[NS];
-  if (V <= kWarpRowSample) {
+  const int steps = (V + 127) >> 7;
+  // One pass over the row in batches of 8 steps of 128 keys: f(st0, v) with
+  // v[u][e] = key 128 (st0 + u) + 32 e + lane (-inf past the row); a batch's
+  // loads are all in flight together and the next batch's lines are
+  // prefetched to L2.
+  auto scan_row = [&](auto f) {
+#pragma unroll 1
+    for (int st0 = 0; st0 < steps; st0 += kWarpRowUnroll) {
+      float v[kWarpRowUnroll][4];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) s[i] = 32 * i + lane < V ? order_bits(__ldg(srcu + 32 * i + lane)) : 0u;
+      for (int u = 0; u < kWarpRowUnroll; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = (st0 + u) * 128 + 32 * e + lane;
+          v[u][e] = i < V ? __ldg(src + i) : -INFINITY;
+        }
+      {
+        const int i = (st0 + kWarpRowUnroll) * 128 + 32 * lane;
+        if (i < V) asm volatile("prefetch.global.L2 [%0];" ::"l"(src + i));
+      }
+      f(st0, v);
+    }
+  };
+
+  // ---- 1. sample (order keys into the band list, which is free until step
+  // 2) and thresholds: the r_hi-th and r_lo-th largest sample keys, by radix
+  // select over the sample
+  // S scales with k V so that the band holds ~800 keys whatever the row length
+  // (q = k S / V stays near k^2 / 16384): 256, 512 or 1024 sample keys
+  const long long kv = (long long)k * V;
+  const int S = V <= kWarpRowSample ? V : (kv <= (4ll << 20) ? 256 : (kv <= (8ll << 20) ? 512 : 1024));
+  if (V <= kWarpRowSample) {
+    for (int i = lane; i < S; i += 32) sm.cand_key[i] = order_bits(__ldg(srcu + i));
   } else {
-    // lane l reads runs 4l .. 4l+3; run j starts at the multiple of 8 at or
-    // below (2j+1) V / 256, kept inside the row
+    // S/8 runs of 8 keys, R = S/256 per lane; run j starts at the multiple of
+    // 8 at or below (2j+1) V / (S/4), kept inside the row
+    const int R = S >> 8;
+    uint32_t sv[32];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int j = 4 * lane + r;
-      const int st = min(V - 8, (int)(((long long)(2 * j + 1) * V) / 256) & ~7);
+      if (r < R) {
+        const int j = R * lane + r;
+        const int st = min(V - 8, (int)(((long long)(2 * j + 1) * V * 4) / S) & ~7);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s[8 * r + e] = order_bits(__ldg(srcu + st + e));
-    }
-  }
-  const float q = (float)k * (float)S / (float)V;   // sample keys expected above the k-th
-  const float mg = 2.6f * sqrtf(q) + 1.f;
-  const int r_hi = max(1, (int)floorf(q - mg));
-  const int r_lo = min(S, (int)ceilf(q + mg));
-  // winners: keys > hiK (none when the sample's top is within the margin);
-  // band: keys in [loK, hiK]
-  const uint32_t hiK = q - mg >= 1.f ? warp_rank_key<NS>(s, r_hi) : 0xFFFFFFFFu;
-  const uint32_t loK = warp_rank_key<NS>(s, r_lo);
-
-  // ---- 2. one pass: winner bits and band keys
-  int nwin = 0, ncand = 0;
-  const int steps = (V + 127) >> 7;
-#pragma unroll 1
-  for (int st0 = 0; st0 < steps; st0 += kWarpRowUnroll) {
-    uint32_t kv[kWarpRowUnroll][4];
-#pragma unroll
-    for (int u = 0; u < kWarpRowUnroll; ++u) {
-      const int i0 = (st0 + u) * 128 + 4 * lane;
-      if (vec && i0 + 3 < V) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(srcu + i0));
-        kv[u][0] = w.x; kv[u][1] = w.y; kv[u][2] = w.z; kv[u][3] = w.w;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) kv[u][e] = i0 + e < V ? __ldg(srcu + i0 + e) : 0u;
+        for (int e = 0; e < 8; ++e) sv[8 * r + e] = __ldg(srcu + st + e);
       }
     }
 #pragma unroll
-    for (int u = 0; u < kWarpRowUnroll; ++u) {
-      const int st = st0 + u;
-      if (st >= steps) break;
-      const int i0 = st * 128 + 4 * lane;
-      uint32_t bw[4], bc[4];
-      int my_c = 0;
-      bool isc[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const bool valid = i0 + e < V;
-        const uint32_t ok = order_bits(kv[u][e]);
-        kv[u][e] = ok;
-        const bool w = valid && ok > hiK;
-        isc[e] = valid && !w && ok >= loK;
-        bw[e] = __ballot_sync(0xffffffffu, w);
-        bc[e] = __ballot_sync(0xffffffffu, isc[e]);
-        my_c += isc[e] ? 1 : 0;
-      }
-      if (lane < 4) {
-        const int sh = 8 * lane;
-        sm.mask[st * 4 + lane] = spread4((bw[0] >> sh) & 0xFFu) | (spread4((bw[1] >> sh) & 0xFFu) << 1) |
-                                 (spread4((bw[2] >> sh) & 0xFFu) << 2) | (spread4((bw[3] >> sh) & 0xFFu) << 3);
-      }
-      nwin += __popc(bw[0]) + __popc(bw[1]) + __popc(bw[2]) + __popc(bw[3]);
-      if (bc[0] | bc[1] | bc[2] | bc[3]) {
-        int at = ncand + __popc(bc[0] & lt) + __popc(bc[1] & lt) + __popc(bc[2] & lt) + __popc(bc[3] & lt);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (isc[e]) {
-            if (at < kWarpRowCand) {
-              sm.cand_key[at] = kv[u][e];
-              sm.cand_idx[at] = (uint16_t)(i0 + e);
-            }
-            ++at;
-          }
-        ncand += __popc(bc[0]) + __popc(bc[1]) + __popc(bc[2]) + __popc(bc[3]);
-      }
-    }
+    for (int i = 0; i < 32; ++i)
+      if (i < 8 * R) sm.cand_key[32 * i + lane] = order_bits(sv[i]);
   }
   __syncwarp();
+  uint32_t smin = 0xFFFFFFFFu, smax = 0u;
+  for (int i = lane; i < S; i += 32) {
+    smin = min(smin, sm.cand_key[i]);
+    smax = max(smax, sm.cand_key[i]);
+  }
+  smin = __reduce_min_sync(0xffffffffu, smin);
+  smax = __reduce_max_sync(0xffffffffu, smax);
+  auto sample_rank = [&](int r) {
+    return warp_radix_select(hist, smin, smax, &r, [&](auto f) {
+      for (int i = lane; i < S; i += 32) f(sm.cand_key[i]);
+    });
+  };
+  const float q = (float)k * (float)S / (float)V;   // sample keys expected above the k-th
+  const float mg = 3.f * sqrtf(q) + 1.f;
+  // winners: keys > hiK (none when the sample's top is within the margin);
+  // band: keys in [loK, hiK]
+  uint32_t hiK = q - mg >= 1.f ? sample_rank(max(1, (int)floorf(q - mg))) : 0xFFFFFFFFu;
+  uint32_t loK = sample_rank(min(S, (int)ceilf(q + mg)));
+  __syncwarp();   // the sample is read before the band list is written
 
-  // ---- 3. the k-th largest key T and the ties kept
-  if (nwin < k && nwin + ncand >= k && ncand <= kWarpRowCand) {
+  // ---- 2. one pass: winner bits (vote over e = mask word 4 st + e) and the
+  // band keys in ascending index order (e first, then lane).  Thresholds
+  // compare as floats (the order of non-NaN floats, -0 == +0).
+  int nwin = 0, ncand = 0;
+  auto band_pass = [&]() {
+    // order keys from +inf up (and the NaN images above it) bound nothing
+    const float hiF = hiK >= 0xFF800000u ? INFINITY : key_float(hiK), loF = key_float(loK);
+    nwin = 0;
+    ncand = 0;
+    // branch-free over the batch (votes first, then the band appends), so
+    // that the steps' work interleaves
+    scan_row([&](int st0, const float (&v)[kWarpRowUnroll][4]) {
+      uint32_t bc[kWarpRowUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kWarpRowUnroll; ++u) {
+        const int st = st0 + u;
+        uint32_t bw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool in = st * 128 + 32 * e + lane < V;
+          const bool w = in && v[u][e] > hiF;
+          bw[e] = __ballot_sync(0xffffffffu, w);
+          bc[u][e] = __ballot_sync(0xffffffffu, in && !w && v[u][e] >= loF);
+        }
+        if (lane < 4 && st < steps)
+          sm.mask[st * 4 + lane] = lane == 0 ? bw[0] : (lane == 1 ? bw[1] : (lane == 2 ? bw[2] : bw[3]));
+        nwin += __popc(bw[0]) + __popc(bw[1]) + __popc(bw[2]) + __popc(bw[3]);
+      }
+#pragma unroll
+      for (int u = 0; u < kWarpRowUnroll; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int a = ncand + __popc(bc[u][e] & lt);
+          if (((bc[u][e] >> lane) & 1u) && a < kWarpRowCand) {
+            sm.cand_key[a] = order_bits(__float_as_uint(v[u][e]));
+            sm.cand_idx[a] = (uint16_t)((st0 + u) * 128 + 32 * e + lane);
+          }
+          ncand += __popc(bc[u][e]);
+        }
+    });
+    __syncwarp();
+  };
+  band_pass();
+
+  // ---- 2'. the sample misled (rare): narrow exactly.  [lo, hi] holds the
+  // k-th largest and `above` keys lie above hi; counting passes split the
+  // range into 256 bins (by the top bits of key - lo) until the k-th's bin
+  // fits the band list or is a single key value, then the band pass runs on
+  // that bin.
+  bool tie_class = false;
+  if (!(nwin < k && nwin + ncand >= k && ncand <= kWarpRowCand)) {
+    uint32_t lo, hi;
+    int above;
+    if (nwin >= k) { lo = hiK + 1u; hi = 0xFFFFFFFFu; above = 0; }
+    else if (nwin + ncand < k) { lo = 0x007FFFFFu; hi = loK - 1u; above = nwin + ncand; }   // from -inf
+    else { lo = loK; hi = hiK; above = nwin; }
+    for (;;) {
+      const uint32_t range = hi - lo;
+      const int nb = range ? 32 - __clz(range) : 0;
+      if (nb == 0) { tie_class = true; break; }
+      const int sh = nb > 8 ? nb - 8 : 0;
+      for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+      __syncwarp();
+      scan_row([&](int st0, const float (&v)[kWarpRowUnroll][4]) {
+#pragma unroll
+        for (int u = 0; u < kWarpRowUnroll; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t kk = order_bits(__float_as_uint(v[u][e]));
+            if ((st0 + u) * 128 + 32 * e + lane < V && kk >= lo && kk <= hi) atomicAdd(&hist[(kk - lo) >> sh], 1u);
+          }
+      });
+      __syncwarp();
+      // the bin holding rank k - above (counted from the top)
+      int krem = k - above, bin = 0, cnt = 0, acc = 0;
+      for (int b = 255; b >= 0; --b) {
+        const int c = (int)hist[b];
+        if (acc + c >= krem) { bin = b; cnt = c; break; }
+        acc += c;
+      }
+      above += acc;
+      const uint32_t nlo = lo + ((uint32_t)bin << sh);
+      const uint32_t nhi = (uint32_t)min((unsigned long long)hi, (unsigned long long)nlo + (1ull << sh) - 1ull);
+      lo = nlo;
+      hi = nhi;
+      __syncwarp();
+      if (cnt <= kWarpRowCand) break;
+    }
+    if (tie_class) {
+      // every key of [lo, hi] is equal: keys above it, then the first
+      // k - above keys equal to it (index order)
+      int ties = 0;
+      const int krem = k - above;
+      scan_row([&](int st0, const float (&v)[kWarpRowUnroll][4]) {
+#pragma unroll
+        for (int u = 0; u < kWarpRowUnroll; ++u)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int st = st0 + u;
+            const uint32_t kk = order_bits(__float_as_uint(v[u][e]));
+            const bool in = st * 128 + 32 * e + lane < V;
+            const bool eq = in && kk == lo;
+            const uint32_t be = __ballot_sync(0xffffffffu, eq);
+            const bool take = (in && kk > lo) || (eq && ties + __popc(be & lt) < krem);
+            const uint32_t word = __ballot_sync(0xffffffffu, take);
+            if (lane == e && st < steps) sm.mask[st * 4 + e] = word;
+            ties += __popc(be);
+          }
+      });
+      __syncwarp();
+    } else {
+      hiK = hi;
+      loK = lo;
+      band_pass();
+    }
+  }
+
+  // ---- 3. the k-th largest key T within the band and the ties kept: the
+  // band's keys above T and its first krem keys equal to T join the mask
+  if (!tie_class) {
     uint32_t cmin = 0xFFFFFFFFu, cmax = 0u;
     for (int i = lane; i < ncand; i += 32) {
       cmin = min(cmin, sm.cand_key[i]);
@@ -990,7 +1072,6 @@ __global__ void __launch_bounds__(kWarpRowWarps * 32) topk_warp(TopkParams p) {
     const uint32_t T = warp_radix_select(hist, cmin, cmax, &krem, [&](auto f) {
       for (int i = lane; i < ncand; i += 32) f(sm.cand_key[i]);
     });
-    // band keys above T, then the first krem keys equal to T (index order)
     int ties = 0;
     for (int c0 = 0; c0 < ncand; c0 += 32) {
       const int i = c0 + lane;
@@ -1004,34 +1085,8 @@ __global__ void __launch_bounds__(kWarpRowWarps * 32) topk_warp(TopkParams p) {
       }
       ties += __popc(be);
     }
-  } else {
-    // the band missed: exact select over the whole row, read again
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i = lane; i < V; i += 32) {
-      const uint32_t kk = order_bits(__ldg(srcu + i));
-      kmin = min(kmin, kk);
-      kmax = max(kmax, kk);
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    int krem = k;
-    const uint32_t T = warp_radix_select(hist, kmin, kmax, &krem, [&](auto f) {
-      for (int i = lane; i < V; i += 32) f(order_bits(__ldg(srcu + i)));
-    });
-    // mark: keys above T, then the first krem keys equal to T in index order
-    int ties = 0;
-    for (int w0 = 0; w0 < nwords; ++w0) {
-      const int i = 32 * w0 + lane;
-      const uint32_t kk = i < V ? order_bits(__ldg(srcu + i)) : 0u;
-      const bool gt = i < V && kk > T, eq = i < V && kk == T;
-      const uint32_t be = __ballot_sync(0xffffffffu, eq);
-      const bool take = gt || (eq && ties + __popc(be & lt) < krem);
-      const uint32_t word = __ballot_sync(0xffffffffu, take);
-      if (lane == 0) sm.mask[w0] = word;
-      ties += __popc(be);
-    }
+    __syncwarp();
   }
-  __syncwarp();
 
   // ---- 4. emit in ascending index order (exactly k bits are set): lane l
   // takes words [l*wpl, (l+1)*wpl)
@@ -1453,7 +1508,9 @@ int launch_topk_warp(const TopkParams &t, long long rows, int Vmax, cudaStream_t
   static std::atomic<bool> attr_dev[kMaxDevices];
   std::atomic<bool> &attr = attr_dev[device_slot()];
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // two CTAs per SM: the whole unified L1 / shared array as shared memory
+    cudaError_t e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(topk_warp, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "top-k warp smem attribute: %s", cudaGetErrorString(e));
     attr = true;
   }

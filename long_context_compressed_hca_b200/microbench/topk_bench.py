@@ -1,7 +1,10 @@
 """Time the index score + top-k call on a slice of a long prefill (each query
 row holds about start_pos/m visible entries) or on a decode batch.
 
-    python -m long_context_compressed_hca_b200.microbench.topk_bench [n_q] [start_pos] [B]
+    python -m long_context_compressed_hca_b200.microbench.topk_bench [n_q] [start_pos] [B] [kernel]
+
+kernel: the top-k kernel (hca_topk_kernel mode: 0 by shape, 1 a CTA per row,
+2 a warp per row, 3 segmented clusters, 4 a cluster per row).
 
 Inputs are seeded N(0,1); per-kernel device times come from CUDA-graph
 replays with the library's event profiler on."""
@@ -17,6 +20,7 @@ def main():
     n_q = int(sys.argv[1]) if len(sys.argv) > 1 else 2048
     start_pos = int(sys.argv[2]) if len(sys.argv) > 2 else 63488
     B = int(sys.argv[3]) if len(sys.argv) > 3 else 1
+    hb.topk_kernel(int(sys.argv[4]) if len(sys.argv) > 4 else 0)
     m, k, n_hI, c_I = 4, 512, 8, 64
     E = (start_pos + n_q) // m
     dev = "cuda"
