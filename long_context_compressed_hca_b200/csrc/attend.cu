@@ -637,18 +637,6 @@ attend_tc(AttendParams p, int n_units) {
               cw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + col_off));
               sc[i] = __ldg(reinterpret_cast<const float *>(rp + sc_off));
             }
-            // the registers hold one tile: pull the next two tiles' codes towards
-            // L2 while this one's loads are in flight
-            for (int ja = j + 1; ja < nt && ja <= j + 2; ++ja) {
-#pragma unroll 4
-              for (int i = 0; i < NR; ++i) {
-                const int kk = (j0 + ja) * KT + prow + i * RPP;
-                bool v;
-                const int row = slot_row(p, ks, b, qi, kk, v);
-                const uint8_t *rp = (kk < ks.nw4 ? wrec : crec) + (long long)row * p.rec;
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(rp + col_off));
-              }
-            }
             if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
