@@ -548,6 +548,14 @@ def roofline_tensor(flops_per_launch, ms_per_launch, peaks, traffic=None):
             "frac_of_sustained": round(ach / peaks["bf16_sus"], 4), "peak_sustained": peaks["bf16_sus"]}
 
 
+# DRAM bytes per query token of the CSA prefill attention kernel (64 heads x 512):
+# read + write counters of one ncu capture of the 16384-token layer (2.157 GB:
+# q read once, o written once, the compressed entries served from L2), which
+# scale with the token count; the traffic of longer launches is this times
+# their tokens.
+CSA_PREFILL_ATTN_DRAM_PER_TOKEN = 2157e6 / 16384
+
+
 def kern_ms(kern, prefix, K):
     tot = sum(v["ms"] for k, v in kern.items() if k.startswith(prefix))
     n = sum(v["launches"] for k, v in kern.items() if k.startswith(prefix))
@@ -688,7 +696,9 @@ def main():
                 "path_ms": round(r["path_ms"], 3),
                 "projections_ms": round(r["glue_ms"], 3),
                 "layer_ms": round(statistics.mean(r["ms"]), 3),
-                "roofline_attention": roofline_tensor(r["att_flops"], att_ms, peaks),
+                "roofline_attention": roofline_tensor(
+                    r["att_flops"], att_ms, peaks,
+                    traffic=round(CSA_PREFILL_ATTN_DRAM_PER_TOKEN * toks) if r["idx_flops"] else None),
                 "kernels_ms": {k: round(v["ms"] / kp, 3) for k, v in r["kern"].items()},
             }
             if r["idx_flops"]:
