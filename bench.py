@@ -482,46 +482,62 @@ def run_oproj(T, K, W, flush, stream):
 
 
 # --------------------------------------------------------------------------- oracle arm
-def oracle_decode_sample(bench: DecodeBench, n_seq: int):
-    """Time the oracle on `n_seq` sequences of one decode step (both layers)."""
-    import numpy as np
-    from oracle import hca_oracle as O
+class OracleStep:
+    """The C++ oracle's inputs for one decode step of a DecodeBench (every
+    sequence, both layers), copied to the host in the bytes the GPU stores
+    (bf16 bits, e4m3 codes and scales); time(n_seq) runs the oracle's decode of
+    the first n_seq sequences of both layers and returns the seconds."""
 
-    wl, pos = bench.wl, bench.wl.pos
-    data = []
-    for li, L in enumerate(wl.layers):
-        ch, ti = bench.caches[li], bench.inputs[li]
-        V = (pos + 1) // L.m
-        per = []
-        for b in range(n_seq):
-            d = dict(q=ti.t["q"][b].double().cpu().numpy(), kvc=ch.kv_comp[b, :V].double().cpu().numpy(),
-                     win=ch.win[b].double().cpu().numpy(), sink=bench.layers[li].t["sink"].double().cpu().numpy())
+    def __init__(self, bench: DecodeBench):
+        import numpy as np
+        from oracle import hca_oracle as O
+        from oracle import hca_oracle_c as OC
+        self.OC = OC
+        wl, pos = bench.wl, bench.wl.pos
+        self.layers = []
+        bits = lambda t: t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        for li, L in enumerate(wl.layers):
+            ch, ti = bench.caches[li], bench.inputs[li]
+            d = dict(L=L, q=ti.t["q"].double().cpu().numpy(), win=bits(ch.win), comp=bits(ch.kv_comp),
+                     order=np.array([p % L.w for p in O.window_positions(pos, L.w)], dtype=np.int32),
+                     sink=bench.layers[li].t["sink"].double().cpu().numpy())
             if L.kind == "csa":
-                if wl.idx_key_dtype == "fp8":
-                    d["KI"] = O.e4m3_to_f64(ch.key_I[b, :V].cpu().numpy()) * \
-                        ch.key_I_scale[b, :V].double().cpu().numpy()[:, None]
+                if bench.idx_key_dtype == "fp8":
+                    d["KI"], d["KI_scale"] = ch.key_I.cpu().numpy(), ch.key_I_scale.cpu().numpy()
                 else:
-                    d["KI"] = ch.key_I[b, :V].double().cpu().numpy()
-                d["qI"] = ti.t["qI"][b].double().cpu().numpy()
-                d["wI"] = ti.t["wI"][b].double().cpu().numpy()
-            per.append(d)
-        data.append(per)
-    t0 = time.perf_counter()
-    for li, L in enumerate(wl.layers):
-        for d in data[li]:
-            wrows = d["win"][[p % L.w for p in O.window_positions(pos, L.w)]]
-            kw = dict(qI_t=d["qI"], w_t=d["wI"], KI=d["KI"]) if L.kind == "csa" else {}
-            O.layer_decode(L, pos, d["q"], d["kvc"], wrows, d["sink"], **kw)
-    return time.perf_counter() - t0
+                    d["KI"], d["KI_scale"] = bits(ch.key_I), None
+                d["qI"] = ti.t["qI"].double().cpu().numpy()
+                d["wI"] = ti.t["wI"].double().cpu().numpy()
+            self.layers.append(d)
+        self.pos = pos
+
+    def time(self, n_seq, threads):
+        self.OC.num_threads(threads)
+        t0 = time.perf_counter()
+        for d in self.layers:
+            L = d["L"]
+            csa = L.kind == "csa"
+            self.OC.decode_batch(L.kind, d["q"][:n_seq], d["win"], d["order"], d["comp"], L.m, d["sink"], L.rd,
+                                 self.pos, k=L.k if csa else 0, qI=d["qI"][:n_seq] if csa else None,
+                                 w=d["wI"][:n_seq] if csa else None, KI=d.get("KI"), KI_scale=d.get("KI_scale"))
+        return time.perf_counter() - t0
 
 
-def cpu_cores():
-    try:
-        from threadpoolctl import threadpool_info
-        n = max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
-        return int(n)
-    except Exception:
-        return os.cpu_count() or 1
+def oracle_baseline(bench: DecodeBench, reps: int, warmup: int):
+    """The C++ oracle (double precision, -O3, OpenMP over the sequences) on the
+    step: every sequence on all host cores, and a bounded sample on one core
+    scaled to the step.  Returns (us per step on all cores, per reps, the
+    one-core figure, the one-core sample size, cores)."""
+    os_ = OracleStep(bench)
+    B = bench.wl.B
+    cores = os_.OC.num_threads(os.cpu_count() or 1)
+    for _ in range(warmup):
+        os_.time(B, cores)
+    all_us = [os_.time(B, cores) * 1e6 for _ in range(reps)]
+    n1 = min(B, 4)
+    one_us = os_.time(n1, 1) * B / n1 * 1e6
+    os_.OC.num_threads(cores)
+    return all_us, one_us, n1, cores
 
 
 # --------------------------------------------------------------------------- main
@@ -569,7 +585,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only-headline", action="store_true")
-    ap.add_argument("--oracle-seqs", type=int, default=2)
     args = ap.parse_args()
     assert args.warmup >= 3, "at least 3 warm-up steps"
 
@@ -593,10 +608,7 @@ def main():
                 torch.distributed.destroy_process_group()
             return
         b = DecodeBench(wl)
-        n = args.oracle_seqs
-        for _ in range(args.warmup):
-            oracle_decode_sample(b, n)
-        times = [oracle_decode_sample(b, n) * wl.B / n * 1e6 for _ in range(args.steps)]
+        times, one_us, n1, cores = oracle_baseline(b, args.steps, args.warmup)
         v = statistics.mean(times)
         line = {"metric": METRIC, "value": round(v, 1), "unit": "us/step", "impl": "reference",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": v / 1e3,
@@ -604,8 +616,11 @@ def main():
                 "data": "synthetic",
                 "config": {"workload": wl.name, "global_batch": wl.B, "seq_len": wl.pos,
                            "parallelism": "single process (CPU oracle)"},
-                "cpu_baseline": {"value": round(v, 1), "unit": "us/step", "cores": cpu_cores(), "kind": "oracle",
-                                 "sample": f"{n} of {wl.B} sequences per step (CSA+HCA layer), scaled x{wl.B / n:g}"},
+                "cpu_baseline": {"value": round(v, 1), "unit": "us/step", "cores": cores, "kind": "oracle",
+                                 "sample": f"all {wl.B} sequences of each step (CSA+HCA layer), C++ oracle, "
+                                           f"double precision, OpenMP over the sequences",
+                                 "single_core_us_per_step": round(one_us, 1),
+                                 "single_core_sample": f"{n1} of {wl.B} sequences, scaled x{wl.B / n1:g}"},
                 "e2e": {"value": round(v, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         if world > 1:
@@ -645,13 +660,15 @@ def main():
     if "sweep" in head:
         extras["decode_steps"] = dict(steady_us=round(step_ms * 1e3, 2), steady_pos=wl.pos, **head["sweep"])
     if rank == 0 and world == 1:
-        # CPU oracle baseline on a bounded sample of the same workload
-        n = args.oracle_seqs
-        oracle_decode_sample(head["bench"], 1)
-        osec = statistics.mean(oracle_decode_sample(head["bench"], n) for _ in range(2))
-        extras["cpu_baseline"] = {"value": round(osec * wl.B / n * 1e6, 1), "unit": "us/step",
-                                  "cores": cpu_cores(), "kind": "oracle",
-                                  "sample": f"{n} of {wl.B} sequences of one step (CSA+HCA), scaled x{wl.B / n:g}"}
+        # the C++ CPU oracle on the same step: every sequence on all host cores,
+        # and a 4-sequence sample on one core
+        all_us, one_us, n1, cores = oracle_baseline(head["bench"], 2, 1)
+        extras["cpu_baseline"] = {"value": round(statistics.mean(all_us), 1), "unit": "us/step",
+                                  "cores": cores, "kind": "oracle",
+                                  "sample": f"all {wl.B} sequences of one step (CSA+HCA), C++ oracle, double "
+                                            f"precision, OpenMP over the sequences",
+                                  "single_core_us_per_step": round(one_us, 1),
+                                  "single_core_sample": f"{n1} of {wl.B} sequences, scaled x{wl.B / n1:g}"}
     del head["bench"]
     torch.cuda.empty_cache()
 
