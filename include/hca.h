@@ -282,6 +282,24 @@ typedef struct {
   const float *compI;  /* [B, 4c_I] (CSA) fp32 */
 } hca_token_in;
 
+/* hybrid_decode_inputs -- the decode token's inputs from hidden states:
+ * h [B, d] (a.dtype) holds one token per sequence, all at position pos; the
+ * call writes the buffers that x points to (allocated by the caller with the
+ * sizes above; the const qualifiers are for hybrid_decode_step, which reads
+ * them): comp = h W_comp^T (fp32, [J] Eq.(9)-(10) / (20)-(21)); q = per-head
+ * RMSNorm of RMSNorm(h W_DQ^T) W_UQ^T, RoPE'd at pos (Eq.(13), (18)); kv =
+ * RMSNorm(h W_KV^T) RoPE'd at pos (the window row, when w > 0); for CSA also
+ * compI = h W_compI^T, qI = RoPE(RMSNorm(h W_DQ^T) W_IUQ^T) at pos (Eq.(14)),
+ * wI = h W_w^T c_I^-1/2 n_hI^-1/2 (Eq.(15)).  These are the prefill's
+ * projections restricted to one token, so a layer's output, projected to
+ * hidden states (hca_output_projection and the caller's residual path), can
+ * feed the next layer's decode step.  Workspace: fp32 / bf16 intermediates
+ * (hybrid_decode_inputs_workspace_size).  Errors: HCA_ERR_INVALID for a null h
+ * or x, a missing output buffer, pos < 0 or a short workspace. */
+size_t hybrid_decode_inputs_workspace_size(const hca_layer *L);
+int hybrid_decode_inputs(const hca_layer *L, const void *h, int pos, const hca_token_in *x, void *ws,
+                         size_t ws_bytes, hca_stream_t stream);
+
 /* hybrid_decode_step -- token at position pos (> 0) for every sequence:
  * stores its window row, advances the compressor states (emitting an entry
  * when (pos+1) % m == 0), scores and selects (CSA), and attends; writes

@@ -107,6 +107,8 @@ def _declare(L):
         "hybrid_decode_step": (I, [C.POINTER(Layer), C.POINTER(TokenIn), C.POINTER(Cache), I, VP, VP,
                                    SZ, VP]),
         "hca_kv_mixed_row_bytes": (SZ, [I, I]),
+        "hybrid_decode_inputs_workspace_size": (SZ, [C.POINTER(Layer)]),
+        "hybrid_decode_inputs": (I, [C.POINTER(Layer), VP, I, C.POINTER(TokenIn), VP, SZ, VP]),
         "hca_static_scratch_bytes": (SZ, []),
         "hca_compress": (I, [C.POINTER(CompressDesc), I, I, VP, VP, VP, VP, LL, LL, VP, VP, VP, VP,
                              VP, LL, VP, VP, VP]),
@@ -351,6 +353,17 @@ def hybrid_layer_forward(L: Layer, H, n, cache: Cache | None, o, ws, stream=None
     nbytes = ws.numel() * ws.element_size()
     return check(lib().hybrid_layer_forward(C.byref(L), ptr(H), n, C.byref(cache) if cache else None,
                                             ptr(o), ptr(ws), nbytes, stream_handle(stream)))
+
+
+def decode_inputs_workspace_size(L: Layer) -> int:
+    return lib().hybrid_decode_inputs_workspace_size(C.byref(L))
+
+
+def hybrid_decode_inputs(L: Layer, h, pos, x: TokenIn, ws, stream=None):
+    """Write the decode token inputs x (buffers the caller allocated) from hidden states h [B, d]."""
+    nbytes = ws.numel() * ws.element_size()
+    return check(lib().hybrid_decode_inputs(C.byref(L), ptr(h), pos, C.byref(x), ptr(ws), nbytes,
+                                            stream_handle(stream)))
 
 
 def decode_workspace_size(L: Layer, pos: int) -> int:

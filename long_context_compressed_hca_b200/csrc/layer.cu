@@ -529,6 +529,102 @@ int hybrid_workspace_map(const hca_layer *L, int n, int decode, hca_ws_map *map)
 }
 
 // ----------------------------------------------------------------- decode
+// ---------------------------------------------------------------- decode inputs
+// The projections of one decode token per sequence from hidden states
+// h [B, d] at position pos, into the buffers of x (the same steps as the
+// prefill's, with every row at position pos): [J] Eq.(9)-(10) / (20)-(21)
+// compressor C/Z, Eq.(13) c^Q = RMSNorm(h W_DQ), Eq.(18) q = per-head RMSNorm
+// of c^Q W_UQ then RoPE, the window row RMSNorm(h W_KV) then RoPE, and for CSA
+// Eq.(14)-(15) q^I = RoPE(c^Q W_IUQ), w^I = h W_w c_I^-1/2 n_hI^-1/2, and the
+// indexer compressor's C/Z.
+struct DecPlan {
+  void *cQ32, *cQ, *q32, *qI32, *kv32;
+  size_t total;
+};
+static DecPlan plan_decode_inputs(const hca_layer *L, void *ws) {
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA;
+  const long long T = a.B;
+  Carver cv(ws);
+  DecPlan P{};
+  P.cQ32 = cv.take(T * L->d_c * 4);
+  P.cQ = cv.take(T * L->d_c * esize(a.dtype));
+  P.q32 = cv.take(T * a.n_h * a.c * 4);
+  P.qI32 = csa ? cv.take(T * a.n_hI * a.c_I * 4) : nullptr;
+  P.kv32 = cv.take(T * a.c * 4);
+  P.total = cv.off;
+  return P;
+}
+
+size_t hybrid_decode_inputs_workspace_size(const hca_layer *L) {
+  if (check_layer(L)) return 0;
+  return plan_decode_inputs(L, nullptr).total;
+}
+
+int hybrid_decode_inputs(const hca_layer *L, const void *h, int pos, const hca_token_in *x, void *ws,
+                         size_t ws_bytes, hca_stream_t stream) {
+  int rc = check_layer(L);
+  if (rc) return rc;
+  const hca_attn_desc &a = L->a;
+  const bool csa = L->kind == HCA_LAYER_CSA, comp = L->kind != HCA_LAYER_SWA;
+  if (!h || !x || pos < 0) return fail(HCA_ERR_INVALID, "h and x must be non-null and pos >= 0");
+  if (!x->q || (a.w > 0 && !x->kv) || (comp && !x->comp) || (csa && (!x->qI || !x->wI || !x->compI)))
+    return fail(HCA_ERR_INVALID, "missing output buffer in x");
+  const DecPlan need = plan_decode_inputs(L, nullptr);
+  if (ws_bytes < need.total || !ws) return fail(HCA_ERR_INVALID, "workspace too small");
+  const DecPlan P = plan_decode_inputs(L, ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const hca_dtype dt = a.dtype;
+  const float theta = rope_theta(a), eps = eps_of(a);
+  const int T = a.B;
+  auto row_op = [&](const void *in, int cols, void *out, hca_dtype odt, int rows, int norm, int rd,
+                    int rows_per_pos) {
+    RowOpParams r{};
+    r.in = static_cast<const float *>(in); r.in_stride = cols; r.out = out; r.out_stride = cols; r.out_dtype = odt;
+    r.rows = rows; r.cols = cols; r.norm = norm; r.eps = eps; r.rd = rd; r.theta = theta;
+    r.rows_per_pos = rows_per_pos; r.pos_mod = 1; r.pos_base = pos; r.scale = 1.f;
+    return launch_row_op(r, s);
+  };
+  void *q = const_cast<void *>(x->q);
+  // compressor C/Z (fp32, [B, ncz c]: C_a | C_b | Z_a | Z_b, or C | Z)
+  if (comp) {
+    const int ncz = csa ? 4 : 2;
+    rc = launch_gemm(dt, h, L->d, L->W_comp, L->d, const_cast<float *>(x->comp), (long long)ncz * a.c, HCA_F32, T,
+                     ncz * a.c, L->d, 1.f, s);
+    if (rc) return rc;
+  }
+  if (csa) {
+    rc = launch_gemm(dt, h, L->d, L->W_compI, L->d, const_cast<float *>(x->compI), 4LL * a.c_I, HCA_F32, T,
+                     4 * a.c_I, L->d, 1.f, s);
+    if (rc) return rc;
+  }
+  // queries
+  if ((rc = launch_gemm(dt, h, L->d, L->W_DQ, L->d, P.cQ32, L->d_c, HCA_F32, T, L->d_c, L->d, 1.f, s)) ||
+      (rc = row_op(P.cQ32, L->d_c, P.cQ, dt, T, 1, 0, 1)))
+    return rc;
+  const int HC = a.n_h * a.c;
+  if ((rc = launch_gemm(dt, P.cQ, L->d_c, L->W_UQ, L->d_c, P.q32, HC, HCA_F32, T, HC, L->d_c, 1.f, s)) ||
+      (rc = row_op(P.q32, a.c, q, dt, T * a.n_h, 1, a.rd, a.n_h)))
+    return rc;
+  if (csa) {
+    const int HI = a.n_hI * a.c_I;
+    if ((rc = launch_gemm(dt, P.cQ, L->d_c, L->W_IUQ, L->d_c, P.qI32, HI, HCA_F32, T, HI, L->d_c, 1.f, s)) ||
+        (rc = row_op(P.qI32, a.c_I, const_cast<void *>(x->qI), dt, T * a.n_hI, 0, a.rd_I, a.n_hI)))
+      return rc;
+    const float wscale = 1.0f / sqrtf((float)a.c_I) / sqrtf((float)a.n_hI);
+    rc = launch_gemm(dt, h, L->d, L->W_w, L->d, const_cast<float *>(x->wI), a.n_hI, HCA_F32, T, a.n_hI, L->d, wscale,
+                     s);
+    if (rc) return rc;
+  }
+  // window row
+  if (a.w > 0) {
+    if ((rc = launch_gemm(dt, h, L->d, L->W_KV, L->d, P.kv32, a.c, HCA_F32, T, a.c, L->d, 1.f, s)) ||
+        (rc = row_op(P.kv32, a.c, const_cast<void *>(x->kv), dt, T, 1, a.rd, 1)))
+      return rc;
+  }
+  return HCA_OK;
+}
+
 size_t hybrid_decode_step_workspace_size(const hca_layer *L, int pos) {
   if (check_layer(L) || pos < 0) return 0;
   size_t b = 0;

@@ -90,3 +90,13 @@ class TokenInputs:
         self.t = dict(q=q, kv=kv, comp=comp, qI=qI, wI=wI, compI=compI)
         p = hb.ptr
         self.struct = hb.TokenIn(p(q), p(qI), p(wI), p(kv), p(comp), p(compI))
+
+    @classmethod
+    def empty(cls, L, B: int, dtype: torch.dtype, device="cuda"):
+        """Buffers for one decode token per sequence of layer shape L (for
+        hybrid_decode_inputs to fill)."""
+        csa = L.kind == "csa"
+        e = lambda *s, dt=dtype: torch.empty(*s, dtype=dt, device=device)
+        return cls(q=e(B, L.n_h, L.c), kv=e(B, L.c), comp=e(B, (4 if csa else 2) * L.c, dt=torch.float32),
+                   qI=e(B, L.n_hI, L.c_I) if csa else None, wI=e(B, L.n_hI, dt=torch.float32) if csa else None,
+                   compI=e(B, 4 * L.c_I, dt=torch.float32) if csa else None)
