@@ -481,6 +481,61 @@ def run_oproj(T, K, W, flush, stream):
     return statistics.mean(ms), flops
 
 
+def run_chained(wl, K, W, flush, stream):
+    """The two layers of the 128K decode step chained through hidden states
+    (d_model 4096, query compression 1024): CSA decode inputs from h0 -> CSA
+    step -> grouped output projection (8 groups of 1024) -> HCA decode inputs ->
+    HCA step, on one stream (each stage needs the previous one's output).
+    Returns (ms per chained step, per-kernel profile)."""
+    d, d_c, g, d_g = 4096, 1024, 8, 1024
+    b = DecodeBench(wl)                      # caches and step inputs at the workload's position
+    B, pos = wl.B, wl.pos
+    Ls = wl.layers
+    lhs, xs, wss = [], [], []
+    for li, L in enumerate(Ls):
+        Wt = synth.layer_weights_on("cuda", L, d, d_c, wl.seed, torch.bfloat16, layer_id=li)
+        lh = LayerHandle(L, Wt, d, d_c, torch.bfloat16, B)   # sequential: every SM for each attention
+        lhs.append(lh)
+        xs.append(TokenInputs.empty(L, B, torch.bfloat16))
+        wss.append(torch.empty(max(hb.decode_inputs_workspace_size(lh.struct), 256), dtype=torch.uint8,
+                               device="cuda"))
+    gw = Ls[0].n_h * Ls[0].c // g
+    wo_a = dev_normal((g, d_g, gw), wl.seed, 21, torch.bfloat16, std=gw ** -0.5)
+    wo_b = dev_normal((d, g * d_g), wl.seed, 22, torch.bfloat16, std=(g * d_g) ** -0.5)
+    od = hb.oproj_desc(B, Ls[0].n_h, Ls[0].c, g, d_g, d, hb.HCA_BF16, hb.HCA_BF16)
+    wso = torch.empty(max(hb.output_projection_workspace_size(od), 256), dtype=torch.uint8, device="cuda")
+    h0 = dev_normal((B, d), wl.seed, 23, torch.bfloat16)
+    h1 = torch.empty(B, d, dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        hb.hybrid_decode_inputs(lhs[0].struct, h0, pos, xs[0].struct, wss[0])
+        hb.hybrid_decode_step(lhs[0].struct, xs[0].struct, b.caches[0].struct, pos, b.outs[0], b.ws[0])
+        hb.output_projection(od, b.outs[0], wo_a, wo_b, h1, wso)
+        hb.hybrid_decode_inputs(lhs[1].struct, h1, pos, xs[1].struct, wss[1])
+        hb.hybrid_decode_step(lhs[1].struct, xs[1].struct, b.caches[1].struct, pos, b.outs[1], b.ws[1])
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    graph = capture_graph(step, stream)
+    for _ in range(W):
+        graph.replay()
+    torch.cuda.synchronize()
+    ms, _, _ = time_steps(graph.replay, K, flush, stream)
+
+    def prof_pass():
+        hb.profile_enable(True)
+        pg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pg, stream=stream):
+            step()
+        torch.cuda.synchronize()
+        return time_steps(pg.replay, K, flush, stream, profile=True, replayed=True)[2]
+    kern = profiled(prof_pass)
+    del graph, b, lhs, xs, wss
+    torch.cuda.empty_cache()
+    return statistics.mean(ms), kern
+
+
 # --------------------------------------------------------------------------- oracle arm
 class OracleStep:
     """The C++ oracle's inputs for one decode step of a DecodeBench (every
@@ -723,6 +778,13 @@ def main():
                 extras[key]["roofline_index"] = roofline_tensor(r["idx_flops"], sc_ms, peaks)
 
     if world == 1 and not args.only_headline:
+        cms, ckern = run_chained(wl, max(3, min(args.steps, 20)), 3, flush, stream)
+        extras["decode_128k_chained"] = {
+            "workload": wl.name + "_chained_d4096",
+            "us_per_step": round(cms * 1e3, 2),
+            "chain": "CSA decode inputs from hidden states -> CSA step -> grouped output projection "
+                     "(8 x 1024 -> 4096) -> HCA decode inputs -> HCA step, one stream",
+            "kernels": {k: round(v["ms"] / max(3, min(args.steps, 20)) * 1e3, 2) for k, v in ckern.items()}}
         oms, ofl = run_oproj(65536, max(3, min(args.steps, 5)), 3, flush, stream)
         extras["output_projection_64k"] = {
             "workload": "grouped output projection, 65536 tokens, 64x512 -> 8x1024 -> 4096, bf16",

@@ -56,6 +56,57 @@ __global__ void __launch_bounds__(256) gemm_simt(const Tab *A, long long lda, co
   }
 }
 
+// ------------------------------------------------------- few output columns
+// C[M, N] for N <= 32 (the head-weight projection W_w, N = n_hI): one CTA per
+// row of A, its threads striding over K (coalesced); each thread keeps N
+// partial sums, reduced across the warps at the end (a fixed order).  A's row
+// is read once, B (N x K) stays in L1/L2 for every row.
+constexpr int kNarrowThreads = 256;
+template <typename Tab, typename Tc, int NT>
+__global__ void __launch_bounds__(kNarrowThreads) gemm_narrow(const Tab *A, long long lda, const Tab *B,
+                                                              long long ldb, Tc *C, long long ldc, int M, int N,
+                                                              int K, float alpha) {
+  __shared__ float part[kNarrowThreads / 32][NT];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long m = blockIdx.x;
+  const Tab *a = A + m * lda;
+  float acc[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j] = 0.f;
+#pragma unroll 4
+  for (int k = threadIdx.x; k < K; k += kNarrowThreads) {
+    const float av = Elt<Tab>::load(a + k);
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+      if (j < N) acc[j] += av * Elt<Tab>::load(B + (long long)j * ldb + k);
+  }
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const float v = warp_sum(acc[j]);
+    if (lane == 0) part[warp][j] = v;
+  }
+  __syncthreads();
+  if (threadIdx.x < N) {
+    float v = 0.f;
+    for (int w = 0; w < kNarrowThreads / 32; ++w) v += part[w][threadIdx.x];
+    Elt<Tc>::store(C + m * ldc + threadIdx.x, v * alpha);
+  }
+}
+
+template <typename Tab, typename Tc>
+int launch_narrow(const Tab *A, long long lda, const Tab *B, long long ldb, Tc *C, long long ldc, int M, int N, int K,
+                  float alpha, cudaStream_t s) {
+  const dim3 grid((unsigned)M);
+  LaunchScope ls_("gemm_narrow", s);
+  if (N <= 8)
+    gemm_narrow<Tab, Tc, 8><<<grid, kNarrowThreads, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, alpha);
+  else if (N <= 16)
+    gemm_narrow<Tab, Tc, 16><<<grid, kNarrowThreads, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, alpha);
+  else
+    gemm_narrow<Tab, Tc, 32><<<grid, kNarrowThreads, 0, s>>>(A, lda, B, ldb, C, ldc, M, N, K, alpha);
+  return ls_.done();
+}
+
 // ------------------------------------------------------------------ row op
 // One warp per row: optional RMS normalisation, gamma, scale, RoPE of the
 // last rd columns (interleaved pairs) and conversion.  cols % 4 == 0 rows
@@ -140,6 +191,17 @@ int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long
   if (ab == HCA_BF16) {
     const int rc = launch_gemm_tc(A, lda, Bm, ldb, C, ldc, cdt, M, N, K, alpha, s);
     if (rc != HCA_ERR_UNSUPPORTED) return rc;
+  }
+  if (N <= 32) {
+    if (ab == HCA_F32)
+      return cdt == HCA_F32 ? launch_narrow((const float *)A, lda, (const float *)Bm, ldb, (float *)C, ldc, M, N, K,
+                                            alpha, s)
+                            : launch_narrow((const float *)A, lda, (const float *)Bm, ldb, (__nv_bfloat16 *)C, ldc,
+                                            M, N, K, alpha, s);
+    return cdt == HCA_F32 ? launch_narrow((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb, (float *)C,
+                                          ldc, M, N, K, alpha, s)
+                          : launch_narrow((const __nv_bfloat16 *)A, lda, (const __nv_bfloat16 *)Bm, ldb,
+                                          (__nv_bfloat16 *)C, ldc, M, N, K, alpha, s);
   }
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
   LaunchScope ls_("gemm_simt", s);

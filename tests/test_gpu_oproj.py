@@ -14,7 +14,9 @@ CASES = [
     # T, n_h, c, g, d_g, d, dtype
     (160, 64, 512, 8, 1024, 4096, BF16),   # V4-Flash widths; a ragged 128-row tile (tensor-core GEMMs)
     (300, 16, 128, 4, 256, 512, BF16),
-    (50, 16, 128, 4, 256, 512, BF16),      # fewer rows than one tile (CUDA-core GEMM)
+    (50, 16, 128, 4, 256, 512, BF16),      # few rows: the swapped skinny tensor-core tile (64 tokens)
+    (32, 64, 512, 8, 1024, 4096, BF16),    # a decode batch of 32 tokens (skinny tile of 32)
+    (5, 16, 128, 4, 256, 512, BF16),       # a ragged skinny tile
     (37, 8, 64, 2, 32, 48, F32),
 ]
 
