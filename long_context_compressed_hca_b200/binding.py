@@ -214,7 +214,7 @@ def profile_collect() -> dict:
 
 TRACE_SLOTS = ("prod_q_free", "prod_stage_free", "mma_q_ready", "mma_tile_ready", "mma_s_free",
                "mma_p_ready", "mma_o_free", "smax_s_ready", "smax_pbuf_free", "smax_rescale_wait",
-               "smax_epi_wait", "-", "epilogue", "total", "rescales", "units", "tiles", "-",
+               "smax_epi_wait", "smax_unit_setup", "epilogue", "total", "rescales", "units", "tiles", "smax_pair_xchg",
                "merge_wait_ready", "merge_wait_full", "merge_push", "merge_weights", "merge_loop",
                "t_setup", "t_first_s", "t_tiles", "t_epilogue", "t_exit", "t_entry_inv", "t_exit_max", "t_ctas")
 

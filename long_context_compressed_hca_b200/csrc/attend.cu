@@ -42,7 +42,7 @@ struct KeySet {
 __device__ __forceinline__ KeySet key_set(const AttendParams &p, int qi) {
   KeySet k;
   const int t = p.start_pos + qi;
-  k.V = (t + 1) / p.m;
+  k.V = fdiv(t + 1, p.fd_m);
   k.nw = min(p.w, t + 1);
   k.t0 = t - k.nw + 1;
   k.nc = p.csa ? min(p.k, k.V) : k.V;
@@ -59,6 +59,47 @@ __device__ __forceinline__ KeySet key_set_tc(const AttendParams &p, int qi) {
   k.nw4 = (k.nw + 3) & ~3;
   k.nk = k.nw4 + k.nc;
   return k;
+}
+
+// Work unit u: sequence b, query group qg (queries qi0 .. qi0 + G - 1), split sp.
+struct Unit {
+  int bq, b, qg, qi0, sp;
+};
+__device__ __forceinline__ Unit unit_of(const AttendParams &p, int u) {
+  Unit x;
+  x.bq = fdiv(u, p.fd_nsplit);
+  x.sp = u - x.bq * p.nsplit;
+  x.b = fdiv(x.bq, p.fd_nqg);
+  x.qg = x.bq - x.b * p.n_qg;
+  x.qi0 = x.qg * p.G;
+  return x;
+}
+
+// Key slots of query group qg: the union of its queries' windows -- one run
+// of tokens, from the first query's first window token to the last query --
+// and the last query's visible entries (the most any query of the group
+// sees).  Each query masks the slots outside its own key set.
+__device__ __forceinline__ KeySet group_key_set(const AttendParams &p, int qg) {
+  if (p.G == 1) return key_set_tc(p, qg);
+  const int qi0 = qg * p.G;
+  const int qi1 = min(p.n_q, qi0 + p.G) - 1;
+  const KeySet a = key_set(p, qi0);
+  KeySet k = key_set(p, qi1);
+  k.t0 = a.t0;
+  k.nw = p.w > 0 ? (p.start_pos + qi1) - a.t0 + 1 : 0;
+  k.nw4 = (k.nw + 3) & ~3;
+  k.nk = k.nw4 + k.nc;
+  return k;
+}
+
+// Whether slot kk (< nk) of a group's key set is a key of query token tq:
+// a window token in (tq - w, tq], or one of its (tq + 1) / m visible entries.
+__device__ __forceinline__ bool slot_of_token(const AttendParams &p, const KeySet &ks, int kk, int tq) {
+  if (kk < ks.nw4) {
+    const int tok = ks.t0 + kk;
+    return kk < ks.nw && tok <= tq && tok > tq - p.w;
+  }
+  return kk - ks.nw4 < fdiv(tq + 1, p.fd_m);
 }
 
 // Source row of slot kk (window tensor if kk < nw4, else compressed tensor)
@@ -289,27 +330,43 @@ struct Bars {
   uint64_t kv_full[8], kv_empty[8], s_full[3], s_empty[3], p_full[3], pv_done[3];
   uint64_t mg_ready, mg_full;    // cluster merge: peers' buffers free / peers' partials delivered
   uint64_t mg_stage;             // cluster merge: this CTA's blocks staged
+  uint64_t pair[4];              // M = 128: the two softmax warps of a TMEM lane quarter
 };
 
-template <int C>
+// Shared and tensor memory of one CTA.  M = 64: one query's (or a group's)
+// heads on 64 rows, S and Q in TMEM lane-half 1 beside O in lane-half 0.
+// M = 128 (c = 128, query groups): row i in TMEM lane i; two O accumulators
+// (one per half of each key tile), S buffers, Q; Q of the next unit is staged
+// in shared memory.
+template <int C, int M = 64>
 struct Layout {
+  static_assert(M == 64 || (M == 128 && C == 128), "M = 128 rows need c = 128");
   static constexpr int NKB = C / 64;
   // key-tile stages: Q lives in tensor memory, so the stages take what the P
-  // buffers leave (192 KB for C = 512 and 256)
-  static constexpr int NS = (C == 512) ? 3 : (C == 256 ? 6 : 8);
+  // buffers leave (192 KB for C = 512 and 256 at M = 64)
+  static constexpr int NS = M == 128 ? 8 : (C == 512) ? 3 : (C == 256 ? 6 : 8);
+  static constexpr uint32_t kPBytes = M * 128;   // P tile: M rows x 64 keys (bf16)
+  static constexpr int SP = M == 128 ? 3 : kSP;    // S / P buffers
   static constexpr uint32_t kv_off = 0;
   static constexpr uint32_t p_off = kv_off + NS * NKB * kTileBytes;
-  static constexpr uint32_t bar_off = p_off + kSP * kTileBytes;
+  static constexpr uint32_t q_off = p_off + SP * kPBytes;             // M = 128: staged Q [128][C] bf16
+  static constexpr uint32_t bar_off = q_off + (M == 128 ? 128u * C * 2 : 0u);
   static constexpr uint32_t misc_off = bar_off + 512;
-  static constexpr uint32_t bytes = misc_off + 2048 + 1024;  // + alignment slack
-  // tensor memory: O in lane-half 0, columns [0, C); in lane-half 1 S buffers
-  // 0 and 1 at columns [0, 128), Q (bf16, two per column) at [q_col, q_col +
-  // C/2), the lanes of S as the A operand of S = Q K^T needs, and S buffer 2
-  // after Q
+  static constexpr uint32_t bytes = misc_off + 8192 + 1024;  // + alignment slack
+  // tensor memory.  M = 64: O in lane-half 0, columns [0, C); in lane-half 1
+  // S buffers 0 and 1 at columns [0, 128), Q (bf16, two per column) at
+  // [q_col, q_col + C/2), the lanes of S as the A operand of S = Q K^T needs,
+  // and S buffer 2 after Q.  M = 128: O accumulators at [0, C) and [C, 2C),
+  // three S buffers from column 2C, Q at [2C + 192, 2C + 192 + C/2).
   static constexpr uint32_t tmem_cols = 512;
-  static constexpr uint32_t q_col = 2 * KT;
-  static_assert(q_col + C / 2 + KT <= tmem_cols, "S buffers and Q exceed tensor memory");
-  static constexpr __host__ __device__ uint32_t s_col(int b) { return b < 2 ? b * KT : q_col + C / 2; }
+  static constexpr uint32_t o_cols = M == 128 ? 2 * C : C;
+  static constexpr uint32_t q_col = M == 64 ? 2 * KT : o_cols + SP * KT;
+  static constexpr uint32_t s_lane = M == 64 ? 16 : 0;   // lane offset of S and Q in each quarter
+  static_assert(q_col + C / 2 + (M == 64 ? KT : 0) <= tmem_cols, "S buffers and Q exceed tensor memory");
+  static_assert(bytes <= 227 * 1024, "shared memory");
+  static constexpr __host__ __device__ uint32_t s_col(int b) {
+    return M == 128 ? o_cols + b * KT : (b < 2 ? b * KT : q_col + C / 2);
+  }
 };
 
 // Trace counters (cycles, summed over CTAs) of the tensor-core kernel's waits.
@@ -502,19 +559,31 @@ __device__ __forceinline__ bool cluster_merge(const AttendParams &p, uint8_t *sm
   return ok;
 }
 
-template <int C, bool TRACE, bool MIX>
+template <int C, int M, bool TRACE, bool MIX>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_tc(AttendParams p, int n_units) {
-  using L = Layout<C>;
+  using L = Layout<C, M>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   Bars *bars = reinterpret_cast<Bars *>(smem + L::bar_off);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
   double *freq = reinterpret_cast<double *>(smem + L::misc_off + 8);      // [32]
-  float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // [4 warps][64]: cos, sin
+  float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // [8 warps][2][64]: cos, sin
+  float *xch = reinterpret_cast<float *>(smem + L::misc_off + 4608);       // [3][8 warps][32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // warp roles: softmax warps first, then the MMA warp, then the loaders.
+  // M = 128: two softmax warps per TMEM lane quarter (each takes 32 of a
+  // tile's 64 keys and half of the O columns) and 4 loaders (c <= 256)
+  constexpr int SMW = M == 128 ? 8 : kSoftmaxWarps;
+  constexpr int MMAW = SMW;
+  constexpr int PW0 = SMW + 1;
+  constexpr int PT = (M == 128 ? 4 : kProdWarps) * 32;
+  static_assert((SMW + 1) * 32 + PT == kThreads, "warp roles");
+  // S / P buffers and how many S tiles the MMA issue runs ahead of P.V
+  constexpr int SP = L::SP;
+  constexpr int LA = M == 128 ? 2 : kLookahead;
   const unsigned long long st_entry = global_ns();
   auto bar = [&](uint64_t &b) { return smem_u32(&b); };
   unsigned long long tr[TR_COUNT];
@@ -530,22 +599,32 @@ attend_tc(AttendParams p, int n_units) {
     tr[slot] += clock64() - t0;
     return ok;
   };
+  // loaders wait for free stages sleeping between polls
+  auto twait_sleep = [&](uint32_t b, uint32_t par, int slot) -> bool {
+    if (!TRACE) return mbar_wait_sleep(b, par, p.status);
+    const long long t0 = clock64();
+    const bool ok = mbar_wait_sleep(b, par, p.status);
+    tr[slot] += clock64() - t0;
+    return ok;
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(bars->q_full), kSoftmaxWarps);
+    mbar_init(bar(bars->q_full), SMW);
     mbar_init(bar(bars->q_empty), 1);
-    mbar_init(bar(bars->o_empty), kSoftmaxWarps);
+    mbar_init(bar(bars->o_empty), SMW);
     mbar_init(bar(bars->mma_done), 1);
     for (int i = 0; i < L::NS; ++i) {
-      mbar_init(bar(bars->kv_full[i]), kProdThreads);
+      mbar_init(bar(bars->kv_full[i]), PT);
       mbar_init(bar(bars->kv_empty[i]), 1);
     }
-    for (int i = 0; i < kSP; ++i) {
+    for (int i = 0; i < SP; ++i) {
       mbar_init(bar(bars->s_full[i]), 1);
-      mbar_init(bar(bars->s_empty[i]), kSoftmaxWarps);
-      mbar_init(bar(bars->p_full[i]), kSoftmaxWarps);
+      mbar_init(bar(bars->s_empty[i]), SMW);
+      mbar_init(bar(bars->p_full[i]), SMW);
       mbar_init(bar(bars->pv_done[i]), 1);
     }
+    if (M == 128)
+      for (int i = 0; i < 4; ++i) mbar_init(bar(bars->pair[i]), 2);
     if (p.cluster) {
       mbar_init(bar(bars->mg_ready), p.nsplit);
       mbar_init(bar(bars->mg_full), 1);
@@ -553,7 +632,7 @@ attend_tc(AttendParams p, int n_units) {
     }
     mbar_fence_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == MMAW) {
     tmem_alloc(smem_u32(tmem_slot), L::tmem_cols);
     tmem_relinquish();
   }
@@ -571,7 +650,7 @@ attend_tc(AttendParams p, int n_units) {
   const unsigned long long st_ready = global_ns();
   if (TRACE && threadIdx.x == 0) ts[1] = global_ns();
 
-  if (warp >= kProdWarp0) {
+  if (warp >= PW0) {
     // ------------------------------------------------------------ loads
     // Q: 2-D tiled TMA (thread 0).  Key rows: cp.async by 8 warps, 16-byte
     // chunks placed at their 128B-swizzled positions; every thread resolves
@@ -581,19 +660,19 @@ attend_tc(AttendParams p, int n_units) {
     [&]() {
     constexpr int NKB = C / 64;
     constexpr int CPR = C / 8;                  // 16-byte chunks per row
-    constexpr int RPP = kProdThreads / CPR;     // rows per pass
+    constexpr int RPP = PT / CPR;               // rows per pass
     constexpr int NR = KT / RPP;                // rows per thread per tile
-    const int pt = threadIdx.x - kProdWarp0 * 32;
+    const int pt = threadIdx.x - PW0 * 32;
     const int chunk = pt % CPR, prow = pt / CPR;
     const uint32_t kb_off = (chunk / 8) * kTileBytes;
     const int cc = chunk % 8;
     uint32_t g = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const int bq = u / p.nsplit, sp = u % p.nsplit;
-      const int b = bq / p.n_q, qi = bq % p.n_q;
-      const KeySet ks = key_set_tc(p, qi);
+      const Unit x = unit_of(p, u);
+      const int b = x.b, qi = x.qi0;
+      const KeySet ks = group_key_set(p, x.qg);
       int j0, nt;
-      split_range(ks, p.nsplit, sp, j0, nt);
+      split_range(ks, p.nsplit, x.sp, j0, nt);
       if (nt == 0) continue;
       if (p.csa && pt < 32) {
         // index lists: this unit's into L1 (read tile by tile below), the next
@@ -603,7 +682,7 @@ attend_tc(AttendParams p, int n_units) {
         for (int x = pt; x < lines; x += 32) asm volatile("prefetch.global.L1 [%0];" ::"l"(il + 32 * x));
         const int un = u + gridDim.x;
         if (un < n_units) {
-          const int32_t *nl = p.idx + (long long)(un / p.nsplit) * p.k;
+          const int32_t *nl = p.idx + (long long)fdiv(un, p.fd_nsplit) * p.k;
           for (int x = pt; x < lines; x += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(nl + 32 * x));
         }
       }
@@ -637,7 +716,7 @@ attend_tc(AttendParams p, int n_units) {
               cw[i] = __ldg(reinterpret_cast<const uint2 *>(rp + col_off));
               sc[i] = __ldg(reinterpret_cast<const float *>(rp + sc_off));
             }
-            if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+            if (!twait_sleep(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
 #pragma unroll
             for (int i = 0; i < NR; ++i) {
               const uint32_t w2[2] = {cw[i].x, cw[i].y};
@@ -663,7 +742,7 @@ attend_tc(AttendParams p, int n_units) {
               const int row = slot_row(p, ks, b, qi, kk, v);
               src8[i] = (kk < ks.nw4 ? wrec : crec) + (long long)row * p.rec + col_off;
             }
-            if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+            if (!twait_sleep(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
 #pragma unroll
             for (int i = 0; i < NR; ++i) cp_async16(tile + sw128_off(prow + i * RPP, cc), src8[i], 16);
             cp_async_arrive_noinc(bar(bars->kv_full[st]));
@@ -681,7 +760,7 @@ attend_tc(AttendParams p, int n_units) {
           const int row = slot_row(p, ks, b, qi, kk, v);
           src[i] = (kk < ks.nw4 ? wbase : cbase) + (long long)row * C + chunk * 8;
         }
-        if (!twait(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
+        if (!twait_sleep(bar(bars->kv_empty[st]), ((g / L::NS) & 1) ^ 1, TR_P_KVEMPTY)) return;
         const uint32_t tile = sbase + L::kv_off + st * NKB * kTileBytes + kb_off;
 #pragma unroll
         for (int i = 0; i < NR; ++i) cp_async16(tile + sw128_off(prow + i * RPP, cc), src[i], 16);
@@ -690,12 +769,11 @@ attend_tc(AttendParams p, int n_units) {
     }
     }();
     cp_async_wait_all();
-    if (p.cluster) {
+    if (M == 64 && p.cluster) {
       // one unit per CTA: join the merge once its last P.V has landed
-      const int u = blockIdx.x;
-      const int bq = u / p.nsplit, sp = u % p.nsplit;
-      const int b = bq / p.n_q, qi = bq % p.n_q;
-      const KeySet ks = key_set_tc(p, qi);
+      const Unit x = unit_of(p, blockIdx.x);
+      const int b = x.b, qi = x.qi0, sp = x.sp;
+      const KeySet ks = group_key_set(p, x.qg);
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
       // the unit's last P.V has landed once the MMA warp's final commit has
@@ -708,31 +786,34 @@ attend_tc(AttendParams p, int n_units) {
         cluster_merge<C>(p, smem, bars, tmem, nt, sp, b, qi, rope_all, nullptr);
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == MMAW) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_bf16(64, KT, 0, 0);
+      constexpr uint32_t IDESC_S = idesc_bf16(M, KT, 0, 0);
       constexpr int NPV = C < 256 ? C : 256;
-      constexpr uint32_t IDESC_PV = idesc_bf16(64, NPV, 0, 1);
-      const uint32_t tS = tmem + (16u << 16);
+      constexpr uint32_t IDESC_PV = idesc_bf16(M, NPV, 0, 1);
+      const uint32_t tS = tmem + (L::s_lane << 16);
       uint32_t g = 0, iq = 0;
       bool ok = true;
       auto issue_pv = [&](uint32_t gg, bool first) -> bool {
-        const int st = gg % kSP;               // S / P buffer
+        const int st = gg % SP;               // S / P buffer
         const int kst = gg % L::NS;            // key-tile stage
-        if (!twait(bar(bars->p_full[st]), (gg / kSP) & 1, TR_M_PFULL)) return false;
+        if (!twait(bar(bars->p_full[st]), (gg / SP) & 1, TR_M_PFULL)) return false;
         if (first && !twait(bar(bars->o_empty), (iq & 1) ^ 1, TR_M_OEMPTY)) return false;
         tc_fence_after();
-        const uint32_t pa = sbase + L::p_off + st * kTileBytes;
+        const uint32_t pa = sbase + L::p_off + st * L::kPBytes;
         const uint32_t va = sbase + L::kv_off + kst * L::NKB * kTileBytes;
         const uint64_t pd = sdesc_sw128(pa, 16, 1024);
         const uint64_t vd = sdesc_sw128(va, kTileBytes, 1024);
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk) {
+          // M = 128: keys [0, 32) of the tile into O accumulator 0, [32, 64) into 1
+          const uint32_t o_acc = M == 128 ? (kk >> 1) * C : 0;
+          const bool reset = first && (M == 128 ? (kk & 1) == 0 : kk == 0);
 #pragma unroll
           for (int nh = 0; nh < C / NPV; ++nh) {
             const uint64_t voff = (nh * (NPV / 64) * kTileBytes + kk * 16 * 128) >> 4;
-            umma_bf16(tmem + nh * NPV, pd + ((kk * 32) >> 4), vd + voff, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+            umma_bf16(tmem + o_acc + nh * NPV, pd + ((kk * 32) >> 4), vd + voff, IDESC_PV, reset ? 0u : 1u);
           }
         }
         umma_commit(bar(bars->kv_empty[kst]));
@@ -740,22 +821,22 @@ attend_tc(AttendParams p, int n_units) {
         return true;
       };
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const int qi = (u / p.nsplit) % p.n_q;
-        const KeySet ks = key_set_tc(p, qi);
+        const Unit x = unit_of(p, u);
+        const KeySet ks = group_key_set(p, x.qg);
         int j0, nt;
-        split_range(ks, p.nsplit, u % p.nsplit, j0, nt);
+        split_range(ks, p.nsplit, x.sp, j0, nt);
         if (nt == 0) continue;
         if (!twait(bar(bars->q_full), iq & 1, TR_M_QFULL)) { ok = false; break; }
         fence_proxy_async();
         tc_fence_after();
-        // S of tile j, then P.V of tile j - kLookahead; the unit's last P.Vs
+        // S of tile j, then P.V of tile j - LA; the unit's last P.Vs
         // are issued before the next unit's Q is awaited (its epilogue waits
         // for them)
         int npv = 0;                           // P.Vs of this unit issued
         for (int j = 0; j < nt && ok; ++j) {
           const uint32_t gj = g + j;
-          const int st = gj % kSP;
-          const uint32_t ph = (gj / kSP) & 1;
+          const int st = gj % SP;
+          const uint32_t ph = (gj / SP) & 1;
           const int kst = gj % L::NS;
           if (!twait(bar(bars->kv_full[kst]), (gj / L::NS) & 1, TR_M_KVFULL) ||
               !twait(bar(bars->s_empty[st]), ph ^ 1, TR_M_SEMPTY)) {
@@ -775,7 +856,7 @@ attend_tc(AttendParams p, int n_units) {
           }
           umma_commit(bar(bars->s_full[st]));
           if (j == nt - 1) umma_commit(bar(bars->q_empty));
-          if (j >= kLookahead) {
+          if (j >= LA) {
             if (!issue_pv(g + npv, npv == 0)) ok = false;
             ++npv;
           }
@@ -789,13 +870,314 @@ attend_tc(AttendParams p, int n_units) {
       mbar_wait(bar(bars->mma_done), 0, p.status);
     }
     __syncwarp();
+  } else if constexpr (M == 128) {
+    // ------------------------------------------------------------ softmax + epilogue, 128 rows
+    // Query groups on 128 rows (c = 128).  Warps w and w + 4 share TMEM lane
+    // quarter w % 4: thread (warp, lane) owns row r = (w % 4) * 32 + lane --
+    // head rh of query rg of the group -- for the keys [32 hf, 32 hf + 32) of
+    // every tile, hf = w / 4, with its own running max and sum and its own O
+    // accumulator (P.V of those keys).  At the end of a unit the two warps
+    // exchange (max, sum) and each combines both accumulators for the O
+    // columns [hf C/2, (hf + 1) C/2).  A warp's rows belong to one query
+    // (n_h >= 32) or two (n_h = 16).
+    [&]() {
+    const int q4 = warp & 3, hf = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const int rg = r / p.n_h, rh = r - rg * p.n_h;
+    const int rg0 = (q4 * 32) / p.n_h, rg1 = (q4 * 32 + 31) / p.n_h;
+    const bool second = rg != rg0;
+    const float *rope_cs = rope_all + warp * 128 + (second ? 64 : 0);
+    const float zs = p.scale * kLog2e;
+    const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+    const uint32_t tO = tmem + lane_base + hf * C;   // this warp's O accumulator
+    constexpr int CH = C / 2;             // O columns (and Q dims) of this warp
+    constexpr int NQC = CH / 8;           // 16-byte chunks of a half row
+    const int col_lo = hf * CH;
+    // bounded rendezvous of the two warps of this lane quarter: their shared
+    // memory writes before it are visible to both after it
+    uint32_t npair = 0;
+    auto pair_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->pair[q4]));
+      return mbar_wait(bar(bars->pair[q4]), (npair++) & 1, p.status);
+    };
+    // Q of the next unit: this thread's half row is copied (cp.async) into
+    // its own shared-memory slot while the current unit runs, then moved to
+    // tensor memory (row r, columns q_col + col_lo/2 ..) once the unit's last
+    // S has been read.  Chunk i sits at slot i ^ (lane & 7) (fewer bank
+    // conflicts on the way out).
+    const uint32_t qstage = sbase + L::q_off + (uint32_t)(r * 2 + hf) * (CH * 2);
+    auto stage_q = [&](int uq) {
+      const Unit xq = unit_of(p, uq);
+      const bool live = xq.qi0 + rg < p.n_q;
+      const long long qrow = live ? ((long long)xq.b * p.n_q + xq.qi0 + rg) * p.n_h + rh : 0;
+      const char *src = reinterpret_cast<const char *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) + qrow * C + col_lo);
+#pragma unroll
+      for (int i = 0; i < NQC; ++i) cp_async16(qstage + ((i ^ (lane & 7)) << 4), src + 16 * i, live ? 16 : 0);
+      cp_async_commit();
+    };
+    uint32_t nq = 0;                      // Q writes so far (q_empty parity)
+    auto write_q = [&]() -> bool {
+      if (nq > 0 && !twait(bar(bars->q_empty), (nq - 1) & 1, TR_P_QEMPTY)) return false;
+      tc_fence_after();
+      cp_async_wait_all();
+      uint32_t v[NQC * 4];
+#pragma unroll
+      for (int i = 0; i < NQC; ++i)
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v[4 * i]), "=r"(v[4 * i + 1]), "=r"(v[4 * i + 2]), "=r"(v[4 * i + 3])
+                     : "r"(qstage + ((i ^ (lane & 7)) << 4))
+                     : "memory");
+      const uint32_t tq = tmem + lane_base + L::q_col + col_lo / 2;
+#pragma unroll
+      for (int y = 0; y < NQC / 4; ++y) tmem_st_32x32b_x16(tq + 16 * y, *reinterpret_cast<const uint32_t(*)[16]>(&v[16 * y]));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->q_full));
+      ++nq;
+      return true;
+    };
+    auto next_unit = [&](int u0) -> int {
+      for (int uu = u0 + gridDim.x; uu < n_units; uu += gridDim.x) {
+        int a0, an;
+        const Unit xu = unit_of(p, uu);
+        split_range(group_key_set(p, xu.qg), p.nsplit, xu.sp, a0, an);
+        if (an > 0) return uu;
+      }
+      return -1;
+    };
+    constexpr double kTwoPi = 6.283185307179586476925286766559, kInvTwoPi = 0.15915494309189533576888376337251;
+    // (the angle is reduced to [-pi, pi] in double; the intrinsic's error there is below 1e-6)
+    int q_ready_u = -1;
+    uint32_t g = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      const long long tu0 = TRACE ? clock64() : 0;
+      const Unit ux = unit_of(p, u);
+      const int b = ux.b, qi = ux.qi0;
+      const bool live = qi + rg < p.n_q;
+      const int tw0 = p.start_pos + qi + rg0, tw1 = p.start_pos + qi + rg1;
+      const KeySet ks = group_key_set(p, ux.qg);
+      int j0, nt;
+      split_range(ks, p.nsplit, ux.sp, j0, nt);
+      // this row's keys among the group's slots: window slots [w_lo, w_hi)
+      // (tokens tq - w + 1 .. tq) and entry slots [nw4, c_hi)
+      const int tq = p.start_pos + qi + rg;
+      const int w_lo = max(0, tq - p.w + 1 - ks.t0), w_hi = p.w > 0 ? min(tq - ks.t0 + 1, ks.nw) : 0;
+      const int c_hi = ks.nw4 + fdiv(tq + 1, p.fd_m);
+      if (nt > 0 && q_ready_u != u) {
+        stage_q(u);
+        if (!write_q()) return;
+        q_ready_u = u;
+      }
+      const int un = nt > 0 ? next_unit(u) : -1;
+      if (un >= 0) stage_q(un);
+      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                            (live ? (((long long)b * p.n_q + qi + rg) * p.n_h + rh) * C : 0);
+      if (nt == 0) {
+        if (live)
+          for (int col = col_lo; col < col_lo + CH; col += 8)
+            *reinterpret_cast<uint4 *>(orow + col) = make_uint4(0, 0, 0, 0);
+        continue;
+      }
+      // RoPE tables of the warp's queries (inverse rotation in the epilogue)
+      __syncwarp();
+      if (lane < p.rd / 2) {
+#pragma unroll
+        for (int k2 = 0; k2 < 2; ++k2) {
+          double ang = (double)(k2 ? tw1 : tw0) * freq[lane];
+          ang -= kTwoPi * rint(ang * kInvTwoPi);
+          float sn, cs;
+          __sincosf((float)ang, &sn, &cs);
+          rope_all[warp * 128 + k2 * 64 + lane] = cs;
+          rope_all[warp * 128 + k2 * 64 + 32 + lane] = sn;
+        }
+      }
+      __syncwarp();
+      // running max (log2 units; -inf until a valid key is seen) and sum
+      float m_used = -INFINITY, l = 0.f;
+      if (TRACE) tr[TR_S_TILE] += clock64() - tu0;   // the unit's setup
+      if (TRACE) { tr[TR_UNITS] += 1; tr[TR_TILES] += nt; }
+      for (int j = 0; j < nt; ++j) {
+        const uint32_t gj = g + j;
+        const int st = gj % SP;
+        const uint32_t ph = (gj / SP) & 1;
+        if (!twait(bar(bars->s_full[st]), ph, TR_S_SFULL)) return;
+        if (TRACE && threadIdx.x == 0 && j == 0 && ts[2] == 0) ts[2] = global_ns();
+        // sub-phase cycles of the tile (the merge slots are unused at M = 128)
+        long long tp = TRACE ? clock64() : 0;
+        auto phase = [&](int slot) {
+          if (TRACE) {
+            const long long t1 = clock64();
+            tr[slot] += t1 - tp;
+            tp = t1;
+          }
+        };
+        tc_fence_after();
+        uint32_t sv[32];
+        tmem_ld_32x32b_x16(tmem + lane_base + L::s_col(st) + 32 * hf, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
+        tmem_ld_32x32b_x16(tmem + lane_base + L::s_col(st) + 32 * hf + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->s_empty[st]));
+        phase(TR_S_MERGE_READY);
+        // this row's valid keys among the warp's 32
+        const int kb = (j0 + j) * KT + 32 * hf;
+        const uint32_t vm = range_bits(kb, w_lo, w_hi) | range_bits(kb, ks.nw4, c_hi);
+        float z[32];
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          z[x] = ((vm >> x) & 1u) ? __uint_as_float(sv[x]) * zs : -INFINITY;
+          mx[x & 3] = fmaxf(mx[x & 3], z[x]);
+        }
+        const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        phase(TR_S_MERGE_FULL);
+        // lazy rescaling: the max moves only when it grows by more than 8
+        bool need = false;
+        float alpha = 1.f;
+        if (tmax != -INFINITY && (m_used == -INFINITY || tmax > m_used + 8.f)) {
+          if (m_used != -INFINITY) {   // before the first valid key O and l are 0
+            need = true;
+            alpha = ex2_approx(m_used - tmax);
+            l *= alpha;
+          }
+          m_used = tmax;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // rescale this warp's O accumulator after the P.V of the previous tile lands
+          const uint32_t gp = gj - 1;
+          if (TRACE) tr[TR_RESCALES] += 1;
+          if (!twait(bar(bars->pv_done[gp % SP]), (gp / SP) & 1, TR_S_RESCALE)) return;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < C; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld_32x32b_x16(tO + c0, ov);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 16; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+            tmem_st_32x32b_x16(tO + c0, ov);
+          }
+          tmem_st_wait();
+        }
+        const float m_eff = m_used == -INFINITY ? 0.f : m_used;
+        float ps[2] = {0.f, 0.f};
+        uint32_t pk[16];
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+          const float p0 = ex2_approx(z[x] - m_eff), p1 = ex2_approx(z[x + 1] - m_eff);
+          ps[(x >> 1) & 1] += p0 + p1;
+          pk[x / 2] = pack_bf16x2(p0, p1);
+        }
+        l += ps[0] + ps[1];
+        phase(TR_S_PUSH);
+        // P buffer `st` is free once the P.V of tile gj - 2 has completed
+        if (!twait(bar(bars->pv_done[st]), ph ^ 1, TR_S_PBUF)) return;
+        const uint32_t prow = sbase + L::p_off + st * L::kPBytes;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, 4 * hf + c4)),
+                       "r"(pk[4 * c4]), "r"(pk[4 * c4 + 1]), "r"(pk[4 * c4 + 2]), "r"(pk[4 * c4 + 3])
+                       : "memory");
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(bars->p_full[st]));
+        phase(TR_S_WEIGHTS);
+        if (j == nt - 1 && un >= 0) {
+          // the unit's last S has been read: the next unit's Q goes in now
+          if (!write_q()) return;
+          q_ready_u = un;
+          phase(TR_S_MERGE_LOOP);
+        }
+      }
+      // -------- epilogue: combine the two halves' accumulators with the
+      // sink, inverse RoPE, store this warp's columns
+      float m_o, l_o;
+      const long long tx0 = TRACE ? clock64() : 0;
+      {
+        float2 *xl = reinterpret_cast<float2 *>(xch);
+        xl[warp * 32 + lane] = make_float2(m_used, l);
+        if (!pair_sync()) return;
+        const float2 o2 = xl[(warp ^ 4) * 32 + lane];
+        m_o = o2.x;
+        l_o = o2.y;
+      }
+      if (TRACE) tr[TR_P_ISSUE] += clock64() - tx0;   // the pair exchange
+      {
+        const uint32_t gl = g + nt - 1;
+        if (!twait(bar(bars->pv_done[gl % SP]), (gl / SP) & 1, TR_S_EPI_WAIT)) return;
+      }
+      if (TRACE && threadIdx.x == 0 && ts[3] == 0) ts[3] = global_ns();
+      const long long te0 = TRACE ? clock64() : 0;
+      tc_fence_after();
+      // weights of accumulator 0 (keys [0, 32) of each tile) and 1
+      const float m0 = hf ? m_o : m_used, m1 = hf ? m_used : m_o;
+      const float l0 = hf ? l_o : l, l1 = hf ? l : l_o;
+      const float mm = fmaxf(m0, m1);
+      float w0 = 0.f, w1 = 0.f, inv = 0.f;
+      if (mm != -INFINITY) {
+        w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - mm);
+        w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mm);
+        const float sink2 = live ? p.sink[rh] * kLog2e : 0.f;
+        inv = 1.f / (w0 * l0 + w1 * l1 + exp2f(sink2 - mm));
+      }
+      w0 *= inv;
+      w1 *= inv;
+#pragma unroll 1
+      for (int c0 = col_lo; c0 < col_lo + CH; c0 += 16) {
+        uint32_t o0[16], o1[16];
+        tmem_ld_32x32b_x16(tmem + lane_base + c0, o0);
+        tmem_ld_32x32b_x16(tmem + lane_base + C + c0, o1);
+        tmem_ld_wait();
+        float v[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] = __uint_as_float(o0[x]) * w0 + __uint_as_float(o1[x]) * w1;
+        if (c0 + 16 > C - p.rd) {
+#pragma unroll
+          for (int x = 0; x < 16; x += 2) {
+            const int col = c0 + x;
+            if (col >= C - p.rd) {
+              const int pi = (col - (C - p.rd)) / 2;
+              const float cs = rope_cs[pi], sn = rope_cs[32 + pi];
+              const float a = v[x], bb = v[x + 1];
+              v[x] = a * cs + bb * sn;
+              v[x + 1] = -a * sn + bb * cs;
+            }
+          }
+        }
+        if (live) {
+          uint4 ww0, ww1;
+          ww0.x = pack_bf16x2(v[0], v[1]); ww0.y = pack_bf16x2(v[2], v[3]);
+          ww0.z = pack_bf16x2(v[4], v[5]); ww0.w = pack_bf16x2(v[6], v[7]);
+          ww1.x = pack_bf16x2(v[8], v[9]); ww1.y = pack_bf16x2(v[10], v[11]);
+          ww1.z = pack_bf16x2(v[12], v[13]); ww1.w = pack_bf16x2(v[14], v[15]);
+          *reinterpret_cast<uint4 *>(orow + c0) = ww0;
+          *reinterpret_cast<uint4 *>(orow + c0 + 8) = ww1;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->o_empty));
+      if (TRACE) tr[TR_S_EPI] += clock64() - te0;
+      if (TRACE && threadIdx.x == 0 && ts[4] == 0) ts[4] = global_ns();
+      g += nt;
+    }
+    cp_async_wait_all();
+    }();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     [&]() {
     float *rope_cs = rope_all + warp * 64;
     const int q4 = warp;                  // TMEM lane quarter
     const int hl = lane & 15, half = lane >> 4;
-    const int r = q4 * 16 + hl;           // head row
+    const int r = q4 * 16 + hl;           // MMA row
+    // row r is head rh of query rg of the unit's group; every row of a warp
+    // belongs to query wg of the group (n_h is a multiple of 16 when G > 1)
+    const int rg = r / p.n_h, rh = r - rg * p.n_h;
+    const int wg = p.G > 1 ? (q4 * 16) / p.n_h : 0;
     const float zs = p.scale * kLog2e;
     const uint32_t lane_S = (uint32_t)(q4 * 32 + 16) << 16;
     const uint32_t lane_O = (uint32_t)(q4 * 32) << 16;
@@ -806,10 +1188,11 @@ attend_tc(AttendParams p, int n_units) {
     auto write_q = [&](int uq) -> bool {
       if (nq > 0 && !twait(bar(bars->q_empty), (nq - 1) & 1, TR_P_QEMPTY)) return false;
       tc_fence_after();
-      const int bqq = uq / p.nsplit;
-      const bool live = r < p.n_h;
+      const Unit xq = unit_of(p, uq);
+      const bool live = rg < p.G && xq.qi0 + rg < p.n_q;
+      const long long qrow = live ? ((long long)xq.b * p.n_q + xq.qi0 + rg) * p.n_h + rh : 0;
       const uint4 *src = reinterpret_cast<const uint4 *>(
-          reinterpret_cast<const __nv_bfloat16 *>(p.q) + ((long long)bqq * p.n_h + (live ? r : 0)) * C + half * (C / 2));
+          reinterpret_cast<const __nv_bfloat16 *>(p.q) + qrow * C + half * (C / 2));
       const uint32_t tq = tmem + lane_S + L::q_col;
       // C/16 uint4 (C/4 words) per thread, in batches of 16 uint4 whose loads are all in flight
       constexpr int PER = C / 16, BATCH = PER < 16 ? PER : 16;
@@ -833,7 +1216,8 @@ attend_tc(AttendParams p, int n_units) {
     auto next_unit = [&](int u0) -> int {
       for (int uu = u0 + gridDim.x; uu < n_units; uu += gridDim.x) {
         int a0, an;
-        split_range(key_set_tc(p, (uu / p.nsplit) % p.n_q), p.nsplit, uu % p.nsplit, a0, an);
+        const Unit xu = unit_of(p, uu);
+        split_range(group_key_set(p, xu.qg), p.nsplit, xu.sp, a0, an);
         if (an > 0) return uu;
       }
       return -1;
@@ -841,10 +1225,11 @@ attend_tc(AttendParams p, int n_units) {
     int q_ready_u = -1;                   // unit whose Q is already in tensor memory
     uint32_t g = 0, iq = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const int bq = u / p.nsplit, sp = u % p.nsplit;
-      const int b = bq / p.n_q, qi = bq % p.n_q;
-      const int t = p.start_pos + qi;
-      const KeySet ks = key_set_tc(p, qi);
+      const Unit ux = unit_of(p, u);
+      const int bq = ux.bq, sp = ux.sp, b = ux.b, qi = ux.qi0;
+      const int t = p.start_pos + qi + wg;   // this warp's query token
+      const bool live = rg < p.G && qi + rg < p.n_q;
+      const KeySet ks = group_key_set(p, ux.qg);
       int j0, nt;
       split_range(ks, p.nsplit, sp, j0, nt);
       if (nt > 0 && q_ready_u != u) {
@@ -855,17 +1240,20 @@ attend_tc(AttendParams p, int n_units) {
         // pull the next unit's Q rows towards L2 now; they are written to tensor
         // memory after this unit's last S
         const int un = next_unit(u);
-        if (un >= 0 && r < p.n_h) {
-          const char *nq = reinterpret_cast<const char *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) +
-                                                          ((long long)(un / p.nsplit) * p.n_h + r) * C + half * (C / 2));
+        const Unit xn = unit_of(p, un < 0 ? 0 : un);
+        if (un >= 0 && rg < p.G && xn.qi0 + rg < p.n_q) {
+          const char *nq = reinterpret_cast<const char *>(
+              reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+              (((long long)xn.b * p.n_q + xn.qi0 + rg) * p.n_h + rh) * C + half * (C / 2));
 #pragma unroll
           for (int x = 0; x < C / 128; ++x) asm volatile("prefetch.global.L2 [%0];" ::"l"(nq + 128 * x));
         }
       }
       if (nt == 0 && p.nsplit > 1 && !p.cluster) continue;   // the combine kernel skips empty ranges
-      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (((long long)b * p.n_q + qi) * p.n_h + r) * C;
+      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) +
+                            (live ? (((long long)b * p.n_q + qi + rg) * p.n_h + rh) * C : 0);
       if (nt == 0 && !p.cluster) {
-        if (r < p.n_h)
+        if (live)
           for (int col = half * (C / 2); col < (half + 1) * (C / 2); col += 8)
             *reinterpret_cast<uint4 *>(orow + col) = make_uint4(0, 0, 0, 0);
         continue;
@@ -886,8 +1274,8 @@ attend_tc(AttendParams p, int n_units) {
       if (TRACE) { tr[TR_UNITS] += 1; tr[TR_TILES] += nt; }
       for (int j = 0; j < nt; ++j) {
         const uint32_t gj = g + j;
-        const int st = gj % kSP;
-        const uint32_t ph = (gj / kSP) & 1;
+        const int st = gj % SP;
+        const uint32_t ph = (gj / SP) & 1;
         if (!twait(bar(bars->s_full[st]), ph, TR_S_SFULL)) return;
         if (TRACE && threadIdx.x == 0 && j == 0 && ts[2] == 0) ts[2] = global_ns();
         tc_fence_after();
@@ -904,8 +1292,13 @@ attend_tc(AttendParams p, int n_units) {
         {
           const int k0 = (j0 + j) * KT + lane, k1 = k0 + 32;
           bool v0 = false, v1 = false;
-          if (k0 < ks.nk) slot_row(p, ks, b, qi, k0, v0);
-          if (k1 < ks.nk) slot_row(p, ks, b, qi, k1, v1);
+          if (p.G > 1) {
+            v0 = k0 < ks.nk && slot_of_token(p, ks, k0, t);
+            v1 = k1 < ks.nk && slot_of_token(p, ks, k1, t);
+          } else {
+            if (k0 < ks.nk) slot_row(p, ks, b, qi, k0, v0);
+            if (k1 < ks.nk) slot_row(p, ks, b, qi, k1, v1);
+          }
           const uint32_t m0 = __ballot_sync(0xffffffffu, v0), m1 = __ballot_sync(0xffffffffu, v1);
           vmask = half ? m1 : m0;
         }
@@ -931,7 +1324,7 @@ attend_tc(AttendParams p, int n_units) {
           // rescale O rows of this warp after the PV of the previous tile lands
           const uint32_t gp = gj - 1;
           if (TRACE) tr[TR_RESCALES] += 1;
-          if (!twait(bar(bars->pv_done[gp % kSP]), (gp / kSP) & 1, TR_S_RESCALE)) return;
+          if (!twait(bar(bars->pv_done[gp % SP]), (gp / SP) & 1, TR_S_RESCALE)) return;
           tc_fence_after();
 #pragma unroll 1
           for (int c0 = 0; c0 < C / 2; c0 += 16) {
@@ -979,7 +1372,7 @@ attend_tc(AttendParams p, int n_units) {
       // -------- epilogue: normalise, inverse RoPE, store
       if (nt > 0) {
         const uint32_t gl = g + nt - 1;
-        if (!twait(bar(bars->pv_done[gl % kSP]), (gl / kSP) & 1, TR_S_EPI_WAIT)) return;
+        if (!twait(bar(bars->pv_done[gl % SP]), (gl / SP) & 1, TR_S_EPI_WAIT)) return;
       }
       if (TRACE && threadIdx.x == 0 && ts[3] == 0) {
         ts[3] = global_ns();
@@ -1034,7 +1427,7 @@ attend_tc(AttendParams p, int n_units) {
         ++iq;
         continue;
       }
-      const float sink2 = (r < p.n_h) ? p.sink[r] * kLog2e : 0.f;
+      const float sink2 = live ? p.sink[rh] * kLog2e : 0.f;
       const float inv = 1.f / (ltot + exp2f(sink2 - m_used));
 #pragma unroll 1
       for (int c0 = 0; c0 < C / 2; c0 += 16) {
@@ -1058,7 +1451,7 @@ attend_tc(AttendParams p, int n_units) {
             }
           }
         }
-        if (r < p.n_h) {
+        if (live) {
           uint4 w0, w1;
           w0.x = pack_bf16x2(v[0], v[1]); w0.y = pack_bf16x2(v[2], v[3]);
           w0.z = pack_bf16x2(v[4], v[5]); w0.w = pack_bf16x2(v[6], v[7]);
@@ -1081,7 +1474,7 @@ attend_tc(AttendParams p, int n_units) {
   if (TRACE) {
     tr[TR_TOTAL] = clock64() - t_start;
     // one thread per role reports: producer thread 0, MMA lane 0, softmax thread 0
-    const bool rep = threadIdx.x == kProdWarp0 * 32 || threadIdx.x == kMmaWarp * 32 || threadIdx.x == 0;
+    const bool rep = threadIdx.x == PW0 * 32 || threadIdx.x == MMAW * 32 || threadIdx.x == 0;
     if (rep)
       for (int i = 0; i < TR_COUNT; ++i)
         if (tr[i]) atomicAdd(&g_attn_trace[i], tr[i]);
@@ -1101,22 +1494,24 @@ attend_tc(AttendParams p, int n_units) {
     atomicAdd(&g_attn_trace[TR_T_CTAS], 1ull);
   }
   if (threadIdx.x == 0) step_trace_record(p.csa ? ST_ATTEND_CSA : ST_ATTEND_HCA, st_entry, st_ready);
-  if (warp == kMmaWarp) tmem_dealloc(tmem, L::tmem_cols);
+  if (warp == MMAW) tmem_dealloc(tmem, L::tmem_cols);
 }
 
-template <int C>
+template <int C, int M>
 int ensure_attr() {
   static std::atomic<bool> attr_set_dev[kMaxDevices];
   std::atomic<bool> &attr_set = attr_set_dev[device_slot()];
   if (!attr_set) {
-    const int smem = (int)Layout<C>::bytes;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int smem = (int)Layout<C, M>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc<C, M, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_tc<C, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_tc<C, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attend_tc<C, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(attend_tc<C, M, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if constexpr (M == 64) {
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attend_tc<C, M, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(attend_tc<C, M, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    }
     if (e != cudaSuccess) return fail(HCA_ERR_CUDA, "attend_tc smem attribute: %s", cudaGetErrorString(e));
     attr_set = true;
   }
@@ -1130,7 +1525,7 @@ int max_active_clusters(int ns) {
   if (ns < 1 || ns > kMaxClusterSplits) return 0;
   std::atomic<int> *cache = cache_dev[device_slot()];
   if (cache[ns]) return cache[ns];
-  if (ensure_attr<C>()) return 0;
+  if (ensure_attr<C, 64>()) return 0;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(ns * 64, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -1143,7 +1538,7 @@ int max_active_clusters(int ns) {
   cfg.attrs = at;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<C, false, false>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, attend_tc<C, 64, false, false>, &cfg) != cudaSuccess) {
     (void)cudaGetLastError();
     n = 0;
   }
@@ -1151,11 +1546,11 @@ int max_active_clusters(int ns) {
   return n;
 }
 
-template <int C>
+template <int C, int M>
 int launch_tc(const AttendParams &p, cudaStream_t s) {
-  const int n_units = p.B * p.n_q * p.nsplit;
-  const size_t smem = Layout<C>::bytes;
-  int rc0 = ensure_attr<C>();
+  const int n_units = p.B * p.n_qg * p.nsplit;
+  const size_t smem = Layout<C, M>::bytes;
+  int rc0 = ensure_attr<C, M>();
   if (rc0) return rc0;
   // cluster merge: one unit per CTA, a query's splits form one cluster
   const int grid = p.cluster ? n_units : (n_units < sm_budget(p) ? n_units : sm_budget(p));
@@ -1175,10 +1570,16 @@ int launch_tc(const AttendParams &p, cudaStream_t s) {
   cfg.attrs = at;
   cfg.numAttrs = p.cluster ? 2 : 1;
   const bool tr = attend_trace_on();
-  const cudaError_t e = p.kv_mixed ? (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, true, true>, p, n_units)
-                                         : cudaLaunchKernelEx(&cfg, attend_tc<C, false, true>, p, n_units))
-                                   : (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, true, false>, p, n_units)
-                                         : cudaLaunchKernelEx(&cfg, attend_tc<C, false, false>, p, n_units));
+  cudaError_t e;
+  if constexpr (M == 128) {
+    e = tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, M, true, false>, p, n_units)
+           : cudaLaunchKernelEx(&cfg, attend_tc<C, M, false, false>, p, n_units);
+  } else {
+    e = p.kv_mixed ? (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, M, true, true>, p, n_units)
+                         : cudaLaunchKernelEx(&cfg, attend_tc<C, M, false, true>, p, n_units))
+                   : (tr ? cudaLaunchKernelEx(&cfg, attend_tc<C, M, true, false>, p, n_units)
+                         : cudaLaunchKernelEx(&cfg, attend_tc<C, M, false, false>, p, n_units));
+  }
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
     return fail(HCA_ERR_CUDA, "attend_tc launch: %s", cudaGetErrorString(e));
@@ -1259,12 +1660,30 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
     p.rope_freq[i] = i < p.rd / 2 ? std::exp2(-2.0 * i / (double)p.rd * std::log2((double)p.theta)) : 0.0;
   p.nsplit = 1;
   p.cluster = 0;
+  p.G = 1;
+  p.n_qg = p.n_q;
+  p.fd_m = make_fastdiv((uint32_t)p.m);
+  p.fd_nsplit = make_fastdiv(1);
+  p.fd_nqg = make_fastdiv((uint32_t)p.n_qg);
   if (p.kv_mixed && !tc_path(p))
     return fail(HCA_ERR_UNSUPPORTED, "mixed-precision KV rows need the tensor-core path (bf16, n_h <= 64, c in {128, 256, 512})");
   if (tc_path(p)) {
     if (!p.kv_comp) p.cap = 0;   // no visible entries: masked slots then read row 0 of the dummy map
     const SplitPlan sp = plan_splits(p, ws && ws_bytes >= attend_workspace_bytes(p));
     const int ns = sp.ns;
+    if (ns == 1 && !p.csa && !p.win_is_ring && p.n_q > 1 && p.n_h % 16 == 0) {
+      // G = rows / n_h queries per unit fill the MMA's 128 rows (c = 128,
+      // bf16 rows) or 64 rows; kept while the groups still give every CTA of
+      // the budget a unit
+      for (int rows = (p.c == 128 && !p.kv_mixed) ? 128 : 64; rows >= 64; rows -= 64) {
+        const int G = rows / p.n_h, n_qg = (p.n_q + G - 1) / G;
+        if (G >= 2 && rows % p.n_h == 0 && (long long)p.B * n_qg >= sm_budget(p)) {
+          p.G = G;
+          p.n_qg = n_qg;
+          break;
+        }
+      }
+    }
     if (sp.cluster) {
       p.nsplit = ns;
       p.cluster = 1;
@@ -1274,11 +1693,14 @@ int run_attend(const AttendParams &p_in, void *ws, size_t ws_bytes, cudaStream_t
       p.part_o = static_cast<float *>(ws);
       p.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + ((q * p.c * 4 + 255) & ~(size_t)255));
     }
+    p.fd_nsplit = make_fastdiv((uint32_t)p.nsplit);
+    p.fd_nqg = make_fastdiv((uint32_t)p.n_qg);
+    const bool m128 = p.G * p.n_h == 128;
     int rc;
     switch (p.c) {
-      case 128: rc = tc::launch_tc<128>(p, s); break;
-      case 256: rc = tc::launch_tc<256>(p, s); break;
-      default: rc = tc::launch_tc<512>(p, s); break;
+      case 128: rc = m128 ? tc::launch_tc<128, 128>(p, s) : tc::launch_tc<128, 64>(p, s); break;
+      case 256: rc = tc::launch_tc<256, 64>(p, s); break;
+      default: rc = tc::launch_tc<512, 64>(p, s); break;
     }
     if (rc || p.nsplit == 1 || p.cluster) return rc;
     return HCA_LAUNCH("attend_combine", s, attend_combine<__nv_bfloat16><<<dim3(p.B * p.n_q, (p.n_h + 3) / 4), 128, 0, s>>>(p));

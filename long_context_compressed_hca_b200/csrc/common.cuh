@@ -81,6 +81,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
   }
 }
 
+// The same wait for threads that are not latency-critical (loaders far ahead
+// of their consumers): they sleep between polls, so that their polling does
+// not take issue slots from the warps of the same scheduler.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, int *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(128);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+      set_timeout_status(status);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- dependent launch
 // Programmatic dependent launch: pdl_trigger lets the next kernel of the
 // stream (launched with programmatic stream serialization) be scheduled and run
@@ -395,6 +411,20 @@ __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
 }
 
 // ---------------------------------------------------------------- numerics
+// 2^x by the special-function unit's approximation (PTX ex2.approx.ftz.f32):
+// relative error near 2^-22, results below 2^-126 flushed to +0, 2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Bits [a - base, b - base) of a 32-bit mask, clipped to [0, 32).
+__device__ __forceinline__ uint32_t range_bits(int base, int a, int b) {
+  const int lo = max(a - base, 0), hi = min(b - base, 32);
+  if (lo >= hi) return 0u;
+  const uint32_t upto = hi == 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return upto & ~((1u << lo) - 1u);
+}
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {

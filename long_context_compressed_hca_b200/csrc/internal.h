@@ -142,6 +142,27 @@ int launch_kv_quant_mixed(const void *x, hca_dtype dt, long long rows, int c, in
 int launch_kv_dequant_mixed(const void *in, long long rows, int c, int rd, void *out, cudaStream_t s);
 
 // ------------------------------------------------------------- attention
+// Division of dividends below 2^31 by an invariant divisor d >= 1 with one
+// multiply-high, an add and a shift (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994): s = ceil(log2 d),
+// mul = floor(2^32 (2^s - d) / d) + 1, n / d = (umulhi(n, mul) + n) >> s.
+struct FastDiv {
+  uint32_t mul, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t s = 0;
+  while ((1ull << s) < d) ++s;
+  FastDiv f;
+  f.mul = (uint32_t)((((1ull << 32) * ((1ull << s) - d)) / d) + 1);
+  f.s = s;
+  return f;
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ int fdiv(int n, const FastDiv &f) {
+  return (int)((__umulhi((uint32_t)n, f.mul) + (uint32_t)n) >> f.s);
+}
+#endif
+
 struct AttendParams {
   int B, n_q, start_pos, n_h, c, rd, w, m, k, cap;
   int csa;                 // 1: compressed set from idx; 0: all visible entries
@@ -167,6 +188,12 @@ struct AttendParams {
   int nsplit;
   int cluster;
   int max_ctas;            // CTA budget of the call (0 = every SM)
+  // query groups: G consecutive queries of one sequence share a work unit
+  // (their G x n_h head rows form the MMA's 64 rows); n_qg = ceil(n_q / G)
+  // groups per sequence.  G > 1 only for the all-entries (HCA) set with a
+  // token-indexed window and one split per group.
+  int G, n_qg;
+  FastDiv fd_m, fd_nsplit, fd_nqg;   // divisions by m, nsplit and n_qg (set at launch)
   float *part_o;           // [B*n_q, nsplit, 64, c]
   float *part_ml;          // [B*n_q, nsplit, 64, 2]
 };

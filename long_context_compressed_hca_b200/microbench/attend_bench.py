@@ -1,7 +1,7 @@
 """Time the tensor-core attention kernel alone on a synthetic prefill batch and
 print the per-role wait-cycle trace.
 
-    python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c]
+    python -m long_context_compressed_hca_b200.microbench.attend_bench <n_q> <csa|hca> [c] [n_h] [B] [m]
     python -m long_context_compressed_hca_b200.microbench.attend_bench decode <csa|hca> [B] [pos] [max_ctas] [mixed]
 
 Inputs are seeded N(0,1) (bf16); CSA index lists take one random visible entry
@@ -121,7 +121,10 @@ def main():
     n_q = int(sys.argv[1]) if len(sys.argv) > 1 else 2048
     kind = sys.argv[2] if len(sys.argv) > 2 else "csa"
     c = int(sys.argv[3]) if len(sys.argv) > 3 else 512
-    B, n_h, rd, w, m, k = 1, 64, 64, 128, 4, 512
+    n_h = int(sys.argv[4]) if len(sys.argv) > 4 else 64
+    B = int(sys.argv[5]) if len(sys.argv) > 5 else 1
+    m = int(sys.argv[6]) if len(sys.argv) > 6 else 4
+    rd, w, k = 64, 128, 512
     cap = n_q // m + 2
     dev = "cuda"
     q = synth.normal_on(dev, (B, n_q, n_h, c), 1, 1, dtype=torch.bfloat16)
@@ -136,7 +139,7 @@ def main():
     g.manual_seed(3)
     u = torch.rand(n_q, k, device=dev, generator=g)
     idx = torch.floor((j[None] + u) * V[:, None].double() / nsel.clamp(min=1)[:, None].double()).long()
-    idx = torch.where(j[None] < nsel[:, None], idx, torch.full_like(idx, -1)).int()[None].contiguous()
+    idx = torch.where(j[None] < nsel[:, None], idx, torch.full_like(idx, -1)).int()[None].expand(B, n_q, k).contiguous()
     o = torch.empty(B, n_q, n_h, c, dtype=torch.bfloat16, device=dev)
     d = hb.attn_desc(B, n_h, c, rd, w, m, k=k, dtype=hb.HCA_BF16)
 
@@ -160,8 +163,8 @@ def main():
     for i in range(n_q):
         vv = (i + 1) // m
         keys += min(w, i + 1) + (min(k, vv) if kind == "csa" else vv)
-    flops = keys * n_h * c * 4
-    print(f"attend {kind} n_q={n_q} c={c}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s")
+    flops = B * keys * n_h * c * 4
+    print(f"attend {kind} B={B} n_q={n_q} n_h={n_h} c={c} m={m}: {ms:.3f} ms, {flops / ms / 1e9:.1f} TFLOP/s")
     hb.trace_attend(1)
     run()
     tr = hb.trace_attend_read()

@@ -408,3 +408,47 @@ def test_attend_prefill_cta_budget(cuda):
 def test_attend_is_deterministic(cuda):
     runs = [_run_attend("csa", BF16, 1, 64, 64, 512, 64, 128, 4, 128, cuda)[-1] for _ in range(2)]
     assert torch.equal(runs[0], runs[1])
+
+
+GROUP_CASES = [
+    # B, n_q, n_h, c, rd, w, m, start_pos, max_ctas
+    (2, 701, 16, 128, 64, 128, 128, 0, 0),       # 8 queries on 128 rows, the last group of 5
+    (1, 603, 32, 256, 64, 100, 16, 0, 0),        # 4 on 128 rows; the visible entries change every 16 tokens
+    (1, 400, 64, 128, 64, 128, 16, 0, 0),        # 2 on 128 rows
+    (2, 1205, 16, 128, 64, 128, 128, 3000, 0),   # a chunk after 3000 tokens: the window's halo rows
+    (2, 600, 16, 128, 64, 5, 128, 0, 0),         # 12-key windows: the tile's upper 32 keys are all masked
+    (2, 600, 16, 128, 64, 0, 128, 0, 0),         # no window: queries before the first entry see no key
+    (2, 450, 16, 128, 64, 128, 128, 1000, 0),    # 57 groups of 8 per sequence are too few: 4 on 64 rows
+    (1, 599, 16, 512, 64, 37, 4, 77, 0),         # c = 512: 4 on 64 rows; short window, m = 4
+    (1, 399, 16, 512, 64, 37, 4, 77, 0),         # 100 groups leave SMs idle: one query per unit
+]
+
+
+@pytest.mark.parametrize("B,n_q,n_h,c,rd,w,m,start_pos,max_ctas", GROUP_CASES)
+def test_attend_query_groups(cuda, B, n_q, n_h, c, rd, w, m, start_pos, max_ctas):
+    """All-entries (HCA) attention over many queries runs 128 / n_h (c <= 256)
+    or 64 / n_h consecutive queries per unit: the union of their key sets is
+    gathered once and each query masks the keys outside its own window and
+    visible entries (juejin "DeepSeek-V4 技术报告简要解读" §2.3.2 Eq.(20)-(23)).
+    Every query is compared with the oracle over its own rows."""
+    seed = 8
+    halo = min(w - 1, start_pos)
+    win_tok0 = start_pos - halo
+    cap = (start_pos + n_q) // m + 1
+    q = rnd((B, n_q, n_h, c), seed, 1, BF16)
+    kv_comp = rnd((B, cap, c), seed, 2, BF16)
+    kv_win = rnd((B, n_q + halo, c), seed, 3, BF16)
+    sink = rnd((n_h,), seed, 4)
+    o = torch.full((B, n_q, n_h, c), float("nan"), dtype=BF16, device=cuda)
+    d = hb.attn_desc(B, n_h, c, rd, w, m, dtype=hb.HCA_BF16, max_ctas=max_ctas)
+    hb.hca_attend(d, q, kv_comp, cap, kv_win, False, sink, n_q, start_pos, o)
+    torch.cuda.synchronize()
+    s64, go = to64(sink), to64(o)
+    for b in range(B):
+        q64, comp, win = to64(q[b]), to64(kv_comp[b]), to64(kv_win[b])
+        for i in range(n_q):
+            t = start_pos + i
+            wpos = O.window_positions(t, w)
+            rows = np.concatenate([win[wpos - win_tok0], comp[:(t + 1) // m]], 0)
+            ref = O.attend_output(q64[i], rows, s64, c ** -0.5, t, rd)
+            assert_close(go[b, i], ref, 2e-2, f"o[{b},{i}]")
