@@ -331,26 +331,32 @@ struct Bars {
   uint64_t mg_ready, mg_full;    // cluster merge: peers' buffers free / peers' partials delivered
   uint64_t mg_stage;             // cluster merge: this CTA's blocks staged
   uint64_t pair[4];              // M = 128: the two softmax warps of a TMEM lane quarter
+  uint64_t us_full[2], us_empty[2];   // M = 128: unit slots (staged Q + RoPE table)
 };
 
 // Shared and tensor memory of one CTA.  M = 64: one query's (or a group's)
 // heads on 64 rows, S and Q in TMEM lane-half 1 beside O in lane-half 0.
 // M = 128 (c = 128, query groups): row i in TMEM lane i; two O accumulators
-// (one per half of each key tile), S buffers, Q; Q of the next unit is staged
-// in shared memory.
+// (one per half of each key tile), S buffers, Q; the loaders stage each
+// unit's Q rows and RoPE table in shared memory ahead of it.
 template <int C, int M = 64>
 struct Layout {
   static_assert(M == 64 || (M == 128 && C == 128), "M = 128 rows need c = 128");
   static constexpr int NKB = C / 64;
   // key-tile stages: Q lives in tensor memory, so the stages take what the P
   // buffers leave (192 KB for C = 512 and 256 at M = 64)
-  static constexpr int NS = M == 128 ? 8 : (C == 512) ? 3 : (C == 256 ? 6 : 8);
+  static constexpr int NS = M == 128 ? 6 : (C == 512) ? 3 : (C == 256 ? 6 : 8);
   static constexpr uint32_t kPBytes = M * 128;   // P tile: M rows x 64 keys (bf16)
   static constexpr int SP = M == 128 ? 3 : kSP;    // S / P buffers
   static constexpr uint32_t kv_off = 0;
   static constexpr uint32_t p_off = kv_off + NS * NKB * kTileBytes;
-  static constexpr uint32_t q_off = p_off + SP * kPBytes;             // M = 128: staged Q [128][C] bf16
-  static constexpr uint32_t bar_off = q_off + (M == 128 ? 128u * C * 2 : 0u);
+  // M = 128: a ring of two unit slots filled by the loaders -- the unit's Q
+  // rows [128][C] bf16 (chunks swizzled by row) and its RoPE table [8
+  // queries][cos 32 | sin 32] fp32
+  static constexpr uint32_t kQStage = 128u * C * 2, kRope = 8u * 64 * 4;
+  static constexpr uint32_t q_off = p_off + SP * kPBytes;
+  static constexpr uint32_t r_off = q_off + (M == 128 ? 2 * kQStage : 0u);
+  static constexpr uint32_t bar_off = r_off + (M == 128 ? 2 * kRope : 0u);
   static constexpr uint32_t misc_off = bar_off + 512;
   static constexpr uint32_t bytes = misc_off + 8192 + 1024;  // + alignment slack
   // tensor memory.  M = 64: O in lane-half 0, columns [0, C); in lane-half 1
@@ -623,8 +629,12 @@ attend_tc(AttendParams p, int n_units) {
       mbar_init(bar(bars->p_full[i]), SMW);
       mbar_init(bar(bars->pv_done[i]), 1);
     }
-    if (M == 128)
+    if (M == 128) {
       for (int i = 0; i < 4; ++i) mbar_init(bar(bars->pair[i]), 2);
+      // per loader thread: its Q copies landed (cp.async arrive) and its RoPE stores
+      for (int i = 0; i < 2; ++i) mbar_init(bar(bars->us_full[i]), 2 * PT);
+      for (int i = 0; i < 2; ++i) mbar_init(bar(bars->us_empty[i]), SMW);
+    }
     if (p.cluster) {
       mbar_init(bar(bars->mg_ready), p.nsplit);
       mbar_init(bar(bars->mg_full), 1);
@@ -666,7 +676,7 @@ attend_tc(AttendParams p, int n_units) {
     const int chunk = pt % CPR, prow = pt / CPR;
     const uint32_t kb_off = (chunk / 8) * kTileBytes;
     const int cc = chunk % 8;
-    uint32_t g = 0;
+    uint32_t g = 0, lv = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const Unit x = unit_of(p, u);
       const int b = x.b, qi = x.qi0;
@@ -674,6 +684,36 @@ attend_tc(AttendParams p, int n_units) {
       int j0, nt;
       split_range(ks, p.nsplit, x.sp, j0, nt);
       if (nt == 0) continue;
+      if constexpr (M == 128) {
+        // the unit's slot: thread pt copies Q row pt (head pt % n_h of query
+        // pt / n_h), 16-byte chunk i to position i ^ (pt & 7), and computes
+        // RoPE entries pt and pt + 128 of the unit's [G][rd/2] table
+        const int slot = lv & 1;
+        if (!twait_sleep(bar(bars->us_empty[slot]), ((lv >> 1) & 1) ^ 1, TR_P_QEMPTY)) return;
+        const int qg = pt / p.n_h, hq = pt - qg * p.n_h;
+        const bool live = qi + qg < p.n_q;
+        const char *src = reinterpret_cast<const char *>(
+            reinterpret_cast<const __nv_bfloat16 *>(p.q) +
+            (live ? (((long long)b * p.n_q + qi + qg) * p.n_h + hq) * C : 0));
+        const uint32_t qrow = sbase + L::q_off + slot * L::kQStage + pt * (C * 2);
+#pragma unroll
+        for (int i = 0; i < C / 8; ++i) cp_async16(qrow + ((i ^ (pt & 7)) << 4), src + 16 * i, live ? 16 : 0);
+        cp_async_arrive_noinc(bar(bars->us_full[slot]));
+        float *rope = reinterpret_cast<float *>(smem + L::r_off + slot * L::kRope);
+        for (int e = pt; e < p.G * 32; e += PT) {
+          const int gq = e >> 5, i = e & 31;
+          if (i < p.rd / 2) {
+            double ang = (double)(p.start_pos + qi + gq) * freq[i];
+            ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533576888376337251);
+            float sn, cs;
+            __sincosf((float)ang, &sn, &cs);   // |ang| <= pi: error below 1e-6
+            rope[gq * 64 + i] = cs;
+            rope[gq * 64 + 32 + i] = sn;
+          }
+        }
+        mbar_arrive(bar(bars->us_full[slot]));
+        ++lv;
+      }
       if (p.csa && pt < 32) {
         // index lists: this unit's into L1 (read tile by tile below), the next
         // unit's of this CTA into L2
@@ -885,8 +925,6 @@ attend_tc(AttendParams p, int n_units) {
     const int r = q4 * 32 + lane;
     const int rg = r / p.n_h, rh = r - rg * p.n_h;
     const int rg0 = (q4 * 32) / p.n_h, rg1 = (q4 * 32 + 31) / p.n_h;
-    const bool second = rg != rg0;
-    const float *rope_cs = rope_all + warp * 128 + (second ? 64 : 0);
     const float zs = p.scale * kLog2e;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + hf * C;   // this warp's O accumulator
@@ -901,32 +939,22 @@ attend_tc(AttendParams p, int n_units) {
       if (lane == 0) mbar_arrive(bar(bars->pair[q4]));
       return mbar_wait(bar(bars->pair[q4]), (npair++) & 1, p.status);
     };
-    // Q of the next unit: this thread's half row is copied (cp.async) into
-    // its own shared-memory slot while the current unit runs, then moved to
-    // tensor memory (row r, columns q_col + col_lo/2 ..) once the unit's last
-    // S has been read.  Chunk i sits at slot i ^ (lane & 7) (fewer bank
-    // conflicts on the way out).
-    const uint32_t qstage = sbase + L::q_off + (uint32_t)(r * 2 + hf) * (CH * 2);
-    auto stage_q = [&](int uq) {
-      const Unit xq = unit_of(p, uq);
-      const bool live = xq.qi0 + rg < p.n_q;
-      const long long qrow = live ? ((long long)xq.b * p.n_q + xq.qi0 + rg) * p.n_h + rh : 0;
-      const char *src = reinterpret_cast<const char *>(reinterpret_cast<const __nv_bfloat16 *>(p.q) + qrow * C + col_lo);
-#pragma unroll
-      for (int i = 0; i < NQC; ++i) cp_async16(qstage + ((i ^ (lane & 7)) << 4), src + 16 * i, live ? 16 : 0);
-      cp_async_commit();
-    };
+    // Q of unit slot lvq (staged by the loaders: row r's 16-byte chunk i at
+    // position i ^ (r & 7)) into tensor memory, row r, columns q_col + col_lo/2 ..,
+    // once the current unit's last S has been read
     uint32_t nq = 0;                      // Q writes so far (q_empty parity)
-    auto write_q = [&]() -> bool {
+    auto write_q = [&](uint32_t lvq) -> bool {
+      const int slot = lvq & 1;
+      if (!twait(bar(bars->us_full[slot]), (lvq >> 1) & 1, TR_P_QEMPTY)) return false;
       if (nq > 0 && !twait(bar(bars->q_empty), (nq - 1) & 1, TR_P_QEMPTY)) return false;
       tc_fence_after();
-      cp_async_wait_all();
+      const uint32_t qrow = sbase + L::q_off + slot * L::kQStage + r * (C * 2);
       uint32_t v[NQC * 4];
 #pragma unroll
       for (int i = 0; i < NQC; ++i)
         asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(v[4 * i]), "=r"(v[4 * i + 1]), "=r"(v[4 * i + 2]), "=r"(v[4 * i + 3])
-                     : "r"(qstage + ((i ^ (lane & 7)) << 4))
+                     : "r"(qrow + (((hf * NQC + i) ^ (r & 7)) << 4))
                      : "memory");
       const uint32_t tq = tmem + lane_base + L::q_col + col_lo / 2;
 #pragma unroll
@@ -947,16 +975,13 @@ attend_tc(AttendParams p, int n_units) {
       }
       return -1;
     };
-    constexpr double kTwoPi = 6.283185307179586476925286766559, kInvTwoPi = 0.15915494309189533576888376337251;
-    // (the angle is reduced to [-pi, pi] in double; the intrinsic's error there is below 1e-6)
     int q_ready_u = -1;
-    uint32_t g = 0;
+    uint32_t g = 0, lv = 0;               // tiles and units (with tiles) so far
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       const long long tu0 = TRACE ? clock64() : 0;
       const Unit ux = unit_of(p, u);
       const int b = ux.b, qi = ux.qi0;
       const bool live = qi + rg < p.n_q;
-      const int tw0 = p.start_pos + qi + rg0, tw1 = p.start_pos + qi + rg1;
       const KeySet ks = group_key_set(p, ux.qg);
       int j0, nt;
       split_range(ks, p.nsplit, ux.sp, j0, nt);
@@ -966,12 +991,10 @@ attend_tc(AttendParams p, int n_units) {
       const int w_lo = max(0, tq - p.w + 1 - ks.t0), w_hi = p.w > 0 ? min(tq - ks.t0 + 1, ks.nw) : 0;
       const int c_hi = ks.nw4 + fdiv(tq + 1, p.fd_m);
       if (nt > 0 && q_ready_u != u) {
-        stage_q(u);
-        if (!write_q()) return;
+        if (!write_q(lv)) return;
         q_ready_u = u;
       }
       const int un = nt > 0 ? next_unit(u) : -1;
-      if (un >= 0) stage_q(un);
       __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) +
                             (live ? (((long long)b * p.n_q + qi + rg) * p.n_h + rh) * C : 0);
       if (nt == 0) {
@@ -980,20 +1003,8 @@ attend_tc(AttendParams p, int n_units) {
             *reinterpret_cast<uint4 *>(orow + col) = make_uint4(0, 0, 0, 0);
         continue;
       }
-      // RoPE tables of the warp's queries (inverse rotation in the epilogue)
-      __syncwarp();
-      if (lane < p.rd / 2) {
-#pragma unroll
-        for (int k2 = 0; k2 < 2; ++k2) {
-          double ang = (double)(k2 ? tw1 : tw0) * freq[lane];
-          ang -= kTwoPi * rint(ang * kInvTwoPi);
-          float sn, cs;
-          __sincosf((float)ang, &sn, &cs);
-          rope_all[warp * 128 + k2 * 64 + lane] = cs;
-          rope_all[warp * 128 + k2 * 64 + 32 + lane] = sn;
-        }
-      }
-      __syncwarp();
+      // this row's query's RoPE table in the unit's slot (inverse rotation in the epilogue)
+      const float *rope_cs = reinterpret_cast<const float *>(smem + L::r_off + (lv & 1) * L::kRope) + rg * 64;
       // running max (log2 units; -inf until a valid key is seen) and sum
       float m_used = -INFINITY, l = 0.f;
       if (TRACE) tr[TR_S_TILE] += clock64() - tu0;   // the unit's setup
@@ -1088,7 +1099,7 @@ attend_tc(AttendParams p, int n_units) {
         phase(TR_S_WEIGHTS);
         if (j == nt - 1 && un >= 0) {
           // the unit's last S has been read: the next unit's Q goes in now
-          if (!write_q()) return;
+          if (!write_q(lv + 1)) return;
           q_ready_u = un;
           phase(TR_S_MERGE_LOOP);
         }
@@ -1160,12 +1171,15 @@ attend_tc(AttendParams p, int n_units) {
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(bars->o_empty));
+      if (lane == 0) {
+        mbar_arrive(bar(bars->o_empty));
+        mbar_arrive(bar(bars->us_empty[lv & 1]));   // the unit's slot is free again
+      }
       if (TRACE) tr[TR_S_EPI] += clock64() - te0;
       if (TRACE && threadIdx.x == 0 && ts[4] == 0) ts[4] = global_ns();
       g += nt;
+      ++lv;
     }
-    cp_async_wait_all();
     }();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
@@ -1341,7 +1355,7 @@ attend_tc(AttendParams p, int n_units) {
         uint32_t pk[16];
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
-          const float p0 = exp2f(z[x] - m_used), p1 = exp2f(z[x + 1] - m_used);
+          const float p0 = ex2_approx(z[x] - m_used), p1 = ex2_approx(z[x + 1] - m_used);
           psum += p0 + p1;
           pk[x / 2] = pack_bf16x2(p0, p1);
         }
