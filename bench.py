@@ -625,6 +625,10 @@ def roofline_tensor(flops_per_launch, ms_per_launch, peaks, traffic=None):
 # scale with the token count; the traffic of longer launches is this times
 # their tokens.
 CSA_PREFILL_ATTN_DRAM_PER_TOKEN = 2157e6 / 16384
+# DRAM bytes of the HCA prefill attention launch (batch 2 x 8192 tokens, 16
+# heads x 128): read + write counters of one ncu capture of that very launch
+# (71.4 MB + 18.3 MB; most of o is still in L2 when the kernel ends).
+HCA_PREFILL_ATTN_DRAM = 89.7e6
 
 
 def kern_ms(kern, prefix, K):
@@ -770,7 +774,8 @@ def main():
                 "layer_ms": round(statistics.mean(r["ms"]), 3),
                 "roofline_attention": roofline_tensor(
                     r["att_flops"], att_ms, peaks,
-                    traffic=round(CSA_PREFILL_ATTN_DRAM_PER_TOKEN * toks) if r["idx_flops"] else None),
+                    traffic=round(CSA_PREFILL_ATTN_DRAM_PER_TOKEN * toks) if r["idx_flops"] else
+                    (round(HCA_PREFILL_ATTN_DRAM) if pwl is workloads.HCA_PREFILL else None)),
                 "kernels_ms": {k: round(v["ms"] / kp, 3) for k, v in r["kern"].items()},
             }
             if r["idx_flops"]:
