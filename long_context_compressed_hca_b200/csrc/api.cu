@@ -262,6 +262,7 @@ int compress_params(const hca_compress_desc *d, int start_pos, int n, const void
   p.B = d->B; p.n = n; p.width = d->width; p.m = d->m; p.overlap = d->overlap;
   p.rd = (d->flags & HCA_COMPRESS_ROPE) ? d->rd : 0; p.flags = d->flags;
   p.eps = d->eps > 0.f ? d->eps : 1e-6f; p.theta = d->rope_theta > 0.f ? d->rope_theta : 10000.f;
+  fill_rope_freq(p.rope_freq, (d->flags & HCA_COMPRESS_ROPE) ? d->rd : 0, p.theta);
   p.Ca = Ca; p.Cb = Cb; p.Za = Za; p.Zb = Zb; p.row_stride = row_stride; p.seq_stride = seq_stride;
   p.Ba = Ba; p.Bb = Bb; p.gamma = gamma; p.out = out; p.out_scale = out_scale; p.out_seq_stride = out_seq_stride;
   p.state_kv = state_kv; p.state_score = state_score; p.in_dtype = d->in_dtype; p.out_dtype = d->out_dtype;

@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(128) attend_combine(AttendParams p) {
   } else if (threadIdx.x >= 32 && threadIdx.x - 32 < p.rd / 2) {
     const int i = threadIdx.x - 32;
     float sn, cs;
-    rope_sincos(t, i, p.rd, p.theta, &sn, &cs);
+    rope_sincos_tab(p.rope_freq, t, i, p.rd, p.theta, &sn, &cs);
     rcs[i] = cs;
     rcs[32 + i] = sn;
   }
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32) attend_simt(AttendParams p) {
     const float other = __shfl_xor_sync(0xffffffffu, v, 1);
     if (col >= p.c - p.rd) {
       float s, cs;
-      rope_sincos(t, (col - (p.c - p.rd)) / 2, p.rd, p.theta, &s, &cs);
+      rope_sincos_tab(p.rope_freq, t, (col - (p.c - p.rd)) / 2, p.rd, p.theta, &s, &cs);
       // inverse rotation: (a, b) -> (a cos + b sin, -a sin + b cos)
       v = (lane & 1) ? (-other * s + v * cs) : (v * cs + other * s);
     }

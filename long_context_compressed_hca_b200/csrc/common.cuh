@@ -466,6 +466,17 @@ __device__ __forceinline__ void store8(float *p, const float (&v)[8]) {
 
 // RoPE angle of pair i at position pos: pos * theta^(-2i/rd), reduced modulo
 // 2*pi in double so that large positions keep full fp32 accuracy.
+// sin / cos of pos * freq (freq = theta^(-2 pair / rd), double): the angle is
+// reduced to [-pi, pi] in double by a multiply with 1 / (2 pi), then sincosf.
+__device__ __forceinline__ void rope_angle_sincos(long long pos, double freq, float *s, float *c) {
+  double ang = (double)pos * freq;
+  ang -= 6.283185307179586476925286766559 * rint(ang * 0.15915494309189533576888376337251);
+  sincosf((float)ang, s, c);
+}
+// The same with the frequencies of the first 32 pairs from a host-computed
+// table (rd <= 64); wider rotations compute theirs.
+__device__ __forceinline__ void rope_sincos_tab(const double *tab, long long pos, int pair, int rd, float theta,
+                                                float *s, float *c);
 __device__ __forceinline__ void rope_sincos(long long pos, int pair, int rd, float theta,
                                             float *s, float *c) {
   const double freq = exp2(-2.0 * (double)pair / (double)rd * log2((double)theta));
@@ -473,6 +484,12 @@ __device__ __forceinline__ void rope_sincos(long long pos, int pair, int rd, flo
   const double two_pi = 6.283185307179586476925286766559;
   ang = ang - two_pi * floor(ang / two_pi);
   sincosf((float)ang, s, c);
+}
+
+__device__ __forceinline__ void rope_sincos_tab(const double *tab, long long pos, int pair, int rd, float theta,
+                                                float *s, float *c) {
+  if (rd <= 64) rope_angle_sincos(pos, tab[pair], s, c);
+  else rope_sincos(pos, pair, rd, theta, s, c);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -85,7 +85,7 @@ __device__ void entry_epilogue(const CompressParams &p, float (&v)[8], bool acti
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float s, c;
-      rope_sincos(pos, (ch0 - (p.width - p.rd)) / 2 + j, p.rd, p.theta, &s, &c);
+      rope_sincos_tab(p.rope_freq, pos, (ch0 - (p.width - p.rd)) / 2 + j, p.rd, p.theta, &s, &c);
       const float a = v[2 * j], bb = v[2 * j + 1];
       v[2 * j] = a * c - bb * s;
       v[2 * j + 1] = a * s + bb * c;
@@ -192,6 +192,123 @@ compress_prefill_kernel(CompressParams p, int epb, int rg) {
     for (int q = 0; q < 8; ++q) v[q] = 0.f;
   }
   entry_epilogue<Tout>(p, v, active, slot, cvi, cv, b, entry - p.e_first, (p.e_pos0 + entry) * p.m, red, red2);
+}
+
+// Prefill with many entries, for widths whose 8-channel groups tile a warp
+// (c/8 a power of two up to 32, or a multiple of 32 up to 256): a thread owns 8 channels of one
+// entry and all of the entry's rows (no partial softmaxes to merge), loading
+// kRowBatch rows at a time with all of their loads in flight; the entry's
+// sums of squares and maxima are reduced by shuffles within its lanes and,
+// when the entry spans several warps, through shared memory under a named
+// barrier of just those warps -- no block-wide barrier.
+constexpr int kRowBatch = 4;
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kThreads) compress_prefill_rows_kernel(CompressParams p) {
+  __shared__ float xbuf[2][kThreads / 32];
+  const int cv = p.width / 8;
+  const int epc = kThreads / cv;                 // entries per block
+  const int tid = threadIdx.x;
+  const int slot = tid / cv, cvi = tid - slot * cv;
+  const int b = blockIdx.y;
+  const int E = p.n / p.m;
+  const long long entry = p.e_first + (long long)blockIdx.x * epc + slot;
+  const bool valid = entry < E;
+  const int R = (p.overlap && entry > 0) ? 2 * p.m : p.m;
+  float mx[8], sum[8], acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { mx[j] = -INFINITY; sum[j] = 0.f; acc[j] = 0.f; }
+  if (valid) {
+    for (int r0 = 0; r0 < R; r0 += kRowBatch) {
+      float z[kRowBatch][8], cval[kRowBatch][8];
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) {
+        const int r = r0 + k;
+        if (r < R) {
+          const bool a_series = r < p.m;
+          const int j = a_series ? r : r - p.m;
+          const long long tok = a_series ? entry * p.m + j : (entry - 1) * p.m + j;
+          load8(row_ptr<Tin>(a_series ? p.Za : p.Zb, p.seq_stride, p.row_stride, b, tok) + cvi * 8, z[k]);
+          load8(row_ptr<Tin>(a_series ? p.Ca : p.Cb, p.seq_stride, p.row_stride, b, tok) + cvi * 8, cval[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kRowBatch; ++k) {
+        const int r = r0 + k;
+        if (r < R) {
+          const bool a_series = r < p.m;
+          const int j = a_series ? r : r - p.m;
+          const float *bp = (a_series ? p.Ba : p.Bb) + (long long)j * p.width + cvi * 8;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float l = z[k][q] + bp[q];
+            const float nm = fmaxf(mx[q], l);
+            const float sc = __expf(mx[q] - nm);   // mx = -inf on the first row -> 0
+            const float e = __expf(l - nm);
+            sum[q] = sum[q] * sc + e;
+            acc[q] = acc[q] * sc + e * cval[k][q];
+            mx[q] = nm;
+          }
+        }
+      }
+    }
+  }
+  float v[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) v[q] = valid ? acc[q] / sum[q] : 0.f;
+  // reduction over the entry's cv lanes (use 0: sums, 1: maxima)
+  auto reduce = [&](float x, bool is_max, int use) -> float {
+    const int g = cv < 32 ? cv : 32;
+    for (int o = g / 2; o > 0; o >>= 1) {
+      const float y = __shfl_xor_sync(0xffffffffu, x, o);
+      x = is_max ? fmaxf(x, y) : x + y;
+    }
+    if (cv <= 32) return x;
+    const int wpe = cv / 32, w = tid >> 5;       // warps per entry, this warp
+    if ((tid & 31) == 0) xbuf[use][w] = x;
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(cv) : "memory");
+    float t = is_max ? 0.f : 0.f;
+    for (int i = 0; i < wpe; ++i) {
+      const float y = xbuf[use][slot * wpe + i];
+      t = is_max ? fmaxf(t, y) : t + y;
+    }
+    return t;
+  };
+  const int ch0 = cvi * 8;
+  if (p.flags & HCA_COMPRESS_NORM) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss += v[j] * v[j];
+    const float tot = reduce(ss, false, 0);
+    const float rn = rsqrtf(tot / (float)p.width + p.eps);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] *= rn * (p.gamma ? p.gamma[ch0 + j] : 1.f);
+  }
+  if ((p.flags & HCA_COMPRESS_ROPE) && p.rd > 0 && ch0 >= p.width - p.rd) {
+    const long long pos = (p.e_pos0 + entry) * p.m;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float sn, cs;
+      rope_sincos_tab(p.rope_freq, pos, (ch0 - (p.width - p.rd)) / 2 + j, p.rd, p.theta, &sn, &cs);
+      const float a = v[2 * j], bb = v[2 * j + 1];
+      v[2 * j] = a * cs - bb * sn;
+      v[2 * j + 1] = a * sn + bb * cs;
+    }
+  }
+  float inv_scale = 1.f;
+  if (p.out_dtype == HCA_FP8E4M3) {
+    float am = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = fmaxf(am, fabsf(v[j]));
+    const float tot = fmaxf(reduce(am, true, 1), 1e-12f);
+    const float scale = tot / 448.f;
+    inv_scale = 1.f / scale;
+    if (valid && cvi == 0) p.out_scale[(long long)b * p.out_seq_stride + (entry - p.e_first)] = scale;
+  }
+  if (valid) {
+    Tout *row = reinterpret_cast<Tout *>(p.out) + ((long long)b * p.out_seq_stride + (entry - p.e_first)) * p.width;
+    EntryWriter<Tout>::put(row, ch0, v, inv_scale);
+  }
 }
 
 // Prefill leaves the state ready for decode at position n (rows of the last
@@ -361,6 +478,22 @@ __global__ void __launch_bounds__(kThreads) decode_ingest_kernel(CompressParams 
 template <typename Tin>
 int launch_prefill_t(const CompressParams &p, cudaStream_t s) {
   const int cv = p.width / 8;
+  const long long E_w = p.n / p.m - p.e_first;   // entries written
+  // a thread per (entry, 8 channels) when that gives half the SMs a block;
+  // few long entries (HCA) split their rows over row groups instead
+  if ((((cv & (cv - 1)) == 0 && cv <= 32) || (cv % 32 == 0 && cv <= kThreads)) &&
+      (long long)p.B * ((E_w + kThreads / cv - 1) / (kThreads / cv)) >= num_sms() / 2) {
+    const long long E = E_w;
+    const int epc = kThreads / cv;
+    dim3 grid((unsigned)((E + epc - 1) / epc), p.B);
+    LaunchScope ls_("compress_prefill", s);
+    switch (p.out_dtype) {
+      case HCA_F32: compress_prefill_rows_kernel<Tin, float><<<grid, kThreads, 0, s>>>(p); break;
+      case HCA_BF16: compress_prefill_rows_kernel<Tin, __nv_bfloat16><<<grid, kThreads, 0, s>>>(p); break;
+      default: compress_prefill_rows_kernel<Tin, uint8_t><<<grid, kThreads, 0, s>>>(p); break;
+    }
+    return ls_.done();
+  }
   const int R = p.overlap ? 2 * p.m : p.m;
   // entries per block: give each entry about cv * R threads, at most kThreads
   int epb = 1;

@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) row_op_kernel(RowOpParams p) {
 #pragma unroll
         for (int j = 0; j < 4; j += 2) {
           float s, cs;
-          rope_sincos(pos, (c + j - c_rope) / 2, p.rd, p.theta, &s, &cs);
+          rope_sincos_tab(p.rope_freq, pos, (c + j - c_rope) / 2, p.rd, p.theta, &s, &cs);
           const float a = v[j], b = v[j + 1];
           v[j] = a * cs - b * s;
           v[j + 1] = a * s + b * cs;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) row_op_kernel(RowOpParams p) {
       float b = in[c + 1] * r * (p.gamma ? p.gamma[c + 1] : 1.f);
       if (c >= c_rope) {
         float s, cs;
-        rope_sincos(pos, (c - c_rope) / 2, p.rd, p.theta, &s, &cs);
+        rope_sincos_tab(p.rope_freq, pos, (c - c_rope) / 2, p.rd, p.theta, &s, &cs);
         const float a2 = a * cs - b * s, b2 = a * s + b * cs;
         a = a2; b = b2;
       }
@@ -219,8 +219,10 @@ int launch_gemm(hca_dtype ab, const void *A, long long lda, const void *Bm, long
   return ls_.done();
 }
 
-int launch_row_op(const RowOpParams &p, cudaStream_t s) {
-  if (p.rows == 0) return HCA_OK;
+int launch_row_op(const RowOpParams &p0, cudaStream_t s) {
+  if (p0.rows == 0) return HCA_OK;
+  RowOpParams p = p0;
+  fill_rope_freq(p.rope_freq, p.rd, p.theta);
   const bool vec = p.cols % 4 == 0 && p.in_stride % 4 == 0 && p.out_stride % 4 == 0 &&
                    (reinterpret_cast<uintptr_t>(p.in) & 15) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0 &&
                    (!p.gamma || (reinterpret_cast<uintptr_t>(p.gamma) & 15) == 0);

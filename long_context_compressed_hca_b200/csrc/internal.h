@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <cmath>
 
 #include "../../include/hca.h"
 
@@ -46,9 +47,16 @@ int encode_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dt, u
 int *device_status_ptr();
 
 // ------------------------------------------------------------- compress
+// theta^(-2i/rd) for the first min(rd/2, 32) rotated pairs (host-computed).
+inline void fill_rope_freq(double (&f)[32], int rd, float theta) {
+  for (int i = 0; i < 32; ++i)
+    f[i] = (rd > 0 && i < rd / 2) ? std::exp2(-2.0 * i / (double)rd * std::log2((double)theta)) : 0.0;
+}
+
 struct CompressParams {
   int B, n, width, m, overlap, rd, flags;
   float eps, theta;
+  double rope_freq[32];    // fill_rope_freq(rd, theta)
   const void *Ca, *Cb, *Za, *Zb;
   long long row_stride, seq_stride;
   const float *Ba, *Bb, *gamma;
@@ -219,6 +227,7 @@ struct RowOpParams {
   int rd; float theta; long long pos0; int rows_per_pos; int pos_mod;
   long long pos_base;   // RoPE position = pos_base + (pos0 + row / rows_per_pos) % pos_mod
   float scale;
+  double rope_freq[32];  // filled by launch_row_op
 };
 int launch_row_op(const RowOpParams &p, cudaStream_t s);
 
