@@ -281,13 +281,34 @@ gemm_tc_skinny(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // rows [z 128/S, (z+1) 128/S) of the tile, summed over the partials in order
         const int r0 = z * 128 / S, r1 = (z + 1) * 128 / S, nr = r1 - r0;
         const uint32_t pbase = smem_u32(P);
-        for (int it = threadIdx.x - 64; it < nr * TN; it += 128) {
-          const int j = it / nr, rr = r0 + it % nr;
-          float acc = 0.f;
-          for (int zz = 0; zz < S; ++zz)
-            acc += __uint_as_float(ld_dsmem_u32(cluster_map(pbase + (uint32_t)((j * 128 + rr) * 4), zz)));
-          const int row = m0 + j, col = n0 + rr;
-          if (row < M && col < N) Elt<TC>::store(C + (long long)row * ldc + col, alpha * acc);
+        // kOut outputs per pass, all of their S partial loads in flight before
+        // any is added; each sum still runs over CTAs 0..S-1 in order
+        constexpr int kOut = 4, kMaxS = 8;
+        const int tot = nr * TN;
+        for (int it0 = threadIdx.x - 64; it0 < tot; it0 += 128 * kOut) {
+          float part[kOut][kMaxS];
+#pragma unroll
+          for (int o = 0; o < kOut; ++o) {
+            const int it = it0 + o * 128;
+            const int j = it / nr, rr = r0 + it % nr;
+#pragma unroll
+            for (int zz = 0; zz < kMaxS; ++zz)
+              part[o][zz] = (it < tot && zz < S)
+                                ? __uint_as_float(ld_dsmem_u32(cluster_map(pbase + (uint32_t)((j * 128 + rr) * 4), zz)))
+                                : 0.f;
+          }
+#pragma unroll
+          for (int o = 0; o < kOut; ++o) {
+            const int it = it0 + o * 128;
+            if (it >= tot) break;
+            const int j = it / nr, rr = r0 + it % nr;
+            float acc = 0.f;
+#pragma unroll
+            for (int zz = 0; zz < kMaxS; ++zz)
+              if (zz < S) acc += part[o][zz];
+            const int row = m0 + j, col = n0 + rr;
+            if (row < M && col < N) Elt<TC>::store(C + (long long)row * ldc + col, alpha * acc);
+          }
         }
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");
