@@ -575,8 +575,8 @@ attend_tc(AttendParams p, int n_units) {
   Bars *bars = reinterpret_cast<Bars *>(smem + L::bar_off);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::misc_off);
   double *freq = reinterpret_cast<double *>(smem + L::misc_off + 8);      // [32]
-  float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // [8 warps][2][64]: cos, sin
-  float *xch = reinterpret_cast<float *>(smem + L::misc_off + 4608);       // [3][8 warps][32]
+  float *rope_all = reinterpret_cast<float *>(smem + L::misc_off + 512);   // M = 64: [4 warps][64]: cos, sin
+  float *xch = reinterpret_cast<float *>(smem + L::misc_off + 4608);       // M = 128: (max, sum) [8 warps][32]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // warp roles: softmax warps first, then the MMA warp, then the loaders.
@@ -924,7 +924,6 @@ attend_tc(AttendParams p, int n_units) {
     const int q4 = warp & 3, hf = warp >> 2;
     const int r = q4 * 32 + lane;
     const int rg = r / p.n_h, rh = r - rg * p.n_h;
-    const int rg0 = (q4 * 32) / p.n_h, rg1 = (q4 * 32 + 31) / p.n_h;
     const float zs = p.scale * kLog2e;
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     const uint32_t tO = tmem + lane_base + hf * C;   // this warp's O accumulator
