@@ -625,7 +625,7 @@ attend_tc(AttendParams p, int n_units) {
     }
     for (int i = 0; i < SP; ++i) {
       mbar_init(bar(bars->s_full[i]), 1);
-      mbar_init(bar(bars->s_empty[i]), SMW);
+      mbar_init(bar(bars->s_empty[i]), M == 128 ? 1 : SMW);   // M = 128: released by the MMA after P.V
       mbar_init(bar(bars->p_full[i]), SMW);
       mbar_init(bar(bars->pv_done[i]), 1);
     }
@@ -853,11 +853,19 @@ attend_tc(AttendParams p, int n_units) {
 #pragma unroll
           for (int nh = 0; nh < C / NPV; ++nh) {
             const uint64_t voff = (nh * (NPV / 64) * kTileBytes + kk * 16 * 128) >> 4;
-            umma_bf16(tmem + o_acc + nh * NPV, pd + ((kk * 32) >> 4), vd + voff, IDESC_PV, reset ? 0u : 1u);
+            if constexpr (M == 128) {
+              // P (bf16) in the tile's S columns: keys [32h, 32h + 32) of
+              // every row at columns s_col + 32h .. + 16, the A operand
+              const uint32_t pa_t = tS + L::s_col(st) + 32 * (kk >> 1) + 8 * (kk & 1);
+              umma_bf16_ts(tmem + o_acc + nh * NPV, pa_t, vd + voff, IDESC_PV, reset ? 0u : 1u);
+            } else {
+              umma_bf16(tmem + o_acc + nh * NPV, pd + ((kk * 32) >> 4), vd + voff, IDESC_PV, reset ? 0u : 1u);
+            }
           }
         }
         umma_commit(bar(bars->kv_empty[kst]));
         umma_commit(bar(bars->pv_done[st]));
+        if (M == 128) umma_commit(bar(bars->s_empty[st]));   // the S / P columns are free
         return true;
       };
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -1028,9 +1036,6 @@ attend_tc(AttendParams p, int n_units) {
         tmem_ld_32x32b_x16(tmem + lane_base + L::s_col(st) + 32 * hf, *reinterpret_cast<uint32_t(*)[16]>(&sv[0]));
         tmem_ld_32x32b_x16(tmem + lane_base + L::s_col(st) + 32 * hf + 16, *reinterpret_cast<uint32_t(*)[16]>(&sv[16]));
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(bars->s_empty[st]));
         phase(TR_S_MERGE_READY);
         // this row's valid keys among the warp's 32
         const int kb = (j0 + j) * KT + 32 * hf;
@@ -1083,15 +1088,10 @@ attend_tc(AttendParams p, int n_units) {
         }
         l += ps[0] + ps[1];
         phase(TR_S_PUSH);
-        // P buffer `st` is free once the P.V of tile gj - 2 has completed
-        if (!twait(bar(bars->pv_done[st]), ph ^ 1, TR_S_PBUF)) return;
-        const uint32_t prow = sbase + L::p_off + st * L::kPBytes;
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(prow + sw128_off(r, 4 * hf + c4)),
-                       "r"(pk[4 * c4]), "r"(pk[4 * c4 + 1]), "r"(pk[4 * c4 + 2]), "r"(pk[4 * c4 + 3])
-                       : "memory");
-        fence_proxy_async();
+        // P (bf16) over the first 16 of this warp's 32 S columns of the tile
+        // (already read); the P.V reads it from tensor memory
+        tmem_st_32x32b_x16(tmem + lane_base + L::s_col(st) + 32 * hf, pk);
+        tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(bars->p_full[st]));
