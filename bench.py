@@ -627,8 +627,8 @@ def roofline_tensor(flops_per_launch, ms_per_launch, peaks, traffic=None):
 CSA_PREFILL_ATTN_DRAM_PER_TOKEN = 2157e6 / 16384
 # DRAM bytes of the HCA prefill attention launch (batch 2 x 8192 tokens, 16
 # heads x 128): read + write counters of one ncu capture of that very launch
-# (71.4 MB + 18.3 MB; most of o is still in L2 when the kernel ends).
-HCA_PREFILL_ATTN_DRAM = 89.7e6
+# (71.4 MB + 20.7 MB; most of o is still in L2 when the kernel ends).
+HCA_PREFILL_ATTN_DRAM = 92.1e6
 
 
 def kern_ms(kern, prefix, K):
